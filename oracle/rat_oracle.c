@@ -1,0 +1,242 @@
+/*
+ * rat_oracle.c -- plain, slow CPU oracle for the RAT+ temporal-mixing operator.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path (the CUDA library and
+ * its Python binding) may include, link or call this file; only the tests, the
+ * smoke check and the benchmark's CPU-baseline leg use it.  It shares no code,
+ * header, table or constant with the CUDA path.
+ *
+ * Everything is computed in IEEE double, straight from the definitions, with no
+ * blocking, fusion or reordering.  OpenMP only spreads independent output rows
+ * or channels over host threads; it does not change any sum's order.
+ *
+ * Sources (titles of the pages the operator is defined on):
+ *   [RAT+]  "RAT+: Train Dense, Infer Sparse -- Recurrence Augmented Attention
+ *           for Dilated Inference": Abstract; Figure 1(a) (full-sequence
+ *           recurrence, L=T); Figure 1(c) (dilated attention, optional local
+ *           attention); Figure 2 (prefill by a scan, decode by a step update).
+ *   [MEM]   "Augmenting Attention with Exponentially Decaying Memory Improves
+ *           Query-Aware KV Sparsity": section 2.1 (key and value states updated
+ *           with an input-dependent gate; exponentially decaying memory).
+ *   [RAT]   "RAT: Bridging RNN Efficiency and Attention Accuracy via
+ *           Chunk-based Sequence Modeling": Approach (gated linear recurrence;
+ *           chunk size L=T makes the layer an RNN).
+ *
+ * Readings taken where the pages leave a step open (each is also listed in the
+ * design notes):
+ *   R1 recurrence: per channel c, s_t = a_t*s_{t-1} + (1-a_t)*x_t with
+ *      a_t = sigmoid(g_t); one gate tensor g drives both the key and the value
+ *      recurrence; s_{-1} = init (zero unless given).
+ *   R2 dilation: query t attends to { j : 0 <= j <= t, (t-j) mod D == 0 }.
+ *   R3 window: W > 0 adds the dense set { j : max(0,t-W+1) <= j <= t }.
+ *   R4 the two parts are two separate softmaxes merged by log-sum-exp, so a
+ *      key in both sets (j = t always is) is counted once in each part.
+ *   R5 score scale s = 1/sqrt(d) unless the caller gives one; the query is not
+ *      recurrence-augmented; both parts read the augmented keys and values.
+ *   R6 a head with recur = 0 uses a = 0, i.e. augmented keys/values equal the
+ *      raw ones (D = 1, a = 0 is plain causal attention).
+ *
+ * Parity pins for every function here live in tests/test_oracle_pins.py.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+/* element (b,t,h,c) of a row-major [B,T,H,d] tensor */
+static size_t idx4(int T, int H, int d, int b, long t, int h, int c)
+{
+    return (((size_t)b * (size_t)T + (size_t)t) * (size_t)H + (size_t)h) * (size_t)d + (size_t)c;
+}
+
+static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
+
+/*
+ * R1: the gated linear recurrence, one channel at a time, t = 0 .. T-1 in order
+ * ([MEM] 2.1; [RAT+] Figure 1(a) L=T; [RAT] Approach).
+ *   x, g   : [B,T,H,d]           input and gate logit
+ *   init   : [B,H,d] or NULL     s_{-1}; NULL means zero
+ *   recur  : [H] or NULL         0 => a = 0 for that head (R6); NULL => all 1
+ *   out    : [B,T,H,d]           s_t for every t
+ *   final  : [B,H,d] or NULL     s_{T-1} (init when T = 0)
+ */
+void oracle_scan(int B, int T, int H, int d, const double *x, const double *g,
+                 const double *init, const unsigned char *recur, double *out,
+                 double *final)
+{
+    long nch = (long)B * H * d;
+#pragma omp parallel for schedule(static)
+    for (long ch = 0; ch < nch; ++ch) {
+        int b = (int)(ch / ((long)H * d));
+        int h = (int)((ch / d) % H);
+        int c = (int)(ch % d);
+        int rec = recur ? (recur[h] != 0) : 1;
+        double s = init ? init[ch] : 0.0;
+        for (long t = 0; t < T; ++t) {
+            size_t e = idx4(T, H, d, b, t, h, c);
+            double a = rec ? sigmoid(g[e]) : 0.0;
+            s = a * s + (1.0 - a) * x[e];
+            out[e] = s;
+        }
+        if (final) final[ch] = s;
+    }
+}
+
+/*
+ * Softmax of q_t against the key set `js` (n entries) of head h in batch b:
+ *   z_j = scale * sum_c q[c]*k_j[c];  lse = log sum_j exp(z_j);
+ *   o[c] = sum_j exp(z_j - lse) * v_j[c].
+ * The maximum is subtracted before exp only to avoid overflow; it cancels.
+ */
+static void softmax_over(int T, int H, int d, const double *qrow, const double *k,
+                         const double *v, int b, int h, const long *js, long n,
+                         double scale, double *o, double *lse, double *z)
+{
+    double m = -INFINITY;
+    for (long i = 0; i < n; ++i) {
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c) acc += qrow[c] * k[idx4(T, H, d, b, js[i], h, c)];
+        z[i] = scale * acc;
+        if (z[i] > m) m = z[i];
+    }
+    double den = 0.0;
+    for (long i = 0; i < n; ++i) den += exp(z[i] - m);
+    for (int c = 0; c < d; ++c) o[c] = 0.0;
+    for (long i = 0; i < n; ++i) {
+        double p = exp(z[i] - m) / den;
+        for (int c = 0; c < d; ++c) o[c] += p * v[idx4(T, H, d, b, js[i], h, c)];
+    }
+    *lse = m + log(den);
+}
+
+/* R4: merge two (output, log-sum-exp) pairs as one softmax over both sets. */
+static void lse_merge(int d, const double *o1, double l1, const double *o2, double l2,
+                      double *o, double *lse)
+{
+    double m = l1 > l2 ? l1 : l2;
+    double w1 = exp(l1 - m), w2 = exp(l2 - m);
+    for (int c = 0; c < d; ++c) o[c] = (w1 * o1[c] + w2 * o2[c]) / (w1 + w2);
+    *lse = m + log(w1 + w2);
+}
+
+/*
+ * One output row per requested (b, h, t) of the attention step over the
+ * augmented keys kt and values vt ([RAT+] Abstract and Figure 1(c)).
+ *   q, kt, vt : [B,T,H,d]
+ *   dil, win  : [H]  dilation D_h >= 1, window W_h >= 0
+ *   parts     : 1 = dilated part only (R2), 2 = window part only (R3),
+ *               3 = the operator's output: dilated part, merged with the window
+ *                   part when W_h > 0 (R4)
+ *   rows      : nrows x 3 int64 (b, h, t)
+ *   o, lse    : nrows x d, nrows
+ * Returns 0, or -1 on an argument error (the outputs are then untouched).
+ */
+int oracle_attn_rows(int B, int T, int H, int d, const double *q, const double *kt,
+                     const double *vt, const int *dil, const int *win, double scale,
+                     int parts, long nrows, const int64_t *rows, double *o, double *lse)
+{
+    if (parts < 1 || parts > 3) return -1;
+    for (long r = 0; r < nrows; ++r) {
+        int64_t b = rows[3 * r], h = rows[3 * r + 1], t = rows[3 * r + 2];
+        if (b < 0 || b >= B || h < 0 || h >= H || t < 0 || t >= T) return -1;
+        if (dil[h] < 1 || win[h] < 0) return -1;
+        if (parts == 2 && win[h] == 0) return -1;
+    }
+    int err = 0;
+#pragma omp parallel
+    {
+        long *js = (long *)malloc(sizeof(long) * (size_t)(T > 0 ? T : 1));
+        double *z = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+        double *o1 = (double *)malloc(sizeof(double) * (size_t)d);
+        double *o2 = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!js || !z || !o1 || !o2) {
+#pragma omp atomic write
+            err = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (long r = 0; r < nrows; ++r) {
+            if (err) continue;
+            int b = (int)rows[3 * r], h = (int)rows[3 * r + 1];
+            long t = (long)rows[3 * r + 2];
+            const double *qrow = q + idx4(T, H, d, b, t, h, 0);
+            int D = dil[h], W = win[h];
+            double l1 = 0.0, l2 = 0.0;
+            if (parts & 1) { /* R2: j <= t with (t - j) mod D == 0 */
+                long n = 0;
+                for (long j = 0; j <= t; ++j)
+                    if ((t - j) % D == 0) js[n++] = j;
+                softmax_over(T, H, d, qrow, kt, vt, b, h, js, n, scale, o1, &l1, z);
+            }
+            if ((parts & 2) && W > 0) { /* R3: max(0, t-W+1) <= j <= t */
+                long n = 0;
+                for (long j = 0; j <= t; ++j)
+                    if (j >= t - W + 1) js[n++] = j;
+                softmax_over(T, H, d, qrow, kt, vt, b, h, js, n, scale, o2, &l2, z);
+            }
+            double *orow = o + (size_t)r * (size_t)d;
+            if (parts == 1 || (parts == 3 && W == 0)) {
+                for (int c = 0; c < d; ++c) orow[c] = o1[c];
+                lse[r] = l1;
+            } else if (parts == 2) {
+                for (int c = 0; c < d; ++c) orow[c] = o2[c];
+                lse[r] = l2;
+            } else {
+                lse_merge(d, o1, l1, o2, l2, orow, &lse[r]);
+            }
+        }
+        free(js); free(z); free(o1); free(o2);
+    }
+    return err ? -1 : 0;
+}
+
+/*
+ * One decode step ([RAT+] Figure 2: "a simple step update" for the recurrence,
+ * then attention of the new query over the cached augmented keys/values).
+ * For every batch entry b the new token sits at position t = pos[b]:
+ *   1. R1 one step: s <- a*s + (1-a)*x for x = k and x = v (a = 0 when
+ *      recur_h = 0), with a = sigmoid(g);
+ *   2. the new augmented key/value s is stored as row t of the history;
+ *   3. the output is oracle_attn_rows' row (b, h, t) with parts = 3 over the
+ *      history rows 0..t.
+ *   q, k, v, g          : [B,H,d]   the new token
+ *   state_k, state_v    : [B,H,d]   s_{t-1} in, s_t out
+ *   hist_k, hist_v      : [B,cap,H,d] augmented keys/values in natural order;
+ *                                      rows < pos[b] are read, row pos[b] written
+ *   o, lse              : [B,H,d], [B,H]
+ * Returns 0, or -1 on an argument error.
+ */
+int oracle_decode_step(int B, int H, int d, int cap, const int *pos, const double *q,
+                       const double *k, const double *v, const double *g,
+                       const int *dil, const int *win, const unsigned char *recur,
+                       double scale, double *state_k, double *state_v, double *hist_k,
+                       double *hist_v, double *o, double *lse)
+{
+    for (int b = 0; b < B; ++b)
+        if (pos[b] < 0 || pos[b] >= cap) return -1;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h)
+            for (int c = 0; c < d; ++c) {
+                size_t e = ((size_t)b * H + h) * d + c;
+                double a = (recur == NULL || recur[h]) ? sigmoid(g[e]) : 0.0;
+                state_k[e] = a * state_k[e] + (1.0 - a) * k[e];
+                state_v[e] = a * state_v[e] + (1.0 - a) * v[e];
+                hist_k[idx4(cap, H, d, b, pos[b], h, c)] = state_k[e];
+                hist_v[idx4(cap, H, d, b, pos[b], h, c)] = state_v[e];
+            }
+    /* the query of the new token laid out as row pos[b] of a [B,cap,H,d] tensor */
+    double *qfull = (double *)calloc((size_t)B * cap * H * d, sizeof(double));
+    int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * 3 * (size_t)B * H);
+    if (!qfull || !rows) { free(qfull); free(rows); return -1; }
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            for (int c = 0; c < d; ++c)
+                qfull[idx4(cap, H, d, b, pos[b], h, c)] = q[((size_t)b * H + h) * d + c];
+            int64_t *rw = rows + 3 * ((size_t)b * H + h);
+            rw[0] = b; rw[1] = h; rw[2] = pos[b];
+        }
+    int rc = oracle_attn_rows(B, cap, H, d, qfull, hist_k, hist_v, dil, win, scale, 3,
+                              (long)B * H, rows, o, lse);
+    free(qfull);
+    free(rows);
+    return rc;
+}
