@@ -1,0 +1,508 @@
+#!/usr/bin/env python
+"""Benchmark of the RAT+ temporal-mixing operator on B200.
+
+Headline workload: prefill of 262144 tokens, B=1, 16 heads x 128 (hidden
+2048), dilation 64 plus a local window of 512 merged by log-sum-exp, bf16
+operands with fp32 state and softmax (the 262K prefill of "RAT+: Train Dense,
+Infer Sparse", Figure 2).  One step = one pass of the whole operator over that
+input: the recurrence scan of k and v, then the dilated + windowed attention.
+Alongside: decode at batch 256, 16 heads x 128, D=16 over a prefilled cache
+(Figure 2's decode scenario), reported in the "decode" object.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
+device synchronize; CUDA events on the launching stream time the whole step
+and each kernel stage; the multi-GPU time is the max over ranks.  Inputs are
+larger than L2 (4.3 GB per prefill step), so no flush is needed.
+
+`--impl reference` times the CPU oracle (the plain fp64 implementation the
+parity tests use) on the host cores on a bounded sample of the same workload.
+
+Prints ONE JSON line on rank 0.
+"""
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "temporal-mix prefill tok/s @262K & decode tok/s; % of HBM/tensor roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------- plumbing
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(world, backend):
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x, world, device):
+    """Max of a float over ranks (identity at world size 1)."""
+    if world == 1:
+        return float(x)
+    import torch.distributed as dist
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        d["_source"] = "measured"
+        return d
+    d = dict(PEAKS_FALLBACK)
+    d["_source"] = "fallback"
+    return d
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.f = None
+
+    def __enter__(self):
+        try:
+            self.f = tempfile.TemporaryFile(mode="w+")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.f is None:
+            return None
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.strip()]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for i, n in enumerate(names):
+                if r[5 + i].lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def profile_traffic(name):
+    """Per-launch DRAM bytes of kernel `name` from its committed ncu summary,
+    or None if there is none or the kernel source changed since the capture."""
+    path = os.path.join(ROOT, "profiles", name + ".md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)\s*\(source sha1 ([0-9a-f]+) of ([\w./]+)\)", txt)
+    if not m:
+        return None
+    src = os.path.join(ROOT, m.group(3))
+    if not os.path.exists(src) or hashlib.sha1(open(src, "rb").read()).hexdigest()[:12] != m.group(2)[:12]:
+        return None
+    return float(m.group(1))
+
+
+# --------------------------------------------------------- algorithmic work
+
+
+def attn_pairs(T, D, W):
+    """Unmasked (query, key) pairs of one head: dilated part + window part."""
+    n = np.array([(T - r + D - 1) // D for r in range(min(D, T))], dtype=np.float64)
+    pairs = float(np.sum(n * (n + 1) / 2))
+    if W > 0:
+        Wm = min(W, T)
+        pairs += Wm * (Wm + 1) / 2 + (T - Wm) * W
+    return pairs
+
+
+def prefill_work(w):
+    """(attention FLOPs, scan bytes) of one prefill step: 4*d FLOPs per pair;
+    10 bytes per (token, channel) of a recurrent head (k, v, g read; kt, vt written)."""
+    flops = 0.0
+    scan_bytes = 0.0
+    elt = 2 if w.dtype == "bf16" else 4
+    for h in range(w.H):
+        flops += w.B * 4.0 * w.d * attn_pairs(w.T, w.dil[h], w.win[h])
+        if w.recur[h]:
+            scan_bytes += w.B * w.T * w.d * 5 * elt
+    return flops, scan_bytes
+
+
+def decode_bytes(B, H, d, t, dil, win, elt=2):
+    """Algorithmic HBM bytes of one decode step at position t: every attended
+    cache row read once (K~ and V~), plus the token's q,k,v,g, o, the fp32 state
+    read+write and the new cache row."""
+    rows = 0
+    for h in range(H):
+        rows += t // dil[h] + (min(win[h], t + 1) - 1 if win[h] > 0 else 0)
+    return B * (rows * 2 * d * elt + H * d * (5 * elt + 16 + 2 * elt))
+
+
+# --------------------------------------------------------------- prefill
+
+
+def bench_prefill(rat, w, steps, warmup, world, rank, dev, e2e_steps):
+    dtype = w.torch_dtype
+    q, k, v, g = wl.prefill_inputs(w.B, w.T, w.H, w.d, w.gate_mean, dtype, device=dev, seed=rank)
+    cfg = rat.Config(w.B, w.T, w.H, w.d, dtype, w.dil, w.win, w.recur)
+    kt, vt = torch.empty_like(k), torch.empty_like(v)
+    o = torch.empty_like(q)
+    lse = torch.empty(w.B, w.H, w.T, dtype=torch.float32, device=dev)
+    fk = torch.empty(w.B, w.H, w.d, dtype=torch.float32, device=dev)
+    fv = torch.empty_like(fk)
+    ws = rat.workspace(cfg, rat.RAT_OP_MIX_CALLER_KV, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        rat.rat_scan_prefill(cfg, k, v, g, None, None, kt, vt, fk, fv, ws=ws, stream=stream)
+        if evs:
+            evs[1].record(stream)
+        rat.rat_dilated_attn_prefill(cfg, q, kt, vt, o, lse, ws=ws, stream=stream)
+        if evs:
+            evs[2].record(stream)
+
+    for _ in range(warmup):
+        step()
+    rat.rat_check_status(ws)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = rat.rat_launch_count()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(steps):
+            step(evs[i])
+        torch.cuda.synchronize()
+    launches = rat.rat_launch_count() - n0
+    barrier(world)
+    rat.rat_check_status(ws)
+    scan_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    total_ms = evs[0][0].elapsed_time(evs[-1][2])
+    total_ms = max_over_ranks(total_ms, world, dev)
+    res = dict(total_ms=total_ms, scan_ms=float(np.mean(scan_ms)), attn_ms=float(np.mean(attn_ms)),
+               launches=launches, clocks=clk.summary())
+
+    # end to end through the user call with host buffers: H2D of q,k,v,g from
+    # pinned memory, rat_mix_prefill, D2H of o
+    if e2e_steps > 0:
+        hq, hk, hv, hg = (x.cpu().pin_memory() for x in (q, k, v, g))
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        wsm = rat.workspace(cfg, rat.RAT_OP_MIX, device=dev)
+        del kt, vt
+        torch.cuda.empty_cache()
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            g.copy_(hg, non_blocking=True)
+            rat.rat_mix_prefill(cfg, q, k, v, g, None, None, o, None, None, None, fk, fv, ws=wsm, stream=stream)
+            ho.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        rat.rat_check_status(wsm)
+        e_ms = max_over_ranks(a.elapsed_time(b), world, dev) / e2e_steps
+        res["e2e_ms"] = e_ms
+        res["h2d_bytes"] = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg))
+        res["d2h_bytes"] = ho.numel() * ho.element_size()
+        del wsm, hq, hk, hv, hg, ho
+    del q, k, v, g, o, lse, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+# ---------------------------------------------------------------- decode
+
+
+def bench_decode(rat, w, ctx, steps, warmup, world, rank, dev, fill_chunk=8):
+    """Fill the cache of `ctx` tokens with batch-chunked rat_scan_prefill, then
+    time `steps` decode steps (positions ctx+warmup .. )."""
+    dtype = w.torch_dtype
+    B = w.decode_batch
+    cap = ctx + warmup + steps
+    cfg = rat.Config(B, ctx, w.H, w.d, dtype, w.dil, w.win, w.recur)
+    R = rat.rat_cache_rows(cfg, cap)
+    ck = torch.empty(B, w.H, R, w.d, dtype=dtype, device=dev)
+    cv = torch.empty_like(ck)
+    sk = torch.empty(B, w.H, w.d, dtype=torch.float32, device=dev)
+    sv = torch.empty_like(sk)
+    ccfg = rat.Config(fill_chunk, ctx, w.H, w.d, dtype, w.dil, w.win, w.recur)
+    wsc = rat.workspace(ccfg, rat.RAT_OP_SCAN, device=dev)
+    per_b = w.H * R * w.d
+    for b0 in range(0, B, fill_chunk):
+        k, v, g = wl.prefill_inputs(fill_chunk, ctx, w.H, w.d, w.gate_mean, dtype, device=dev,
+                                    seed=1000 + rank * 997 + b0)[1:]
+        rat.rat_scan_prefill(ccfg, k, v, g, None, None, None, None, sk[b0:b0 + fill_chunk], sv[b0:b0 + fill_chunk],
+                             ck.view(-1)[b0 * per_b:(b0 + fill_chunk) * per_b],
+                             cv.view(-1)[b0 * per_b:(b0 + fill_chunk) * per_b], cap, ws=wsc)
+        del k, v, g
+    rat.rat_check_status(wsc)
+    del wsc
+    n = warmup + steps
+    toks = [wl.token_inputs(B, w.H, w.d, w.gate_mean, dtype, device=dev, seed=5000 + i) for i in range(n)]
+    poss = [torch.full((B,), ctx + i, dtype=torch.int32, device=dev) for i in range(n)]
+    o = torch.empty(B, w.H, w.d, dtype=dtype, device=dev)
+    wsd = rat.workspace(cfg, rat.RAT_OP_DECODE, cap, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        tq, tk, tv, tg = toks[i]
+        rat.rat_decode_step(cfg, tq, tk, tv, tg, sk, sv, ck, cv, cap, poss[i], o, None, ws=wsd, stream=stream)
+
+    for i in range(warmup):
+        step(i)
+    rat.rat_check_status(wsd)
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = rat.rat_launch_count()
+    a.record(stream)
+    for i in range(warmup, n):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    launches = rat.rat_launch_count() - n0
+    rat.rat_check_status(wsd)
+    ms = max_over_ranks(a.elapsed_time(b), world, dev) / steps
+    t_mid = ctx + warmup + steps // 2
+    byts = decode_bytes(B, w.H, w.d, t_mid, w.dil, w.win)
+    del ck, cv, toks
+    torch.cuda.empty_cache()
+    return dict(ms=ms, bytes=byts, launches=launches, ctx=ctx)
+
+
+# ------------------------------------------------------------ CPU oracle
+
+
+def oracle_sample(w, n_rows, seed=0, rows_offset=0.5):
+    """Time the CPU oracle on head 0 of the workload: the full-length scan of k
+    and v, then `n_rows` query rows spread evenly over T.  Returns the
+    extrapolated whole-operator throughput (tokens/s over all heads)."""
+    import oracle
+
+    q, k, v, g = wl.prefill_inputs(w.B, w.T, 1, w.d, w.gate_mean, w.torch_dtype, device="cpu", seed=seed)
+    f = lambda x: x.float().numpy().astype(np.float64)
+    q, k, v, g = f(q), f(k), f(v), f(g)
+    t0 = time.perf_counter()
+    kt, _ = oracle.scan(k, g, None, [w.recur[0]])
+    vt, _ = oracle.scan(v, g, None, [w.recur[0]])
+    t_scan = time.perf_counter() - t0
+    ts = ((np.arange(n_rows) + rows_offset) * w.T / n_rows).astype(np.int64)
+    rows = np.stack([np.zeros_like(ts), np.zeros_like(ts), ts], axis=1)
+    t0 = time.perf_counter()
+    oracle.attn_rows(q, kt, vt, [w.dil[0]], [w.win[0]], rows, parts=3)
+    t_rows = time.perf_counter() - t0
+    per_head = t_scan + t_rows * (w.T / n_rows)
+    tok_s = w.B * w.T / (per_head * w.H)
+    return tok_s, t_scan + t_rows
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle as it stands, rank 0 only."""
+    if rank != 0:
+        return
+    w = wl.PREFILL_262K
+    n_rows = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample(w, max(16, n_rows // 8))
+    vals, secs = [], []
+    for i in range(args.steps):
+        v, s = oracle_sample(w, n_rows, rows_offset=(i % 4 + 0.5) / 4)
+        vals.append(v)
+        secs.append(s)
+    value = float(np.mean(vals))
+    cores = host_cores()
+    sample = ("head 0 of %d: full scan of k and v over T=%d plus %d query rows spread over T per step; "
+              "extrapolated to all heads" % (w.H, w.T, n_rows))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": float(np.mean(secs)) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.T, "parallelism": "host threads"},
+            "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-ctx", type=str, default="4096,16384,32768")
+    ap.add_argument("--decode-steps", type=int, default=64)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-rows", type=int, default=2048, help="oracle rows timed for cpu_baseline")
+    ap.add_argument("--ref-rows", type=int, default=512, help="oracle rows per reference-arm step")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        init_dist(world, "gloo")
+        run_reference(args, world, rank)
+        return
+
+    import recurrence_augmented_dilated_gated_b200 as rat
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    rat.load_library()
+    peaks = load_peaks()
+
+    w = wl.PREFILL_262K
+    pre = bench_prefill(rat, w, args.steps, args.warmup, world, rank, dev, args.e2e_steps)
+    flops, scan_bytes = prefill_work(w)
+    tokens = w.B * w.T * world
+    step_ms = pre["total_ms"] / args.steps
+    value = tokens / (step_ms * 1e-3)
+
+    dec = []
+    for ctx in [int(c) for c in args.decode_ctx.split(",") if c]:
+        dec.append(bench_decode(rat, wl.DECODE_D16, ctx, args.decode_steps, args.warmup, world, rank, dev))
+
+    if rank != 0:
+        return
+    attn_tflops = flops / (pre["attn_ms"] * 1e-3) / 1e12
+    scan_gbs = scan_bytes / (pre["scan_ms"] * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tok/s",
+        "value_is": "prefill tokens/s of the whole operator (scan + dilated/window attention) at T=262144",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (q,k,v ~ N(0,1), gate logits ~ N(2,1), seeded)",
+        "config": {"workload": w.name, "global_batch": w.B * world, "seq_len": w.T,
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (4.3 GB per step), no flush"},
+        "roofline": {"bound": "tensor", "kernel": "attention (dilated + window + LSE merge)",
+                     "achieved": attn_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": attn_tflops / peaks["bf16_tflops"],
+                     "traffic": profile_traffic("attn_prefill262k"),
+                     "algorithmic": "%.4g FLOP per launch (4*d per unmasked pair)" % flops,
+                     "peak_source": peaks["_source"] + " bf16 dense burst"},
+        "scan_roofline": {"bound": "hbm", "achieved": scan_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                          "frac": scan_gbs / peaks["hbm_gbs"], "traffic": profile_traffic("scan_prefill262k"),
+                          "algorithmic": "%.4g bytes per launch (10 B per token-channel)" % scan_bytes,
+                          "peak_source": peaks["_source"] + " copy"},
+        "kernels_ms": {"scan": pre["scan_ms"], "attention": pre["attn_ms"]},
+        "gpu_launches": pre["launches"],
+        "clocks": pre["clocks"],
+    }
+    if "e2e_ms" in pre:
+        line["e2e"] = {"value": tokens / (pre["e2e_ms"] * 1e-3), "unit": "tok/s",
+                       "h2d_bytes_per_step": pre["h2d_bytes"], "d2h_bytes_per_step": pre["d2h_bytes"],
+                       "call": "rat_mix_prefill with pinned-host inputs copied in and o copied out every step"}
+    if dec:
+        wd = wl.DECODE_D16
+        line["decode"] = {
+            "metric": "decode tok/s (batch %d, H%d d%d D%d)" % (wd.decode_batch, wd.H, wd.d, wd.dil[0]),
+            "unit": "tok/s",
+            "steps": args.decode_steps,
+            "by_ctx": [{"ctx": r["ctx"], "value": wd.decode_batch * world / (r["ms"] * 1e-3), "ms_per_step": r["ms"],
+                        "roofline": {"bound": "hbm", "achieved": r["bytes"] / (r["ms"] * 1e-3) / 1e9,
+                                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                     "frac": r["bytes"] / (r["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                     "traffic": profile_traffic("decode_ctx%d" % r["ctx"])},
+                        "gpu_launches": r["launches"]} for r in dec],
+        }
+    if not args.no_cpu and world == 1:
+        v, secs = oracle_sample(w, args.cpu_rows)
+        line["cpu_baseline"] = {"value": v, "unit": "tok/s", "cores": host_cores(), "kind": "oracle",
+                                "sample": "head 0 of %d: full scan over T=%d + %d query rows spread over T "
+                                          "(%.1f s); extrapolated to all heads" % (w.H, w.T, args.cpu_rows, secs)}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

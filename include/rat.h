@@ -1,0 +1,227 @@
+/*
+ * rat.h -- C ABI of librat.so, the B200 (sm_100a) implementation of the RAT+
+ * temporal-mixing operator: a per-channel gated linear recurrence over keys and
+ * values, then causal softmax attention over the recurrence-augmented keys and
+ * values with dilation D and an optional dense local window W, the two parts
+ * merged by log-sum-exp.
+ *
+ * Sources (page titles and the passages each entry point follows):
+ *   "RAT+: Train Dense, Infer Sparse -- Recurrence Augmented Attention for
+ *    Dilated Inference": Abstract (dilated attention cuts attention FLOPs and
+ *    KV cache by D; optional local windows; hybrid head compositions),
+ *    Figure 1(a) (full-sequence recurrence, L = T), Figure 1(c) (dilated
+ *    attention with optional local attention), Figure 2 (prefill = scan of the
+ *    recurrence + dilated attention; decode = a step update of the recurrence
+ *    + attention over the cache), Figure 9 (non-zero initial cell state).
+ *   "Augmenting Attention with Exponentially Decaying Memory Improves
+ *    Query-Aware KV Sparsity", section 2.1 (key and value states updated with
+ *    an input-dependent gate; O(1) extra compute and storage per token).
+ *
+ * Definitions used by every entry point (the pages give the method at the
+ * level of captions; these are the plain readings of them):
+ *   recurrence   s_t = a_t * s_{t-1} + (1 - a_t) * x_t per channel, for x = k
+ *                and x = v, with a_t = sigmoid(g_t) from one gate tensor g;
+ *                s_{-1} = init (zero when not given).  A head with recur = 0
+ *                has a = 0: its augmented keys/values are the raw ones.
+ *   dilation     query t attends to { j <= t : (t - j) mod D == 0 }.
+ *   window       W > 0 adds a second softmax over { max(0, t-W+1) <= j <= t }.
+ *   merge        the two softmaxes are merged by log-sum-exp (a key in both
+ *                sets counts in both).
+ *   scale        scores are scale * <q_t, k~_j>, scale = 1/sqrt(d) by default.
+ *
+ * Conventions shared by all calls
+ *   - Tensors are dense row-major.  Token tensors are [B, T, H, d] (d fastest);
+ *     lse is [B, H, T] fp32; states are [B, H, d] fp32.
+ *   - Element type of q/k/v/g/o/kt/vt/cache is cfg->dtype (RAT_BF16 or
+ *     RAT_F32).  States, init and lse are always fp32.
+ *   - Every device pointer must be 16-byte aligned.
+ *   - Ownership: the caller owns every buffer and the stream.  The library
+ *     allocates no device memory, keeps no global state and may be called from
+ *     several host threads on different workspaces.  Calls are asynchronous on
+ *     `stream`; inputs must stay valid until the stream reaches the call.
+ *   - Workspace: `ws` is caller-allocated device memory of at least
+ *     rat_workspace_size() bytes, zero-filled once before its first use
+ *     (rat_workspace_init does that).  Calls that share a workspace must be
+ *     ordered on one stream.
+ *   - Errors: argument errors return RAT_ERR_INVALID / RAT_ERR_UNSUPPORTED /
+ *     RAT_ERR_WORKSPACE before anything is launched.  A failed launch returns
+ *     RAT_ERR_CUDA.  A device-side error (a bounded wait that gave up) is
+ *     recorded in the workspace and returned by rat_check_status().
+ *     rat_last_error() gives a one-line reason for the calling thread's last
+ *     non-OK return.
+ */
+#ifndef RAT_H
+#define RAT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported symbol marker (the library is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define RAT_API __attribute__((visibility("default")))
+#else
+#define RAT_API
+#endif
+
+/* A cudaStream_t (same underlying type); NULL is the legacy default stream. */
+typedef struct CUstream_st *rat_stream_t;
+
+typedef enum {
+    RAT_OK = 0,
+    RAT_ERR_INVALID = 1,     /* null / misaligned pointer, out-of-range size or parameter */
+    RAT_ERR_UNSUPPORTED = 2, /* valid request with no kernel in this build (e.g. d not 64/128) */
+    RAT_ERR_CUDA = 3,        /* a CUDA runtime call or a kernel launch failed */
+    RAT_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up (rat_check_status) */
+    RAT_ERR_WORKSPACE = 5    /* ws_bytes below rat_workspace_size() */
+} rat_status;
+
+typedef enum { RAT_F32 = 0, RAT_BF16 = 1 } rat_dtype;
+
+/* Workspace requests (the `op` argument of rat_workspace_size). */
+typedef enum {
+    RAT_OP_SCAN = 0,          /* rat_scan_prefill */
+    RAT_OP_ATTN = 1,          /* rat_dilated_attn_prefill */
+    RAT_OP_MIX = 2,           /* rat_mix_prefill with kt = vt = NULL (K~/V~ kept in ws) */
+    RAT_OP_MIX_CALLER_KV = 3, /* rat_mix_prefill with caller-provided kt and vt */
+    RAT_OP_DECODE = 4         /* rat_decode_step */
+} rat_op;
+
+/*
+ * Operator configuration.  The per-head arrays are HOST memory, read during
+ * the call only.  Head h uses dilation dil[h] >= 1, window win[h] >= 0 (0 = no
+ * window) and recurrence flag recur[h] (0 = no recurrence; NULL = all heads
+ * recurrent) -- the hybrid head compositions of the RAT+ Abstract.
+ * Limits of this build: d in {64, 128}; 1 <= H <= 256; B, T >= 0;
+ * B*T*H*d < 2^40 elements.  An empty batch or sequence (B*T == 0) launches
+ * no kernel; a prefill then only copies init (or zero) to final.
+ */
+typedef struct {
+    int B, T, H, d;
+    int dtype;               /* rat_dtype */
+    const int32_t *dil;      /* host [H] */
+    const int32_t *win;      /* host [H] */
+    const uint8_t *recur;    /* host [H] or NULL */
+    float scale;             /* <= 0 selects 1/sqrt(d) */
+} rat_cfg;
+
+/* Bytes of workspace `op` needs for `cfg` (cache_cap: decode capacity, else
+ * ignored).  Returns 0 when cfg is invalid. */
+RAT_API size_t rat_workspace_size(const rat_cfg *cfg, int op, int cache_cap);
+
+/* Zero the workspace header (status word and debug fields). */
+RAT_API rat_status rat_workspace_init(void *ws, size_t ws_bytes, rat_stream_t stream);
+
+/*
+ * Decode cache layout ("dilated KV cache", RAT+ Abstract and Figure 2).
+ * A cache tensor is [B, H, R, d] in cfg->dtype with R = rat_cache_rows(cfg,
+ * cap).  Position j of head h is stored at row
+ *     (j mod D_h) * ceil(cap / D_h) + floor(j / D_h)
+ * i.e. residue-major: the rows a decode query at position t reads for its
+ * dilated part (all j == t mod D_h, j <= t) form one contiguous slab.
+ * Returns 0 when cfg or cap is invalid.
+ */
+RAT_API int64_t rat_cache_rows(const rat_cfg *cfg, int cap);
+
+/*
+ * Prefill recurrence (RAT+ Figure 1(a) and Figure 2 "associative scan";
+ * Exponentially Decaying Memory section 2.1).
+ *   k, v, g          in  [B,T,H,d]  keys, values, gate logits
+ *   init_k, init_v   in  [B,H,d] fp32 or NULL (zero initial state; RAT+ Figure 9)
+ *   kt, vt           out [B,T,H,d]  augmented keys/values, or NULL when a cache
+ *                        is given (recur = 0 heads receive a copy of k / v)
+ *   final_k, final_v out [B,H,d] fp32 s_{T-1}, or NULL
+ *   cache_k, cache_v out decode cache tensors (layout above) for positions
+ *                        0..T-1, or NULL; requires T <= cache_cap
+ * At least one of (kt, vt) or (cache_k, cache_v) must be given, as pairs.
+ */
+RAT_API rat_status rat_scan_prefill(const rat_cfg *cfg, const void *k, const void *v, const void *g,
+                            const float *init_k, const float *init_v, void *kt, void *vt,
+                            float *final_k, float *final_v, void *cache_k, void *cache_v,
+                            int cache_cap, void *ws, size_t ws_bytes, rat_stream_t stream);
+
+/*
+ * Attention step over augmented keys/values (RAT+ Abstract, Figure 1(c)):
+ * dilated causal attention, plus the local window for heads with win > 0,
+ * merged by log-sum-exp.
+ *   q, kt, vt  in  [B,T,H,d]
+ *   o          out [B,T,H,d]
+ *   lse        out [B,H,T] fp32 natural-log log-sum-exp of the merged softmax, or NULL
+ */
+RAT_API rat_status rat_dilated_attn_prefill(const rat_cfg *cfg, const void *q, const void *kt, const void *vt,
+                                    void *o, float *lse, void *ws, size_t ws_bytes,
+                                    rat_stream_t stream);
+
+/*
+ * The whole temporal-mixing operator for a prefill: rat_scan_prefill of k and
+ * v followed by rat_dilated_attn_prefill.  kt/vt may be NULL (kept in the
+ * workspace, size RAT_OP_MIX) or caller buffers (RAT_OP_MIX_CALLER_KV) that
+ * receive the augmented keys/values.  Heads with recur = 0 attend to k and v
+ * directly.  final_k/final_v (nullable) receive the recurrent state after
+ * token T-1, which a decode continues from.
+ */
+RAT_API rat_status rat_mix_prefill(const rat_cfg *cfg, const void *q, const void *k, const void *v,
+                           const void *g, const float *init_k, const float *init_v, void *o,
+                           float *lse, void *kt, void *vt, float *final_k, float *final_v,
+                           void *ws, size_t ws_bytes, rat_stream_t stream);
+
+/*
+ * One decode step for every batch entry (RAT+ Figure 2: "a simple step update"
+ * of the recurrence, then attention over the dilated KV cache).  cfg->T is
+ * ignored.  For batch entry b the new token is at position t = pos[b]:
+ *   1. s <- a*s + (1-a)*x for x = k and v (a = sigmoid(g), a = 0 if recur = 0),
+ *      updating state_k / state_v in place (fp32 [B,H,d]);
+ *   2. the new augmented key/value (rounded to cfg->dtype) is stored at t's
+ *      cache row;
+ *   3. o[b,h] = merged attention of q over the cache rows j <= t of the
+ *      dilated set (and window) of t.
+ *   q, k, v, g   in  [B,H,d]
+ *   cache_k/v    in/out [B,H,R,d], R = rat_cache_rows(cfg, cache_cap); rows of
+ *                positions < pos[b] must hold earlier augmented keys/values
+ *   pos          in  DEVICE int32 [B], 0 <= pos[b] < cache_cap (a position out
+ *                of range makes the kernel skip that entry and record
+ *                RAT_ERR_INVALID for rat_check_status)
+ *   o            out [B,H,d];  lse out [B,H] fp32 or NULL
+ */
+RAT_API rat_status rat_decode_step(const rat_cfg *cfg, const void *q, const void *k, const void *v,
+                           const void *g, float *state_k, float *state_v, void *cache_k,
+                           void *cache_v, int cache_cap, const int32_t *pos, void *o, float *lse,
+                           void *ws, size_t ws_bytes, rat_stream_t stream);
+
+/*
+ * Synchronises `stream`, returns the first device-side error recorded in `ws`
+ * since the last check (RAT_OK if none) and clears it.  RAT_ERR_CUDA if the
+ * synchronisation itself fails.
+ */
+RAT_API rat_status rat_check_status(void *ws, rat_stream_t stream);
+
+/* Static string for a status code. */
+RAT_API const char *rat_status_string(rat_status s);
+
+/* One-line reason for the calling thread's last non-OK return ("" if none). */
+RAT_API const char *rat_last_error(void);
+
+/* ABI version of this header (major * 100 + minor). */
+RAT_API int rat_version(void);
+
+/* Number of kernels this library has launched in this process so far. */
+RAT_API long long rat_launch_count(void);
+
+/*
+ * Failure-injection hooks for tests of the bounded device-side waits.
+ * rat_debug_set_scan_stall makes scan chunk `ticket` (0-based launch order;
+ * -1 = off) never publish its carry, so the chunks after it must give up after
+ * `spin_limit_ns` (0 = the default of one second) and record RAT_ERR_TIMEOUT.
+ * Stored in the workspace header; no effect on other workspaces.
+ */
+RAT_API rat_status rat_debug_set_scan_stall(void *ws, size_t ws_bytes, int64_t ticket, int64_t spin_limit_ns,
+                                    rat_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RAT_H */

@@ -13,7 +13,7 @@ import os
 
 import numpy as np
 
-from .build import build
+from .build import build as build_library
 
 _lib = None
 
@@ -23,7 +23,7 @@ def _load():
     if _lib is None:
         # RAT_ORACLE_LIB points at another build of rat_oracle.c (the mutation
         # test loads deliberately broken copies through it).
-        path = os.environ.get("RAT_ORACLE_LIB") or build()
+        path = os.environ.get("RAT_ORACLE_LIB") or build_library()
         lib = ctypes.CDLL(path)
         dp = ctypes.POINTER(ctypes.c_double)
         ip = ctypes.POINTER(ctypes.c_int)

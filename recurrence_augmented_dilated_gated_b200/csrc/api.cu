@@ -1,0 +1,409 @@
+// api.cu -- the C ABI of librat.so (declared in include/rat.h): argument
+// checks, workspace layout and kernel dispatch.  Every step of the operator
+// runs in this library's kernels; there is no host or library fallback.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <atomic>
+
+#include "rat_internal.cuh"
+
+using namespace rat;
+
+namespace rat {
+static std::atomic<long long> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+}  // namespace rat
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+rat_status fail(rat_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+rat_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(RAT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+size_t elt_size(int dtype) { return dtype == RAT_F32 ? 4 : 2; }
+
+// scan geometry: 256 threads, d/4 threads per token row, 16 tokens per group
+constexpr int kScanSub = 16;
+int scan_chunk_len(int d) { return (256 / (d / 4)) * kScanSub; }
+
+constexpr int kDecodeRowsPerSplit = 1024;
+
+rat_status check_cfg(const rat_cfg *c, bool need_T = true) {
+    if (!c) return fail(RAT_ERR_INVALID, "cfg is NULL");
+    if (c->B < 0 || c->H < 1 || c->d < 1 || (need_T && c->T < 0))
+        return fail(RAT_ERR_INVALID, "need B >= 0, T >= 0, H >= 1, d >= 1 (B=%d T=%d H=%d d=%d)", c->B, c->T,
+                    c->H, c->d);
+    if (c->H > kMaxHeads) return fail(RAT_ERR_UNSUPPORTED, "H=%d exceeds %d heads", c->H, kMaxHeads);
+    if (c->d != 64 && c->d != 128) return fail(RAT_ERR_UNSUPPORTED, "head_dim d=%d (supported: 64, 128)", c->d);
+    if (c->dtype != RAT_F32 && c->dtype != RAT_BF16) return fail(RAT_ERR_INVALID, "dtype %d", c->dtype);
+    if (!c->dil || !c->win) return fail(RAT_ERR_INVALID, "cfg->dil / cfg->win is NULL");
+    for (int h = 0; h < c->H; ++h) {
+        if (c->dil[h] < 1) return fail(RAT_ERR_INVALID, "dil[%d]=%d < 1", h, c->dil[h]);
+        if (c->win[h] < 0) return fail(RAT_ERR_INVALID, "win[%d]=%d < 0", h, c->win[h]);
+    }
+    const double elems = (double)c->B * (need_T ? (double)c->T : 1.0) * c->H * c->d;
+    if (elems >= 1099511627776.0) return fail(RAT_ERR_INVALID, "B*T*H*d too large");
+    if (!(c->scale == c->scale)) return fail(RAT_ERR_INVALID, "scale is NaN");
+    return RAT_OK;
+}
+
+bool head_recur(const rat_cfg *c, int h) { return c->recur == nullptr || c->recur[h] != 0; }
+
+float scale_of(const rat_cfg *c) { return c->scale > 0.f ? c->scale : 1.0f / sqrtf((float)c->d); }
+
+int64_t cache_rows(const rat_cfg *c, int cap) {
+    int64_t R = 0;
+    for (int h = 0; h < c->H; ++h) {
+        const int64_t D = c->dil[h];
+        R = std::max<int64_t>(R, D * ((cap + D - 1) / D));
+    }
+    return R;
+}
+
+struct Layout {
+    size_t ticket = 0, flags = 0, agg = 0, incl = 0;  // scan
+    size_t lse_dil = 0;                               // attention
+    size_t kt = 0, vt = 0;                            // mix scratch
+    size_t part = 0;                                  // decode
+    int nchunks = 0, items_per_b = 0;
+    size_t total = 0;
+};
+
+int decode_items(const rat_cfg *c, int cap, int *nsplit, int *item0) {
+    int items = 0;
+    for (int h = 0; h < c->H; ++h) {
+        const int slab = (cap + c->dil[h] - 1) / c->dil[h];
+        const int ns = (slab + kDecodeRowsPerSplit - 1) / kDecodeRowsPerSplit;
+        if (nsplit) nsplit[h] = ns;
+        if (item0) item0[h] = items;
+        items += ns + 1;
+    }
+    if (item0) item0[c->H] = items;
+    return items;
+}
+
+Layout layout(const rat_cfg *c, int op, int cap) {
+    Layout L;
+    size_t off = sizeof(WsHeader);
+    const size_t elt = elt_size(c->dtype);
+    if (op == RAT_OP_SCAN || op == RAT_OP_MIX || op == RAT_OP_MIX_CALLER_KV) {
+        const int clen = scan_chunk_len(c->d);
+        L.nchunks = (c->T + clen - 1) / clen;
+        const size_t units = (size_t)c->B * c->H * L.nchunks;
+        L.ticket = off; off += 256;
+        L.flags = off; off = align256(off + units * sizeof(int));
+        L.agg = off; off = align256(off + units * 3 * c->d * sizeof(float));
+        L.incl = off; off = align256(off + units * 2 * c->d * sizeof(float));
+    }
+    if (op == RAT_OP_ATTN || op == RAT_OP_MIX || op == RAT_OP_MIX_CALLER_KV) {
+        L.lse_dil = off; off = align256(off + (size_t)c->B * c->H * c->T * sizeof(float));
+    }
+    if (op == RAT_OP_MIX) {
+        const size_t bytes = (size_t)c->B * c->T * c->H * c->d * elt;
+        L.kt = off; off = align256(off + bytes);
+        L.vt = off; off = align256(off + bytes);
+    }
+    if (op == RAT_OP_DECODE) {
+        L.items_per_b = decode_items(c, cap, nullptr, nullptr);
+        L.part = off; off = align256(off + (size_t)c->B * L.items_per_b * (c->d + 2) * sizeof(float));
+    }
+    L.total = off;
+    return L;
+}
+
+rat_status check_ws(const rat_cfg *c, int op, int cap, void *ws, size_t ws_bytes, Layout *L) {
+    if (!ws) return fail(RAT_ERR_INVALID, "workspace is NULL");
+    if (((uintptr_t)ws & 255u) != 0) return fail(RAT_ERR_INVALID, "workspace must be 256-byte aligned");
+    *L = layout(c, op, cap);
+    if (ws_bytes < L->total)
+        return fail(RAT_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, L->total);
+    return RAT_OK;
+}
+
+#define CHECK_PTR(p, name)                                                                   \
+    do {                                                                                     \
+        if (!(p)) return fail(RAT_ERR_INVALID, "%s is NULL", name);                         \
+        if (!aligned16(p)) return fail(RAT_ERR_INVALID, "%s is not 16-byte aligned", name); \
+    } while (0)
+#define CHECK_OPT(p, name)                                                                   \
+    do {                                                                                     \
+        if ((p) && !aligned16(p)) return fail(RAT_ERR_INVALID, "%s is not 16-byte aligned", name); \
+    } while (0)
+
+bool empty(const rat_cfg *c) { return (size_t)c->B * (size_t)c->T == 0; }
+
+// An empty prefill leaves the state where it was: final = init (or zero).
+rat_status empty_prefill_state(const rat_cfg *c, const float *ik, const float *iv, float *fk, float *fv,
+                               cudaStream_t s) {
+    const size_t bytes = (size_t)c->B * c->H * c->d * sizeof(float);
+    if (bytes == 0) return RAT_OK;
+    const float *src[2] = {ik, iv};
+    float *dst[2] = {fk, fv};
+    for (int i = 0; i < 2; ++i) {
+        if (!dst[i]) continue;
+        cudaError_t e = src[i] ? cudaMemcpyAsync(dst[i], src[i], bytes, cudaMemcpyDeviceToDevice, s)
+                               : cudaMemsetAsync(dst[i], 0, bytes, s);
+        if (e != cudaSuccess) return cuda_fail(e, "empty prefill state copy");
+    }
+    return RAT_OK;
+}
+
+// Scan of the selected heads into kt/vt and/or the cache.
+rat_status run_scan(const rat_cfg *c, const Layout &L, const void *k, const void *v, const void *g,
+                    const float *ik, const float *iv, void *kt, void *vt, float *fk, float *fv,
+                    void *ck, void *cv, int cap, char *ws, bool only_recurrent, cudaStream_t s) {
+    ScanParams p;
+    memset(&p, 0, sizeof(p));
+    p.x[0] = k; p.x[1] = v; p.g = g;
+    p.init[0] = ik; p.init[1] = iv;
+    p.out[0] = kt; p.out[1] = vt;
+    p.fin[0] = fk; p.fin[1] = fv;
+    p.cache[0] = ck; p.cache[1] = cv;
+    p.cap = cap;
+    p.cache_R = ck ? cache_rows(c, cap) : 0;
+    p.B = c->B; p.T = c->T; p.H = c->H; p.d = c->d;
+    int n = 0;
+    for (int h = 0; h < c->H; ++h) {
+        p.head_recur[h] = head_recur(c, h) ? 1 : 0;
+        p.head_dil[h] = c->dil[h];
+        if (!only_recurrent || p.head_recur[h]) p.head_list[n++] = (unsigned char)h;
+    }
+    if (n == 0) return RAT_OK;
+    p.nheads = n;
+    p.nslices = c->B * n;
+    p.nchunks = L.nchunks;
+    p.chunk_len = scan_chunk_len(c->d);
+    p.sub_len = kScanSub;
+    p.ticket = reinterpret_cast<unsigned *>(ws + L.ticket);
+    p.flags = reinterpret_cast<int *>(ws + L.flags);
+    p.agg = reinterpret_cast<float *>(ws + L.agg);
+    p.incl = reinterpret_cast<float *>(ws + L.incl);
+    p.hdr = reinterpret_cast<WsHeader *>(ws);
+    // zero the ticket and the chunk flags (one contiguous range)
+    cudaError_t e = cudaMemsetAsync(ws + L.ticket, 0, L.agg - L.ticket, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(scan flags)");
+    e = launch_scan(p, c->dtype, s);
+    if (e != cudaSuccess) return cuda_fail(e, "scan launch");
+    return RAT_OK;
+}
+
+rat_status run_attn(const rat_cfg *c, const Layout &L, const void *q, const void *kt, const void *vt,
+                    const void *kraw, const void *vraw, bool raw_for_plain_heads, void *o, float *lse,
+                    char *ws, cudaStream_t s) {
+    AttnParams p;
+    memset(&p, 0, sizeof(p));
+    p.q = q; p.kt = kt; p.vt = vt; p.kraw = kraw; p.vraw = vraw;
+    p.o = o; p.lse = lse;
+    p.B = c->B; p.T = c->T; p.H = c->H; p.d = c->d;
+    p.scale_log2 = scale_of(c) * 1.4426950408889634f;
+    for (int h = 0; h < c->H; ++h) {
+        p.dil[h] = c->dil[h];
+        p.win[h] = c->win[h];
+        p.use_raw[h] = (raw_for_plain_heads && !head_recur(c, h)) ? 1 : 0;
+    }
+    p.hdr = reinterpret_cast<WsHeader *>(ws);
+    (void)L;
+    cudaError_t e = launch_attn_simt(p, c->dtype, s);
+    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    return RAT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int rat_version(void) { return 100; }
+
+long long rat_launch_count(void) { return rat::g_launches.load(std::memory_order_relaxed); }
+
+const char *rat_last_error(void) { return g_last_error; }
+
+const char *rat_status_string(rat_status s) {
+    switch (s) {
+    case RAT_OK: return "RAT_OK";
+    case RAT_ERR_INVALID: return "RAT_ERR_INVALID: invalid argument";
+    case RAT_ERR_UNSUPPORTED: return "RAT_ERR_UNSUPPORTED: no kernel for this configuration";
+    case RAT_ERR_CUDA: return "RAT_ERR_CUDA: CUDA runtime or launch failure";
+    case RAT_ERR_TIMEOUT: return "RAT_ERR_TIMEOUT: a bounded device-side wait gave up";
+    case RAT_ERR_WORKSPACE: return "RAT_ERR_WORKSPACE: workspace too small";
+    }
+    return "unknown rat_status";
+}
+
+size_t rat_workspace_size(const rat_cfg *cfg, int op, int cache_cap) {
+    if (op < RAT_OP_SCAN || op > RAT_OP_DECODE) return 0;
+    if (check_cfg(cfg, op != RAT_OP_DECODE) != RAT_OK) return 0;
+    if (op == RAT_OP_DECODE && cache_cap < 1) return 0;
+    return layout(cfg, op, cache_cap).total;
+}
+
+rat_status rat_workspace_init(void *ws, size_t ws_bytes, rat_stream_t stream) {
+    if (!ws || ws_bytes < sizeof(WsHeader)) return fail(RAT_ERR_INVALID, "workspace NULL or < 256 bytes");
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(WsHeader), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(workspace header)");
+    return RAT_OK;
+}
+
+int64_t rat_cache_rows(const rat_cfg *cfg, int cap) {
+    if (check_cfg(cfg, false) != RAT_OK || cap < 1) return 0;
+    return cache_rows(cfg, cap);
+}
+
+rat_status rat_scan_prefill(const rat_cfg *cfg, const void *k, const void *v, const void *g,
+                            const float *init_k, const float *init_v, void *kt, void *vt,
+                            float *final_k, float *final_v, void *cache_k, void *cache_v,
+                            int cache_cap, void *ws, size_t ws_bytes, rat_stream_t stream) {
+    rat_status st = check_cfg(cfg);
+    if (st != RAT_OK) return st;
+    CHECK_OPT(init_k, "init_k"); CHECK_OPT(init_v, "init_v");
+    CHECK_OPT(final_k, "final_k"); CHECK_OPT(final_v, "final_v");
+    if (empty(cfg)) return empty_prefill_state(cfg, init_k, init_v, final_k, final_v, (cudaStream_t)stream);
+    CHECK_PTR(k, "k"); CHECK_PTR(v, "v"); CHECK_PTR(g, "g");
+    CHECK_OPT(init_k, "init_k"); CHECK_OPT(init_v, "init_v");
+    CHECK_OPT(kt, "kt"); CHECK_OPT(vt, "vt");
+    CHECK_OPT(final_k, "final_k"); CHECK_OPT(final_v, "final_v");
+    CHECK_OPT(cache_k, "cache_k"); CHECK_OPT(cache_v, "cache_v");
+    if ((kt == nullptr) != (vt == nullptr)) return fail(RAT_ERR_INVALID, "kt and vt must be given together");
+    if ((cache_k == nullptr) != (cache_v == nullptr))
+        return fail(RAT_ERR_INVALID, "cache_k and cache_v must be given together");
+    if (!kt && !cache_k) return fail(RAT_ERR_INVALID, "no output: give kt/vt and/or cache_k/cache_v");
+    if (cache_k && cache_cap < cfg->T) return fail(RAT_ERR_INVALID, "cache_cap %d < T %d", cache_cap, cfg->T);
+    Layout L;
+    st = check_ws(cfg, RAT_OP_SCAN, 0, ws, ws_bytes, &L);
+    if (st != RAT_OK) return st;
+    return run_scan(cfg, L, k, v, g, init_k, init_v, kt, vt, final_k, final_v, cache_k, cache_v,
+                    cache_cap, static_cast<char *>(ws), false, (cudaStream_t)stream);
+}
+
+rat_status rat_dilated_attn_prefill(const rat_cfg *cfg, const void *q, const void *kt, const void *vt,
+                                    void *o, float *lse, void *ws, size_t ws_bytes, rat_stream_t stream) {
+    rat_status st = check_cfg(cfg);
+    if (st != RAT_OK) return st;
+    if (empty(cfg)) return RAT_OK;
+    CHECK_PTR(q, "q"); CHECK_PTR(kt, "kt"); CHECK_PTR(vt, "vt"); CHECK_PTR(o, "o");
+    CHECK_OPT(lse, "lse");
+    Layout L;
+    st = check_ws(cfg, RAT_OP_ATTN, 0, ws, ws_bytes, &L);
+    if (st != RAT_OK) return st;
+    return run_attn(cfg, L, q, kt, vt, nullptr, nullptr, false, o, lse, static_cast<char *>(ws),
+                    (cudaStream_t)stream);
+}
+
+rat_status rat_mix_prefill(const rat_cfg *cfg, const void *q, const void *k, const void *v,
+                           const void *g, const float *init_k, const float *init_v, void *o,
+                           float *lse, void *kt, void *vt, float *final_k, float *final_v,
+                           void *ws, size_t ws_bytes, rat_stream_t stream) {
+    rat_status st = check_cfg(cfg);
+    if (st != RAT_OK) return st;
+    CHECK_OPT(init_k, "init_k"); CHECK_OPT(init_v, "init_v");
+    CHECK_OPT(final_k, "final_k"); CHECK_OPT(final_v, "final_v");
+    if (empty(cfg)) return empty_prefill_state(cfg, init_k, init_v, final_k, final_v, (cudaStream_t)stream);
+    CHECK_PTR(q, "q"); CHECK_PTR(k, "k"); CHECK_PTR(v, "v"); CHECK_PTR(g, "g"); CHECK_PTR(o, "o");
+    CHECK_OPT(lse, "lse");
+    CHECK_OPT(kt, "kt"); CHECK_OPT(vt, "vt");
+    CHECK_OPT(final_k, "final_k"); CHECK_OPT(final_v, "final_v");
+    if ((kt == nullptr) != (vt == nullptr)) return fail(RAT_ERR_INVALID, "kt and vt must be given together");
+    const bool caller_kv = kt != nullptr;
+    Layout L;
+    st = check_ws(cfg, caller_kv ? RAT_OP_MIX_CALLER_KV : RAT_OP_MIX, 0, ws, ws_bytes, &L);
+    if (st != RAT_OK) return st;
+    char *w = static_cast<char *>(ws);
+    if (!caller_kv) {
+        kt = w + L.kt;
+        vt = w + L.vt;
+    }
+    const cudaStream_t s = (cudaStream_t)stream;
+    // Heads without recurrence attend to k/v directly, unless the caller asked
+    // for the complete augmented tensors.
+    st = run_scan(cfg, L, k, v, g, init_k, init_v, kt, vt, final_k, final_v, nullptr, nullptr, 0, w,
+                  !caller_kv, s);
+    if (st != RAT_OK) return st;
+    return run_attn(cfg, L, q, kt, vt, k, v, !caller_kv, o, lse, w, s);
+}
+
+rat_status rat_decode_step(const rat_cfg *cfg, const void *q, const void *k, const void *v,
+                           const void *g, float *state_k, float *state_v, void *cache_k,
+                           void *cache_v, int cache_cap, const int32_t *pos, void *o, float *lse,
+                           void *ws, size_t ws_bytes, rat_stream_t stream) {
+    rat_status st = check_cfg(cfg, false);
+    if (st != RAT_OK) return st;
+    if (cfg->B == 0) return RAT_OK;
+    CHECK_PTR(q, "q"); CHECK_PTR(k, "k"); CHECK_PTR(v, "v"); CHECK_PTR(g, "g");
+    CHECK_PTR(state_k, "state_k"); CHECK_PTR(state_v, "state_v");
+    CHECK_PTR(cache_k, "cache_k"); CHECK_PTR(cache_v, "cache_v");
+    CHECK_PTR(pos, "pos"); CHECK_PTR(o, "o"); CHECK_OPT(lse, "lse");
+    if (cache_cap < 1) return fail(RAT_ERR_INVALID, "cache_cap %d < 1", cache_cap);
+    Layout L;
+    st = check_ws(cfg, RAT_OP_DECODE, cache_cap, ws, ws_bytes, &L);
+    if (st != RAT_OK) return st;
+    DecodeParams p;
+    memset(&p, 0, sizeof(p));
+    p.q = q; p.k = k; p.v = v; p.g = g;
+    p.state[0] = state_k; p.state[1] = state_v;
+    p.cache[0] = cache_k; p.cache[1] = cache_v;
+    p.pos = pos; p.o = o; p.lse = lse;
+    p.part = reinterpret_cast<float *>(static_cast<char *>(ws) + L.part);
+    p.cache_R = cache_rows(cfg, cache_cap);
+    p.cap = cache_cap; p.B = cfg->B; p.H = cfg->H; p.d = cfg->d;
+    p.rows_per_split = kDecodeRowsPerSplit;
+    p.scale_log2 = scale_of(cfg) * 1.4426950408889634f;
+    p.items_per_b = decode_items(cfg, cache_cap, p.nsplit, p.item0);
+    for (int h = 0; h < cfg->H; ++h) {
+        p.dil[h] = cfg->dil[h];
+        p.win[h] = cfg->win[h];
+        p.slab[h] = (cache_cap + cfg->dil[h] - 1) / cfg->dil[h];
+        p.recur[h] = head_recur(cfg, h) ? 1 : 0;
+    }
+    p.hdr = reinterpret_cast<WsHeader *>(ws);
+    cudaError_t e = launch_decode(p, cfg->dtype, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    return RAT_OK;
+}
+
+rat_status rat_check_status(void *ws, rat_stream_t stream) {
+    if (!ws) return fail(RAT_ERR_INVALID, "workspace is NULL");
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int hdr[2] = {0, 0};
+    e = cudaMemcpy(hdr, ws, sizeof(hdr), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(status)");
+    if (hdr[0] != 0) {
+        const int zero[2] = {0, 0};
+        e = cudaMemcpy(ws, zero, sizeof(zero), cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(clear status)");
+        return fail((rat_status)hdr[0], "device reported %s (unit %d)", rat_status_string((rat_status)hdr[0]),
+                    hdr[1]);
+    }
+    return RAT_OK;
+}
+
+rat_status rat_debug_set_scan_stall(void *ws, size_t ws_bytes, int64_t ticket, int64_t spin_limit_ns,
+                                    rat_stream_t stream) {
+    if (!ws || ws_bytes < sizeof(WsHeader)) return fail(RAT_ERR_INVALID, "workspace NULL or too small");
+    long long v[2] = {ticket < 0 ? 0LL : (long long)ticket + 1, spin_limit_ns > 0 ? (long long)spin_limit_ns : 0LL};
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaMemcpy(static_cast<char *>(ws) + offsetof(WsHeader, stall_ticket_plus1), v,
+                                         sizeof(v), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "set scan stall");
+    return RAT_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,147 @@
+// rat_internal.cuh -- parameter blocks and device helpers shared by the kernels
+// of librat.so.  Nothing here is part of the public ABI (include/rat.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "rat.h"
+
+namespace rat {
+
+constexpr int kMaxHeads = 256;
+constexpr long long kDefaultSpinNs = 1000000000LL;  // 1 s bound on every device-side wait
+
+// First 256 bytes of every workspace.
+struct WsHeader {
+    int status;                    // first device-side error (a rat_status), 0 = none
+    int detail;                    // which unit reported it (e.g. a scan ticket)
+    long long stall_ticket_plus1;  // failure injection for the scan look-back, 0 = off
+    long long spin_limit_ns;       // 0 = kDefaultSpinNs
+    long long pad[29];
+};
+static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
+
+__device__ __forceinline__ void report_error(WsHeader *hdr, int code, int detail) {
+    if (atomicCAS(&hdr->status, 0, code) == 0) hdr->detail = detail;
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ int ld_acquire(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release(int *p, int v) {
+    asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// ---------------------------------------------------------------- 4-wide I/O
+// Four consecutive channels of a token row: 8 bytes of bf16 or 16 bytes of f32.
+template <typename T> struct IO4;
+
+template <> struct IO4<float> {
+    static __device__ __forceinline__ float4 load(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+    static __device__ __forceinline__ void store(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+};
+
+template <> struct IO4<__nv_bfloat16> {
+    static __device__ __forceinline__ float4 load(const __nv_bfloat16 *p) {
+        uint2 raw = *reinterpret_cast<const uint2 *>(p);
+        float2 lo = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw.x));
+        float2 hi = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&raw.y));
+        return make_float4(lo.x, lo.y, hi.x, hi.y);
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, float4 v) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(v.z, v.w);
+        uint2 raw;
+        raw.x = *reinterpret_cast<uint32_t *>(&lo);
+        raw.y = *reinterpret_cast<uint32_t *>(&hi);
+        *reinterpret_cast<uint2 *>(p) = raw;
+    }
+};
+
+__device__ __forceinline__ float f4get(const float4 &v, int i) {
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// --------------------------------------------------------------- scan (K1)
+struct ScanParams {
+    const void *x[2];       // k, v            [B,T,H,d]
+    const void *g;          // gate logits     [B,T,H,d]
+    const float *init[2];   // [B,H,d] or null
+    void *out[2];           // kt, vt or null
+    float *fin[2];          // final state [B,H,d] or null
+    void *cache[2];         // decode cache [B,H,R,d] or null
+    long long cache_R;      // rows per (b,h) cache block
+    int cap;
+    int B, T, H, d;
+    int nslices;            // B * nheads
+    int nchunks;            // chunks along T per slice
+    int chunk_len, sub_len; // timesteps per chunk / per thread group
+    int nheads;             // heads taken by this launch
+    unsigned char head_list[kMaxHeads];
+    unsigned char head_recur[kMaxHeads];
+    int head_dil[kMaxHeads];
+    unsigned int *ticket;   // dynamic chunk ticket counter (zeroed per launch)
+    int *flags;             // [nslices * nchunks] 0 none, 1 aggregate, 2 inclusive
+    float *agg;             // [nslices * nchunks][3][d]  (A, b_k, b_v)
+    float *incl;            // [nslices * nchunks][2][d]  state after the chunk
+    WsHeader *hdr;
+};
+
+// ---------------------------------------------------------- attention (K2/K3)
+struct AttnParams {
+    const void *q;          // [B,T,H,d]
+    const void *kt, *vt;    // augmented keys / values [B,T,H,d]
+    const void *kraw, *vraw;// raw keys / values for heads with use_raw (or null)
+    void *o;                // [B,T,H,d]
+    float *lse;             // [B,H,T] or null
+    int B, T, H, d;
+    float scale_log2;       // scale * log2(e)
+    int dil[kMaxHeads];
+    int win[kMaxHeads];
+    unsigned char use_raw[kMaxHeads];
+    WsHeader *hdr;
+};
+
+// -------------------------------------------------------------- decode (K4/K5)
+struct DecodeParams {
+    const void *q, *k, *v, *g;   // [B,H,d]
+    float *state[2];             // [B,H,d] fp32, in place
+    void *cache[2];              // [B,H,R,d]
+    const int *pos;              // device [B]
+    void *o;                     // [B,H,d]
+    float *lse;                  // [B,H] or null
+    float *part;                 // [B][items][d + 2]  (acc[d], m, l) per work item
+    long long cache_R;
+    int cap, B, H, d;
+    int items_per_b;             // sum over heads of (nsplit_h + 1)
+    int rows_per_split;
+    float scale_log2;
+    int dil[kMaxHeads];
+    int win[kMaxHeads];
+    int slab[kMaxHeads];         // ceil(cap / dil)
+    int nsplit[kMaxHeads];       // dilated splits of head h (the +1 tail item follows them)
+    int item0[kMaxHeads + 1];    // first item of head h within a batch entry
+    unsigned char recur[kMaxHeads];
+    WsHeader *hdr;
+};
+
+// Process-wide count of kernels this library has launched (rat_launch_count).
+void count_launches(int n);
+
+// launchers (defined in the kernel files); return cudaGetLastError()
+cudaError_t launch_scan(const ScanParams &p, int dtype, cudaStream_t s);
+cudaError_t launch_attn_simt(const AttnParams &p, int dtype, cudaStream_t s);
+cudaError_t launch_decode(const DecodeParams &p, int dtype, cudaStream_t s);
+
+}  // namespace rat

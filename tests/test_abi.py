@@ -1,0 +1,116 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel launched).
+
+* librat.so builds, loads and exports every function include/rat.h declares;
+* argument validation returns the documented status before any launch;
+* workspace sizes and the decode-cache layout are as documented.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import recurrence_augmented_dilated_gated_b200 as rat
+from recurrence_augmented_dilated_gated_b200 import build as rat_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    rat_build.build()
+    return rat.load_library()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "rat.h")).read()
+    return sorted(set(re.findall(r"RAT_API\s+[\w\s\*]+?\b(rat_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(rat.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert lib.rat_version() == 100
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert lib.rat_status_string(s).decode().startswith(rat.STATUS_NAMES[s])
+
+
+def cfg(**kw):
+    a = dict(B=1, T=100, H=2, d=128, dtype=rat.RAT_BF16, dil=[4, 4], win=[0, 8], recur=None, scale=0.0)
+    a.update(kw)
+    return rat.Config(**a)
+
+
+def test_workspace_size_rejects_bad_configs(lib):
+    c = cfg()
+    assert lib.rat_workspace_size(c.ref(), rat.RAT_OP_MIX, 0) > 0
+    for bad in (cfg(d=96), cfg(d=32), cfg(H=300, dil=[1] * 300, win=[0] * 300), cfg(dil=[0, 4]),
+                cfg(win=[-1, 0]), cfg(dtype=7), cfg(B=-1)):
+        assert lib.rat_workspace_size(bad.ref(), rat.RAT_OP_MIX, 0) == 0
+    assert lib.rat_workspace_size(c.ref(), 99, 0) == 0
+    assert lib.rat_workspace_size(c.ref(), rat.RAT_OP_DECODE, 0) == 0  # decode needs a capacity
+
+
+def test_workspace_grows_with_what_it_holds(lib):
+    c = cfg(T=4096)
+    scan = lib.rat_workspace_size(c.ref(), rat.RAT_OP_SCAN, 0)
+    mix = lib.rat_workspace_size(c.ref(), rat.RAT_OP_MIX, 0)
+    mixkv = lib.rat_workspace_size(c.ref(), rat.RAT_OP_MIX_CALLER_KV, 0)
+    kv_bytes = 2 * 1 * 4096 * 2 * 128 * 2
+    assert mix - mixkv >= kv_bytes and mixkv > scan
+    d1 = lib.rat_workspace_size(c.ref(), rat.RAT_OP_DECODE, 1000)
+    d2 = lib.rat_workspace_size(c.ref(), rat.RAT_OP_DECODE, 100000)
+    assert d2 > d1 > 0
+
+
+def test_cache_rows_layout(lib):
+    # rows per (b,h) block = max_h D_h * ceil(cap / D_h)
+    c = cfg(H=3, dil=[1, 16, 64], win=[0, 0, 256])
+    for cap in (1, 63, 64, 65, 4096, 33792):
+        expect = max(D * -(-cap // D) for D in (1, 16, 64))
+        assert lib.rat_cache_rows(c.ref(), cap) == expect
+    assert lib.rat_cache_rows(c.ref(), 0) == 0
+
+
+def call_scan(lib, c, **ptrs):
+    P = dict(k=16, v=16, g=16, init_k=None, init_v=None, kt=16, vt=16, fk=None, fv=None, ck=None, cv=None, cap=0,
+             ws=256, wsb=1 << 40)
+    P.update(ptrs)
+    return lib.rat_scan_prefill(c.ref(), P["k"], P["v"], P["g"], P["init_k"], P["init_v"], P["kt"], P["vt"],
+                                P["fk"], P["fv"], P["ck"], P["cv"], P["cap"], P["ws"], P["wsb"], None)
+
+
+def test_argument_errors_return_before_launch(lib):
+    # fake (never dereferenced) addresses: every call below must fail in validation
+    c = cfg()
+    assert call_scan(lib, c, k=None) == rat.RAT_ERR_INVALID
+    assert call_scan(lib, c, k=8) == rat.RAT_ERR_INVALID                     # misaligned
+    assert call_scan(lib, c, kt=None, vt=None) == rat.RAT_ERR_INVALID         # no output
+    assert call_scan(lib, c, vt=None) == rat.RAT_ERR_INVALID                  # unpaired
+    assert call_scan(lib, c, ck=16, cv=16, cap=50) == rat.RAT_ERR_INVALID    # cap < T
+    assert call_scan(lib, c, wsb=16) == rat.RAT_ERR_WORKSPACE
+    assert call_scan(lib, c, ws=None) == rat.RAT_ERR_INVALID
+    assert call_scan(lib, c, ws=272) == rat.RAT_ERR_INVALID                   # ws not 256-aligned
+    assert call_scan(lib, cfg(d=96)) == rat.RAT_ERR_UNSUPPORTED
+    assert b"aligned" in lib.rat_last_error() or len(lib.rat_last_error()) > 0
+    bad = lib.rat_dilated_attn_prefill(c.ref(), 16, 16, 16, None, None, 256, 1 << 40, None)
+    assert bad == rat.RAT_ERR_INVALID
+    bad = lib.rat_decode_step(c.ref(), 16, 16, 16, 16, 16, 16, 16, 16, 0, 16, 16, None, 256, 1 << 40, None)
+    assert bad == rat.RAT_ERR_INVALID                                          # cap < 1
+    assert lib.rat_check_status(None, None) == rat.RAT_ERR_INVALID
+
+
+def test_binding_refuses_cpu_tensors():
+    c = cfg(T=8)
+    x = torch.zeros(1, 8, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        rat.rat_scan_prefill(c, x, x, x, kt=x, vt=x, ws=torch.zeros(1 << 20, dtype=torch.uint8))

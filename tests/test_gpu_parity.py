@@ -1,0 +1,346 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Inputs come from workloads.py (seeded; q, k, v ~ N(0,1), gate logits ~ N(mu,1)).
+The oracle consumes the exact input values the GPU consumed (bf16 inputs are
+converted to fp64 on the host).  Bar: max-abs 1e-4 (fp32), relative L2 1e-2
+(bf16).  Small cases compare every element; the full-size workloads compare
+sampled heads and rows that always include t=0, t<D, residue and window
+boundaries and the last rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from parity import assert_close, f64, sample_rows
+
+rat = pytest.importorskip("recurrence_augmented_dilated_gated_b200")
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def make_cfg(B, T, H, d, dtype, dil, win, recur=None, scale=0.0):
+    return rat.Config(B, T, H, d, dtype, dil, win, recur, scale)
+
+
+def inputs(B, T, H, d, dtype, mu=2.0, seed=0, device="cpu"):
+    q, k, v, g = wl.prefill_inputs(B, T, H, d, mu, dtype, device=device, seed=seed)
+    return [x.to(DEV) for x in (q, k, v, g)]
+
+
+def oracle_prefill(q, k, v, g, dil, win, recur, init_k=None, init_v=None, scale=None):
+    return oracle.mix_prefill(f64(q), f64(k), f64(v), f64(g), dil, win, recur,
+                              None if init_k is None else f64(init_k), None if init_v is None else f64(init_v),
+                              scale=scale)
+
+
+# ------------------------------------------------------------------ small cases
+
+
+def test_tiny_f32_operator_every_element():
+    w = wl.TINY_F32
+    cfg = make_cfg(w.B, w.T, w.H, w.d, rat.RAT_F32, w.dil, w.win, w.recur)
+    q, k, v, g = inputs(w.B, w.T, w.H, w.d, torch.float32, w.gate_mean)
+    out = rat.mix_prefill(cfg, q, k, v, g, want_kv=True)
+    rat.rat_check_status(out["ws"])
+    ref = oracle_prefill(q, k, v, g, w.dil, w.win, w.recur)
+    for key in ("o", "lse", "kt", "vt", "final_k", "final_v"):
+        assert_close(out[key], ref[key], torch.float32, key)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("T", [1, 77, 1000, 5003])
+def test_scan_every_element(dtype, d, T):
+    # ragged T spans one to dozens of chunks (look-back exercised); init given
+    B, H = 2, 3
+    q, k, v, g = inputs(B, T, H, d, dtype, seed=T)
+    init_k = wl.random_state(B, H, d, seed=1).to(DEV)
+    init_v = wl.random_state(B, H, d, seed=2).to(DEV)
+    recur = [1, 0, 1]
+    cfg = make_cfg(B, T, H, d, dtype, [4] * H, [0] * H, recur)
+    kt, vt = torch.empty_like(k), torch.empty_like(v)
+    fk = torch.empty(B, H, d, device=DEV)
+    fv = torch.empty_like(fk)
+    ws = rat.workspace(cfg, rat.RAT_OP_SCAN)
+    rat.rat_scan_prefill(cfg, k, v, g, init_k, init_v, kt, vt, fk, fv, ws=ws)
+    rat.rat_check_status(ws)
+    rk, rfk = oracle.scan(f64(k), f64(g), f64(init_k), recur)
+    rv, rfv = oracle.scan(f64(v), f64(g), f64(init_v), recur)
+    assert_close(kt, rk, dtype, "kt")
+    assert_close(vt, rv, dtype, "vt")
+    assert_close(fk, rfk, torch.float32 if dtype == torch.float32 else dtype, "final_k")
+    assert_close(fv, rfv, torch.float32 if dtype == torch.float32 else dtype, "final_v")
+    # heads without recurrence are copied exactly
+    assert torch.equal(kt[:, :, 1], k[:, :, 1]) and torch.equal(vt[:, :, 1], v[:, :, 1])
+
+
+ATTN_CASES = [
+    # (T, dil per head, win per head)
+    (700, [1, 3], [0, 0]),
+    (700, [16, 5], [64, 1]),
+    (333, [7, 400], [5, 333]),     # D > T for one head, W = T
+    (129, [1, 2], [1000, 2]),      # W > T
+    (1024, [64, 16], [512, 0]),
+]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("case", range(len(ATTN_CASES)))
+def test_attention_every_element(dtype, d, case):
+    T, dil, win = ATTN_CASES[case]
+    B, H = 2, 2
+    q, kt, vt, _ = inputs(B, T, H, d, dtype, seed=100 + case)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, T, device=DEV)
+    ws = rat.workspace(cfg, rat.RAT_OP_ATTN)
+    rat.rat_dilated_attn_prefill(cfg, q, kt, vt, o, lse, ws)
+    rat.rat_check_status(ws)
+    ro, rl = oracle.attention(f64(q), f64(kt), f64(vt), dil, win)
+    assert_close(o, ro, dtype, "o")
+    assert_close(lse, rl, dtype if dtype == torch.bfloat16 else torch.float32, "lse")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_mix_hybrid_heads_every_element(dtype):
+    # dense heads (D=1, no recurrence) next to dilated + windowed recurrent heads
+    B, T, H, d = 2, 900, 4, 128
+    dil, win, recur = [1, 1, 8, 16], [0, 0, 32, 100], [0, 0, 1, 1]
+    q, k, v, g = inputs(B, T, H, d, dtype, mu=3.0, seed=7)
+    init_k = wl.random_state(B, H, d, seed=3).to(DEV)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur)
+    for want_kv in (False, True):
+        out = rat.mix_prefill(cfg, q, k, v, g, init_k=init_k, want_kv=want_kv)
+        rat.rat_check_status(out["ws"])
+        ref = oracle_prefill(q, k, v, g, dil, win, recur, init_k=init_k)
+        assert_close(out["o"], ref["o"], dtype, "o")
+        assert_close(out["lse"], ref["lse"], torch.float32 if dtype == torch.float32 else dtype, "lse")
+        if want_kv:
+            assert_close(out["kt"], ref["kt"], dtype, "kt")
+
+
+def test_custom_scale():
+    B, T, H, d = 1, 300, 2, 64
+    dtype = torch.bfloat16
+    q, k, v, g = inputs(B, T, H, d, dtype, seed=11)
+    cfg = make_cfg(B, T, H, d, dtype, [3, 3], [10, 0], scale=0.05)
+    out = rat.mix_prefill(cfg, q, k, v, g)
+    ref = oracle_prefill(q, k, v, g, [3, 3], [10, 0], None, scale=0.05)
+    assert_close(out["o"], ref["o"], dtype, "o")
+
+
+def test_empty_inputs():
+    B, T, H, d = 2, 0, 2, 64
+    cfg = make_cfg(B, T, H, d, torch.float32, [2, 2], [0, 0])
+    e = torch.empty(B, T, H, d, device=DEV)
+    init = wl.random_state(B, H, d, seed=5).to(DEV)
+    fk = torch.full((B, H, d), 7.0, device=DEV)
+    fv = torch.full((B, H, d), 7.0, device=DEV)
+    ws = rat.workspace(make_cfg(B, 1, H, d, torch.float32, [2, 2], [0, 0]), rat.RAT_OP_MIX)
+    rat.rat_mix_prefill(cfg, e, e, e, e, init, None, e, None, None, None, fk, fv, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(fk, init) and torch.all(fv == 0)
+
+
+def test_decode_cache_layout_from_scan():
+    # cache row of position j in head h: (j mod D_h) * ceil(cap/D_h) + j // D_h
+    B, T, H, d = 2, 300, 3, 64
+    dtype = torch.bfloat16
+    dil = [1, 4, 7]
+    cap = 333
+    q, k, v, g = inputs(B, T, H, d, dtype, seed=9)
+    cfg = make_cfg(B, T, H, d, dtype, dil, [0] * H)
+    R = rat.rat_cache_rows(cfg, cap)
+    ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
+    cv = torch.zeros_like(ck)
+    kt, vt = torch.empty_like(k), torch.empty_like(v)
+    ws = rat.workspace(cfg, rat.RAT_OP_SCAN)
+    rat.rat_scan_prefill(cfg, k, v, g, None, None, kt, vt, None, None, ck, cv, cap, ws)
+    torch.cuda.synchronize()
+    for h, D in enumerate(dil):
+        S = -(-cap // D)
+        j = torch.arange(T, device=DEV)
+        rows = (j % D) * S + j // D
+        assert torch.equal(ck[:, h, rows], kt[:, :, h])
+        assert torch.equal(cv[:, h, rows], vt[:, :, h])
+
+
+def run_decode_case(B, T, steps, H, d, dtype, dil, win, recur, mu, seed, cap=None, check_b=None, check_h=None,
+                    gen_device="cpu"):
+    """Prefill T tokens into the cache with rat_scan_prefill, then decode `steps`
+    tokens with rat_decode_step; compare every step with the oracle's rows
+    (on the batch entries check_b and heads check_h; all by default)."""
+    Tt = T + steps
+    cap = cap or Tt
+    q, k, v, g = inputs(B, Tt, H, d, dtype, mu=mu, seed=seed, device=gen_device)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur)
+    R = rat.rat_cache_rows(cfg, cap)
+    ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
+    cv = torch.zeros_like(ck)
+    sk = torch.empty(B, H, d, device=DEV)
+    sv = torch.empty_like(sk)
+    ws = rat.workspace(cfg, rat.RAT_OP_SCAN)
+    rat.rat_scan_prefill(cfg, k[:, :T].contiguous(), v[:, :T].contiguous(), g[:, :T].contiguous(), None, None,
+                         None, None, sk, sv, ck, cv, cap, ws)
+    rat.rat_check_status(ws)
+    del ws
+    wsd = rat.workspace(cfg, rat.RAT_OP_DECODE, cap)
+    outs = []
+    for s in range(steps):
+        t = T + s
+        pos = torch.full((B,), t, dtype=torch.int32, device=DEV)
+        o = torch.empty(B, H, d, dtype=dtype, device=DEV)
+        lse = torch.empty(B, H, device=DEV)
+        rat.rat_decode_step(cfg, q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(),
+                            g[:, t].contiguous(), sk, sv, ck, cv, cap, pos, o, lse, wsd)
+        outs.append((o, lse))
+    rat.rat_check_status(wsd)
+    bsel = list(range(B)) if check_b is None else check_b
+    hsel = list(range(H)) if check_h is None else check_h
+    sl = lambda x: f64(x[bsel][:, :, hsel])
+    dsel, wsel, rsel = [dil[h] for h in hsel], [win[h] for h in hsel], [recur[h] for h in hsel]
+    kt, fk = oracle.scan(sl(k), sl(g), None, rsel)
+    vt, fv = oracle.scan(sl(v), sl(g), None, rsel)
+    rows = np.array([(b, i, t) for b in range(len(bsel)) for i in range(len(hsel)) for t in range(T, Tt)])
+    ro, rl = oracle.attn_rows(sl(q), kt, vt, dsel, wsel, rows, parts=3)
+    ro = ro.reshape(len(bsel), len(hsel), steps, d)
+    rl = rl.reshape(len(bsel), len(hsel), steps)
+    ft = torch.float32 if dtype == torch.float32 else dtype
+    for s, (o, lse) in enumerate(outs):
+        assert_close(o[bsel][:, hsel], ro[:, :, s], dtype, "decode o step %d" % s)
+        assert_close(lse[bsel][:, hsel], rl[:, :, s], ft, "decode lse step %d" % s)
+    assert_close(sk[bsel][:, hsel], fk, ft, "state_k")
+    assert_close(sv[bsel][:, hsel], fv, ft, "state_v")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_steps_every_element(dtype, d):
+    run_decode_case(B=3, T=1500, steps=5, H=4, d=d, dtype=dtype, dil=[1, 4, 16, 3], win=[0, 0, 64, 1500],
+                    recur=[0, 1, 1, 1], mu=2.0, seed=21)
+
+
+def test_decode_from_empty_history():
+    # the first token decoded with nothing in the cache (t = 0), then a few more
+    run_decode_case(B=2, T=1, steps=4, H=2, d=128, dtype=torch.bfloat16, dil=[2, 1], win=[3, 0],
+                    recur=[1, 0], mu=2.0, seed=5, cap=8)
+
+
+def test_decode_long_slab_spans_several_splits():
+    # 2500 old rows in the residue slab: three split items plus the tail item
+    run_decode_case(B=1, T=5000, steps=2, H=2, d=128, dtype=torch.bfloat16, dil=[2, 1], win=[0, 7],
+                    recur=[1, 1], mu=2.0, seed=6)
+
+
+def test_decode_bad_position_is_reported():
+    B, H, d = 2, 2, 64
+    cfg = make_cfg(B, 1, H, d, torch.bfloat16, [2, 2], [0, 0])
+    cap = 16
+    R = rat.rat_cache_rows(cfg, cap)
+    ck = torch.zeros(B, H, R, d, dtype=torch.bfloat16, device=DEV)
+    cv = torch.zeros_like(ck)
+    x = torch.zeros(B, H, d, dtype=torch.bfloat16, device=DEV)
+    s = torch.zeros(B, H, d, device=DEV)
+    ws = rat.workspace(cfg, rat.RAT_OP_DECODE, cap)
+    pos = torch.tensor([3, cap], dtype=torch.int32, device=DEV)   # second entry out of range
+    o = torch.empty_like(x)
+    rat.rat_decode_step(cfg, x, x, x, x, s, s.clone(), ck, cv, cap, pos, o, None, ws)
+    with pytest.raises(rat.RatError) as ei:
+        rat.rat_check_status(ws)
+    assert ei.value.status == rat.RAT_ERR_INVALID
+    rat.rat_check_status(ws)  # cleared
+
+
+def test_scan_lookback_timeout_is_reported_and_recovers():
+    # one chunk never publishes its carry: its successors give up after the
+    # bounded wait, record RAT_ERR_TIMEOUT, and the workspace stays usable
+    B, T, H, d = 1, 4096, 2, 128
+    dtype = torch.bfloat16
+    q, k, v, g = inputs(B, T, H, d, dtype, seed=3)
+    cfg = make_cfg(B, T, H, d, dtype, [1, 1], [0, 0])
+    kt, vt = torch.empty_like(k), torch.empty_like(v)
+    ws = rat.workspace(cfg, rat.RAT_OP_SCAN)
+    rat.rat_debug_set_scan_stall(ws, ticket=5, spin_limit_ns=20_000_000)
+    rat.rat_scan_prefill(cfg, k, v, g, kt=kt, vt=vt, ws=ws)
+    with pytest.raises(rat.RatError) as ei:
+        rat.rat_check_status(ws)
+    assert ei.value.status == rat.RAT_ERR_TIMEOUT
+    rat.rat_debug_set_scan_stall(ws, ticket=-1)
+    rat.rat_scan_prefill(cfg, k, v, g, kt=kt, vt=vt, ws=ws)
+    rat.rat_check_status(ws)
+    rk, _ = oracle.scan(f64(k), f64(g))
+    assert_close(kt, rk, dtype, "kt after recovery")
+
+
+# ------------------------------------------------------ full-size workloads
+
+
+def large_prefill_check(w, heads, n_random=24, seed=0):
+    """Run the whole operator at the workload's full size on the GPU; compare
+    sampled heads and rows with the oracle (which runs on those heads only)."""
+    dtype = w.torch_dtype
+    q, k, v, g = wl.prefill_inputs(w.B, w.T, w.H, w.d, w.gate_mean, dtype, device=DEV, seed=seed)
+    cfg = make_cfg(w.B, w.T, w.H, w.d, dtype, w.dil, w.win, w.recur)
+    out = rat.mix_prefill(cfg, q, k, v, g)
+    rat.rat_check_status(out["ws"])
+    sl = lambda x: x[:, :, heads]
+    dil = [w.dil[h] for h in heads]
+    win = [w.win[h] for h in heads]
+    recur = [w.recur[h] for h in heads]
+    kt, fk = oracle.scan(f64(sl(k)), f64(sl(g)), None, recur)
+    vt, fv = oracle.scan(f64(sl(v)), f64(sl(g)), None, recur)
+    qh = f64(sl(q))
+    rows = []
+    for b in range(w.B):
+        for i, h in enumerate(heads):
+            for t in sample_rows(w.T, dil[i], win[i], n_random=n_random, seed=seed + h):
+                rows.append((b, i, t))
+    rows = np.array(rows)
+    ro, rl = oracle.attn_rows(qh, kt, vt, dil, win, rows, parts=3)
+    hsel = torch.tensor([heads[i] for i in rows[:, 1]])
+    got_o = out["o"][rows[:, 0], rows[:, 2], hsel]
+    got_l = out["lse"][rows[:, 0], hsel, rows[:, 2]]
+    assert_close(got_o, ro, dtype, "o rows")
+    assert_close(got_l, rl, dtype, "lse rows")
+    assert_close(out["final_k"][:, heads], fk, dtype, "final_k")
+    del out, q, k, v, g
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.slow
+def test_full_prefill_16k():
+    large_prefill_check(wl.PREFILL_16K, heads=[0, 7, 15])
+
+
+@pytest.mark.slow
+def test_full_prefill_262k_window():
+    large_prefill_check(wl.PREFILL_262K, heads=[0, 9], n_random=16)
+
+
+@pytest.mark.slow
+def test_full_prefill_hybrid():
+    large_prefill_check(wl.HYBRID, heads=[0, 3, 4, 31], n_random=12)
+
+
+@pytest.mark.slow
+def test_full_decode_batch256_ctx4096():
+    # the decode workload at its full batch and head count, context 4096
+    w = wl.DECODE_D16
+    run_decode_case(B=w.decode_batch, T=4096, steps=3, H=w.H, d=w.d, dtype=torch.bfloat16, dil=w.dil, win=w.win,
+                    recur=w.recur, mu=w.gate_mean, seed=0, check_b=[0, 97, 255], check_h=[0, 5, 15],
+                    gen_device=DEV)
+
+
+@pytest.mark.slow
+def test_hybrid_decode_full_context():
+    # the hybrid workload's decode at its full 65536-token context (batch 8 of
+    # the 128: the batch entries are independent)
+    w = wl.HYBRID
+    run_decode_case(B=8, T=65536, steps=2, H=w.H, d=w.d, dtype=torch.bfloat16, dil=w.dil, win=w.win,
+                    recur=w.recur, mu=w.gate_mean, seed=0, check_b=[0, 7], check_h=[0, 3, 4, 31],
+                    gen_device=DEV)
