@@ -192,6 +192,33 @@ RAT_API rat_status rat_decode_step(const rat_cfg *cfg, const void *q, const void
                            void *ws, size_t ws_bytes, rat_stream_t stream);
 
 /*
+ * rat_decode_step without a workspace, for callers that cannot allocate
+ * device memory when they decode: a plugin inside an inference engine that
+ * owns all device memory and gives its plugins no scratch buffer, or a serving
+ * loop whose device-memory budget is fixed at start-up.  The operator paper
+ * has no counterpart to this call; it only moves rat_decode_step's scratch.
+ * Arguments and results are those of rat_decode_step minus (ws, ws_bytes).
+ *   - Scratch: a static 16 MiB device array inside librat.so, held by every
+ *     GPU that loads the library until the process exits.  A step needs
+ *     256 + B * items * (d + 2) * 4 bytes, items = sum over heads of
+ *     ceil(ceil(cache_cap / D_h) / 1024) + 1; a larger step returns
+ *     RAT_ERR_UNSUPPORTED with the sizes in rat_last_error().
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address (cudaGetSymbolAddress) and caches it; make that
+ *     first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents
+ *     (no call needs it cleared).  Calls whose kernels overlap on a GPU race
+ *     on it: order them on one stream.
+ *   - Never allocates or frees device memory.  An out-of-range pos[b] still
+ *     makes the kernel skip that entry (its o is zero), but is not reported:
+ *     there is no workspace for rat_check_status to read.
+ */
+RAT_API rat_status rat_decode_step_noalloc(const rat_cfg *cfg, const void *q, const void *k, const void *v,
+                                           const void *g, float *state_k, float *state_v, void *cache_k,
+                                           void *cache_v, int cache_cap, const int32_t *pos, void *o,
+                                           float *lse, rat_stream_t stream);
+
+/*
  * Synchronises `stream`, returns the first device-side error recorded in `ws`
  * since the last check (RAT_OK if none) and clears it.  RAT_ERR_CUDA if the
  * synchronisation itself fails.

@@ -24,7 +24,8 @@ RAT_OP_SCAN, RAT_OP_ATTN, RAT_OP_MIX, RAT_OP_MIX_CALLER_KV, RAT_OP_DECODE = rang
 
 EXPORTS = ["rat_workspace_size", "rat_workspace_init", "rat_cache_rows", "rat_scan_prefill",
            "rat_dilated_attn_prefill", "rat_mix_prefill", "rat_decode_step", "rat_check_status",
-           "rat_status_string", "rat_last_error", "rat_version", "rat_launch_count", "rat_debug_set_scan_stall"]
+           "rat_status_string", "rat_last_error", "rat_version", "rat_launch_count", "rat_debug_set_scan_stall",
+           "rat_decode_step_noalloc"]
 
 
 class RatError(RuntimeError):
@@ -66,6 +67,7 @@ def load_library(path=LIB_PATH):
     lib.rat_dilated_attn_prefill.argtypes = [cfgp, P, P, P, P, P, P, S, P]
     lib.rat_mix_prefill.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P]
     lib.rat_decode_step.argtypes = [cfgp, P, P, P, P, P, P, P, P, I, P, P, P, P, S, P]
+    lib.rat_decode_step_noalloc.argtypes = [cfgp, P, P, P, P, P, P, P, P, I, P, P, P, P]
     lib.rat_check_status.argtypes = [P, P]
     lib.rat_status_string.argtypes = [I]
     lib.rat_status_string.restype = ctypes.c_char_p
@@ -75,7 +77,7 @@ def load_library(path=LIB_PATH):
     lib.rat_launch_count.restype = ctypes.c_longlong
     lib.rat_debug_set_scan_stall.argtypes = [P, S, ctypes.c_int64, ctypes.c_int64, P]
     for name in ("rat_workspace_init", "rat_scan_prefill", "rat_dilated_attn_prefill", "rat_mix_prefill",
-                 "rat_decode_step", "rat_check_status", "rat_debug_set_scan_stall"):
+                 "rat_decode_step", "rat_check_status", "rat_debug_set_scan_stall", "rat_decode_step_noalloc"):
         getattr(lib, name).restype = I
     _lib = lib
     return lib
@@ -230,6 +232,24 @@ def rat_decode_step(cfg, q, k, v, g, state_k, state_v, cache_k, cache_v, cache_c
             _ptr(lse, "lse", torch.float32, (c.B, c.H), True), _ptr(ws, "ws", torch.uint8), ws.numel(),
             _stream(stream)]
     _check(load_library().rat_decode_step(cfg.ref(), *args), "rat_decode_step")
+
+
+def rat_decode_step_noalloc(cfg, q, k, v, g, state_k, state_v, cache_k, cache_v, cache_cap, pos, o, lse=None,
+                            stream=None):
+    """rat_decode_step without a workspace: for callers that cannot allocate
+    device memory while decoding (its scratch is a static 16 MiB array inside
+    the library).  Calls whose kernels overlap on the GPU race on that array."""
+    c = cfg.c
+    tok = (c.B, c.H, c.d)
+    dt = cfg.torch_dtype
+    R = rat_cache_rows(cfg, cache_cap)
+    cshape = (c.B, c.H, R, c.d)
+    args = [_ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, tok),
+            _ptr(state_k, "state_k", torch.float32, tok), _ptr(state_v, "state_v", torch.float32, tok),
+            _ptr(cache_k, "cache_k", dt, cshape), _ptr(cache_v, "cache_v", dt, cshape), int(cache_cap),
+            _ptr(pos, "pos", torch.int32, (c.B,)), _ptr(o, "o", dt, tok),
+            _ptr(lse, "lse", torch.float32, (c.B, c.H), True), _stream(stream)]
+    _check(load_library().rat_decode_step_noalloc(cfg.ref(), *args), "rat_decode_step_noalloc")
 
 
 def rat_check_status(ws, stream=None):

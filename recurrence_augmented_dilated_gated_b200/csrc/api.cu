@@ -30,6 +30,15 @@ rat_status fail(rat_status s, const char *fmt, ...) {
     return s;
 }
 
+}  // namespace
+
+rat_status rat::set_last_error(rat_status s, const char *msg) {
+    snprintf(g_last_error, sizeof(g_last_error), "%s", msg);
+    return s;
+}
+
+namespace {
+
 rat_status cuda_fail(cudaError_t e, const char *what) {
     return fail(RAT_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }

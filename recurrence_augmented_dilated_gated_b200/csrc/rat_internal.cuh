@@ -139,6 +139,9 @@ struct DecodeParams {
 // Process-wide count of kernels this library has launched (rat_launch_count).
 void count_launches(int n);
 
+// Record the calling thread's rat_last_error() message; returns s.
+rat_status set_last_error(rat_status s, const char *msg);
+
 // launchers (defined in the kernel files); return cudaGetLastError()
 cudaError_t launch_scan(const ScanParams &p, int dtype, cudaStream_t s);
 cudaError_t launch_attn_simt(const AttnParams &p, int dtype, cudaStream_t s);
