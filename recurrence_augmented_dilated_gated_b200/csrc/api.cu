@@ -9,6 +9,7 @@
 #include <algorithm>
 #include <atomic>
 
+#include "attn_tc.cuh"
 #include "rat_internal.cuh"
 
 using namespace rat;
@@ -189,11 +190,21 @@ rat_status run_scan(const rat_cfg *c, const Layout &L, const void *k, const void
     p.cap = cap;
     p.cache_R = ck ? cache_rows(c, cap) : 0;
     p.B = c->B; p.T = c->T; p.H = c->H; p.d = c->d;
-    int n = 0;
+    int n = 0, n_plain = 0;
+    unsigned char plain[kMaxHeads];
     for (int h = 0; h < c->H; ++h) {
         p.head_recur[h] = head_recur(c, h) ? 1 : 0;
         p.head_dil[h] = c->dil[h];
         if (!only_recurrent || p.head_recur[h]) p.head_list[n++] = (unsigned char)h;
+        else plain[n_plain++] = (unsigned char)h;
+    }
+    if (n_plain > 0 && (fk || fv)) {
+        // skipped heads still report their final state (a = 0: the last token)
+        ScanParams pp = p;
+        memcpy(pp.head_list, plain, n_plain);
+        pp.nheads = n_plain;
+        cudaError_t e = launch_final_of_plain_heads(pp, c->dtype, s);
+        if (e != cudaSuccess) return cuda_fail(e, "final-state launch");
     }
     if (n == 0) return RAT_OK;
     p.nheads = n;
@@ -214,24 +225,124 @@ rat_status run_scan(const rat_cfg *c, const Layout &L, const void *k, const void
     return RAT_OK;
 }
 
+// A head runs on the tensor-core kernel when its operands are bf16 and its
+// dilation divides T (the strided TMA view needs whole subsequences);
+// otherwise the fp32 CUDA-core kernel computes it.
+bool tc_head(const rat_cfg *c, int h) { return c->dtype == RAT_BF16 && c->T % c->dil[h] == 0; }
+
+// One tensor-core launch over `heads` (dilated part, or window part when
+// window_mode), grouped into classes of equal (dilation, K/V source).
+rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, bool window_mode, const void *q,
+                          const void *kt, const void *vt, const void *kraw, const void *vraw,
+                          const bool *raw_head, void *o, float *lse, float *lse_dil, char *ws, cudaStream_t s) {
+    struct Key { int D; int raw; };
+    int done = 0;
+    bool taken[kMaxHeads] = {false};
+    while (done < nheads) {
+        TcParams P;
+        memset(&P, 0, sizeof(P));
+        P.B = c->B; P.T = c->T; P.H = c->H;
+        P.window_mode = window_mode ? 1 : 0;
+        P.scale_log2 = scale_of(c) * 1.4426950408889634f;
+        P.o = o; P.lse_user = lse; P.lse_dil = lse_dil;
+        P.hdr = reinterpret_cast<WsHeader *>(ws);
+        for (int h = 0; h < c->H; ++h) P.win[h] = c->win[h];
+        // collect up to kTcMaxClasses classes
+        Key keys[kTcMaxClasses];
+        int ncls = 0, nh = 0;
+        int cls_heads[kTcMaxClasses][kMaxHeads];
+        int cls_n[kTcMaxClasses] = {0};
+        for (int i = 0; i < nheads; ++i) {
+            const int h = heads[i];
+            if (taken[i]) continue;
+            const Key k{window_mode ? 1 : c->dil[h], raw_head[h] ? 1 : 0};
+            int ci = -1;
+            for (int j = 0; j < ncls; ++j)
+                if (keys[j].D == k.D && keys[j].raw == k.raw) ci = j;
+            if (ci < 0) {
+                if (ncls == kTcMaxClasses) continue;  // next launch
+                ci = ncls++;
+                keys[ci] = k;
+            }
+            cls_heads[ci][cls_n[ci]++] = h;
+            taken[i] = true;
+            ++done;
+        }
+        // order classes by query tiles per subsequence, descending (heaviest first)
+        int order[kTcMaxClasses];
+        for (int i = 0; i < ncls; ++i) order[i] = i;
+        std::sort(order, order + ncls, [&](int a, int b) { return keys[a].D < keys[b].D; });
+        P.ncls = ncls;
+        long long pref = 0;
+        for (int oi = 0; oi < ncls; ++oi) {
+            const int ci = order[oi];
+            TcClass &C = P.cls[oi];
+            C.D = keys[ci].D;
+            C.n = c->T / C.D;
+            C.mtiles = (C.n + 127) / 128;
+            C.nheads = cls_n[ci];
+            C.head0 = nh;
+            for (int j = 0; j < cls_n[ci]; ++j) P.heads[nh++] = (unsigned char)cls_heads[ci][j];
+            P.prefix[oi] = pref;
+            pref += (long long)c->B * C.nheads * C.D;
+            const void *kb = keys[ci].raw ? kraw : kt;
+            const void *vb = keys[ci].raw ? vraw : vt;
+            if (!encode_map_5d(&P.tq[oi], q, c->B, c->T, c->H, c->d, C.D) ||
+                !encode_map_5d(&P.tk[oi], kb, c->B, c->T, c->H, c->d, C.D) ||
+                !encode_map_5d(&P.tv[oi], vb, c->B, c->T, c->H, c->d, C.D))
+                return fail(RAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (dilation %d)", C.D);
+        }
+        P.prefix[ncls] = pref;
+        for (int oi = 0; oi < ncls; ++oi) P.total_units += (long long)P.cls[oi].mtiles * (c->B * (long long)P.cls[oi].nheads * P.cls[oi].D);
+        cudaError_t e = launch_attn_tc(P, c->d, s);
+        if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
+    }
+    return RAT_OK;
+}
+
 rat_status run_attn(const rat_cfg *c, const Layout &L, const void *q, const void *kt, const void *vt,
                     const void *kraw, const void *vraw, bool raw_for_plain_heads, void *o, float *lse,
                     char *ws, cudaStream_t s) {
-    AttnParams p;
-    memset(&p, 0, sizeof(p));
-    p.q = q; p.kt = kt; p.vt = vt; p.kraw = kraw; p.vraw = vraw;
-    p.o = o; p.lse = lse;
-    p.B = c->B; p.T = c->T; p.H = c->H; p.d = c->d;
-    p.scale_log2 = scale_of(c) * 1.4426950408889634f;
+    bool raw_head[kMaxHeads];
+    int tc_all[kMaxHeads], tc_win[kMaxHeads];
+    int n_tc = 0, n_win = 0, n_simt = 0;
     for (int h = 0; h < c->H; ++h) {
-        p.dil[h] = c->dil[h];
-        p.win[h] = c->win[h];
-        p.use_raw[h] = (raw_for_plain_heads && !head_recur(c, h)) ? 1 : 0;
+        raw_head[h] = raw_for_plain_heads && !head_recur(c, h);
+        if (tc_head(c, h)) {
+            tc_all[n_tc++] = h;
+            if (c->win[h] > 0) tc_win[n_win++] = h;
+        } else {
+            ++n_simt;
+        }
     }
-    p.hdr = reinterpret_cast<WsHeader *>(ws);
-    (void)L;
-    cudaError_t e = launch_attn_simt(p, c->dtype, s);
-    if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    float *lse_dil = reinterpret_cast<float *>(ws + L.lse_dil);
+    if (n_tc > 0) {
+        // The sort in launch_tc_part orders classes by dilation; with T fixed,
+        // a smaller dilation means longer subsequences, i.e. more query tiles.
+        rat_status st = launch_tc_part(c, tc_all, n_tc, false, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws, s);
+        if (st != RAT_OK) return st;
+        if (n_win > 0) {
+            st = launch_tc_part(c, tc_win, n_win, true, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws, s);
+            if (st != RAT_OK) return st;
+        }
+    }
+    if (n_simt > 0) {
+        AttnParams p;
+        memset(&p, 0, sizeof(p));
+        p.q = q; p.kt = kt; p.vt = vt; p.kraw = kraw; p.vraw = vraw;
+        p.o = o; p.lse = lse;
+        p.B = c->B; p.T = c->T; p.H = c->H; p.d = c->d;
+        p.scale_log2 = scale_of(c) * 1.4426950408889634f;
+        for (int h = 0; h < c->H; ++h) {
+            p.dil[h] = c->dil[h];
+            p.win[h] = c->win[h];
+            p.use_raw[h] = raw_head[h] ? 1 : 0;
+            p.skip[h] = tc_head(c, h) ? 1 : 0;
+        }
+        p.hdr = reinterpret_cast<WsHeader *>(ws);
+        cudaError_t e = launch_attn_simt(p, c->dtype, s);
+        if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+    }
     return RAT_OK;
 }
 

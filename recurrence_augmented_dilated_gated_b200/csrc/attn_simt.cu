@@ -67,6 +67,7 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(const AttnParams
     const long long t = row % p.T;
     const int h = (int)((row / p.T) % p.H);
     const int b = (int)(row / ((long long)p.T * p.H));
+    if (p.skip[h]) return;  // uniform across the warp (one row per warp)
     const int d = p.d;
     const size_t rs = (size_t)p.H * d;
     const size_t hb = ((size_t)b * p.T * p.H + h) * d;  // (b, t=0, h, 0)

@@ -1,0 +1,46 @@
+// attn_tc.cuh -- parameters of the tensor-core attention kernel (attn_tc.cu).
+#pragma once
+
+#include <cuda.h>
+
+#include "rat_internal.cuh"
+
+namespace rat {
+
+constexpr int kTcMaxClasses = 8;
+
+// Heads of one launch that share a dilation and a K/V source.
+struct TcClass {
+    int D;       // dilation (1 in the window launch: natural order)
+    int n;       // rows of one residue subsequence (T / D)
+    int mtiles;  // query tiles per subsequence, ceil(n / 128)
+    int nheads;  // heads in the class
+    int head0;   // first entry of the class in TcParams::heads
+    int pad;
+};
+
+struct TcParams {
+    CUtensorMap tq[kTcMaxClasses];  // 5-D maps (d, H, D, T/D, B), box (64, 1, 1, 128, 1), 128B swizzle
+    CUtensorMap tk[kTcMaxClasses];
+    CUtensorMap tv[kTcMaxClasses];
+    TcClass cls[kTcMaxClasses];     // sorted by mtiles, descending
+    long long prefix[kTcMaxClasses + 1];  // prefix[c] = sum of units-per-level of classes < c
+    int ncls;
+    int B, T, H;
+    int window_mode;                // 0: dilated part; 1: window part merged with the dilated part
+    float scale_log2;
+    void *o;                        // [B,T,H,d] bf16
+    float *lse_user;                // [B,H,T] or null
+    float *lse_dil;                 // [B,H,T] scratch: lse of the dilated part of windowed heads
+    WsHeader *hdr;
+    long long total_units;
+    unsigned char heads[kMaxHeads];
+    int win[kMaxHeads];
+};
+
+size_t attn_tc_smem_bytes(int hd);
+cudaError_t launch_attn_tc(const TcParams &p, int hd, cudaStream_t s);
+// 5-D TMA map of a [B,T,H,d] bf16 tensor viewed as (d, H, D, T/D, B); requires T % D == 0.
+bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int H, int d, int D);
+
+}  // namespace rat

@@ -110,6 +110,7 @@ struct AttnParams {
     int dil[kMaxHeads];
     int win[kMaxHeads];
     unsigned char use_raw[kMaxHeads];
+    unsigned char skip[kMaxHeads];   // heads another kernel computes
     WsHeader *hdr;
 };
 
@@ -144,6 +145,8 @@ rat_status set_last_error(rat_status s, const char *msg);
 
 // launchers (defined in the kernel files); return cudaGetLastError()
 cudaError_t launch_scan(const ScanParams &p, int dtype, cudaStream_t s);
+// final state of the heads in p.head_list, which have no recurrence
+cudaError_t launch_final_of_plain_heads(const ScanParams &p, int dtype, cudaStream_t s);
 cudaError_t launch_attn_simt(const AttnParams &p, int dtype, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, int dtype, cudaStream_t s);
 

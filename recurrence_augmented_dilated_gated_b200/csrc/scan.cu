@@ -313,7 +313,30 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const ScanParams p) {
     }
 }
 
+// Final state of heads without recurrence (a = 0): s_{T-1} = x_{T-1}.  Used
+// when the scan itself skips those heads (their attention reads k, v directly).
+template <typename T>
+__global__ void final_of_plain_heads_kernel(const ScanParams p) {
+    const int b = blockIdx.x;
+    const T *xs[2] = {static_cast<const T *>(p.x[0]), static_cast<const T *>(p.x[1])};
+    for (int i = threadIdx.x; i < p.nheads * p.d; i += blockDim.x) {
+        const int h = p.head_list[i / p.d], c = i % p.d;
+        const size_t src = (((size_t)b * p.T + (p.T - 1)) * p.H + h) * p.d + c;
+        const size_t dst = ((size_t)b * p.H + h) * p.d + c;
+        for (int j = 0; j < 2; ++j)
+            if (p.fin[j]) p.fin[j][dst] = (float)xs[j][src];
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_final_of_plain_heads(const ScanParams &p, int dtype, cudaStream_t s) {
+    if (p.B == 0 || p.T == 0 || p.nheads == 0) return cudaSuccess;
+    if (dtype == RAT_BF16) final_of_plain_heads_kernel<__nv_bfloat16><<<p.B, 256, 0, s>>>(p);
+    else final_of_plain_heads_kernel<float><<<p.B, 256, 0, s>>>(p);
+    count_launches(1);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_scan(const ScanParams &p, int dtype, cudaStream_t s) {
     const unsigned grid = (unsigned)p.nslices * (unsigned)p.nchunks;
