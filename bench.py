@@ -91,9 +91,10 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms, with host
+    timestamps, so the samples inside the timed region can be picked out."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -102,17 +103,17 @@ class ClockSampler:
         self.proc = None
         self.f = None
 
-    def __enter__(self):
+    def start(self):
         try:
             self.f = tempfile.TemporaryFile(mode="w+")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, ValueError):
             self.proc = None
         return self
 
-    def __exit__(self, *a):
+    def stop(self):
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -120,29 +121,38 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self):
+    def summary(self, t0=None, t1=None):
+        """Median SM clock and active throttle reasons of the samples taken in
+        [t0, t1] (host epoch seconds); all samples when fewer than 2 fall there."""
+        import datetime
+
         if self.proc is None or self.f is None:
             return None
         self.f.seek(0)
-        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.strip()]
-        sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            r = [x.strip() for x in r]
-            if len(r) < 9:
+        samples = []
+        for line in self.f.read().strip().splitlines():
+            r = [x.strip() for x in line.split(",")]
+            if len(r) < 10:
                 continue
             try:
-                sm.append(float(r[1]))
-                mx.append(float(r[2]))
+                ts = datetime.datetime.strptime(r[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                sm, mx = float(r[2]), float(r[3])
             except ValueError:
                 continue
-            for i, n in enumerate(names):
-                if r[5 + i].lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
+            active = {n for i, n in enumerate(names) if r[6 + i].lower().startswith("active")}
+            samples.append((ts, sm, mx, active))
+        if not samples:
             return None
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(mx)), "samples": len(sm),
-                "reasons": sorted(reasons)}
+        window = "timed region"
+        sel = [x for x in samples if t0 is not None and t0 - 0.05 <= x[0] <= t1 + 0.05]
+        if len(sel) < 2:
+            sel, window = samples, "warm-up + timed region (timed region shorter than the sampling interval)"
+        reasons = set()
+        for x in sel:
+            reasons |= x[3]
+        return {"sm_mhz": float(np.median([x[1] for x in sel])), "sm_max_mhz": float(max(x[2] for x in sel)),
+                "samples": len(sel), "reasons": sorted(reasons), "window": window}
 
 
 def profile_traffic(name):
@@ -222,6 +232,7 @@ def bench_prefill(rat, w, steps, warmup, world, rank, dev, e2e_steps):
         if evs:
             evs[2].record(stream)
 
+    clk = ClockSampler(torch.cuda.current_device()).start()
     for _ in range(warmup):
         step()
     rat.rat_check_status(ws)
@@ -229,10 +240,12 @@ def bench_prefill(rat, w, steps, warmup, world, rank, dev, e2e_steps):
     barrier(world)
     torch.cuda.synchronize()
     n0 = rat.rat_launch_count()
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        for i in range(steps):
-            step(evs[i])
-        torch.cuda.synchronize()
+    t_host0 = time.time()
+    for i in range(steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    t_host1 = time.time()
+    clk.stop()
     launches = rat.rat_launch_count() - n0
     barrier(world)
     rat.rat_check_status(ws)
@@ -241,7 +254,7 @@ def bench_prefill(rat, w, steps, warmup, world, rank, dev, e2e_steps):
     total_ms = evs[0][0].elapsed_time(evs[-1][2])
     total_ms = max_over_ranks(total_ms, world, dev)
     res = dict(total_ms=total_ms, scan_ms=float(np.mean(scan_ms)), attn_ms=float(np.mean(attn_ms)),
-               launches=launches, clocks=clk.summary())
+               launches=launches, clocks=clk.summary(t_host0, t_host1))
 
     # end to end through the user call with host buffers: H2D of q,k,v,g from
     # pinned memory, rat_mix_prefill, D2H of o

@@ -279,12 +279,12 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, bool w
             TcClass &C = P.cls[oi];
             C.D = keys[ci].D;
             C.n = c->T / C.D;
-            C.mtiles = (C.n + 127) / 128;
+            C.mtiles = (C.n + 255) / 256;   // 256-row units per (b, h, residue) group
             C.nheads = cls_n[ci];
             C.head0 = nh;
             for (int j = 0; j < cls_n[ci]; ++j) P.heads[nh++] = (unsigned char)cls_heads[ci][j];
             P.prefix[oi] = pref;
-            pref += (long long)c->B * C.nheads * C.D;
+            pref += (long long)c->B * C.nheads * C.D * C.mtiles;
             const void *kb = keys[ci].raw ? kraw : kt;
             const void *vb = keys[ci].raw ? vraw : vt;
             if (!encode_map_5d(&P.tq[oi], q, c->B, c->T, c->H, c->d, C.D) ||
@@ -293,7 +293,7 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, bool w
                 return fail(RAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (dilation %d)", C.D);
         }
         P.prefix[ncls] = pref;
-        for (int oi = 0; oi < ncls; ++oi) P.total_units += (long long)P.cls[oi].mtiles * (c->B * (long long)P.cls[oi].nheads * P.cls[oi].D);
+        P.total_units = pref;
         cudaError_t e = launch_attn_tc(P, c->d, s);
         if (e != cudaSuccess) return cuda_fail(e, "tensor-core attention launch");
     }

@@ -7,40 +7,46 @@
 // merged by log-sum-exp.  The dilated set of residue r = t mod D is a dense
 // causal problem on the interleaved subsequence r, r+D, r+2D, ..., so the
 // dilated part is D independent causal flash attentions per head.  A 5-D TMA
-// map (d, H, D, T/D, B) turns the residue into a coordinate: one box load
-// fetches 128 rows of one subsequence.
+// map (d, H, D, T/D, B) makes the residue a coordinate: one box load fetches
+// 128 rows of one subsequence.
 //
-// One CTA computes one 128-row query tile (one work unit):
-//   warp 0      TMA producer: the Q tile once, then K and V tiles (2-stage rings)
-//   warp 1      TMEM owner and MMA issuer: S = Q K^T into a double-buffered
-//               TMEM S, then O += P V into TMEM O (one elected thread)
-//   warps 2..5  softmax: thread i owns query row i (TMEM lane i); online
-//               softmax in the log2 domain, P written to shared memory in the
-//               128B-swizzled K-major layout the tensor core reads; O is
-//               rescaled in TMEM only when the running max grows by more than
-//               2^8 (the stale max bounds every P by 256).
-// Launch 1 (dilated part): work units are (b, h, residue, query tile), issued
-// heaviest first.  Heads without a window write o and lse directly; heads with
-// one write o (bf16) and lse into scratch.  Launch 2 (window part): 128
-// consecutive query positions against the ceil((W+127)/128) key tiles ending
-// at the diagonal; the epilogue merges with launch 1's (o, lse) by LSE.
+// One CTA computes one work unit: 256 query rows as two 128-row sub-tiles that
+// share every K/V tile load (ping-pong, as in FlashAttention-4):
+//   warp 0      TMA producer: Q0/Q1 once, then K and V tiles (2-stage rings)
+//   warp 1      TMEM owner and MMA issuer (one elected thread), in the order
+//               PV0(j) QK0(j+1) PV1(j) QK1(j+1), so the tensor core works on
+//               one sub-tile while the softmax of the other runs
+//   warps 2..9  two softmax warpgroups, one per sub-tile; thread i of a group
+//               owns query row i (TMEM lane i).  Online softmax in the log2
+//               domain; P (bf16) is written back into TMEM over its own S and
+//               read from there by the PV MMA; O is rescaled in TMEM only when
+//               the running max grows by more than 8 (P stays <= 2^8).
+// TMEM: S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [256+d,256+2d).
+// Launch 1 (dilated part): units are (b, h, residue, 256-row block), grouped
+// by (b, h, residue) with the heaviest block first, so the blocks that share a
+// subsequence's K/V run together and hit L2.  Heads without a window write o
+// and lse; heads with one write o (bf16) and lse into scratch.  Launch 2
+// (window part): 256 consecutive positions against the key tiles covering
+// [t0-W+1, t0+255]; the epilogue merges with launch 1's (o, lse) by LSE.
 //
 // Every mbarrier wait is bounded (globaltimer); on expiry the CTA records
 // RAT_ERR_TIMEOUT, raises a shared abort flag, waits (bounded) for its own
 // copies and MMAs in flight, frees its TMEM and exits.
 #include <cuda.h>
 
-#include "attn_tc.cuh"
-
 #include <mutex>
+
+#include "attn_tc.cuh"
+#include "tmem_io.cuh"
 
 namespace rat {
 
 namespace {
 
 constexpr int BM = 128, BN = 128;
-constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 512;   // S0 [0,128) S1 [128,256) O [256, 256+d)
+constexpr int kSub = 2;                        // query sub-tiles per CTA
+constexpr int kThreads = 64 + kSub * 128;      // TMA warp, MMA warp, two softmax warpgroups
+constexpr uint32_t kTmemCols = 512;
 constexpr long long kWaitNs = 2000000000LL;
 
 // ------------------------------------------------------------ PTX helpers
@@ -113,12 +119,10 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-__device__ __forceinline__ void fence_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
-__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                         uint32_t accumulate) {
+// D(tmem) (+)= A(smem) * B(smem)
+__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
@@ -127,49 +131,21 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint6
         : "memory");
 }
 
+// D(tmem) (+)= A(tmem) * B(smem)
+__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                      smem_u32(bar))
                  : "memory");
-}
-
-// 32 consecutive fp32 columns of this thread's TMEM lane; the load and its
-// completion wait are one asm statement, so no use can move above the wait.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr)
-        : "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n\t"
-        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
-        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
-        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
-        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
-        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
-        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
-        : "memory");
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -183,7 +159,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Shared-memory matrix descriptors (tcgen05 "matrix descriptor"): start
+// Shared-memory matrix descriptor (tcgen05 "matrix descriptor"): start
 // address, leading / stride byte offsets (16-byte units), version 1, and the
 // 128-byte swizzle layout (2).
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -191,8 +167,8 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// Instruction descriptor of kind::f16: fp32 accumulate, bf16 A and B,
-// A K-major, B K-major (b_mn = 0) or MN-major (b_mn = 1), shape M x N.
+// Instruction descriptor of kind::f16: fp32 accumulate, bf16 A and B, A
+// K-major, B K-major (b_mn = 0) or MN-major (b_mn = 1), shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) |
            ((uint32_t)(M >> 4) << 24);
@@ -200,63 +176,128 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {
 
 // ------------------------------------------------------------ work units
 struct Unit {
-    int m;       // query tile index within the subsequence (dilated) or sequence (window)
-    int cls;     // class
-    int b, h, r; // batch, head, residue
+    int m;        // 256-row block index within the subsequence (dilated) or sequence (window)
+    int cls;      // class
+    int b, h, r;  // batch, head, residue
 };
 
+// Units of class c occupy [prefix[c], prefix[c+1]); inside a class, groups of
+// units share (b, h, residue) and list their blocks heaviest (last) first.
 __device__ __forceinline__ Unit decode_unit(const TcParams &p, long long u) {
-    // Classes are sorted by mtiles descending; units go level by level from the
-    // top query tile down, and within a level class by class.
-    Unit out{0, 0, 0, 0, 0};
-    long long rem = u;
-    int k = 0;
-    for (; k < p.ncls; ++k) {
-        const int hi = p.cls[k].mtiles;
-        const int lo = (k + 1 < p.ncls) ? p.cls[k + 1].mtiles : 0;
-        const long long S = p.prefix[k + 1];
-        const long long seg = (long long)(hi - lo) * S;
-        if (rem < seg) {
-            out.m = hi - 1 - (int)(rem / S);
-            rem %= S;
-            break;
-        }
-        rem -= seg;
-    }
     int c = 0;
-    while (c < k && p.prefix[c + 1] <= rem) ++c;
-    long long idx = rem - p.prefix[c];
+    while (c + 1 < p.ncls && p.prefix[c + 1] <= u) ++c;
     const TcClass &C = p.cls[c];
+    const long long rem = u - p.prefix[c];
+    long long g = rem / C.mtiles;
+    Unit out;
     out.cls = c;
-    out.r = (int)(idx % C.D);
-    idx /= C.D;
-    out.h = p.heads[C.head0 + (int)(idx % C.nheads)];
-    out.b = (int)(idx / C.nheads);
+    out.m = C.mtiles - 1 - (int)(rem % C.mtiles);
+    out.r = (int)(g % C.D);
+    g /= C.D;
+    out.h = p.heads[C.head0 + (int)(g % C.nheads)];
+    out.b = (int)(g / C.nheads);
     return out;
 }
 
-// KV tiles of a unit: first key row (subsequence row for the dilated part,
-// position for the window part) of tile j, and the tile count.
-struct KvPlan {
-    int nkv, ks0;
+// Key tiles (128 key rows each, first row 128*j) of a unit: tiles [jlo, jhi];
+// sub-tile i takes [lo[i], hi[i]] (none when its rows all lie past the end).
+struct Plan {
+    int jlo, jhi;
+    int lo[kSub], hi[kSub];
+    bool valid[kSub];
 };
 
-__device__ __forceinline__ KvPlan kv_plan(const TcParams &p, const Unit &u) {
-    if (!p.window_mode) return KvPlan{u.m + 1, 0};
+__device__ __forceinline__ Plan make_plan(const TcParams &p, const Unit &u, int n) {
+    Plan pl;
+    const int q0 = 2 * BM * u.m;
     const int W = p.win[u.h];
-    const int nwt = (W + BN - 1 + BM - 1) / BN;  // tiles covering [t0 - W + 1, t0 + 127]
-    const int j0 = max(0, nwt - u.m - 1);        // skip tiles entirely before position 0
-    return KvPlan{nwt - j0, BM * (u.m + 1 - nwt + j0)};
+    for (int i = 0; i < kSub; ++i) {
+        const int qmin = q0 + BM * i;
+        pl.valid[i] = qmin < n;
+        pl.hi[i] = qmin / BN;
+        if (!p.window_mode) {
+            pl.lo[i] = 0;
+        } else {
+            const int first = qmin - W + 1;  // earliest key of the sub-tile's first row
+            pl.lo[i] = first > 0 ? first / BN : 0;
+        }
+    }
+    pl.jlo = pl.lo[0];
+    pl.jhi = pl.valid[1] ? pl.hi[1] : pl.hi[0];
+    return pl;
+}
+
+__device__ __forceinline__ bool takes(const Plan &pl, int i, int j) {
+    return pl.valid[i] && j >= pl.lo[i] && j <= pl.hi[i];
+}
+
+// Softmax passes over one 128-key row of S in TMEM, in two 64-column halves
+// (the register budget of 10 warps per CTA does not hold a whole row).  MODE:
+// 0 = every key valid, 1 = causal (key k valid iff k <= lim), 2 = window
+// (valid iff lo < k <= lim); k counts keys from the tile's first column and
+// the limits are this row's, so each test is one compare per element.
+template <int MODE>
+__device__ __forceinline__ bool key_ok(int k, int lo, int lim) {
+    return MODE == 0 ? true : MODE == 1 ? (k <= lim) : (k <= lim && k > lo);
+}
+
+// Max of the valid raw scores of this thread's row.
+template <int MODE>
+__device__ __forceinline__ float row_max(uint32_t t_s, int lo, int lim) {
+    float mx8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        uint32_t sr[64];
+        tmem_ld64(t_s + 64 * half, sr);
+#pragma unroll
+        for (int k = 0; k < 64; ++k) {
+            const float x = __uint_as_float(sr[k]);
+            mx8[k & 7] = key_ok<MODE>(64 * half + k, lo, lim) ? fmaxf(mx8[k & 7], x) : mx8[k & 7];
+        }
+    }
+    return fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+}
+
+// P = 2^(s * c - m) (0 for masked keys), packed to bf16 pairs over the first
+// 64 columns of the row: half h lands on columns [32h, 32h+32), which the max
+// pass and half 0 have already consumed.  Returns the row sum of P.
+template <int MODE>
+__device__ __forceinline__ float row_exp_pack(uint32_t t_s, int lo, int lim, float c, float m) {
+    float rs8[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) rs8[k] = 0.f;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        uint32_t sr[64];
+        tmem_ld64(t_s + 64 * half, sr);
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            float e[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int kk = 2 * k + q;
+                const float v = ex2(fmaf(__uint_as_float(sr[kk]), c, -m));
+                e[q] = key_ok<MODE>(64 * half + kk, lo, lim) ? v : 0.f;
+                rs8[kk & 7] += e[q];
+            }
+            pk[k] = pack_bf16(e[0], e[1]);
+        }
+        tmem_st32(t_s + 32 * half, pk);
+    }
+    return ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
 }
 
 template <int HD>
 struct Smem {
-    static constexpr int kTile = BM * HD * 2;         // one Q/K/V tile (bytes)
-    static constexpr int kQ = 0;
-    static constexpr int kK = kQ + kTile;              // 2 stages
-    static constexpr int kV = kK + 2 * kTile;          // 2 stages
-    static constexpr int kP = kV + 2 * kTile;          // 128 x 128 bf16
-    static constexpr int kBytes = kP + BM * BN * 2;
+    static constexpr int kTile = BM * HD * 2;   // one 128-row tile of Q, K or V (bytes)
+    static constexpr int kQ = 0;                 // kSub tiles
+    static constexpr int kK = kQ + kSub * kTile; // 2 stages
+    static constexpr int kV = kK + 2 * kTile;    // 2 stages
+    static constexpr int kBytes = kV + 2 * kTile;
 };
 
 // ------------------------------------------------------------------ kernel
@@ -269,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const uint32_t sbase = smem_u32(smem);
 
     __shared__ uint64_t bar_q, bar_kfull[2], bar_kempty[2], bar_vfull[2], bar_vempty[2];
-    __shared__ uint64_t bar_sfull[2], bar_sfree[2], bar_pfull, bar_pvdone, bar_drain;
+    __shared__ uint64_t bar_sfull[kSub], bar_pfull[kSub], bar_pvdone[kSub], bar_drain;
     __shared__ uint32_t s_tmem;
     __shared__ volatile int s_abort;
 
@@ -278,8 +319,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // remaining work units (the error is already recorded for rat_check_status)
     if (*reinterpret_cast<volatile int *>(&p.hdr->status) == RAT_ERR_TIMEOUT) return;
     const Unit u = decode_unit(p, blockIdx.x);
-    const KvPlan plan = kv_plan(p, u);
     const TcClass &C = p.cls[u.cls];
+    const Plan pl = make_plan(p, u, C.n);
+    const int ntiles = pl.jhi - pl.jlo + 1;
 
     if (threadIdx.x == 0) {
         s_abort = 0;
@@ -289,11 +331,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             mbar_init(&bar_kempty[i], 1);
             mbar_init(&bar_vfull[i], 1);
             mbar_init(&bar_vempty[i], 1);
-            mbar_init(&bar_sfull[i], 1);
-            mbar_init(&bar_sfree[i], 4);
         }
-        mbar_init(&bar_pfull, 4);
-        mbar_init(&bar_pvdone, 1);
+        for (int i = 0; i < kSub; ++i) {
+            mbar_init(&bar_sfull[i], 1);
+            mbar_init(&bar_pfull[i], 4);
+            mbar_init(&bar_pvdone[i], 1);
+        }
         mbar_init(&bar_drain, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -312,26 +355,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const CUtensorMap *mq = &p.tq[u.cls];
             const CUtensorMap *mk = &p.tk[u.cls];
             const CUtensorMap *mv = &p.tv[u.cls];
-            const int qrow = BM * u.m;
-            mbar_expect_tx(&bar_q, L::kTile);
-            for (int cb = 0; cb < NCB; ++cb)
-                tma_load_5d(sbase + L::kQ + cb * BM * 128, mq, &bar_q, cb * 64, u.h, u.r, qrow, u.b);
+            const int nq = pl.valid[1] ? 2 : 1;
+            mbar_expect_tx(&bar_q, nq * L::kTile);
+            for (int i = 0; i < nq; ++i)
+                for (int cb = 0; cb < NCB; ++cb)
+                    tma_load_5d(sbase + L::kQ + i * L::kTile + cb * BM * 128, mq, &bar_q, cb * 64, u.h, u.r,
+                                2 * BM * u.m + BM * i, u.b);
             bool ok = true;
-            int j = 0;
-            for (; j < plan.nkv && ok; ++j) {
-                const int st = j & 1;
-                const uint32_t ph = (uint32_t)(j >> 1) & 1u;
-                const int krow = plan.ks0 + BN * j;
-                if (j >= 2) ok = mbar_wait(&bar_kempty[st], ph ^ 1u, &s_abort);
+            int t = 0;
+            for (; t < ntiles && ok; ++t) {
+                const int st = t & 1;
+                const uint32_t ph = (uint32_t)(t >> 1) & 1u;
+                const int krow = BN * (pl.jlo + t);
+                if (t >= 2) ok = mbar_wait(&bar_kempty[st], ph ^ 1u, &s_abort);
                 if (!ok) break;
                 mbar_expect_tx(&bar_kfull[st], L::kTile);
                 for (int cb = 0; cb < NCB; ++cb)
                     tma_load_5d(sbase + L::kK + st * L::kTile + cb * BN * 128, mk, &bar_kfull[st], cb * 64, u.h,
                                 u.r, krow, u.b);
-                if (j >= 2) ok = mbar_wait(&bar_vempty[st], ph ^ 1u, &s_abort);
+                if (t >= 2) ok = mbar_wait(&bar_vempty[st], ph ^ 1u, &s_abort);
                 if (!ok) {
-                    // K of this tile is in flight: let it land before leaving
-                    mbar_wait(&bar_kfull[st], ph, &s_abort);
+                    volatile int never = 0;
+                    mbar_wait(&bar_kfull[st], ph, &never);  // K of this tile is in flight
                     break;
                 }
                 mbar_expect_tx(&bar_vfull[st], L::kTile);
@@ -342,15 +387,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (!ok) {
                 s_abort = 1;
                 report_error(p.hdr, RAT_ERR_TIMEOUT, (int)blockIdx.x);
-                // copies already issued complete on their own: wait for the last of each ring
-                for (int jj = max(0, j - 2); jj < j; ++jj) {
-                    const int st = jj & 1;
-                    const uint32_t ph = (uint32_t)(jj >> 1) & 1u;
-                    volatile int never = 0;
-                    mbar_wait(&bar_kfull[st], ph, &never);
-                    mbar_wait(&bar_vfull[st], ph, &never);
-                }
                 volatile int never = 0;
+                for (int tt = max(0, t - 2); tt < t; ++tt) {  // the last copies of each ring
+                    const uint32_t ph = (uint32_t)(tt >> 1) & 1u;
+                    mbar_wait(&bar_kfull[tt & 1], ph, &never);
+                    mbar_wait(&bar_vfull[tt & 1], ph, &never);
+                }
                 mbar_wait(&bar_q, 0, &never);
             }
         }
@@ -359,210 +401,216 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16(BM, BN, 0);
             const uint32_t id_pv = idesc_bf16(BM, HD, 1);
-            const uint32_t tq = sbase + L::kQ, tp = sbase + L::kP;
-            bool ok = mbar_wait(&bar_q, 0, &s_abort);
-            int issued_pv = 0;
-            auto issue_pv = [&](int jj) -> bool {
-                const int st = jj & 1;
-                if (!mbar_wait(&bar_pfull, (uint32_t)jj & 1u, &s_abort)) return false;
-                if (!mbar_wait(&bar_vfull[st], (uint32_t)(jj >> 1) & 1u, &s_abort)) return false;
-                tc_fence_after();
-                const uint32_t tv = sbase + L::kV + st * L::kTile;
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t a = sdesc(tp + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
-                    const uint64_t b = sdesc(tv + kk * 16 * 128, BN * 128, 1024);
-                    umma_f16(tmem + 256, a, b, id_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(&bar_pvdone);
-                umma_commit(&bar_vempty[st]);
-                issued_pv = jj + 1;
-                return true;
-            };
-            for (int j = 0; j < plan.nkv && ok; ++j) {
-                const int st = j & 1, sb = j & 1;
-                ok = mbar_wait(&bar_kfull[st], (uint32_t)(j >> 1) & 1u, &s_abort);
-                if (ok && j >= 2) ok = mbar_wait(&bar_sfree[sb], (uint32_t)((j >> 1) - 1) & 1u, &s_abort);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t tk = sbase + L::kK + st * L::kTile;
+            int n_pv[kSub] = {0, 0};
+            auto qk = [&](int i, int t) {  // S_i = Q_i K_t
+                const uint32_t tq = sbase + L::kQ + i * L::kTile;
+                const uint32_t tk = sbase + L::kK + (t & 1) * L::kTile;
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
                     const uint64_t a = sdesc(tq + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
                     const uint64_t b = sdesc(tk + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024);
-                    umma_f16(tmem + sb * BN, a, b, id_qk, kk > 0 ? 1u : 0u);
+                    umma_ss(tmem + BM * i, a, b, id_qk, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&bar_sfull[sb]);
-                umma_commit(&bar_kempty[st]);
-                if (j >= 1) ok = issue_pv(j - 1);
+                umma_commit(&bar_sfull[i]);
+            };
+            auto pv = [&](int i, int t) -> bool {  // O_i += P_i V_t, P_i read from TMEM over S_i
+                if (!mbar_wait(&bar_pfull[i], (uint32_t)n_pv[i] & 1u, &s_abort)) return false;
+                tc_fence_after();
+                const uint32_t tv = sbase + L::kV + (t & 1) * L::kTile;
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    const uint64_t b = sdesc(tv + kk * 16 * 128, BN * 128, 1024);
+                    umma_ts(tmem + 256 + HD * i, tmem + BM * i + 8 * kk, b, id_pv, (n_pv[i] > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(&bar_pvdone[i]);
+                ++n_pv[i];
+                return true;
+            };
+            bool ok = mbar_wait(&bar_q, 0, &s_abort);
+            if (ok) ok = mbar_wait(&bar_kfull[0], 0, &s_abort);
+            if (ok) {
+                tc_fence_after();
+#pragma unroll
+                for (int i = 0; i < kSub; ++i)
+                    if (takes(pl, i, pl.jlo)) qk(i, 0);
+                umma_commit(&bar_kempty[0]);
             }
-            if (ok) ok = issue_pv(plan.nkv - 1);
+            for (int t = 0; t < ntiles && ok; ++t) {
+                const int j = pl.jlo + t;
+                bool v_ready = false, k_ready = false;
+#pragma unroll
+                for (int i = 0; i < kSub; ++i) {
+                    if (!ok) break;
+                    if (takes(pl, i, j)) {
+                        if (!v_ready) {
+                            ok = mbar_wait(&bar_vfull[t & 1], (uint32_t)(t >> 1) & 1u, &s_abort);
+                            if (!ok) break;
+                            v_ready = true;
+                        }
+                        ok = pv(i, t);
+                        if (!ok) break;
+                    }
+                    if (t + 1 < ntiles && takes(pl, i, j + 1)) {
+                        if (!k_ready) {
+                            ok = mbar_wait(&bar_kfull[(t + 1) & 1], (uint32_t)((t + 1) >> 1) & 1u, &s_abort);
+                            if (!ok) break;
+                            tc_fence_after();
+                            k_ready = true;
+                        }
+                        qk(i, t + 1);
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&bar_vempty[t & 1]);
+                if (t + 1 < ntiles) {
+                    if (!k_ready) ok = mbar_wait(&bar_kfull[(t + 1) & 1], (uint32_t)((t + 1) >> 1) & 1u, &s_abort);
+                    umma_commit(&bar_kempty[(t + 1) & 1]);
+                }
+            }
             if (!ok) {
                 s_abort = 1;
                 report_error(p.hdr, RAT_ERR_TIMEOUT, (int)blockIdx.x);
-                // let every MMA already issued finish before TMEM is released:
+                // every MMA already issued must finish before TMEM is released:
                 // a commit arrives once all prior tcgen05 operations are done
-                (void)issued_pv;
                 umma_commit(&bar_drain);
                 volatile int never = 0;
                 mbar_wait(&bar_drain, 0, &never);
             }
         }
     } else {
-        // ------------------------------------------------ softmax warps 2..5
+        // ------------------------------------------------ softmax warpgroups
+        const int sub = (warp - 2) >> 2;         // sub-tile of this warpgroup
         const int q4 = warp & 3;                 // TMEM lane quarter of this warp
-        const int row = q4 * 32 + lane;          // query row of this thread
+        const int row = q4 * 32 + lane;          // query row within the sub-tile
         const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-        const int qi = BM * u.m + row;           // subsequence row (dilated) / position (window)
+        const uint32_t t_s = tmem + lane_base + BM * sub;         // S (and P) of this row
+        const uint32_t t_o = tmem + lane_base + 256 + HD * sub;   // O of this row
+        const int qmin = 2 * BM * u.m + BM * sub;                 // first row of the sub-tile
+        const int qi = qmin + row;                                // subsequence row / position
         const int W = p.win[u.h];
+        const int lo_s = sub ? pl.lo[1] : pl.lo[0];
+        const int nt = (sub ? pl.valid[1] : pl.valid[0]) ? (sub ? pl.hi[1] : pl.hi[0]) - lo_s + 1 : 0;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
-        uint8_t *prow = smem + L::kP + row * 128;
-        for (int j = 0; j < plan.nkv; ++j) {
-            const int sb = j & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfull[sb], (uint32_t)(j >> 1) & 1u, &s_abort));
+        for (int c = 0; c < nt; ++c) {
+            const int j = lo_s + c;
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfull[sub], (uint32_t)c & 1u, &s_abort));
             if (!ok) break;
             tc_fence_after();
-            float s[BN];
-#pragma unroll
-            for (int c = 0; c < BN / 32; ++c) tmem_ld32(tmem + lane_base + sb * BN + c * 32, s + c * 32);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_sfree[sb]);
-
-            // mask: dilated part is causal on subsequence rows; window part keeps
-            // keys in (qi - W, qi]
-            const int ks = plan.ks0 + BN * j;
-            bool full;
-            if (!p.window_mode) full = (j < u.m);
-            else full = (ks + BN - 1 <= BM * u.m) && (ks > BM * u.m + BM - 1 - W);
-            float mx = -INFINITY;
-            if (full) {
-#pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    s[c] *= p.scale_log2;
-                    mx = fmaxf(mx, s[c]);
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    const int kp = ks + c;
-                    const bool valid = p.window_mode ? (kp <= qi && kp > qi - W) : (kp <= qi);
-                    s[c] = valid ? s[c] * p.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, s[c]);
-                }
-            }
+            // mask: causal on subsequence rows (dilated part); keys in (qi - W, qi] (window part)
+            const int ks = BN * j;
+            const bool full = !p.window_mode ? (ks + BN - 1 <= qmin)
+                                             : (ks + BN - 1 <= qmin && ks > qmin + BM - 1 - W);
+            // row limits in keys from the tile's first column
+            const int lim = qi - ks;            // key k valid iff k <= lim (both parts)
+            const int lo = qi - W - ks;         // window part: and k > lo
+            const int mode = full ? 0 : (p.window_mode ? 2 : 1);
+            const float mraw = mode == 0 ? row_max<0>(t_s, lo, lim)
+                             : mode == 1 ? row_max<1>(t_s, lo, lim) : row_max<2>(t_s, lo, lim);
+            const float mx = mraw * p.scale_log2;   // scale > 0 commutes with max
             // running max with lazy rescale: keep the stale max unless the new
             // one exceeds it by more than 8 (P stays <= 2^8)
             float m_new = m_run;
             bool rescale = false;
             if (mx > m_run + 8.f || m_run == -INFINITY) {
                 m_new = mx;
-                rescale = (j > 0) && (m_run != -INFINITY);
+                rescale = (c > 0) && (m_run != -INFINITY);
             }
             const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-            float rs = 0.f;
-#pragma unroll
-            for (int c = 0; c < BN; ++c) {
-                s[c] = ex2(s[c] - m_use);
-                rs += s[c];
-            }
             const float alpha = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_use);
-            l_run = l_run * alpha + rs;
-            m_run = m_new;
-            // O and the P buffer are free once the previous PV has completed
-            if (j > 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bar_pvdone, (uint32_t)(j - 1) & 1u, &s_abort));
+            // O and the TMEM holding the previous P are free once the previous PV completed
+            if (c > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar_pvdone[sub], (uint32_t)(c - 1) & 1u, &s_abort));
                 if (!ok) break;
                 tc_fence_after();
                 if (__any_sync(0xffffffffu, rescale)) {
                     const float f = rescale ? alpha : 1.f;
 #pragma unroll
-                    for (int c = 0; c < HD / 32; ++c) {
-                        float o[32];
-                        tmem_ld32(tmem + lane_base + 256 + c * 32, o);
+                    for (int cc = 0; cc < HD / 32; ++cc) {
+                        uint32_t o[32];
+                        tmem_ld32(t_o + cc * 32, o);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] *= f;
-                        tmem_st32(tmem + lane_base + 256 + c * 32, o);
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+                        tmem_st32(t_o + cc * 32, o);
                     }
                 }
             }
-            // P row -> shared memory, 128B-swizzled K-major (16-byte chunk q of a
-            // 128-byte row lands at chunk q ^ (row & 7))
-#pragma unroll
-            for (int q = 0; q < BN / 8; ++q) {
-                uint4 w;
-                w.x = pack_bf16(s[8 * q + 0], s[8 * q + 1]);
-                w.y = pack_bf16(s[8 * q + 2], s[8 * q + 3]);
-                w.z = pack_bf16(s[8 * q + 4], s[8 * q + 5]);
-                w.w = pack_bf16(s[8 * q + 6], s[8 * q + 7]);
-                const int blk = q >> 3, ch = (q & 7) ^ (row & 7);
-                *reinterpret_cast<uint4 *>(prow + blk * (BM * 128) + ch * 16) = w;
-            }
-            fence_async_smem();
+            const float rs = mode == 0 ? row_exp_pack<0>(t_s, lo, lim, p.scale_log2, m_use)
+                           : mode == 1 ? row_exp_pack<1>(t_s, lo, lim, p.scale_log2, m_use)
+                                       : row_exp_pack<2>(t_s, lo, lim, p.scale_log2, m_use);
+            l_run = l_run * alpha + rs;
+            m_run = m_new;
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_pfull);
+            if (lane == 0) mbar_arrive(&bar_pfull[sub]);
         }
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar_pvdone, (uint32_t)(plan.nkv - 1) & 1u, &s_abort));
-        if (!ok) {
-            s_abort = 1;
-            report_error(p.hdr, RAT_ERR_TIMEOUT, (int)blockIdx.x);
-        } else {
-            tc_fence_after();
-            // ---- epilogue: o = O / l, lse = ln(2) * (m + log2 l)
-            const bool valid_row = qi < C.n;
-            const long long t = p.window_mode ? (long long)qi : (long long)u.r + (long long)C.D * qi;
-            const size_t orow = (((size_t)u.b * p.T + (size_t)t) * p.H + u.h) * HD;
-            const size_t lrow = ((size_t)u.b * p.H + u.h) * p.T + (size_t)t;
-            const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-            float lse2 = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;   // log2 domain
-            __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.o);
-            const bool merge = p.window_mode != 0;
-            float w_self = 1.f, w_dil = 0.f;
-            if (merge && valid_row) {
-                // merge with the dilated part: weights e^(lse_i - max) / sum
-                const float ld2 = p.lse_dil[lrow] * 1.4426950408889634f;
-                const float mm = fmaxf(ld2, lse2);
-                const float e1 = ex2(ld2 - mm), e2 = ex2(lse2 - mm);
-                w_dil = e1 / (e1 + e2);
-                w_self = e2 / (e1 + e2);
-                lse2 = mm + __log2f(e1 + e2);
-            }
+        if (nt > 0) {
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar_pvdone[sub], (uint32_t)(nt - 1) & 1u, &s_abort));
+            if (!ok) {
+                s_abort = 1;
+                report_error(p.hdr, RAT_ERR_TIMEOUT, (int)blockIdx.x);
+            } else {
+                tc_fence_after();
+                // ---- epilogue: o = O / l, lse = ln(2) * (m + log2 l)
+                const bool valid_row = qi < C.n;
+                const long long t = p.window_mode ? (long long)qi : (long long)u.r + (long long)C.D * qi;
+                const size_t orow = (((size_t)u.b * p.T + (size_t)t) * p.H + u.h) * HD;
+                const size_t lrow = ((size_t)u.b * p.H + u.h) * p.T + (size_t)t;
+                const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+                float lse2 = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;  // log2 domain
+                __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.o);
+                const bool merge = p.window_mode != 0;
+                float w_self = 1.f, w_dil = 0.f;
+                if (merge && valid_row) {
+                    // merge with the dilated part: weights e^(lse_i - max) / sum
+                    const float ld2 = p.lse_dil[lrow] * 1.4426950408889634f;
+                    const float mm = fmaxf(ld2, lse2);
+                    const float e1 = ex2(ld2 - mm), e2 = ex2(lse2 - mm);
+                    w_dil = e1 / (e1 + e2);
+                    w_self = e2 / (e1 + e2);
+                    lse2 = mm + __log2f(e1 + e2);
+                }
 #pragma unroll
-            for (int c = 0; c < HD / 32; ++c) {
-                float ov[32];
-                tmem_ld32(tmem + lane_base + 256 + c * 32, ov);
-                if (valid_row) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(o + orow + c * 32);
+                for (int cc = 0; cc < HD / 32; ++cc) {
+                    float ov[32];
+                    {
+                        uint32_t raw[32];
+                        tmem_ld32(t_o + cc * 32, raw);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        float v8[8];
+                        for (int i = 0; i < 32; ++i) ov[i] = __uint_as_float(raw[i]);
+                    }
+                    if (valid_row) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(o + orow + cc * 32);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) v8[i] = ov[8 * q + i] * inv_l * w_self;
-                        if (merge) {
-                            const uint4 prev = dst[q];
-                            const uint32_t pw[4] = {prev.x, prev.y, prev.z, prev.w};
+                        for (int q = 0; q < 4; ++q) {
+                            float v8[8];
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pw[i]));
-                                v8[2 * i] += w_dil * f.x;
-                                v8[2 * i + 1] += w_dil * f.y;
+                            for (int i = 0; i < 8; ++i) v8[i] = ov[8 * q + i] * inv_l * w_self;
+                            if (merge) {
+                                const uint4 prev = dst[q];
+                                const uint32_t pw[4] = {prev.x, prev.y, prev.z, prev.w};
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    const float2 f =
+                                        __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pw[i]));
+                                    v8[2 * i] += w_dil * f.x;
+                                    v8[2 * i + 1] += w_dil * f.y;
+                                }
                             }
+                            uint4 w;
+                            w.x = pack_bf16(v8[0], v8[1]);
+                            w.y = pack_bf16(v8[2], v8[3]);
+                            w.z = pack_bf16(v8[4], v8[5]);
+                            w.w = pack_bf16(v8[6], v8[7]);
+                            dst[q] = w;
                         }
-                        uint4 w;
-                        w.x = pack_bf16(v8[0], v8[1]);
-                        w.y = pack_bf16(v8[2], v8[3]);
-                        w.z = pack_bf16(v8[4], v8[5]);
-                        w.w = pack_bf16(v8[6], v8[7]);
-                        dst[q] = w;
                     }
                 }
-            }
-            if (valid_row) {
-                const float lse = lse2 * 0.69314718055994531f;
-                if (!merge && p.win[u.h] > 0) p.lse_dil[lrow] = lse;   // the window launch merges later
-                else if (p.lse_user) p.lse_user[lrow] = lse;
+                if (valid_row) {
+                    const float lse = lse2 * 0.69314718055994531f;
+                    if (!merge && p.win[u.h] > 0) p.lse_dil[lrow] = lse;  // the window launch merges later
+                    else if (p.lse_user) p.lse_user[lrow] = lse;
+                }
             }
         }
     }

@@ -13,7 +13,7 @@ constexpr int kTcMaxClasses = 8;
 struct TcClass {
     int D;       // dilation (1 in the window launch: natural order)
     int n;       // rows of one residue subsequence (T / D)
-    int mtiles;  // query tiles per subsequence, ceil(n / 128)
+    int mtiles;  // 256-row work units per subsequence, ceil(n / 256)
     int nheads;  // heads in the class
     int head0;   // first entry of the class in TcParams::heads
     int pad;
@@ -24,7 +24,7 @@ struct TcParams {
     CUtensorMap tk[kTcMaxClasses];
     CUtensorMap tv[kTcMaxClasses];
     TcClass cls[kTcMaxClasses];     // sorted by mtiles, descending
-    long long prefix[kTcMaxClasses + 1];  // prefix[c] = sum of units-per-level of classes < c
+    long long prefix[kTcMaxClasses + 1];  // prefix[c] = work units of the classes before c
     int ncls;
     int B, T, H;
     int window_mode;                // 0: dilated part; 1: window part merged with the dilated part
