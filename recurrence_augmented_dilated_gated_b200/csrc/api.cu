@@ -50,9 +50,7 @@ bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 size_t elt_size(int dtype) { return dtype == RAT_F32 ? 4 : 2; }
 
-// scan geometry: 256 threads, d/4 threads per token row, 16 tokens per group
-constexpr int kScanSub = 16;
-int scan_chunk_len(int d) { return (256 / (d / 4)) * kScanSub; }
+int scan_chunk_len(int d) { return scan_chunk_tokens(d); }
 
 constexpr int kDecodeRowsPerSplit = 1024;
 
@@ -211,7 +209,12 @@ rat_status run_scan(const rat_cfg *c, const Layout &L, const void *k, const void
     p.nslices = c->B * n;
     p.nchunks = L.nchunks;
     p.chunk_len = scan_chunk_len(c->d);
-    p.sub_len = kScanSub;
+    p.sub_len = 0;
+    const void *srcs[5] = {k, v, g, kt, vt};
+    p.use_tma_out = kt != nullptr ? 1 : 0;
+    for (int i = 0; i < (p.use_tma_out ? 5 : 3); ++i)
+        if (!encode_map_tokens(&p.tmap[i], srcs[i], c->dtype, c->B, c->T, c->H, c->d, p.chunk_len))
+            return fail(RAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (scan operand %d)", i);
     p.ticket = reinterpret_cast<unsigned *>(ws + L.ticket);
     p.flags = reinterpret_cast<int *>(ws + L.flags);
     p.agg = reinterpret_cast<float *>(ws + L.agg);

@@ -663,6 +663,20 @@ bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int H, int 
 
 // One CTA per SM: each CTA allocates all 512 TMEM columns, so the d = 64
 // variant also asks for more than half of the shared memory.
+bool encode_map_tokens(CUtensorMap *map, const void *base, int dtype, int B, int T, int H, int d, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t e = dtype == RAT_BF16 ? 2 : 4;
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {e * d, e * d * H, e * d * H * T};
+    const cuuint32_t box[4] = {(cuuint32_t)d, 1, (cuuint32_t)box_rows, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(map, dtype == RAT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+              const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 size_t attn_tc_smem_bytes(int hd) {
     const size_t need = (hd == 128 ? (size_t)Smem<128>::kBytes : (size_t)Smem<64>::kBytes) + 1024;
     return need > 120 * 1024 ? need : 120 * 1024;

@@ -2,6 +2,7 @@
 // of librat.so.  Nothing here is part of the public ABI (include/rat.h).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -75,6 +76,10 @@ __device__ __forceinline__ float f4get(const float4 &v, int i) {
 
 // --------------------------------------------------------------- scan (K1)
 struct ScanParams {
+    // 4-D TMA maps (d, H, T, B) of k, v, g (loads) and kt, vt (stores), box
+    // (d, 1, chunk_len, 1); the T extent clips every box at its batch's end
+    CUtensorMap tmap[5];
+    int use_tma_out;        // kt / vt maps are valid
     const void *x[2];       // k, v            [B,T,H,d]
     const void *g;          // gate logits     [B,T,H,d]
     const float *init[2];   // [B,H,d] or null
@@ -145,6 +150,10 @@ rat_status set_last_error(rat_status s, const char *msg);
 
 // launchers (defined in the kernel files); return cudaGetLastError()
 cudaError_t launch_scan(const ScanParams &p, int dtype, cudaStream_t s);
+// tokens per scan chunk for head dimension d
+int scan_chunk_tokens(int d);
+// 4-D TMA map (d, H, T, B) of a [B,T,H,d] tensor, box (d, 1, box_rows, 1), no swizzle
+bool encode_map_tokens(CUtensorMap *map, const void *base, int dtype, int B, int T, int H, int d, int box_rows);
 // final state of the heads in p.head_list, which have no recurrence
 cudaError_t launch_final_of_plain_heads(const ScanParams &p, int dtype, cudaStream_t s);
 cudaError_t launch_attn_simt(const AttnParams &p, int dtype, cudaStream_t s);

@@ -14,18 +14,22 @@
 //   * a CTA takes a dynamic ticket -> (slice = one (b,h) head, chunk of time);
 //     tickets are handed out in launch order, so every predecessor chunk of a
 //     running CTA has already started (forward progress);
-//   * pass 1: each group of d/4 threads (4 channels per thread, one token row
-//     per group) folds its sub-chunk into (A, b_k, b_v), reading g, k, v once;
+//   * three TMA loads stage the chunk's k, v, g rows (d channels of one head)
+//     in shared memory; nothing else reads HBM;
+//   * pass 1: each group of d/4 threads (4 channels per thread) folds its
+//     sub-chunk of rows into (A, b_k, b_v);
 //   * the CTA folds its groups, publishes its aggregate, looks back over
 //     predecessor chunks (aggregates or inclusive states) to get the state
 //     entering the chunk, and publishes its inclusive state;
-//   * pass 2: each group replays its sub-chunk from its carried-in state and
-//     writes the augmented rows (and decode-cache rows).  The pass-2 reads hit
-//     L2: the chunk was read microseconds earlier by the same CTA.
+//   * pass 2: each group replays its sub-chunk from its carried-in state,
+//     overwriting k and v in shared memory with K~ and V~, which two TMA
+//     stores write back (and decode-cache rows are written directly).
 // HBM traffic is the algorithmic 3 reads + 2 writes per (token, channel).
-// Every wait on a predecessor is bounded by the workspace's spin limit; on
-// expiry the CTA records RAT_ERR_TIMEOUT, continues from a zero state and still
-// publishes, so no successor waits forever.
+// Every wait is bounded by the workspace's spin limit; on expiry the CTA
+// records RAT_ERR_TIMEOUT, continues from a zero state and still publishes, so
+// no successor waits forever.
+#include <cuda_fp16.h>
+
 #include "rat_internal.cuh"
 
 namespace rat {
@@ -33,7 +37,11 @@ namespace rat {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 8;
+constexpr int kSub = 16;   // tokens per thread group
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
 
 template <bool kAccurate>
 __device__ __forceinline__ void gate(float g, float &a, float &oma) {
@@ -51,17 +59,41 @@ __device__ __forceinline__ void gate(float g, float &a, float &oma) {
     }
 }
 
+// 4 consecutive channels of one token row in shared memory
+template <typename T> struct Smem4;
+template <> struct Smem4<__nv_bfloat16> {
+    static __device__ __forceinline__ float4 load(const __nv_bfloat16 *p) { return IO4<__nv_bfloat16>::load(p); }
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, float4 v) { IO4<__nv_bfloat16>::store(p, v); }
+};
+template <> struct Smem4<float> {
+    static __device__ __forceinline__ float4 load(const float *p) { return IO4<float>::load(p); }
+    static __device__ __forceinline__ void store(float *p, float4 v) { IO4<float>::store(p, v); }
+};
+
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreads) scan_kernel(const ScanParams p) {
-    constexpr int LPR = D / 4;            // threads per token row
-    constexpr int G = kThreads / LPR;     // thread groups (sub-chunks) per CTA
+__global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ ScanParams p) {
+    constexpr int LPR = D / 4;             // threads per token row (4 channels each)
+    constexpr int G = kThreads / LPR;      // thread groups (sub-chunks) per CTA
+    constexpr int C = G * kSub;            // tokens per chunk
+    constexpr uint32_t kTile = C * D * sizeof(T);
     constexpr bool kAccurate = sizeof(T) == 4;
+    extern __shared__ __align__(128) uint8_t sbuf[];
+    T *tile_k = reinterpret_cast<T *>(sbuf);
+    T *tile_v = reinterpret_cast<T *>(sbuf + kTile);
+    T *tile_g = reinterpret_cast<T *>(sbuf + 2 * kTile);
     __shared__ unsigned s_ticket;
-    __shared__ float s_agg[G][3][D];      // per group (A, b_k, b_v)
-    __shared__ float s_carry[G][2][D];    // state entering each group's sub-chunk
+    __shared__ __align__(8) uint64_t s_bar;
+    __shared__ int s_load_ok;
+    // per group (A, b_k, b_v); after the look-back, slots 1 and 2 hold the
+    // state entering the group's sub-chunk (k and v)
+    __shared__ float s_agg[G][3][D];
 
     const int tid = threadIdx.x;
-    if (tid == 0) s_ticket = atomicAdd(p.ticket, 1u);
+    if (tid == 0) {
+        s_ticket = atomicAdd(p.ticket, 1u);
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&s_bar)) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
     __syncthreads();
     const unsigned ticket = s_ticket;
     const int slice = (int)(ticket % (unsigned)p.nslices);
@@ -70,38 +102,71 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const ScanParams p) {
     const int h = p.head_list[slice % p.nheads];
     const bool rec = p.head_recur[h] != 0;
     const int grp = tid / LPR, c0 = (tid % LPR) * 4;
+    const int tc0 = chunk * C;                                   // first token of the chunk
+    const int r0 = grp * kSub;                                   // first row of this group
+    const int r1 = min(r0 + kSub, p.T - tc0);                    // rows of this group (may be <= r0)
+    const long long limit = p.hdr->spin_limit_ns > 0 ? p.hdr->spin_limit_ns : kDefaultSpinNs;
 
-    const T *xk = static_cast<const T *>(p.x[0]);
-    const T *xv = static_cast<const T *>(p.x[1]);
-    const T *gg = static_cast<const T *>(p.g);
-    const size_t rs = (size_t)p.H * D;                         // stride between tokens
-    const size_t base = ((size_t)b * p.T * p.H + h) * D + c0;  // (b, t=0, h, c0)
-    const long long t0 = (long long)chunk * p.chunk_len + (long long)grp * p.sub_len;
-    const long long t1 = min(t0 + (long long)p.sub_len, (long long)p.T);
+    // ---- stage the chunk: TMA loads of k, v (and g) rows of this head
+    if (tid == 0) {
+        const uint32_t bar = smem_u32(&s_bar);
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+                     "r"((rec ? 3u : 2u) * kTile)
+                     : "memory");
+        for (int i = 0; i < (rec ? 3 : 2); ++i)
+            asm volatile(
+                "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(sbuf + i * kTile)),
+                "l"(reinterpret_cast<uint64_t>(&p.tmap[i])), "r"(0), "r"(h), "r"(tc0), "r"(b), "r"(bar)
+                : "memory");
+        // bounded wait for the bytes to land
+        const unsigned long long t0 = global_ns();
+        int ok = 1;
+        for (uint32_t w = 0;; ++w) {
+            uint32_t done;
+            asm volatile(
+                "{\n\t.reg .pred q;\n\tmbarrier.try_wait.parity.shared::cta.b64 q, [%1], 0;\n\t"
+                "selp.u32 %0, 1, 0, q;\n\t}\n"
+                : "=r"(done)
+                : "r"(bar)
+                : "memory");
+            if (done) break;
+            if ((w & 63u) == 63u && (long long)(global_ns() - t0) > limit) {
+                ok = 0;
+                break;
+            }
+        }
+        s_load_ok = ok;
+        if (!ok) report_error(p.hdr, RAT_ERR_TIMEOUT, (int)ticket);
+    }
+    __syncthreads();
+    const bool loaded = s_load_ok != 0;
 
     // ---- pass 1: fold the sub-chunk into one affine map per channel
     float A[4] = {1.f, 1.f, 1.f, 1.f}, bk[4] = {0.f, 0.f, 0.f, 0.f}, bv[4] = {0.f, 0.f, 0.f, 0.f};
-    for (long long t = t0; t < t1; t += kUnroll) {
-        float4 kk[kUnroll], vv[kUnroll], ga[kUnroll];
+    if (loaded) {
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            if (t + u < t1) {
-                size_t e = base + (size_t)(t + u) * rs;
-                kk[u] = IO4<T>::load(xk + e);
-                vv[u] = IO4<T>::load(xv + e);
-                ga[u] = rec ? IO4<T>::load(gg + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            if (t + u < t1) {
+        for (int r = r0; r < r0 + kSub; ++r) {
+            if (r < r1) {
+                const float4 kk = Smem4<T>::load(tile_k + r * D + c0);
+                const float4 vv = Smem4<T>::load(tile_v + r * D + c0);
+                const float4 gg = rec ? Smem4<T>::load(tile_g + r * D + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
+                float om[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     float a = 0.f, oma = 1.f;
-                    if (rec) gate<kAccurate>(f4get(ga[u], c), a, oma);
+                    if (rec) gate<kAccurate>(f4get(gg, c), a, oma);
+                    om[c] = oma;
                     A[c] *= a;
-                    bk[c] = a * bk[c] + oma * f4get(kk[u], c);
-                    bv[c] = a * bv[c] + oma * f4get(vv[u], c);
+                    bk[c] = a * bk[c] + oma * f4get(kk, c);
+                    bv[c] = a * bv[c] + oma * f4get(vv, c);
+                }
+                if (!kAccurate && rec) {
+                    // keep 1 - a for pass 2 (fp16: relative precision 2^-11)
+                    // over the gate logit this thread has just consumed
+                    __half2 *gh = reinterpret_cast<__half2 *>(tile_g + r * D + c0);
+                    gh[0] = __floats2half2_rn(om[0], om[1]);
+                    gh[1] = __floats2half2_rn(om[2], om[3]);
                 }
             }
         }
@@ -131,7 +196,8 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const ScanParams p) {
                 }
             }
         }
-        const size_t my = (size_t)slice * p.nchunks + chunk;
+        const size_t sbase = (size_t)slice * p.nchunks;
+        const size_t my = sbase + chunk;
         const bool stalled = p.hdr->stall_ticket_plus1 == (long long)ticket + 1;
         float sk[4] = {0.f, 0.f, 0.f, 0.f}, sv[4] = {0.f, 0.f, 0.f, 0.f};  // state entering the chunk
         if (chunk == 0) {
@@ -158,30 +224,67 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const ScanParams p) {
             __syncwarp();
             if (lane == 0) st_release(p.flags + my, 1);
 
-            // look back: fold predecessor aggregates until an inclusive state
+            // Warp-parallel look-back: lane l inspects chunk base - l, so one
+            // round trip finds the nearest inclusive state among 32
+            // predecessors; every aggregate in between is folded in.
             float accA[4] = {1.f, 1.f, 1.f, 1.f}, acck[4] = {0.f, 0.f, 0.f, 0.f}, accv[4] = {0.f, 0.f, 0.f, 0.f};
-            const long long limit = p.hdr->spin_limit_ns > 0 ? p.hdr->spin_limit_ns : kDefaultSpinNs;
             const unsigned long long start = global_ns();
-            int pred = chunk - 1;
+            int base = chunk - 1;
             bool timed_out = false;
+            int spins = 0;
             while (true) {
-                const int *fp = p.flags + (size_t)slice * p.nchunks + pred;
-                int f = ld_acquire(fp);
-                int spins = 0;
-                while (__any_sync(0xffffffffu, f == 0)) {
-                    if (__any_sync(0xffffffffu, (long long)(global_ns() - start) > limit)) {
+                const int mine = base - lane;
+                const int f = mine >= 0 ? ld_acquire(p.flags + sbase + mine) : 0;
+                const unsigned incl = __ballot_sync(0xffffffffu, f == 2);
+                const unsigned none = __ballot_sync(0xffffffffu, f == 0);
+                const int lstar = incl ? __ffs(incl) - 1 : 32;   // nearest inclusive predecessor
+                const unsigned before = lstar == 32 ? 0xffffffffu : ((1u << lstar) - 1u);
+                if (none & before) {  // an aggregate in between is not out yet: look again
+                    if ((long long)(global_ns() - start) > limit) {
                         timed_out = true;
                         break;
                     }
-                    if (++spins > 8) __nanosleep(64);
-                    f = ld_acquire(fp);
+                    if (++spins > 4) __nanosleep(32);
+                    continue;
                 }
-                if (timed_out) break;
-                f = __reduce_min_sync(0xffffffffu, f);
-                const size_t pi = (size_t)slice * p.nchunks + pred;
-                if (f == 2) {
+                __syncwarp();  // the flags acquired by every lane order the reads below
+                // fold aggregates of chunks base, base-1, ..., base-lstar+1
+                if (owns) {
+                    int j = 0;
+                    for (; j + 4 <= lstar; j += 4) {
+                        float ag4[4][12];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float *ag = p.agg + (sbase + (base - j - q)) * 3 * D + cc;
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                ag4[q][c] = ag[c];
+                                ag4[q][4 + c] = ag[D + c];
+                                ag4[q][8 + c] = ag[2 * D + c];
+                            }
+                        }
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                acck[c] = accA[c] * ag4[q][4 + c] + acck[c];
+                                accv[c] = accA[c] * ag4[q][8 + c] + accv[c];
+                                accA[c] *= ag4[q][c];
+                            }
+                    }
+                    for (; j < lstar; ++j) {
+                        const float *ag = p.agg + (sbase + (base - j)) * 3 * D + cc;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            acck[c] = accA[c] * ag[D + c] + acck[c];
+                            accv[c] = accA[c] * ag[2 * D + c] + accv[c];
+                            accA[c] *= ag[c];
+                        }
+                    }
+                }
+                if (lstar < 32) {
                     if (owns) {
-                        const float *in = p.incl + pi * 2 * D + cc;
+                        const float *in = p.incl + (sbase + (base - lstar)) * 2 * D + cc;
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {
                             sk[c] = accA[c] * in[c] + acck[c];
@@ -190,18 +293,8 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const ScanParams p) {
                     }
                     break;
                 }
-                // aggregate of chunk `pred`: acc <- acc o agg(pred)
-                if (owns) {
-                    const float *ag = p.agg + pi * 3 * D + cc;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        float a = ag[c];
-                        acck[c] = accA[c] * ag[D + c] + acck[c];
-                        accv[c] = accA[c] * ag[2 * D + c] + accv[c];
-                        accA[c] *= a;
-                    }
-                }
-                --pred;  // chunk 0 always publishes inclusive, so pred stays >= 0
+                base -= 32;  // 32 aggregates folded, none inclusive: next window
+                spins = 0;
             }
             if (timed_out) {
                 if (lane == 0) report_error(p.hdr, RAT_ERR_TIMEOUT, (int)ticket);
@@ -240,75 +333,94 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const ScanParams p) {
                 if (p.fin[1]) p.fin[1][ib + c] = iv[c];
             }
         }
-        // state entering each group's sub-chunk
+        // state entering each group's sub-chunk (over the consumed b_k, b_v slots)
         if (owns) {
             for (int gi = 0; gi < G; ++gi) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    s_carry[gi][0][cc + c] = sk[c];
-                    s_carry[gi][1][cc + c] = sv[c];
-                    float a = s_agg[gi][0][cc + c];
-                    sk[c] = a * sk[c] + s_agg[gi][1][cc + c];
-                    sv[c] = a * sv[c] + s_agg[gi][2][cc + c];
+                    const float a = s_agg[gi][0][cc + c];
+                    const float ak = s_agg[gi][1][cc + c], av = s_agg[gi][2][cc + c];
+                    s_agg[gi][1][cc + c] = sk[c];
+                    s_agg[gi][2][cc + c] = sv[c];
+                    sk[c] = a * sk[c] + ak;
+                    sv[c] = a * sv[c] + av;
                 }
             }
         }
     }
     __syncthreads();
 
-    // ---- pass 2: replay the sub-chunk from its carried-in state, write rows
+    // ---- pass 2: replay the sub-chunk from its carried-in state; K~ and V~
+    // overwrite k and v in shared memory (same thread, same slot)
     float sk[4], sv[4];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-        sk[c] = s_carry[grp][0][c0 + c];
-        sv[c] = s_carry[grp][1][c0 + c];
+        sk[c] = s_agg[grp][1][c0 + c];
+        sv[c] = s_agg[grp][2][c0 + c];
     }
-    T *ok = static_cast<T *>(p.out[0]);
-    T *ov = static_cast<T *>(p.out[1]);
     T *ck = static_cast<T *>(p.cache[0]);
     T *cv = static_cast<T *>(p.cache[1]);
     const int Dh = p.head_dil[h];
     const long long S = ((long long)p.cap + Dh - 1) / Dh;
     const size_t cbase = ((size_t)b * p.H + h) * (size_t)p.cache_R * D + c0;
-    for (long long t = t0; t < t1; t += kUnroll) {
-        float4 kk[kUnroll], vv[kUnroll], ga[kUnroll];
+    if (loaded) {
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            if (t + u < t1) {
-                size_t e = base + (size_t)(t + u) * rs;
-                kk[u] = IO4<T>::load(xk + e);
-                vv[u] = IO4<T>::load(xv + e);
-                ga[u] = rec ? IO4<T>::load(gg + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            if (t + u < t1) {
+        for (int r = r0; r < r0 + kSub; ++r) {
+            if (r < r1) {
+                const float4 kk = Smem4<T>::load(tile_k + r * D + c0);
+                const float4 vv = Smem4<T>::load(tile_v + r * D + c0);
+                float4 gg = make_float4(0.f, 0.f, 0.f, 0.f);
+                float omc[4] = {1.f, 1.f, 1.f, 1.f};
+                if (rec) {
+                    if (kAccurate) {
+                        gg = Smem4<T>::load(tile_g + r * D + c0);
+                    } else {
+                        const __half2 *gh = reinterpret_cast<const __half2 *>(tile_g + r * D + c0);
+                        const float2 o01 = __half22float2(gh[0]), o23 = __half22float2(gh[1]);
+                        omc[0] = o01.x; omc[1] = o01.y; omc[2] = o23.x; omc[3] = o23.y;
+                    }
+                }
                 float rk[4], rv[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     float a = 0.f, oma = 1.f;
-                    if (rec) gate<kAccurate>(f4get(ga[u], c), a, oma);
-                    sk[c] = a * sk[c] + oma * f4get(kk[u], c);
-                    sv[c] = a * sv[c] + oma * f4get(vv[u], c);
+                    if (rec) {
+                        if (kAccurate) gate<kAccurate>(f4get(gg, c), a, oma);
+                        else { oma = omc[c]; a = 1.f - oma; }
+                    }
+                    sk[c] = a * sk[c] + oma * f4get(kk, c);
+                    sv[c] = a * sv[c] + oma * f4get(vv, c);
                     rk[c] = sk[c];
                     rv[c] = sv[c];
                 }
                 const float4 wk = make_float4(rk[0], rk[1], rk[2], rk[3]);
                 const float4 wv = make_float4(rv[0], rv[1], rv[2], rv[3]);
-                const long long tt = t + u;
-                if (ok) {
-                    size_t e = base + (size_t)tt * rs;
-                    IO4<T>::store(ok + e, wk);
-                    IO4<T>::store(ov + e, wv);
-                }
+                Smem4<T>::store(tile_k + r * D + c0, wk);
+                Smem4<T>::store(tile_v + r * D + c0, wv);
                 if (ck) {
-                    long long row = (tt % Dh) * S + tt / Dh;
-                    size_t e = cbase + (size_t)row * D;
+                    const long long tt = tc0 + r;
+                    const long long row = (tt % Dh) * S + tt / Dh;
+                    const size_t e = cbase + (size_t)row * D;
                     IO4<T>::store(ck + e, wk);
                     IO4<T>::store(cv + e, wv);
                 }
             }
+        }
+    }
+    if (p.use_tma_out && loaded) {
+        // generic-proxy writes of K~ / V~ must be visible to the TMA engine
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncthreads();
+        if (tid == 0) {
+            for (int i = 0; i < 2; ++i)
+                asm volatile(
+                    "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"(
+                        reinterpret_cast<uint64_t>(&p.tmap[3 + i])),
+                    "r"(0), "r"(h), "r"(tc0), "r"(b), "r"(smem_u32(sbuf + i * kTile))
+                    : "memory");
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            // the stores must have read shared memory before the CTA exits
+            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
         }
     }
 }
@@ -316,7 +428,7 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const ScanParams p) {
 // Final state of heads without recurrence (a = 0): s_{T-1} = x_{T-1}.  Used
 // when the scan itself skips those heads (their attention reads k, v directly).
 template <typename T>
-__global__ void final_of_plain_heads_kernel(const ScanParams p) {
+__global__ void final_of_plain_heads_kernel(const __grid_constant__ ScanParams p) {
     const int b = blockIdx.x;
     const T *xs[2] = {static_cast<const T *>(p.x[0]), static_cast<const T *>(p.x[1])};
     for (int i = threadIdx.x; i < p.nheads * p.d; i += blockDim.x) {
@@ -328,7 +440,24 @@ __global__ void final_of_plain_heads_kernel(const ScanParams p) {
     }
 }
 
+template <typename T, int D>
+size_t scan_smem() {
+    constexpr int C = (kThreads / (D / 4)) * kSub;
+    return 3 * (size_t)C * D * sizeof(T);   // k, v, g of one chunk
+}
+
+template <typename T, int D>
+cudaError_t launch_one(const ScanParams &p, unsigned tickets, cudaStream_t s) {
+    const size_t smem = scan_smem<T, D>();
+    cudaError_t e = cudaFuncSetAttribute(scan_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    scan_kernel<T, D><<<tickets, kThreads, smem, s>>>(p);
+    return cudaSuccess;
+}
+
 }  // namespace
+
+int scan_chunk_tokens(int d) { return (kThreads / (d / 4)) * kSub; }
 
 cudaError_t launch_final_of_plain_heads(const ScanParams &p, int dtype, cudaStream_t s) {
     if (p.B == 0 || p.T == 0 || p.nheads == 0) return cudaSuccess;
@@ -341,13 +470,10 @@ cudaError_t launch_final_of_plain_heads(const ScanParams &p, int dtype, cudaStre
 cudaError_t launch_scan(const ScanParams &p, int dtype, cudaStream_t s) {
     const unsigned grid = (unsigned)p.nslices * (unsigned)p.nchunks;
     if (grid == 0) return cudaSuccess;
-    if (dtype == RAT_BF16) {
-        if (p.d == 128) scan_kernel<__nv_bfloat16, 128><<<grid, kThreads, 0, s>>>(p);
-        else scan_kernel<__nv_bfloat16, 64><<<grid, kThreads, 0, s>>>(p);
-    } else {
-        if (p.d == 128) scan_kernel<float, 128><<<grid, kThreads, 0, s>>>(p);
-        else scan_kernel<float, 64><<<grid, kThreads, 0, s>>>(p);
-    }
+    cudaError_t e;
+    if (dtype == RAT_BF16) e = p.d == 128 ? launch_one<__nv_bfloat16, 128>(p, grid, s) : launch_one<__nv_bfloat16, 64>(p, grid, s);
+    else e = p.d == 128 ? launch_one<float, 128>(p, grid, s) : launch_one<float, 64>(p, grid, s);
+    if (e != cudaSuccess) return e;
     count_launches(1);
     return cudaGetLastError();
 }
