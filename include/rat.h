@@ -200,15 +200,16 @@ RAT_API rat_status rat_decode_step(const rat_cfg *cfg, const void *q, const void
  * Arguments and results are those of rat_decode_step minus (ws, ws_bytes).
  *   - Scratch: a static 16 MiB device array inside librat.so, held by every
  *     GPU that loads the library until the process exits.  A step needs
- *     256 + B * items * (d + 2) * 4 bytes, items = sum over heads of
- *     ceil(ceil(cache_cap / D_h) / 1024) + 1; a larger step returns
+ *     about 256 + B * items * (d + 2) * 4 + B * H * 4 bytes, items = sum over
+ *     heads of ceil(ceil(cache_cap / D_h) / 512); a larger step returns
  *     RAT_ERR_UNSUPPORTED with the sizes in rat_last_error().
  *   - The first call on a device (with that device current) looks up the
  *     array's device address (cudaGetSymbolAddress) and caches it; make that
  *     first call before any stream capture.
- *   - All calls share the one array and it keeps the last call's contents
- *     (no call needs it cleared).  Calls whose kernels overlap on a GPU race
- *     on it: order them on one stream.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     each call clears the part that must start at zero (its completion
+ *     counters) itself.  Calls whose kernels overlap on a GPU race on it:
+ *     order them on one stream.
  *   - Never allocates or frees device memory.  An out-of-range pos[b] still
  *     makes the kernel skip that entry (its o is zero), but is not reported:
  *     there is no workspace for rat_check_status to read.

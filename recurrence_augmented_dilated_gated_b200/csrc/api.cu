@@ -52,7 +52,6 @@ size_t elt_size(int dtype) { return dtype == RAT_F32 ? 4 : 2; }
 
 int scan_chunk_len(int d) { return scan_chunk_tokens(d); }
 
-constexpr int kDecodeRowsPerSplit = 1024;
 
 rat_status check_cfg(const rat_cfg *c, bool need_T = true) {
     if (!c) return fail(RAT_ERR_INVALID, "cfg is NULL");
@@ -95,19 +94,6 @@ struct Layout {
     size_t total = 0;
 };
 
-int decode_items(const rat_cfg *c, int cap, int *nsplit, int *item0) {
-    int items = 0;
-    for (int h = 0; h < c->H; ++h) {
-        const int slab = (cap + c->dil[h] - 1) / c->dil[h];
-        const int ns = (slab + kDecodeRowsPerSplit - 1) / kDecodeRowsPerSplit;
-        if (nsplit) nsplit[h] = ns;
-        if (item0) item0[h] = items;
-        items += ns + 1;
-    }
-    if (item0) item0[c->H] = items;
-    return items;
-}
-
 Layout layout(const rat_cfg *c, int op, int cap) {
     Layout L;
     size_t off = sizeof(WsHeader);
@@ -130,8 +116,11 @@ Layout layout(const rat_cfg *c, int op, int cap) {
         L.vt = off; off = align256(off + bytes);
     }
     if (op == RAT_OP_DECODE) {
-        L.items_per_b = decode_items(c, cap, nullptr, nullptr);
-        L.part = off; off = align256(off + (size_t)c->B * L.items_per_b * (c->d + 2) * sizeof(float));
+        DecodeParams tmp;
+        memset(&tmp, 0, sizeof(tmp));
+        L.part = off;
+        off = align256(off + decode_plan(c, cap, &tmp));
+        L.items_per_b = tmp.items_per_b;
     }
     L.total = off;
     return L;
@@ -479,23 +468,21 @@ rat_status rat_decode_step(const rat_cfg *cfg, const void *q, const void *k, con
     if (st != RAT_OK) return st;
     DecodeParams p;
     memset(&p, 0, sizeof(p));
+    decode_plan(cfg, cache_cap, &p);
     p.q = q; p.k = k; p.v = v; p.g = g;
     p.state[0] = state_k; p.state[1] = state_v;
     p.cache[0] = cache_k; p.cache[1] = cache_v;
     p.pos = pos; p.o = o; p.lse = lse;
-    p.part = reinterpret_cast<float *>(static_cast<char *>(ws) + L.part);
-    p.cache_R = cache_rows(cfg, cache_cap);
+    char *w = static_cast<char *>(ws);
+    p.part = reinterpret_cast<float *>(w + L.part);
+    const size_t part_bytes = align256((size_t)cfg->B * p.items_per_b * (cfg->d + 2) * sizeof(float));
+    p.counter = reinterpret_cast<int *>(w + L.part + part_bytes);
     p.cap = cache_cap; p.B = cfg->B; p.H = cfg->H; p.d = cfg->d;
-    p.rows_per_split = kDecodeRowsPerSplit;
     p.scale_log2 = scale_of(cfg) * 1.4426950408889634f;
-    p.items_per_b = decode_items(cfg, cache_cap, p.nsplit, p.item0);
-    for (int h = 0; h < cfg->H; ++h) {
-        p.dil[h] = cfg->dil[h];
-        p.win[h] = cfg->win[h];
-        p.slab[h] = (cache_cap + cfg->dil[h] - 1) / cfg->dil[h];
-        p.recur[h] = head_recur(cfg, h) ? 1 : 0;
-    }
     p.hdr = reinterpret_cast<WsHeader *>(ws);
+    // per-(b,h) completion counters start from zero on every call
+    cudaError_t ez = cudaMemsetAsync(p.counter, 0, (size_t)cfg->B * cfg->H * sizeof(int), (cudaStream_t)stream);
+    if (ez != cudaSuccess) return cuda_fail(ez, "cudaMemsetAsync(decode counters)");
     cudaError_t e = launch_decode(p, cfg->dtype, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     return RAT_OK;

@@ -1,4 +1,4 @@
-// decode.cu -- K4/K5: one decode step of the temporal-mixing operator
+// decode.cu -- K4: one decode step of the temporal-mixing operator
 // ("RAT+: Train Dense, Infer Sparse", Figure 2: decode updates the recurrence
 // with a simple step and attends over the dilated KV cache; Abstract: the
 // dilated pattern cuts the KV cache a step reads by D).
@@ -8,14 +8,16 @@
 //   the new augmented row is stored at cache row (t mod D)*S + t/D,
 //   o = softmax over the multiset  { j <= t, j == t mod D }  (+)  { t-W+1..t }.
 // Softmaxes over disjoint pieces of a key multiset combine exactly by
-// log-sum-exp, so the step is split into independent work items whose partial
-// (unnormalised accumulator, running max, running sum) are merged by K5:
-//   * items 0..nsplit_h-1 : consecutive runs of `rows_per_split` old rows of the
-//     residue slab (t mod D) -- one contiguous, coalesced stream per item;
-//   * the tail item       : the step update of the recurrent state, the append
-//     of the new row, the new row's dilated score, and the window rows.
-// Only the tail item touches the state and the new cache row, and no other
-// item reads that row, so the items need no ordering among themselves.
+// log-sum-exp, so the step is split into independent work items:
+//   * item i of (b, h) streams its run of old rows of the residue slab
+//     (t mod D), one contiguous coalesced region;
+//   * the last item also does the step update of the recurrent state, the
+//     append of the new row, the new row's dilated score and the window rows.
+// Only the last item touches the state and the new cache row, and no other
+// item reads that row, so the items need no ordering among themselves.  Each
+// item writes a partial (unnormalised accumulator, max, sum); the last item
+// of a (b, h) to finish (a per-(b,h) atomic counter, reset by that item)
+// combines the partials by log-sum-exp and writes o and lse.
 // The work is HBM-bound: each cache row is read once, 2*d bytes of bf16 per
 // row and tensor (K~ and V~).
 #include "rat_internal.cuh"
@@ -25,7 +27,8 @@ namespace rat {
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kUnroll = 4;
+constexpr int kBatch = 4;            // rows scored together per row group
+constexpr int kRowsTarget = 512;     // slab rows per work item (upper bound)
 
 // 8 consecutive channels (16 bytes of bf16, 32 bytes of f32) as floats
 template <typename T> struct IO8;
@@ -68,11 +71,6 @@ __device__ __forceinline__ int find_head(const DecodeParams &p, int it) {
     return lo;
 }
 
-// Per row-group online softmax state (log2-domain scores).
-struct Acc8 {
-    float m, l, o[8];
-};
-
 // Sum over the LPR lanes of one row group.  The row groups of a warp can take
 // different branches (their rows differ), so the shuffle names only the lanes
 // of the calling group; every xor partner (offset < LPR) lies inside it.
@@ -84,20 +82,37 @@ __device__ __forceinline__ unsigned group_mask() {
 }
 
 template <int LPR>
-__device__ __forceinline__ float group_sum(float s) {
-    const unsigned mask = group_mask<LPR>();
+__device__ __forceinline__ float group_sum(float s, unsigned mask) {
 #pragma unroll
     for (int off = LPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(mask, s, off);
     return s;
 }
 
-__device__ __forceinline__ void acc_add(Acc8 &a, float s, const float *v) {
-    const float mn = fmaxf(a.m, s);
-    const float corr = exp2f(a.m - mn);
-    const float pj = exp2f(s - mn);
-    a.l = a.l * corr + pj;
+// Online softmax state of one row group (log2-domain scores); o holds this
+// lane's 8 channels of the unnormalised accumulator.
+struct Acc8 {
+    float m, l, o[8];
+};
+
+// Adds the first n <= NB keys (scores s[], values v[][]) in one rescale;
+// fully unrolled and predicated so the arrays stay in registers.
+template <int NB>
+__device__ __forceinline__ void acc_add_batch(Acc8 &a, const float *s, const float (*v)[8], int n) {
+    float mb = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) a.o[i] = a.o[i] * corr + pj * v[i];
+    for (int u = 0; u < NB; ++u) mb = u < n ? fmaxf(mb, s[u]) : mb;
+    const float mn = fmaxf(a.m, mb);
+    const float corr = a.m == -INFINITY ? 0.f : exp2f(a.m - mn);
+    a.l *= corr;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a.o[i] *= corr;
+#pragma unroll
+    for (int u = 0; u < NB; ++u) {
+        const float pj = u < n ? exp2f(s[u] - mn) : 0.f;
+        a.l += pj;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a.o[i] += pj * v[u][i];
+    }
     a.m = mn;
 }
 
@@ -108,124 +123,139 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     __shared__ float s_new[2][D];              // new augmented key / value (rounded)
     __shared__ float s_m[NG], s_l[NG];
     __shared__ float s_o[NG][D];
+    __shared__ int s_last;
 
     const int tid = threadIdx.x;
     const int b = blockIdx.x / p.items_per_b;
     const int it = blockIdx.x % p.items_per_b;
     const int h = find_head(p, it);
     const int li = it - p.item0[h];
-    const bool tail = li == p.nsplit[h];
+    const bool last = li == p.nsplit[h] - 1;
     float *part = p.part + ((size_t)b * p.items_per_b + it) * (D + 2);
     const int t = p.pos[b];
-    if (t < 0 || t >= p.cap) {
-        if (tid == 0) report_error(p.hdr, RAT_ERR_INVALID, b);
-        for (int c = tid; c < D; c += kThreads) part[c] = 0.f;
-        if (tid == 0) { part[D] = -INFINITY; part[D + 1] = 0.f; }
-        return;
-    }
-    const int Dh = p.dil[h], W = p.win[h];
-    const long long S = p.slab[h];
-    const int r = t % Dh;
-    const int n_old = t / Dh;                  // old rows of the residue slab
-    const size_t bh = (size_t)b * p.H + h;
-    const T *ck = static_cast<const T *>(p.cache[0]) + bh * (size_t)p.cache_R * D;
-    const T *cv = static_cast<const T *>(p.cache[1]) + bh * (size_t)p.cache_R * D;
-
     const int grp = tid / LPR, gl = tid % LPR, c0 = gl * 8;
-    float q[8];
-    {
-        const T *qp = static_cast<const T *>(p.q) + bh * D + c0;
-        IO8<T>::load(qp, q);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) q[i] *= p.scale_log2;
-    }
+    const unsigned gmask = group_mask<LPR>();
     Acc8 acc;
     acc.m = -INFINITY;
     acc.l = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc.o[i] = 0.f;
+    const bool valid_pos = t >= 0 && t < p.cap;
+    const size_t bh = (size_t)b * p.H + h;
 
-    if (!tail) {
-        // a run of old rows of the residue slab: rows [i0, i1) at cache rows r*S + i
-        const int i0 = li * p.rows_per_split;
-        const int i1 = min(i0 + p.rows_per_split, n_old);
+    if (!valid_pos) {
+        if (tid == 0) report_error(p.hdr, RAT_ERR_INVALID, b);
+    } else {
+        const int Dh = p.dil[h], W = p.win[h];
+        const long long S = p.slab[h];
+        const int r = t % Dh;
+        const int n_old = t / Dh;              // old rows of the residue slab
+        const T *ck = static_cast<const T *>(p.cache[0]) + bh * (size_t)p.cache_R * D;
+        const T *cv = static_cast<const T *>(p.cache[1]) + bh * (size_t)p.cache_R * D;
+        float q[8];
+        IO8<T>::load(static_cast<const T *>(p.q) + bh * D + c0, q);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) q[i] *= p.scale_log2;
+
+        if (last) {
+            // step update of the recurrent state and append of the new row
+            for (int c = tid; c < D; c += kThreads) {
+                const size_t e = bh * D + c;
+                const float xk = (float)static_cast<const T *>(p.k)[e];
+                const float xv = (float)static_cast<const T *>(p.v)[e];
+                float a = 0.f, oma = 1.f;
+                if (p.recur[h]) {
+                    const float gl_ = fminf(fmaxf((float)static_cast<const T *>(p.g)[e], -80.f), 80.f);
+                    const float ex = expf(-gl_);
+                    a = 1.f / (1.f + ex);
+                    oma = ex * a;
+                }
+                const float sk = a * p.state[0][e] + oma * xk;
+                const float sv = a * p.state[1][e] + oma * xv;
+                p.state[0][e] = sk;
+                p.state[1][e] = sv;
+                const size_t row = (size_t)r * S + n_old;
+                static_cast<T *>(p.cache[0])[bh * (size_t)p.cache_R * D + row * D + c] = to_t<T>(sk);
+                static_cast<T *>(p.cache[1])[bh * (size_t)p.cache_R * D + row * D + c] = to_t<T>(sv);
+                s_new[0][c] = round_to<T>(sk);
+                s_new[1][c] = round_to<T>(sv);
+            }
+        }
+
+        // this item's run of old rows of the residue slab: [i0, i1)
+        const int i0 = li * p.rows_per_item[h];
+        const int i1 = min(i0 + p.rows_per_item[h], n_old);
         const T *kb = ck + ((size_t)r * S) * D + c0;
         const T *vb = cv + ((size_t)r * S) * D + c0;
-        for (int i = i0 + grp; i < i1; i += NG * kUnroll) {
-            float kf[kUnroll][8], vf[kUnroll][8];
+        for (int i = i0 + grp * kBatch; i < i1; i += NG * kBatch) {
+            float kf[kBatch][8], vf[kBatch][8], sc[kBatch];
+            const int n = min(kBatch, i1 - i);
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int ii = i + u * NG;
-                if (ii < i1) {
-                    IO8<T>::load(kb + (size_t)ii * D, kf[u]);
-                    IO8<T>::load(vb + (size_t)ii * D, vf[u]);
+            for (int u = 0; u < kBatch; ++u) {
+                if (u < n) {
+                    IO8<T>::load(kb + (size_t)(i + u) * D, kf[u]);
+                    IO8<T>::load(vb + (size_t)(i + u) * D, vf[u]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) kf[u][c] = vf[u][c] = 0.f;
                 }
             }
 #pragma unroll
-            for (int u = 0; u < kUnroll; ++u) {
-                const int ii = i + u * NG;
-                if (ii < i1) {  // uniform across the row group
-                    float s = 0.f;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) s += q[c] * kf[u][c];
-                    s = group_sum<LPR>(s);
-                    acc_add(acc, s, vf[u]);
-                }
-            }
-        }
-    } else {
-        // step update of the recurrent state and append of the new row
-        for (int c = tid; c < D; c += kThreads) {
-            const size_t e = bh * D + c;
-            const float xk = (float)static_cast<const T *>(p.k)[e];
-            const float xv = (float)static_cast<const T *>(p.v)[e];
-            float a = 0.f, oma = 1.f;
-            if (p.recur[h]) {
-                float gl_ = fminf(fmaxf((float)static_cast<const T *>(p.g)[e], -80.f), 80.f);
-                float ex = expf(-gl_);
-                a = 1.f / (1.f + ex);
-                oma = ex * a;
-            }
-            const float sk = a * p.state[0][e] + oma * xk;
-            const float sv = a * p.state[1][e] + oma * xv;
-            p.state[0][e] = sk;
-            p.state[1][e] = sv;
-            const size_t row = (size_t)r * S + n_old;
-            static_cast<T *>(p.cache[0])[bh * (size_t)p.cache_R * D + row * D + c] = to_t<T>(sk);
-            static_cast<T *>(p.cache[1])[bh * (size_t)p.cache_R * D + row * D + c] = to_t<T>(sv);
-            s_new[0][c] = round_to<T>(sk);
-            s_new[1][c] = round_to<T>(sv);
-        }
-        __syncthreads();
-        // old rows of the window: j in [max(0, t-W+1), t-1]
-        if (W > 0) {
-            const int j0 = max(0, t - W + 1);
-            for (int j = j0 + grp; j < t; j += NG) {
-                const size_t row = (size_t)(j % Dh) * S + (size_t)(j / Dh);
-                float kf[8], vf[8];
-                IO8<T>::load(ck + row * D + c0, kf);
-                IO8<T>::load(cv + row * D + c0, vf);
+            for (int u = 0; u < kBatch; ++u) {
                 float s = 0.f;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) s += q[c] * kf[c];
-                s = group_sum<LPR>(s);
-                acc_add(acc, s, vf);
+                for (int c = 0; c < 8; ++c) s += q[c] * kf[u][c];
+                sc[u] = group_sum<LPR>(s, gmask);   // every lane of the group, u < n or not
             }
+            acc_add_batch<kBatch>(acc, sc, vf, n);
         }
-        // the new row: once in the dilated set, once more in the window
-        if (grp == 0) {
-            float kf[8], vf[8];
+
+        if (last) {
+            __syncthreads();  // the new row is in shared memory
+            // old rows of the window: j in [max(0, t-W+1), t-1]
+            if (W > 0) {
+                const int j0 = max(0, t - W + 1);
+                for (int j = j0 + grp * kBatch; j < t; j += NG * kBatch) {
+                    float kf[kBatch][8], vf[kBatch][8], sc[kBatch];
+                    const int n = min(kBatch, t - j);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                kf[c] = s_new[0][c0 + c];
-                vf[c] = s_new[1][c0 + c];
+                    for (int u = 0; u < kBatch; ++u) {
+                        if (u < n) {
+                            const int jj = j + u;
+                            const size_t row = (size_t)(jj % Dh) * S + (size_t)(jj / Dh);
+                            IO8<T>::load(ck + row * D + c0, kf[u]);
+                            IO8<T>::load(cv + row * D + c0, vf[u]);
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) kf[u][c] = vf[u][c] = 0.f;
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < kBatch; ++u) {
+                        float s = 0.f;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) s += q[c] * kf[u][c];
+                        sc[u] = group_sum<LPR>(s, gmask);
+                    }
+                    acc_add_batch<kBatch>(acc, sc, vf, n);
+                }
             }
-            float s = 0.f;
+            // the new row: once in the dilated set, once more in the window
+            if (grp == 0) {
+                float kv[2][8], sc[2];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) s += q[c] * kf[c];
-            s = group_sum<LPR>(s);
-            acc_add(acc, s, vf);
-            if (W > 0) acc_add(acc, s, vf);
+                for (int c = 0; c < 8; ++c) {
+                    kv[0][c] = s_new[1][c0 + c];
+                    kv[1][c] = kv[0][c];
+                }
+                float s = 0.f;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) s += q[c] * s_new[0][c0 + c];
+                s = group_sum<LPR>(s, gmask);
+                sc[0] = s;
+                sc[1] = s;
+                acc_add_batch<2>(acc, sc, kv, W > 0 ? 2 : 1);
+            }
         }
     }
 
@@ -252,56 +282,78 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         part[D] = M;
         part[D + 1] = L;
     }
-}
 
-// K5: log-sum-exp combine of the items of one (b, h).
-template <typename T, int D>
-__global__ void __launch_bounds__(D) decode_combine_kernel(const DecodeParams p) {
-    const int b = blockIdx.x / p.H, h = blockIdx.x % p.H;
-    const int c = threadIdx.x;
-    const int i0 = p.item0[h], i1 = p.item0[h + 1];
-    const float *base = p.part + (size_t)b * p.items_per_b * (D + 2);
-    float M = -INFINITY;
-    for (int i = i0; i < i1; ++i) M = fmaxf(M, base[(size_t)i * (D + 2) + D]);
-    float L = 0.f, o = 0.f;
-    if (M != -INFINITY) {
-        for (int i = i0; i < i1; ++i) {
-            const float *pi = base + (size_t)i * (D + 2);
-            if (pi[D] == -INFINITY) continue;
-            const float w = exp2f(pi[D] - M);
-            L += pi[D + 1] * w;
-            o += pi[c] * w;
-        }
+    // the last item of (b, h) to finish combines all of them
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        const int done = atomicAdd(p.counter + bh, 1);
+        s_last = done == p.nsplit[h] - 1;
     }
-    const size_t e = ((size_t)b * p.H + h) * D + c;
-    static_cast<T *>(p.o)[e] = to_t<T>(L > 0.f ? o / L : 0.f);
-    if (p.lse && c == 0) p.lse[(size_t)b * p.H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const float *base = p.part + ((size_t)b * p.items_per_b + p.item0[h]) * (D + 2);
+    const int ni = p.nsplit[h];
+    float Mx = -INFINITY;
+    for (int i = 0; i < ni; ++i) Mx = fmaxf(Mx, __ldcg(base + (size_t)i * (D + 2) + D));
+    for (int c = tid; c < D; c += kThreads) {
+        float L = 0.f, o = 0.f;
+        if (Mx != -INFINITY) {
+            for (int i = 0; i < ni; ++i) {
+                const float *pi = base + (size_t)i * (D + 2);
+                const float mi = __ldcg(pi + D);
+                if (mi == -INFINITY) continue;
+                const float w = exp2f(mi - Mx);
+                L += __ldcg(pi + D + 1) * w;
+                o += __ldcg(pi + c) * w;
+            }
+        }
+        static_cast<T *>(p.o)[bh * D + c] = to_t<T>(L > 0.f ? o / L : 0.f);
+        if (p.lse && c == 0) p.lse[bh] = L > 0.f ? (Mx + log2f(L)) * 0.69314718055994531f : -INFINITY;
+    }
+    if (tid == 0) p.counter[bh] = 0;  // ready for the next step
 }
 
 }  // namespace
 
+size_t decode_plan(const rat_cfg *c, int cap, DecodeParams *p) {
+    int items = 0;
+    long long R = 0;
+    for (int h = 0; h < c->H; ++h) {
+        const int D = c->dil[h];
+        const int slab = (cap + D - 1) / D;
+        const int ns = (slab + kRowsTarget - 1) / kRowsTarget;
+        const int n = ns > 0 ? ns : 1;
+        p->dil[h] = D;
+        p->win[h] = c->win[h];
+        p->slab[h] = slab;
+        p->nsplit[h] = n;
+        p->rows_per_item[h] = (slab + n - 1) / n;   // balanced runs
+        p->item0[h] = items;
+        p->recur[h] = (c->recur == nullptr || c->recur[h] != 0) ? 1 : 0;
+        items += n;
+        R = R > (long long)D * slab ? R : (long long)D * slab;
+    }
+    p->item0[c->H] = items;
+    p->items_per_b = items;
+    p->cache_R = R;
+    const size_t part = (size_t)c->B * items * (c->d + 2) * sizeof(float);
+    const size_t part_al = (part + 255) & ~(size_t)255;
+    return part_al + (size_t)c->B * c->H * sizeof(int);
+}
+
 cudaError_t launch_decode(const DecodeParams &p, int dtype, cudaStream_t s) {
     const unsigned grid = (unsigned)p.B * (unsigned)p.items_per_b;
-    const unsigned grid2 = (unsigned)p.B * (unsigned)p.H;
     if (grid == 0) return cudaSuccess;
     if (dtype == RAT_BF16) {
-        if (p.d == 128) {
-            decode_kernel<__nv_bfloat16, 128><<<grid, kThreads, 0, s>>>(p);
-            decode_combine_kernel<__nv_bfloat16, 128><<<grid2, 128, 0, s>>>(p);
-        } else {
-            decode_kernel<__nv_bfloat16, 64><<<grid, kThreads, 0, s>>>(p);
-            decode_combine_kernel<__nv_bfloat16, 64><<<grid2, 64, 0, s>>>(p);
-        }
+        if (p.d == 128) decode_kernel<__nv_bfloat16, 128><<<grid, kThreads, 0, s>>>(p);
+        else decode_kernel<__nv_bfloat16, 64><<<grid, kThreads, 0, s>>>(p);
     } else {
-        if (p.d == 128) {
-            decode_kernel<float, 128><<<grid, kThreads, 0, s>>>(p);
-            decode_combine_kernel<float, 128><<<grid2, 128, 0, s>>>(p);
-        } else {
-            decode_kernel<float, 64><<<grid, kThreads, 0, s>>>(p);
-            decode_combine_kernel<float, 64><<<grid2, 64, 0, s>>>(p);
-        }
+        if (p.d == 128) decode_kernel<float, 128><<<grid, kThreads, 0, s>>>(p);
+        else decode_kernel<float, 64><<<grid, kThreads, 0, s>>>(p);
     }
-    count_launches(2);
+    count_launches(1);
     return cudaGetLastError();
 }
 

@@ -83,23 +83,7 @@ extern "C" rat_status rat_decode_step_noalloc(const rat_cfg *cfg, const void *q,
 
     DecodeParams p;
     memset(&p, 0, sizeof(p));
-    const int rps = 1024;  // rows of a residue slab per split item, as in rat_decode_step
-    int items = 0;
-    int64_t R = 0;
-    for (int h = 0; h < cfg->H; ++h) {
-        const int D = cfg->dil[h];
-        const int slab = (cache_cap + D - 1) / D;
-        p.dil[h] = D;
-        p.win[h] = cfg->win[h];
-        p.slab[h] = slab;
-        p.nsplit[h] = (slab + rps - 1) / rps;
-        p.item0[h] = items;
-        p.recur[h] = (cfg->recur == nullptr || cfg->recur[h] != 0) ? 1 : 0;
-        items += p.nsplit[h] + 1;
-        R = R > (int64_t)D * slab ? R : (int64_t)D * slab;
-    }
-    p.item0[cfg->H] = items;
-    const size_t need = sizeof(WsHeader) + (size_t)cfg->B * items * (cfg->d + 2) * sizeof(float);
+    const size_t need = sizeof(WsHeader) + decode_plan(cfg, cache_cap, &p);
     if (need > kScratchBytes) {
         char msg[200];
         snprintf(msg, sizeof(msg),
@@ -115,15 +99,17 @@ extern "C" rat_status rat_decode_step_noalloc(const rat_cfg *cfg, const void *q,
     p.state[0] = state_k; p.state[1] = state_v;
     p.cache[0] = cache_k; p.cache[1] = cache_v;
     p.pos = pos; p.o = o; p.lse = lse;
-    // every work item writes its whole partial, so nothing needs clearing first
-    p.hdr = static_cast<WsHeader *>(scratch);
-    p.part = reinterpret_cast<float *>(static_cast<char *>(scratch) + sizeof(WsHeader));
-    p.cache_R = R;
+    char *w = static_cast<char *>(scratch);
+    p.hdr = reinterpret_cast<WsHeader *>(w);
+    p.part = reinterpret_cast<float *>(w + sizeof(WsHeader));
+    const size_t part_bytes = ((size_t)cfg->B * p.items_per_b * (cfg->d + 2) * sizeof(float) + 255) & ~(size_t)255;
+    p.counter = reinterpret_cast<int *>(w + sizeof(WsHeader) + part_bytes);
     p.cap = cache_cap; p.B = cfg->B; p.H = cfg->H; p.d = cfg->d;
-    p.items_per_b = items;
-    p.rows_per_split = rps;
     const float scale = cfg->scale > 0.f ? cfg->scale : 1.0f / sqrtf((float)cfg->d);
     p.scale_log2 = scale * 1.4426950408889634f;
+    // the per-(b,h) completion counters must start from zero
+    cudaError_t ez = cudaMemsetAsync(p.counter, 0, (size_t)cfg->B * cfg->H * sizeof(int), (cudaStream_t)stream);
+    if (ez != cudaSuccess) return set_last_error(RAT_ERR_CUDA, "rat_decode_step_noalloc: counter reset failed");
     cudaError_t e = launch_decode(p, cfg->dtype, (cudaStream_t)stream);
     if (e != cudaSuccess) return set_last_error(RAT_ERR_CUDA, "rat_decode_step_noalloc: launch failed");
     return RAT_OK;

@@ -128,19 +128,25 @@ struct DecodeParams {
     void *o;                     // [B,H,d]
     float *lse;                  // [B,H] or null
     float *part;                 // [B][items][d + 2]  (acc[d], m, l) per work item
+    int *counter;                // [B][H] items finished (the last one combines and resets it)
     long long cache_R;
     int cap, B, H, d;
-    int items_per_b;             // sum over heads of (nsplit_h + 1)
-    int rows_per_split;
+    int items_per_b;             // sum over heads of nsplit
     float scale_log2;
     int dil[kMaxHeads];
     int win[kMaxHeads];
     int slab[kMaxHeads];         // ceil(cap / dil)
-    int nsplit[kMaxHeads];       // dilated splits of head h (the +1 tail item follows them)
+    int nsplit[kMaxHeads];       // work items of head h (the last also does the step update)
+    int rows_per_item[kMaxHeads];// slab rows per work item
     int item0[kMaxHeads + 1];    // first item of head h within a batch entry
     unsigned char recur[kMaxHeads];
     WsHeader *hdr;
 };
+
+// Fills the per-head split plan, items_per_b and cache_R of `p` for a decode
+// step with capacity `cap` (host).  Returns the scratch bytes the step needs
+// after the workspace header: partials plus per-(b,h) counters.
+size_t decode_plan(const rat_cfg *c, int cap, DecodeParams *p);
 
 // Process-wide count of kernels this library has launched (rat_launch_count).
 void count_launches(int n);
