@@ -26,9 +26,44 @@ namespace rat {
 
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kCompute = 128;        // threads that score rows (4 warps)
+constexpr int kThreads = kCompute + 32;  // plus one producer warp
 constexpr int kBatch = 4;            // rows scored together per row group
 constexpr int kRowsTarget = 512;     // slab rows per work item (upper bound)
+constexpr int kStages = 4;           // shared-memory ring of K/V row blocks
+constexpr long long kWaitNs = 2000000000LL;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase with `parity`; false on timeout or abort.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (*abort_flag) return false;
+            if ((long long)(global_ns() - t0) > kWaitNs) return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void compute_sync() {  // the kCompute scoring threads only
+    asm volatile("bar.sync 1, %0;" ::"n"(kCompute) : "memory");
+}
 
 // 8 consecutive channels (16 bytes of bf16, 32 bytes of f32) as floats
 template <typename T> struct IO8;
@@ -119,13 +154,20 @@ __device__ __forceinline__ void acc_add_batch(Acc8 &a, const float *s, const flo
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) {
     constexpr int LPR = D / 8;                 // lanes per cache row (8 channels each)
-    constexpr int NG = kThreads / LPR;         // row groups per CTA
+    constexpr int NG = kCompute / LPR;         // row groups
+    constexpr int RS = NG * kBatch;            // rows per ring stage
+    constexpr uint32_t kRowBytes = D * sizeof(T);
+    constexpr uint32_t kStageBytes = 2 * RS * kRowBytes;   // K and V rows
+    extern __shared__ __align__(128) uint8_t ring[];
+    __shared__ __align__(8) uint64_t s_full[kStages], s_empty[kStages];
     __shared__ float s_new[2][D];              // new augmented key / value (rounded)
     __shared__ float s_m[NG], s_l[NG];
     __shared__ float s_o[NG][D];
     __shared__ int s_last;
+    __shared__ volatile int s_abort;
 
     const int tid = threadIdx.x;
+    const int warp = tid >> 5;
     const int b = blockIdx.x / p.items_per_b;
     const int it = blockIdx.x % p.items_per_b;
     const int h = find_head(p, it);
@@ -133,25 +175,81 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     const bool last = li == p.nsplit[h] - 1;
     float *part = p.part + ((size_t)b * p.items_per_b + it) * (D + 2);
     const int t = p.pos[b];
-    const int grp = tid / LPR, gl = tid % LPR, c0 = gl * 8;
-    const unsigned gmask = group_mask<LPR>();
+    const bool valid_pos = t >= 0 && t < p.cap;
+    const size_t bh = (size_t)b * p.H + h;
+    const int Dh = p.dil[h], W = p.win[h];
+    const long long S = p.slab[h];
+    const int r = valid_pos ? t % Dh : 0;
+    const int n_old = valid_pos ? t / Dh : 0;    // old rows of the residue slab
+    const int i0 = li * p.rows_per_item[h];      // this item's run of old rows: [i0, i1)
+    const int i1 = min(i0 + p.rows_per_item[h], n_old);
+    const int nrows = max(0, i1 - i0);
+    const int nst = (nrows + RS - 1) / RS;       // ring stages this item streams
+    const T *ck = static_cast<const T *>(p.cache[0]) + bh * (size_t)p.cache_R * D;
+    const T *cv = static_cast<const T *>(p.cache[1]) + bh * (size_t)p.cache_R * D;
+
+    if (tid == 0) {
+        s_abort = 0;
+        for (int i = 0; i < kStages; ++i) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&s_full[i])) : "memory");
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&s_empty[i])), "r"(kCompute / 32)
+                         : "memory");
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        if (!valid_pos) report_error(p.hdr, RAT_ERR_INVALID, b);
+    }
+    __syncthreads();
+
     Acc8 acc;
     acc.m = -INFINITY;
     acc.l = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc.o[i] = 0.f;
-    const bool valid_pos = t >= 0 && t < p.cap;
-    const size_t bh = (size_t)b * p.H + h;
+    const int grp = tid / LPR, gl = tid % LPR, c0 = gl * 8;
 
-    if (!valid_pos) {
-        if (tid == 0) report_error(p.hdr, RAT_ERR_INVALID, b);
-    } else {
-        const int Dh = p.dil[h], W = p.win[h];
-        const long long S = p.slab[h];
-        const int r = t % Dh;
-        const int n_old = t / Dh;              // old rows of the residue slab
-        const T *ck = static_cast<const T *>(p.cache[0]) + bh * (size_t)p.cache_R * D;
-        const T *cv = static_cast<const T *>(p.cache[1]) + bh * (size_t)p.cache_R * D;
+    if (warp == kCompute / 32) {
+        // ------------------------------------------------ producer: stream the
+        // item's contiguous run of K~ and V~ rows through the ring
+        if ((tid & 31) == 0 && valid_pos) {
+            const char *kb = reinterpret_cast<const char *>(ck + ((size_t)r * S + i0) * D);
+            const char *vb = reinterpret_cast<const char *>(cv + ((size_t)r * S + i0) * D);
+            int sidx = 0;
+            bool ok = true;
+            for (; sidx < nst; ++sidx) {
+                const int st = sidx % kStages;
+                if (sidx >= kStages &&
+                    !mbar_wait(smem_u32(&s_empty[st]), (uint32_t)(sidx / kStages - 1) & 1u, &s_abort)) {
+                    ok = false;
+                    break;
+                }
+                const int nr = min(RS, nrows - sidx * RS);
+                const uint32_t bytes = (uint32_t)nr * kRowBytes;
+                const uint32_t full = smem_u32(&s_full[st]);
+                const uint32_t dk = smem_u32(ring + st * kStageBytes);
+                const uint32_t dv = dk + RS * kRowBytes;
+                const size_t off = (size_t)sidx * RS * kRowBytes;
+                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full), "r"(2 * bytes)
+                             : "memory");
+                asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                                 dk),
+                             "l"(kb + off), "r"(bytes), "r"(full)
+                             : "memory");
+                asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                                 dv),
+                             "l"(vb + off), "r"(bytes), "r"(full)
+                             : "memory");
+            }
+            if (!ok) {
+                s_abort = 1;
+                report_error(p.hdr, RAT_ERR_TIMEOUT, (int)blockIdx.x);
+                volatile int never = 0;
+                for (int q = max(0, sidx - kStages); q < sidx; ++q)  // copies still in flight
+                    mbar_wait(smem_u32(&s_full[q % kStages]), (uint32_t)(q / kStages) & 1u, &never);
+            }
+        }
+    } else if (valid_pos) {
+        // ------------------------------------------------ scoring warps
+        const unsigned gmask = group_mask<LPR>();
         float q[8];
         IO8<T>::load(static_cast<const T *>(p.q) + bh * D + c0, q);
 #pragma unroll
@@ -159,7 +257,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
 
         if (last) {
             // step update of the recurrent state and append of the new row
-            for (int c = tid; c < D; c += kThreads) {
+            for (int c = tid; c < D; c += kCompute) {
                 const size_t e = bh * D + c;
                 const float xk = (float)static_cast<const T *>(p.k)[e];
                 const float xv = (float)static_cast<const T *>(p.v)[e];
@@ -182,36 +280,47 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
             }
         }
 
-        // this item's run of old rows of the residue slab: [i0, i1)
-        const int i0 = li * p.rows_per_item[h];
-        const int i1 = min(i0 + p.rows_per_item[h], n_old);
-        const T *kb = ck + ((size_t)r * S) * D + c0;
-        const T *vb = cv + ((size_t)r * S) * D + c0;
-        for (int i = i0 + grp * kBatch; i < i1; i += NG * kBatch) {
+        // the item's old rows, one ring stage at a time; group grp takes rows
+        // [grp*kBatch, grp*kBatch + kBatch) of each stage
+        bool ok = true;
+        for (int sidx = 0; sidx < nst; ++sidx) {
+            const int st = sidx % kStages;
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(smem_u32(&s_full[st]), (uint32_t)(sidx / kStages) & 1u, &s_abort));
+            if (!ok) break;
+            const int nr = min(RS, nrows - sidx * RS);
+            const int n = max(0, min(kBatch, nr - grp * kBatch));
+            const T *sk_ = reinterpret_cast<const T *>(ring + st * kStageBytes);
+            const T *sv_ = sk_ + RS * D;
             float kf[kBatch][8], vf[kBatch][8], sc[kBatch];
-            const int n = min(kBatch, i1 - i);
 #pragma unroll
             for (int u = 0; u < kBatch; ++u) {
                 if (u < n) {
-                    IO8<T>::load(kb + (size_t)(i + u) * D, kf[u]);
-                    IO8<T>::load(vb + (size_t)(i + u) * D, vf[u]);
+                    IO8<T>::load(sk_ + (grp * kBatch + u) * D + c0, kf[u]);
+                    IO8<T>::load(sv_ + (grp * kBatch + u) * D + c0, vf[u]);
                 } else {
 #pragma unroll
                     for (int c = 0; c < 8; ++c) kf[u][c] = vf[u][c] = 0.f;
                 }
             }
+            __syncwarp();
+            if ((tid & 31) == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&s_empty[st])) : "memory");
 #pragma unroll
             for (int u = 0; u < kBatch; ++u) {
-                float s = 0.f;
+                float s2 = 0.f;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) s += q[c] * kf[u][c];
-                sc[u] = group_sum<LPR>(s, gmask);   // every lane of the group, u < n or not
+                for (int c = 0; c < 8; ++c) s2 += q[c] * kf[u][c];
+                sc[u] = group_sum<LPR>(s2, gmask);
             }
             acc_add_batch<kBatch>(acc, sc, vf, n);
         }
+        if (!ok) {
+            s_abort = 1;
+            if (tid == 0) report_error(p.hdr, RAT_ERR_TIMEOUT, (int)blockIdx.x);
+        }
 
         if (last) {
-            __syncthreads();  // the new row is in shared memory
+            compute_sync();  // the new row is in shared memory
             // old rows of the window: j in [max(0, t-W+1), t-1]
             if (W > 0) {
                 const int j0 = max(0, t - W + 1);
@@ -232,10 +341,10 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                     }
 #pragma unroll
                     for (int u = 0; u < kBatch; ++u) {
-                        float s = 0.f;
+                        float s2 = 0.f;
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) s += q[c] * kf[u][c];
-                        sc[u] = group_sum<LPR>(s, gmask);
+                        for (int c = 0; c < 8; ++c) s2 += q[c] * kf[u][c];
+                        sc[u] = group_sum<LPR>(s2, gmask);
                     }
                     acc_add_batch<kBatch>(acc, sc, vf, n);
                 }
@@ -248,39 +357,41 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                     kv[0][c] = s_new[1][c0 + c];
                     kv[1][c] = kv[0][c];
                 }
-                float s = 0.f;
+                float s2 = 0.f;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) s += q[c] * s_new[0][c0 + c];
-                s = group_sum<LPR>(s, gmask);
-                sc[0] = s;
-                sc[1] = s;
+                for (int c = 0; c < 8; ++c) s2 += q[c] * s_new[0][c0 + c];
+                s2 = group_sum<LPR>(s2, gmask);
+                sc[0] = s2;
+                sc[1] = s2;
                 acc_add_batch<2>(acc, sc, kv, W > 0 ? 2 : 1);
             }
         }
     }
 
-    // fold the row groups of this CTA into one partial
-    if (gl == 0) {
-        s_m[grp] = acc.m;
-        s_l[grp] = acc.l;
-    }
+    // fold the row groups into one partial (scoring threads)
+    if (tid < kCompute) {
+        if (gl == 0) {
+            s_m[grp] = acc.m;
+            s_l[grp] = acc.l;
+        }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) s_o[grp][c0 + i] = acc.o[i];
-    __syncthreads();
-    float M = -INFINITY;
-    for (int g2 = 0; g2 < NG; ++g2) M = fmaxf(M, s_m[g2]);
-    for (int c = tid; c < D; c += kThreads) {
-        float o = 0.f;
-        for (int g2 = 0; g2 < NG; ++g2)
-            if (s_m[g2] != -INFINITY) o += s_o[g2][c] * exp2f(s_m[g2] - M);
-        part[c] = o;
-    }
-    if (tid == 0) {
-        float L = 0.f;
-        for (int g2 = 0; g2 < NG; ++g2)
-            if (s_m[g2] != -INFINITY) L += s_l[g2] * exp2f(s_m[g2] - M);
-        part[D] = M;
-        part[D + 1] = L;
+        for (int i = 0; i < 8; ++i) s_o[grp][c0 + i] = acc.o[i];
+        compute_sync();
+        float M = -INFINITY;
+        for (int g2 = 0; g2 < NG; ++g2) M = fmaxf(M, s_m[g2]);
+        for (int c = tid; c < D; c += kCompute) {
+            float o = 0.f;
+            for (int g2 = 0; g2 < NG; ++g2)
+                if (s_m[g2] != -INFINITY) o += s_o[g2][c] * exp2f(s_m[g2] - M);
+            part[c] = o;
+        }
+        if (tid == 0) {
+            float L = 0.f;
+            for (int g2 = 0; g2 < NG; ++g2)
+                if (s_m[g2] != -INFINITY) L += s_l[g2] * exp2f(s_m[g2] - M);
+            part[D] = M;
+            part[D + 1] = L;
+        }
     }
 
     // the last item of (b, h) to finish combines all of them
@@ -291,13 +402,13 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         s_last = done == p.nsplit[h] - 1;
     }
     __syncthreads();
-    if (!s_last) return;
+    if (!s_last || tid >= kCompute) return;
     __threadfence();
     const float *base = p.part + ((size_t)b * p.items_per_b + p.item0[h]) * (D + 2);
     const int ni = p.nsplit[h];
     float Mx = -INFINITY;
     for (int i = 0; i < ni; ++i) Mx = fmaxf(Mx, __ldcg(base + (size_t)i * (D + 2) + D));
-    for (int c = tid; c < D; c += kThreads) {
+    for (int c = tid; c < D; c += kCompute) {
         float L = 0.f, o = 0.f;
         if (Mx != -INFINITY) {
             for (int i = 0; i < ni; ++i) {
@@ -313,6 +424,16 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         if (p.lse && c == 0) p.lse[bh] = L > 0.f ? (Mx + log2f(L)) * 0.69314718055994531f : -INFINITY;
     }
     if (tid == 0) p.counter[bh] = 0;  // ready for the next step
+}
+
+template <typename T, int D>
+cudaError_t launch_typed(const DecodeParams &p, unsigned grid, cudaStream_t s) {
+    constexpr int RS = (kCompute / (D / 8)) * kBatch;
+    const size_t smem = (size_t)kStages * 2 * RS * D * sizeof(T);
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    decode_kernel<T, D><<<grid, kThreads, smem, s>>>(p);
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -346,13 +467,10 @@ size_t decode_plan(const rat_cfg *c, int cap, DecodeParams *p) {
 cudaError_t launch_decode(const DecodeParams &p, int dtype, cudaStream_t s) {
     const unsigned grid = (unsigned)p.B * (unsigned)p.items_per_b;
     if (grid == 0) return cudaSuccess;
-    if (dtype == RAT_BF16) {
-        if (p.d == 128) decode_kernel<__nv_bfloat16, 128><<<grid, kThreads, 0, s>>>(p);
-        else decode_kernel<__nv_bfloat16, 64><<<grid, kThreads, 0, s>>>(p);
-    } else {
-        if (p.d == 128) decode_kernel<float, 128><<<grid, kThreads, 0, s>>>(p);
-        else decode_kernel<float, 64><<<grid, kThreads, 0, s>>>(p);
-    }
+    cudaError_t e;
+    if (dtype == RAT_BF16) e = p.d == 128 ? launch_typed<__nv_bfloat16, 128>(p, grid, s) : launch_typed<__nv_bfloat16, 64>(p, grid, s);
+    else e = p.d == 128 ? launch_typed<float, 128>(p, grid, s) : launch_typed<float, 64>(p, grid, s);
+    if (e != cudaSuccess) return e;
     count_launches(1);
     return cudaGetLastError();
 }
