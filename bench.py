@@ -155,14 +155,16 @@ class ClockSampler:
                 "samples": len(sel), "reasons": sorted(reasons), "window": window}
 
 
-def profile_traffic(name):
-    """Per-launch DRAM bytes of kernel `name` from its committed ncu summary,
-    or None if there is none or the kernel source changed since the capture."""
+def profile_traffic(name, key=None):
+    """Per-launch DRAM bytes from the committed ncu summary profiles/<name>.md
+    (line `traffic_bytes_per_launch[key]: ...` when key is given), or None if
+    there is none or the kernel source changed since the capture."""
     path = os.path.join(ROOT, "profiles", name + ".md")
     if not os.path.exists(path):
         return None
     txt = open(path).read()
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)\s*\(source sha1 ([0-9a-f]+) of ([\w./]+)\)", txt)
+    tag = r"\[" + re.escape(key) + r"\]" if key else ""
+    m = re.search(r"traffic_bytes_per_launch" + tag + r":\s*([0-9.eE+]+)\s*\(source sha1 ([0-9a-f]+) of ([\w./]+)\)", txt)
     if not m:
         return None
     src = os.path.join(ROOT, m.group(3))
@@ -506,7 +508,7 @@ def main():
                         "roofline": {"bound": "hbm", "achieved": r["bytes"] / (r["ms"] * 1e-3) / 1e9,
                                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                      "frac": r["bytes"] / (r["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                                     "traffic": profile_traffic("decode_ctx%d" % r["ctx"])},
+                                     "traffic": profile_traffic("decode_batch256", "decode_ctx%d" % r["ctx"])},
                         "gpu_launches": r["launches"]} for r in dec],
         }
     if not args.no_cpu and world == 1:
