@@ -138,6 +138,57 @@ def test_tensor_core_attention_every_element(d, case):
     assert float(err.max()) < 5e-2, "worst row rel err %.3g" % float(err.max())
 
 
+def test_many_dilation_classes_split_over_launches():
+    # 12 distinct dilations (more than one tensor-core launch holds) plus a
+    # window on some heads; every head still matches the oracle
+    B, T, d = 1, 2048, 64
+    dil = [1, 2, 4, 8, 16, 32, 64, 128, 256, 512, 1024, 2048] * 2
+    win = [0] * 12 + [3, 0, 17, 0, 64, 0, 129, 0, 1, 0, 2048, 5]
+    H = len(dil)
+    dtype = torch.bfloat16
+    q, kt, vt, _ = inputs(B, T, H, d, dtype, seed=400)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, T, device=DEV)
+    ws = rat.workspace(cfg, rat.RAT_OP_ATTN)
+    rat.rat_dilated_attn_prefill(cfg, q, kt, vt, o, lse, ws)
+    rat.rat_check_status(ws)
+    ro, rl = oracle.attention(f64(q), f64(kt), f64(vt), dil, win)
+    for h in range(H):
+        assert_close(o[:, :, h], ro[:, :, h], dtype, "o head %d (D=%d W=%d)" % (h, dil[h], win[h]))
+    assert_close(lse, rl, dtype, "lse")
+
+
+@pytest.mark.parametrize("T", [1, 2, 130])
+def test_short_sequences_on_both_paths(T):
+    # T = 1 (one row, one key), tiny T, and T just past one tile, for D | T
+    # (tensor-core kernel) and D not dividing T (CUDA-core kernel)
+    B, H, d = 2, 4, 128
+    dil, win, recur = [1, 1, 3, T + 1], [0, 2, 1, 0], [0, 1, 1, 1]
+    dtype = torch.bfloat16
+    q, k, v, g = inputs(B, T, H, d, dtype, seed=500 + T)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur)
+    out = rat.mix_prefill(cfg, q, k, v, g, want_kv=True)
+    rat.rat_check_status(out["ws"])
+    ref = oracle_prefill(q, k, v, g, dil, win, recur)
+    for key in ("o", "lse", "kt", "vt", "final_k", "final_v"):
+        assert_close(out[key], ref[key], dtype, key)
+
+
+def test_maximum_head_count():
+    # H = 256, the largest head count of this build, mixed dilations
+    B, T, H, d = 1, 64, 256, 64
+    dil = [1 + (h % 4) for h in range(H)]
+    win = [(h % 3) * 4 for h in range(H)]
+    dtype = torch.bfloat16
+    q, k, v, g = inputs(B, T, H, d, dtype, seed=600)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win)
+    out = rat.mix_prefill(cfg, q, k, v, g)
+    rat.rat_check_status(out["ws"])
+    ref = oracle_prefill(q, k, v, g, dil, win, None)
+    assert_close(out["o"], ref["o"], dtype, "o")
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_mix_hybrid_heads_every_element(dtype):
     # dense heads (D=1, no recurrence) next to dilated + windowed recurrent heads
