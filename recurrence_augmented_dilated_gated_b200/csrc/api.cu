@@ -52,6 +52,10 @@ size_t elt_size(int dtype) { return dtype == RAT_F32 ? 4 : 2; }
 
 int scan_chunk_len(int d) { return scan_chunk_tokens(d); }
 
+// Work-unit counters for the tensor-core attention launches of one call
+// (each launch takes up to 8 classes of heads, so 256 heads need at most 64).
+constexpr int kAttnTickets = 128;
+
 
 rat_status check_cfg(const rat_cfg *c, bool need_T = true) {
     if (!c) return fail(RAT_ERR_INVALID, "cfg is NULL");
@@ -87,7 +91,7 @@ int64_t cache_rows(const rat_cfg *c, int cap) {
 
 struct Layout {
     size_t ticket = 0, flags = 0, agg = 0, incl = 0;  // scan
-    size_t lse_dil = 0;                               // attention
+    size_t lse_dil = 0, att_ticket = 0;               // attention
     size_t kt = 0, vt = 0;                            // mix scratch
     size_t part = 0;                                  // decode
     int nchunks = 0, items_per_b = 0;
@@ -109,6 +113,7 @@ Layout layout(const rat_cfg *c, int op, int cap) {
     }
     if (op == RAT_OP_ATTN || op == RAT_OP_MIX || op == RAT_OP_MIX_CALLER_KV) {
         L.lse_dil = off; off = align256(off + (size_t)c->B * c->H * c->T * sizeof(float));
+        L.att_ticket = off; off += kAttnTickets * sizeof(unsigned);   // one work counter per launch
     }
     if (op == RAT_OP_MIX) {
         const size_t bytes = (size_t)c->B * c->T * c->H * c->d * elt;
@@ -226,7 +231,8 @@ bool tc_head(const rat_cfg *c, int h) { return c->dtype == RAT_BF16 && c->T % c-
 // window_mode), grouped into classes of equal (dilation, K/V source).
 rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, bool window_mode, const void *q,
                           const void *kt, const void *vt, const void *kraw, const void *vraw,
-                          const bool *raw_head, void *o, float *lse, float *lse_dil, char *ws, cudaStream_t s) {
+                          const bool *raw_head, void *o, float *lse, float *lse_dil, char *ws, unsigned *tickets,
+                          int *n_launch, cudaStream_t s) {
     struct Key { int D; int raw; };
     int done = 0;
     bool taken[kMaxHeads] = {false};
@@ -238,6 +244,8 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, bool w
         P.scale_log2 = scale_of(c) * 1.4426950408889634f;
         P.o = o; P.lse_user = lse; P.lse_dil = lse_dil;
         P.hdr = reinterpret_cast<WsHeader *>(ws);
+        if (*n_launch >= kAttnTickets) return fail(RAT_ERR_UNSUPPORTED, "more than %d attention launches", kAttnTickets);
+        P.ticket = tickets + (*n_launch)++;
         for (int h = 0; h < c->H; ++h) P.win[h] = c->win[h];
         // collect up to kTcMaxClasses classes
         Key keys[kTcMaxClasses];
@@ -279,9 +287,9 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, bool w
             pref += (long long)c->B * C.nheads * C.D * C.mtiles;
             const void *kb = keys[ci].raw ? kraw : kt;
             const void *vb = keys[ci].raw ? vraw : vt;
-            if (!encode_map_5d(&P.tq[oi], q, c->B, c->T, c->H, c->d, C.D) ||
-                !encode_map_5d(&P.tk[oi], kb, c->B, c->T, c->H, c->d, C.D) ||
-                !encode_map_5d(&P.tv[oi], vb, c->B, c->T, c->H, c->d, C.D))
+            if (!encode_map_5d(&P.tq[oi], q, c->B, c->T, c->H, c->d, C.D, kTcRowsQ) ||
+                !encode_map_5d(&P.tk[oi], kb, c->B, c->T, c->H, c->d, C.D, kTcRowsKV) ||
+                !encode_map_5d(&P.tv[oi], vb, c->B, c->T, c->H, c->d, C.D, kTcRowsKV))
                 return fail(RAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (dilation %d)", C.D);
         }
         P.prefix[ncls] = pref;
@@ -309,12 +317,18 @@ rat_status run_attn(const rat_cfg *c, const Layout &L, const void *q, const void
     }
     float *lse_dil = reinterpret_cast<float *>(ws + L.lse_dil);
     if (n_tc > 0) {
+        unsigned *tickets = reinterpret_cast<unsigned *>(ws + L.att_ticket);
+        int n_launch = 0;
+        cudaError_t e = cudaMemsetAsync(tickets, 0, kAttnTickets * sizeof(unsigned), s);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(attention tickets)");
         // The sort in launch_tc_part orders classes by dilation; with T fixed,
         // a smaller dilation means longer subsequences, i.e. more query tiles.
-        rat_status st = launch_tc_part(c, tc_all, n_tc, false, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws, s);
+        rat_status st = launch_tc_part(c, tc_all, n_tc, false, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws,
+                                       tickets, &n_launch, s);
         if (st != RAT_OK) return st;
         if (n_win > 0) {
-            st = launch_tc_part(c, tc_win, n_win, true, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws, s);
+            st = launch_tc_part(c, tc_win, n_win, true, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws,
+                                tickets, &n_launch, s);
             if (st != RAT_OK) return st;
         }
     }

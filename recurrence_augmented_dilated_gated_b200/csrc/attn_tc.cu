@@ -34,6 +34,7 @@
 // copies and MMAs in flight, frees its TMEM and exits.
 #include <cuda.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "attn_tc.cuh"
@@ -43,7 +44,7 @@ namespace rat {
 
 namespace {
 
-constexpr int BM = 128, BN = 128;
+constexpr int BM = kTcRowsQ, BN = kTcRowsKV;   // query rows per sub-tile, keys per K/V tile (128 each)
 constexpr int kSub = 2;                        // query sub-tiles per CTA
 constexpr int kThreads = 64 + kSub * 128;      // TMA warp, MMA warp, two softmax warpgroups
 constexpr uint32_t kTmemCols = 512;
@@ -301,6 +302,16 @@ struct Smem {
 };
 
 // ------------------------------------------------------------------ kernel
+// Persistent: one CTA per SM takes work units from a ticket counter in the
+// order of the unit list (so the blocks of one subsequence still run close
+// together and share its K/V in L2).  The roles run ahead across units: the
+// producer loads the next unit's Q as soon as the last QK of the current one
+// has read its Q, and K/V tiles flow through the same rings; the MMA issuer
+// starts the next unit's first QK while the softmax warps write the current
+// unit's output.  O_i needs no barrier of its own: the next PV into O_i waits
+// for that warpgroup's next P, which it writes only after its epilogue has
+// read O_i (ordered by the tcgen05 fences around bar_pfull).  Unit tickets
+// reach the other roles through a 2-slot ring in shared memory.
 template <int HD>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
     using L = Smem<HD>;
@@ -309,28 +320,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
 
-    __shared__ uint64_t bar_q, bar_kfull[2], bar_kempty[2], bar_vfull[2], bar_vempty[2];
+    __shared__ uint64_t bar_q, bar_qempty, bar_kfull[2], bar_kempty[2], bar_vfull[2], bar_vempty[2];
     __shared__ uint64_t bar_sfull[kSub], bar_pfull[kSub], bar_pvdone[kSub], bar_drain;
+    __shared__ uint64_t bar_ufull[2], bar_uempty[2];
+    __shared__ long long s_unit[2];
     __shared__ uint32_t s_tmem;
     __shared__ volatile int s_abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // a bounded wait of an earlier CTA on this workspace gave up: skip the
-    // remaining work units (the error is already recorded for rat_check_status)
+    // a bounded wait of an earlier launch on this workspace gave up: skip the
+    // work (the error is already recorded for rat_check_status)
     if (*reinterpret_cast<volatile int *>(&p.hdr->status) == RAT_ERR_TIMEOUT) return;
-    const Unit u = decode_unit(p, blockIdx.x);
-    const TcClass &C = p.cls[u.cls];
-    const Plan pl = make_plan(p, u, C.n);
-    const int ntiles = pl.jhi - pl.jlo + 1;
 
     if (threadIdx.x == 0) {
         s_abort = 0;
         mbar_init(&bar_q, 1);
+        mbar_init(&bar_qempty, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bar_kfull[i], 1);
             mbar_init(&bar_kempty[i], 1);
             mbar_init(&bar_vfull[i], 1);
             mbar_init(&bar_vempty[i], 1);
+            mbar_init(&bar_ufull[i], 1);
+            mbar_init(&bar_uempty[i], 1 + 4 * kSub);  // MMA issuer + every softmax warp
         }
         for (int i = 0; i < kSub; ++i) {
             mbar_init(&bar_sfull[i], 1);
@@ -352,59 +364,70 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            const CUtensorMap *mq = &p.tq[u.cls];
-            const CUtensorMap *mk = &p.tk[u.cls];
-            const CUtensorMap *mv = &p.tv[u.cls];
-            const int nq = pl.valid[1] ? 2 : 1;
-            mbar_expect_tx(&bar_q, nq * L::kTile);
-            for (int i = 0; i < nq; ++i)
-                for (int cb = 0; cb < NCB; ++cb)
-                    tma_load_5d(sbase + L::kQ + i * L::kTile + cb * BM * 128, mq, &bar_q, cb * 64, u.h, u.r,
-                                2 * BM * u.m + BM * i, u.b);
+            int nk = 0, nv = 0, nqu = 0;  // K tiles, V tiles, Q units issued so far
             bool ok = true;
-            int t = 0;
-            for (; t < ntiles && ok; ++t) {
-                const int st = t & 1;
-                const uint32_t ph = (uint32_t)(t >> 1) & 1u;
-                const int krow = BN * (pl.jlo + t);
-                if (t >= 2) ok = mbar_wait(&bar_kempty[st], ph ^ 1u, &s_abort);
-                if (!ok) break;
-                mbar_expect_tx(&bar_kfull[st], L::kTile);
-                for (int cb = 0; cb < NCB; ++cb)
-                    tma_load_5d(sbase + L::kK + st * L::kTile + cb * BN * 128, mk, &bar_kfull[st], cb * 64, u.h,
-                                u.r, krow, u.b);
-                if (t >= 2) ok = mbar_wait(&bar_vempty[st], ph ^ 1u, &s_abort);
-                if (!ok) {
-                    volatile int never = 0;
-                    mbar_wait(&bar_kfull[st], ph, &never);  // K of this tile is in flight
+            for (int it = 0; ok; ++it) {
+                const int slot = it & 1;
+                if (it >= 2 && !(ok = mbar_wait(&bar_uempty[slot], (uint32_t)((it >> 1) - 1) & 1u, &s_abort)))
                     break;
+                const long long un = (long long)atomicAdd(p.ticket, 1u);
+                s_unit[slot] = un;
+                mbar_arrive(&bar_ufull[slot]);
+                if (un >= p.total_units) break;
+                const Unit u = decode_unit(p, un);
+                const Plan pl = make_plan(p, u, p.cls[u.cls].n);
+                const int ntiles = pl.jhi - pl.jlo + 1;
+                const CUtensorMap *mq = &p.tq[u.cls];
+                const CUtensorMap *mk = &p.tk[u.cls];
+                const CUtensorMap *mv = &p.tv[u.cls];
+                // Q of the previous unit has been read by its last QK
+                if (it >= 1 && !(ok = mbar_wait(&bar_qempty, (uint32_t)(it - 1) & 1u, &s_abort))) break;
+                const int nq = pl.valid[1] ? 2 : 1;
+                mbar_expect_tx(&bar_q, nq * L::kTile);
+                for (int i = 0; i < nq; ++i)
+                    for (int cb = 0; cb < NCB; ++cb)
+                        tma_load_5d(sbase + L::kQ + i * L::kTile + cb * BM * 128, mq, &bar_q, cb * 64, u.h, u.r,
+                                    2 * BM * u.m + BM * i, u.b);
+                ++nqu;
+                for (int t = 0; t < ntiles; ++t) {
+                    const int krow = BN * (pl.jlo + t);
+                    const int st = nk & 1;
+                    const uint32_t ph = (uint32_t)(nk >> 1) & 1u;
+                    if (nk >= 2 && !(ok = mbar_wait(&bar_kempty[st], ph ^ 1u, &s_abort))) break;
+                    mbar_expect_tx(&bar_kfull[st], L::kTile);
+                    for (int cb = 0; cb < NCB; ++cb)
+                        tma_load_5d(sbase + L::kK + st * L::kTile + cb * BN * 128, mk, &bar_kfull[st], cb * 64,
+                                    u.h, u.r, krow, u.b);
+                    ++nk;
+                    if (nv >= 2 && !(ok = mbar_wait(&bar_vempty[st], ph ^ 1u, &s_abort))) break;
+                    mbar_expect_tx(&bar_vfull[st], L::kTile);
+                    for (int cb = 0; cb < NCB; ++cb)
+                        tma_load_5d(sbase + L::kV + st * L::kTile + cb * BN * 128, mv, &bar_vfull[st], cb * 64,
+                                    u.h, u.r, krow, u.b);
+                    ++nv;
                 }
-                mbar_expect_tx(&bar_vfull[st], L::kTile);
-                for (int cb = 0; cb < NCB; ++cb)
-                    tma_load_5d(sbase + L::kV + st * L::kTile + cb * BN * 128, mv, &bar_vfull[st], cb * 64, u.h,
-                                u.r, krow, u.b);
             }
             if (!ok) {
                 s_abort = 1;
                 report_error(p.hdr, RAT_ERR_TIMEOUT, (int)blockIdx.x);
-                volatile int never = 0;
-                for (int tt = max(0, t - 2); tt < t; ++tt) {  // the last copies of each ring
-                    const uint32_t ph = (uint32_t)(tt >> 1) & 1u;
-                    mbar_wait(&bar_kfull[tt & 1], ph, &never);
-                    mbar_wait(&bar_vfull[tt & 1], ph, &never);
-                }
-                mbar_wait(&bar_q, 0, &never);
             }
+            // Before the CTA exits, every copy it issued must have landed (the
+            // consumers have waited for all of them unless a role gave up): the
+            // last one issued into each ring slot and the last Q; bounded.
+            volatile int never = 0;
+            for (int n = max(0, nk - 2); n < nk; ++n) mbar_wait(&bar_kfull[n & 1], (uint32_t)(n >> 1) & 1u, &never);
+            for (int n = max(0, nv - 2); n < nv; ++n) mbar_wait(&bar_vfull[n & 1], (uint32_t)(n >> 1) & 1u, &never);
+            if (nqu > 0) mbar_wait(&bar_q, (uint32_t)(nqu - 1) & 1u, &never);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t id_qk = idesc_bf16(BM, BN, 0);
             const uint32_t id_pv = idesc_bf16(BM, HD, 1);
-            int n_pv[kSub] = {0, 0};
-            auto qk = [&](int i, int t) {  // S_i = Q_i K_t
+            int n_pv[kSub] = {0, 0};   // PV MMAs issued per sub-tile (pfull phases)
+            auto qk = [&](int i, int n) {  // S_i = Q_i K(ring tile n)
                 const uint32_t tq = sbase + L::kQ + i * L::kTile;
-                const uint32_t tk = sbase + L::kK + (t & 1) * L::kTile;
+                const uint32_t tk = sbase + L::kK + (n & 1) * L::kTile;
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
                     const uint64_t a = sdesc(tq + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
@@ -413,69 +436,87 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 }
                 umma_commit(&bar_sfull[i]);
             };
-            auto pv = [&](int i, int t) -> bool {  // O_i += P_i V_t, P_i read from TMEM over S_i
+            // O_i (+)= P_i V(ring tile n), P_i read from TMEM over S_i
+            auto pv = [&](int i, int n, bool acc) -> bool {
                 if (!mbar_wait(&bar_pfull[i], (uint32_t)n_pv[i] & 1u, &s_abort)) return false;
                 tc_fence_after();
-                const uint32_t tv = sbase + L::kV + (t & 1) * L::kTile;
+                const uint32_t tv = sbase + L::kV + (n & 1) * L::kTile;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     const uint64_t b = sdesc(tv + kk * 16 * 128, BN * 128, 1024);
-                    umma_ts(tmem + 256 + HD * i, tmem + BM * i + 8 * kk, b, id_pv, (n_pv[i] > 0 || kk > 0) ? 1u : 0u);
+                    umma_ts(tmem + 256 + HD * i, tmem + BM * i + 8 * kk, b, id_pv, (acc || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(&bar_pvdone[i]);
                 ++n_pv[i];
                 return true;
             };
-            bool ok = mbar_wait(&bar_q, 0, &s_abort);
-            if (ok) ok = mbar_wait(&bar_kfull[0], 0, &s_abort);
-            if (ok) {
+            int kv = 0;  // K/V ring tiles consumed before this unit
+            bool ok = true;
+            for (int it = 0; ok; ++it) {
+                const int slot = it & 1;
+                if (!(ok = mbar_wait(&bar_ufull[slot], (uint32_t)(it >> 1) & 1u, &s_abort))) break;
+                const long long un = s_unit[slot];
+                mbar_arrive(&bar_uempty[slot]);
+                if (un >= p.total_units) break;
+                const Unit u = decode_unit(p, un);
+                const Plan pl = make_plan(p, u, p.cls[u.cls].n);
+                const int ntiles = pl.jhi - pl.jlo + 1;
+                ok = mbar_wait(&bar_q, (uint32_t)it & 1u, &s_abort);
+                if (ok) ok = mbar_wait(&bar_kfull[kv & 1], (uint32_t)(kv >> 1) & 1u, &s_abort);
+                if (!ok) break;
                 tc_fence_after();
 #pragma unroll
                 for (int i = 0; i < kSub; ++i)
-                    if (takes(pl, i, pl.jlo)) qk(i, 0);
-                umma_commit(&bar_kempty[0]);
-            }
-            for (int t = 0; t < ntiles && ok; ++t) {
-                const int j = pl.jlo + t;
-                bool v_ready = false, k_ready = false;
+                    if (takes(pl, i, pl.jlo)) qk(i, kv);
+                umma_commit(&bar_kempty[kv & 1]);
+                if (ntiles == 1) umma_commit(&bar_qempty);
+                bool started[kSub] = {false, false};  // a PV of this unit has written O_i (accumulate)
+                for (int t = 0; t < ntiles && ok; ++t) {
+                    const int j = pl.jlo + t;
+                    const int cur = kv + t, nxt = cur + 1;
+                    bool v_ready = false, k_ready = false;
 #pragma unroll
-                for (int i = 0; i < kSub; ++i) {
-                    if (!ok) break;
-                    if (takes(pl, i, j)) {
-                        if (!v_ready) {
-                            ok = mbar_wait(&bar_vfull[t & 1], (uint32_t)(t >> 1) & 1u, &s_abort);
-                            if (!ok) break;
-                            v_ready = true;
-                        }
-                        ok = pv(i, t);
+                    for (int i = 0; i < kSub; ++i) {
                         if (!ok) break;
-                    }
-                    if (t + 1 < ntiles && takes(pl, i, j + 1)) {
-                        if (!k_ready) {
-                            ok = mbar_wait(&bar_kfull[(t + 1) & 1], (uint32_t)((t + 1) >> 1) & 1u, &s_abort);
+                        if (takes(pl, i, j)) {
+                            if (!v_ready) {
+                                ok = mbar_wait(&bar_vfull[cur & 1], (uint32_t)(cur >> 1) & 1u, &s_abort);
+                                if (!ok) break;
+                                v_ready = true;
+                            }
+                            ok = pv(i, cur, started[i]);
                             if (!ok) break;
-                            tc_fence_after();
-                            k_ready = true;
+                            started[i] = true;
                         }
-                        qk(i, t + 1);
+                        if (t + 1 < ntiles && takes(pl, i, j + 1)) {
+                            if (!k_ready) {
+                                ok = mbar_wait(&bar_kfull[nxt & 1], (uint32_t)(nxt >> 1) & 1u, &s_abort);
+                                if (!ok) break;
+                                tc_fence_after();
+                                k_ready = true;
+                            }
+                            qk(i, nxt);
+                        }
+                    }
+                    if (!ok) break;
+                    umma_commit(&bar_vempty[cur & 1]);
+                    if (t + 1 < ntiles) {
+                        if (!k_ready) ok = mbar_wait(&bar_kfull[nxt & 1], (uint32_t)(nxt >> 1) & 1u, &s_abort);
+                        umma_commit(&bar_kempty[nxt & 1]);
+                        if (t + 2 == ntiles) umma_commit(&bar_qempty);  // the unit's last QK is issued
                     }
                 }
-                if (!ok) break;
-                umma_commit(&bar_vempty[t & 1]);
-                if (t + 1 < ntiles) {
-                    if (!k_ready) ok = mbar_wait(&bar_kfull[(t + 1) & 1], (uint32_t)((t + 1) >> 1) & 1u, &s_abort);
-                    umma_commit(&bar_kempty[(t + 1) & 1]);
-                }
+                kv += ntiles;
             }
             if (!ok) {
                 s_abort = 1;
                 report_error(p.hdr, RAT_ERR_TIMEOUT, (int)blockIdx.x);
-                // every MMA already issued must finish before TMEM is released:
-                // a commit arrives once all prior tcgen05 operations are done
-                umma_commit(&bar_drain);
-                volatile int never = 0;
-                mbar_wait(&bar_drain, 0, &never);
             }
+            // every MMA already issued must finish before TMEM is released
+            // (a commit arrives once all prior tcgen05 operations are done)
+            umma_commit(&bar_drain);
+            volatile int never = 0;
+            mbar_wait(&bar_drain, 0, &never);
         }
     } else {
         // ------------------------------------------------ softmax warpgroups
@@ -485,85 +526,107 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
         const uint32_t t_s = tmem + lane_base + BM * sub;         // S (and P) of this row
         const uint32_t t_o = tmem + lane_base + 256 + HD * sub;   // O of this row
-        const int qmin = 2 * BM * u.m + BM * sub;                 // first row of the sub-tile
-        const int qi = qmin + row;                                // subsequence row / position
-        const int W = p.win[u.h];
-        const int lo_s = sub ? pl.lo[1] : pl.lo[0];
-        const int nt = (sub ? pl.valid[1] : pl.valid[0]) ? (sub ? pl.hi[1] : pl.hi[0]) - lo_s + 1 : 0;
-        float m_run = -INFINITY, l_run = 0.f;
+        int n_s = 0, n_pv = 0;   // S tiles and PV MMAs of this sub-tile consumed so far
         bool ok = true;
-        for (int c = 0; c < nt; ++c) {
-            const int j = lo_s + c;
-            ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfull[sub], (uint32_t)c & 1u, &s_abort));
+        for (int it = 0; ok; ++it) {
+            const int slot = it & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar_ufull[slot], (uint32_t)(it >> 1) & 1u, &s_abort));
             if (!ok) break;
-            tc_fence_after();
-            // mask: causal on subsequence rows (dilated part); keys in (qi - W, qi] (window part)
-            const int ks = BN * j;
-            const bool full = !p.window_mode ? (ks + BN - 1 <= qmin)
-                                             : (ks + BN - 1 <= qmin && ks > qmin + BM - 1 - W);
-            // row limits in keys from the tile's first column
-            const int lim = qi - ks;            // key k valid iff k <= lim (both parts)
-            const int lo = qi - W - ks;         // window part: and k > lo
-            const int mode = full ? 0 : (p.window_mode ? 2 : 1);
-            const float mraw = mode == 0 ? row_max<0>(t_s, lo, lim)
-                             : mode == 1 ? row_max<1>(t_s, lo, lim) : row_max<2>(t_s, lo, lim);
-            const float mx = mraw * p.scale_log2;   // scale > 0 commutes with max
-            // running max with lazy rescale: keep the stale max unless the new
-            // one exceeds it by more than 8 (P stays <= 2^8)
-            float m_new = m_run;
-            bool rescale = false;
-            if (mx > m_run + 8.f || m_run == -INFINITY) {
-                m_new = mx;
-                rescale = (c > 0) && (m_run != -INFINITY);
-            }
-            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-            const float alpha = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_use);
-            // O and the TMEM holding the previous P are free once the previous PV completed
-            if (c > 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bar_pvdone[sub], (uint32_t)(c - 1) & 1u, &s_abort));
+            const long long un = s_unit[slot];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_uempty[slot]);
+            if (un >= p.total_units) break;
+            const Unit u = decode_unit(p, un);
+            const TcClass &C = p.cls[u.cls];
+            const Plan pl = make_plan(p, u, C.n);
+            const int qmin = 2 * BM * u.m + BM * sub;                 // first row of the sub-tile
+            const int qi = qmin + row;                                // subsequence row / position
+            const int W = p.win[u.h];
+            const int lo_s = sub ? pl.lo[1] : pl.lo[0];
+            const int nt = (sub ? pl.valid[1] : pl.valid[0]) ? (sub ? pl.hi[1] : pl.hi[0]) - lo_s + 1 : 0;
+            float m_run = -INFINITY, l_run = 0.f;
+            for (int c = 0; c < nt; ++c) {
+                const int j = lo_s + c;
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar_sfull[sub], (uint32_t)n_s & 1u, &s_abort));
                 if (!ok) break;
+                ++n_s;
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, rescale)) {
-                    const float f = rescale ? alpha : 1.f;
+                // mask: causal on subsequence rows (dilated part); keys in (qi - W, qi] (window part)
+                const int ks = BN * j;
+                const bool full = !p.window_mode ? (ks + BN - 1 <= qmin)
+                                                 : (ks + BN - 1 <= qmin && ks > qmin + BM - 1 - W);
+                // row limits in keys from the tile's first column
+                const int lim = qi - ks;            // key k valid iff k <= lim (both parts)
+                const int lo = qi - W - ks;         // window part: and k > lo
+                const int mode = full ? 0 : (p.window_mode ? 2 : 1);
+                const float mraw = mode == 0 ? row_max<0>(t_s, lo, lim)
+                                 : mode == 1 ? row_max<1>(t_s, lo, lim) : row_max<2>(t_s, lo, lim);
+                const float mx = mraw * p.scale_log2;   // scale > 0 commutes with max
+                // running max with lazy rescale: keep the stale max unless the new
+                // one exceeds it by more than 8 (P stays <= 2^8)
+                float m_new = m_run;
+                bool rescale = false;
+                if (mx > m_run + 8.f || m_run == -INFINITY) {
+                    m_new = mx;
+                    rescale = (c > 0) && (m_run != -INFINITY);
+                }
+                const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+                const float alpha = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_use);
+                // O and the TMEM holding the previous P are free once the previous PV completed
+                if (c > 0) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(&bar_pvdone[sub], (uint32_t)n_pv & 1u, &s_abort));
+                    if (!ok) break;
+                    ++n_pv;
+                    tc_fence_after();
+                    if (__any_sync(0xffffffffu, rescale)) {
+                        const float f = rescale ? alpha : 1.f;
 #pragma unroll
-                    for (int cc = 0; cc < HD / 32; ++cc) {
-                        uint32_t o[32];
-                        tmem_ld32(t_o + cc * 32, o);
+                        for (int cc = 0; cc < HD / 32; ++cc) {
+                            uint32_t o[32];
+                            tmem_ld32(t_o + cc * 32, o);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-                        tmem_st32(t_o + cc * 32, o);
+                            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+                            tmem_st32(t_o + cc * 32, o);
+                        }
                     }
                 }
+                const float rs = mode == 0 ? row_exp_pack<0>(t_s, lo, lim, p.scale_log2, m_use)
+                               : mode == 1 ? row_exp_pack<1>(t_s, lo, lim, p.scale_log2, m_use)
+                                           : row_exp_pack<2>(t_s, lo, lim, p.scale_log2, m_use);
+                l_run = l_run * alpha + rs;
+                m_run = m_new;
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_pfull[sub]);
             }
-            const float rs = mode == 0 ? row_exp_pack<0>(t_s, lo, lim, p.scale_log2, m_use)
-                           : mode == 1 ? row_exp_pack<1>(t_s, lo, lim, p.scale_log2, m_use)
-                                       : row_exp_pack<2>(t_s, lo, lim, p.scale_log2, m_use);
-            l_run = l_run * alpha + rs;
-            m_run = m_new;
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_pfull[sub]);
-        }
-        if (nt > 0) {
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar_pvdone[sub], (uint32_t)(nt - 1) & 1u, &s_abort));
-            if (!ok) {
-                s_abort = 1;
-                report_error(p.hdr, RAT_ERR_TIMEOUT, (int)blockIdx.x);
-            } else {
-                tc_fence_after();
-                // ---- epilogue: o = O / l, lse = ln(2) * (m + log2 l)
+            if (!ok) break;
+            if (nt > 0) {
                 const bool valid_row = qi < C.n;
                 const long long t = p.window_mode ? (long long)qi : (long long)u.r + (long long)C.D * qi;
                 const size_t orow = (((size_t)u.b * p.T + (size_t)t) * p.H + u.h) * HD;
                 const size_t lrow = ((size_t)u.b * p.H + u.h) * p.T + (size_t)t;
-                const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-                float lse2 = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;  // log2 domain
                 __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.o);
                 const bool merge = p.window_mode != 0;
+                // The window launch merges with the dilated part's row (o, lse),
+                // written by the previous launch: fetch it while the last PV runs.
+                uint4 prev[HD / 8];
+                float ld2 = 0.f;
+                if (merge && valid_row) {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(o + orow);
+#pragma unroll
+                    for (int q = 0; q < HD / 8; ++q) prev[q] = src[q];
+                    ld2 = p.lse_dil[lrow] * 1.4426950408889634f;
+                }
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar_pvdone[sub], (uint32_t)n_pv & 1u, &s_abort));
+                if (!ok) break;
+                ++n_pv;
+                tc_fence_after();
+                // ---- epilogue: o = O / l, lse = ln(2) * (m + log2 l)
+                const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+                float lse2 = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;  // log2 domain
                 float w_self = 1.f, w_dil = 0.f;
                 if (merge && valid_row) {
                     // merge with the dilated part: weights e^(lse_i - max) / sum
-                    const float ld2 = p.lse_dil[lrow] * 1.4426950408889634f;
                     const float mm = fmaxf(ld2, lse2);
                     const float e1 = ex2(ld2 - mm), e2 = ex2(lse2 - mm);
                     w_dil = e1 / (e1 + e2);
@@ -587,8 +650,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 #pragma unroll
                             for (int i = 0; i < 8; ++i) v8[i] = ov[8 * q + i] * inv_l * w_self;
                             if (merge) {
-                                const uint4 prev = dst[q];
-                                const uint32_t pw[4] = {prev.x, prev.y, prev.z, prev.w};
+                                const uint4 pq = prev[cc * 4 + q];
+                                const uint32_t pw[4] = {pq.x, pq.y, pq.z, pq.w};
 #pragma unroll
                                 for (int i = 0; i < 4; ++i) {
                                     const float2 f =
@@ -612,6 +675,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     else if (p.lse_user) p.lse_user[lrow] = lse;
                 }
             }
+        }
+        if (!ok) {
+            s_abort = 1;
+            report_error(p.hdr, RAT_ERR_TIMEOUT, (int)blockIdx.x);
         }
     }
 
@@ -648,13 +715,13 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int H, int d, int D) {
+bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int H, int d, int D, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn || D < 1 || T % D != 0) return false;
     const cuuint64_t e = 2;  // bf16
     const cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)D, (cuuint64_t)(T / D), (cuuint64_t)B};
     const cuuint64_t strides[4] = {e * d, e * d * H, e * d * H * D, e * d * H * T};
-    const cuuint32_t box[5] = {64, 1, 1, 128, 1};
+    const cuuint32_t box[5] = {64, 1, 1, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -685,15 +752,20 @@ size_t attn_tc_smem_bytes(int hd) {
 cudaError_t launch_attn_tc(const TcParams &p, int hd, cudaStream_t s) {
     if (p.total_units == 0) return cudaSuccess;
     const size_t smem = attn_tc_smem_bytes(hd);
-    cudaError_t e;
+    int dev = 0, nsm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    // persistent: one CTA per SM (the shared memory and TMEM of one CTA fill an SM)
+    const unsigned grid = (unsigned)std::min<long long>(p.total_units, (long long)nsm);
     if (hd == 128) {
         e = cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        attn_tc_kernel<128><<<(unsigned)p.total_units, kThreads, smem, s>>>(p);
+        attn_tc_kernel<128><<<grid, kThreads, smem, s>>>(p);
     } else {
         e = cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        attn_tc_kernel<64><<<(unsigned)p.total_units, kThreads, smem, s>>>(p);
+        attn_tc_kernel<64><<<grid, kThreads, smem, s>>>(p);
     }
     count_launches(1);
     return cudaGetLastError();

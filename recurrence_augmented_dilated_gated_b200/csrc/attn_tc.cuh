@@ -8,6 +8,8 @@
 namespace rat {
 
 constexpr int kTcMaxClasses = 8;
+constexpr int kTcRowsQ = 128;   // query rows per sub-tile (Q box height)
+constexpr int kTcRowsKV = 128;  // keys per K/V tile (K/V box height)
 
 // Heads of one launch that share a dilation and a K/V source.
 struct TcClass {
@@ -20,8 +22,8 @@ struct TcClass {
 };
 
 struct TcParams {
-    CUtensorMap tq[kTcMaxClasses];  // 5-D maps (d, H, D, T/D, B), box (64, 1, 1, 128, 1), 128B swizzle
-    CUtensorMap tk[kTcMaxClasses];
+    CUtensorMap tq[kTcMaxClasses];  // 5-D maps (d, H, D, T/D, B), box (64, 1, 1, rows, 1), 128B swizzle:
+    CUtensorMap tk[kTcMaxClasses];  // Q boxes of kTcRowsQ rows, K and V boxes of kTcRowsKV rows
     CUtensorMap tv[kTcMaxClasses];
     TcClass cls[kTcMaxClasses];     // sorted by mtiles, descending
     long long prefix[kTcMaxClasses + 1];  // prefix[c] = work units of the classes before c
@@ -33,6 +35,7 @@ struct TcParams {
     float *lse_user;                // [B,H,T] or null
     float *lse_dil;                 // [B,H,T] scratch: lse of the dilated part of windowed heads
     WsHeader *hdr;
+    unsigned int *ticket;           // work-unit counter of this launch (zero at launch)
     long long total_units;
     unsigned char heads[kMaxHeads];
     int win[kMaxHeads];
@@ -40,7 +43,8 @@ struct TcParams {
 
 size_t attn_tc_smem_bytes(int hd);
 cudaError_t launch_attn_tc(const TcParams &p, int hd, cudaStream_t s);
-// 5-D TMA map of a [B,T,H,d] bf16 tensor viewed as (d, H, D, T/D, B); requires T % D == 0.
-bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int H, int d, int D);
+// 5-D TMA map of a [B,T,H,d] bf16 tensor viewed as (d, H, D, T/D, B), box
+// (64, 1, 1, box_rows, 1); requires T % D == 0.
+bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int H, int d, int D, int box_rows);
 
 }  // namespace rat

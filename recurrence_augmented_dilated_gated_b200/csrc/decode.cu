@@ -29,7 +29,9 @@ namespace {
 constexpr int kCompute = 128;        // threads that score rows (4 warps)
 constexpr int kThreads = kCompute + 32;  // plus one producer warp
 constexpr int kBatch = 4;            // rows scored together per row group
-constexpr int kRowsTarget = 512;     // slab rows per work item (upper bound)
+constexpr int kRowsMax = 2048;       // slab rows per work item, at most ...
+constexpr int kRowsMin = 256;        // ... and at least, when the batch alone cannot fill the GPU
+constexpr int kItemsWanted = 4 * 148;  // work items per step that keep every SM busy
 constexpr int kStages = 4;           // shared-memory ring of K/V row blocks
 constexpr long long kWaitNs = 2000000000LL;
 
@@ -439,12 +441,24 @@ cudaError_t launch_typed(const DecodeParams &p, unsigned grid, cudaStream_t s) {
 }  // namespace
 
 size_t decode_plan(const rat_cfg *c, int cap, DecodeParams *p) {
+    // Longer items mean fewer partial results to merge; split further only
+    // while the batch's items would leave SMs idle.
+    int target = kRowsMax;
+    while (target > kRowsMin) {
+        long long n_items = 0;
+        for (int h = 0; h < c->H; ++h) {
+            const long long slab = ((long long)cap + c->dil[h] - 1) / c->dil[h];
+            n_items += slab > 0 ? (slab + target - 1) / target : 1;
+        }
+        if (n_items * c->B >= kItemsWanted) break;
+        target /= 2;
+    }
     int items = 0;
     long long R = 0;
     for (int h = 0; h < c->H; ++h) {
         const int D = c->dil[h];
         const int slab = (cap + D - 1) / D;
-        const int ns = (slab + kRowsTarget - 1) / kRowsTarget;
+        const int ns = (slab + target - 1) / target;
         const int n = ns > 0 ? ns : 1;
         p->dil[h] = D;
         p->win[h] = c->win[h];
