@@ -35,6 +35,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <climits>
 #include <mutex>
 
 #include "attn_tc.cuh"
@@ -232,30 +233,32 @@ __device__ __forceinline__ bool takes(const Plan &pl, int i, int j) {
     return pl.valid[i] && j >= pl.lo[i] && j <= pl.hi[i];
 }
 
-// Softmax passes over one 128-key row of S in TMEM, in two 64-column halves
-// (the register budget of 10 warps per CTA does not hold a whole row).  MODE:
-// 0 = every key valid, 1 = causal (key k valid iff k <= lim), 2 = window
-// (valid iff lo < k <= lim); k counts keys from the tile's first column and
-// the limits are this row's, so each test is one compare per element.
+// Softmax passes over one 128-key row of S in TMEM, in four 32-column chunks
+// in a loop that is not unrolled: the small code keeps both softmax
+// warpgroups' instruction streams in cache, which measured faster than 64-
+// or 128-column bodies unrolled per mask mode.  MODE: 0 = every key valid,
+// 2 = masked, key k valid iff lo < k <= lim (causal: lo below every key).  k
+// counts keys from the tile's first column and the limits are this row's, so
+// each test is at most two compares per element.
 template <int MODE>
 __device__ __forceinline__ bool key_ok(int k, int lo, int lim) {
-    return MODE == 0 ? true : MODE == 1 ? (k <= lim) : (k <= lim && k > lo);
+    return MODE == 0 ? true : (k <= lim && k > lo);
 }
 
 // Max of the valid raw scores of this thread's row.
 template <int MODE>
-__device__ __forceinline__ float row_max(uint32_t t_s, int lo, int lim) {
+__device__ __forceinline__ float row_max_s(uint32_t t_s, int lo, int lim) {
     float mx8[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+        uint32_t sr[32];
+        tmem_ld32(t_s + 32 * q, sr);
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        uint32_t sr[64];
-        tmem_ld64(t_s + 64 * half, sr);
-#pragma unroll
-        for (int k = 0; k < 64; ++k) {
+        for (int k = 0; k < 32; ++k) {
             const float x = __uint_as_float(sr[k]);
-            mx8[k & 7] = key_ok<MODE>(64 * half + k, lo, lim) ? fmaxf(mx8[k & 7], x) : mx8[k & 7];
+            mx8[k & 7] = key_ok<MODE>(32 * q + k, lo, lim) ? fmaxf(mx8[k & 7], x) : mx8[k & 7];
         }
     }
     return fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
@@ -263,31 +266,31 @@ __device__ __forceinline__ float row_max(uint32_t t_s, int lo, int lim) {
 }
 
 // P = 2^(s * c - m) (0 for masked keys), packed to bf16 pairs over the first
-// 64 columns of the row: half h lands on columns [32h, 32h+32), which the max
-// pass and half 0 have already consumed.  Returns the row sum of P.
+// 64 columns of the row: chunk q lands on columns [16q, 16q+16), which this
+// and the earlier chunks have already consumed.  Returns the row sum of P.
 template <int MODE>
-__device__ __forceinline__ float row_exp_pack(uint32_t t_s, int lo, int lim, float c, float m) {
+__device__ __forceinline__ float row_exp_s(uint32_t t_s, int lo, int lim, float c, float m) {
     float rs8[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) rs8[k] = 0.f;
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+        uint32_t sr[32];
+        tmem_ld32(t_s + 32 * q, sr);
+        uint32_t pk[16];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        uint32_t sr[64];
-        tmem_ld64(t_s + 64 * half, sr);
-        uint32_t pk[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
+        for (int k = 0; k < 16; ++k) {
             float e[2];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int kk = 2 * k + q;
+            for (int h = 0; h < 2; ++h) {
+                const int kk = 2 * k + h;
                 const float v = ex2(fmaf(__uint_as_float(sr[kk]), c, -m));
-                e[q] = key_ok<MODE>(64 * half + kk, lo, lim) ? v : 0.f;
-                rs8[kk & 7] += e[q];
+                e[h] = key_ok<MODE>(32 * q + kk, lo, lim) ? v : 0.f;
+                rs8[kk & 7] += e[h];
             }
             pk[k] = pack_bf16(e[0], e[1]);
         }
-        tmem_st32(t_s + 32 * half, pk);
+        tmem_st16(t_s + 16 * q, pk);
     }
     return ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
 }
@@ -557,10 +560,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                                                  : (ks + BN - 1 <= qmin && ks > qmin + BM - 1 - W);
                 // row limits in keys from the tile's first column
                 const int lim = qi - ks;            // key k valid iff k <= lim (both parts)
-                const int lo = qi - W - ks;         // window part: and k > lo
-                const int mode = full ? 0 : (p.window_mode ? 2 : 1);
-                const float mraw = mode == 0 ? row_max<0>(t_s, lo, lim)
-                                 : mode == 1 ? row_max<1>(t_s, lo, lim) : row_max<2>(t_s, lo, lim);
+                // window part: and k > lo (no lower limit in the dilated part)
+                const int lo = p.window_mode ? qi - W - ks : INT_MIN / 2;
+                const int mode = full ? 0 : 2;
+                const float mraw = mode == 0 ? row_max_s<0>(t_s, lo, lim) : row_max_s<2>(t_s, lo, lim);
                 const float mx = mraw * p.scale_log2;   // scale > 0 commutes with max
                 // running max with lazy rescale: keep the stale max unless the new
                 // one exceeds it by more than 8 (P stays <= 2^8)
@@ -590,9 +593,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                         }
                     }
                 }
-                const float rs = mode == 0 ? row_exp_pack<0>(t_s, lo, lim, p.scale_log2, m_use)
-                               : mode == 1 ? row_exp_pack<1>(t_s, lo, lim, p.scale_log2, m_use)
-                                           : row_exp_pack<2>(t_s, lo, lim, p.scale_log2, m_use);
+                const float rs = mode == 0 ? row_exp_s<0>(t_s, lo, lim, p.scale_log2, m_use)
+                                           : row_exp_s<2>(t_s, lo, lim, p.scale_log2, m_use);
                 l_run = l_run * alpha + rs;
                 m_run = m_new;
                 tc_fence_before();
