@@ -245,24 +245,53 @@ __device__ __forceinline__ bool key_ok(int k, int lo, int lim) {
     return MODE == 0 ? true : (k <= lim && k > lo);
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: one issue for two elements).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// max of three (sm_100 three-input max)
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // Max of the valid raw scores of this thread's row.
 template <int MODE>
 __device__ __forceinline__ float row_max_s(uint32_t t_s, int lo, int lim) {
-    float mx8[8];
+    float mx4[4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
+    for (int k = 0; k < 4; ++k) mx4[k] = -INFINITY;
 #pragma unroll 1
     for (int q = 0; q < 4; ++q) {
         uint32_t sr[32];
         tmem_ld32(t_s + 32 * q, sr);
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            const float x = __uint_as_float(sr[k]);
-            mx8[k & 7] = key_ok<MODE>(32 * q + k, lo, lim) ? fmaxf(mx8[k & 7], x) : mx8[k & 7];
+        for (int k = 0; k < 16; ++k) {
+            float a = __uint_as_float(sr[2 * k]), b = __uint_as_float(sr[2 * k + 1]);
+            if (MODE != 0) {
+                a = key_ok<MODE>(32 * q + 2 * k, lo, lim) ? a : -INFINITY;
+                b = key_ok<MODE>(32 * q + 2 * k + 1, lo, lim) ? b : -INFINITY;
+            }
+            mx4[k & 3] = max3(mx4[k & 3], a, b);
         }
     }
-    return fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+    return max3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
 }
 
 // P = 2^(s * c - m) (0 for masked keys), packed to bf16 pairs over the first
@@ -270,9 +299,10 @@ __device__ __forceinline__ float row_max_s(uint32_t t_s, int lo, int lim) {
 // and the earlier chunks have already consumed.  Returns the row sum of P.
 template <int MODE>
 __device__ __forceinline__ float row_exp_s(uint32_t t_s, int lo, int lim, float c, float m) {
-    float rs8[8];
+    uint64_t rs2[4];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) rs8[k] = 0.f;
+    for (int k = 0; k < 4; ++k) rs2[k] = f2_pack(0.f, 0.f);
+    const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m, -m);
 #pragma unroll 1
     for (int q = 0; q < 4; ++q) {
         uint32_t sr[32];
@@ -280,19 +310,22 @@ __device__ __forceinline__ float row_exp_s(uint32_t t_s, int lo, int lim, float 
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-            float e[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int kk = 2 * k + h;
-                const float v = ex2(fmaf(__uint_as_float(sr[kk]), c, -m));
-                e[h] = key_ok<MODE>(32 * q + kk, lo, lim) ? v : 0.f;
-                rs8[kk & 7] += e[h];
+            float t0, t1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])), c2, nm2), t0, t1);
+            float e0 = ex2(t0), e1 = ex2(t1);
+            if (MODE != 0) {
+                e0 = key_ok<MODE>(32 * q + 2 * k, lo, lim) ? e0 : 0.f;
+                e1 = key_ok<MODE>(32 * q + 2 * k + 1, lo, lim) ? e1 : 0.f;
             }
-            pk[k] = pack_bf16(e[0], e[1]);
+            rs2[k & 3] = f2_add(rs2[k & 3], f2_pack(e0, e1));
+            pk[k] = pack_bf16(e0, e1);
         }
         tmem_st16(t_s + 16 * q, pk);
     }
-    return ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+    float r[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) f2_unpack(rs2[k], r[2 * k], r[2 * k + 1]);
+    return ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
 }
 
 template <int HD>
