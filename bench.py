@@ -90,9 +90,60 @@ def load_peaks():
     return d
 
 
+class NvmlSampler:
+    """SM clock and throttle reasons read through NVML every ~5 ms on a host
+    thread, with host timestamps, so that even a short timed region holds
+    several samples.  The GPU is found by its PCI bus id (CUDA and NVML
+    number devices differently when CUDA_VISIBLE_DEVICES is set)."""
+
+    PERIOD_S = 0.005
+
+    def __init__(self, cuda_index):
+        import threading
+
+        import pynvml
+
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        pr = torch.cuda.get_device_properties(cuda_index)
+        bus = "%08x:%02x:%02x.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+        self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        bits = {"hw_slowdown": "HwSlowdown", "hw_thermal_slowdown": "HwThermalSlowdown",
+                "sw_thermal_slowdown": "SwThermalSlowdown", "sw_power_cap": "SwPowerCap"}
+        self.bits = {k: getattr(pynvml, "nvmlClocksEventReason" + v, None) or
+                     getattr(pynvml, "nvmlClocksThrottleReason" + v) for k, v in bits.items()}
+        self.reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        self.samples = []
+        self._stop = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            t = time.time()
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = int(self.reasons_fn(self.h))
+            except nv.NVMLError:
+                break
+            self.samples.append((t, sm, self.max_mhz, {k for k, b in self.bits.items() if r & b}))
+            self._stop.wait(self.PERIOD_S)
+
+    def start(self):
+        self.thread.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        self.thread.join(timeout=5)
+
+
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 100 ms, with host
-    timestamps, so the samples inside the timed region can be picked out."""
+    """SM clocks and throttle reasons during the run: NVML every ~5 ms, or
+    nvidia-smi every 100 ms where NVML cannot be used; host timestamps let
+    summary() pick the samples inside the timed region."""
 
     Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -102,8 +153,14 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.f = None
+        self.nvml = None
 
     def start(self):
+        try:
+            self.nvml = NvmlSampler(self.gpu).start()
+            return self
+        except Exception:  # no NVML here: fall back to nvidia-smi
+            self.nvml = None
         try:
             self.f = tempfile.TemporaryFile(mode="w+")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
@@ -114,6 +171,8 @@ class ClockSampler:
         return self
 
     def stop(self):
+        if self.nvml is not None:
+            self.nvml.stop()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -126,12 +185,16 @@ class ClockSampler:
         [t0, t1] (host epoch seconds); all samples when fewer than 2 fall there."""
         import datetime
 
-        if self.proc is None or self.f is None:
-            return None
-        self.f.seek(0)
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         samples = []
-        for line in self.f.read().strip().splitlines():
+        source = "nvidia-smi, 100 ms"
+        if self.nvml is not None:
+            samples, source = list(self.nvml.samples), "nvml, 5 ms"
+        elif self.proc is None or self.f is None:
+            return None
+        else:
+            self.f.seek(0)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in ([] if self.nvml is not None else self.f.read().strip().splitlines()):
             r = [x.strip() for x in line.split(",")]
             if len(r) < 10:
                 continue
@@ -152,7 +215,7 @@ class ClockSampler:
         for x in sel:
             reasons |= x[3]
         return {"sm_mhz": float(np.median([x[1] for x in sel])), "sm_max_mhz": float(max(x[2] for x in sel)),
-                "samples": len(sel), "reasons": sorted(reasons), "window": window}
+                "samples": len(sel), "reasons": sorted(reasons), "window": window, "source": source}
 
 
 def profile_traffic(name, key=None):
