@@ -59,6 +59,66 @@ __device__ __forceinline__ void gate(float g, float &a, float &oma) {
     }
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: one issue for two channels).
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f2_split(uint64_t v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+// a bf16 pair (one 32-bit word, low half first) as an fp32 pair
+__device__ __forceinline__ uint64_t bf2_f2(uint32_t w) {
+    return f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ uint32_t f2_bf2(uint64_t v) {
+    const float2 x = f2_split(v);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(x.x, x.y);
+    return *reinterpret_cast<const uint32_t *>(&b);
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// One gate pair of the bf16 path: a = sigmoid(g), 1 - a = e * a with
+// e = 2^(-g log2 e).  Only g >= -80 needs clamping (e stays finite); large g
+// gives e -> 0, a -> 1, 1 - a -> 0 without it.
+__device__ __forceinline__ void gate2(uint32_t gw, uint64_t &a, uint64_t &oma) {
+    const uint64_t g = bf2_f2(gw);
+    const float2 gs = f2_split(g);
+    const float2 t = f2_split(f2_mul(f2(fmaxf(gs.x, -80.f), fmaxf(gs.y, -80.f)),
+                                     f2(-1.4426950408889634f, -1.4426950408889634f)));
+    const uint64_t e = f2(ex2_approx(t.x), ex2_approx(t.y));
+    const float2 den = f2_split(f2_add(e, f2(1.f, 1.f)));
+    a = f2(rcp_approx(den.x), rcp_approx(den.y));
+    oma = f2_mul(e, a);
+}
+
 // 4 consecutive channels of one token row in shared memory
 template <typename T> struct Smem4;
 template <> struct Smem4<__nv_bfloat16> {
@@ -144,7 +204,42 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
 
     // ---- pass 1: fold the sub-chunk into one affine map per channel
     float A[4] = {1.f, 1.f, 1.f, 1.f}, bk[4] = {0.f, 0.f, 0.f, 0.f}, bv[4] = {0.f, 0.f, 0.f, 0.f};
-    if (loaded) {
+    if (loaded && !kAccurate && rec) {
+        // bf16: channel pairs in f32x2 arithmetic
+        uint64_t A2[2] = {f2(1.f, 1.f), f2(1.f, 1.f)}, bk2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)},
+                 bv2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+#pragma unroll
+        for (int r = r0; r < r0 + kSub; ++r) {
+            if (r < r1) {
+                const uint2 kw = *reinterpret_cast<const uint2 *>(tile_k + r * D + c0);
+                const uint2 vw = *reinterpret_cast<const uint2 *>(tile_v + r * D + c0);
+                const uint2 gw = *reinterpret_cast<const uint2 *>(tile_g + r * D + c0);
+                const uint32_t kq[2] = {kw.x, kw.y}, vq[2] = {vw.x, vw.y}, gq[2] = {gw.x, gw.y};
+                uint32_t oh[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint64_t a, oma;
+                    gate2(gq[h], a, oma);
+                    A2[h] = f2_mul(A2[h], a);
+                    bk2[h] = f2_fma(a, bk2[h], f2_mul(oma, bf2_f2(kq[h])));
+                    bv2[h] = f2_fma(a, bv2[h], f2_mul(oma, bf2_f2(vq[h])));
+                    const float2 o = f2_split(oma);
+                    const __half2 hh = __floats2half2_rn(o.x, o.y);
+                    oh[h] = *reinterpret_cast<const uint32_t *>(&hh);
+                }
+                // keep 1 - a for pass 2 (fp16: relative precision 2^-11)
+                // over the gate logits this thread has just consumed
+                *reinterpret_cast<uint2 *>(tile_g + r * D + c0) = make_uint2(oh[0], oh[1]);
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float2 x = f2_split(A2[h]), y = f2_split(bk2[h]), z = f2_split(bv2[h]);
+            A[2 * h] = x.x; A[2 * h + 1] = x.y;
+            bk[2 * h] = y.x; bk[2 * h + 1] = y.y;
+            bv[2 * h] = z.x; bv[2 * h + 1] = z.y;
+        }
+    } else if (loaded) {
 #pragma unroll
         for (int r = r0; r < r0 + kSub; ++r) {
             if (r < r1) {
@@ -220,7 +315,8 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
                     ag[2 * D + c] = Tv[c];
                 }
             }
-            __threadfence();
+            // the warp barrier orders every lane's stores before lane 0's
+            // release store of the flag, whose release is cumulative
             __syncwarp();
             if (lane == 0) st_release(p.flags + my, 1);
 
@@ -321,7 +417,6 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
                     in[D + c] = iv[c];
                 }
             }
-            __threadfence();
             __syncwarp();
             if (lane == 0) st_release(p.flags + my, 2);
         }
@@ -363,7 +458,39 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
     const int Dh = p.head_dil[h];
     const long long S = ((long long)p.cap + Dh - 1) / Dh;
     const size_t cbase = ((size_t)b * p.H + h) * (size_t)p.cache_R * D + c0;
-    if (loaded) {
+    if (loaded && !kAccurate && rec) {
+        // bf16: a = 1 - (1 - a) from the fp16 cache, channel pairs in f32x2
+        uint64_t sk2[2] = {f2(sk[0], sk[1]), f2(sk[2], sk[3])}, sv2[2] = {f2(sv[0], sv[1]), f2(sv[2], sv[3])};
+#pragma unroll
+        for (int r = r0; r < r0 + kSub; ++r) {
+            if (r < r1) {
+                const uint2 kw = *reinterpret_cast<const uint2 *>(tile_k + r * D + c0);
+                const uint2 vw = *reinterpret_cast<const uint2 *>(tile_v + r * D + c0);
+                const uint2 ow = *reinterpret_cast<const uint2 *>(tile_g + r * D + c0);
+                const uint32_t kq[2] = {kw.x, kw.y}, vq[2] = {vw.x, vw.y}, oq[2] = {ow.x, ow.y};
+                uint32_t wk[2], wv[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float2 of = __half22float2(*reinterpret_cast<const __half2 *>(&oq[h]));
+                    const uint64_t oma = f2(of.x, of.y);
+                    const uint64_t a = f2_fma(oma, f2(-1.f, -1.f), f2(1.f, 1.f));
+                    sk2[h] = f2_fma(a, sk2[h], f2_mul(oma, bf2_f2(kq[h])));
+                    sv2[h] = f2_fma(a, sv2[h], f2_mul(oma, bf2_f2(vq[h])));
+                    wk[h] = f2_bf2(sk2[h]);
+                    wv[h] = f2_bf2(sv2[h]);
+                }
+                *reinterpret_cast<uint2 *>(tile_k + r * D + c0) = make_uint2(wk[0], wk[1]);
+                *reinterpret_cast<uint2 *>(tile_v + r * D + c0) = make_uint2(wv[0], wv[1]);
+                if (ck) {
+                    const long long tt = tc0 + r;
+                    const long long row = (tt % Dh) * S + tt / Dh;
+                    const size_t e = cbase + (size_t)row * D;
+                    *reinterpret_cast<uint2 *>(ck + e) = make_uint2(wk[0], wk[1]);
+                    *reinterpret_cast<uint2 *>(cv + e) = make_uint2(wv[0], wv[1]);
+                }
+            }
+        }
+    } else if (loaded) {
 #pragma unroll
         for (int r = r0; r < r0 + kSub; ++r) {
             if (r < r1) {
