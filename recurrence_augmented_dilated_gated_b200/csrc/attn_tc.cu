@@ -348,7 +348,7 @@ struct Smem {
 // for that warpgroup's next P, which it writes only after its epilogue has
 // read O_i (ordered by the tcgen05 fences around bar_pfull).  Unit tickets
 // reach the other roles through a 2-slot ring in shared memory.
-template <int HD>
+template <int HD, bool kWin>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
     using L = Smem<HD>;
     constexpr int NCB = HD / 64;  // 64-column (128-byte) blocks of a head row
@@ -589,12 +589,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 tc_fence_after();
                 // mask: causal on subsequence rows (dilated part); keys in (qi - W, qi] (window part)
                 const int ks = BN * j;
-                const bool full = !p.window_mode ? (ks + BN - 1 <= qmin)
+                const bool full = !kWin ? (ks + BN - 1 <= qmin)
                                                  : (ks + BN - 1 <= qmin && ks > qmin + BM - 1 - W);
                 // row limits in keys from the tile's first column
                 const int lim = qi - ks;            // key k valid iff k <= lim (both parts)
                 // window part: and k > lo (no lower limit in the dilated part)
-                const int lo = p.window_mode ? qi - W - ks : INT_MIN / 2;
+                const int lo = kWin ? qi - W - ks : INT_MIN / 2;
                 const int mode = full ? 0 : 2;
                 const float mraw = mode == 0 ? row_max_s<0>(t_s, lo, lim) : row_max_s<2>(t_s, lo, lim);
                 const float mx = mraw * p.scale_log2;   // scale > 0 commutes with max
@@ -616,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     tc_fence_after();
                     if (__any_sync(0xffffffffu, rescale)) {
                         const float f = rescale ? alpha : 1.f;
-#pragma unroll
+#pragma unroll 1
                         for (int cc = 0; cc < HD / 32; ++cc) {
                             uint32_t o[32];
                             tmem_ld32(t_o + cc * 32, o);
@@ -637,11 +637,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (!ok) break;
             if (nt > 0) {
                 const bool valid_row = qi < C.n;
-                const long long t = p.window_mode ? (long long)qi : (long long)u.r + (long long)C.D * qi;
+                const long long t = kWin ? (long long)qi : (long long)u.r + (long long)C.D * qi;
                 const size_t orow = (((size_t)u.b * p.T + (size_t)t) * p.H + u.h) * HD;
                 const size_t lrow = ((size_t)u.b * p.H + u.h) * p.T + (size_t)t;
                 __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.o);
-                const bool merge = p.window_mode != 0;
+                constexpr bool merge = kWin;
                 // The window launch merges with the dilated part's row (o, lse),
                 // written by the previous launch: fetch it while the last PV runs.
                 uint4 prev[HD / 8];
@@ -668,39 +668,78 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     w_self = e2 / (e1 + e2);
                     lse2 = mm + __log2f(e1 + e2);
                 }
+                if constexpr (merge) {
 #pragma unroll
-                for (int cc = 0; cc < HD / 32; ++cc) {
-                    float ov[32];
-                    {
-                        uint32_t raw[32];
-                        tmem_ld32(t_o + cc * 32, raw);
+                    for (int cc = 0; cc < HD / 32; ++cc) {
+                        float ov[32];
+                        {
+                            uint32_t raw[32];
+                            tmem_ld32(t_o + cc * 32, raw);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) ov[i] = __uint_as_float(raw[i]);
-                    }
-                    if (valid_row) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(o + orow + cc * 32);
+                            for (int i = 0; i < 32; ++i) ov[i] = __uint_as_float(raw[i]);
+                        }
+                        if (valid_row) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(o + orow + cc * 32);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            float v8[8];
+                            for (int q = 0; q < 4; ++q) {
+                                float v8[8];
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) v8[i] = ov[8 * q + i] * inv_l * w_self;
-                            if (merge) {
-                                const uint4 pq = prev[cc * 4 + q];
-                                const uint32_t pw[4] = {pq.x, pq.y, pq.z, pq.w};
+                                for (int i = 0; i < 8; ++i) v8[i] = ov[8 * q + i] * inv_l * w_self;
+                                if constexpr (merge) {
+                                    const uint4 pq = prev[cc * 4 + q];
+                                    const uint32_t pw[4] = {pq.x, pq.y, pq.z, pq.w};
 #pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    const float2 f =
-                                        __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pw[i]));
-                                    v8[2 * i] += w_dil * f.x;
-                                    v8[2 * i + 1] += w_dil * f.y;
+                                    for (int i = 0; i < 4; ++i) {
+                                        const float2 f =
+                                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pw[i]));
+                                        v8[2 * i] += w_dil * f.x;
+                                        v8[2 * i + 1] += w_dil * f.y;
+                                    }
                                 }
+                                uint4 w;
+                                w.x = pack_bf16(v8[0], v8[1]);
+                                w.y = pack_bf16(v8[2], v8[3]);
+                                w.z = pack_bf16(v8[4], v8[5]);
+                                w.w = pack_bf16(v8[6], v8[7]);
+                                dst[q] = w;
                             }
-                            uint4 w;
-                            w.x = pack_bf16(v8[0], v8[1]);
-                            w.y = pack_bf16(v8[2], v8[3]);
-                            w.z = pack_bf16(v8[4], v8[5]);
-                            w.w = pack_bf16(v8[6], v8[7]);
-                            dst[q] = w;
+                        }
+                    }
+                } else {
+#pragma unroll 1
+                    for (int cc = 0; cc < HD / 32; ++cc) {
+                        float ov[32];
+                        {
+                            uint32_t raw[32];
+                            tmem_ld32(t_o + cc * 32, raw);
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) ov[i] = __uint_as_float(raw[i]);
+                        }
+                        if (valid_row) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(o + orow + cc * 32);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                float v8[8];
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) v8[i] = ov[8 * q + i] * inv_l * w_self;
+                                if constexpr (merge) {
+                                    const uint4 pq = prev[cc * 4 + q];
+                                    const uint32_t pw[4] = {pq.x, pq.y, pq.z, pq.w};
+#pragma unroll
+                                    for (int i = 0; i < 4; ++i) {
+                                        const float2 f =
+                                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&pw[i]));
+                                        v8[2 * i] += w_dil * f.x;
+                                        v8[2 * i + 1] += w_dil * f.y;
+                                    }
+                                }
+                                uint4 w;
+                                w.x = pack_bf16(v8[0], v8[1]);
+                                w.y = pack_bf16(v8[2], v8[3]);
+                                w.z = pack_bf16(v8[4], v8[5]);
+                                w.w = pack_bf16(v8[6], v8[7]);
+                                dst[q] = w;
+                            }
                         }
                     }
                 }
@@ -793,15 +832,17 @@ cudaError_t launch_attn_tc(const TcParams &p, int hd, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM (the shared memory and TMEM of one CTA fill an SM)
     const unsigned grid = (unsigned)std::min<long long>(p.total_units, (long long)nsm);
-    if (hd == 128) {
-        e = cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        attn_tc_kernel<128><<<grid, kThreads, smem, s>>>(p);
-    } else {
-        e = cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        attn_tc_kernel<64><<<grid, kThreads, smem, s>>>(p);
-    }
+    auto go = [&](auto kern) -> cudaError_t {
+        cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (r != cudaSuccess) return r;
+        kern<<<grid, kThreads, smem, s>>>(p);
+        return cudaSuccess;
+    };
+    // the dilated and window launches are separate instantiations, so each
+    // carries only its own epilogue and masks (instruction-cache footprint)
+    if (hd == 128) e = p.window_mode ? go(attn_tc_kernel<128, true>) : go(attn_tc_kernel<128, false>);
+    else e = p.window_mode ? go(attn_tc_kernel<64, true>) : go(attn_tc_kernel<64, false>);
+    if (e != cudaSuccess) return e;
     count_launches(1);
     return cudaGetLastError();
 }
