@@ -344,6 +344,16 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
                     continue;
                 }
                 __syncwarp();  // the flags acquired by every lane order the reads below
+                // the inclusive state found, loaded with the aggregates (one round trip)
+                float inK[4] = {0.f, 0.f, 0.f, 0.f}, inV[4] = {0.f, 0.f, 0.f, 0.f};
+                if (lstar < 32 && owns) {
+                    const float *in = p.incl + (sbase + (base - lstar)) * 2 * D + cc;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        inK[c] = in[c];
+                        inV[c] = in[D + c];
+                    }
+                }
                 // fold aggregates of chunks base, base-1, ..., base-lstar+1
                 if (owns) {
                     int j = 0;
@@ -380,11 +390,10 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
                 }
                 if (lstar < 32) {
                     if (owns) {
-                        const float *in = p.incl + (sbase + (base - lstar)) * 2 * D + cc;
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {
-                            sk[c] = accA[c] * in[c] + acck[c];
-                            sv[c] = accA[c] * in[D + c] + accv[c];
+                            sk[c] = accA[c] * inK[c] + acck[c];
+                            sv[c] = accA[c] * inV[c] + accv[c];
                         }
                     }
                     break;
