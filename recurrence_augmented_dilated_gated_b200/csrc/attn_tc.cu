@@ -472,8 +472,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 }
                 umma_commit(&bar_sfull[i]);
             };
-            // O_i (+)= P_i V(ring tile n), P_i read from TMEM over S_i
-            auto pv = [&](int i, int n, bool acc) -> bool {
+            // O_i (+)= P_i V(ring tile n), P_i read from TMEM over S_i.  Only the
+            // unit's last PV of a sub-tile signals bar_pvdone (for the epilogue):
+            // the commit after QK_i(j+1), issued after PV_i(j), already tells the
+            // softmax that O_i holds tile j when S_i(j+1) is ready.
+            auto pv = [&](int i, int n, bool acc, bool last) -> bool {
                 if (!mbar_wait(&bar_pfull[i], (uint32_t)n_pv[i] & 1u, &s_abort)) return false;
                 tc_fence_after();
                 const uint32_t tv = sbase + L::kV + (n & 1) * L::kTile;
@@ -482,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     const uint64_t b = sdesc(tv + kk * 16 * 128, BN * 128, 1024);
                     umma_ts(tmem + 256 + HD * i, tmem + BM * i + 8 * kk, b, id_pv, (acc || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(&bar_pvdone[i]);
+                if (last) umma_commit(&bar_pvdone[i]);
                 ++n_pv[i];
                 return true;
             };
@@ -520,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                                 if (!ok) break;
                                 v_ready = true;
                             }
-                            ok = pv(i, cur, started[i]);
+                            ok = pv(i, cur, started[i], !takes(pl, i, j + 1));
                             if (!ok) break;
                             started[i] = true;
                         }
@@ -562,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
         const uint32_t t_s = tmem + lane_base + BM * sub;         // S (and P) of this row
         const uint32_t t_o = tmem + lane_base + 256 + HD * sub;   // O of this row
-        int n_s = 0, n_pv = 0;   // S tiles and PV MMAs of this sub-tile consumed so far
+        int n_s = 0, n_pv = 0;   // S tiles, and units whose last PV was awaited, of this sub-tile
         bool ok = true;
         for (int it = 0; ok; ++it) {
             const int slot = it & 1;
@@ -608,12 +611,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 }
                 const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
                 const float alpha = (m_run == -INFINITY) ? 0.f : ex2(m_run - m_use);
-                // O and the TMEM holding the previous P are free once the previous PV completed
+                // S(c) is complete only after every earlier MMA of this CTA, so O
+                // already holds tiles 0..c-1: rescale it before PV(c) adds to it
                 if (c > 0) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(&bar_pvdone[sub], (uint32_t)n_pv & 1u, &s_abort));
-                    if (!ok) break;
-                    ++n_pv;
-                    tc_fence_after();
                     if (__any_sync(0xffffffffu, rescale)) {
                         const float f = rescale ? alpha : 1.f;
 #pragma unroll 1
