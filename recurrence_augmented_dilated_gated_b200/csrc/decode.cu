@@ -257,29 +257,18 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
 #pragma unroll
         for (int i = 0; i < 8; ++i) q[i] *= p.scale_log2;
 
-        if (last) {
-            // step update of the recurrent state and append of the new row
-            for (int c = tid; c < D; c += kCompute) {
-                const size_t e = bh * D + c;
-                const float xk = (float)static_cast<const T *>(p.k)[e];
-                const float xv = (float)static_cast<const T *>(p.v)[e];
-                float a = 0.f, oma = 1.f;
-                if (p.recur[h]) {
-                    const float gl_ = fminf(fmaxf((float)static_cast<const T *>(p.g)[e], -80.f), 80.f);
-                    const float ex = expf(-gl_);
-                    a = 1.f / (1.f + ex);
-                    oma = ex * a;
-                }
-                const float sk = a * p.state[0][e] + oma * xk;
-                const float sv = a * p.state[1][e] + oma * xv;
-                p.state[0][e] = sk;
-                p.state[1][e] = sv;
-                const size_t row = (size_t)r * S + n_old;
-                static_cast<T *>(p.cache[0])[bh * (size_t)p.cache_R * D + row * D + c] = to_t<T>(sk);
-                static_cast<T *>(p.cache[1])[bh * (size_t)p.cache_R * D + row * D + c] = to_t<T>(sv);
-                s_new[0][c] = round_to<T>(sk);
-                s_new[1][c] = round_to<T>(sv);
-            }
+        // The last item's step update of the recurrent state: its inputs are
+        // loaded now and used after the old rows, so their latency overlaps
+        // the stream (channel tid; kCompute >= D)
+        static_assert(kCompute >= D, "one channel per scoring thread");
+        float in_k = 0.f, in_v = 0.f, in_g = 0.f, st_k = 0.f, st_v = 0.f;
+        const size_t e_new = bh * D + tid;
+        if (last && tid < D) {
+            in_k = (float)static_cast<const T *>(p.k)[e_new];
+            in_v = (float)static_cast<const T *>(p.v)[e_new];
+            if (p.recur[h]) in_g = (float)static_cast<const T *>(p.g)[e_new];
+            st_k = p.state[0][e_new];
+            st_v = p.state[1][e_new];
         }
 
         // the item's old rows, one ring stage at a time; group grp takes rows
@@ -322,6 +311,25 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         }
 
         if (last) {
+            // step update and append of the new row (no item reads it this step)
+            if (tid < D) {
+                float a = 0.f, oma = 1.f;
+                if (p.recur[h]) {
+                    const float gl_ = fminf(fmaxf(in_g, -80.f), 80.f);
+                    const float ex = expf(-gl_);
+                    a = 1.f / (1.f + ex);
+                    oma = ex * a;
+                }
+                const float sk = a * st_k + oma * in_k;
+                const float sv = a * st_v + oma * in_v;
+                p.state[0][e_new] = sk;
+                p.state[1][e_new] = sv;
+                const size_t row = (size_t)r * S + n_old;
+                static_cast<T *>(p.cache[0])[bh * (size_t)p.cache_R * D + row * D + tid] = to_t<T>(sk);
+                static_cast<T *>(p.cache[1])[bh * (size_t)p.cache_R * D + row * D + tid] = to_t<T>(sv);
+                s_new[0][tid] = round_to<T>(sk);
+                s_new[1][tid] = round_to<T>(sv);
+            }
             compute_sync();  // the new row is in shared memory
             // old rows of the window: j in [max(0, t-W+1), t-1]
             if (W > 0) {
@@ -381,20 +389,36 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         compute_sync();
         float M = -INFINITY;
         for (int g2 = 0; g2 < NG; ++g2) M = fmaxf(M, s_m[g2]);
-        for (int c = tid; c < D; c += kCompute) {
-            float o = 0.f;
-            for (int g2 = 0; g2 < NG; ++g2)
-                if (s_m[g2] != -INFINITY) o += s_o[g2][c] * exp2f(s_m[g2] - M);
-            part[c] = o;
-        }
-        if (tid == 0) {
+        if (p.nsplit[h] == 1) {
+            // the only item of (b, h): write o and lse directly (an invalid
+            // position leaves every row group empty: o = 0, lse = -inf)
             float L = 0.f;
             for (int g2 = 0; g2 < NG; ++g2)
                 if (s_m[g2] != -INFINITY) L += s_l[g2] * exp2f(s_m[g2] - M);
-            part[D] = M;
-            part[D + 1] = L;
+            for (int c = tid; c < D; c += kCompute) {
+                float o = 0.f;
+                for (int g2 = 0; g2 < NG; ++g2)
+                    if (s_m[g2] != -INFINITY) o += s_o[g2][c] * exp2f(s_m[g2] - M);
+                static_cast<T *>(p.o)[bh * D + c] = to_t<T>(L > 0.f ? o / L : 0.f);
+                if (p.lse && c == 0) p.lse[bh] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+            }
+        } else {
+            for (int c = tid; c < D; c += kCompute) {
+                float o = 0.f;
+                for (int g2 = 0; g2 < NG; ++g2)
+                    if (s_m[g2] != -INFINITY) o += s_o[g2][c] * exp2f(s_m[g2] - M);
+                part[c] = o;
+            }
+            if (tid == 0) {
+                float L = 0.f;
+                for (int g2 = 0; g2 < NG; ++g2)
+                    if (s_m[g2] != -INFINITY) L += s_l[g2] * exp2f(s_m[g2] - M);
+                part[D] = M;
+                part[D + 1] = L;
+            }
         }
     }
+    if (p.nsplit[h] == 1) return;   // nothing to combine
 
     // the last item of (b, h) to finish combines all of them
     __threadfence();
