@@ -72,6 +72,23 @@ def test_workspace_grows_with_what_it_holds(lib):
     assert d2 > d1 > 0
 
 
+def test_decode_split_adapts_to_the_batch(lib):
+    # Decode splits each (b, h) slab into work items of at most 2048 rows, and
+    # halves that (down to 256) while batch x items would leave SMs idle.  The
+    # workspace holds one (d + 2)-float partial per item, so its size per batch
+    # entry shows the split: 16 heads at D = 16, capacity 32768 (2048-row slabs).
+    def part_floats_per_b(B):
+        c = cfg(B=B, H=16, dil=[16] * 16, win=[0] * 16)
+        return lib.rat_workspace_size(c.ref(), rat.RAT_OP_DECODE, 32768)
+    big, small = part_floats_per_b(256), part_floats_per_b(1)
+    items_big = 16 * 1      # one 2048-row item per head already fills the GPU at batch 256
+    items_small = 16 * 8    # batch 1: 256-row items
+    per_item = (128 + 2) * 4
+    assert big >= 256 * items_big * per_item
+    assert big < 256 * 2 * items_big * per_item      # not split further
+    assert small >= items_small * per_item            # split down to 256-row items
+
+
 def test_cache_rows_layout(lib):
     # rows per (b,h) block = max_h D_h * ceil(cap / D_h)
     c = cfg(H=3, dil=[1, 16, 64], win=[0, 0, 256])

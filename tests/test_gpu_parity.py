@@ -318,7 +318,8 @@ def test_decode_from_empty_history():
 
 
 def test_decode_long_slab_spans_several_splits():
-    # 2500 old rows in the residue slab: three split items plus the tail item
+    # 2500 old rows in the residue slab: at batch 1 the plan splits it into ten
+    # 256-row items (the last one also does the step update), combined by LSE
     run_decode_case(B=1, T=5000, steps=2, H=2, d=128, dtype=torch.bfloat16, dil=[2, 1], win=[0, 7],
                     recur=[1, 1], mu=2.0, seed=6)
 
