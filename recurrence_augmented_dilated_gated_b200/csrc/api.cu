@@ -203,7 +203,6 @@ rat_status run_scan(const rat_cfg *c, const Layout &L, const void *k, const void
     p.nslices = c->B * n;
     p.nchunks = L.nchunks;
     p.chunk_len = scan_chunk_len(c->d);
-    p.sub_len = 0;
     const void *srcs[5] = {k, v, g, kt, vt};
     p.use_tma_out = kt != nullptr ? 1 : 0;
     for (int i = 0; i < (p.use_tma_out ? 5 : 3); ++i)

@@ -91,7 +91,7 @@ struct ScanParams {
     int B, T, H, d;
     int nslices;            // B * nheads
     int nchunks;            // chunks along T per slice
-    int chunk_len, sub_len; // timesteps per chunk / per thread group
+    int chunk_len;          // timesteps per chunk
     int nheads;             // heads taken by this launch
     unsigned char head_list[kMaxHeads];
     unsigned char head_recur[kMaxHeads];
