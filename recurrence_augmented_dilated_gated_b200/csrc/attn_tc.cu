@@ -823,6 +823,15 @@ size_t attn_tc_smem_bytes(int hd) {
     return need > 120 * 1024 ? need : 120 * 1024;
 }
 
+template <int HD, bool kWin>
+cudaError_t launch_inst(const TcParams &p, unsigned grid, size_t smem, cudaStream_t s) {
+    static std::atomic<unsigned long long> smem_set{0};
+    cudaError_t e = ensure_smem_limit(attn_tc_kernel<HD, kWin>, smem, smem_set);
+    if (e != cudaSuccess) return e;
+    attn_tc_kernel<HD, kWin><<<grid, kThreads, smem, s>>>(p);
+    return cudaSuccess;
+}
+
 cudaError_t launch_attn_tc(const TcParams &p, int hd, cudaStream_t s) {
     if (p.total_units == 0) return cudaSuccess;
     const size_t smem = attn_tc_smem_bytes(hd);
@@ -832,16 +841,10 @@ cudaError_t launch_attn_tc(const TcParams &p, int hd, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM (the shared memory and TMEM of one CTA fill an SM)
     const unsigned grid = (unsigned)std::min<long long>(p.total_units, (long long)nsm);
-    auto go = [&](auto kern) -> cudaError_t {
-        cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (r != cudaSuccess) return r;
-        kern<<<grid, kThreads, smem, s>>>(p);
-        return cudaSuccess;
-    };
     // the dilated and window launches are separate instantiations, so each
     // carries only its own epilogue and masks (instruction-cache footprint)
-    if (hd == 128) e = p.window_mode ? go(attn_tc_kernel<128, true>) : go(attn_tc_kernel<128, false>);
-    else e = p.window_mode ? go(attn_tc_kernel<64, true>) : go(attn_tc_kernel<64, false>);
+    if (hd == 128) e = p.window_mode ? launch_inst<128, true>(p, grid, smem, s) : launch_inst<128, false>(p, grid, smem, s);
+    else e = p.window_mode ? launch_inst<64, true>(p, grid, smem, s) : launch_inst<64, false>(p, grid, smem, s);
     if (e != cudaSuccess) return e;
     count_launches(1);
     return cudaGetLastError();

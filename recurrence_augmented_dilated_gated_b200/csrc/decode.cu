@@ -456,7 +456,8 @@ template <typename T, int D>
 cudaError_t launch_typed(const DecodeParams &p, unsigned grid, cudaStream_t s) {
     constexpr int RS = (kCompute / (D / 8)) * kBatch;
     const size_t smem = (size_t)kStages * 2 * RS * D * sizeof(T);
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<unsigned long long> smem_set{0};
+    cudaError_t e = ensure_smem_limit(decode_kernel<T, D>, smem, smem_set);
     if (e != cudaSuccess) return e;
     decode_kernel<T, D><<<grid, kThreads, smem, s>>>(p);
     return cudaSuccess;

@@ -7,9 +7,27 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "rat.h"
 
 namespace rat {
+
+// Raise a kernel's dynamic shared-memory limit once per device.  The setting
+// persists, so repeating it on every launch would only add a host call to
+// every step (and one more call that stream capture has to tolerate).
+// `done` holds one bit per device and must be distinct per kernel.
+template <typename Kernel>
+cudaError_t ensure_smem_limit(Kernel kernel, size_t bytes, std::atomic<unsigned long long> &done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
 
 constexpr int kMaxHeads = 256;
 constexpr long long kDefaultSpinNs = 1000000000LL;  // 1 s bound on every device-side wait

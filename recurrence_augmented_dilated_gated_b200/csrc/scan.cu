@@ -585,7 +585,8 @@ size_t scan_smem() {
 template <typename T, int D>
 cudaError_t launch_one(const ScanParams &p, unsigned tickets, cudaStream_t s) {
     const size_t smem = scan_smem<T, D>();
-    cudaError_t e = cudaFuncSetAttribute(scan_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static std::atomic<unsigned long long> smem_set{0};
+    cudaError_t e = ensure_smem_limit(scan_kernel<T, D>, smem, smem_set);
     if (e != cudaSuccess) return e;
     scan_kernel<T, D><<<tickets, kThreads, smem, s>>>(p);
     return cudaSuccess;

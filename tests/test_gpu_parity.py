@@ -324,6 +324,104 @@ def test_decode_long_slab_spans_several_splits():
                     recur=[1, 1], mu=2.0, seed=6)
 
 
+def _prefill_cache_per_entry(cfg1, k, v, g, T_b, cap, ck, cv, sk, sv):
+    """Fill batch entry b's cache rows and state from its own T_b tokens (one
+    B = 1 scan per entry, writing into that entry's slices)."""
+    for b, Tb in enumerate(T_b):
+        c = cfg1.replace(B=1, T=Tb)
+        ws = rat.workspace(c, rat.RAT_OP_SCAN)
+        rat.rat_scan_prefill(c, k[b:b + 1, :Tb].contiguous(), v[b:b + 1, :Tb].contiguous(),
+                             g[b:b + 1, :Tb].contiguous(), None, None, None, None, sk[b:b + 1], sv[b:b + 1],
+                             ck[b:b + 1], cv[b:b + 1], cap, ws)
+        rat.rat_check_status(ws)
+
+
+def test_decode_ragged_positions():
+    # each sequence of the batch at its own position (pos is per entry): a
+    # batch entry reads only its own residue slab and window
+    B, H, d, dtype = 4, 3, 128, torch.bfloat16
+    dil, win, recur = [1, 8, 5], [0, 16, 33], [0, 1, 1]
+    T_b = [1, 700, 1299, 2048]
+    steps, cap = 3, max(T_b) + 3
+    Tt = max(T_b) + steps
+    q, k, v, g = inputs(B, Tt, H, d, dtype, seed=31)
+    cfg = make_cfg(B, max(T_b), H, d, dtype, dil, win, recur)
+    R = rat.rat_cache_rows(cfg, cap)
+    ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
+    cv = torch.zeros_like(ck)
+    sk = torch.empty(B, H, d, device=DEV)
+    sv = torch.empty_like(sk)
+    _prefill_cache_per_entry(cfg, k, v, g, T_b, cap, ck, cv, sk, sv)
+    wsd = rat.workspace(cfg, rat.RAT_OP_DECODE, cap)
+    kt, _ = oracle.scan(f64(k), f64(g), None, recur)
+    vt, _ = oracle.scan(f64(v), f64(g), None, recur)
+    for s in range(steps):
+        pos_l = [t + s for t in T_b]
+        pos = torch.tensor(pos_l, dtype=torch.int32, device=DEV)
+        tok = lambda x: torch.stack([x[b, pos_l[b]] for b in range(B)]).contiguous()
+        o = torch.empty(B, H, d, dtype=dtype, device=DEV)
+        lse = torch.empty(B, H, device=DEV)
+        rat.rat_decode_step(cfg, tok(q), tok(k), tok(v), tok(g), sk, sv, ck, cv, cap, pos, o, lse, wsd)
+        rows = np.array([(b, h, pos_l[b]) for b in range(B) for h in range(H)])
+        ro, rl = oracle.attn_rows(f64(q), kt, vt, dil, win, rows, parts=3)
+        assert_close(o, ro.reshape(B, H, d), dtype, "ragged decode o step %d" % s)
+        assert_close(lse, rl.reshape(B, H), torch.float32 if dtype == torch.float32 else dtype,
+                     "ragged decode lse step %d" % s)
+    rat.rat_check_status(wsd)
+
+
+def test_decode_step_replays_from_a_cuda_graph():
+    # one rat_decode_step captured in a CUDA graph (its counter reset and its
+    # kernel), replayed for several tokens with the inputs and positions
+    # refreshed in place between replays
+    B, H, d, dtype = 2, 2, 128, torch.bfloat16
+    dil, win, recur = [4, 1], [8, 0], [1, 0]
+    T, steps = 1000, 4
+    cap = T + steps
+    q, k, v, g = inputs(B, T + steps, H, d, dtype, seed=41)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur)
+    R = rat.rat_cache_rows(cfg, cap)
+    ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
+    cv = torch.zeros_like(ck)
+    sk = torch.empty(B, H, d, device=DEV)
+    sv = torch.empty_like(sk)
+    _prefill_cache_per_entry(cfg, k, v, g, [T] * B, cap, ck, cv, sk, sv)
+    wsd = rat.workspace(cfg, rat.RAT_OP_DECODE, cap)
+    xq, xk, xv, xg = (torch.empty(B, H, d, dtype=dtype, device=DEV) for _ in range(4))
+    pos = torch.full((B,), T, dtype=torch.int32, device=DEV)
+    o = torch.empty(B, H, d, dtype=dtype, device=DEV)
+    lse = torch.empty(B, H, device=DEV)
+    # a first eager step (also warms up), then capture the same step
+    for x_, src in zip((xq, xk, xv, xg), (q, k, v, g)):
+        x_.copy_(src[:, T])
+    rat.rat_decode_step(cfg, xq, xk, xv, xg, sk, sv, ck, cv, cap, pos, o, lse, wsd)
+    torch.cuda.synchronize()
+    outs = [(o.clone(), lse.clone())]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        rat.rat_decode_step(cfg, xq, xk, xv, xg, sk, sv, ck, cv, cap, pos, o, lse, wsd)
+    for s in range(1, steps):
+        for x_, src in zip((xq, xk, xv, xg), (q, k, v, g)):
+            x_.copy_(src[:, T + s])
+        pos.fill_(T + s)
+        graph.replay()
+        outs.append((o.clone(), lse.clone()))
+    torch.cuda.synchronize()
+    rat.rat_check_status(wsd)
+    kt, fk = oracle.scan(f64(k), f64(g), None, recur)
+    vt, fv = oracle.scan(f64(v), f64(g), None, recur)
+    rows = np.array([(b, h, t) for b in range(B) for h in range(H) for t in range(T, T + steps)])
+    ro, rl = oracle.attn_rows(f64(q), kt, vt, dil, win, rows, parts=3)
+    ro = ro.reshape(B, H, steps, d)
+    rl = rl.reshape(B, H, steps)
+    for s, (os_, ls_) in enumerate(outs):
+        assert_close(os_, ro[:, :, s], dtype, "graph decode o step %d" % s)
+        assert_close(ls_, rl[:, :, s], dtype, "graph decode lse step %d" % s)
+    assert_close(sk, fk, dtype, "state_k after the replays")
+    assert_close(sv, fv, dtype, "state_v after the replays")
+    del graph
+
+
 def test_decode_bad_position_is_reported():
     B, H, d = 2, 2, 64
     cfg = make_cfg(B, 1, H, d, torch.bfloat16, [2, 2], [0, 0])
