@@ -73,7 +73,7 @@ typedef struct CUstream_st *rat_stream_t;
 typedef enum {
     RAT_OK = 0,
     RAT_ERR_INVALID = 1,     /* null / misaligned pointer, out-of-range size or parameter */
-    RAT_ERR_UNSUPPORTED = 2, /* valid request with no kernel in this build (e.g. d not 64/128) */
+    RAT_ERR_UNSUPPORTED = 2, /* valid request with no kernel in this library (e.g. d not 64/128) */
     RAT_ERR_CUDA = 3,        /* a CUDA runtime call or a kernel launch failed */
     RAT_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up (rat_check_status) */
     RAT_ERR_WORKSPACE = 5    /* ws_bytes below rat_workspace_size() */
@@ -95,7 +95,7 @@ typedef enum {
  * the call only.  Head h uses dilation dil[h] >= 1, window win[h] >= 0 (0 = no
  * window) and recurrence flag recur[h] (0 = no recurrence; NULL = all heads
  * recurrent) -- the hybrid head compositions of the RAT+ Abstract.
- * Limits of this build: d in {64, 128}; 1 <= H <= 256; B, T >= 0;
+ * Limits of this library version: d in {64, 128}; 1 <= H <= 256; B, T >= 0;
  * B*T*H*d < 2^40 elements.  An empty batch or sequence (B*T == 0) launches
  * no kernel; a prefill then only copies init (or zero) to final.
  */

@@ -176,7 +176,7 @@ def test_short_sequences_on_both_paths(T):
 
 
 def test_maximum_head_count():
-    # H = 256, the largest head count of this build, mixed dilations
+    # H = 256, the largest head count the library accepts, mixed dilations
     B, T, H, d = 1, 64, 256, 64
     dil = [1 + (h % 4) for h in range(H)]
     win = [(h % 3) * 4 for h in range(H)]
