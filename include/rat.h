@@ -36,9 +36,12 @@
  *     RAT_F32).  States, init and lse are always fp32.
  *   - Every device pointer must be 16-byte aligned.
  *   - Ownership: the caller owns every buffer and the stream.  The library
- *     allocates no device memory, keeps no global state and may be called from
- *     several host threads on different workspaces.  Calls are asynchronous on
- *     `stream`; inputs must stay valid until the stream reaches the call.
+ *     allocates no device memory and may be called from several host threads
+ *     on different workspaces.  Its only process-wide state is a launch
+ *     counter, a per-thread last-error string, each kernel's shared-memory
+ *     limit (raised once per device), and the static scratch of
+ *     rat_decode_step_noalloc.  Calls are asynchronous on `stream`; inputs
+ *     must stay valid until the stream reaches the call.
  *   - Workspace: `ws` is caller-allocated device memory of at least
  *     rat_workspace_size() bytes, zero-filled once before its first use
  *     (rat_workspace_init does that).  Calls that share a workspace must be
@@ -185,6 +188,10 @@ RAT_API rat_status rat_mix_prefill(const rat_cfg *cfg, const void *q, const void
  *                of range makes the kernel skip that entry and record
  *                RAT_ERR_INVALID for rat_check_status)
  *   o            out [B,H,d];  lse out [B,H] fp32 or NULL
+ * Positions may differ between batch entries (a ragged batch).  A step issues
+ * one memset (its combine counters) and one kernel on `stream`, and after the
+ * first call on a device no other CUDA runtime call, so a step can be captured
+ * in a CUDA graph and replayed with the inputs and pos refreshed in place.
  */
 RAT_API rat_status rat_decode_step(const rat_cfg *cfg, const void *q, const void *k, const void *v,
                            const void *g, float *state_k, float *state_v, void *cache_k,
@@ -201,7 +208,8 @@ RAT_API rat_status rat_decode_step(const rat_cfg *cfg, const void *q, const void
  *   - Scratch: a static 16 MiB device array inside librat.so, held by every
  *     GPU that loads the library until the process exits.  A step needs
  *     about 256 + B * items * (d + 2) * 4 + B * H * 4 bytes, items = sum over
- *     heads of ceil(ceil(cache_cap / D_h) / 512); a larger step returns
+ *     heads of ceil(ceil(cache_cap / D_h) / r), where r = 2048 rows is halved
+ *     (down to 256) while B * items < 592; a larger step returns
  *     RAT_ERR_UNSUPPORTED with the sizes in rat_last_error().
  *   - The first call on a device (with that device current) looks up the
  *     array's device address (cudaGetSymbolAddress) and caches it; make that
