@@ -35,6 +35,8 @@
  *      recurrence-augmented; both parts read the augmented keys and values.
  *   R6 a head with recur = 0 uses a = 0, i.e. augmented keys/values equal the
  *      raw ones (D = 1, a = 0 is plain causal attention).
+ *   R7 (a second reading, kept for comparison) fixed-grid dilation: query t
+ *      attends to { j <= t : j mod D == D - 1 } plus t (oracle_attn_rows_grid).
  *
  * Parity pins for every function here live in tests/test_oracle_pins.py.
  */
@@ -131,9 +133,10 @@ static void lse_merge(int d, const double *o1, double l1, const double *o2, doub
  *   o, lse    : nrows x d, nrows
  * Returns 0, or -1 on an argument error (the outputs are then untouched).
  */
-int oracle_attn_rows(int B, int T, int H, int d, const double *q, const double *kt,
-                     const double *vt, const int *dil, const int *win, double scale,
-                     int parts, long nrows, const int64_t *rows, double *o, double *lse)
+static int attn_rows_impl(int B, int T, int H, int d, const double *q, const double *kt,
+                          const double *vt, const int *dil, const int *win, double scale,
+                          int parts, long nrows, const int64_t *rows, double *o, double *lse,
+                          int grid)
 {
     if (parts < 1 || parts > 3) return -1;
     for (long r = 0; r < nrows; ++r) {
@@ -161,10 +164,15 @@ int oracle_attn_rows(int B, int T, int H, int d, const double *q, const double *
             const double *qrow = q + idx4(T, H, d, b, t, h, 0);
             int D = dil[h], W = win[h];
             double l1 = 0.0, l2 = 0.0;
-            if (parts & 1) { /* R2: j <= t with (t - j) mod D == 0 */
+            if (parts & 1) {
                 long n = 0;
-                for (long j = 0; j <= t; ++j)
-                    if ((t - j) % D == 0) js[n++] = j;
+                if (!grid) { /* R2: j <= t with (t - j) mod D == 0 */
+                    for (long j = 0; j <= t; ++j)
+                        if ((t - j) % D == 0) js[n++] = j;
+                } else {    /* fixed grid: j <= t on the grid j mod D == D - 1, plus t */
+                    for (long j = 0; j <= t; ++j)
+                        if (j % D == D - 1 || j == t) js[n++] = j;
+                }
                 softmax_over(T, H, d, qrow, kt, vt, b, h, js, n, scale, o1, &l1, z);
             }
             if ((parts & 2) && W > 0) { /* R3: max(0, t-W+1) <= j <= t */
@@ -187,6 +195,29 @@ int oracle_attn_rows(int B, int T, int H, int d, const double *q, const double *
         free(js); free(z); free(o1); free(o2);
     }
     return err ? -1 : 0;
+}
+
+int oracle_attn_rows(int B, int T, int H, int d, const double *q, const double *kt,
+                     const double *vt, const int *dil, const int *win, double scale,
+                     int parts, long nrows, const int64_t *rows, double *o, double *lse)
+{
+    return attn_rows_impl(B, T, H, d, q, kt, vt, dil, win, scale, parts, nrows, rows, o, lse, 0);
+}
+
+/*
+ * The same rows under the fixed-grid reading of dilation, kept for comparison
+ * with R4 ([RAT+] Abstract: dilation cuts the KV cache by a factor of D;
+ * [RAT] Approach: attention over chunk-level keys, one per chunk of D tokens).
+ * Query t's dilated part attends to the keys on a grid shared by all queries,
+ * { j <= t : j mod D == D - 1 }, plus t itself; so a decode cache needs only
+ * one row per D positions.  For t with t mod D == D - 1 the set equals R2's.
+ * The window part and the merge are R3 and R4, unchanged.
+ */
+int oracle_attn_rows_grid(int B, int T, int H, int d, const double *q, const double *kt,
+                          const double *vt, const int *dil, const int *win, double scale,
+                          int parts, long nrows, const int64_t *rows, double *o, double *lse)
+{
+    return attn_rows_impl(B, T, H, d, q, kt, vt, dil, win, scale, parts, nrows, rows, o, lse, 1);
 }
 
 /*

@@ -3,7 +3,8 @@
 Each mutant is rat_oracle.c with one textual change (a swapped gate, a wrong
 sign, a dropped term, a wrong dilation residue, a window off by one, a wrong
 merge, a dropped scale, a transposed operand, a gate one step late, a decode
-that ignores the per-head recurrence flag).  It is compiled into a temporary
+that ignores the per-head recurrence flag, a fixed grid on the wrong residue
+or without the query's own key).  It is compiled into a temporary
 directory and the pin suite is run against it in a subprocess; the suite must
 fail.  The shipped oracle is never modified.
 """
@@ -32,6 +33,8 @@ MUTANTS = {
                          "acc += qrow[c] * v[idx4(T, H, d, b, js[i], h, c)];"),
     "decode_ignores_recur": ("double a = (recur == NULL || recur[h]) ? sigmoid(g[e]) : 0.0;",
                              "double a = sigmoid(g[e]);"),
+    "grid_on_residue_zero": ("if (j % D == D - 1 || j == t) js[n++] = j;", "if (j % D == 0 || j == t) js[n++] = j;"),
+    "grid_without_self": ("if (j % D == D - 1 || j == t) js[n++] = j;", "if (j % D == D - 1) js[n++] = j;"),
 }
 
 

@@ -251,6 +251,68 @@ def test_first_row_and_convex_hull():
         assert np.all(o[:, t] >= lo - 1e-12) and np.all(o[:, t] <= hi + 1e-12)
 
 
+# -------------------------------------------------- fixed-grid dilation (comparison)
+# The fixed-grid reading: query t's dilated part takes the keys j <= t with
+# j mod D == D - 1 (one per chunk of D tokens, shared by all queries) plus t.
+
+
+@pytest.mark.parametrize("T", [1, 19])
+def test_grid_with_d_1_is_dense_causal(T):
+    B, H, d = 1, 2, 6
+    q, k, v = rand_qkv(B, T, H, d)
+    o, _ = oracle.attention(q, k, v, [1] * H, [0] * H, grid=True)
+    for h in range(H):
+        np.testing.assert_allclose(o[0, :, h], sdpa_causal(q[0, :, h], k[0, :, h], v[0, :, h], 1 / math.sqrt(d)),
+                                   rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("T,D", [(37, 3), (37, 5), (20, 8), (9, 12)])
+def test_grid_equals_masked_sdpa(T, D):
+    # brute force: SDPA with the boolean mask of the grid set
+    B, H, d = 1, 1, 7
+    q, k, v = rand_qkv(B, T, H, d)
+    scale = 0.45
+    o, _ = oracle.attention(q, k, v, [D], [0], parts=1, scale=scale, grid=True)
+    i, j = np.meshgrid(np.arange(T), np.arange(T), indexing="ij")
+    mask = (j <= i) & ((j % D == D - 1) | (j == i))
+    np.testing.assert_allclose(o[0, :, 0], sdpa_causal(q[0, :, 0], k[0, :, 0], v[0, :, 0], scale, mask),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_grid_rows_on_the_grid_equal_the_residue_reading():
+    # for t with t mod D == D - 1 both readings select the same keys
+    B, T, H, d = 1, 50, 2, 5
+    q, k, v = rand_qkv(B, T, H, d)
+    dil = [4, 7]
+    rows = [(0, h, t) for h in range(H) for t in range(T) if t % dil[h] == dil[h] - 1]
+    og, lg = oracle.attn_rows(q, k, v, dil, [0, 0], rows, parts=1, grid=True)
+    orr, lr = oracle.attn_rows(q, k, v, dil, [0, 0], rows, parts=1)
+    np.testing.assert_allclose(og, orr, rtol=0, atol=0)
+    np.testing.assert_allclose(lg, lr, rtol=0, atol=0)
+
+
+def test_grid_rows_before_the_first_grid_key_see_only_themselves():
+    B, T, H, d, D = 1, 6, 1, 4, 8
+    q, k, v = rand_qkv(B, T, H, d)
+    o, lse = oracle.attention(q, k, v, [D], [0], parts=1, scale=0.5, grid=True)
+    np.testing.assert_allclose(o[0, :, 0], v[0, :, 0], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(lse[0, 0], 0.5 * np.einsum("tc,tc->t", q[0, :, 0], k[0, :, 0]), rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("T,D,W", [(40, 4, 6), (23, 6, 2)])
+def test_grid_merge_is_one_softmax_over_both_sets(T, D, W):
+    B, H, d = 1, 1, 5
+    q, k, v = rand_qkv(B, T, H, d)
+    scale = 0.6
+    o, lse = oracle.attention(q, k, v, [D], [W], parts=3, scale=scale, grid=True)
+    for t in range(T):
+        keys = [j for j in range(t + 1) if j % D == D - 1 or j == t] + [j for j in range(max(0, t - W + 1), t + 1)]
+        z = torch.from_numpy(scale * k[0, keys, 0] @ q[0, t, 0])
+        p = torch.softmax(z, dim=0).numpy()
+        np.testing.assert_allclose(o[0, t, 0], p @ v[0, keys, 0], rtol=1e-12, atol=1e-12)
+        assert abs(lse[0, 0, t] - torch.logsumexp(z, 0).item()) < 1e-12
+
+
 # --------------------------------------------------------------------------- decode
 
 
