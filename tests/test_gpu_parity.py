@@ -233,6 +233,26 @@ def test_empty_inputs():
     assert torch.equal(fk, init) and torch.all(fv == 0)
 
 
+def test_workspace_reused_across_calls():
+    # one workspace for several calls with different inputs: the per-call
+    # reset of the attention work counters and of the scan's chunk flags
+    B, T, H, d, dtype = 1, 2048, 3, 128, torch.bfloat16
+    dil, win, recur = [16, 1, 4], [128, 0, 0], [1, 0, 1]
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur)
+    ws = rat.workspace(cfg, rat.RAT_OP_MIX)
+    o = torch.empty(B, T, H, d, dtype=dtype, device=DEV)
+    lse = torch.empty(B, H, T, device=DEV)
+    for call in range(3):
+        q, k, v, g = inputs(B, T, H, d, dtype, seed=900 + call)
+        rat.rat_mix_prefill(cfg, q, k, v, g, None, None, o, lse, None, None, None, None, ws)
+        rat.rat_check_status(ws)
+        kt, _ = oracle.scan(f64(k), f64(g), None, recur)
+        vt, _ = oracle.scan(f64(v), f64(g), None, recur)
+        ro, rl = oracle.attention(f64(q), kt, vt, dil, win)
+        assert_close(o, ro, dtype, "o, call %d" % call)
+        assert_close(lse, rl, dtype, "lse, call %d" % call)
+
+
 def test_decode_cache_layout_from_scan():
     # cache row of position j in head h: (j mod D_h) * ceil(cap/D_h) + j // D_h
     B, T, H, d = 2, 300, 3, 64
