@@ -36,6 +36,8 @@ def _load():
         lib.oracle_attn_rows.restype = ctypes.c_int
         lib.oracle_attn_rows_grid.argtypes = lib.oracle_attn_rows.argtypes
         lib.oracle_attn_rows_grid.restype = ctypes.c_int
+        lib.oracle_attn_rows_ex.argtypes = lib.oracle_attn_rows.argtypes + [ctypes.c_int, ctypes.c_int]
+        lib.oracle_attn_rows_ex.restype = ctypes.c_int
         lib.oracle_decode_step.argtypes = [ctypes.c_int] * 4 + [ip, dp, dp, dp, dp, ip, ip, up,
                                                                 ctypes.c_double, dp, dp, dp, dp, dp, dp]
         lib.oracle_decode_step.restype = ctypes.c_int
@@ -77,10 +79,11 @@ def scan(x, g, init=None, recur=None):
     return out, final
 
 
-def attn_rows(q, kt, vt, dil, win, rows, parts=3, scale=None, grid=False):
+def attn_rows(q, kt, vt, dil, win, rows, parts=3, scale=None, grid=False, dedupe=False):
     """Rows (b, h, t) of the attention step; returns (o [n,d], lse [n]).
     grid=True takes the fixed-grid reading of the dilated part (keys j <= t
-    with j mod D == D - 1, plus t) instead of the residue set."""
+    with j mod D == D - 1, plus t) instead of the residue set; dedupe=True
+    counts a key that both parts hold once (the window part skips it)."""
     lib = _load()
     q, kt, vt = _f64(q), _f64(kt), _f64(vt)
     B, T, H, d = q.shape
@@ -90,11 +93,11 @@ def attn_rows(q, kt, vt, dil, win, rows, parts=3, scale=None, grid=False):
     o = np.empty((n, d), dtype=np.float64)
     lse = np.empty((n,), dtype=np.float64)
     s = default_scale(d) if scale is None else float(scale)
-    fn = lib.oracle_attn_rows_grid if grid else lib.oracle_attn_rows
-    rc = fn(B, T, H, d, _dp(q), _dp(kt), _dp(vt),
-                              dil.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
-                              win.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), s, int(parts), n,
-                              rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), _dp(o), _dp(lse))
+    rc = lib.oracle_attn_rows_ex(B, T, H, d, _dp(q), _dp(kt), _dp(vt),
+                                 dil.ctypes.data_as(ctypes.POINTER(ctypes.c_int)),
+                                 win.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), s, int(parts), n,
+                                 rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), _dp(o), _dp(lse),
+                                 int(bool(grid)), int(bool(dedupe)))
     if rc != 0:
         raise ValueError("oracle_attn_rows: invalid arguments")
     return o, lse
@@ -106,11 +109,11 @@ def all_rows(B, T, H):
     return np.stack([b.ravel(), h.ravel(), t.ravel()], axis=1)
 
 
-def attention(q, kt, vt, dil, win, parts=3, scale=None, grid=False):
+def attention(q, kt, vt, dil, win, parts=3, scale=None, grid=False, dedupe=False):
     """Every row of the attention step as full tensors: (o [B,T,H,d], lse [B,H,T])."""
     B, T, H, d = q.shape
     rows = all_rows(B, T, H)
-    o, lse = attn_rows(q, kt, vt, dil, win, rows, parts=parts, scale=scale, grid=grid)
+    o, lse = attn_rows(q, kt, vt, dil, win, rows, parts=parts, scale=scale, grid=grid, dedupe=dedupe)
     o = o.reshape(B, H, T, d).transpose(0, 2, 1, 3).copy()
     return o, lse.reshape(B, H, T)
 

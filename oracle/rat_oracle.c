@@ -37,6 +37,9 @@
  *      raw ones (D = 1, a = 0 is plain causal attention).
  *   R7 (a second reading, kept for comparison) fixed-grid dilation: query t
  *      attends to { j <= t : j mod D == D - 1 } plus t (oracle_attn_rows_grid).
+ *   R8 (a variant, off by default) dedupe: a key in both parts counts once,
+ *      i.e. the window part skips the keys of the dilated set
+ *      (oracle_attn_rows_ex).
  *
  * Parity pins for every function here live in tests/test_oracle_pins.py.
  */
@@ -136,7 +139,7 @@ static void lse_merge(int d, const double *o1, double l1, const double *o2, doub
 static int attn_rows_impl(int B, int T, int H, int d, const double *q, const double *kt,
                           const double *vt, const int *dil, const int *win, double scale,
                           int parts, long nrows, const int64_t *rows, double *o, double *lse,
-                          int grid)
+                          int grid, int dedupe)
 {
     if (parts < 1 || parts > 3) return -1;
     for (long r = 0; r < nrows; ++r) {
@@ -179,6 +182,15 @@ static int attn_rows_impl(int B, int T, int H, int d, const double *q, const dou
                 long n = 0;
                 for (long j = 0; j <= t; ++j)
                     if (j >= t - W + 1) js[n++] = j;
+                if (dedupe) { /* R8: keys the dilated part holds count once */
+                    long n2 = 0;
+                    for (long i = 0; i < n; ++i) {
+                        const long j = js[i];
+                        const int in_dil = grid ? (j % D == D - 1 || j == t) : ((t - j) % D == 0);
+                        if (!in_dil) js[n2++] = j;
+                    }
+                    n = n2;
+                }
                 softmax_over(T, H, d, qrow, kt, vt, b, h, js, n, scale, o2, &l2, z);
             }
             double *orow = o + (size_t)r * (size_t)d;
@@ -201,7 +213,7 @@ int oracle_attn_rows(int B, int T, int H, int d, const double *q, const double *
                      const double *vt, const int *dil, const int *win, double scale,
                      int parts, long nrows, const int64_t *rows, double *o, double *lse)
 {
-    return attn_rows_impl(B, T, H, d, q, kt, vt, dil, win, scale, parts, nrows, rows, o, lse, 0);
+    return attn_rows_impl(B, T, H, d, q, kt, vt, dil, win, scale, parts, nrows, rows, o, lse, 0, 0);
 }
 
 /*
@@ -217,7 +229,22 @@ int oracle_attn_rows_grid(int B, int T, int H, int d, const double *q, const dou
                           const double *vt, const int *dil, const int *win, double scale,
                           int parts, long nrows, const int64_t *rows, double *o, double *lse)
 {
-    return attn_rows_impl(B, T, H, d, q, kt, vt, dil, win, scale, parts, nrows, rows, o, lse, 1);
+    return attn_rows_impl(B, T, H, d, q, kt, vt, dil, win, scale, parts, nrows, rows, o, lse, 1, 0);
+}
+
+/*
+ * Both readings and both merge variants in one call: grid != 0 takes the
+ * fixed-grid dilated set (R7), dedupe != 0 drops from the window part the keys
+ * the dilated part already holds (R8), so that the merge is one softmax over
+ * the union of the two sets rather than over their multiset.
+ */
+int oracle_attn_rows_ex(int B, int T, int H, int d, const double *q, const double *kt,
+                        const double *vt, const int *dil, const int *win, double scale,
+                        int parts, long nrows, const int64_t *rows, double *o, double *lse,
+                        int grid, int dedupe)
+{
+    return attn_rows_impl(B, T, H, d, q, kt, vt, dil, win, scale, parts, nrows, rows, o, lse,
+                          grid != 0, dedupe != 0);
 }
 
 /*

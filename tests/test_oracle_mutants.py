@@ -4,7 +4,7 @@ Each mutant is rat_oracle.c with one textual change (a swapped gate, a wrong
 sign, a dropped term, a wrong dilation residue, a window off by one, a wrong
 merge, a dropped scale, a transposed operand, a gate one step late, a decode
 that ignores the per-head recurrence flag, a fixed grid on the wrong residue
-or without the query's own key).  It is compiled into a temporary
+or without the query's own key, a dedupe that keeps the shared keys).  It is compiled into a temporary
 directory and the pin suite is run against it in a subprocess; the suite must
 fail.  The shipped oracle is never modified.
 """
@@ -35,6 +35,7 @@ MUTANTS = {
                              "double a = sigmoid(g[e]);"),
     "grid_on_residue_zero": ("if (j % D == D - 1 || j == t) js[n++] = j;", "if (j % D == 0 || j == t) js[n++] = j;"),
     "grid_without_self": ("if (j % D == D - 1 || j == t) js[n++] = j;", "if (j % D == D - 1) js[n++] = j;"),
+    "dedupe_ignored": ("if (!in_dil) js[n2++] = j;", "js[n2++] = j;"),
 }
 
 

@@ -313,6 +313,45 @@ def test_grid_merge_is_one_softmax_over_both_sets(T, D, W):
         assert abs(lse[0, 0, t] - torch.logsumexp(z, 0).item()) < 1e-12
 
 
+# ------------------------------------------------- dedupe variant of the merge
+# With dedupe, a key in both parts counts once: the merge is one softmax over
+# the union of the dilated and window sets (the default counts the multiset).
+
+
+@pytest.mark.parametrize("T,D,W,grid", [(40, 4, 6, False), (33, 5, 1, False), (20, 3, 40, False),
+                                        (29, 4, 9, True), (25, 6, 3, True)])
+def test_dedupe_merge_is_one_softmax_over_the_union(T, D, W, grid):
+    B, H, d = 1, 1, 5
+    q, k, v = rand_qkv(B, T, H, d)
+    scale = 0.6
+    o, lse = oracle.attention(q, k, v, [D], [W], parts=3, scale=scale, grid=grid, dedupe=True)
+    for t in range(T):
+        dil_set = {j for j in range(t + 1) if ((j % D == D - 1 or j == t) if grid else (t - j) % D == 0)}
+        keys = sorted(dil_set | set(range(max(0, t - W + 1), t + 1)))
+        z = torch.from_numpy(scale * k[0, keys, 0] @ q[0, t, 0])
+        p = torch.softmax(z, dim=0).numpy()
+        np.testing.assert_allclose(o[0, t, 0], p @ v[0, keys, 0], rtol=1e-12, atol=1e-12)
+        assert abs(lse[0, 0, t] - torch.logsumexp(z, 0).item()) < 1e-12
+
+
+def test_dedupe_with_d_1_is_dense_causal():
+    # every window key is already a dilated key at D = 1
+    B, T, H, d = 1, 26, 1, 6
+    q, k, v = rand_qkv(B, T, H, d)
+    o, _ = oracle.attention(q, k, v, [1], [5], dedupe=True)
+    np.testing.assert_allclose(o[0, :, 0], sdpa_causal(q[0, :, 0], k[0, :, 0], v[0, :, 0], 1 / math.sqrt(d)),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_dedupe_without_window_changes_nothing():
+    B, T, H, d = 1, 30, 2, 4
+    q, k, v = rand_qkv(B, T, H, d)
+    a = oracle.attention(q, k, v, [3, 7], [0, 0])
+    b = oracle.attention(q, k, v, [3, 7], [0, 0], dedupe=True)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+
+
 # --------------------------------------------------------------------------- decode
 
 
