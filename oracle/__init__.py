@@ -38,6 +38,10 @@ def _load():
         lib.oracle_attn_rows_grid.restype = ctypes.c_int
         lib.oracle_attn_rows_ex.argtypes = lib.oracle_attn_rows.argtypes + [ctypes.c_int, ctypes.c_int]
         lib.oracle_attn_rows_ex.restype = ctypes.c_int
+        lib.oracle_attn_rows_topk.argtypes = [ctypes.c_int] * 4 + [dp, dp, dp, ctypes.c_int, ctypes.c_int,
+                                                                  ctypes.c_int, ctypes.c_double, ctypes.c_long,
+                                                                  lp, dp, dp]
+        lib.oracle_attn_rows_topk.restype = ctypes.c_int
         lib.oracle_decode_step.argtypes = [ctypes.c_int] * 4 + [ip, dp, dp, dp, dp, ip, ip, up,
                                                                 ctypes.c_double, dp, dp, dp, dp, dp, dp]
         lib.oracle_decode_step.restype = ctypes.c_int
@@ -100,6 +104,26 @@ def attn_rows(q, kt, vt, dil, win, rows, parts=3, scale=None, grid=False, dedupe
                                  int(bool(grid)), int(bool(dedupe)))
     if rc != 0:
         raise ValueError("oracle_attn_rows: invalid arguments")
+    return o, lse
+
+
+def attn_rows_topk(q, kt, vt, block, K, mode, rows, scale=None):
+    """Rows (b, h, t) of top-k block attention (mode "quest": per-channel
+    min/max block statistics; "moba": mean-pooled block keys); returns
+    (o [n,d], lse [n])."""
+    lib = _load()
+    q, kt, vt = _f64(q), _f64(kt), _f64(vt)
+    B, T, H, d = q.shape
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+    n = rows.shape[0]
+    o = np.empty((n, d), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    s = default_scale(d) if scale is None else float(scale)
+    m = {"quest": 0, "moba": 1}[mode]
+    rc = lib.oracle_attn_rows_topk(B, T, H, d, _dp(q), _dp(kt), _dp(vt), int(block), int(K), m, s, n,
+                                   rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), _dp(o), _dp(lse))
+    if rc != 0:
+        raise ValueError("oracle_attn_rows_topk: invalid arguments")
     return o, lse
 
 

@@ -40,6 +40,11 @@
  *   R8 (a variant, off by default) dedupe: a key in both parts counts once,
  *      i.e. the window part skips the keys of the dilated set
  *      (oracle_attn_rows_ex).
+ *   R9 top-k block attention (oracle_attn_rows_topk): blocks of bs keys; the
+ *      first and the query's own block are always kept, K more are chosen by
+ *      score; the Quest-style score is the per-channel min/max upper bound
+ *      sum_c max(q_c*kmin_c, q_c*kmax_c), the MoBA-style score q . mean(k);
+ *      ties go to the lower block index; blocks hold the augmented keys.
  *
  * Parity pins for every function here live in tests/test_oracle_pins.py.
  */
@@ -245,6 +250,93 @@ int oracle_attn_rows_ex(int B, int T, int H, int d, const double *q, const doubl
 {
     return attn_rows_impl(B, T, H, d, q, kt, vt, dil, win, scale, parts, nrows, rows, o, lse,
                           grid != 0, dedupe != 0);
+}
+
+/*
+ * Top-k block attention over the augmented keys/values, the sparse-inference
+ * setting the pages evaluate on RAT+ ([RAT+] Figure 3 and Tables 17-18;
+ * [MEM] "Sparse inference settings").  Keys are grouped into blocks of `bs`
+ * consecutive positions.  Query t (in block c = floor(t / bs)) attends, over
+ * j <= t, to the keys of
+ *   - block 0 and block c (the first and the local block are always kept),
+ *   - the K highest-scoring of blocks 1 .. c-1 (all of them when there are at
+ *     most K; equal scores go to the lower block index).
+ * A block's score against q_t:
+ *   mode 0 (Quest-style, per-channel min/max statistics of the block's keys):
+ *          sum_c max(q_c * kmin_c, q_c * kmax_c), an upper bound of q.k over
+ *          any key inside the block's per-channel ranges;
+ *   mode 1 (MoBA-style, mean-pooled keys): q . mean_j(k_j).
+ * Reading R9 (the pages name the methods and their statistics but print no
+ * formula): the Quest score is that upper bound; K counts the blocks chosen
+ * besides the first and the local one; the blocks hold the augmented keys.
+ * Output and log-sum-exp are those of one softmax over the attended keys
+ * (scale as in R5).  Returns 0, or -1 on an argument error.
+ */
+int oracle_attn_rows_topk(int B, int T, int H, int d, const double *q, const double *kt,
+                          const double *vt, int bs, int K, int mode, double scale, long nrows,
+                          const int64_t *rows, double *o, double *lse)
+{
+    if (bs < 1 || K < 0 || (mode != 0 && mode != 1)) return -1;
+    for (long r = 0; r < nrows; ++r) {
+        int64_t b = rows[3 * r], h = rows[3 * r + 1], t = rows[3 * r + 2];
+        if (b < 0 || b >= B || h < 0 || h >= H || t < 0 || t >= T) return -1;
+    }
+    const long nblk = (T + bs - 1) / bs;
+    int err = 0;
+#pragma omp parallel
+    {
+        long *js = (long *)malloc(sizeof(long) * (size_t)(T > 0 ? T : 1));
+        double *z = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+        double *score = (double *)malloc(sizeof(double) * (size_t)nblk);
+        unsigned char *keep = (unsigned char *)malloc((size_t)nblk);
+        if (!js || !z || !score || !keep) {
+#pragma omp atomic write
+            err = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (long r = 0; r < nrows; ++r) {
+            if (err) continue;
+            int b = (int)rows[3 * r], h = (int)rows[3 * r + 1];
+            long t = (long)rows[3 * r + 2];
+            const double *qrow = q + idx4(T, H, d, b, t, h, 0);
+            const long c = t / bs;
+            for (long blk = 0; blk <= c; ++blk) keep[blk] = (blk == 0 || blk == c);
+            /* scores of the candidate blocks 1 .. c-1 (whole blocks, all j < c*bs <= t) */
+            for (long blk = 1; blk < c; ++blk) {
+                double sc = 0.0;
+                for (int ch = 0; ch < d; ++ch) {
+                    double lo = INFINITY, hi = -INFINITY, sum = 0.0;
+                    for (long j = blk * bs; j < (blk + 1) * bs; ++j) {
+                        const double x = kt[idx4(T, H, d, b, j, h, ch)];
+                        if (x < lo) lo = x;
+                        if (x > hi) hi = x;
+                        sum += x;
+                    }
+                    if (mode == 0) {
+                        const double a1 = qrow[ch] * lo, a2 = qrow[ch] * hi;
+                        sc += a1 > a2 ? a1 : a2;
+                    } else {
+                        sc += qrow[ch] * (sum / (double)bs);
+                    }
+                }
+                score[blk] = sc;
+            }
+            /* the K best candidates, ties to the lower index */
+            for (int pick = 0; pick < K; ++pick) {
+                long best = -1;
+                for (long blk = 1; blk < c; ++blk)
+                    if (!keep[blk] && (best < 0 || score[blk] > score[best])) best = blk;
+                if (best < 0) break;
+                keep[best] = 1;
+            }
+            long n = 0;
+            for (long j = 0; j <= t; ++j)
+                if (keep[j / bs]) js[n++] = j;
+            softmax_over(T, H, d, qrow, kt, vt, b, h, js, n, scale, o + (size_t)r * (size_t)d, &lse[r], z);
+        }
+        free(js); free(z); free(score); free(keep);
+    }
+    return err ? -1 : 0;
 }
 
 /*

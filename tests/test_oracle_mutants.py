@@ -4,7 +4,9 @@ Each mutant is rat_oracle.c with one textual change (a swapped gate, a wrong
 sign, a dropped term, a wrong dilation residue, a window off by one, a wrong
 merge, a dropped scale, a transposed operand, a gate one step late, a decode
 that ignores the per-head recurrence flag, a fixed grid on the wrong residue
-or without the query's own key, a dedupe that keeps the shared keys).  It is compiled into a temporary
+or without the query's own key, a dedupe that keeps the shared keys,
+a top-k block selection with a one-sided bound, a dropped first or local
+block, ties to the wrong block or one block too many).  It is compiled into a temporary
 directory and the pin suite is run against it in a subprocess; the suite must
 fail.  The shipped oracle is never modified.
 """
@@ -36,6 +38,11 @@ MUTANTS = {
     "grid_on_residue_zero": ("if (j % D == D - 1 || j == t) js[n++] = j;", "if (j % D == 0 || j == t) js[n++] = j;"),
     "grid_without_self": ("if (j % D == D - 1 || j == t) js[n++] = j;", "if (j % D == D - 1) js[n++] = j;"),
     "dedupe_ignored": ("if (!in_dil) js[n2++] = j;", "js[n2++] = j;"),
+    "topk_quest_upper_end_only": ("sc += a1 > a2 ? a1 : a2;", "sc += a2;"),
+    "topk_local_block_dropped": ("keep[blk] = (blk == 0 || blk == c);", "keep[blk] = (blk == 0);"),
+    "topk_first_block_dropped": ("keep[blk] = (blk == 0 || blk == c);", "keep[blk] = (blk == c);"),
+    "topk_ties_to_higher_block": ("(best < 0 || score[blk] > score[best])", "(best < 0 || score[blk] >= score[best])"),
+    "topk_one_block_too_many": ("for (int pick = 0; pick < K; ++pick)", "for (int pick = 0; pick <= K; ++pick)"),
 }
 
 

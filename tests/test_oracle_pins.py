@@ -352,6 +352,107 @@ def test_dedupe_without_window_changes_nothing():
         np.testing.assert_array_equal(x, y)
 
 
+# --------------------------------------------------------------------------- top-k blocks
+
+
+def topk_rows(T, H=1, B=1):
+    return [(b, h, t) for b in range(B) for h in range(H) for t in range(T)]
+
+
+def masked_rows(q, k, v, keysets, scale):
+    """Softmax attention of row t of q over the explicit key set keysets[t]."""
+    out, lses = [], []
+    for t, keys in enumerate(keysets):
+        keys = sorted(keys)
+        z = torch.from_numpy(scale * k[keys] @ q[t])
+        out.append(torch.softmax(z, dim=0).numpy() @ v[keys])
+        lses.append(torch.logsumexp(z, 0).item())
+    return np.array(out), np.array(lses)
+
+
+@pytest.mark.parametrize("mode", ["quest", "moba"])
+@pytest.mark.parametrize("T,bs", [(29, 4), (16, 16), (7, 3)])
+def test_topk_with_every_block_kept_is_dense_causal(mode, T, bs):
+    B, H, d = 1, 2, 5
+    q, k, v = rand_qkv(B, T, H, d)
+    rows = topk_rows(T, H)
+    o, lse = oracle.attn_rows_topk(q, k, v, bs, T, mode, rows)
+    for h in range(H):
+        ref = sdpa_causal(q[0, :, h], k[0, :, h], v[0, :, h], 1 / math.sqrt(d))
+        np.testing.assert_allclose(o[h * T:(h + 1) * T], ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", ["quest", "moba"])
+def test_topk_with_k_0_keeps_first_and_local_block(mode):
+    B, T, H, d, bs = 1, 23, 1, 4, 5
+    q, k, v = rand_qkv(B, T, H, d)
+    o, lse = oracle.attn_rows_topk(q, k, v, bs, 0, mode, topk_rows(T), scale=0.7)
+    sets = [[j for j in range(t + 1) if j < bs or j >= (t // bs) * bs] for t in range(T)]
+    ro, rl = masked_rows(q[0, :, 0], k[0, :, 0], v[0, :, 0], sets, 0.7)
+    np.testing.assert_allclose(o, ro, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse, rl, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", ["quest", "moba"])
+@pytest.mark.parametrize("K", [1, 3])
+def test_topk_with_blocks_of_one_key_is_top_k_keys(mode, K):
+    # a one-key block has kmin = kmax = mean = k, so both scores are q.k and the
+    # selection is the K largest dot products among keys 1 .. t-1
+    B, T, H, d = 1, 19, 1, 6
+    q, k, v = rand_qkv(B, T, H, d)
+    o, lse = oracle.attn_rows_topk(q, k, v, 1, K, mode, topk_rows(T))
+    qq, kk = q[0, :, 0], k[0, :, 0]
+    sets = []
+    for t in range(T):
+        cand = list(range(1, t))
+        best = sorted(cand, key=lambda j: -float(kk[j] @ qq[t]))[:K]
+        sets.append(set([0, t] + best))
+    ro, rl = masked_rows(qq, kk, v[0, :, 0], sets, 1 / math.sqrt(d))
+    np.testing.assert_allclose(o, ro, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse, rl, rtol=1e-12, atol=1e-12)
+
+
+def test_topk_quest_and_moba_worked_example():
+    # blocks of 2 over T = 8 (blocks 0..3); rows 6 and 7 sit in block 3, one
+    # candidate (K = 1) among blocks 1 and 2, d = 2:
+    #   block 1 keys (-3, 0), (5, 0): mean (1, 0);   block 2 keys (-2, 1) twice
+    #   row 7, q = (-1, 0.5): Quest bound  block1 = 3 + 0 = 3,  block2 = 2 + 0.5 = 2.5 -> block 1
+    #                        MoBA mean     block1 = -1,        block2 = 2.5        -> block 2
+    #   row 6, q = (1, 0):    Quest bound  block1 = 5,          block2 = -2         -> block 1
+    #                        MoBA mean     block1 = 1,          block2 = -2         -> block 1
+    k = np.zeros((1, 8, 1, 2))
+    k[0, :, 0] = [[0.3, -0.2], [0.1, 0.4], [-3, 0], [5, 0], [-2, 1], [-2, 1], [0.2, 0.2], [-0.1, 0.3]]
+    q = np.zeros((1, 8, 1, 2))
+    q[0, 6, 0] = [1, 0]
+    q[0, 7, 0] = [-1, 0.5]
+    v = rng.standard_normal((1, 8, 1, 2))
+    rows = [(0, 0, 6), (0, 0, 7)]
+    expect = {"quest": [{0, 1, 2, 3, 6}, {0, 1, 2, 3, 6, 7}],
+              "moba": [{0, 1, 2, 3, 6}, {0, 1, 4, 5, 6, 7}]}
+    for mode, sets in expect.items():
+        o, lse = oracle.attn_rows_topk(q, k, v, 2, 1, mode, rows, scale=0.5)
+        ro, rl = masked_rows(q[0, 6:, 0], k[0, :, 0], v[0, :, 0], sets, 0.5)
+        np.testing.assert_allclose(o, ro, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(lse, rl, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", ["quest", "moba"])
+def test_topk_equal_scores_go_to_the_lower_block(mode):
+    B, T, H, d, bs = 1, 12, 1, 3, 3
+    q, k, v = rand_qkv(B, T, H, d)
+    k[0, 6:9] = k[0, 3:6]          # blocks 1 and 2 hold the same keys
+    o, _ = oracle.attn_rows_topk(q, k, v, bs, 1, mode, [(0, 0, 11)])
+    ro, _ = masked_rows(q[0, 11:, 0], k[0, :, 0], v[0, :, 0], [{0, 1, 2, 3, 4, 5, 9, 10, 11}], 1 / math.sqrt(d))
+    np.testing.assert_allclose(o, ro, rtol=1e-12, atol=1e-12)
+
+
+def test_topk_invalid_arguments_are_rejected():
+    q, k, v = rand_qkv(1, 4, 1, 2)
+    for bs, K, rows in [(0, 1, [(0, 0, 1)]), (2, -1, [(0, 0, 1)]), (2, 1, [(0, 0, 4)])]:
+        with pytest.raises(ValueError):
+            oracle.attn_rows_topk(q, k, v, bs, K, "quest", rows)
+
+
 # --------------------------------------------------------------------------- decode
 
 
