@@ -23,7 +23,11 @@
  *                and x = v, with a_t = sigmoid(g_t) from one gate tensor g;
  *                s_{-1} = init (zero when not given).  A head with recur = 0
  *                has a = 0: its augmented keys/values are the raw ones.
- *   dilation     query t attends to { j <= t : (t - j) mod D == 0 }.
+ *   dilation     query t attends to { j <= t : (t - j) mod D == 0 }.  With
+ *                RAT_FLAG_GRID_DILATION it attends instead to the fixed grid
+ *                { j <= t : j mod D == D - 1 } plus itself (j = t, once): the
+ *                chunk-end keys of the RAT page's Approach (chunk size D),
+ *                which a decode can keep in a cache D times smaller.
  *   window       W > 0 adds a second softmax over { max(0, t-W+1) <= j <= t }.
  *   merge        the two softmaxes are merged by log-sum-exp (a key in both
  *                sets counts in both).
@@ -109,7 +113,12 @@ typedef struct {
     const int32_t *win;      /* host [H] */
     const uint8_t *recur;    /* host [H] or NULL */
     float scale;             /* <= 0 selects 1/sqrt(d) */
+    uint32_t flags;          /* RAT_FLAG_* bits, 0 = the defaults above */
 } rat_cfg;
+
+/* Fixed-grid reading of dilation (see "dilation" above) for every head of the
+ * call, and the matching decode-cache layout (see rat_cache_rows). */
+#define RAT_FLAG_GRID_DILATION 1u
 
 /* Bytes of workspace `op` needs for `cfg` (cache_cap: decode capacity, else
  * ignored).  Returns 0 when cfg is invalid. */
@@ -125,6 +134,11 @@ RAT_API rat_status rat_workspace_init(void *ws, size_t ws_bytes, rat_stream_t st
  *     (j mod D_h) * ceil(cap / D_h) + floor(j / D_h)
  * i.e. residue-major: the rows a decode query at position t reads for its
  * dilated part (all j == t mod D_h, j <= t) form one contiguous slab.
+ * With RAT_FLAG_GRID_DILATION a head keeps only its grid: position j with
+ * j mod D_h == D_h - 1 at row floor(j / D_h), rows [0, ceil(cap / D_h)).  A
+ * head with D_h > 1 and a window W_h > 0 also keeps a ring of its last W_h
+ * positions after the grid: position j at row ceil(cap / D_h) + (j mod W_h).
+ * R is the largest head's row count in either layout.
  * Returns 0 when cfg or cap is invalid.
  */
 RAT_API int64_t rat_cache_rows(const rat_cfg *cfg, int cap);
@@ -138,7 +152,9 @@ RAT_API int64_t rat_cache_rows(const rat_cfg *cfg, int cap);
  *                        is given (recur = 0 heads receive a copy of k / v)
  *   final_k, final_v out [B,H,d] fp32 s_{T-1}, or NULL
  *   cache_k, cache_v out decode cache tensors (layout above) for positions
- *                        0..T-1, or NULL; requires T <= cache_cap
+ *                        0..T-1 (under the fixed grid: the grid rows, and
+ *                        the ring rows of positions T-W_h .. T-1), or NULL;
+ *                        requires T <= cache_cap
  * At least one of (kt, vt) or (cache_k, cache_v) must be given, as pairs.
  */
 RAT_API rat_status rat_scan_prefill(const rat_cfg *cfg, const void *k, const void *v, const void *g,
@@ -178,12 +194,15 @@ RAT_API rat_status rat_mix_prefill(const rat_cfg *cfg, const void *q, const void
  *   1. s <- a*s + (1-a)*x for x = k and v (a = sigmoid(g), a = 0 if recur = 0),
  *      updating state_k / state_v in place (fp32 [B,H,d]);
  *   2. the new augmented key/value (rounded to cfg->dtype) is stored at t's
- *      cache row;
+ *      cache row (under the fixed grid: at its grid row when t is on the
+ *      grid, and at its ring row when the head keeps a ring);
  *   3. o[b,h] = merged attention of q over the cache rows j <= t of the
  *      dilated set (and window) of t.
  *   q, k, v, g   in  [B,H,d]
  *   cache_k/v    in/out [B,H,R,d], R = rat_cache_rows(cfg, cache_cap); rows of
  *                positions < pos[b] must hold earlier augmented keys/values
+ *                (under the fixed grid: the grid rows below t and the ring
+ *                rows of t-W_h+1 .. t-1)
  *   pos          in  DEVICE int32 [B], 0 <= pos[b] < cache_cap (a position out
  *                of range makes the kernel skip that entry and record
  *                RAT_ERR_INVALID for rat_check_status)

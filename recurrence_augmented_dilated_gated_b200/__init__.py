@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(HERE, "librat.so")
 RAT_OK, RAT_ERR_INVALID, RAT_ERR_UNSUPPORTED, RAT_ERR_CUDA, RAT_ERR_TIMEOUT, RAT_ERR_WORKSPACE = range(6)
 RAT_F32, RAT_BF16 = 0, 1
 RAT_OP_SCAN, RAT_OP_ATTN, RAT_OP_MIX, RAT_OP_MIX_CALLER_KV, RAT_OP_DECODE = range(5)
+RAT_FLAG_GRID_DILATION = 1
 
 EXPORTS = ["rat_workspace_size", "rat_workspace_init", "rat_cache_rows", "rat_scan_prefill",
            "rat_dilated_attn_prefill", "rat_mix_prefill", "rat_decode_step", "rat_check_status",
@@ -42,7 +43,7 @@ class rat_cfg(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("dil", ctypes.POINTER(ctypes.c_int32)),
                 ("win", ctypes.POINTER(ctypes.c_int32)), ("recur", ctypes.POINTER(ctypes.c_uint8)),
-                ("scale", ctypes.c_float)]
+                ("scale", ctypes.c_float), ("flags", ctypes.c_uint32)]
 
 
 _lib = None
@@ -86,7 +87,7 @@ def load_library(path=LIB_PATH):
 class Config:
     """Owns a rat_cfg and the host arrays it points to."""
 
-    def __init__(self, B, T, H, d, dtype, dil, win, recur=None, scale=0.0):
+    def __init__(self, B, T, H, d, dtype, dil, win, recur=None, scale=0.0, flags=0):
         self.dil = np.ascontiguousarray(dil, dtype=np.int32)
         self.win = np.ascontiguousarray(win, dtype=np.int32)
         self.recur = None if recur is None else np.ascontiguousarray(recur, dtype=np.uint8)
@@ -97,7 +98,7 @@ class Config:
                          self.dil.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
                          self.win.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
                          None if self.recur is None else self.recur.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
-                         float(scale))
+                         float(scale), int(flags))
 
     @property
     def torch_dtype(self):
@@ -105,7 +106,7 @@ class Config:
 
     def replace(self, **kw):
         args = dict(B=self.c.B, T=self.c.T, H=self.c.H, d=self.c.d, dtype=self.c.dtype, dil=self.dil,
-                    win=self.win, recur=self.recur, scale=self.c.scale)
+                    win=self.win, recur=self.recur, scale=self.c.scale, flags=self.c.flags)
         args.update(kw)
         return Config(**args)
 

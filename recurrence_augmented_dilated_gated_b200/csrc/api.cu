@@ -73,18 +73,24 @@ rat_status check_cfg(const rat_cfg *c, bool need_T = true) {
     const double elems = (double)c->B * (need_T ? (double)c->T : 1.0) * c->H * c->d;
     if (elems >= 1099511627776.0) return fail(RAT_ERR_INVALID, "B*T*H*d too large");
     if (!(c->scale == c->scale)) return fail(RAT_ERR_INVALID, "scale is NaN");
+    if (c->flags & ~RAT_FLAG_GRID_DILATION) return fail(RAT_ERR_INVALID, "unknown flags 0x%x", c->flags);
     return RAT_OK;
 }
 
 bool head_recur(const rat_cfg *c, int h) { return c->recur == nullptr || c->recur[h] != 0; }
 
+bool grid_mode(const rat_cfg *c) { return (c->flags & RAT_FLAG_GRID_DILATION) != 0; }
+
 float scale_of(const rat_cfg *c) { return c->scale > 0.f ? c->scale : 1.0f / sqrtf((float)c->d); }
 
+// Rows of one (b, h) block of the decode cache: residue-major, all positions;
+// or, under the fixed grid, the grid rows plus the window ring (D > 1, W > 0).
 int64_t cache_rows(const rat_cfg *c, int cap) {
     int64_t R = 0;
     for (int h = 0; h < c->H; ++h) {
-        const int64_t D = c->dil[h];
-        R = std::max<int64_t>(R, D * ((cap + D - 1) / D));
+        const int64_t D = c->dil[h], S = (cap + D - 1) / D;
+        const int64_t rows = grid_mode(c) ? S + (D > 1 ? (int64_t)c->win[h] : 0) : D * S;
+        R = std::max<int64_t>(R, rows);
     }
     return R;
 }
@@ -181,12 +187,14 @@ rat_status run_scan(const rat_cfg *c, const Layout &L, const void *k, const void
     p.cache[0] = ck; p.cache[1] = cv;
     p.cap = cap;
     p.cache_R = ck ? cache_rows(c, cap) : 0;
+    p.grid = grid_mode(c) ? 1 : 0;
     p.B = c->B; p.T = c->T; p.H = c->H; p.d = c->d;
     int n = 0, n_plain = 0;
     unsigned char plain[kMaxHeads];
     for (int h = 0; h < c->H; ++h) {
         p.head_recur[h] = head_recur(c, h) ? 1 : 0;
         p.head_dil[h] = c->dil[h];
+        p.head_win[h] = c->win[h];
         if (!only_recurrent || p.head_recur[h]) p.head_list[n++] = (unsigned char)h;
         else plain[n_plain++] = (unsigned char)h;
     }
@@ -221,14 +229,18 @@ rat_status run_scan(const rat_cfg *c, const Layout &L, const void *k, const void
     return RAT_OK;
 }
 
+// Kind of a head's dilated part on the tensor cores: the residue subsequences,
+// or (fixed grid, D > 1) every position against the grid subsequence.
+bool grid_head(const rat_cfg *c, int h) { return grid_mode(c) && c->dil[h] > 1; }
+
 // A head runs on the tensor-core kernel when its operands are bf16 and its
 // dilation divides T (the strided TMA view needs whole subsequences);
 // otherwise the fp32 CUDA-core kernel computes it.
 bool tc_head(const rat_cfg *c, int h) { return c->dtype == RAT_BF16 && c->T % c->dil[h] == 0; }
 
-// One tensor-core launch over `heads` (dilated part, or window part when
-// window_mode), grouped into classes of equal (dilation, K/V source).
-rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, bool window_mode, const void *q,
+// One tensor-core launch over `heads` (kind kTcDilated, kTcWindow or kTcGrid),
+// grouped into classes of equal (dilation, K/V source).
+rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, int kind, const void *q,
                           const void *kt, const void *vt, const void *kraw, const void *vraw,
                           const bool *raw_head, void *o, float *lse, float *lse_dil, char *ws, unsigned *tickets,
                           int *n_launch, cudaStream_t s) {
@@ -239,7 +251,8 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, bool w
         TcParams P;
         memset(&P, 0, sizeof(P));
         P.B = c->B; P.T = c->T; P.H = c->H;
-        P.window_mode = window_mode ? 1 : 0;
+        P.kind = kind;
+        P.q = q;
         P.scale_log2 = scale_of(c) * 1.4426950408889634f;
         P.o = o; P.lse_user = lse; P.lse_dil = lse_dil;
         P.hdr = reinterpret_cast<WsHeader *>(ws);
@@ -254,7 +267,7 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, bool w
         for (int i = 0; i < nheads; ++i) {
             const int h = heads[i];
             if (taken[i]) continue;
-            const Key k{window_mode ? 1 : c->dil[h], raw_head[h] ? 1 : 0};
+            const Key k{kind == kTcWindow ? 1 : c->dil[h], raw_head[h] ? 1 : 0};
             int ci = -1;
             for (int j = 0; j < ncls; ++j)
                 if (keys[j].D == k.D && keys[j].raw == k.raw) ci = j;
@@ -277,16 +290,21 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, bool w
             const int ci = order[oi];
             TcClass &C = P.cls[oi];
             C.D = keys[ci].D;
-            C.n = c->T / C.D;
+            // query rows per group: a residue subsequence, or every position
+            C.n = kind == kTcDilated ? c->T / C.D : c->T;
+            C.nres = kind == kTcDilated ? C.D : 1;
+            C.kres = kind == kTcGrid ? C.D - 1 : 0;   // the grid is residue D-1
             C.mtiles = (C.n + 255) / 256;   // 256-row units per (b, h, residue) group
             C.nheads = cls_n[ci];
             C.head0 = nh;
             for (int j = 0; j < cls_n[ci]; ++j) P.heads[nh++] = (unsigned char)cls_heads[ci][j];
             P.prefix[oi] = pref;
-            pref += (long long)c->B * C.nheads * C.D * C.mtiles;
+            pref += (long long)c->B * C.nheads * C.nres * C.mtiles;
             const void *kb = keys[ci].raw ? kraw : kt;
             const void *vb = keys[ci].raw ? vraw : vt;
-            if (!encode_map_5d(&P.tq[oi], q, c->B, c->T, c->H, c->d, C.D, kTcRowsQ) ||
+            P.kself[oi] = kb;
+            P.vself[oi] = vb;
+            if (!encode_map_5d(&P.tq[oi], q, c->B, c->T, c->H, c->d, kind == kTcGrid ? 1 : C.D, kTcRowsQ) ||
                 !encode_map_5d(&P.tk[oi], kb, c->B, c->T, c->H, c->d, C.D, kTcRowsKV) ||
                 !encode_map_5d(&P.tv[oi], vb, c->B, c->T, c->H, c->d, C.D, kTcRowsKV))
                 return fail(RAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (dilation %d)", C.D);
@@ -303,30 +321,37 @@ rat_status run_attn(const rat_cfg *c, const Layout &L, const void *q, const void
                     const void *kraw, const void *vraw, bool raw_for_plain_heads, void *o, float *lse,
                     char *ws, cudaStream_t s) {
     bool raw_head[kMaxHeads];
-    int tc_all[kMaxHeads], tc_win[kMaxHeads];
-    int n_tc = 0, n_win = 0, n_simt = 0;
+    int tc_all[kMaxHeads], tc_grid[kMaxHeads], tc_win[kMaxHeads];
+    int n_tc = 0, n_grid = 0, n_win = 0, n_simt = 0;
     for (int h = 0; h < c->H; ++h) {
         raw_head[h] = raw_for_plain_heads && !head_recur(c, h);
         if (tc_head(c, h)) {
-            tc_all[n_tc++] = h;
+            if (grid_head(c, h)) tc_grid[n_grid++] = h;
+            else tc_all[n_tc++] = h;
             if (c->win[h] > 0) tc_win[n_win++] = h;
         } else {
             ++n_simt;
         }
     }
     float *lse_dil = reinterpret_cast<float *>(ws + L.lse_dil);
-    if (n_tc > 0) {
+    if (n_tc + n_grid > 0) {
         unsigned *tickets = reinterpret_cast<unsigned *>(ws + L.att_ticket);
         int n_launch = 0;
         cudaError_t e = cudaMemsetAsync(tickets, 0, kAttnTickets * sizeof(unsigned), s);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(attention tickets)");
         // The sort in launch_tc_part orders classes by dilation; with T fixed,
         // a smaller dilation means longer subsequences, i.e. more query tiles.
-        rat_status st = launch_tc_part(c, tc_all, n_tc, false, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws,
-                                       tickets, &n_launch, s);
+        rat_status st = RAT_OK;
+        if (n_tc > 0)
+            st = launch_tc_part(c, tc_all, n_tc, kTcDilated, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws,
+                                tickets, &n_launch, s);
+        if (st != RAT_OK) return st;
+        if (n_grid > 0)
+            st = launch_tc_part(c, tc_grid, n_grid, kTcGrid, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws,
+                                tickets, &n_launch, s);
         if (st != RAT_OK) return st;
         if (n_win > 0) {
-            st = launch_tc_part(c, tc_win, n_win, true, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws,
+            st = launch_tc_part(c, tc_win, n_win, kTcWindow, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws,
                                 tickets, &n_launch, s);
             if (st != RAT_OK) return st;
         }
@@ -338,6 +363,7 @@ rat_status run_attn(const rat_cfg *c, const Layout &L, const void *q, const void
         p.o = o; p.lse = lse;
         p.B = c->B; p.T = c->T; p.H = c->H; p.d = c->d;
         p.scale_log2 = scale_of(c) * 1.4426950408889634f;
+        p.grid = grid_mode(c) ? 1 : 0;
         for (int h = 0; h < c->H; ++h) {
             p.dil[h] = c->dil[h];
             p.win[h] = c->win[h];
@@ -355,7 +381,7 @@ rat_status run_attn(const rat_cfg *c, const Layout &L, const void *q, const void
 
 extern "C" {
 
-int rat_version(void) { return 100; }
+int rat_version(void) { return 101; }
 
 long long rat_launch_count(void) { return rat::g_launches.load(std::memory_order_relaxed); }
 

@@ -3,7 +3,8 @@
 // "RAT+: Train Dense, Infer Sparse", Abstract and Figure 1(c): query t attends
 // to the dilated set { j <= t : (t-j) mod D == 0 } and, when the head has a
 // window W > 0, in a second softmax to { max(0, t-W+1) <= j <= t }; the two
-// softmaxes are merged by log-sum-exp.
+// softmaxes are merged by log-sum-exp.  Under the fixed-grid reading the
+// dilated set is { j <= t : j mod D == D-1 } plus t itself (once).
 //
 // One warp owns one query row: each lane holds d/32 channels of q and of the
 // running output, the score of every key is a warp-wide dot product, and the
@@ -82,7 +83,14 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(const AttnParams
     const int D = p.dil[h], W = p.win[h];
     RowState<CPL> dil, wnd;
     dil.init();
-    attend<T, CPL>(dil, q, kb, vb, rs, t % D, t, D, lane);
+    if (p.grid && D > 1) {
+        // the grid keys up to t, then t itself unless it is on the grid
+        const long long g_hi = (t + 1) / D * D - 1;
+        attend<T, CPL>(dil, q, kb, vb, rs, D - 1, g_hi, D, lane);
+        if (t % D != D - 1) attend<T, CPL>(dil, q, kb, vb, rs, t, t, 1, lane);
+    } else {
+        attend<T, CPL>(dil, q, kb, vb, rs, t % D, t, D, lane);
+    }
     float m = dil.m, l = dil.l;
     float acc[CPL];
 #pragma unroll

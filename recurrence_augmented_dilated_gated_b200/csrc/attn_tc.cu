@@ -28,6 +28,12 @@
 // and lse; heads with one write o (bf16) and lse into scratch.  Launch 2
 // (window part): 256 consecutive positions against the key tiles covering
 // [t0-W+1, t0+255]; the epilogue merges with launch 1's (o, lse) by LSE.
+// Under the fixed-grid reading of dilation (query t attends to the keys
+// j <= t with j mod D == D-1, plus its own key) the dilated launch is replaced
+// by a grid launch: units are 256 consecutive positions against the key tiles
+// of the residue-(D-1) subsequence up to the last row's grid key, masked per
+// row; the epilogue adds the row's own key (when it is off the grid) by LSE,
+// scoring it from q and K~ in global memory.
 //
 // Every mbarrier wait is bounded (globaltimer); on expiry the CTA records
 // RAT_ERR_TIMEOUT, raises a shared abort flag, waits (bounded) for its own
@@ -194,8 +200,8 @@ __device__ __forceinline__ Unit decode_unit(const TcParams &p, long long u) {
     Unit out;
     out.cls = c;
     out.m = C.mtiles - 1 - (int)(rem % C.mtiles);
-    out.r = (int)(g % C.D);
-    g /= C.D;
+    out.r = (int)(g % C.nres);
+    g /= C.nres;
     out.h = p.heads[C.head0 + (int)(g % C.nheads)];
     out.b = (int)(g / C.nheads);
     return out;
@@ -209,15 +215,25 @@ struct Plan {
     bool valid[kSub];
 };
 
-__device__ __forceinline__ Plan make_plan(const TcParams &p, const Unit &u, int n) {
+template <int kKind>
+__device__ __forceinline__ Plan make_plan(const TcParams &p, const Unit &u) {
     Plan pl;
+    const TcClass &C = p.cls[u.cls];
+    const int n = C.n;
     const int q0 = 2 * BM * u.m;
     const int W = p.win[u.h];
     for (int i = 0; i < kSub; ++i) {
         const int qmin = q0 + BM * i;
         pl.valid[i] = qmin < n;
-        pl.hi[i] = qmin / BN;
-        if (!p.window_mode) {
+        if (kKind == kTcGrid) {
+            // grid keys g <= (t+1)/D - 1 for the sub-tile's last row t; a tile
+            // whose rows have no grid key yet keeps tile 0, fully masked
+            const int qlast = min(qmin + BM - 1, n - 1);
+            pl.hi[i] = max(0, ((qlast + 1) / C.D - 1) / BN);
+        } else {
+            pl.hi[i] = qmin / BN;
+        }
+        if (kKind != kTcWindow) {
             pl.lo[i] = 0;
         } else {
             const int first = qmin - W + 1;  // earliest key of the sub-tile's first row
@@ -348,9 +364,11 @@ struct Smem {
 // for that warpgroup's next P, which it writes only after its epilogue has
 // read O_i (ordered by the tcgen05 fences around bar_pfull).  Unit tickets
 // reach the other roles through a 2-slot ring in shared memory.
-template <int HD, bool kWin>
+template <int HD, int kKind>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
     using L = Smem<HD>;
+    constexpr bool kWin = kKind == kTcWindow;
+    constexpr bool kGrid = kKind == kTcGrid;
     constexpr int NCB = HD / 64;  // 64-column (128-byte) blocks of a head row
     extern __shared__ uint8_t dsmem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
@@ -411,11 +429,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 mbar_arrive(&bar_ufull[slot]);
                 if (un >= p.total_units) break;
                 const Unit u = decode_unit(p, un);
-                const Plan pl = make_plan(p, u, p.cls[u.cls].n);
+                const Plan pl = make_plan<kKind>(p, u);
                 const int ntiles = pl.jhi - pl.jlo + 1;
                 const CUtensorMap *mq = &p.tq[u.cls];
                 const CUtensorMap *mk = &p.tk[u.cls];
                 const CUtensorMap *mv = &p.tv[u.cls];
+                const int rk = u.r + p.cls[u.cls].kres;   // K/V residue coordinate
                 // Q of the previous unit has been read by its last QK
                 if (it >= 1 && !(ok = mbar_wait(&bar_qempty, (uint32_t)(it - 1) & 1u, &s_abort))) break;
                 const int nq = pl.valid[1] ? 2 : 1;
@@ -433,13 +452,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     mbar_expect_tx(&bar_kfull[st], L::kTile);
                     for (int cb = 0; cb < NCB; ++cb)
                         tma_load_5d(sbase + L::kK + st * L::kTile + cb * BN * 128, mk, &bar_kfull[st], cb * 64,
-                                    u.h, u.r, krow, u.b);
+                                    u.h, rk, krow, u.b);
                     ++nk;
                     if (nv >= 2 && !(ok = mbar_wait(&bar_vempty[st], ph ^ 1u, &s_abort))) break;
                     mbar_expect_tx(&bar_vfull[st], L::kTile);
                     for (int cb = 0; cb < NCB; ++cb)
                         tma_load_5d(sbase + L::kV + st * L::kTile + cb * BN * 128, mv, &bar_vfull[st], cb * 64,
-                                    u.h, u.r, krow, u.b);
+                                    u.h, rk, krow, u.b);
                     ++nv;
                 }
             }
@@ -498,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 mbar_arrive(&bar_uempty[slot]);
                 if (un >= p.total_units) break;
                 const Unit u = decode_unit(p, un);
-                const Plan pl = make_plan(p, u, p.cls[u.cls].n);
+                const Plan pl = make_plan<kKind>(p, u);
                 const int ntiles = pl.jhi - pl.jlo + 1;
                 ok = mbar_wait(&bar_q, (uint32_t)it & 1u, &s_abort);
                 if (ok) ok = mbar_wait(&bar_kfull[kv & 1], (uint32_t)(kv >> 1) & 1u, &s_abort);
@@ -577,7 +596,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (un >= p.total_units) break;
             const Unit u = decode_unit(p, un);
             const TcClass &C = p.cls[u.cls];
-            const Plan pl = make_plan(p, u, C.n);
+            const Plan pl = make_plan<kKind>(p, u);
             const int qmin = 2 * BM * u.m + BM * sub;                 // first row of the sub-tile
             const int qi = qmin + row;                                // subsequence row / position
             const int W = p.win[u.h];
@@ -590,12 +609,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 if (!ok) break;
                 ++n_s;
                 tc_fence_after();
-                // mask: causal on subsequence rows (dilated part); keys in (qi - W, qi] (window part)
+                // mask: causal on subsequence rows (dilated part); keys in (qi - W, qi] (window
+                // part); grid keys g <= (qi+1)/D - 1 (grid part)
                 const int ks = BN * j;
-                const bool full = !kWin ? (ks + BN - 1 <= qmin)
-                                                 : (ks + BN - 1 <= qmin && ks > qmin + BM - 1 - W);
-                // row limits in keys from the tile's first column
-                const int lim = qi - ks;            // key k valid iff k <= lim (both parts)
+                const bool full = kGrid ? (ks + BN - 1 <= (qmin + 1) / C.D - 1)
+                                  : !kWin ? (ks + BN - 1 <= qmin)
+                                          : (ks + BN - 1 <= qmin && ks > qmin + BM - 1 - W);
+                // row limits in keys from the tile's first column: key k valid iff k <= lim
+                const int lim = kGrid ? (qi + 1) / C.D - 1 - ks : qi - ks;
                 // window part: and k > lo (no lower limit in the dilated part)
                 const int lo = kWin ? qi - W - ks : INT_MIN / 2;
                 const int mode = full ? 0 : 2;
@@ -637,20 +658,49 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (!ok) break;
             if (nt > 0) {
                 const bool valid_row = qi < C.n;
-                const long long t = kWin ? (long long)qi : (long long)u.r + (long long)C.D * qi;
+                const long long t = kKind != kTcDilated ? (long long)qi : (long long)u.r + (long long)C.D * qi;
                 const size_t orow = (((size_t)u.b * p.T + (size_t)t) * p.H + u.h) * HD;
                 const size_t lrow = ((size_t)u.b * p.H + u.h) * p.T + (size_t)t;
                 __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.o);
-                constexpr bool merge = kWin;
-                // The window launch merges with the dilated part's row (o, lse),
-                // written by the previous launch: fetch it while the last PV runs.
+                constexpr bool merge = kWin || kGrid;
+                // The row's other part, merged by LSE: for the window launch the
+                // dilated part's row (o, lse) written by the previous launch; for
+                // the grid launch the row's own key (V~_t, score s q_t.K~_t) when
+                // t is off the grid.  Fetched while the last PV runs.
+                const bool mrow = merge && valid_row && (!kGrid || t % C.D != C.D - 1);
                 uint4 prev[HD / 8];
                 float ld2 = 0.f;
-                if (merge && valid_row) {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(o + orow);
+                if (mrow) {
+                    if constexpr (kGrid) {
+                        const uint4 *qs = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.q) + orow);
+                        const uint4 *ks4 =
+                            reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.kself[u.cls]) + orow);
+                        const uint4 *vs4 =
+                            reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.vself[u.cls]) + orow);
+                        float z = 0.f;
 #pragma unroll
-                    for (int q = 0; q < HD / 8; ++q) prev[q] = src[q];
-                    ld2 = p.lse_dil[lrow] * 1.4426950408889634f;
+                        for (int q = 0; q < HD / 8; ++q) {
+                            const uint4 a = qs[q], k4 = ks4[q];
+                            const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, kw[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&aw[i]));
+                                const float2 fk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kw[i]));
+                                z = fmaf(fa.x, fk.x, z);
+                                z = fmaf(fa.y, fk.y, z);
+                            }
+                            prev[q] = vs4[q];
+                        }
+                        ld2 = z * p.scale_log2;
+                    } else {
+                        const uint4 *src = reinterpret_cast<const uint4 *>(o + orow);
+#pragma unroll
+                        for (int q = 0; q < HD / 8; ++q) prev[q] = src[q];
+                        ld2 = p.lse_dil[lrow] * 1.4426950408889634f;
+                    }
+                } else if constexpr (merge) {
+#pragma unroll
+                    for (int q = 0; q < HD / 8; ++q) prev[q] = make_uint4(0u, 0u, 0u, 0u);
                 }
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar_pvdone[sub], (uint32_t)n_pv & 1u, &s_abort));
                 if (!ok) break;
@@ -659,9 +709,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 // ---- epilogue: o = O / l, lse = ln(2) * (m + log2 l)
                 const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
                 float lse2 = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;  // log2 domain
+                // weights of this launch's part (w_self) and of the other part (w_dil)
                 float w_self = 1.f, w_dil = 0.f;
-                if (merge && valid_row) {
-                    // merge with the dilated part: weights e^(lse_i - max) / sum
+                if (mrow) {
+                    // merge with the other part: weights e^(lse_i - max) / sum
                     const float mm = fmaxf(ld2, lse2);
                     const float e1 = ex2(ld2 - mm), e2 = ex2(lse2 - mm);
                     w_dil = e1 / (e1 + e2);
@@ -745,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 }
                 if (valid_row) {
                     const float lse = lse2 * 0.69314718055994531f;
-                    if (!merge && p.win[u.h] > 0) p.lse_dil[lrow] = lse;  // the window launch merges later
+                    if (!kWin && p.win[u.h] > 0) p.lse_dil[lrow] = lse;  // the window launch merges later
                     else if (p.lse_user) p.lse_user[lrow] = lse;
                 }
             }
@@ -823,13 +874,22 @@ size_t attn_tc_smem_bytes(int hd) {
     return need > 120 * 1024 ? need : 120 * 1024;
 }
 
-template <int HD, bool kWin>
+template <int HD, int kKind>
 cudaError_t launch_inst(const TcParams &p, unsigned grid, size_t smem, cudaStream_t s) {
     static std::atomic<unsigned long long> smem_set{0};
-    cudaError_t e = ensure_smem_limit(attn_tc_kernel<HD, kWin>, smem, smem_set);
+    cudaError_t e = ensure_smem_limit(attn_tc_kernel<HD, kKind>, smem, smem_set);
     if (e != cudaSuccess) return e;
-    attn_tc_kernel<HD, kWin><<<grid, kThreads, smem, s>>>(p);
+    attn_tc_kernel<HD, kKind><<<grid, kThreads, smem, s>>>(p);
     return cudaSuccess;
+}
+
+template <int HD>
+cudaError_t launch_kind(const TcParams &p, unsigned grid, size_t smem, cudaStream_t s) {
+    switch (p.kind) {
+    case kTcWindow: return launch_inst<HD, kTcWindow>(p, grid, smem, s);
+    case kTcGrid: return launch_inst<HD, kTcGrid>(p, grid, smem, s);
+    default: return launch_inst<HD, kTcDilated>(p, grid, smem, s);
+    }
 }
 
 cudaError_t launch_attn_tc(const TcParams &p, int hd, cudaStream_t s) {
@@ -841,10 +901,9 @@ cudaError_t launch_attn_tc(const TcParams &p, int hd, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM (the shared memory and TMEM of one CTA fill an SM)
     const unsigned grid = (unsigned)std::min<long long>(p.total_units, (long long)nsm);
-    // the dilated and window launches are separate instantiations, so each
-    // carries only its own epilogue and masks (instruction-cache footprint)
-    if (hd == 128) e = p.window_mode ? launch_inst<128, true>(p, grid, smem, s) : launch_inst<128, false>(p, grid, smem, s);
-    else e = p.window_mode ? launch_inst<64, true>(p, grid, smem, s) : launch_inst<64, false>(p, grid, smem, s);
+    // each launch kind is its own instantiation, carrying only its own
+    // epilogue and masks (instruction-cache footprint)
+    e = hd == 128 ? launch_kind<128>(p, grid, smem, s) : launch_kind<64>(p, grid, smem, s);
     if (e != cudaSuccess) return e;
     count_launches(1);
     return cudaGetLastError();

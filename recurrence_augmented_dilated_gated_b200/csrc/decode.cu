@@ -7,6 +7,10 @@
 //   s <- a*s + (1-a)*x (x = k, v; a = sigmoid(g), a = 0 without recurrence),
 //   the new augmented row is stored at cache row (t mod D)*S + t/D,
 //   o = softmax over the multiset  { j <= t, j == t mod D }  (+)  { t-W+1..t }.
+// Under the fixed-grid reading the dilated set is { j < t, j mod D == D-1 }
+// plus t, the slab is the grid (rows 0 .. t/D - 1, the same count), the new
+// row is stored at its grid row only when t is on the grid, and the window
+// rows come from a ring of the last W positions (D > 1).
 // Softmaxes over disjoint pieces of a key multiset combine exactly by
 // log-sum-exp, so the step is split into independent work items:
 //   * item i of (b, h) streams its run of old rows of the residue slab
@@ -182,7 +186,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     const int Dh = p.dil[h], W = p.win[h];
     const long long S = p.slab[h];
     const int r = valid_pos ? t % Dh : 0;
-    const int n_old = valid_pos ? t / Dh : 0;    // old rows of the residue slab
+    const int n_old = valid_pos ? t / Dh : 0;    // old rows of the residue slab (or grid)
+    const size_t slab0 = p.grid ? 0 : (size_t)r * S;   // first cache row of the slab
     const int i0 = li * p.rows_per_item[h];      // this item's run of old rows: [i0, i1)
     const int i1 = min(i0 + p.rows_per_item[h], n_old);
     const int nrows = max(0, i1 - i0);
@@ -213,8 +218,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         // ------------------------------------------------ producer: stream the
         // item's contiguous run of K~ and V~ rows through the ring
         if ((tid & 31) == 0 && valid_pos) {
-            const char *kb = reinterpret_cast<const char *>(ck + ((size_t)r * S + i0) * D);
-            const char *vb = reinterpret_cast<const char *>(cv + ((size_t)r * S + i0) * D);
+            const char *kb = reinterpret_cast<const char *>(ck + (slab0 + i0) * D);
+            const char *vb = reinterpret_cast<const char *>(cv + (slab0 + i0) * D);
             int sidx = 0;
             bool ok = true;
             for (; sidx < nst; ++sidx) {
@@ -324,9 +329,18 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                 const float sv = a * st_v + oma * in_v;
                 p.state[0][e_new] = sk;
                 p.state[1][e_new] = sv;
-                const size_t row = (size_t)r * S + n_old;
-                static_cast<T *>(p.cache[0])[bh * (size_t)p.cache_R * D + row * D + tid] = to_t<T>(sk);
-                static_cast<T *>(p.cache[1])[bh * (size_t)p.cache_R * D + row * D + tid] = to_t<T>(sv);
+                long long row0, row1;
+                cache_rows_of(t, Dh, W, S, p.grid, row0, row1);
+                T *dk = static_cast<T *>(p.cache[0]) + bh * (size_t)p.cache_R * D + tid;
+                T *dv = static_cast<T *>(p.cache[1]) + bh * (size_t)p.cache_R * D + tid;
+                if (row0 >= 0) {
+                    dk[(size_t)row0 * D] = to_t<T>(sk);
+                    dv[(size_t)row0 * D] = to_t<T>(sv);
+                }
+                if (row1 >= 0) {  // the ring slot of t - W, which no window needs any more
+                    dk[(size_t)row1 * D] = to_t<T>(sk);
+                    dv[(size_t)row1 * D] = to_t<T>(sv);
+                }
                 s_new[0][tid] = round_to<T>(sk);
                 s_new[1][tid] = round_to<T>(sv);
             }
@@ -341,7 +355,9 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                     for (int u = 0; u < kBatch; ++u) {
                         if (u < n) {
                             const int jj = j + u;
-                            const size_t row = (size_t)(jj % Dh) * S + (size_t)(jj / Dh);
+                            long long row0, row1;
+                            cache_rows_of(jj, Dh, W, S, p.grid, row0, row1);
+                            const size_t row = (size_t)(row1 >= 0 ? row1 : row0);
                             IO8<T>::load(ck + row * D + c0, kf[u]);
                             IO8<T>::load(cv + row * D + c0, vf[u]);
                         } else {
@@ -493,8 +509,11 @@ size_t decode_plan(const rat_cfg *c, int cap, DecodeParams *p) {
         p->item0[h] = items;
         p->recur[h] = (c->recur == nullptr || c->recur[h] != 0) ? 1 : 0;
         items += n;
-        R = R > (long long)D * slab ? R : (long long)D * slab;
+        const bool grid = (c->flags & RAT_FLAG_GRID_DILATION) != 0;
+        const long long rows = grid ? (long long)slab + (D > 1 ? c->win[h] : 0) : (long long)D * slab;
+        R = R > rows ? R : rows;
     }
+    p->grid = (c->flags & RAT_FLAG_GRID_DILATION) ? 1 : 0;
     p->item0[c->H] = items;
     p->items_per_b = items;
     p->cache_R = R;

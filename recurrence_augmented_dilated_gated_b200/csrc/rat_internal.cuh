@@ -92,6 +92,21 @@ __device__ __forceinline__ float f4get(const float4 &v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
+// Decode-cache rows of position j for a head with dilation D, window W and
+// S = ceil(cap / D) (layout in include/rat.h).  Residue-major: one row.  Fixed
+// grid: the grid row when j is on the grid (j mod D == D - 1), and the window
+// ring row when the head keeps a ring (D > 1, W > 0); -1 where there is none.
+__host__ __device__ __forceinline__ void cache_rows_of(long long j, int D, int W, long long S, int grid,
+                                                       long long &grid_row, long long &ring_row) {
+    if (!grid) {
+        grid_row = (j % D) * S + j / D;
+        ring_row = -1;
+        return;
+    }
+    grid_row = (j % D == D - 1) ? j / D : -1;
+    ring_row = (D > 1 && W > 0) ? S + j % W : -1;
+}
+
 // --------------------------------------------------------------- scan (K1)
 struct ScanParams {
     // 4-D TMA maps (d, H, T, B) of k, v, g (loads) and kt, vt (stores), box
@@ -106,6 +121,7 @@ struct ScanParams {
     void *cache[2];         // decode cache [B,H,R,d] or null
     long long cache_R;      // rows per (b,h) cache block
     int cap;
+    int grid;               // cache layout of the fixed-grid reading (grid rows + window ring)
     int B, T, H, d;
     int nslices;            // B * nheads
     int nchunks;            // chunks along T per slice
@@ -114,6 +130,7 @@ struct ScanParams {
     unsigned char head_list[kMaxHeads];
     unsigned char head_recur[kMaxHeads];
     int head_dil[kMaxHeads];
+    int head_win[kMaxHeads];
     unsigned int *ticket;   // dynamic chunk ticket counter (zeroed per launch)
     int *flags;             // [nslices * nchunks] 0 none, 1 aggregate, 2 inclusive
     float *agg;             // [nslices * nchunks][3][d]  (A, b_k, b_v)
@@ -130,6 +147,7 @@ struct AttnParams {
     float *lse;             // [B,H,T] or null
     int B, T, H, d;
     float scale_log2;       // scale * log2(e)
+    int grid;               // fixed-grid reading of dilation
     int dil[kMaxHeads];
     int win[kMaxHeads];
     unsigned char use_raw[kMaxHeads];
@@ -150,6 +168,7 @@ struct DecodeParams {
     long long cache_R;
     int cap, B, H, d;
     int items_per_b;             // sum over heads of nsplit
+    int grid;                    // fixed-grid reading and its cache layout
     float scale_log2;
     int dil[kMaxHeads];
     int win[kMaxHeads];

@@ -464,8 +464,10 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
     }
     T *ck = static_cast<T *>(p.cache[0]);
     T *cv = static_cast<T *>(p.cache[1]);
-    const int Dh = p.head_dil[h];
+    const int Dh = p.head_dil[h], Wh = p.head_win[h];
     const long long S = ((long long)p.cap + Dh - 1) / Dh;
+    // the window ring keeps the prefill's last W positions (one writer per row)
+    const long long ring_from = (long long)p.T - Wh;
     const size_t cbase = ((size_t)b * p.H + h) * (size_t)p.cache_R * D + c0;
     if (loaded && !kAccurate && rec) {
         // bf16: a = 1 - (1 - a) from the fp16 cache, channel pairs in f32x2
@@ -492,10 +494,18 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
                 *reinterpret_cast<uint2 *>(tile_v + r * D + c0) = make_uint2(wv[0], wv[1]);
                 if (ck) {
                     const long long tt = tc0 + r;
-                    const long long row = (tt % Dh) * S + tt / Dh;
-                    const size_t e = cbase + (size_t)row * D;
-                    *reinterpret_cast<uint2 *>(ck + e) = make_uint2(wk[0], wk[1]);
-                    *reinterpret_cast<uint2 *>(cv + e) = make_uint2(wv[0], wv[1]);
+                    long long row0, row1;
+                    cache_rows_of(tt, Dh, Wh, S, p.grid, row0, row1);
+                    if (row0 >= 0) {
+                        const size_t e = cbase + (size_t)row0 * D;
+                        *reinterpret_cast<uint2 *>(ck + e) = make_uint2(wk[0], wk[1]);
+                        *reinterpret_cast<uint2 *>(cv + e) = make_uint2(wv[0], wv[1]);
+                    }
+                    if (row1 >= 0 && tt >= ring_from) {
+                        const size_t e = cbase + (size_t)row1 * D;
+                        *reinterpret_cast<uint2 *>(ck + e) = make_uint2(wk[0], wk[1]);
+                        *reinterpret_cast<uint2 *>(cv + e) = make_uint2(wv[0], wv[1]);
+                    }
                 }
             }
         }
@@ -535,10 +545,16 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
                 Smem4<T>::store(tile_v + r * D + c0, wv);
                 if (ck) {
                     const long long tt = tc0 + r;
-                    const long long row = (tt % Dh) * S + tt / Dh;
-                    const size_t e = cbase + (size_t)row * D;
-                    IO4<T>::store(ck + e, wk);
-                    IO4<T>::store(cv + e, wv);
+                    long long row0, row1;
+                    cache_rows_of(tt, Dh, Wh, S, p.grid, row0, row1);
+                    if (row0 >= 0) {
+                        IO4<T>::store(ck + cbase + (size_t)row0 * D, wk);
+                        IO4<T>::store(cv + cbase + (size_t)row0 * D, wv);
+                    }
+                    if (row1 >= 0 && tt >= ring_from) {
+                        IO4<T>::store(ck + cbase + (size_t)row1 * D, wk);
+                        IO4<T>::store(cv + cbase + (size_t)row1 * D, wv);
+                    }
                 }
             }
         }

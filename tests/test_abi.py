@@ -36,7 +36,7 @@ def test_header_declares_the_binding_exports():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.rat_version() == 100
+    assert lib.rat_version() == 101
 
 
 def test_status_strings(lib):
@@ -96,6 +96,22 @@ def test_cache_rows_layout(lib):
         expect = max(D * -(-cap // D) for D in (1, 16, 64))
         assert lib.rat_cache_rows(c.ref(), cap) == expect
     assert lib.rat_cache_rows(c.ref(), 0) == 0
+
+
+
+def test_cache_rows_layout_fixed_grid(lib):
+    # fixed grid: ceil(cap / D) grid rows, plus a ring of W rows when D > 1 and W > 0
+    c = cfg(H=4, dil=[1, 16, 64, 8], win=[32, 0, 256, 0], flags=rat.RAT_FLAG_GRID_DILATION)
+    for cap in (1, 63, 64, 65, 4096, 33792):
+        expect = max(-(-cap // D) + (W if D > 1 else 0) for D, W in ((1, 32), (16, 0), (64, 256), (8, 0)))
+        assert lib.rat_cache_rows(c.ref(), cap) == expect
+    # the decode plan strides the cache by the same row count (workspace stays defined)
+    assert lib.rat_workspace_size(c.ref(), rat.RAT_OP_DECODE, 4096) > 0
+
+
+def test_unknown_flags_are_rejected(lib):
+    assert lib.rat_workspace_size(cfg(flags=2).ref(), rat.RAT_OP_MIX, 0) == 0
+    assert lib.rat_workspace_size(cfg(flags=rat.RAT_FLAG_GRID_DILATION).ref(), rat.RAT_OP_MIX, 0) > 0
 
 
 def call_scan(lib, c, **ptrs):

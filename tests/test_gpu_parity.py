@@ -22,8 +22,8 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def make_cfg(B, T, H, d, dtype, dil, win, recur=None, scale=0.0):
-    return rat.Config(B, T, H, d, dtype, dil, win, recur, scale)
+def make_cfg(B, T, H, d, dtype, dil, win, recur=None, scale=0.0, grid=False):
+    return rat.Config(B, T, H, d, dtype, dil, win, recur, scale, rat.RAT_FLAG_GRID_DILATION if grid else 0)
 
 
 def inputs(B, T, H, d, dtype, mu=2.0, seed=0, device="cpu"):
@@ -277,14 +277,15 @@ def test_decode_cache_layout_from_scan():
 
 
 def run_decode_case(B, T, steps, H, d, dtype, dil, win, recur, mu, seed, cap=None, check_b=None, check_h=None,
-                    gen_device="cpu"):
+                    gen_device="cpu", grid=False):
     """Prefill T tokens into the cache with rat_scan_prefill, then decode `steps`
     tokens with rat_decode_step; compare every step with the oracle's rows
-    (on the batch entries check_b and heads check_h; all by default)."""
+    (on the batch entries check_b and heads check_h; all by default).  grid:
+    the fixed-grid reading of dilation and its cache layout."""
     Tt = T + steps
     cap = cap or Tt
     q, k, v, g = inputs(B, Tt, H, d, dtype, mu=mu, seed=seed, device=gen_device)
-    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur, grid=grid)
     R = rat.rat_cache_rows(cfg, cap)
     ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
     cv = torch.zeros_like(ck)
@@ -313,7 +314,7 @@ def run_decode_case(B, T, steps, H, d, dtype, dil, win, recur, mu, seed, cap=Non
     kt, fk = oracle.scan(sl(k), sl(g), None, rsel)
     vt, fv = oracle.scan(sl(v), sl(g), None, rsel)
     rows = np.array([(b, i, t) for b in range(len(bsel)) for i in range(len(hsel)) for t in range(T, Tt)])
-    ro, rl = oracle.attn_rows(sl(q), kt, vt, dsel, wsel, rows, parts=3)
+    ro, rl = oracle.attn_rows(sl(q), kt, vt, dsel, wsel, rows, parts=3, grid=grid)
     ro = ro.reshape(len(bsel), len(hsel), steps, d)
     rl = rl.reshape(len(bsel), len(hsel), steps)
     ft = torch.float32 if dtype == torch.float32 else dtype
@@ -440,6 +441,102 @@ def test_decode_step_replays_from_a_cuda_graph():
     assert_close(sk, fk, dtype, "state_k after the replays")
     assert_close(sv, fv, dtype, "state_v after the replays")
     del graph
+
+
+# ------------------------------------------------- fixed-grid reading of dilation
+# Query t attends to { j <= t : j mod D == D-1 } plus itself, and the decode
+# cache keeps only the grid rows plus a ring of the last W positions.
+
+GRID_CASES = [
+    # (B, T, dil per head, win per head)
+    (2, 2048, [4, 64], [0, 100]),        # tensor-core grid launch, one head windowed
+    (1, 12800, [64, 128], [1, 3000]),    # 200 and 100 grid rows: full and partial key tiles
+    (2, 1024, [256, 1], [0, 64]),        # D = 256: the first query tiles have no grid key yet
+    (2, 1000, [8, 3], [127, 0]),         # 3 does not divide T: that head runs on CUDA cores
+]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("case", range(len(GRID_CASES)))
+def test_grid_attention_every_element(dtype, d, case):
+    B, T, dil, win = GRID_CASES[case]
+    H = len(dil)
+    q, kt, vt, _ = inputs(B, T, H, d, dtype, seed=700 + case)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, grid=True)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, T, device=DEV)
+    ws = rat.workspace(cfg, rat.RAT_OP_ATTN)
+    rat.rat_dilated_attn_prefill(cfg, q, kt, vt, o, lse, ws)
+    rat.rat_check_status(ws)
+    ro, rl = oracle.attention(f64(q), f64(kt), f64(vt), dil, win, grid=True)
+    assert_close(o, ro, dtype, "o")
+    assert_close(lse, rl, dtype if dtype == torch.bfloat16 else torch.float32, "lse")
+    err = np.linalg.norm(f64(o) - ro, axis=-1) / np.maximum(np.linalg.norm(ro, axis=-1), 1e-30)
+    assert float(err.max()) < 5e-2, "worst row rel err %.3g" % float(err.max())
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_grid_mix_hybrid_heads_every_element(dtype):
+    # a dense head without recurrence next to dilated recurrent heads
+    B, T, d = 2, 1536, 128
+    dil, win, recur = [1, 16, 64], [0, 0, 256], [0, 1, 1]
+    H = len(dil)
+    q, k, v, g = inputs(B, T, H, d, dtype, seed=77)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur, grid=True)
+    out = rat.mix_prefill(cfg, q, k, v, g)
+    rat.rat_check_status(out["ws"])
+    rk, _ = oracle.scan(f64(k), f64(g), None, recur)
+    rv, _ = oracle.scan(f64(v), f64(g), None, recur)
+    ro, rl = oracle.attention(f64(q), rk, rv, dil, win, grid=True)
+    assert_close(out["o"], ro, dtype, "o")
+    assert_close(out["lse"], rl, dtype if dtype == torch.bfloat16 else torch.float32, "lse")
+
+
+def test_grid_decode_cache_layout_from_scan():
+    # grid row of j (j mod D == D-1): j // D; ring row (D > 1, W > 0) of the
+    # prefill's last W positions: ceil(cap / D) + j mod W
+    B, T, H, d = 2, 300, 4, 64
+    dtype = torch.bfloat16
+    dil, win = [1, 4, 7, 16], [5, 0, 40, 512]
+    cap = 333
+    q, k, v, g = inputs(B, T, H, d, dtype, seed=19)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, grid=True)
+    R = rat.rat_cache_rows(cfg, cap)
+    ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
+    cv = torch.zeros_like(ck)
+    kt, vt = torch.empty_like(k), torch.empty_like(v)
+    ws = rat.workspace(cfg, rat.RAT_OP_SCAN)
+    rat.rat_scan_prefill(cfg, k, v, g, None, None, kt, vt, None, None, ck, cv, cap, ws)
+    rat.rat_check_status(ws)
+    for h, (D, W) in enumerate(zip(dil, win)):
+        S = -(-cap // D)
+        j = torch.arange(D - 1, T, D, device=DEV)
+        assert torch.equal(ck[:, h, j // D], kt[:, j, h])
+        assert torch.equal(cv[:, h, j // D], vt[:, j, h])
+        if D > 1 and W > 0:
+            j = torch.arange(max(0, T - W), T, device=DEV)
+            assert torch.equal(ck[:, h, S + j % W], kt[:, j, h])
+            assert torch.equal(cv[:, h, S + j % W], vt[:, j, h])
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+def test_grid_decode_steps_every_element(dtype, d):
+    # positions 1500..1504 put t on the grid of D = 4, 16 and 3 once each
+    run_decode_case(B=3, T=1500, steps=5, H=4, d=d, dtype=dtype, dil=[1, 4, 16, 3], win=[0, 0, 64, 1500],
+                    recur=[0, 1, 1, 1], mu=2.0, seed=21, grid=True)
+
+
+def test_grid_decode_from_empty_history():
+    # the ring fills while the first positions are decoded (cap 8 < W for one head)
+    run_decode_case(B=2, T=1, steps=6, H=3, d=128, dtype=torch.bfloat16, dil=[2, 1, 3], win=[3, 0, 10],
+                    recur=[1, 0, 1], mu=2.0, seed=5, cap=8, grid=True)
+
+
+def test_grid_decode_long_slab_spans_several_splits():
+    run_decode_case(B=1, T=5000, steps=2, H=2, d=128, dtype=torch.bfloat16, dil=[2, 1], win=[9, 7],
+                    recur=[1, 1], mu=2.0, seed=6, grid=True)
 
 
 def test_decode_bad_position_is_reported():
