@@ -30,7 +30,7 @@
  *                which a decode can keep in a cache D times smaller.
  *   window       W > 0 adds a second softmax over { max(0, t-W+1) <= j <= t }.
  *   merge        the two softmaxes are merged by log-sum-exp (a key in both
- *                sets counts in both).
+ *                sets counts in both; with RAT_FLAG_DEDUPE, once).
  *   scale        scores are scale * <q_t, k~_j>, scale = 1/sqrt(d) by default.
  *
  * Conventions shared by all calls
@@ -119,6 +119,9 @@ typedef struct {
 /* Fixed-grid reading of dilation (see "dilation" above) for every head of the
  * call, and the matching decode-cache layout (see rat_cache_rows). */
 #define RAT_FLAG_GRID_DILATION 1u
+/* A key in both the dilated set and the window counts once: the window part
+ * skips the keys the dilated set holds (with D = 1 the window adds nothing). */
+#define RAT_FLAG_DEDUPE 2u
 
 /* Bytes of workspace `op` needs for `cfg` (cache_cap: decode capacity, else
  * ignored).  Returns 0 when cfg is invalid. */

@@ -22,6 +22,7 @@ RAT_OK, RAT_ERR_INVALID, RAT_ERR_UNSUPPORTED, RAT_ERR_CUDA, RAT_ERR_TIMEOUT, RAT
 RAT_F32, RAT_BF16 = 0, 1
 RAT_OP_SCAN, RAT_OP_ATTN, RAT_OP_MIX, RAT_OP_MIX_CALLER_KV, RAT_OP_DECODE = range(5)
 RAT_FLAG_GRID_DILATION = 1
+RAT_FLAG_DEDUPE = 2
 
 EXPORTS = ["rat_workspace_size", "rat_workspace_init", "rat_cache_rows", "rat_scan_prefill",
            "rat_dilated_attn_prefill", "rat_mix_prefill", "rat_decode_step", "rat_check_status",

@@ -73,13 +73,20 @@ rat_status check_cfg(const rat_cfg *c, bool need_T = true) {
     const double elems = (double)c->B * (need_T ? (double)c->T : 1.0) * c->H * c->d;
     if (elems >= 1099511627776.0) return fail(RAT_ERR_INVALID, "B*T*H*d too large");
     if (!(c->scale == c->scale)) return fail(RAT_ERR_INVALID, "scale is NaN");
-    if (c->flags & ~RAT_FLAG_GRID_DILATION) return fail(RAT_ERR_INVALID, "unknown flags 0x%x", c->flags);
+    if (c->flags & ~(RAT_FLAG_GRID_DILATION | RAT_FLAG_DEDUPE))
+        return fail(RAT_ERR_INVALID, "unknown flags 0x%x", c->flags);
     return RAT_OK;
 }
 
 bool head_recur(const rat_cfg *c, int h) { return c->recur == nullptr || c->recur[h] != 0; }
 
 bool grid_mode(const rat_cfg *c) { return (c->flags & RAT_FLAG_GRID_DILATION) != 0; }
+
+bool dedupe_mode(const rat_cfg *c) { return (c->flags & RAT_FLAG_DEDUPE) != 0; }
+
+// The window a head's attention runs: with dedupe a D = 1 head's window keys
+// all lie in its dilated set, so it has no window part.
+int attn_window(const rat_cfg *c, int h) { return dedupe_mode(c) && c->dil[h] == 1 ? 0 : c->win[h]; }
 
 float scale_of(const rat_cfg *c) { return c->scale > 0.f ? c->scale : 1.0f / sqrtf((float)c->d); }
 
@@ -244,7 +251,7 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, int ki
                           const void *kt, const void *vt, const void *kraw, const void *vraw,
                           const bool *raw_head, void *o, float *lse, float *lse_dil, char *ws, unsigned *tickets,
                           int *n_launch, cudaStream_t s) {
-    struct Key { int D; int raw; };
+    struct Key { int D; int raw; int xd; };
     int done = 0;
     bool taken[kMaxHeads] = {false};
     while (done < nheads) {
@@ -258,7 +265,8 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, int ki
         P.hdr = reinterpret_cast<WsHeader *>(ws);
         if (*n_launch >= kAttnTickets) return fail(RAT_ERR_UNSUPPORTED, "more than %d attention launches", kAttnTickets);
         P.ticket = tickets + (*n_launch)++;
-        for (int h = 0; h < c->H; ++h) P.win[h] = c->win[h];
+        P.grid = grid_mode(c) ? 1 : 0;
+        for (int h = 0; h < c->H; ++h) P.win[h] = attn_window(c, h);
         // collect up to kTcMaxClasses classes
         Key keys[kTcMaxClasses];
         int ncls = 0, nh = 0;
@@ -267,10 +275,12 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, int ki
         for (int i = 0; i < nheads; ++i) {
             const int h = heads[i];
             if (taken[i]) continue;
-            const Key k{kind == kTcWindow ? 1 : c->dil[h], raw_head[h] ? 1 : 0};
+            const bool win_kind = kind == kTcWindow || kind == kTcWindowDedupe;
+            // the dedupe window launch also tells the heads' dilations apart
+            const Key k{win_kind ? 1 : c->dil[h], raw_head[h] ? 1 : 0, kind == kTcWindowDedupe ? c->dil[h] : 1};
             int ci = -1;
             for (int j = 0; j < ncls; ++j)
-                if (keys[j].D == k.D && keys[j].raw == k.raw) ci = j;
+                if (keys[j].D == k.D && keys[j].raw == k.raw && keys[j].xd == k.xd) ci = j;
             if (ci < 0) {
                 if (ncls == kTcMaxClasses) continue;  // next launch
                 ci = ncls++;
@@ -294,6 +304,7 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, int ki
             C.n = kind == kTcDilated ? c->T / C.D : c->T;
             C.nres = kind == kTcDilated ? C.D : 1;
             C.kres = kind == kTcGrid ? C.D - 1 : 0;   // the grid is residue D-1
+            C.xd = keys[ci].xd;
             C.mtiles = (C.n + 255) / 256;   // 256-row units per (b, h, residue) group
             C.nheads = cls_n[ci];
             C.head0 = nh;
@@ -328,7 +339,7 @@ rat_status run_attn(const rat_cfg *c, const Layout &L, const void *q, const void
         if (tc_head(c, h)) {
             if (grid_head(c, h)) tc_grid[n_grid++] = h;
             else tc_all[n_tc++] = h;
-            if (c->win[h] > 0) tc_win[n_win++] = h;
+            if (attn_window(c, h) > 0) tc_win[n_win++] = h;
         } else {
             ++n_simt;
         }
@@ -351,7 +362,7 @@ rat_status run_attn(const rat_cfg *c, const Layout &L, const void *q, const void
                                 tickets, &n_launch, s);
         if (st != RAT_OK) return st;
         if (n_win > 0) {
-            st = launch_tc_part(c, tc_win, n_win, kTcWindow, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws,
+            st = launch_tc_part(c, tc_win, n_win, dedupe_mode(c) ? kTcWindowDedupe : kTcWindow, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws,
                                 tickets, &n_launch, s);
             if (st != RAT_OK) return st;
         }
@@ -364,9 +375,10 @@ rat_status run_attn(const rat_cfg *c, const Layout &L, const void *q, const void
         p.B = c->B; p.T = c->T; p.H = c->H; p.d = c->d;
         p.scale_log2 = scale_of(c) * 1.4426950408889634f;
         p.grid = grid_mode(c) ? 1 : 0;
+        p.dedupe = dedupe_mode(c) ? 1 : 0;
         for (int h = 0; h < c->H; ++h) {
             p.dil[h] = c->dil[h];
-            p.win[h] = c->win[h];
+            p.win[h] = attn_window(c, h);
             p.use_raw[h] = raw_head[h] ? 1 : 0;
             p.skip[h] = tc_head(c, h) ? 1 : 0;
         }

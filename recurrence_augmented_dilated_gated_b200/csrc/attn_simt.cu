@@ -4,7 +4,8 @@
 // to the dilated set { j <= t : (t-j) mod D == 0 } and, when the head has a
 // window W > 0, in a second softmax to { max(0, t-W+1) <= j <= t }; the two
 // softmaxes are merged by log-sum-exp.  Under the fixed-grid reading the
-// dilated set is { j <= t : j mod D == D-1 } plus t itself (once).
+// dilated set is { j <= t : j mod D == D-1 } plus t itself (once).  With
+// dedupe the window part skips the keys of the dilated set.
 //
 // One warp owns one query row: each lane holds d/32 channels of q and of the
 // running output, the score of every key is a warp-wide dot product, and the
@@ -36,11 +37,15 @@ struct RowState {
     }
 };
 
-// Online softmax over keys j = jhi, jhi - step, ..., >= jlo (log2-domain scores).
+// Online softmax over keys j = jhi, jhi - step, ..., >= jlo (log2-domain scores);
+// with skip_d > 0, keys in the dilated set of row t (dilation skip_d; fixed
+// grid when grid) are left out.
 template <typename T, int CPL>
 __device__ __forceinline__ void attend(RowState<CPL> &st, const float *q, const T *kb, const T *vb,
-                                       size_t rs, long long jlo, long long jhi, long long step, int lane) {
+                                       size_t rs, long long jlo, long long jhi, long long step, int lane,
+                                       int skip_d = 0, long long t = 0, int grid = 0) {
     for (long long j = jhi; j >= jlo; j -= step) {
+        if (skip_d > 0 && (grid ? (j % skip_d == skip_d - 1 || j == t) : ((t - j) % skip_d == 0))) continue;
         const T *kr = kb + (size_t)j * rs;
         const T *vr = vb + (size_t)j * rs;
         float s = 0.f;
@@ -97,7 +102,7 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(const AttnParams
     for (int i = 0; i < CPL; ++i) acc[i] = dil.acc[i];
     if (W > 0) {
         wnd.init();
-        attend<T, CPL>(wnd, q, kb, vb, rs, max(0LL, t - W + 1), t, 1, lane);
+        attend<T, CPL>(wnd, q, kb, vb, rs, max(0LL, t - W + 1), t, 1, lane, p.dedupe ? D : 0, t, p.grid);
         // log-sum-exp merge of two (unnormalised) softmax accumulators
         const float mn = fmaxf(dil.m, wnd.m);
         const float c1 = exp2f(dil.m - mn), c2 = exp2f(wnd.m - mn);

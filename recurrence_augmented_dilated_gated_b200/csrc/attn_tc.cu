@@ -34,6 +34,9 @@
 // of the residue-(D-1) subsequence up to the last row's grid key, masked per
 // row; the epilogue adds the row's own key (when it is off the grid) by LSE,
 // scoring it from q and K~ in global memory.
+// With dedupe the window launch also masks, in every tile, the keys of the
+// row's dilated set (a periodic bit pattern per 32-column chunk), so a key in
+// both sets counts once.
 //
 // Every mbarrier wait is bounded (globaltimer); on expiry the CTA records
 // RAT_ERR_TIMEOUT, raises a shared abort flag, waits (bounded) for its own
@@ -233,7 +236,7 @@ __device__ __forceinline__ Plan make_plan(const TcParams &p, const Unit &u) {
         } else {
             pl.hi[i] = qmin / BN;
         }
-        if (kKind != kTcWindow) {
+        if (kKind != kTcWindow && kKind != kTcWindowDedupe) {
             pl.lo[i] = 0;
         } else {
             const int first = qmin - W + 1;  // earliest key of the sub-tile's first row
@@ -344,6 +347,87 @@ __device__ __forceinline__ float row_exp_s(uint32_t t_s, int lo, int lim, float 
     return ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
 }
 
+// Keys the dilated set already holds, for the window part with dedupe: in a
+// tile, key k is excluded when k == e0 (mod xd).  base has a bit at every
+// multiple of xd below 32 (one bit when xd > 32); e is the offset of the first
+// excluded key of the current 32-column chunk, d32 = 32 mod xd steps it on.
+struct Excl {
+    uint32_t base;
+    int d32, xd;
+};
+
+__device__ __forceinline__ Excl make_excl(int xd) {
+    Excl x;
+    x.xd = xd;
+    x.d32 = 32 % xd;
+    x.base = 0u;
+    for (int k = 0; k < 32; k += xd) x.base |= 1u << k;
+    return x;
+}
+
+__device__ __forceinline__ uint32_t excl_word(const Excl &x, int e) { return e < 32 ? x.base << e : 0u; }
+
+__device__ __forceinline__ int excl_next(const Excl &x, int e) {
+    e -= x.d32;
+    return e < 0 ? e + x.xd : e;
+}
+
+// row_max_s / row_exp_s with the masked test and the exclusion pattern
+// starting at offset e0 of the tile.
+__device__ __forceinline__ float row_max_x(uint32_t t_s, int lo, int lim, const Excl &x, int e0) {
+    float mx4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) mx4[k] = -INFINITY;
+    int e = e0;
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+        uint32_t sr[32];
+        tmem_ld32(t_s + 32 * q, sr);
+        const uint32_t xw = excl_word(x, e);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            float a = __uint_as_float(sr[2 * k]), b = __uint_as_float(sr[2 * k + 1]);
+            a = key_ok<2>(32 * q + 2 * k, lo, lim) && !((xw >> (2 * k)) & 1u) ? a : -INFINITY;
+            b = key_ok<2>(32 * q + 2 * k + 1, lo, lim) && !((xw >> (2 * k + 1)) & 1u) ? b : -INFINITY;
+            mx4[k & 3] = max3(mx4[k & 3], a, b);
+        }
+        e = excl_next(x, e);
+    }
+    return max3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+}
+
+__device__ __forceinline__ float row_exp_x(uint32_t t_s, int lo, int lim, const Excl &x, int e0, float c,
+                                           float m) {
+    uint64_t rs2[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) rs2[k] = f2_pack(0.f, 0.f);
+    const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m, -m);
+    int e = e0;
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+        uint32_t sr[32];
+        tmem_ld32(t_s + 32 * q, sr);
+        const uint32_t xw = excl_word(x, e);
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            float t0, t1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])), c2, nm2), t0, t1);
+            float e0_ = ex2(t0), e1_ = ex2(t1);
+            e0_ = key_ok<2>(32 * q + 2 * k, lo, lim) && !((xw >> (2 * k)) & 1u) ? e0_ : 0.f;
+            e1_ = key_ok<2>(32 * q + 2 * k + 1, lo, lim) && !((xw >> (2 * k + 1)) & 1u) ? e1_ : 0.f;
+            rs2[k & 3] = f2_add(rs2[k & 3], f2_pack(e0_, e1_));
+            pk[k] = pack_bf16(e0_, e1_);
+        }
+        tmem_st16(t_s + 16 * q, pk);
+        e = excl_next(x, e);
+    }
+    float r[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) f2_unpack(rs2[k], r[2 * k], r[2 * k + 1]);
+    return ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
+}
+
 template <int HD>
 struct Smem {
     static constexpr int kTile = BM * HD * 2;   // one 128-row tile of Q, K or V (bytes)
@@ -367,8 +451,9 @@ struct Smem {
 template <int HD, int kKind>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
     using L = Smem<HD>;
-    constexpr bool kWin = kKind == kTcWindow;
+    constexpr bool kWin = kKind == kTcWindow || kKind == kTcWindowDedupe;
     constexpr bool kGrid = kKind == kTcGrid;
+    constexpr bool kDedupe = kKind == kTcWindowDedupe;
     constexpr int NCB = HD / 64;  // 64-column (128-byte) blocks of a head row
     extern __shared__ uint8_t dsmem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
@@ -602,6 +687,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const int W = p.win[u.h];
             const int lo_s = sub ? pl.lo[1] : pl.lo[0];
             const int nt = (sub ? pl.valid[1] : pl.valid[0]) ? (sub ? pl.hi[1] : pl.hi[0]) - lo_s + 1 : 0;
+            Excl xcl;
+            if constexpr (kDedupe) xcl = make_excl(C.xd);
             float m_run = -INFINITY, l_run = 0.f;
             for (int c = 0; c < nt; ++c) {
                 const int j = lo_s + c;
@@ -620,7 +707,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 // window part: and k > lo (no lower limit in the dilated part)
                 const int lo = kWin ? qi - W - ks : INT_MIN / 2;
                 const int mode = full ? 0 : 2;
-                const float mraw = mode == 0 ? row_max_s<0>(t_s, lo, lim) : row_max_s<2>(t_s, lo, lim);
+                // dedupe: the dilated set's keys in this tile are k == e0 (mod xd):
+                // k == lim for the residue reading (the row's own key among them);
+                // the grid positions ks + k == xd - 1 (mod xd) for the fixed grid,
+                // whose own key leaves through the limit instead
+                int e0 = 0, limx = lim;
+                if constexpr (kDedupe) {
+                    const int r0 = p.grid ? (C.xd - 1 - ks) % C.xd : lim % C.xd;
+                    e0 = r0 < 0 ? r0 + C.xd : r0;
+                    if (p.grid) limx = lim - 1;
+                }
+                float mraw;
+                if constexpr (kDedupe) mraw = row_max_x(t_s, lo, limx, xcl, e0);
+                else mraw = mode == 0 ? row_max_s<0>(t_s, lo, lim) : row_max_s<2>(t_s, lo, lim);
                 const float mx = mraw * p.scale_log2;   // scale > 0 commutes with max
                 // running max with lazy rescale: keep the stale max unless the new
                 // one exceeds it by more than 8 (P stays <= 2^8)
@@ -647,8 +746,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                         }
                     }
                 }
-                const float rs = mode == 0 ? row_exp_s<0>(t_s, lo, lim, p.scale_log2, m_use)
-                                           : row_exp_s<2>(t_s, lo, lim, p.scale_log2, m_use);
+                float rs;
+                if constexpr (kDedupe) rs = row_exp_x(t_s, lo, limx, xcl, e0, p.scale_log2, m_use);
+                else rs = mode == 0 ? row_exp_s<0>(t_s, lo, lim, p.scale_log2, m_use)
+                                    : row_exp_s<2>(t_s, lo, lim, p.scale_log2, m_use);
                 l_run = l_run * alpha + rs;
                 m_run = m_new;
                 tc_fence_before();
@@ -888,6 +989,7 @@ cudaError_t launch_kind(const TcParams &p, unsigned grid, size_t smem, cudaStrea
     switch (p.kind) {
     case kTcWindow: return launch_inst<HD, kTcWindow>(p, grid, smem, s);
     case kTcGrid: return launch_inst<HD, kTcGrid>(p, grid, smem, s);
+    case kTcWindowDedupe: return launch_inst<HD, kTcWindowDedupe>(p, grid, smem, s);
     default: return launch_inst<HD, kTcDilated>(p, grid, smem, s);
     }
 }

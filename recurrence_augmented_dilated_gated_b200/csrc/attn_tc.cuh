@@ -14,7 +14,8 @@ constexpr int kTcRowsKV = 128;  // keys per K/V tile (K/V box height)
 // Launch kinds: the residue subsequences of the dilated part; the window part
 // (merged with the dilated part); the fixed-grid reading of the dilated part
 // (every position against the subsequence of residue D-1, plus its own key).
-constexpr int kTcDilated = 0, kTcWindow = 1, kTcGrid = 2;
+// kTcWindowDedupe is the window part that skips the keys of the dilated set.
+constexpr int kTcDilated = 0, kTcWindow = 1, kTcGrid = 2, kTcWindowDedupe = 3;
 
 // Heads of one launch that share a dilation and a K/V source.
 struct TcClass {
@@ -25,7 +26,7 @@ struct TcClass {
     int head0;   // first entry of the class in TcParams::heads
     int nres;    // groups per (b, h): D residues (dilated part), else 1
     int kres;    // residue coordinate of K/V relative to Q's (D - 1 for the grid)
-    int pad;
+    int xd;      // dilation of the heads (the dedupe window launch), else 1
 };
 
 struct TcParams {
@@ -36,7 +37,8 @@ struct TcParams {
     long long prefix[kTcMaxClasses + 1];  // prefix[c] = work units of the classes before c
     int ncls;
     int B, T, H;
-    int kind;                       // kTcDilated, kTcWindow or kTcGrid
+    int kind;                       // kTcDilated, kTcWindow, kTcGrid or kTcWindowDedupe
+    int grid;                       // fixed-grid reading (the dedupe window's excluded keys)
     float scale_log2;
     const void *q;                  // [B,T,H,d] bf16 (the grid's own-key score)
     const void *kself[kTcMaxClasses];  // K/V source of each class, [B,T,H,d] bf16

@@ -10,7 +10,8 @@
 // Under the fixed-grid reading the dilated set is { j < t, j mod D == D-1 }
 // plus t, the slab is the grid (rows 0 .. t/D - 1, the same count), the new
 // row is stored at its grid row only when t is on the grid, and the window
-// rows come from a ring of the last W positions (D > 1).
+// rows come from a ring of the last W positions (D > 1).  With dedupe the
+// window part skips the keys of the dilated set, the new row among them.
 // Softmaxes over disjoint pieces of a key multiset combine exactly by
 // log-sum-exp, so the step is split into independent work items:
 //   * item i of (b, h) streams its run of old rows of the residue slab
@@ -135,13 +136,15 @@ struct Acc8 {
     float m, l, o[8];
 };
 
-// Adds the first n <= NB keys (scores s[], values v[][]) in one rescale;
-// fully unrolled and predicated so the arrays stay in registers.
+// Adds the first n <= NB keys (scores s[], values v[][]) in one rescale,
+// leaving out key u when bit u of `skip` is set; fully unrolled and predicated
+// so the arrays stay in registers.
 template <int NB>
-__device__ __forceinline__ void acc_add_batch(Acc8 &a, const float *s, const float (*v)[8], int n) {
+__device__ __forceinline__ void acc_add_batch(Acc8 &a, const float *s, const float (*v)[8], int n,
+                                              unsigned skip = 0u) {
     float mb = -INFINITY;
 #pragma unroll
-    for (int u = 0; u < NB; ++u) mb = u < n ? fmaxf(mb, s[u]) : mb;
+    for (int u = 0; u < NB; ++u) mb = (u < n && !((skip >> u) & 1u)) ? fmaxf(mb, s[u]) : mb;
     const float mn = fmaxf(a.m, mb);
     const float corr = a.m == -INFINITY ? 0.f : exp2f(a.m - mn);
     a.l *= corr;
@@ -149,7 +152,7 @@ __device__ __forceinline__ void acc_add_batch(Acc8 &a, const float *s, const flo
     for (int i = 0; i < 8; ++i) a.o[i] *= corr;
 #pragma unroll
     for (int u = 0; u < NB; ++u) {
-        const float pj = u < n ? exp2f(s[u] - mn) : 0.f;
+        const float pj = (u < n && !((skip >> u) & 1u)) ? exp2f(s[u] - mn) : 0.f;
         a.l += pj;
 #pragma unroll
         for (int i = 0; i < 8; ++i) a.o[i] += pj * v[u][i];
@@ -351,10 +354,12 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                 for (int j = j0 + grp * kBatch; j < t; j += NG * kBatch) {
                     float kf[kBatch][8], vf[kBatch][8], sc[kBatch];
                     const int n = min(kBatch, t - j);
+                    unsigned skip = 0u;
 #pragma unroll
                     for (int u = 0; u < kBatch; ++u) {
                         if (u < n) {
                             const int jj = j + u;
+                            if (p.dedupe && (p.grid ? jj % Dh == Dh - 1 : (t - jj) % Dh == 0)) skip |= 1u << u;
                             long long row0, row1;
                             cache_rows_of(jj, Dh, W, S, p.grid, row0, row1);
                             const size_t row = (size_t)(row1 >= 0 ? row1 : row0);
@@ -372,10 +377,11 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                         for (int c = 0; c < 8; ++c) s2 += q[c] * kf[u][c];
                         sc[u] = group_sum<LPR>(s2, gmask);
                     }
-                    acc_add_batch<kBatch>(acc, sc, vf, n);
+                    acc_add_batch<kBatch>(acc, sc, vf, n, skip);
                 }
             }
             // the new row: once in the dilated set, once more in the window
+            // (not with dedupe)
             if (grp == 0) {
                 float kv[2][8], sc[2];
 #pragma unroll
@@ -389,7 +395,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                 s2 = group_sum<LPR>(s2, gmask);
                 sc[0] = s2;
                 sc[1] = s2;
-                acc_add_batch<2>(acc, sc, kv, W > 0 ? 2 : 1);
+                acc_add_batch<2>(acc, sc, kv, W > 0 && !p.dedupe ? 2 : 1);
             }
         }
     }
@@ -502,7 +508,8 @@ size_t decode_plan(const rat_cfg *c, int cap, DecodeParams *p) {
         const int ns = (slab + target - 1) / target;
         const int n = ns > 0 ? ns : 1;
         p->dil[h] = D;
-        p->win[h] = c->win[h];
+        // with dedupe a D = 1 head's window keys are all in its dilated set
+        p->win[h] = (c->flags & RAT_FLAG_DEDUPE) && D == 1 ? 0 : c->win[h];
         p->slab[h] = slab;
         p->nsplit[h] = n;
         p->rows_per_item[h] = (slab + n - 1) / n;   // balanced runs
@@ -514,6 +521,7 @@ size_t decode_plan(const rat_cfg *c, int cap, DecodeParams *p) {
         R = R > rows ? R : rows;
     }
     p->grid = (c->flags & RAT_FLAG_GRID_DILATION) ? 1 : 0;
+    p->dedupe = (c->flags & RAT_FLAG_DEDUPE) ? 1 : 0;
     p->item0[c->H] = items;
     p->items_per_b = items;
     p->cache_R = R;

@@ -148,6 +148,7 @@ struct AttnParams {
     int B, T, H, d;
     float scale_log2;       // scale * log2(e)
     int grid;               // fixed-grid reading of dilation
+    int dedupe;             // the window part skips the dilated set's keys
     int dil[kMaxHeads];
     int win[kMaxHeads];
     unsigned char use_raw[kMaxHeads];
@@ -169,6 +170,7 @@ struct DecodeParams {
     int cap, B, H, d;
     int items_per_b;             // sum over heads of nsplit
     int grid;                    // fixed-grid reading and its cache layout
+    int dedupe;                  // the window part skips the dilated set's keys
     float scale_log2;
     int dil[kMaxHeads];
     int win[kMaxHeads];

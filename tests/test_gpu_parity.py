@@ -22,8 +22,9 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def make_cfg(B, T, H, d, dtype, dil, win, recur=None, scale=0.0, grid=False):
-    return rat.Config(B, T, H, d, dtype, dil, win, recur, scale, rat.RAT_FLAG_GRID_DILATION if grid else 0)
+def make_cfg(B, T, H, d, dtype, dil, win, recur=None, scale=0.0, grid=False, dedupe=False):
+    flags = (rat.RAT_FLAG_GRID_DILATION if grid else 0) | (rat.RAT_FLAG_DEDUPE if dedupe else 0)
+    return rat.Config(B, T, H, d, dtype, dil, win, recur, scale, flags)
 
 
 def inputs(B, T, H, d, dtype, mu=2.0, seed=0, device="cpu"):
@@ -277,15 +278,16 @@ def test_decode_cache_layout_from_scan():
 
 
 def run_decode_case(B, T, steps, H, d, dtype, dil, win, recur, mu, seed, cap=None, check_b=None, check_h=None,
-                    gen_device="cpu", grid=False):
+                    gen_device="cpu", grid=False, dedupe=False):
     """Prefill T tokens into the cache with rat_scan_prefill, then decode `steps`
     tokens with rat_decode_step; compare every step with the oracle's rows
     (on the batch entries check_b and heads check_h; all by default).  grid:
-    the fixed-grid reading of dilation and its cache layout."""
+    the fixed-grid reading of dilation and its cache layout; dedupe: a key in
+    both parts counts once."""
     Tt = T + steps
     cap = cap or Tt
     q, k, v, g = inputs(B, Tt, H, d, dtype, mu=mu, seed=seed, device=gen_device)
-    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur, grid=grid)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur, grid=grid, dedupe=dedupe)
     R = rat.rat_cache_rows(cfg, cap)
     ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
     cv = torch.zeros_like(ck)
@@ -314,7 +316,7 @@ def run_decode_case(B, T, steps, H, d, dtype, dil, win, recur, mu, seed, cap=Non
     kt, fk = oracle.scan(sl(k), sl(g), None, rsel)
     vt, fv = oracle.scan(sl(v), sl(g), None, rsel)
     rows = np.array([(b, i, t) for b in range(len(bsel)) for i in range(len(hsel)) for t in range(T, Tt)])
-    ro, rl = oracle.attn_rows(sl(q), kt, vt, dsel, wsel, rows, parts=3, grid=grid)
+    ro, rl = oracle.attn_rows(sl(q), kt, vt, dsel, wsel, rows, parts=3, grid=grid, dedupe=dedupe)
     ro = ro.reshape(len(bsel), len(hsel), steps, d)
     rl = rl.reshape(len(bsel), len(hsel), steps)
     ft = torch.float32 if dtype == torch.float32 else dtype
@@ -537,6 +539,44 @@ def test_grid_decode_from_empty_history():
 def test_grid_decode_long_slab_spans_several_splits():
     run_decode_case(B=1, T=5000, steps=2, H=2, d=128, dtype=torch.bfloat16, dil=[2, 1], win=[9, 7],
                     recur=[1, 1], mu=2.0, seed=6, grid=True)
+
+
+# ------------------------------------------------- dedupe: a shared key counts once
+
+DEDUPE_CASES = [
+    # (B, T, dil per head, win per head): windows wider and narrower than D
+    (2, 2048, [4, 64], [100, 512]),
+    (1, 1056, [1, 33], [64, 1000]),       # D = 1: no window part; D = 33 > 32 (one key per chunk)
+    (2, 768, [2, 3], [1, 300]),           # W = 1 leaves the window part empty (residue reading)
+    (2, 1000, [8, 7], [127, 50]),         # 7 does not divide T: CUDA cores
+]
+
+
+@pytest.mark.parametrize("grid", [False, True])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("case", range(len(DEDUPE_CASES)))
+def test_dedupe_attention_every_element(grid, dtype, case):
+    B, T, dil, win = DEDUPE_CASES[case]
+    H, d = len(dil), 128
+    q, kt, vt, _ = inputs(B, T, H, d, dtype, seed=900 + case)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, grid=grid, dedupe=True)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, T, device=DEV)
+    ws = rat.workspace(cfg, rat.RAT_OP_ATTN)
+    rat.rat_dilated_attn_prefill(cfg, q, kt, vt, o, lse, ws)
+    rat.rat_check_status(ws)
+    ro, rl = oracle.attention(f64(q), f64(kt), f64(vt), dil, win, grid=grid, dedupe=True)
+    assert_close(o, ro, dtype, "o")
+    assert_close(lse, rl, dtype if dtype == torch.bfloat16 else torch.float32, "lse")
+    err = np.linalg.norm(f64(o) - ro, axis=-1) / np.maximum(np.linalg.norm(ro, axis=-1), 1e-30)
+    assert float(err.max()) < 5e-2, "worst row rel err %.3g" % float(err.max())
+
+
+@pytest.mark.parametrize("grid", [False, True])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_dedupe_decode_steps_every_element(grid, dtype):
+    run_decode_case(B=3, T=1500, steps=5, H=4, d=128, dtype=dtype, dil=[1, 4, 16, 3], win=[8, 9, 64, 1500],
+                    recur=[0, 1, 1, 1], mu=2.0, seed=23, grid=grid, dedupe=True)
 
 
 def test_decode_bad_position_is_reported():
