@@ -42,6 +42,9 @@ def _load():
                                                                   ctypes.c_int, ctypes.c_double, ctypes.c_long,
                                                                   lp, dp, dp]
         lib.oracle_attn_rows_topk.restype = ctypes.c_int
+        lib.oracle_topk_select.argtypes = [ctypes.c_int] * 4 + [dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                              ctypes.c_long, lp, ctypes.POINTER(ctypes.c_int), dp]
+        lib.oracle_topk_select.restype = ctypes.c_int
         lib.oracle_decode_step.argtypes = [ctypes.c_int] * 4 + [ip, dp, dp, dp, dp, ip, ip, up,
                                                                 ctypes.c_double, dp, dp, dp, dp, dp, dp]
         lib.oracle_decode_step.restype = ctypes.c_int
@@ -125,6 +128,26 @@ def attn_rows_topk(q, kt, vt, block, K, mode, rows, scale=None):
     if rc != 0:
         raise ValueError("oracle_attn_rows_topk: invalid arguments")
     return o, lse
+
+
+def topk_select(q, kt, block, K, mode, rows):
+    """The block selection of attn_rows_topk for each row: (sel [n, K] int32 in
+    pick order, -1 padded; gap [n]: last pick's score minus the best score
+    left out, +inf when nothing is left out)."""
+    lib = _load()
+    q, kt = _f64(q), _f64(kt)
+    B, T, H, d = q.shape
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+    n = rows.shape[0]
+    sel = np.empty((n, max(int(K), 1)), dtype=np.int32)
+    gap = np.empty((n,), dtype=np.float64)
+    m = {"quest": 0, "moba": 1}[mode]
+    rc = lib.oracle_topk_select(B, T, H, d, _dp(q), _dp(kt), int(block), int(K), m, n,
+                                rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                sel.ctypes.data_as(ctypes.POINTER(ctypes.c_int)), _dp(gap))
+    if rc != 0:
+        raise ValueError("oracle_topk_select: invalid arguments")
+    return sel[:, :K], gap
 
 
 def all_rows(B, T, H):

@@ -270,8 +270,59 @@ int oracle_attn_rows_ex(int B, int T, int H, int d, const double *q, const doubl
  * formula): the Quest score is that upper bound; K counts the blocks chosen
  * besides the first and the local one; the blocks hold the augmented keys.
  * Output and log-sum-exp are those of one softmax over the attended keys
- * (scale as in R5).  Returns 0, or -1 on an argument error.
+ * (scale as in R5).
  */
+
+/* R9 block selection for query row t of (b, h): marks keep[0 .. c] (c = t/bs)
+ * and lists the picked candidates in picks[0 .. K) in the order they are
+ * taken (-1 when fewer than K candidates exist).  *gap receives the score of
+ * the last pick minus the best score left out (+inf when nothing is left out
+ * or nothing is picked), how far the selection is from a tie. */
+static void topk_pick(int T, int H, int d, const double *qrow, const double *kt, int b, int h, long t,
+                      int bs, int K, int mode, double *score, unsigned char *keep, int *picks, double *gap)
+{
+    const long c = t / bs;
+    for (long blk = 0; blk <= c; ++blk) keep[blk] = (blk == 0 || blk == c);
+    /* scores of the candidate blocks 1 .. c-1 (whole blocks, all j < c*bs <= t) */
+    for (long blk = 1; blk < c; ++blk) {
+        double sc = 0.0;
+        for (int ch = 0; ch < d; ++ch) {
+            double lo = INFINITY, hi = -INFINITY, sum = 0.0;
+            for (long j = blk * bs; j < (blk + 1) * bs; ++j) {
+                const double x = kt[idx4(T, H, d, b, j, h, ch)];
+                if (x < lo) lo = x;
+                if (x > hi) hi = x;
+                sum += x;
+            }
+            if (mode == 0) {
+                const double a1 = qrow[ch] * lo, a2 = qrow[ch] * hi;
+                sc += a1 > a2 ? a1 : a2;
+            } else {
+                sc += qrow[ch] * (sum / (double)bs);
+            }
+        }
+        score[blk] = sc;
+    }
+    /* the K best candidates, ties to the lower index */
+    double last = INFINITY;
+    for (int pick = 0; pick < K; ++pick) {
+        long best = -1;
+        for (long blk = 1; blk < c; ++blk)
+            if (!keep[blk] && (best < 0 || score[blk] > score[best])) best = blk;
+        if (picks) picks[pick] = (int)best;
+        if (best < 0) continue;
+        keep[best] = 1;
+        last = score[best];
+    }
+    if (gap) {
+        double rest = -INFINITY;
+        for (long blk = 1; blk < c; ++blk)
+            if (!keep[blk] && score[blk] > rest) rest = score[blk];
+        *gap = (rest == -INFINITY || last == INFINITY) ? INFINITY : last - rest;
+    }
+}
+
+/* Rows of top-k block attention.  Returns 0, or -1 on an argument error. */
 int oracle_attn_rows_topk(int B, int T, int H, int d, const double *q, const double *kt,
                           const double *vt, int bs, int K, int mode, double scale, long nrows,
                           const int64_t *rows, double *o, double *lse)
@@ -287,8 +338,8 @@ int oracle_attn_rows_topk(int B, int T, int H, int d, const double *q, const dou
     {
         long *js = (long *)malloc(sizeof(long) * (size_t)(T > 0 ? T : 1));
         double *z = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
-        double *score = (double *)malloc(sizeof(double) * (size_t)nblk);
-        unsigned char *keep = (unsigned char *)malloc((size_t)nblk);
+        double *score = (double *)malloc(sizeof(double) * (size_t)(nblk > 0 ? nblk : 1));
+        unsigned char *keep = (unsigned char *)malloc((size_t)(nblk > 0 ? nblk : 1));
         if (!js || !z || !score || !keep) {
 #pragma omp atomic write
             err = 1;
@@ -299,42 +350,46 @@ int oracle_attn_rows_topk(int B, int T, int H, int d, const double *q, const dou
             int b = (int)rows[3 * r], h = (int)rows[3 * r + 1];
             long t = (long)rows[3 * r + 2];
             const double *qrow = q + idx4(T, H, d, b, t, h, 0);
-            const long c = t / bs;
-            for (long blk = 0; blk <= c; ++blk) keep[blk] = (blk == 0 || blk == c);
-            /* scores of the candidate blocks 1 .. c-1 (whole blocks, all j < c*bs <= t) */
-            for (long blk = 1; blk < c; ++blk) {
-                double sc = 0.0;
-                for (int ch = 0; ch < d; ++ch) {
-                    double lo = INFINITY, hi = -INFINITY, sum = 0.0;
-                    for (long j = blk * bs; j < (blk + 1) * bs; ++j) {
-                        const double x = kt[idx4(T, H, d, b, j, h, ch)];
-                        if (x < lo) lo = x;
-                        if (x > hi) hi = x;
-                        sum += x;
-                    }
-                    if (mode == 0) {
-                        const double a1 = qrow[ch] * lo, a2 = qrow[ch] * hi;
-                        sc += a1 > a2 ? a1 : a2;
-                    } else {
-                        sc += qrow[ch] * (sum / (double)bs);
-                    }
-                }
-                score[blk] = sc;
-            }
-            /* the K best candidates, ties to the lower index */
-            for (int pick = 0; pick < K; ++pick) {
-                long best = -1;
-                for (long blk = 1; blk < c; ++blk)
-                    if (!keep[blk] && (best < 0 || score[blk] > score[best])) best = blk;
-                if (best < 0) break;
-                keep[best] = 1;
-            }
+            topk_pick(T, H, d, qrow, kt, b, h, t, bs, K, mode, score, keep, NULL, NULL);
             long n = 0;
             for (long j = 0; j <= t; ++j)
                 if (keep[j / bs]) js[n++] = j;
             softmax_over(T, H, d, qrow, kt, vt, b, h, js, n, scale, o + (size_t)r * (size_t)d, &lse[r], z);
         }
         free(js); free(z); free(score); free(keep);
+    }
+    return err ? -1 : 0;
+}
+
+/* The R9 selection itself for each row: sel (nrows x K, in pick order, -1
+ * padded) and gap (nrows), as topk_pick defines them.  Returns 0 or -1. */
+int oracle_topk_select(int B, int T, int H, int d, const double *q, const double *kt, int bs, int K,
+                       int mode, long nrows, const int64_t *rows, int *sel, double *gap)
+{
+    if (bs < 1 || K < 0 || (mode != 0 && mode != 1)) return -1;
+    for (long r = 0; r < nrows; ++r) {
+        int64_t b = rows[3 * r], h = rows[3 * r + 1], t = rows[3 * r + 2];
+        if (b < 0 || b >= B || h < 0 || h >= H || t < 0 || t >= T) return -1;
+    }
+    const long nblk = (T + bs - 1) / bs;
+    int err = 0;
+#pragma omp parallel
+    {
+        double *score = (double *)malloc(sizeof(double) * (size_t)(nblk > 0 ? nblk : 1));
+        unsigned char *keep = (unsigned char *)malloc((size_t)(nblk > 0 ? nblk : 1));
+        if (!score || !keep) {
+#pragma omp atomic write
+            err = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (long r = 0; r < nrows; ++r) {
+            if (err) continue;
+            int b = (int)rows[3 * r], h = (int)rows[3 * r + 1];
+            long t = (long)rows[3 * r + 2];
+            topk_pick(T, H, d, q + idx4(T, H, d, b, t, h, 0), kt, b, h, t, bs, K, mode, score, keep,
+                      sel + (size_t)r * (size_t)K, &gap[r]);
+        }
+        free(score); free(keep);
     }
     return err ? -1 : 0;
 }

@@ -6,7 +6,8 @@ merge, a dropped scale, a transposed operand, a gate one step late, a decode
 that ignores the per-head recurrence flag, a fixed grid on the wrong residue
 or without the query's own key, a dedupe that keeps the shared keys,
 a top-k block selection with a one-sided bound, a dropped first or local
-block, ties to the wrong block or one block too many).  It is compiled into a temporary
+block, ties to the wrong block, one block too many or a selection gap of
+the wrong sign).  It is compiled into a temporary
 directory and the pin suite is run against it in a subprocess; the suite must
 fail.  The shipped oracle is never modified.
 """
@@ -43,6 +44,7 @@ MUTANTS = {
     "topk_first_block_dropped": ("keep[blk] = (blk == 0 || blk == c);", "keep[blk] = (blk == c);"),
     "topk_ties_to_higher_block": ("(best < 0 || score[blk] > score[best])", "(best < 0 || score[blk] >= score[best])"),
     "topk_one_block_too_many": ("for (int pick = 0; pick < K; ++pick)", "for (int pick = 0; pick <= K; ++pick)"),
+    "topk_gap_sign": ("last - rest;", "rest - last;"),
 }
 
 

@@ -446,6 +446,60 @@ def test_topk_equal_scores_go_to_the_lower_block(mode):
     np.testing.assert_allclose(o, ro, rtol=1e-12, atol=1e-12)
 
 
+@pytest.mark.parametrize("mode", ["quest", "moba"])
+def test_topk_selection_is_what_the_rows_attend(mode):
+    # the exported selection and the attention rows agree: each row equals a
+    # softmax over the first block, its own block and the selected ones
+    B, T, H, d, bs, K = 1, 41, 1, 4, 4, 2
+    q, k, v = rand_qkv(B, T, H, d)
+    rows = topk_rows(T)
+    o, lse = oracle.attn_rows_topk(q, k, v, bs, K, mode, rows)
+    sel, gap = oracle.topk_select(q, k, bs, K, mode, rows)
+    sets = []
+    for t in range(T):
+        blocks = {0, t // bs} | {int(x) for x in sel[t] if x >= 0}
+        sets.append({j for j in range(t + 1) if j // bs in blocks})
+        ncand = max(0, t // bs - 1)
+        assert (sel[t] >= 0).sum() == min(K, ncand)
+        assert all(1 <= x < t // bs for x in sel[t] if x >= 0)
+    ro, rl = masked_rows(q[0, :, 0], k[0, :, 0], v[0, :, 0], sets, 1 / math.sqrt(d))
+    np.testing.assert_allclose(o, ro, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse, rl, rtol=1e-12, atol=1e-12)
+
+
+def test_topk_selection_with_blocks_of_one_key_sorts_dot_products():
+    # one-key blocks: picks in descending q.k among keys 1 .. t-1, and the gap
+    # is the K-th largest minus the (K+1)-th
+    B, T, H, d, K = 1, 23, 1, 5, 3
+    q, k, _ = rand_qkv(B, T, H, d)
+    sel, gap = oracle.topk_select(q, k, 1, K, "moba", topk_rows(T))
+    for t in range(T):
+        dots = {j: float(k[0, j, 0] @ q[0, t, 0]) for j in range(1, t)}
+        order = sorted(dots, key=lambda j: -dots[j])
+        want = order[:K] + [-1] * (K - len(order[:K]))
+        assert list(sel[t]) == want
+        if len(order) > K:
+            assert abs(gap[t] - (dots[order[K - 1]] - dots[order[K]])) < 1e-12
+        else:
+            assert gap[t] == np.inf
+
+
+def test_topk_selection_worked_example():
+    # the hand-worked blocks of test_topk_quest_and_moba_worked_example:
+    #   row 7: Quest 3 vs 2.5 -> picks block 1, gap 0.5; MoBA 2.5 vs -1 -> block 2, gap 3.5
+    #   row 6: Quest 5 vs -2 -> block 1, gap 7;         MoBA 1 vs -2 -> block 1, gap 3
+    k = np.zeros((1, 8, 1, 2))
+    k[0, :, 0] = [[0.3, -0.2], [0.1, 0.4], [-3, 0], [5, 0], [-2, 1], [-2, 1], [0.2, 0.2], [-0.1, 0.3]]
+    q = np.zeros((1, 8, 1, 2))
+    q[0, 6, 0] = [1, 0]
+    q[0, 7, 0] = [-1, 0.5]
+    rows = [(0, 0, 6), (0, 0, 7)]
+    sel, gap = oracle.topk_select(q, k, 2, 1, "quest", rows)
+    assert sel.tolist() == [[1], [1]] and np.allclose(gap, [7.0, 0.5], rtol=0, atol=1e-12)
+    sel, gap = oracle.topk_select(q, k, 2, 1, "moba", rows)
+    assert sel.tolist() == [[1], [2]] and np.allclose(gap, [3.0, 3.5], rtol=0, atol=1e-12)
+
+
 def test_topk_invalid_arguments_are_rejected():
     q, k, v = rand_qkv(1, 4, 1, 2)
     for bs, K, rows in [(0, 1, [(0, 0, 1)]), (2, -1, [(0, 0, 1)]), (2, 1, [(0, 0, 4)])]:
