@@ -94,7 +94,8 @@ typedef enum {
     RAT_OP_ATTN = 1,          /* rat_dilated_attn_prefill */
     RAT_OP_MIX = 2,           /* rat_mix_prefill with kt = vt = NULL (K~/V~ kept in ws) */
     RAT_OP_MIX_CALLER_KV = 3, /* rat_mix_prefill with caller-provided kt and vt */
-    RAT_OP_DECODE = 4         /* rat_decode_step */
+    RAT_OP_DECODE = 4,        /* rat_decode_step */
+    RAT_OP_TOPK_DECODE = 5    /* rat_topk_decode_step */
 } rat_op;
 
 /*
@@ -248,6 +249,54 @@ RAT_API rat_status rat_decode_step_noalloc(const rat_cfg *cfg, const void *q, co
                                            const void *g, float *state_k, float *state_v, void *cache_k,
                                            void *cache_v, int cache_cap, const int32_t *pos, void *o,
                                            float *lse, rat_stream_t stream);
+
+/*
+ * Top-k block attention for decoding over the augmented keys/values (RAT+
+ * Figure 3 and Tables 17-18; Exponentially Decaying Memory, section 2.2,
+ * sparse inference settings).  Keys are grouped in blocks of `block`
+ * consecutive positions.  The query at t (block c = t / block) attends, in one
+ * softmax, to the rows j <= t of block 0, of block c, and of the `topk` best
+ * of blocks 1 .. c-1 (all of them when there are fewer), ranked by
+ *   RAT_TOPK_QUEST  sum_ch max(q_ch * kmin_ch, q_ch * kmax_ch) over the block's
+ *                   per-channel key range (an upper bound of q.k in the block)
+ *   RAT_TOPK_MOBA   q . mean of the block's keys
+ * with equal scores going to the lower block.  The cache is the dense layout:
+ * every head must have dil = 1 and win = 0 (the sparse selection replaces
+ * dilation and window), so position j of a head is row j.
+ *
+ * Block statistics: `stats` is caller memory of rat_topk_stats_size() bytes,
+ * fp32 [B, H, ceil(cache_cap / block), 2, d]: per block the channel minima and
+ * maxima (Quest), or the channel sums and zeros (MoBA), of the cached keys.
+ * Limits: 1 <= block; 0 <= topk <= 64; ceil(cache_cap / block) <= 16384.
+ */
+typedef enum { RAT_TOPK_QUEST = 0, RAT_TOPK_MOBA = 1 } rat_topk_mode;
+
+/* Bytes of the block-statistics buffer (0 when an argument is invalid). */
+RAT_API size_t rat_topk_stats_size(const rat_cfg *cfg, int block, int cache_cap);
+
+/*
+ * Statistics of the blocks of positions 0 .. cfg->T - 1 (the tokens a prefill
+ * wrote into cache_k with rat_scan_prefill), in `mode`; a last partial block
+ * covers the positions it has.  Blocks at or past cfg->T are left as they are.
+ */
+RAT_API rat_status rat_topk_build_stats(const rat_cfg *cfg, int block, int mode, const void *cache_k,
+                                        int cache_cap, float *stats, rat_stream_t stream);
+
+/*
+ * One decode step with top-k block attention.  As rat_decode_step (the state
+ * update, the append of the new row at row t = pos[b], ragged positions, the
+ * error behaviour), plus: the new key is folded into its block's statistics,
+ * which must hold blocks 0 .. c of the positions before t; `sel` (nullable,
+ * device int32 [B, H, topk]) receives the selected blocks in selection order,
+ * -1 where fewer were available.  ws: rat_workspace_size(cfg,
+ * RAT_OP_TOPK_DECODE, cache_cap) bytes.  One kernel per step, no other CUDA
+ * call after the first on a device (graph-capturable).
+ */
+RAT_API rat_status rat_topk_decode_step(const rat_cfg *cfg, int block, int topk, int mode, const void *q,
+                                        const void *k, const void *v, const void *g, float *state_k,
+                                        float *state_v, void *cache_k, void *cache_v, int cache_cap,
+                                        float *stats, const int32_t *pos, void *o, float *lse, int32_t *sel,
+                                        void *ws, size_t ws_bytes, rat_stream_t stream);
 
 /*
  * Synchronises `stream`, returns the first device-side error recorded in `ws`

@@ -20,14 +20,15 @@ LIB_PATH = os.path.join(HERE, "librat.so")
 
 RAT_OK, RAT_ERR_INVALID, RAT_ERR_UNSUPPORTED, RAT_ERR_CUDA, RAT_ERR_TIMEOUT, RAT_ERR_WORKSPACE = range(6)
 RAT_F32, RAT_BF16 = 0, 1
-RAT_OP_SCAN, RAT_OP_ATTN, RAT_OP_MIX, RAT_OP_MIX_CALLER_KV, RAT_OP_DECODE = range(5)
+RAT_OP_SCAN, RAT_OP_ATTN, RAT_OP_MIX, RAT_OP_MIX_CALLER_KV, RAT_OP_DECODE, RAT_OP_TOPK_DECODE = range(6)
+RAT_TOPK_QUEST, RAT_TOPK_MOBA = 0, 1
 RAT_FLAG_GRID_DILATION = 1
 RAT_FLAG_DEDUPE = 2
 
 EXPORTS = ["rat_workspace_size", "rat_workspace_init", "rat_cache_rows", "rat_scan_prefill",
            "rat_dilated_attn_prefill", "rat_mix_prefill", "rat_decode_step", "rat_check_status",
            "rat_status_string", "rat_last_error", "rat_version", "rat_launch_count", "rat_debug_set_scan_stall",
-           "rat_decode_step_noalloc"]
+           "rat_decode_step_noalloc", "rat_topk_stats_size", "rat_topk_build_stats", "rat_topk_decode_step"]
 
 
 class RatError(RuntimeError):
@@ -70,6 +71,10 @@ def load_library(path=LIB_PATH):
     lib.rat_mix_prefill.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P]
     lib.rat_decode_step.argtypes = [cfgp, P, P, P, P, P, P, P, P, I, P, P, P, P, S, P]
     lib.rat_decode_step_noalloc.argtypes = [cfgp, P, P, P, P, P, P, P, P, I, P, P, P, P]
+    lib.rat_topk_stats_size.argtypes = [cfgp, I, I]
+    lib.rat_topk_stats_size.restype = S
+    lib.rat_topk_build_stats.argtypes = [cfgp, I, I, P, I, P, P]
+    lib.rat_topk_decode_step.argtypes = [cfgp, I, I, I, P, P, P, P, P, P, P, P, I, P, P, P, P, P, P, S, P]
     lib.rat_check_status.argtypes = [P, P]
     lib.rat_status_string.argtypes = [I]
     lib.rat_status_string.restype = ctypes.c_char_p
@@ -79,7 +84,8 @@ def load_library(path=LIB_PATH):
     lib.rat_launch_count.restype = ctypes.c_longlong
     lib.rat_debug_set_scan_stall.argtypes = [P, S, ctypes.c_int64, ctypes.c_int64, P]
     for name in ("rat_workspace_init", "rat_scan_prefill", "rat_dilated_attn_prefill", "rat_mix_prefill",
-                 "rat_decode_step", "rat_check_status", "rat_debug_set_scan_stall", "rat_decode_step_noalloc"):
+                 "rat_decode_step", "rat_check_status", "rat_debug_set_scan_stall", "rat_decode_step_noalloc",
+                 "rat_topk_build_stats", "rat_topk_decode_step"):
         getattr(lib, name).restype = I
     _lib = lib
     return lib
@@ -252,6 +258,46 @@ def rat_decode_step_noalloc(cfg, q, k, v, g, state_k, state_v, cache_k, cache_v,
             _ptr(pos, "pos", torch.int32, (c.B,)), _ptr(o, "o", dt, tok),
             _ptr(lse, "lse", torch.float32, (c.B, c.H), True), _stream(stream)]
     _check(load_library().rat_decode_step_noalloc(cfg.ref(), *args), "rat_decode_step_noalloc")
+
+
+def rat_topk_stats_size(cfg, block, cache_cap):
+    n = load_library().rat_topk_stats_size(cfg.ref(), int(block), int(cache_cap))
+    if n == 0:
+        raise RatError(RAT_ERR_INVALID, "rat_topk_stats_size: " + load_library().rat_last_error().decode())
+    return n
+
+
+def topk_stats_shape(cfg, block, cache_cap):
+    """Shape of the fp32 block-statistics tensor: [B, H, ceil(cap / block), 2, d]."""
+    c = cfg.c
+    return (c.B, c.H, -(-int(cache_cap) // int(block)), 2, c.d)
+
+
+def rat_topk_build_stats(cfg, block, mode, cache_k, cache_cap, stats, stream=None):
+    c = cfg.c
+    R = rat_cache_rows(cfg, cache_cap)
+    args = [int(block), int(mode), _ptr(cache_k, "cache_k", cfg.torch_dtype, (c.B, c.H, R, c.d)), int(cache_cap),
+            _ptr(stats, "stats", torch.float32, topk_stats_shape(cfg, block, cache_cap)), _stream(stream)]
+    _check(load_library().rat_topk_build_stats(cfg.ref(), *args), "rat_topk_build_stats")
+
+
+def rat_topk_decode_step(cfg, block, topk, mode, q, k, v, g, state_k, state_v, cache_k, cache_v, cache_cap, stats,
+                         pos, o, lse=None, sel=None, ws=None, stream=None):
+    c = cfg.c
+    tok = (c.B, c.H, c.d)
+    dt = cfg.torch_dtype
+    R = rat_cache_rows(cfg, cache_cap)
+    cshape = (c.B, c.H, R, c.d)
+    args = [int(block), int(topk), int(mode),
+            _ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, tok),
+            _ptr(state_k, "state_k", torch.float32, tok), _ptr(state_v, "state_v", torch.float32, tok),
+            _ptr(cache_k, "cache_k", dt, cshape), _ptr(cache_v, "cache_v", dt, cshape), int(cache_cap),
+            _ptr(stats, "stats", torch.float32, topk_stats_shape(cfg, block, cache_cap)),
+            _ptr(pos, "pos", torch.int32, (c.B,)), _ptr(o, "o", dt, tok),
+            _ptr(lse, "lse", torch.float32, (c.B, c.H), True),
+            _ptr(sel, "sel", torch.int32, (c.B, c.H, int(topk)), True),
+            _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream)]
+    _check(load_library().rat_topk_decode_step(cfg.ref(), *args), "rat_topk_decode_step")
 
 
 def rat_check_status(ws, stream=None):

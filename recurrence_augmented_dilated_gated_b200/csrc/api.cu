@@ -412,9 +412,11 @@ const char *rat_status_string(rat_status s) {
 }
 
 size_t rat_workspace_size(const rat_cfg *cfg, int op, int cache_cap) {
-    if (op < RAT_OP_SCAN || op > RAT_OP_DECODE) return 0;
-    if (check_cfg(cfg, op != RAT_OP_DECODE) != RAT_OK) return 0;
-    if (op == RAT_OP_DECODE && cache_cap < 1) return 0;
+    if (op < RAT_OP_SCAN || op > RAT_OP_TOPK_DECODE) return 0;
+    const bool dec = op == RAT_OP_DECODE || op == RAT_OP_TOPK_DECODE;
+    if (check_cfg(cfg, !dec) != RAT_OK) return 0;
+    if (dec && cache_cap < 1) return 0;
+    if (op == RAT_OP_TOPK_DECODE) return sizeof(WsHeader);   // the status word only
     return layout(cfg, op, cache_cap).total;
 }
 
@@ -536,6 +538,85 @@ rat_status rat_decode_step(const rat_cfg *cfg, const void *q, const void *k, con
     if (ez != cudaSuccess) return cuda_fail(ez, "cudaMemsetAsync(decode counters)");
     cudaError_t e = launch_decode(p, cfg->dtype, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    return RAT_OK;
+}
+
+// ---------------------------------------------------------- top-k block decode
+
+namespace {
+
+rat_status check_topk(const rat_cfg *c, int block, int topk, int mode, int cap) {
+    rat_status st = check_cfg(c, false);
+    if (st != RAT_OK) return st;
+    if (block < 1) return fail(RAT_ERR_INVALID, "block %d < 1", block);
+    if (topk < 0 || topk > kTopkMaxK) return fail(RAT_ERR_INVALID, "topk %d outside [0, %d]", topk, kTopkMaxK);
+    if (mode != RAT_TOPK_QUEST && mode != RAT_TOPK_MOBA) return fail(RAT_ERR_INVALID, "top-k mode %d", mode);
+    if (cap < 1) return fail(RAT_ERR_INVALID, "cache_cap %d < 1", cap);
+    if ((cap + (long long)block - 1) / block > kTopkMaxBlocks)
+        return fail(RAT_ERR_UNSUPPORTED, "ceil(cache_cap / block) exceeds %d blocks", kTopkMaxBlocks);
+    for (int h = 0; h < c->H; ++h)
+        if (c->dil[h] != 1 || c->win[h] != 0)
+            return fail(RAT_ERR_INVALID, "top-k decoding needs dil = 1 and win = 0 (head %d)", h);
+    return RAT_OK;
+}
+
+TopkParams topk_params(const rat_cfg *c, int block, int topk, int mode, int cap, float *stats) {
+    TopkParams p;
+    memset(&p, 0, sizeof(p));
+    p.cache_R = cache_rows(c, cap);
+    p.cap = cap; p.B = c->B; p.H = c->H; p.d = c->d;
+    p.bs = block; p.K = topk; p.mode = mode;
+    p.nblk = (int)((cap + (long long)block - 1) / block);
+    p.stats = stats;
+    p.scale_log2 = scale_of(c) * 1.4426950408889634f;
+    for (int h = 0; h < c->H; ++h) p.recur[h] = head_recur(c, h) ? 1 : 0;
+    return p;
+}
+
+}  // namespace
+
+size_t rat_topk_stats_size(const rat_cfg *cfg, int block, int cache_cap) {
+    if (check_topk(cfg, block, 0, RAT_TOPK_QUEST, cache_cap) != RAT_OK) return 0;
+    const size_t nblk = (size_t)((cache_cap + (long long)block - 1) / block);
+    return (size_t)cfg->B * cfg->H * nblk * 2 * cfg->d * sizeof(float);
+}
+
+rat_status rat_topk_build_stats(const rat_cfg *cfg, int block, int mode, const void *cache_k, int cache_cap,
+                                float *stats, rat_stream_t stream) {
+    rat_status st = check_topk(cfg, block, 0, mode, cache_cap);
+    if (st != RAT_OK) return st;
+    if (cfg->T < 0 || cfg->T > cache_cap) return fail(RAT_ERR_INVALID, "T %d outside [0, cache_cap]", cfg->T);
+    if ((size_t)cfg->B * cfg->T == 0) return RAT_OK;
+    CHECK_PTR(cache_k, "cache_k"); CHECK_PTR(stats, "stats");
+    TopkParams p = topk_params(cfg, block, 0, mode, cache_cap, stats);
+    p.cache[0] = const_cast<void *>(cache_k);
+    cudaError_t e = launch_topk_stats(p, cfg->T, cfg->dtype, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "top-k statistics launch");
+    return RAT_OK;
+}
+
+rat_status rat_topk_decode_step(const rat_cfg *cfg, int block, int topk, int mode, const void *q, const void *k,
+                                const void *v, const void *g, float *state_k, float *state_v, void *cache_k,
+                                void *cache_v, int cache_cap, float *stats, const int32_t *pos, void *o,
+                                float *lse, int32_t *sel, void *ws, size_t ws_bytes, rat_stream_t stream) {
+    rat_status st = check_topk(cfg, block, topk, mode, cache_cap);
+    if (st != RAT_OK) return st;
+    if (cfg->B == 0) return RAT_OK;
+    CHECK_PTR(q, "q"); CHECK_PTR(k, "k"); CHECK_PTR(v, "v"); CHECK_PTR(g, "g");
+    CHECK_PTR(state_k, "state_k"); CHECK_PTR(state_v, "state_v");
+    CHECK_PTR(cache_k, "cache_k"); CHECK_PTR(cache_v, "cache_v"); CHECK_PTR(stats, "stats");
+    CHECK_PTR(pos, "pos"); CHECK_PTR(o, "o"); CHECK_OPT(lse, "lse"); CHECK_OPT(sel, "sel");
+    Layout L;
+    st = check_ws(cfg, RAT_OP_TOPK_DECODE, cache_cap, ws, ws_bytes, &L);
+    if (st != RAT_OK) return st;
+    TopkParams p = topk_params(cfg, block, topk, mode, cache_cap, stats);
+    p.q = q; p.k = k; p.v = v; p.g = g;
+    p.state[0] = state_k; p.state[1] = state_v;
+    p.cache[0] = cache_k; p.cache[1] = cache_v;
+    p.pos = pos; p.o = o; p.lse = lse; p.sel = sel;
+    p.hdr = reinterpret_cast<WsHeader *>(ws);
+    cudaError_t e = launch_topk_decode(p, cfg->dtype, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "top-k decode launch");
     return RAT_OK;
 }
 

@@ -182,6 +182,27 @@ struct DecodeParams {
     WsHeader *hdr;
 };
 
+// -------------------------------------------------- top-k block decode (K6)
+constexpr int kTopkMaxK = 64;          // selected blocks per query, at most
+constexpr int kTopkMaxBlocks = 16384;  // blocks of one (b, h) cache, at most (scores in shared memory)
+
+struct TopkParams {
+    const void *q, *k, *v, *g;   // [B,H,d]
+    float *state[2];             // [B,H,d] fp32, in place
+    void *cache[2];              // [B,H,R,d], dense layout: position j at row j
+    float *stats;                // [B,H,nblk,2,d] fp32 block statistics
+    const int *pos;              // device [B]
+    void *o;                     // [B,H,d]
+    float *lse;                  // [B,H] or null
+    int *sel;                    // [B,H,K] selected blocks or null
+    long long cache_R;
+    int cap, B, H, d;
+    int bs, K, mode, nblk;       // block size, blocks to select, RAT_TOPK_*, ceil(cap / bs)
+    float scale_log2;
+    unsigned char recur[kMaxHeads];
+    WsHeader *hdr;
+};
+
 // Fills the per-head split plan, items_per_b and cache_R of `p` for a decode
 // step with capacity `cap` (host).  Returns the scratch bytes the step needs
 // after the workspace header: partials plus per-(b,h) counters.
@@ -203,5 +224,8 @@ bool encode_map_tokens(CUtensorMap *map, const void *base, int dtype, int B, int
 cudaError_t launch_final_of_plain_heads(const ScanParams &p, int dtype, cudaStream_t s);
 cudaError_t launch_attn_simt(const AttnParams &p, int dtype, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, int dtype, cudaStream_t s);
+// block statistics of positions [0, n_tok) of the cache
+cudaError_t launch_topk_stats(const TopkParams &p, int n_tok, int dtype, cudaStream_t s);
+cudaError_t launch_topk_decode(const TopkParams &p, int dtype, cudaStream_t s);
 
 }  // namespace rat

@@ -115,6 +115,25 @@ def test_unknown_flags_are_rejected(lib):
         assert lib.rat_workspace_size(cfg(flags=f).ref(), rat.RAT_OP_MIX, 0) > 0
 
 
+
+def test_topk_sizes_and_argument_checks(lib):
+    c = cfg(B=2, H=2, dil=[1, 1], win=[0, 0])
+    # statistics: [B, H, ceil(cap / block), 2, d] fp32
+    assert lib.rat_topk_stats_size(c.ref(), 64, 4000) == 2 * 2 * 63 * 2 * 128 * 4
+    assert lib.rat_topk_stats_size(cfg().ref(), 64, 4096) == 0          # dilated heads: not the dense layout
+    assert lib.rat_topk_stats_size(cfg(dil=[1, 1]).ref(), 64, 4096) == 0  # a window
+    assert lib.rat_topk_stats_size(c.ref(), 0, 4096) == 0
+    assert lib.rat_topk_stats_size(c.ref(), 1, 16385) == 0               # more blocks than the kernel holds
+    assert lib.rat_workspace_size(c.ref(), rat.RAT_OP_TOPK_DECODE, 4096) == 256
+    P = 16
+    for block, topk, mode in ((64, 65, 0), (64, -1, 0), (64, 4, 2), (0, 4, 0)):
+        rc = lib.rat_topk_decode_step(c.ref(), block, topk, mode, P, P, P, P, P, P, P, P, 4096, P, P, P, None,
+                                      None, 256, 256, None)
+        assert rc == rat.RAT_ERR_INVALID, (block, topk, mode)
+    rc = lib.rat_topk_build_stats(c.replace(T=5000).ref(), 64, 0, P, 4096, P, None)
+    assert rc == rat.RAT_ERR_INVALID     # more tokens than the cache holds
+
+
 def call_scan(lib, c, **ptrs):
     P = dict(k=16, v=16, g=16, init_k=None, init_v=None, kt=16, vt=16, fk=None, fv=None, ck=None, cv=None, cap=0,
              ws=256, wsb=1 << 40)

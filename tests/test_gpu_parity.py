@@ -579,6 +579,95 @@ def test_dedupe_decode_steps_every_element(grid, dtype):
                     recur=[0, 1, 1, 1], mu=2.0, seed=23, grid=grid, dedupe=True)
 
 
+# ------------------------------------------- top-k block attention for decoding
+
+
+def run_topk_case(B, T, steps, H, d, dtype, block, topk, mode, recur, seed, cap=None, margin=0.02):
+    """Prefill T tokens into a dense cache, build the block statistics, decode
+    `steps` tokens with rat_topk_decode_step; compare with the oracle's top-k
+    rows.  The block choice is an integer decision: the oracle takes it on its
+    K~ rounded to the cache's precision, as the kernel does, and rows whose
+    K-th and (K+1)-th block scores lie within `margin` (rounding could swap
+    them) are only checked for a valid selection."""
+    Tt = T + steps
+    cap = cap or Tt
+    q, k, v, g = inputs(B, Tt, H, d, dtype, mu=2.0, seed=seed)
+    cfg = make_cfg(B, T, H, d, dtype, [1] * H, [0] * H, recur)
+    R = rat.rat_cache_rows(cfg, cap)
+    ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
+    cv = torch.zeros_like(ck)
+    sk = torch.empty(B, H, d, device=DEV)
+    sv = torch.empty_like(sk)
+    ws = rat.workspace(cfg, rat.RAT_OP_SCAN)
+    rat.rat_scan_prefill(cfg, k[:, :T].contiguous(), v[:, :T].contiguous(), g[:, :T].contiguous(), None, None,
+                         None, None, sk, sv, ck, cv, cap, ws)
+    rat.rat_check_status(ws)
+    stats = torch.full(rat.topk_stats_shape(cfg, block, cap), float("nan"), device=DEV)
+    rat.rat_topk_build_stats(cfg, block, mode, ck, cap, stats)
+    wsd = rat.workspace(cfg, rat.RAT_OP_TOPK_DECODE, cap)
+    outs = []
+    for s in range(steps):
+        t = T + s
+        pos = torch.full((B,), t, dtype=torch.int32, device=DEV)
+        o = torch.empty(B, H, d, dtype=dtype, device=DEV)
+        lse = torch.empty(B, H, device=DEV)
+        sel = torch.empty(B, H, topk, dtype=torch.int32, device=DEV)
+        rat.rat_topk_decode_step(cfg, block, topk, mode, q[:, t].contiguous(), k[:, t].contiguous(),
+                                 v[:, t].contiguous(), g[:, t].contiguous(), sk, sv, ck, cv, cap, stats, pos, o,
+                                 lse, sel, wsd)
+        outs.append((o, lse, sel))
+    rat.rat_check_status(wsd)
+    kt, fk = oracle.scan(f64(k), f64(g), None, recur)
+    vt, fv = oracle.scan(f64(v), f64(g), None, recur)
+    ft = torch.float32 if dtype == torch.float32 else dtype
+    assert_close(ck[:, :, :Tt].transpose(1, 2), kt, dtype, "cache_k")
+    assert_close(cv[:, :, :Tt].transpose(1, 2), vt, dtype, "cache_v")
+    assert_close(sk, fk, ft, "state_k")
+    # the cache's precision for the oracle's keys and values
+    kq = torch.from_numpy(kt).to(dtype).double().numpy()
+    vq = torch.from_numpy(vt).to(dtype).double().numpy()
+    name = {rat.RAT_TOPK_QUEST: "quest", rat.RAT_TOPK_MOBA: "moba"}[mode]
+    rows = np.array([(b, h, t) for b in range(B) for h in range(H) for t in range(T, Tt)])
+    ro, rl = oracle.attn_rows_topk(f64(q), kq, vq, block, topk, name, rows)
+    rsel, gap = oracle.topk_select(f64(q), kq, block, topk, name, rows)
+    got_o = np.stack([f64(o) for o, _, _ in outs], axis=2).reshape(-1, d)      # (b, h, step) order
+    got_l = np.stack([f64(l) for _, l, _ in outs], axis=2).reshape(-1)
+    got_s = np.stack([x[2].cpu().numpy() for x in outs], axis=2).reshape(-1, topk)
+    clear = gap > margin
+    assert clear.mean() >= 0.6, "too many near-ties: %d of %d rows" % (int((~clear).sum()), len(clear))
+    for i in np.nonzero(clear)[0]:
+        assert sorted(got_s[i]) == sorted(rsel[i]), (rows[i], got_s[i], rsel[i])
+    assert_close(got_o[clear], ro[clear], dtype, "top-k o")
+    assert_close(got_l[clear], rl[clear], ft, "top-k lse")
+    for i in np.nonzero(~clear)[0]:   # a near-tie: any valid selection of distinct candidates
+        c = rows[i][2] // block
+        picked = [x for x in got_s[i] if x >= 0]
+        assert len(set(picked)) == len(picked) == min(topk, max(0, c - 1))
+        assert all(1 <= x < c for x in picked)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+def test_topk_decode_steps(mode, dtype, d):
+    # positions 1021 .. 1025 cross into a new 64-row block at 1024
+    run_topk_case(B=2, T=1021, steps=5, H=3, d=d, dtype=dtype, block=64, topk=4, mode=mode, recur=[0, 1, 1],
+                  seed=31 + mode)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_topk_decode_from_empty_history(mode):
+    # blocks of 4 from t = 1: no candidates, then fewer than K, then more
+    run_topk_case(B=2, T=1, steps=30, H=2, d=128, dtype=torch.bfloat16, block=4, topk=3, mode=mode,
+                  recur=[1, 0], seed=41, cap=40)
+
+
+def test_topk_decode_keeps_every_block_when_k_is_large():
+    # K >= number of candidates: the step is dense causal attention
+    run_topk_case(B=1, T=500, steps=3, H=2, d=128, dtype=torch.bfloat16, block=32, topk=64, mode=0,
+                  recur=[1, 1], seed=43)
+
+
 def test_decode_bad_position_is_reported():
     B, H, d = 2, 2, 64
     cfg = make_cfg(B, 1, H, d, torch.bfloat16, [2, 2], [0, 0])
