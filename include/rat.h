@@ -20,7 +20,8 @@
  * Definitions used by every entry point (the pages give the method at the
  * level of captions; these are the plain readings of them):
  *   recurrence   s_t = a_t * s_{t-1} + (1 - a_t) * x_t per channel, for x = k
- *                and x = v, with a_t = sigmoid(g_t) from one gate tensor g;
+ *                and x = v, with a_t = sigmoid(g_t) from one gate tensor g
+ *                (one per tensor with RAT_FLAG_SEPARATE_GATES);
  *                s_{-1} = init (zero when not given).  A head with recur = 0
  *                has a = 0: its augmented keys/values are the raw ones.
  *   dilation     query t attends to { j <= t : (t - j) mod D == 0 }.  With
@@ -123,6 +124,10 @@ typedef struct {
 /* A key in both the dilated set and the window counts once: the window part
  * skips the keys the dilated set holds (with D = 1 the window adds nothing). */
 #define RAT_FLAG_DEDUPE 2u
+/* Separate gates for keys and values: the gate tensor g holds two tensors of
+ * the usual shape, g[0] for the key recurrence and g[1] for the value
+ * recurrence ([2, B, T, H, d] in a prefill, [2, B, H, d] in a decode step). */
+#define RAT_FLAG_SEPARATE_GATES 4u
 
 /* Bytes of workspace `op` needs for `cfg` (cache_cap: decode capacity, else
  * ignored).  Returns 0 when cfg is invalid. */

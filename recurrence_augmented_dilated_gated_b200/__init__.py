@@ -24,6 +24,7 @@ RAT_OP_SCAN, RAT_OP_ATTN, RAT_OP_MIX, RAT_OP_MIX_CALLER_KV, RAT_OP_DECODE, RAT_O
 RAT_TOPK_QUEST, RAT_TOPK_MOBA = 0, 1
 RAT_FLAG_GRID_DILATION = 1
 RAT_FLAG_DEDUPE = 2
+RAT_FLAG_SEPARATE_GATES = 4
 
 EXPORTS = ["rat_workspace_size", "rat_workspace_init", "rat_cache_rows", "rat_scan_prefill",
            "rat_dilated_attn_prefill", "rat_mix_prefill", "rat_decode_step", "rat_check_status",
@@ -120,6 +121,11 @@ class Config:
     def ref(self):
         return ctypes.byref(self.c)
 
+    def gate_shape(self, tok):
+        """Shape of the gate tensor for token tensors of shape `tok` (a second,
+        leading axis of 2 with separate key and value gates)."""
+        return ((2,) + tuple(tok)) if self.c.flags & RAT_FLAG_SEPARATE_GATES else tuple(tok)
+
 
 def _ptr(t, name, dtype=None, shape=None, optional=False):
     if t is None:
@@ -192,7 +198,7 @@ def rat_scan_prefill(cfg, k, v, g, init_k=None, init_v=None, kt=None, vt=None, f
     tok = (c.B, c.T, c.H, c.d)
     st = (c.B, c.H, c.d)
     dt = cfg.torch_dtype
-    args = [_ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, tok),
+    args = [_ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
             _ptr(init_k, "init_k", torch.float32, st, True), _ptr(init_v, "init_v", torch.float32, st, True),
             _ptr(kt, "kt", dt, tok, True), _ptr(vt, "vt", dt, tok, True),
             _ptr(final_k, "final_k", torch.float32, st, True), _ptr(final_v, "final_v", torch.float32, st, True),
@@ -217,7 +223,7 @@ def rat_mix_prefill(cfg, q, k, v, g, init_k=None, init_v=None, o=None, lse=None,
     tok = (c.B, c.T, c.H, c.d)
     st = (c.B, c.H, c.d)
     dt = cfg.torch_dtype
-    args = [_ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, tok),
+    args = [_ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
             _ptr(init_k, "init_k", torch.float32, st, True), _ptr(init_v, "init_v", torch.float32, st, True),
             _ptr(o, "o", dt, tok), _ptr(lse, "lse", torch.float32, (c.B, c.H, c.T), True),
             _ptr(kt, "kt", dt, tok, True), _ptr(vt, "vt", dt, tok, True),
@@ -233,7 +239,7 @@ def rat_decode_step(cfg, q, k, v, g, state_k, state_v, cache_k, cache_v, cache_c
     dt = cfg.torch_dtype
     R = rat_cache_rows(cfg, cache_cap)
     cshape = (c.B, c.H, R, c.d)
-    args = [_ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, tok),
+    args = [_ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
             _ptr(state_k, "state_k", torch.float32, tok), _ptr(state_v, "state_v", torch.float32, tok),
             _ptr(cache_k, "cache_k", dt, cshape), _ptr(cache_v, "cache_v", dt, cshape), int(cache_cap),
             _ptr(pos, "pos", torch.int32, (c.B,)), _ptr(o, "o", dt, tok),
@@ -252,7 +258,7 @@ def rat_decode_step_noalloc(cfg, q, k, v, g, state_k, state_v, cache_k, cache_v,
     dt = cfg.torch_dtype
     R = rat_cache_rows(cfg, cache_cap)
     cshape = (c.B, c.H, R, c.d)
-    args = [_ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, tok),
+    args = [_ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
             _ptr(state_k, "state_k", torch.float32, tok), _ptr(state_v, "state_v", torch.float32, tok),
             _ptr(cache_k, "cache_k", dt, cshape), _ptr(cache_v, "cache_v", dt, cshape), int(cache_cap),
             _ptr(pos, "pos", torch.int32, (c.B,)), _ptr(o, "o", dt, tok),
@@ -289,7 +295,7 @@ def rat_topk_decode_step(cfg, block, topk, mode, q, k, v, g, state_k, state_v, c
     R = rat_cache_rows(cfg, cache_cap)
     cshape = (c.B, c.H, R, c.d)
     args = [int(block), int(topk), int(mode),
-            _ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, tok),
+            _ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
             _ptr(state_k, "state_k", torch.float32, tok), _ptr(state_v, "state_v", torch.float32, tok),
             _ptr(cache_k, "cache_k", dt, cshape), _ptr(cache_v, "cache_v", dt, cshape), int(cache_cap),
             _ptr(stats, "stats", torch.float32, topk_stats_shape(cfg, block, cache_cap)),

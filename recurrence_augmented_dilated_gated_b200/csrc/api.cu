@@ -73,7 +73,7 @@ rat_status check_cfg(const rat_cfg *c, bool need_T = true) {
     const double elems = (double)c->B * (need_T ? (double)c->T : 1.0) * c->H * c->d;
     if (elems >= 1099511627776.0) return fail(RAT_ERR_INVALID, "B*T*H*d too large");
     if (!(c->scale == c->scale)) return fail(RAT_ERR_INVALID, "scale is NaN");
-    if (c->flags & ~(RAT_FLAG_GRID_DILATION | RAT_FLAG_DEDUPE))
+    if (c->flags & ~(RAT_FLAG_GRID_DILATION | RAT_FLAG_DEDUPE | RAT_FLAG_SEPARATE_GATES))
         return fail(RAT_ERR_INVALID, "unknown flags 0x%x", c->flags);
     return RAT_OK;
 }
@@ -181,6 +181,24 @@ rat_status empty_prefill_state(const rat_cfg *c, const float *ik, const float *i
     return RAT_OK;
 }
 
+bool separate_gates(const rat_cfg *c) { return (c->flags & RAT_FLAG_SEPARATE_GATES) != 0; }
+
+// One scan launch: tensor maps of its operands, zeroed ticket and chunk flags.
+rat_status scan_pass(const rat_cfg *c, const Layout &L, ScanParams &p, char *ws, cudaStream_t s) {
+    // the one-tensor form reads slot 1 of neither list: repeat slot 0 there
+    const void *srcs[5] = {p.x[0], p.x[1] ? p.x[1] : p.x[0], p.g, p.out[0], p.out[1] ? p.out[1] : p.out[0]};
+    p.use_tma_out = p.out[0] != nullptr ? 1 : 0;
+    for (int i = 0; i < (p.use_tma_out ? 5 : 3); ++i)
+        if (!encode_map_tokens(&p.tmap[i], srcs[i], c->dtype, c->B, c->T, c->H, c->d, p.chunk_len))
+            return fail(RAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (scan operand %d)", i);
+    // zero the ticket and the chunk flags (one contiguous range)
+    cudaError_t e = cudaMemsetAsync(ws + L.ticket, 0, L.agg - L.ticket, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(scan flags)");
+    e = launch_scan(p, c->dtype, s);
+    if (e != cudaSuccess) return cuda_fail(e, "scan launch");
+    return RAT_OK;
+}
+
 // Scan of the selected heads into kt/vt and/or the cache.
 rat_status run_scan(const rat_cfg *c, const Layout &L, const void *k, const void *v, const void *g,
                     const float *ik, const float *iv, void *kt, void *vt, float *fk, float *fv,
@@ -218,22 +236,23 @@ rat_status run_scan(const rat_cfg *c, const Layout &L, const void *k, const void
     p.nslices = c->B * n;
     p.nchunks = L.nchunks;
     p.chunk_len = scan_chunk_len(c->d);
-    const void *srcs[5] = {k, v, g, kt, vt};
-    p.use_tma_out = kt != nullptr ? 1 : 0;
-    for (int i = 0; i < (p.use_tma_out ? 5 : 3); ++i)
-        if (!encode_map_tokens(&p.tmap[i], srcs[i], c->dtype, c->B, c->T, c->H, c->d, p.chunk_len))
-            return fail(RAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (scan operand %d)", i);
     p.ticket = reinterpret_cast<unsigned *>(ws + L.ticket);
     p.flags = reinterpret_cast<int *>(ws + L.flags);
     p.agg = reinterpret_cast<float *>(ws + L.agg);
     p.incl = reinterpret_cast<float *>(ws + L.incl);
     p.hdr = reinterpret_cast<WsHeader *>(ws);
-    // zero the ticket and the chunk flags (one contiguous range)
-    cudaError_t e = cudaMemsetAsync(ws + L.ticket, 0, L.agg - L.ticket, s);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(scan flags)");
-    e = launch_scan(p, c->dtype, s);
-    if (e != cudaSuccess) return cuda_fail(e, "scan launch");
-    return RAT_OK;
+    if (!separate_gates(c)) return scan_pass(c, L, p, ws, s);
+    // separate gates: the keys with g[0], then the values with g[1], each in
+    // the one-tensor form of the scan (ordered on the stream, one workspace)
+    ScanParams pk = p, pv = p;
+    pk.one = pv.one = 1;
+    pk.x[1] = nullptr; pk.init[1] = nullptr; pk.out[1] = nullptr; pk.fin[1] = nullptr; pk.cache[1] = nullptr;
+    pv.x[0] = v; pv.init[0] = iv; pv.out[0] = vt; pv.fin[0] = fv; pv.cache[0] = cv;
+    pv.x[1] = nullptr; pv.init[1] = nullptr; pv.out[1] = nullptr; pv.fin[1] = nullptr; pv.cache[1] = nullptr;
+    pv.g = static_cast<const char *>(g) + (size_t)c->B * c->T * c->H * c->d * elt_size(c->dtype);
+    rat_status st = scan_pass(c, L, pk, ws, s);
+    if (st != RAT_OK) return st;
+    return scan_pass(c, L, pv, ws, s);
 }
 
 // Kind of a head's dilated part on the tensor cores: the residue subsequences,
@@ -566,6 +585,7 @@ TopkParams topk_params(const rat_cfg *c, int block, int topk, int mode, int cap,
     p.cache_R = cache_rows(c, cap);
     p.cap = cap; p.B = c->B; p.H = c->H; p.d = c->d;
     p.bs = block; p.K = topk; p.mode = mode;
+    p.sep = separate_gates(c) ? 1 : 0;
     p.nblk = (int)((cap + (long long)block - 1) / block);
     p.stats = stats;
     p.scale_log2 = scale_of(c) * 1.4426950408889634f;

@@ -269,12 +269,16 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         // loaded now and used after the old rows, so their latency overlaps
         // the stream (channel tid; kCompute >= D)
         static_assert(kCompute >= D, "one channel per scoring thread");
-        float in_k = 0.f, in_v = 0.f, in_g = 0.f, st_k = 0.f, st_v = 0.f;
+        float in_k = 0.f, in_v = 0.f, in_g = 0.f, in_gv = 0.f, st_k = 0.f, st_v = 0.f;
         const size_t e_new = bh * D + tid;
         if (last && tid < D) {
             in_k = (float)static_cast<const T *>(p.k)[e_new];
             in_v = (float)static_cast<const T *>(p.v)[e_new];
-            if (p.recur[h]) in_g = (float)static_cast<const T *>(p.g)[e_new];
+            if (p.recur[h]) {
+                in_g = (float)static_cast<const T *>(p.g)[e_new];
+                // separate gates: the value gate is the second [B,H,d] tensor
+                in_gv = p.sep ? (float)static_cast<const T *>(p.g)[(size_t)p.B * p.H * D + e_new] : in_g;
+            }
             st_k = p.state[0][e_new];
             st_v = p.state[1][e_new];
         }
@@ -321,15 +325,23 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         if (last) {
             // step update and append of the new row (no item reads it this step)
             if (tid < D) {
-                float a = 0.f, oma = 1.f;
+                float a = 0.f, oma = 1.f, av = 0.f, omav = 1.f;
                 if (p.recur[h]) {
                     const float gl_ = fminf(fmaxf(in_g, -80.f), 80.f);
                     const float ex = expf(-gl_);
                     a = 1.f / (1.f + ex);
                     oma = ex * a;
+                    av = a;
+                    omav = oma;
+                    if (p.sep) {
+                        const float gv_ = fminf(fmaxf(in_gv, -80.f), 80.f);
+                        const float exv = expf(-gv_);
+                        av = 1.f / (1.f + exv);
+                        omav = exv * av;
+                    }
                 }
                 const float sk = a * st_k + oma * in_k;
-                const float sv = a * st_v + oma * in_v;
+                const float sv = av * st_v + omav * in_v;
                 p.state[0][e_new] = sk;
                 p.state[1][e_new] = sv;
                 long long row0, row1;
@@ -522,6 +534,7 @@ size_t decode_plan(const rat_cfg *c, int cap, DecodeParams *p) {
     }
     p->grid = (c->flags & RAT_FLAG_GRID_DILATION) ? 1 : 0;
     p->dedupe = (c->flags & RAT_FLAG_DEDUPE) ? 1 : 0;
+    p->sep = (c->flags & RAT_FLAG_SEPARATE_GATES) ? 1 : 0;
     p->item0[c->H] = items;
     p->items_per_b = items;
     p->cache_R = R;

@@ -122,6 +122,7 @@ struct ScanParams {
     long long cache_R;      // rows per (b,h) cache block
     int cap;
     int grid;               // cache layout of the fixed-grid reading (grid rows + window ring)
+    int one;                // one-tensor form: x[0], g -> out[0] (separate gates, run per tensor)
     int B, T, H, d;
     int nslices;            // B * nheads
     int nchunks;            // chunks along T per slice
@@ -171,6 +172,7 @@ struct DecodeParams {
     int items_per_b;             // sum over heads of nsplit
     int grid;                    // fixed-grid reading and its cache layout
     int dedupe;                  // the window part skips the dilated set's keys
+    int sep;                     // separate key and value gates: g is [2,B,H,d]
     float scale_log2;
     int dil[kMaxHeads];
     int win[kMaxHeads];
@@ -198,6 +200,7 @@ struct TopkParams {
     long long cache_R;
     int cap, B, H, d;
     int bs, K, mode, nblk;       // block size, blocks to select, RAT_TOPK_*, ceil(cap / bs)
+    int sep;                     // separate key and value gates: g is [2,B,H,d]
     float scale_log2;
     unsigned char recur[kMaxHeads];
     WsHeader *hdr;

@@ -146,15 +146,19 @@ __global__ void __launch_bounds__(kThreads) topk_decode_kernel(const TopkParams 
     // (A) step update of channel tid, append of row t, statistics of block c
     if (tid < D) {
         const size_t e = bh * D + tid;
-        float a = 0.f, oma = 1.f;
+        float a[2] = {0.f, 0.f}, oma[2] = {1.f, 1.f};   // keys, values
         if (p.recur[h]) {
-            const float g = fminf(fmaxf(to_f<T>(static_cast<const T *>(p.g)[e]), -80.f), 80.f);
-            const float ex = expf(-g);
-            a = 1.f / (1.f + ex);
-            oma = ex * a;
+            for (int i = 0; i < 2; ++i) {
+                // separate gates: the value gate is the second [B,H,d] tensor
+                const size_t ge = (p.sep && i == 1) ? (size_t)p.B * p.H * D + e : e;
+                const float g = fminf(fmaxf(to_f<T>(static_cast<const T *>(p.g)[ge]), -80.f), 80.f);
+                const float ex = expf(-g);
+                a[i] = 1.f / (1.f + ex);
+                oma[i] = ex * a[i];
+            }
         }
-        const float sk = a * p.state[0][e] + oma * to_f<T>(static_cast<const T *>(p.k)[e]);
-        const float sv = a * p.state[1][e] + oma * to_f<T>(static_cast<const T *>(p.v)[e]);
+        const float sk = a[0] * p.state[0][e] + oma[0] * to_f<T>(static_cast<const T *>(p.k)[e]);
+        const float sv = a[1] * p.state[1][e] + oma[1] * to_f<T>(static_cast<const T *>(p.v)[e]);
         p.state[0][e] = sk;
         p.state[1][e] = sv;
         const T rk = from_f<T>(sk);

@@ -110,8 +110,9 @@ def test_cache_rows_layout_fixed_grid(lib):
 
 
 def test_unknown_flags_are_rejected(lib):
-    assert lib.rat_workspace_size(cfg(flags=4).ref(), rat.RAT_OP_MIX, 0) == 0
-    for f in (rat.RAT_FLAG_GRID_DILATION, rat.RAT_FLAG_DEDUPE, rat.RAT_FLAG_GRID_DILATION | rat.RAT_FLAG_DEDUPE):
+    assert lib.rat_workspace_size(cfg(flags=8).ref(), rat.RAT_OP_MIX, 0) == 0
+    for f in (rat.RAT_FLAG_GRID_DILATION, rat.RAT_FLAG_DEDUPE, rat.RAT_FLAG_SEPARATE_GATES,
+              rat.RAT_FLAG_GRID_DILATION | rat.RAT_FLAG_DEDUPE | rat.RAT_FLAG_SEPARATE_GATES):
         assert lib.rat_workspace_size(cfg(flags=f).ref(), rat.RAT_OP_MIX, 0) > 0
 
 

@@ -22,8 +22,9 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def make_cfg(B, T, H, d, dtype, dil, win, recur=None, scale=0.0, grid=False, dedupe=False):
+def make_cfg(B, T, H, d, dtype, dil, win, recur=None, scale=0.0, grid=False, dedupe=False, sep=False):
     flags = (rat.RAT_FLAG_GRID_DILATION if grid else 0) | (rat.RAT_FLAG_DEDUPE if dedupe else 0)
+    flags |= rat.RAT_FLAG_SEPARATE_GATES if sep else 0
     return rat.Config(B, T, H, d, dtype, dil, win, recur, scale, flags)
 
 
@@ -278,23 +279,26 @@ def test_decode_cache_layout_from_scan():
 
 
 def run_decode_case(B, T, steps, H, d, dtype, dil, win, recur, mu, seed, cap=None, check_b=None, check_h=None,
-                    gen_device="cpu", grid=False, dedupe=False):
+                    gen_device="cpu", grid=False, dedupe=False, sep=False):
     """Prefill T tokens into the cache with rat_scan_prefill, then decode `steps`
     tokens with rat_decode_step; compare every step with the oracle's rows
     (on the batch entries check_b and heads check_h; all by default).  grid:
     the fixed-grid reading of dilation and its cache layout; dedupe: a key in
-    both parts counts once."""
+    both parts counts once; sep: separate key and value gates."""
     Tt = T + steps
     cap = cap or Tt
     q, k, v, g = inputs(B, Tt, H, d, dtype, mu=mu, seed=seed, device=gen_device)
-    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur, grid=grid, dedupe=dedupe)
+    gv = inputs(B, Tt, H, d, dtype, mu=mu, seed=seed + 1000, device=gen_device)[3] if sep else g
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur, grid=grid, dedupe=dedupe, sep=sep)
+    # the gate argument: [2, B, T, H, d] with separate gates
+    gate = (lambda sl: torch.stack([g[sl], gv[sl]]).contiguous()) if sep else (lambda sl: g[sl].contiguous())
     R = rat.rat_cache_rows(cfg, cap)
     ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
     cv = torch.zeros_like(ck)
     sk = torch.empty(B, H, d, device=DEV)
     sv = torch.empty_like(sk)
     ws = rat.workspace(cfg, rat.RAT_OP_SCAN)
-    rat.rat_scan_prefill(cfg, k[:, :T].contiguous(), v[:, :T].contiguous(), g[:, :T].contiguous(), None, None,
+    rat.rat_scan_prefill(cfg, k[:, :T].contiguous(), v[:, :T].contiguous(), gate(np.s_[:, :T]), None, None,
                          None, None, sk, sv, ck, cv, cap, ws)
     rat.rat_check_status(ws)
     del ws
@@ -306,7 +310,7 @@ def run_decode_case(B, T, steps, H, d, dtype, dil, win, recur, mu, seed, cap=Non
         o = torch.empty(B, H, d, dtype=dtype, device=DEV)
         lse = torch.empty(B, H, device=DEV)
         rat.rat_decode_step(cfg, q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(),
-                            g[:, t].contiguous(), sk, sv, ck, cv, cap, pos, o, lse, wsd)
+                            gate(np.s_[:, t]), sk, sv, ck, cv, cap, pos, o, lse, wsd)
         outs.append((o, lse))
     rat.rat_check_status(wsd)
     bsel = list(range(B)) if check_b is None else check_b
@@ -314,7 +318,7 @@ def run_decode_case(B, T, steps, H, d, dtype, dil, win, recur, mu, seed, cap=Non
     sl = lambda x: f64(x[bsel][:, :, hsel])
     dsel, wsel, rsel = [dil[h] for h in hsel], [win[h] for h in hsel], [recur[h] for h in hsel]
     kt, fk = oracle.scan(sl(k), sl(g), None, rsel)
-    vt, fv = oracle.scan(sl(v), sl(g), None, rsel)
+    vt, fv = oracle.scan(sl(v), sl(gv), None, rsel)
     rows = np.array([(b, i, t) for b in range(len(bsel)) for i in range(len(hsel)) for t in range(T, Tt)])
     ro, rl = oracle.attn_rows(sl(q), kt, vt, dsel, wsel, rows, parts=3, grid=grid, dedupe=dedupe)
     ro = ro.reshape(len(bsel), len(hsel), steps, d)
@@ -666,6 +670,70 @@ def test_topk_decode_keeps_every_block_when_k_is_large():
     # K >= number of candidates: the step is dense causal attention
     run_topk_case(B=1, T=500, steps=3, H=2, d=128, dtype=torch.bfloat16, block=32, topk=64, mode=0,
                   recur=[1, 1], seed=43)
+
+
+# ------------------------------------------------- separate key and value gates
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("T", [77, 5003])
+def test_separate_gates_scan_every_element(dtype, d, T):
+    B, H = 2, 3
+    q, k, v, g = inputs(B, T, H, d, dtype, seed=T + 1)
+    gv = inputs(B, T, H, d, dtype, mu=0.5, seed=T + 2)[3]
+    init_k = wl.random_state(B, H, d, seed=3).to(DEV)
+    init_v = wl.random_state(B, H, d, seed=4).to(DEV)
+    recur = [1, 0, 1]
+    cap = T + 5
+    cfg = make_cfg(B, T, H, d, dtype, [1, 4, 7], [0, 0, 9], recur, sep=True)
+    kt, vt = torch.empty_like(k), torch.empty_like(v)
+    fk = torch.empty(B, H, d, device=DEV)
+    fv = torch.empty_like(fk)
+    R = rat.rat_cache_rows(cfg, cap)
+    ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
+    cv = torch.zeros_like(ck)
+    ws = rat.workspace(cfg, rat.RAT_OP_SCAN)
+    rat.rat_scan_prefill(cfg, k, v, torch.stack([g, gv]).contiguous(), init_k, init_v, kt, vt, fk, fv, ck, cv,
+                         cap, ws)
+    rat.rat_check_status(ws)
+    rk, rfk = oracle.scan(f64(k), f64(g), f64(init_k), recur)
+    rv, rfv = oracle.scan(f64(v), f64(gv), f64(init_v), recur)
+    ft = torch.float32 if dtype == torch.float32 else dtype
+    assert_close(kt, rk, dtype, "kt")
+    assert_close(vt, rv, dtype, "vt")
+    assert_close(fk, rfk, ft, "final_k")
+    assert_close(fv, rfv, ft, "final_v")
+    for h, D in enumerate([1, 4, 7]):   # both caches written, each from its own pass
+        S = -(-cap // D)
+        j = torch.arange(T, device=DEV)
+        rows = (j % D) * S + j // D
+        assert torch.equal(ck[:, h, rows], kt[:, :, h]) and torch.equal(cv[:, h, rows], vt[:, :, h])
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_separate_gates_mix_every_element(dtype):
+    B, T, H, d = 2, 2048, 3, 128
+    dil, win, recur = [1, 16, 64], [0, 0, 256], [0, 1, 1]
+    q, k, v, g = inputs(B, T, H, d, dtype, seed=51)
+    gv = inputs(B, T, H, d, dtype, mu=-1.0, seed=52)[3]
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur, sep=True)
+    out = rat.mix_prefill(cfg, q, k, v, torch.stack([g, gv]).contiguous())
+    rat.rat_check_status(out["ws"])
+    rk, rfk = oracle.scan(f64(k), f64(g), None, recur)
+    rv, rfv = oracle.scan(f64(v), f64(gv), None, recur)
+    ro, rl = oracle.attention(f64(q), rk, rv, dil, win)
+    ft = torch.float32 if dtype == torch.float32 else dtype
+    assert_close(out["o"], ro, dtype, "o")
+    assert_close(out["lse"], rl, ft, "lse")
+    assert_close(out["final_k"], rfk, ft, "final_k")
+    assert_close(out["final_v"], rfv, ft, "final_v")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_separate_gates_decode_steps(dtype):
+    run_decode_case(B=3, T=1500, steps=4, H=4, d=128, dtype=dtype, dil=[1, 4, 16, 3], win=[0, 0, 64, 1500],
+                    recur=[0, 1, 1, 1], mu=2.0, seed=25, sep=True)
 
 
 def test_decode_bad_position_is_reported():
