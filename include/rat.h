@@ -227,6 +227,38 @@ RAT_API rat_status rat_decode_step(const rat_cfg *cfg, const void *q, const void
                            void *ws, size_t ws_bytes, rat_stream_t stream);
 
 /*
+ * Paged decode cache, for serving engines that hand out KV memory in pages.
+ * The logical rows of a (b, h) block -- the layout of rat_cache_rows, in
+ * either dilation reading -- live in pages of page_rows rows: logical row r of
+ * batch entry b, head h is row (r mod page_rows) of page
+ * page_table[b * pages_per_seq + r / page_rows] of the pools, which are
+ * [num_pages, H, page_rows, d] in cfg->dtype.  pages_per_seq * page_rows must
+ * cover rat_cache_rows(cfg, cache_cap).  Only the pages of the rows a call
+ * touches need valid entries; a touched entry outside [0, num_pages) is never
+ * dereferenced: the prefill leaves that row unwritten and the decode step
+ * skips each (b, h) whose step touches it (o = 0, state unchanged), and either
+ * records RAT_ERR_INVALID for rat_check_status.  The caller owns pools and
+ * table (device memory).
+ */
+typedef struct {
+    void *pool_k, *pool_v;        /* [num_pages, H, page_rows, d] */
+    const int32_t *page_table;    /* device int32 [B, pages_per_seq] */
+    int page_rows, pages_per_seq, num_pages;
+} rat_paged_cache;
+
+/* rat_scan_prefill writing a paged cache (cache_cap as there). */
+RAT_API rat_status rat_scan_prefill_paged(const rat_cfg *cfg, const void *k, const void *v, const void *g,
+                                          const float *init_k, const float *init_v, void *kt, void *vt,
+                                          float *final_k, float *final_v, const rat_paged_cache *cache,
+                                          int cache_cap, void *ws, size_t ws_bytes, rat_stream_t stream);
+
+/* rat_decode_step over a paged cache; the ring's copies split at page ends. */
+RAT_API rat_status rat_decode_step_paged(const rat_cfg *cfg, const void *q, const void *k, const void *v,
+                                         const void *g, float *state_k, float *state_v,
+                                         const rat_paged_cache *cache, int cache_cap, const int32_t *pos,
+                                         void *o, float *lse, void *ws, size_t ws_bytes, rat_stream_t stream);
+
+/*
  * rat_decode_step without a workspace, for callers that cannot allocate
  * device memory when they decode: a plugin inside an inference engine that
  * owns all device memory and gives its plugins no scratch buffer, or a serving

@@ -29,7 +29,8 @@ RAT_FLAG_SEPARATE_GATES = 4
 EXPORTS = ["rat_workspace_size", "rat_workspace_init", "rat_cache_rows", "rat_scan_prefill",
            "rat_dilated_attn_prefill", "rat_mix_prefill", "rat_decode_step", "rat_check_status",
            "rat_status_string", "rat_last_error", "rat_version", "rat_launch_count", "rat_debug_set_scan_stall",
-           "rat_decode_step_noalloc", "rat_topk_stats_size", "rat_topk_build_stats", "rat_topk_decode_step"]
+           "rat_decode_step_noalloc", "rat_topk_stats_size", "rat_topk_build_stats", "rat_topk_decode_step",
+           "rat_scan_prefill_paged", "rat_decode_step_paged"]
 
 
 class RatError(RuntimeError):
@@ -47,6 +48,11 @@ class rat_cfg(ctypes.Structure):
                 ("dtype", ctypes.c_int), ("dil", ctypes.POINTER(ctypes.c_int32)),
                 ("win", ctypes.POINTER(ctypes.c_int32)), ("recur", ctypes.POINTER(ctypes.c_uint8)),
                 ("scale", ctypes.c_float), ("flags", ctypes.c_uint32)]
+
+
+class rat_paged_cache(ctypes.Structure):
+    _fields_ = [("pool_k", ctypes.c_void_p), ("pool_v", ctypes.c_void_p), ("page_table", ctypes.c_void_p),
+                ("page_rows", ctypes.c_int), ("pages_per_seq", ctypes.c_int), ("num_pages", ctypes.c_int)]
 
 
 _lib = None
@@ -76,6 +82,9 @@ def load_library(path=LIB_PATH):
     lib.rat_topk_stats_size.restype = S
     lib.rat_topk_build_stats.argtypes = [cfgp, I, I, P, I, P, P]
     lib.rat_topk_decode_step.argtypes = [cfgp, I, I, I, P, P, P, P, P, P, P, P, I, P, P, P, P, P, P, S, P]
+    pcp = ctypes.POINTER(rat_paged_cache)
+    lib.rat_scan_prefill_paged.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, pcp, I, P, S, P]
+    lib.rat_decode_step_paged.argtypes = [cfgp, P, P, P, P, P, P, pcp, I, P, P, P, P, S, P]
     lib.rat_check_status.argtypes = [P, P]
     lib.rat_status_string.argtypes = [I]
     lib.rat_status_string.restype = ctypes.c_char_p
@@ -86,7 +95,8 @@ def load_library(path=LIB_PATH):
     lib.rat_debug_set_scan_stall.argtypes = [P, S, ctypes.c_int64, ctypes.c_int64, P]
     for name in ("rat_workspace_init", "rat_scan_prefill", "rat_dilated_attn_prefill", "rat_mix_prefill",
                  "rat_decode_step", "rat_check_status", "rat_debug_set_scan_stall", "rat_decode_step_noalloc",
-                 "rat_topk_build_stats", "rat_topk_decode_step"):
+                 "rat_topk_build_stats", "rat_topk_decode_step", "rat_scan_prefill_paged",
+                 "rat_decode_step_paged"):
         getattr(lib, name).restype = I
     _lib = lib
     return lib
@@ -304,6 +314,51 @@ def rat_topk_decode_step(cfg, block, topk, mode, q, k, v, g, state_k, state_v, c
             _ptr(sel, "sel", torch.int32, (c.B, c.H, int(topk)), True),
             _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream)]
     _check(load_library().rat_topk_decode_step(cfg.ref(), *args), "rat_topk_decode_step")
+
+
+def paged_cache(cfg, pool_k, pool_v, page_table, cache_cap):
+    """A rat_paged_cache over torch tensors: pools [num_pages, H, page_rows, d]
+    in the cfg's dtype and a device int32 table [B, pages_per_seq]."""
+    c = cfg.c
+    if pool_k.dim() != 4 or pool_k.shape[1] != c.H or pool_k.shape[3] != c.d:
+        raise ValueError("pool_k must be [num_pages, H, page_rows, d]")
+    n, _, P, _ = pool_k.shape
+    _ptr(pool_k, "pool_k", cfg.torch_dtype)
+    _ptr(pool_v, "pool_v", cfg.torch_dtype, tuple(pool_k.shape))
+    _ptr(page_table, "page_table", torch.int32)
+    if page_table.dim() != 2 or page_table.shape[0] != c.B:
+        raise ValueError("page_table must be [B, pages_per_seq]")
+    return rat_paged_cache(pool_k.data_ptr(), pool_v.data_ptr(), page_table.data_ptr(), int(P),
+                           int(page_table.shape[1]), int(n))
+
+
+def rat_scan_prefill_paged(cfg, k, v, g, init_k=None, init_v=None, kt=None, vt=None, final_k=None, final_v=None,
+                           cache=None, cache_cap=0, ws=None, stream=None):
+    """rat_scan_prefill into a paged cache (a rat_paged_cache from paged_cache())."""
+    c = cfg.c
+    tok = (c.B, c.T, c.H, c.d)
+    st = (c.B, c.H, c.d)
+    dt = cfg.torch_dtype
+    args = [_ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
+            _ptr(init_k, "init_k", torch.float32, st, True), _ptr(init_v, "init_v", torch.float32, st, True),
+            _ptr(kt, "kt", dt, tok, True), _ptr(vt, "vt", dt, tok, True),
+            _ptr(final_k, "final_k", torch.float32, st, True), _ptr(final_v, "final_v", torch.float32, st, True),
+            ctypes.byref(cache), int(cache_cap), _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream)]
+    _check(load_library().rat_scan_prefill_paged(cfg.ref(), *args), "rat_scan_prefill_paged")
+
+
+def rat_decode_step_paged(cfg, q, k, v, g, state_k, state_v, cache, cache_cap, pos, o, lse=None, ws=None,
+                          stream=None):
+    """rat_decode_step over a paged cache (a rat_paged_cache from paged_cache())."""
+    c = cfg.c
+    tok = (c.B, c.H, c.d)
+    dt = cfg.torch_dtype
+    args = [_ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
+            _ptr(state_k, "state_k", torch.float32, tok), _ptr(state_v, "state_v", torch.float32, tok),
+            ctypes.byref(cache), int(cache_cap), _ptr(pos, "pos", torch.int32, (c.B,)), _ptr(o, "o", dt, tok),
+            _ptr(lse, "lse", torch.float32, (c.B, c.H), True), _ptr(ws, "ws", torch.uint8), ws.numel(),
+            _stream(stream)]
+    _check(load_library().rat_decode_step_paged(cfg.ref(), *args), "rat_decode_step_paged")
 
 
 def rat_check_status(ws, stream=None):

@@ -202,9 +202,16 @@ rat_status scan_pass(const rat_cfg *c, const Layout &L, ScanParams &p, char *ws,
 // Scan of the selected heads into kt/vt and/or the cache.
 rat_status run_scan(const rat_cfg *c, const Layout &L, const void *k, const void *v, const void *g,
                     const float *ik, const float *iv, void *kt, void *vt, float *fk, float *fv,
-                    void *ck, void *cv, int cap, char *ws, bool only_recurrent, cudaStream_t s) {
+                    void *ck, void *cv, int cap, char *ws, bool only_recurrent, cudaStream_t s,
+                    const rat_paged_cache *pc = nullptr) {
     ScanParams p;
     memset(&p, 0, sizeof(p));
+    if (pc) {
+        p.page_table = pc->page_table;
+        p.page_rows = pc->page_rows;
+        p.pps = pc->pages_per_seq;
+        p.num_pages = pc->num_pages;
+    }
     p.x[0] = k; p.x[1] = v; p.g = g;
     p.init[0] = ik; p.init[1] = iv;
     p.out[0] = kt; p.out[1] = vt;
@@ -408,6 +415,91 @@ rat_status run_attn(const rat_cfg *c, const Layout &L, const void *q, const void
     return RAT_OK;
 }
 
+// A paged cache descriptor: pools and table given, pages cover the logical rows.
+rat_status check_paged(const rat_cfg *c, const rat_paged_cache *pc, int cap) {
+    if (!pc) return fail(RAT_ERR_INVALID, "paged cache descriptor is NULL");
+    CHECK_PTR(pc->pool_k, "pool_k"); CHECK_PTR(pc->pool_v, "pool_v"); CHECK_PTR(pc->page_table, "page_table");
+    if (pc->page_rows < 1 || pc->num_pages < 1 || pc->pages_per_seq < 1)
+        return fail(RAT_ERR_INVALID, "page_rows %d, num_pages %d, pages_per_seq %d must be >= 1", pc->page_rows,
+                    pc->num_pages, pc->pages_per_seq);
+    if (cap < 1) return fail(RAT_ERR_INVALID, "cache_cap %d < 1", cap);
+    const long long R = cache_rows(c, cap);
+    if ((long long)pc->pages_per_seq * pc->page_rows < R)
+        return fail(RAT_ERR_INVALID, "pages_per_seq x page_rows < %lld cache rows", R);
+    return RAT_OK;
+}
+
+// rat_decode_step with a dense cache (pc = NULL) or a paged one.
+rat_status decode_step(const rat_cfg *cfg, const void *q, const void *k, const void *v, const void *g,
+                       float *state_k, float *state_v, void *cache_k, void *cache_v, const rat_paged_cache *pc,
+                       int cache_cap, const int32_t *pos, void *o, float *lse, void *ws, size_t ws_bytes,
+                       rat_stream_t stream) {
+    rat_status st = check_cfg(cfg, false);
+    if (st != RAT_OK) return st;
+    if (cfg->B == 0) return RAT_OK;
+    CHECK_PTR(q, "q"); CHECK_PTR(k, "k"); CHECK_PTR(v, "v"); CHECK_PTR(g, "g");
+    CHECK_PTR(state_k, "state_k"); CHECK_PTR(state_v, "state_v");
+    CHECK_PTR(cache_k, "cache_k"); CHECK_PTR(cache_v, "cache_v");
+    CHECK_PTR(pos, "pos"); CHECK_PTR(o, "o"); CHECK_OPT(lse, "lse");
+    if (cache_cap < 1) return fail(RAT_ERR_INVALID, "cache_cap %d < 1", cache_cap);
+    Layout L;
+    st = check_ws(cfg, RAT_OP_DECODE, cache_cap, ws, ws_bytes, &L);
+    if (st != RAT_OK) return st;
+    DecodeParams p;
+    memset(&p, 0, sizeof(p));
+    decode_plan(cfg, cache_cap, &p);
+    p.q = q; p.k = k; p.v = v; p.g = g;
+    p.state[0] = state_k; p.state[1] = state_v;
+    p.cache[0] = cache_k; p.cache[1] = cache_v;
+    if (pc) {
+        p.page_table = pc->page_table;
+        p.page_rows = pc->page_rows;
+        p.pps = pc->pages_per_seq;
+        p.num_pages = pc->num_pages;
+    }
+    p.pos = pos; p.o = o; p.lse = lse;
+    char *w = static_cast<char *>(ws);
+    p.part = reinterpret_cast<float *>(w + L.part);
+    const size_t part_bytes = align256((size_t)cfg->B * p.items_per_b * (cfg->d + 2) * sizeof(float));
+    p.counter = reinterpret_cast<int *>(w + L.part + part_bytes);
+    p.cap = cache_cap; p.B = cfg->B; p.H = cfg->H; p.d = cfg->d;
+    p.scale_log2 = scale_of(cfg) * 1.4426950408889634f;
+    p.hdr = reinterpret_cast<WsHeader *>(ws);
+    // per-(b,h) completion counters start from zero on every call
+    cudaError_t ez = cudaMemsetAsync(p.counter, 0, (size_t)cfg->B * cfg->H * sizeof(int), (cudaStream_t)stream);
+    if (ez != cudaSuccess) return cuda_fail(ez, "cudaMemsetAsync(decode counters)");
+    cudaError_t e = launch_decode(p, cfg->dtype, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    return RAT_OK;
+}
+
+// rat_scan_prefill with a dense cache (pc = NULL) or a paged one.
+rat_status scan_prefill(const rat_cfg *cfg, const void *k, const void *v, const void *g, const float *init_k,
+                        const float *init_v, void *kt, void *vt, float *final_k, float *final_v, void *cache_k,
+                        void *cache_v, const rat_paged_cache *pc, int cache_cap, void *ws, size_t ws_bytes,
+                        rat_stream_t stream) {
+    rat_status st = check_cfg(cfg);
+    if (st != RAT_OK) return st;
+    CHECK_OPT(init_k, "init_k"); CHECK_OPT(init_v, "init_v");
+    CHECK_OPT(final_k, "final_k"); CHECK_OPT(final_v, "final_v");
+    if (empty(cfg)) return empty_prefill_state(cfg, init_k, init_v, final_k, final_v, (cudaStream_t)stream);
+    CHECK_PTR(k, "k"); CHECK_PTR(v, "v"); CHECK_PTR(g, "g");
+    CHECK_OPT(init_k, "init_k"); CHECK_OPT(init_v, "init_v");
+    CHECK_OPT(kt, "kt"); CHECK_OPT(vt, "vt");
+    CHECK_OPT(final_k, "final_k"); CHECK_OPT(final_v, "final_v");
+    CHECK_OPT(cache_k, "cache_k"); CHECK_OPT(cache_v, "cache_v");
+    if ((kt == nullptr) != (vt == nullptr)) return fail(RAT_ERR_INVALID, "kt and vt must be given together");
+    if ((cache_k == nullptr) != (cache_v == nullptr))
+        return fail(RAT_ERR_INVALID, "cache_k and cache_v must be given together");
+    if (!kt && !cache_k) return fail(RAT_ERR_INVALID, "no output: give kt/vt and/or cache_k/cache_v");
+    if (cache_k && cache_cap < cfg->T) return fail(RAT_ERR_INVALID, "cache_cap %d < T %d", cache_cap, cfg->T);
+    Layout L;
+    st = check_ws(cfg, RAT_OP_SCAN, 0, ws, ws_bytes, &L);
+    if (st != RAT_OK) return st;
+    return run_scan(cfg, L, k, v, g, init_k, init_v, kt, vt, final_k, final_v, cache_k, cache_v,
+                    cache_cap, static_cast<char *>(ws), false, (cudaStream_t)stream, pc);
+}
+
 }  // namespace
 
 extern "C" {
@@ -455,26 +547,20 @@ rat_status rat_scan_prefill(const rat_cfg *cfg, const void *k, const void *v, co
                             const float *init_k, const float *init_v, void *kt, void *vt,
                             float *final_k, float *final_v, void *cache_k, void *cache_v,
                             int cache_cap, void *ws, size_t ws_bytes, rat_stream_t stream) {
+    return scan_prefill(cfg, k, v, g, init_k, init_v, kt, vt, final_k, final_v, cache_k, cache_v, nullptr,
+                        cache_cap, ws, ws_bytes, stream);
+}
+
+rat_status rat_scan_prefill_paged(const rat_cfg *cfg, const void *k, const void *v, const void *g,
+                                  const float *init_k, const float *init_v, void *kt, void *vt, float *final_k,
+                                  float *final_v, const rat_paged_cache *cache, int cache_cap, void *ws,
+                                  size_t ws_bytes, rat_stream_t stream) {
     rat_status st = check_cfg(cfg);
     if (st != RAT_OK) return st;
-    CHECK_OPT(init_k, "init_k"); CHECK_OPT(init_v, "init_v");
-    CHECK_OPT(final_k, "final_k"); CHECK_OPT(final_v, "final_v");
-    if (empty(cfg)) return empty_prefill_state(cfg, init_k, init_v, final_k, final_v, (cudaStream_t)stream);
-    CHECK_PTR(k, "k"); CHECK_PTR(v, "v"); CHECK_PTR(g, "g");
-    CHECK_OPT(init_k, "init_k"); CHECK_OPT(init_v, "init_v");
-    CHECK_OPT(kt, "kt"); CHECK_OPT(vt, "vt");
-    CHECK_OPT(final_k, "final_k"); CHECK_OPT(final_v, "final_v");
-    CHECK_OPT(cache_k, "cache_k"); CHECK_OPT(cache_v, "cache_v");
-    if ((kt == nullptr) != (vt == nullptr)) return fail(RAT_ERR_INVALID, "kt and vt must be given together");
-    if ((cache_k == nullptr) != (cache_v == nullptr))
-        return fail(RAT_ERR_INVALID, "cache_k and cache_v must be given together");
-    if (!kt && !cache_k) return fail(RAT_ERR_INVALID, "no output: give kt/vt and/or cache_k/cache_v");
-    if (cache_k && cache_cap < cfg->T) return fail(RAT_ERR_INVALID, "cache_cap %d < T %d", cache_cap, cfg->T);
-    Layout L;
-    st = check_ws(cfg, RAT_OP_SCAN, 0, ws, ws_bytes, &L);
+    st = check_paged(cfg, cache, cache_cap);
     if (st != RAT_OK) return st;
-    return run_scan(cfg, L, k, v, g, init_k, init_v, kt, vt, final_k, final_v, cache_k, cache_v,
-                    cache_cap, static_cast<char *>(ws), false, (cudaStream_t)stream);
+    return scan_prefill(cfg, k, v, g, init_k, init_v, kt, vt, final_k, final_v, cache->pool_k, cache->pool_v,
+                        cache, cache_cap, ws, ws_bytes, stream);
 }
 
 rat_status rat_dilated_attn_prefill(const rat_cfg *cfg, const void *q, const void *kt, const void *vt,
@@ -527,37 +613,20 @@ rat_status rat_decode_step(const rat_cfg *cfg, const void *q, const void *k, con
                            const void *g, float *state_k, float *state_v, void *cache_k,
                            void *cache_v, int cache_cap, const int32_t *pos, void *o, float *lse,
                            void *ws, size_t ws_bytes, rat_stream_t stream) {
+    return decode_step(cfg, q, k, v, g, state_k, state_v, cache_k, cache_v, nullptr, cache_cap, pos, o, lse, ws,
+                       ws_bytes, stream);
+}
+
+rat_status rat_decode_step_paged(const rat_cfg *cfg, const void *q, const void *k, const void *v, const void *g,
+                                 float *state_k, float *state_v, const rat_paged_cache *cache, int cache_cap,
+                                 const int32_t *pos, void *o, float *lse, void *ws, size_t ws_bytes,
+                                 rat_stream_t stream) {
     rat_status st = check_cfg(cfg, false);
     if (st != RAT_OK) return st;
-    if (cfg->B == 0) return RAT_OK;
-    CHECK_PTR(q, "q"); CHECK_PTR(k, "k"); CHECK_PTR(v, "v"); CHECK_PTR(g, "g");
-    CHECK_PTR(state_k, "state_k"); CHECK_PTR(state_v, "state_v");
-    CHECK_PTR(cache_k, "cache_k"); CHECK_PTR(cache_v, "cache_v");
-    CHECK_PTR(pos, "pos"); CHECK_PTR(o, "o"); CHECK_OPT(lse, "lse");
-    if (cache_cap < 1) return fail(RAT_ERR_INVALID, "cache_cap %d < 1", cache_cap);
-    Layout L;
-    st = check_ws(cfg, RAT_OP_DECODE, cache_cap, ws, ws_bytes, &L);
+    st = check_paged(cfg, cache, cache_cap);
     if (st != RAT_OK) return st;
-    DecodeParams p;
-    memset(&p, 0, sizeof(p));
-    decode_plan(cfg, cache_cap, &p);
-    p.q = q; p.k = k; p.v = v; p.g = g;
-    p.state[0] = state_k; p.state[1] = state_v;
-    p.cache[0] = cache_k; p.cache[1] = cache_v;
-    p.pos = pos; p.o = o; p.lse = lse;
-    char *w = static_cast<char *>(ws);
-    p.part = reinterpret_cast<float *>(w + L.part);
-    const size_t part_bytes = align256((size_t)cfg->B * p.items_per_b * (cfg->d + 2) * sizeof(float));
-    p.counter = reinterpret_cast<int *>(w + L.part + part_bytes);
-    p.cap = cache_cap; p.B = cfg->B; p.H = cfg->H; p.d = cfg->d;
-    p.scale_log2 = scale_of(cfg) * 1.4426950408889634f;
-    p.hdr = reinterpret_cast<WsHeader *>(ws);
-    // per-(b,h) completion counters start from zero on every call
-    cudaError_t ez = cudaMemsetAsync(p.counter, 0, (size_t)cfg->B * cfg->H * sizeof(int), (cudaStream_t)stream);
-    if (ez != cudaSuccess) return cuda_fail(ez, "cudaMemsetAsync(decode counters)");
-    cudaError_t e = launch_decode(p, cfg->dtype, (cudaStream_t)stream);
-    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-    return RAT_OK;
+    return decode_step(cfg, q, k, v, g, state_k, state_v, cache->pool_k, cache->pool_v, cache, cache_cap, pos, o,
+                       lse, ws, ws_bytes, stream);
 }
 
 // ---------------------------------------------------------- top-k block decode

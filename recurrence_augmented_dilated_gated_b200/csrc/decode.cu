@@ -10,7 +10,9 @@
 // Under the fixed-grid reading the dilated set is { j < t, j mod D == D-1 }
 // plus t, the slab is the grid (rows 0 .. t/D - 1, the same count), the new
 // row is stored at its grid row only when t is on the grid, and the window
-// rows come from a ring of the last W positions (D > 1).  With dedupe the
+// rows come from a ring of the last W positions (D > 1).  A paged cache
+// (kPaged) keeps the same logical rows in pages named by a page table; the
+// ring's bulk copies split where a run of rows crosses a page.  With dedupe the
 // window part skips the keys of the dilated set, the new row among them.
 // Softmaxes over disjoint pieces of a key multiset combine exactly by
 // log-sum-exp, so the step is split into independent work items:
@@ -160,7 +162,7 @@ __device__ __forceinline__ void acc_add_batch(Acc8 &a, const float *s, const flo
     a.m = mn;
 }
 
-template <typename T, int D>
+template <typename T, int D, bool kPaged>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) {
     constexpr int LPR = D / 8;                 // lanes per cache row (8 channels each)
     constexpr int NG = kCompute / LPR;         // row groups
@@ -195,8 +197,32 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     const int i1 = min(i0 + p.rows_per_item[h], n_old);
     const int nrows = max(0, i1 - i0);
     const int nst = (nrows + RS - 1) / RS;       // ring stages this item streams
-    const T *ck = static_cast<const T *>(p.cache[0]) + bh * (size_t)p.cache_R * D;
-    const T *cv = static_cast<const T *>(p.cache[1]) + bh * (size_t)p.cache_R * D;
+    const T *ck = static_cast<const T *>(p.cache[0]);   // cache bases: rows at row_off(row)
+    const T *cv = static_cast<const T *>(p.cache[1]);
+    // element offset of logical cache row `row` of (b, h); -1 for a page the
+    // table does not name validly
+    auto row_off = [&](long long row) -> long long {
+        if (kPaged) return cache_offset(p.page_table, p.pps, p.page_rows, p.num_pages, p.cache_R, p.H, D, b, h, row);
+        return ((long long)bh * p.cache_R + row) * D;
+    };
+    // a paged cache: every page the step of (b, h) touches must be valid, else
+    // the pair is skipped (o = 0) and reported like an invalid position.  Every
+    // item checks the pages of the whole step, so all items of (b, h) agree.
+    int bad = 0;
+    if (kPaged && valid_pos) {
+        if (n_old > 0)
+            for (long long pg = (long long)slab0 / p.page_rows + tid;
+                 pg <= (long long)(slab0 + n_old - 1) / p.page_rows; pg += kThreads)
+                bad |= row_off(pg * p.page_rows) < 0;
+        long long ra, rb;
+        cache_rows_of(t, Dh, W, S, p.grid, ra, rb);
+        if (tid == 0) bad |= (ra >= 0 && row_off(ra) < 0) || (rb >= 0 && row_off(rb) < 0);
+        if (W > 0)
+            for (int jj = max(0, t - W + 1) + tid; jj < t; jj += kThreads) {
+                cache_rows_of(jj, Dh, W, S, p.grid, ra, rb);
+                bad |= row_off(rb >= 0 ? rb : ra) < 0;
+            }
+    }
 
     if (tid == 0) {
         s_abort = 0;
@@ -208,7 +234,9 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         if (!valid_pos) report_error(p.hdr, RAT_ERR_INVALID, b);
     }
-    __syncthreads();
+    bad = __syncthreads_or(bad);
+    const bool valid = valid_pos && !bad;
+    if (tid == 0 && valid_pos && bad) report_error(p.hdr, RAT_ERR_INVALID, b);
 
     Acc8 acc;
     acc.m = -INFINITY;
@@ -220,9 +248,9 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     if (warp == kCompute / 32) {
         // ------------------------------------------------ producer: stream the
         // item's contiguous run of K~ and V~ rows through the ring
-        if ((tid & 31) == 0 && valid_pos) {
-            const char *kb = reinterpret_cast<const char *>(ck + (slab0 + i0) * D);
-            const char *vb = reinterpret_cast<const char *>(cv + (slab0 + i0) * D);
+        if ((tid & 31) == 0 && valid) {
+            const char *kb = reinterpret_cast<const char *>(ck + (kPaged ? 0 : row_off(slab0 + i0)));
+            const char *vb = reinterpret_cast<const char *>(cv + (kPaged ? 0 : row_off(slab0 + i0)));
             int sidx = 0;
             bool ok = true;
             for (; sidx < nst; ++sidx) {
@@ -240,14 +268,34 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                 const size_t off = (size_t)sidx * RS * kRowBytes;
                 asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full), "r"(2 * bytes)
                              : "memory");
-                asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                                 dk),
-                             "l"(kb + off), "r"(bytes), "r"(full)
-                             : "memory");
-                asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                                 dv),
-                             "l"(vb + off), "r"(bytes), "r"(full)
-                             : "memory");
+                if (!kPaged) {
+                    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                                     dk),
+                                 "l"(kb + off), "r"(bytes), "r"(full)
+                                 : "memory");
+                    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                                     dv),
+                                 "l"(vb + off), "r"(bytes), "r"(full)
+                                 : "memory");
+                } else {
+                    // one copy per page the stage's rows touch (all validated above)
+                    const long long ra = (long long)(slab0 + i0) + (long long)sidx * RS;
+                    for (int done = 0; done < nr;) {
+                        const long long row = ra + done;
+                        const int n = (int)min((long long)(nr - done), (long long)p.page_rows - row % p.page_rows);
+                        const long long ofs = row_off(row);
+                        const uint32_t nb = (uint32_t)n * kRowBytes, so = (uint32_t)done * kRowBytes;
+                        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                                         dk + so),
+                                     "l"(ck + ofs), "r"(nb), "r"(full)
+                                     : "memory");
+                        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                                         dv + so),
+                                     "l"(cv + ofs), "r"(nb), "r"(full)
+                                     : "memory");
+                        done += n;
+                    }
+                }
             }
             if (!ok) {
                 s_abort = 1;
@@ -257,7 +305,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                     mbar_wait(smem_u32(&s_full[q % kStages]), (uint32_t)(q / kStages) & 1u, &never);
             }
         }
-    } else if (valid_pos) {
+    } else if (valid) {
         // ------------------------------------------------ scoring warps
         const unsigned gmask = group_mask<LPR>();
         float q[8];
@@ -346,15 +394,15 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                 p.state[1][e_new] = sv;
                 long long row0, row1;
                 cache_rows_of(t, Dh, W, S, p.grid, row0, row1);
-                T *dk = static_cast<T *>(p.cache[0]) + bh * (size_t)p.cache_R * D + tid;
-                T *dv = static_cast<T *>(p.cache[1]) + bh * (size_t)p.cache_R * D + tid;
+                T *dk = static_cast<T *>(p.cache[0]) + tid;
+                T *dv = static_cast<T *>(p.cache[1]) + tid;
                 if (row0 >= 0) {
-                    dk[(size_t)row0 * D] = to_t<T>(sk);
-                    dv[(size_t)row0 * D] = to_t<T>(sv);
+                    dk[row_off(row0)] = to_t<T>(sk);
+                    dv[row_off(row0)] = to_t<T>(sv);
                 }
                 if (row1 >= 0) {  // the ring slot of t - W, which no window needs any more
-                    dk[(size_t)row1 * D] = to_t<T>(sk);
-                    dv[(size_t)row1 * D] = to_t<T>(sv);
+                    dk[row_off(row1)] = to_t<T>(sk);
+                    dv[row_off(row1)] = to_t<T>(sv);
                 }
                 s_new[0][tid] = round_to<T>(sk);
                 s_new[1][tid] = round_to<T>(sv);
@@ -374,9 +422,9 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                             if (p.dedupe && (p.grid ? jj % Dh == Dh - 1 : (t - jj) % Dh == 0)) skip |= 1u << u;
                             long long row0, row1;
                             cache_rows_of(jj, Dh, W, S, p.grid, row0, row1);
-                            const size_t row = (size_t)(row1 >= 0 ? row1 : row0);
-                            IO8<T>::load(ck + row * D + c0, kf[u]);
-                            IO8<T>::load(cv + row * D + c0, vf[u]);
+                            const long long ofs = row_off(row1 >= 0 ? row1 : row0);
+                            IO8<T>::load(ck + ofs + c0, kf[u]);
+                            IO8<T>::load(cv + ofs + c0, vf[u]);
                         } else {
 #pragma unroll
                             for (int c = 0; c < 8; ++c) kf[u][c] = vf[u][c] = 0.f;
@@ -486,15 +534,20 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     if (tid == 0) p.counter[bh] = 0;  // ready for the next step
 }
 
-template <typename T, int D>
-cudaError_t launch_typed(const DecodeParams &p, unsigned grid, cudaStream_t s) {
+template <typename T, int D, bool kPaged>
+cudaError_t launch_form(const DecodeParams &p, unsigned grid, cudaStream_t s) {
     constexpr int RS = (kCompute / (D / 8)) * kBatch;
     const size_t smem = (size_t)kStages * 2 * RS * D * sizeof(T);
     static std::atomic<unsigned long long> smem_set{0};
-    cudaError_t e = ensure_smem_limit(decode_kernel<T, D>, smem, smem_set);
+    cudaError_t e = ensure_smem_limit(decode_kernel<T, D, kPaged>, smem, smem_set);
     if (e != cudaSuccess) return e;
-    decode_kernel<T, D><<<grid, kThreads, smem, s>>>(p);
+    decode_kernel<T, D, kPaged><<<grid, kThreads, smem, s>>>(p);
     return cudaSuccess;
+}
+
+template <typename T, int D>
+cudaError_t launch_typed(const DecodeParams &p, unsigned grid, cudaStream_t s) {
+    return p.page_table ? launch_form<T, D, true>(p, grid, s) : launch_form<T, D, false>(p, grid, s);
 }
 
 }  // namespace

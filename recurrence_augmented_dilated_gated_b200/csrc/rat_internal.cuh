@@ -107,6 +107,18 @@ __host__ __device__ __forceinline__ void cache_rows_of(long long j, int D, int W
     ring_row = (D > 1 && W > 0) ? S + j % W : -1;
 }
 
+// Element offset of (logical row `row`, channel 0) of (b, h) in a cache: the
+// dense [B,H,R,d] block, or the page the table names ([num_pages,H,P,d]); -1
+// when the table names no valid page.
+__host__ __device__ __forceinline__ long long cache_offset(const int *table, int pps, int page_rows, int num_pages,
+                                                           long long cache_R, int H, int d, int b, int h,
+                                                           long long row) {
+    if (!table) return (((long long)b * H + h) * cache_R + row) * d;
+    const int pg = table[(long long)b * pps + row / page_rows];
+    if (pg < 0 || pg >= num_pages) return -1;
+    return (((long long)pg * H + h) * page_rows + row % page_rows) * d;
+}
+
 // --------------------------------------------------------------- scan (K1)
 struct ScanParams {
     // 4-D TMA maps (d, H, T, B) of k, v, g (loads) and kt, vt (stores), box
@@ -123,6 +135,8 @@ struct ScanParams {
     int cap;
     int grid;               // cache layout of the fixed-grid reading (grid rows + window ring)
     int one;                // one-tensor form: x[0], g -> out[0] (separate gates, run per tensor)
+    const int *page_table;  // paged cache (null: dense), as DecodeParams
+    int page_rows, pps, num_pages;
     int B, T, H, d;
     int nslices;            // B * nheads
     int nchunks;            // chunks along T per slice
@@ -173,6 +187,10 @@ struct DecodeParams {
     int grid;                    // fixed-grid reading and its cache layout
     int dedupe;                  // the window part skips the dilated set's keys
     int sep;                     // separate key and value gates: g is [2,B,H,d]
+    // paged cache (null table: one dense [B,H,R,d] block): logical row r of
+    // (b, h) at page table[b * pps + r / page_rows], [num_pages, H, page_rows, d]
+    const int *page_table;
+    int page_rows, pps, num_pages;
     float scale_log2;
     int dil[kMaxHeads];
     int win[kMaxHeads];

@@ -472,7 +472,14 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
     const long long S = ((long long)p.cap + Dh - 1) / Dh;
     // the window ring keeps the prefill's last W positions (one writer per row)
     const long long ring_from = (long long)p.T - Wh;
-    const size_t cbase = ((size_t)b * p.H + h) * (size_t)p.cache_R * D + c0;
+    // element offset of (cache row `row`, channel c0) of this head: the dense
+    // block or a page of a paged cache; a page the table does not name validly
+    // is reported and the row left unwritten
+    auto crow = [&](long long row) -> long long {
+        const long long o = cache_offset(p.page_table, p.pps, p.page_rows, p.num_pages, p.cache_R, p.H, D, b, h, row);
+        if (o < 0) report_error(p.hdr, RAT_ERR_INVALID, (int)ticket);
+        return o < 0 ? -1 : o + c0;
+    };
     if (loaded && !kAccurate && rec) {
         // bf16: a = 1 - (1 - a) from the fp16 cache, channel pairs in f32x2
         uint64_t sk2[2] = {f2(sk[0], sk[1]), f2(sk[2], sk[3])}, sv2[2] = {f2(sv[0], sv[1]), f2(sv[2], sv[3])};
@@ -500,15 +507,15 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
                     const long long tt = tc0 + r;
                     long long row0, row1;
                     cache_rows_of(tt, Dh, Wh, S, p.grid, row0, row1);
-                    if (row0 >= 0) {
-                        const size_t e = cbase + (size_t)row0 * D;
-                        *reinterpret_cast<uint2 *>(ck + e) = make_uint2(wk[0], wk[1]);
-                        if (!kOne) *reinterpret_cast<uint2 *>(cv + e) = make_uint2(wv[0], wv[1]);
+                    const long long e0 = row0 >= 0 ? crow(row0) : -1;
+                    if (e0 >= 0) {
+                        *reinterpret_cast<uint2 *>(ck + e0) = make_uint2(wk[0], wk[1]);
+                        if (!kOne) *reinterpret_cast<uint2 *>(cv + e0) = make_uint2(wv[0], wv[1]);
                     }
-                    if (row1 >= 0 && tt >= ring_from) {
-                        const size_t e = cbase + (size_t)row1 * D;
-                        *reinterpret_cast<uint2 *>(ck + e) = make_uint2(wk[0], wk[1]);
-                        if (!kOne) *reinterpret_cast<uint2 *>(cv + e) = make_uint2(wv[0], wv[1]);
+                    const long long e1 = (row1 >= 0 && tt >= ring_from) ? crow(row1) : -1;
+                    if (e1 >= 0) {
+                        *reinterpret_cast<uint2 *>(ck + e1) = make_uint2(wk[0], wk[1]);
+                        if (!kOne) *reinterpret_cast<uint2 *>(cv + e1) = make_uint2(wv[0], wv[1]);
                     }
                 }
             }
@@ -551,13 +558,15 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
                     const long long tt = tc0 + r;
                     long long row0, row1;
                     cache_rows_of(tt, Dh, Wh, S, p.grid, row0, row1);
-                    if (row0 >= 0) {
-                        IO4<T>::store(ck + cbase + (size_t)row0 * D, wk);
-                        if (!kOne) IO4<T>::store(cv + cbase + (size_t)row0 * D, wv);
+                    const long long e0 = row0 >= 0 ? crow(row0) : -1;
+                    if (e0 >= 0) {
+                        IO4<T>::store(ck + e0, wk);
+                        if (!kOne) IO4<T>::store(cv + e0, wv);
                     }
-                    if (row1 >= 0 && tt >= ring_from) {
-                        IO4<T>::store(ck + cbase + (size_t)row1 * D, wk);
-                        if (!kOne) IO4<T>::store(cv + cbase + (size_t)row1 * D, wv);
+                    const long long e1 = (row1 >= 0 && tt >= ring_from) ? crow(row1) : -1;
+                    if (e1 >= 0) {
+                        IO4<T>::store(ck + e1, wk);
+                        if (!kOne) IO4<T>::store(cv + e1, wv);
                     }
                 }
             }

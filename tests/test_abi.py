@@ -135,6 +135,28 @@ def test_topk_sizes_and_argument_checks(lib):
     assert rc == rat.RAT_ERR_INVALID     # more tokens than the cache holds
 
 
+
+def test_paged_cache_descriptor_checks(lib):
+    # host-side checks of the page descriptor, before any launch
+    c = cfg(B=2, H=2, dil=[1, 4], win=[0, 8])
+    cap = 1000
+    R = lib.rat_cache_rows(c.ref(), cap)
+    P = 16
+
+    def step(desc):
+        return lib.rat_decode_step_paged(c.ref(), P, P, P, P, P, P, ctypes.byref(desc), cap, P, P, None, 256, 1 << 30,
+                                         None)
+
+    good = dict(pool_k=16, pool_v=32, page_table=48, page_rows=64, pages_per_seq=-(-R // 64), num_pages=64)
+    for bad in (dict(page_rows=0), dict(num_pages=0), dict(pages_per_seq=-(-R // 64) - 1), dict(pool_k=None),
+                dict(page_table=8)):
+        d = dict(good)
+        d.update(bad)
+        assert step(rat.rat_paged_cache(**d)) == rat.RAT_ERR_INVALID, bad
+    assert lib.rat_decode_step_paged(c.ref(), P, P, P, P, P, P, None, cap, P, P, None, 256, 1 << 30,
+                                     None) == rat.RAT_ERR_INVALID
+
+
 def call_scan(lib, c, **ptrs):
     P = dict(k=16, v=16, g=16, init_k=None, init_v=None, kt=16, vt=16, fk=None, fv=None, ck=None, cv=None, cap=0,
              ws=256, wsb=1 << 40)

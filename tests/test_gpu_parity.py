@@ -736,6 +736,90 @@ def test_separate_gates_decode_steps(dtype):
                     recur=[0, 1, 1, 1], mu=2.0, seed=25, sep=True)
 
 
+# ---------------------------------------------------------- paged decode cache
+
+
+def _paged_setup(grid):
+    B, T, steps, H, d = 3, 700, 4, 3, 128
+    dil, win, recur = [1, 4, 7], [0, 16, 100], [0, 1, 1]
+    cap = T + steps
+    dtype = torch.bfloat16
+    q, k, v, g = inputs(B, T + steps, H, d, dtype, seed=61)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur, grid=grid)
+    R = rat.rat_cache_rows(cfg, cap)
+    P = 48                      # not a multiple of a ring stage (64 rows): stages straddle pages
+    pps = -(-R // P)
+    num_pages = B * pps + 5
+    perm = torch.randperm(num_pages, generator=torch.Generator().manual_seed(7))[:B * pps]
+    table = perm.view(B, pps).to(torch.int32).to(DEV)
+    return B, T, steps, H, d, cap, dtype, q, k, v, g, cfg, R, P, num_pages, table
+
+
+@pytest.mark.parametrize("grid", [False, True])
+def test_paged_decode_equals_dense(grid):
+    # the same logical rows in shuffled pages: every output bit-identical
+    B, T, steps, H, d, cap, dtype, q, k, v, g, cfg, R, P, num_pages, table = _paged_setup(grid)
+    ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
+    cv = torch.zeros_like(ck)
+    pool_k = torch.zeros(num_pages, H, P, d, dtype=dtype, device=DEV)
+    pool_v = torch.zeros_like(pool_k)
+    cache = rat.paged_cache(cfg, pool_k, pool_v, table, cap)
+    states = [torch.empty(B, H, d, device=DEV) for _ in range(4)]
+    ws = rat.workspace(cfg, rat.RAT_OP_SCAN)
+    pre = (k[:, :T].contiguous(), v[:, :T].contiguous(), g[:, :T].contiguous())
+    rat.rat_scan_prefill(cfg, *pre, None, None, None, None, states[0], states[1], ck, cv, cap, ws)
+    rat.rat_scan_prefill_paged(cfg, *pre, None, None, None, None, states[2], states[3], cache=cache, cache_cap=cap,
+                               ws=ws)
+    rat.rat_check_status(ws)
+    wsd = rat.workspace(cfg, rat.RAT_OP_DECODE, cap)
+    for s in range(steps):
+        t = T + s
+        pos = torch.full((B,), t, dtype=torch.int32, device=DEV)
+        tok = (q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(), g[:, t].contiguous())
+        o1, o2 = torch.empty(B, H, d, dtype=dtype, device=DEV), torch.empty(B, H, d, dtype=dtype, device=DEV)
+        l1, l2 = torch.empty(B, H, device=DEV), torch.empty(B, H, device=DEV)
+        rat.rat_decode_step(cfg, *tok, states[0], states[1], ck, cv, cap, pos, o1, l1, wsd)
+        rat.rat_decode_step_paged(cfg, *tok, states[2], states[3], cache, cap, pos, o2, l2, wsd)
+        rat.rat_check_status(wsd)
+        assert torch.equal(o1, o2) and torch.equal(l1, l2), "step %d" % s
+    assert torch.equal(states[0], states[2]) and torch.equal(states[1], states[3])
+    # every logical row sits in the page the table names
+    r = torch.arange(R, device=DEV)
+    for b in range(B):
+        pg = table[b, r // P].long()
+        for h in range(H):
+            assert torch.equal(pool_k[pg, h, r % P], ck[b, h]) and torch.equal(pool_v[pg, h, r % P], cv[b, h])
+
+
+def test_paged_decode_invalid_page_is_reported():
+    # a table entry of -1 on a page the step reads: every head of entry 1 reads
+    # logical rows from 0 at t = 700 (residue 0 of D = 1, 4, 7), so all are
+    # skipped (o = 0) and RAT_ERR_INVALID recorded; the other entries are not
+    B, T, steps, H, d, cap, dtype, q, k, v, g, cfg, R, P, num_pages, table = _paged_setup(False)
+    pool_k = torch.zeros(num_pages, H, P, d, dtype=dtype, device=DEV)
+    pool_v = torch.zeros_like(pool_k)
+    cache = rat.paged_cache(cfg, pool_k, pool_v, table, cap)
+    sk, sv = torch.empty(B, H, d, device=DEV), torch.empty(B, H, d, device=DEV)
+    ws = rat.workspace(cfg, rat.RAT_OP_SCAN)
+    rat.rat_scan_prefill_paged(cfg, k[:, :T].contiguous(), v[:, :T].contiguous(), g[:, :T].contiguous(), None,
+                               None, None, None, sk, sv, cache=cache, cache_cap=cap, ws=ws)
+    rat.rat_check_status(ws)
+    ok = table.clone()
+    table[1, 0] = -1            # head 0 of entry 1 (D = 1) reads logical rows from 0
+    t = T
+    pos = torch.full((B,), t, dtype=torch.int32, device=DEV)
+    o = torch.empty(B, H, d, dtype=dtype, device=DEV)
+    wsd = rat.workspace(cfg, rat.RAT_OP_DECODE, cap)
+    rat.rat_decode_step_paged(cfg, q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(),
+                              g[:, t].contiguous(), sk, sv, cache, cap, pos, o, None, wsd)
+    with pytest.raises(rat.RatError) as err:
+        rat.rat_check_status(wsd)
+    assert err.value.status == rat.RAT_ERR_INVALID
+    assert torch.count_nonzero(o[1]) == 0
+    assert torch.count_nonzero(o[0]) > 0 and torch.count_nonzero(o[2]) > 0
+    table.copy_(ok)
+
+
 def test_decode_bad_position_is_reported():
     B, H, d = 2, 2, 64
     cfg = make_cfg(B, 1, H, d, torch.bfloat16, [2, 2], [0, 0])
