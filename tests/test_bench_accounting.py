@@ -65,3 +65,15 @@ def test_profile_traffic_needs_the_captured_source(tmp_path, monkeypatch):
     assert bench.profile_traffic("missing") is None
     src.write_text("kernel source, changed\n")
     assert bench.profile_traffic("k_case", "x") is None       # the counters belong to older code
+
+
+@pytest.mark.parametrize("t,block,K", [(0, 4, 2), (3, 4, 2), (4, 4, 2), (9, 4, 2), (40, 4, 2), (40, 4, 64),
+                                       (16450, 64, 16)])
+def test_topk_decode_bytes_read_the_kept_rows_and_the_candidates(t, block, K):
+    B, H, d, elt = 2, 3, 128, 2
+    c = t // block
+    cand = list(range(1, c))
+    kept = {0, c} | set(cand[:K])          # which K does not matter for the byte count
+    rows = sum(1 for j in range(t) if j // block in kept)      # old rows; the new one is in registers
+    per = len(cand) * 2 * d * 4 + rows * 2 * d * elt + d * (5 * elt + 16 + 2 * elt) + 2 * 2 * d * 4
+    assert bench.topk_decode_bytes(B, H, d, t, block, K, elt) == B * H * per
