@@ -249,6 +249,27 @@ def attn_pairs(T, D, W):
     return pairs
 
 
+def variant_pairs(T, D, W, grid=False, dedupe=False):
+    """Unmasked (query, key) pairs of one head under the fixed-grid reading
+    (keys j <= t with j mod D == D-1, plus t once) and/or dedupe (the window
+    part skips the dilated set's keys), in closed form per row."""
+    t = np.arange(T, dtype=np.int64)
+    lo = np.maximum(0, t - W + 1)
+    if grid:
+        on = (t % D) == D - 1
+        n_dil = (t + 1) // D + np.where(on, 0, 1)
+    else:
+        n_dil = t // D + 1
+    n_win = np.minimum(W, t + 1) if W > 0 else np.zeros_like(t)
+    if dedupe and W > 0:
+        if grid:    # grid positions in [lo, t], plus t itself when it is off the grid
+            shared = (t + 1) // D - lo // D + np.where(on, 0, 1)
+        else:       # t, t-D, ... down to lo
+            shared = (t - lo) // D + 1
+        n_win = n_win - shared
+    return float(np.sum(n_dil + n_win))
+
+
 def prefill_work(w):
     """(attention FLOPs, scan bytes) of one prefill step: 4*d FLOPs per pair;
     10 bytes per (token, channel) of a recurrent head (k, v, g read; kt, vt written)."""
@@ -470,6 +491,35 @@ def bench_decode(rat, w, ctx, steps, warmup, world, rank, dev, fill_chunk=8, fla
     return dict(ms=ms, bytes=byts, launches=launches, ctx=ctx)
 
 
+def bench_attn_variant(rat, w, flags, steps, warmup, world, rank, dev):
+    """The attention step alone (rat_dilated_attn_prefill) on the prefill
+    workload under RAT_FLAG_* `flags`; returns ms per launch."""
+    dtype = w.torch_dtype
+    q, k, v, _ = wl.prefill_inputs(w.B, w.T, w.H, w.d, w.gate_mean, dtype, device=dev, seed=11 + rank)
+    cfg = rat.Config(w.B, w.T, w.H, w.d, dtype, w.dil, w.win, w.recur, flags=flags)
+    o = torch.empty_like(q)
+    ws = rat.workspace(cfg, rat.RAT_OP_ATTN, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        rat.rat_dilated_attn_prefill(cfg, q, k, v, o, None, ws, stream=stream)
+    rat.rat_check_status(ws)
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = rat.rat_launch_count()
+    a.record(stream)
+    for _ in range(steps):
+        rat.rat_dilated_attn_prefill(cfg, q, k, v, o, None, ws, stream=stream)
+    b.record(stream)
+    torch.cuda.synchronize()
+    launches = rat.rat_launch_count() - n0
+    rat.rat_check_status(ws)
+    ms = max_over_ranks(a.elapsed_time(b), world, dev) / steps
+    del q, k, v, o, ws
+    torch.cuda.empty_cache()
+    return dict(ms=ms, launches=launches)
+
+
 def topk_decode_bytes(B, H, d, t, block, K, elt=2):
     """Algorithmic HBM bytes of one top-k decode step at position t: the fp32
     statistics of the candidate blocks, the old rows (before t) of the first,
@@ -654,6 +704,8 @@ def main():
                                           flags=rat.RAT_FLAG_GRID_DILATION)
         nxt["paged_decode"] = bench_decode(rat, wd, 4096, args.decode_steps, args.warmup, world, rank, dev,
                                            page_rows=256)
+        att_var = {name: bench_attn_variant(rat, w, f, 3, args.warmup, world, rank, dev)
+                   for name, f in (("grid", rat.RAT_FLAG_GRID_DILATION), ("dedupe", rat.RAT_FLAG_DEDUPE))}
         nxt["topk_decode"] = bench_topk(rat, wd.decode_batch, wd.H, wd.d, 16384, 64, 16, rat.RAT_TOPK_QUEST,
                                         args.decode_steps, args.warmup, world, rank, dev)
 
@@ -712,6 +764,18 @@ def main():
                         "gpu_launches": r["launches"]} for r in dec],
         }
     if nxt:
+        line["attention_variants"] = {}
+        for name, r in att_var.items():
+            fl = sum(w.B * 4.0 * w.d * variant_pairs(w.T, w.dil[h], w.win[h], grid=name == "grid",
+                                                     dedupe=name == "dedupe") for h in range(w.H))
+            tf = fl / (r["ms"] * 1e-3) / 1e12
+            line["attention_variants"][name] = {
+                "what": {"grid": "fixed-grid dilation (j mod D == D-1, plus t)",
+                         "dedupe": "window part without the dilated set's keys"}[name],
+                "ms_per_launch": r["ms"], "value": w.B * w.T * world / (r["ms"] * 1e-3), "unit": "tok/s",
+                "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": tf / peaks["bf16_tflops"], "traffic": None},
+                "gpu_launches": r["launches"]}
         wd = wl.DECODE_D16
         desc = {"grid_decode": "fixed-grid dilation, grid cache + window ring, ctx 4096",
                 "paged_decode": "residue cache in 256-row pages (shuffled), ctx 4096",

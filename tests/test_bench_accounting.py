@@ -77,3 +77,17 @@ def test_topk_decode_bytes_read_the_kept_rows_and_the_candidates(t, block, K):
     rows = sum(1 for j in range(t) if j // block in kept)      # old rows; the new one is in registers
     per = len(cand) * 2 * d * 4 + rows * 2 * d * elt + d * (5 * elt + 16 + 2 * elt) + 2 * 2 * d * 4
     assert bench.topk_decode_bytes(B, H, d, t, block, K, elt) == B * H * per
+
+
+@pytest.mark.parametrize("grid", [False, True])
+@pytest.mark.parametrize("dedupe", [False, True])
+@pytest.mark.parametrize("T,D,W", [(1, 1, 0), (37, 4, 5), (50, 7, 100), (64, 1, 8), (100, 9, 1), (90, 30, 61)])
+def test_variant_pairs_count_the_reading_key_sets(grid, dedupe, T, D, W):
+    n = 0
+    for t in range(T):
+        dil = {j for j in range(t + 1) if ((j % D == D - 1 or j == t) if grid else (t - j) % D == 0)}
+        win = {j for j in range(t + 1) if W > 0 and j >= t - W + 1}
+        n += len(dil) + len(win - dil if dedupe else win)
+    assert bench.variant_pairs(T, D, W, grid=grid, dedupe=dedupe) == n
+    if not grid and not dedupe:
+        assert bench.attn_pairs(T, D, W) == n
