@@ -105,7 +105,17 @@ typedef enum {
  * window) and recurrence flag recur[h] (0 = no recurrence; NULL = all heads
  * recurrent) -- the hybrid head compositions of the RAT+ Abstract.
  * Limits of this library version: d in {64, 128}; 1 <= H <= 256; B, T >= 0;
- * B*T*H*d < 2^40 elements.  An empty batch or sequence (B*T == 0) launches
+ * B*T*H*d < 2^40 elements.
+ *
+ * Chunked prefill (t0 > 0): a call covers positions t0 .. t0+T-1 of its
+ * sequences.  Token inputs (q, k, v, g) and outputs (o, lse) hold those T
+ * positions; the augmented keys/values kt, vt are history buffers
+ * [B, t_cap, H, d] (t_cap = 0 means t0 + T) whose rows 0 .. t0+T-1 hold
+ * positions 0 .. t0+T-1, so one buffer serves every chunk: the scan writes rows t0 ..
+ * t0+T-1 (init_k/init_v carry the state after position t0-1) and the
+ * attention reads all rows, so the chunks of a prefill give the one-shot
+ * result.  Decode-cache rows go to positions t0 + t.  rat_mix_prefill then
+ * needs caller kt/vt.  Decode steps ignore t0.  An empty batch or sequence (B*T == 0) launches
  * no kernel; a prefill then only copies init (or zero) to final.
  */
 typedef struct {
@@ -116,6 +126,8 @@ typedef struct {
     const uint8_t *recur;    /* host [H] or NULL */
     float scale;             /* <= 0 selects 1/sqrt(d) */
     uint32_t flags;          /* RAT_FLAG_* bits, 0 = the defaults above */
+    int t0;                  /* position of this call's first token (chunked prefill), 0 = a whole prefill */
+    int t_cap;               /* rows per batch entry of the kt/vt history, >= t0 + T; 0 = t0 + T */
 } rat_cfg;
 
 /* Fixed-grid reading of dilation (see "dilation" above) for every head of the

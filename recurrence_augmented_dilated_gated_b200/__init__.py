@@ -47,7 +47,7 @@ class rat_cfg(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("dil", ctypes.POINTER(ctypes.c_int32)),
                 ("win", ctypes.POINTER(ctypes.c_int32)), ("recur", ctypes.POINTER(ctypes.c_uint8)),
-                ("scale", ctypes.c_float), ("flags", ctypes.c_uint32)]
+                ("scale", ctypes.c_float), ("flags", ctypes.c_uint32), ("t0", ctypes.c_int), ("t_cap", ctypes.c_int)]
 
 
 class rat_paged_cache(ctypes.Structure):
@@ -105,7 +105,7 @@ def load_library(path=LIB_PATH):
 class Config:
     """Owns a rat_cfg and the host arrays it points to."""
 
-    def __init__(self, B, T, H, d, dtype, dil, win, recur=None, scale=0.0, flags=0):
+    def __init__(self, B, T, H, d, dtype, dil, win, recur=None, scale=0.0, flags=0, t0=0, t_cap=0):
         self.dil = np.ascontiguousarray(dil, dtype=np.int32)
         self.win = np.ascontiguousarray(win, dtype=np.int32)
         self.recur = None if recur is None else np.ascontiguousarray(recur, dtype=np.uint8)
@@ -116,7 +116,7 @@ class Config:
                          self.dil.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
                          self.win.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
                          None if self.recur is None else self.recur.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
-                         float(scale), int(flags))
+                         float(scale), int(flags), int(t0), int(t_cap))
 
     @property
     def torch_dtype(self):
@@ -124,12 +124,18 @@ class Config:
 
     def replace(self, **kw):
         args = dict(B=self.c.B, T=self.c.T, H=self.c.H, d=self.c.d, dtype=self.c.dtype, dil=self.dil,
-                    win=self.win, recur=self.recur, scale=self.c.scale, flags=self.c.flags)
+                    win=self.win, recur=self.recur, scale=self.c.scale, flags=self.c.flags, t0=self.c.t0,
+                    t_cap=self.c.t_cap)
         args.update(kw)
         return Config(**args)
 
     def ref(self):
         return ctypes.byref(self.c)
+
+    @property
+    def history_shape(self):
+        """Shape of kt / vt: [B, t_cap or t0 + T, H, d] (the history in a chunked prefill)."""
+        return (self.c.B, self.c.t_cap or self.c.t0 + self.c.T, self.c.H, self.c.d)
 
     def gate_shape(self, tok):
         """Shape of the gate tensor for token tensors of shape `tok` (a second,
@@ -210,7 +216,7 @@ def rat_scan_prefill(cfg, k, v, g, init_k=None, init_v=None, kt=None, vt=None, f
     dt = cfg.torch_dtype
     args = [_ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
             _ptr(init_k, "init_k", torch.float32, st, True), _ptr(init_v, "init_v", torch.float32, st, True),
-            _ptr(kt, "kt", dt, tok, True), _ptr(vt, "vt", dt, tok, True),
+            _ptr(kt, "kt", dt, cfg.history_shape, True), _ptr(vt, "vt", dt, cfg.history_shape, True),
             _ptr(final_k, "final_k", torch.float32, st, True), _ptr(final_v, "final_v", torch.float32, st, True),
             _ptr(cache_k, "cache_k", dt, None, True), _ptr(cache_v, "cache_v", dt, None, True), int(cache_cap),
             _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream)]
@@ -221,7 +227,8 @@ def rat_dilated_attn_prefill(cfg, q, kt, vt, o, lse=None, ws=None, stream=None):
     c = cfg.c
     tok = (c.B, c.T, c.H, c.d)
     dt = cfg.torch_dtype
-    args = [_ptr(q, "q", dt, tok), _ptr(kt, "kt", dt, tok), _ptr(vt, "vt", dt, tok), _ptr(o, "o", dt, tok),
+    args = [_ptr(q, "q", dt, tok), _ptr(kt, "kt", dt, cfg.history_shape), _ptr(vt, "vt", dt, cfg.history_shape),
+            _ptr(o, "o", dt, tok),
             _ptr(lse, "lse", torch.float32, (c.B, c.H, c.T), True), _ptr(ws, "ws", torch.uint8), ws.numel(),
             _stream(stream)]
     _check(load_library().rat_dilated_attn_prefill(cfg.ref(), *args), "rat_dilated_attn_prefill")
@@ -236,7 +243,7 @@ def rat_mix_prefill(cfg, q, k, v, g, init_k=None, init_v=None, o=None, lse=None,
     args = [_ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
             _ptr(init_k, "init_k", torch.float32, st, True), _ptr(init_v, "init_v", torch.float32, st, True),
             _ptr(o, "o", dt, tok), _ptr(lse, "lse", torch.float32, (c.B, c.H, c.T), True),
-            _ptr(kt, "kt", dt, tok, True), _ptr(vt, "vt", dt, tok, True),
+            _ptr(kt, "kt", dt, cfg.history_shape, True), _ptr(vt, "vt", dt, cfg.history_shape, True),
             _ptr(final_k, "final_k", torch.float32, st, True), _ptr(final_v, "final_v", torch.float32, st, True),
             _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream)]
     _check(load_library().rat_mix_prefill(cfg.ref(), *args), "rat_mix_prefill")
@@ -341,7 +348,7 @@ def rat_scan_prefill_paged(cfg, k, v, g, init_k=None, init_v=None, kt=None, vt=N
     dt = cfg.torch_dtype
     args = [_ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
             _ptr(init_k, "init_k", torch.float32, st, True), _ptr(init_v, "init_v", torch.float32, st, True),
-            _ptr(kt, "kt", dt, tok, True), _ptr(vt, "vt", dt, tok, True),
+            _ptr(kt, "kt", dt, cfg.history_shape, True), _ptr(vt, "vt", dt, cfg.history_shape, True),
             _ptr(final_k, "final_k", torch.float32, st, True), _ptr(final_v, "final_v", torch.float32, st, True),
             ctypes.byref(cache), int(cache_cap), _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream)]
     _check(load_library().rat_scan_prefill_paged(cfg.ref(), *args), "rat_scan_prefill_paged")
@@ -375,8 +382,11 @@ def rat_debug_set_scan_stall(ws, ticket, spin_limit_ns=0, stream=None):
 
 
 def mix_prefill(cfg, q, k, v, g, init_k=None, init_v=None, want_kv=False, want_lse=True, ws=None, stream=None):
-    """Allocate outputs with torch and run rat_mix_prefill.  Returns a dict."""
+    """Allocate outputs with torch and run rat_mix_prefill.  Returns a dict.
+    (A chunked prefill, t0 > 0, calls rat_mix_prefill with its kt/vt history.)"""
     c = cfg.c
+    if c.t0 > 0:
+        raise ValueError("mix_prefill allocates its own kt/vt: with t0 > 0 call rat_mix_prefill with the history")
     dev = q.device
     o = torch.empty_like(q)
     lse = torch.empty((c.B, c.H, c.T), dtype=torch.float32, device=dev) if want_lse else None

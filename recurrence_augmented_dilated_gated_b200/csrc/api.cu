@@ -73,6 +73,11 @@ rat_status check_cfg(const rat_cfg *c, bool need_T = true) {
     const double elems = (double)c->B * (need_T ? (double)c->T : 1.0) * c->H * c->d;
     if (elems >= 1099511627776.0) return fail(RAT_ERR_INVALID, "B*T*H*d too large");
     if (!(c->scale == c->scale)) return fail(RAT_ERR_INVALID, "scale is NaN");
+    if (c->t0 < 0 || (long long)c->t0 + c->T > 0x7fffffffLL) return fail(RAT_ERR_INVALID, "t0 %d out of range", c->t0);
+    if (c->t_cap != 0 && (long long)c->t_cap < (long long)c->t0 + c->T)
+        return fail(RAT_ERR_INVALID, "t_cap %d < t0 + T", c->t_cap);
+    if (need_T && (double)c->B * ((double)c->t0 + c->T + c->t_cap) * c->H * c->d >= 1099511627776.0)
+        return fail(RAT_ERR_INVALID, "B*(t0+T)*H*d too large");
     if (c->flags & ~(RAT_FLAG_GRID_DILATION | RAT_FLAG_DEDUPE | RAT_FLAG_SEPARATE_GATES))
         return fail(RAT_ERR_INVALID, "unknown flags 0x%x", c->flags);
     return RAT_OK;
@@ -81,6 +86,9 @@ rat_status check_cfg(const rat_cfg *c, bool need_T = true) {
 bool head_recur(const rat_cfg *c, int h) { return c->recur == nullptr || c->recur[h] != 0; }
 
 bool grid_mode(const rat_cfg *c) { return (c->flags & RAT_FLAG_GRID_DILATION) != 0; }
+
+// rows per batch entry of the kt/vt history (t0 + T unless the caller's buffer is longer)
+int hist_rows(const rat_cfg *c) { return c->t_cap ? c->t_cap : c->t0 + c->T; }
 
 bool dedupe_mode(const rat_cfg *c) { return (c->flags & RAT_FLAG_DEDUPE) != 0; }
 
@@ -188,8 +196,10 @@ rat_status scan_pass(const rat_cfg *c, const Layout &L, ScanParams &p, char *ws,
     // the one-tensor form reads slot 1 of neither list: repeat slot 0 there
     const void *srcs[5] = {p.x[0], p.x[1] ? p.x[1] : p.x[0], p.g, p.out[0], p.out[1] ? p.out[1] : p.out[0]};
     p.use_tma_out = p.out[0] != nullptr ? 1 : 0;
+    // inputs hold the call's T positions; kt / vt are the [B, t0+T, H, d] history
     for (int i = 0; i < (p.use_tma_out ? 5 : 3); ++i)
-        if (!encode_map_tokens(&p.tmap[i], srcs[i], c->dtype, c->B, c->T, c->H, c->d, p.chunk_len))
+        if (!encode_map_tokens(&p.tmap[i], srcs[i], c->dtype, c->B, i < 3 ? c->T : c->t0 + c->T,
+                               i < 3 ? c->T : hist_rows(c), c->H, c->d, p.chunk_len))
             return fail(RAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (scan operand %d)", i);
     // zero the ticket and the chunk flags (one contiguous range)
     cudaError_t e = cudaMemsetAsync(ws + L.ticket, 0, L.agg - L.ticket, s);
@@ -221,6 +231,7 @@ rat_status run_scan(const rat_cfg *c, const Layout &L, const void *k, const void
     p.cache_R = ck ? cache_rows(c, cap) : 0;
     p.grid = grid_mode(c) ? 1 : 0;
     p.B = c->B; p.T = c->T; p.H = c->H; p.d = c->d;
+    p.t0 = c->t0;
     int n = 0, n_plain = 0;
     unsigned char plain[kMaxHeads];
     for (int h = 0; h < c->H; ++h) {
@@ -269,7 +280,11 @@ bool grid_head(const rat_cfg *c, int h) { return grid_mode(c) && c->dil[h] > 1; 
 // A head runs on the tensor-core kernel when its operands are bf16 and its
 // dilation divides T (the strided TMA view needs whole subsequences);
 // otherwise the fp32 CUDA-core kernel computes it.
-bool tc_head(const rat_cfg *c, int h) { return c->dtype == RAT_BF16 && c->T % c->dil[h] == 0; }
+// (A chunked prefill also needs t0 % D == 0: its residues line up with the
+// history's.)
+bool tc_head(const rat_cfg *c, int h) {
+    return c->dtype == RAT_BF16 && c->T % c->dil[h] == 0 && c->t0 % c->dil[h] == 0;
+}
 
 // One tensor-core launch over `heads` (kind kTcDilated, kTcWindow or kTcGrid),
 // grouped into classes of equal (dilation, K/V source).
@@ -286,6 +301,9 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, int ki
         P.B = c->B; P.T = c->T; P.H = c->H;
         P.kind = kind;
         P.q = q;
+        P.t0 = c->t0;
+        P.Tk = c->t0 + c->T;
+        P.Th = hist_rows(c);
         P.scale_log2 = scale_of(c) * 1.4426950408889634f;
         P.o = o; P.lse_user = lse; P.lse_dil = lse_dil;
         P.hdr = reinterpret_cast<WsHeader *>(ws);
@@ -341,9 +359,11 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, int ki
             const void *vb = keys[ci].raw ? vraw : vt;
             P.kself[oi] = kb;
             P.vself[oi] = vb;
-            if (!encode_map_5d(&P.tq[oi], q, c->B, c->T, c->H, c->d, kind == kTcGrid ? 1 : C.D, kTcRowsQ) ||
-                !encode_map_5d(&P.tk[oi], kb, c->B, c->T, c->H, c->d, C.D, kTcRowsKV) ||
-                !encode_map_5d(&P.tv[oi], vb, c->B, c->T, c->H, c->d, C.D, kTcRowsKV))
+            // raw k / v (heads without recurrence, mix prefill) hold the call's rows only
+            const int kv_rows = keys[ci].raw ? c->T : P.Th;
+            if (!encode_map_5d(&P.tq[oi], q, c->B, c->T, c->T, c->H, c->d, kind == kTcGrid ? 1 : C.D, kTcRowsQ) ||
+                !encode_map_5d(&P.tk[oi], kb, c->B, P.Tk, kv_rows, c->H, c->d, C.D, kTcRowsKV) ||
+                !encode_map_5d(&P.tv[oi], vb, c->B, P.Tk, kv_rows, c->H, c->d, C.D, kTcRowsKV))
                 return fail(RAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (dilation %d)", C.D);
         }
         P.prefix[ncls] = pref;
@@ -399,6 +419,8 @@ rat_status run_attn(const rat_cfg *c, const Layout &L, const void *q, const void
         p.q = q; p.kt = kt; p.vt = vt; p.kraw = kraw; p.vraw = vraw;
         p.o = o; p.lse = lse;
         p.B = c->B; p.T = c->T; p.H = c->H; p.d = c->d;
+        p.t0 = c->t0;
+        p.Th = hist_rows(c);
         p.scale_log2 = scale_of(c) * 1.4426950408889634f;
         p.grid = grid_mode(c) ? 1 : 0;
         p.dedupe = dedupe_mode(c) ? 1 : 0;
@@ -492,7 +514,8 @@ rat_status scan_prefill(const rat_cfg *cfg, const void *k, const void *v, const 
     if ((cache_k == nullptr) != (cache_v == nullptr))
         return fail(RAT_ERR_INVALID, "cache_k and cache_v must be given together");
     if (!kt && !cache_k) return fail(RAT_ERR_INVALID, "no output: give kt/vt and/or cache_k/cache_v");
-    if (cache_k && cache_cap < cfg->T) return fail(RAT_ERR_INVALID, "cache_cap %d < T %d", cache_cap, cfg->T);
+    if (cache_k && cache_cap < (long long)cfg->t0 + cfg->T)
+        return fail(RAT_ERR_INVALID, "cache_cap %d < t0 + T = %lld", cache_cap, (long long)cfg->t0 + cfg->T);
     Layout L;
     st = check_ws(cfg, RAT_OP_SCAN, 0, ws, ws_bytes, &L);
     if (st != RAT_OK) return st;
@@ -592,6 +615,10 @@ rat_status rat_mix_prefill(const rat_cfg *cfg, const void *q, const void *k, con
     CHECK_OPT(final_k, "final_k"); CHECK_OPT(final_v, "final_v");
     if ((kt == nullptr) != (vt == nullptr)) return fail(RAT_ERR_INVALID, "kt and vt must be given together");
     const bool caller_kv = kt != nullptr;
+    if (cfg->t0 > 0 && !caller_kv)
+        return fail(RAT_ERR_INVALID, "a chunked prefill (t0 > 0) needs the caller's kt/vt history");
+    if (!caller_kv && cfg->t_cap != 0 && cfg->t_cap != cfg->T)
+        return fail(RAT_ERR_INVALID, "t_cap describes the caller's kt/vt; the workspace keeps T rows");
     Layout L;
     st = check_ws(cfg, caller_kv ? RAT_OP_MIX_CALLER_KV : RAT_OP_MIX, 0, ws, ws_bytes, &L);
     if (st != RAT_OK) return st;

@@ -69,21 +69,24 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(const AttnParams
     const long long row = (long long)blockIdx.x * kWarps + (threadIdx.x >> 5);
     const long long nrows = (long long)p.B * p.H * p.T;
     if (row >= nrows) return;
-    // rows ordered (b, h, t)
-    const long long t = row % p.T;
+    // rows ordered (b, h, t); t is the position, tl the row of this call
+    const long long tl = row % p.T;
+    const long long t = p.t0 + tl;
     const int h = (int)((row / p.T) % p.H);
     const int b = (int)(row / ((long long)p.T * p.H));
     if (p.skip[h]) return;  // uniform across the warp (one row per warp)
     const int d = p.d;
     const size_t rs = (size_t)p.H * d;
-    const size_t hb = ((size_t)b * p.T * p.H + h) * d;  // (b, t=0, h, 0)
+    const size_t hb = ((size_t)b * p.T * p.H + h) * d;                        // (b, row 0, h, 0) of q and o
+    // (b, position 0, h, 0) of kt, vt: Th rows per batch entry (raw k, v: the call's T)
+    const size_t hk = ((size_t)b * (size_t)(p.use_raw[h] ? p.T : p.Th) * p.H + h) * d;
     const T *qb = static_cast<const T *>(p.q) + hb;
-    const T *kb = static_cast<const T *>(p.use_raw[h] ? p.kraw : p.kt) + hb;
-    const T *vb = static_cast<const T *>(p.use_raw[h] ? p.vraw : p.vt) + hb;
+    const T *kb = static_cast<const T *>(p.use_raw[h] ? p.kraw : p.kt) + hk;
+    const T *vb = static_cast<const T *>(p.use_raw[h] ? p.vraw : p.vt) + hk;
 
     float q[CPL];
 #pragma unroll
-    for (int i = 0; i < CPL; ++i) q[i] = ld1<T>(qb + (size_t)t * rs + lane + 32 * i) * p.scale_log2;
+    for (int i = 0; i < CPL; ++i) q[i] = ld1<T>(qb + (size_t)tl * rs + lane + 32 * i) * p.scale_log2;
 
     const int D = p.dil[h], W = p.win[h];
     RowState<CPL> dil, wnd;
@@ -112,11 +115,11 @@ __global__ void __launch_bounds__(kWarps * 32) attn_simt_kernel(const AttnParams
         m = mn;
     }
     const float inv = 1.f / l;
-    T *ob = static_cast<T *>(p.o) + hb + (size_t)t * rs;
+    T *ob = static_cast<T *>(p.o) + hb + (size_t)tl * rs;
 #pragma unroll
     for (int i = 0; i < CPL; ++i) st1<T>(ob + lane + 32 * i, acc[i] * inv);
     if (p.lse && lane == 0)
-        p.lse[((size_t)b * p.H + h) * p.T + t] = (m + log2f(l)) * 0.69314718055994531f;
+        p.lse[((size_t)b * p.H + h) * p.T + tl] = (m + log2f(l)) * 0.69314718055994531f;
 }
 
 }  // namespace

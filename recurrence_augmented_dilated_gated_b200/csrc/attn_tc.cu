@@ -218,6 +218,14 @@ struct Plan {
     bool valid[kSub];
 };
 
+// Where a unit's query rows sit in the key rows: a chunked prefill's queries
+// start at position t0, i.e. subsequence row t0 / D of the dilated part (t0 is
+// a multiple of D there) and position t0 of the window and grid parts.
+template <int kKind>
+__device__ __forceinline__ int query_offset(const TcParams &p, const TcClass &C) {
+    return kKind == kTcDilated ? p.t0 / C.D : p.t0;
+}
+
 template <int kKind>
 __device__ __forceinline__ Plan make_plan(const TcParams &p, const Unit &u) {
     Plan pl;
@@ -225,21 +233,22 @@ __device__ __forceinline__ Plan make_plan(const TcParams &p, const Unit &u) {
     const int n = C.n;
     const int q0 = 2 * BM * u.m;
     const int W = p.win[u.h];
+    const int qo = query_offset<kKind>(p, C);
     for (int i = 0; i < kSub; ++i) {
         const int qmin = q0 + BM * i;
         pl.valid[i] = qmin < n;
+        const int qlast = qo + min(qmin + BM - 1, n - 1);   // the sub-tile's last row, in key units
         if (kKind == kTcGrid) {
             // grid keys g <= (t+1)/D - 1 for the sub-tile's last row t; a tile
             // whose rows have no grid key yet keeps tile 0, fully masked
-            const int qlast = min(qmin + BM - 1, n - 1);
             pl.hi[i] = max(0, ((qlast + 1) / C.D - 1) / BN);
         } else {
-            pl.hi[i] = qmin / BN;
+            pl.hi[i] = qlast / BN;
         }
         if (kKind != kTcWindow && kKind != kTcWindowDedupe) {
             pl.lo[i] = 0;
         } else {
-            const int first = qmin - W + 1;  // earliest key of the sub-tile's first row
+            const int first = qo + qmin - W + 1;  // earliest key of the sub-tile's first row
             pl.lo[i] = first > 0 ? first / BN : 0;
         }
     }
@@ -685,6 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const int qmin = 2 * BM * u.m + BM * sub;                 // first row of the sub-tile
             const int qi = qmin + row;                                // subsequence row / position
             const int W = p.win[u.h];
+            const int qo = query_offset<kKind>(p, C);
             const int lo_s = sub ? pl.lo[1] : pl.lo[0];
             const int nt = (sub ? pl.valid[1] : pl.valid[0]) ? (sub ? pl.hi[1] : pl.hi[0]) - lo_s + 1 : 0;
             Excl xcl;
@@ -699,13 +709,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 // mask: causal on subsequence rows (dilated part); keys in (qi - W, qi] (window
                 // part); grid keys g <= (qi+1)/D - 1 (grid part)
                 const int ks = BN * j;
-                const bool full = kGrid ? (ks + BN - 1 <= (qmin + 1) / C.D - 1)
-                                  : !kWin ? (ks + BN - 1 <= qmin)
-                                          : (ks + BN - 1 <= qmin && ks > qmin + BM - 1 - W);
+                const int qa = qo + qi, qamin = qo + qmin;   // the row and the sub-tile's first, in key units
+                const bool full = kGrid ? (ks + BN - 1 <= (qamin + 1) / C.D - 1)
+                                  : !kWin ? (ks + BN - 1 <= qamin)
+                                          : (ks + BN - 1 <= qamin && ks > qamin + BM - 1 - W);
                 // row limits in keys from the tile's first column: key k valid iff k <= lim
-                const int lim = kGrid ? (qi + 1) / C.D - 1 - ks : qi - ks;
+                const int lim = kGrid ? (qa + 1) / C.D - 1 - ks : qa - ks;
                 // window part: and k > lo (no lower limit in the dilated part)
-                const int lo = kWin ? qi - W - ks : INT_MIN / 2;
+                const int lo = kWin ? qa - W - ks : INT_MIN / 2;
                 const int mode = full ? 0 : 2;
                 // dedupe: the dilated set's keys in this tile are k == e0 (mod xd):
                 // k == lim for the residue reading (the row's own key among them);
@@ -768,16 +779,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 // dilated part's row (o, lse) written by the previous launch; for
                 // the grid launch the row's own key (V~_t, score s q_t.K~_t) when
                 // t is off the grid.  Fetched while the last PV runs.
-                const bool mrow = merge && valid_row && (!kGrid || t % C.D != C.D - 1);
+                const bool mrow = merge && valid_row && (!kGrid || (p.t0 + t) % C.D != C.D - 1);
                 uint4 prev[HD / 8];
                 float ld2 = 0.f;
                 if (mrow) {
                     if constexpr (kGrid) {
                         const uint4 *qs = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.q) + orow);
+                        // the row's own key and value: row t0 + t of the [B, t0+T, H, d] history
+                        const size_t hrow = (((size_t)u.b * p.Th + (size_t)(p.t0 + t)) * p.H + u.h) * HD;
                         const uint4 *ks4 =
-                            reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.kself[u.cls]) + orow);
+                            reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.kself[u.cls]) + hrow);
                         const uint4 *vs4 =
-                            reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.vself[u.cls]) + orow);
+                            reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.vself[u.cls]) + hrow);
                         float z = 0.f;
 #pragma unroll
                         for (int q = 0; q < HD / 8; ++q) {
@@ -941,12 +954,12 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int H, int d, int D, int box_rows) {
+bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int Ts, int H, int d, int D, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn || D < 1 || T % D != 0) return false;
     const cuuint64_t e = 2;  // bf16
     const cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)D, (cuuint64_t)(T / D), (cuuint64_t)B};
-    const cuuint64_t strides[4] = {e * d, e * d * H, e * d * H * D, e * d * H * T};
+    const cuuint64_t strides[4] = {e * d, e * d * H, e * d * H * D, e * d * H * Ts};
     const cuuint32_t box[5] = {64, 1, 1, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
@@ -956,12 +969,13 @@ bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int H, int 
 
 // One CTA per SM: each CTA allocates all 512 TMEM columns, so the d = 64
 // variant also asks for more than half of the shared memory.
-bool encode_map_tokens(CUtensorMap *map, const void *base, int dtype, int B, int T, int H, int d, int box_rows) {
+bool encode_map_tokens(CUtensorMap *map, const void *base, int dtype, int B, int T, int Ts, int H, int d,
+                       int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t e = dtype == RAT_BF16 ? 2 : 4;
     const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {e * d, e * d * H, e * d * H * T};
+    const cuuint64_t strides[3] = {e * d, e * d * H, e * d * H * Ts};
     const cuuint32_t box[4] = {(cuuint32_t)d, 1, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(map, dtype == RAT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,

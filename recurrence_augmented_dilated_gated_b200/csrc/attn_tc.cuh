@@ -38,6 +38,8 @@ struct TcParams {
     int ncls;
     int B, T, H;
     int kind;                       // kTcDilated, kTcWindow, kTcGrid or kTcWindowDedupe
+    int t0, Tk, Th;                 // chunked prefill: queries at t0 + t; K/V maps cover Tk = t0 + T rows
+                                    // of a history with Th rows per batch entry
     int grid;                       // fixed-grid reading (the dedupe window's excluded keys)
     float scale_log2;
     const void *q;                  // [B,T,H,d] bf16 (the grid's own-key score)
@@ -55,8 +57,9 @@ struct TcParams {
 
 size_t attn_tc_smem_bytes(int hd);
 cudaError_t launch_attn_tc(const TcParams &p, int hd, cudaStream_t s);
-// 5-D TMA map of a [B,T,H,d] bf16 tensor viewed as (d, H, D, T/D, B), box
-// (64, 1, 1, box_rows, 1); requires T % D == 0.
-bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int H, int d, int D, int box_rows);
+// 5-D TMA map of the first T rows of a [B,Ts,H,d] bf16 tensor (Ts rows per
+// batch entry) viewed as (d, H, D, T/D, B), box (64, 1, 1, box_rows, 1);
+// requires T % D == 0.
+bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int Ts, int H, int d, int D, int box_rows);
 
 }  // namespace rat

@@ -135,6 +135,7 @@ struct ScanParams {
     int cap;
     int grid;               // cache layout of the fixed-grid reading (grid rows + window ring)
     int one;                // one-tensor form: x[0], g -> out[0] (separate gates, run per tensor)
+    int t0;                 // position of the call's first token: out rows and cache positions are t0 + t
     const int *page_table;  // paged cache (null: dense), as DecodeParams
     int page_rows, pps, num_pages;
     int B, T, H, d;
@@ -162,6 +163,8 @@ struct AttnParams {
     float *lse;             // [B,H,T] or null
     int B, T, H, d;
     float scale_log2;       // scale * log2(e)
+    int t0;                 // chunked prefill: rows are positions t0 + t; kt/vt hold t0 + T rows
+    int Th;                 // rows per batch entry of kt/vt
     int grid;               // fixed-grid reading of dilation
     int dedupe;             // the window part skips the dilated set's keys
     int dil[kMaxHeads];
@@ -239,8 +242,10 @@ rat_status set_last_error(rat_status s, const char *msg);
 cudaError_t launch_scan(const ScanParams &p, int dtype, cudaStream_t s);
 // tokens per scan chunk for head dimension d
 int scan_chunk_tokens(int d);
-// 4-D TMA map (d, H, T, B) of a [B,T,H,d] tensor, box (d, 1, box_rows, 1), no swizzle
-bool encode_map_tokens(CUtensorMap *map, const void *base, int dtype, int B, int T, int H, int d, int box_rows);
+// 4-D TMA map (d, H, T, B) of the first T rows of a [B,Ts,H,d] tensor (Ts rows
+// per batch entry), box (d, 1, box_rows, 1), no swizzle
+bool encode_map_tokens(CUtensorMap *map, const void *base, int dtype, int B, int T, int Ts, int H, int d,
+                       int box_rows);
 // final state of the heads in p.head_list, which have no recurrence
 cudaError_t launch_final_of_plain_heads(const ScanParams &p, int dtype, cudaStream_t s);
 cudaError_t launch_attn_simt(const AttnParams &p, int dtype, cudaStream_t s);

@@ -471,7 +471,7 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
     const int Dh = p.head_dil[h], Wh = p.head_win[h];
     const long long S = ((long long)p.cap + Dh - 1) / Dh;
     // the window ring keeps the prefill's last W positions (one writer per row)
-    const long long ring_from = (long long)p.T - Wh;
+    const long long ring_from = (long long)p.t0 + p.T - Wh;
     // element offset of (cache row `row`, channel c0) of this head: the dense
     // block or a page of a paged cache; a page the table does not name validly
     // is reported and the row left unwritten
@@ -504,7 +504,7 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
                 *reinterpret_cast<uint2 *>(tile_k + r * D + c0) = make_uint2(wk[0], wk[1]);
                 *reinterpret_cast<uint2 *>(tile_v + r * D + c0) = make_uint2(wv[0], wv[1]);
                 if (ck) {
-                    const long long tt = tc0 + r;
+                    const long long tt = (long long)p.t0 + tc0 + r;
                     long long row0, row1;
                     cache_rows_of(tt, Dh, Wh, S, p.grid, row0, row1);
                     const long long e0 = row0 >= 0 ? crow(row0) : -1;
@@ -555,7 +555,7 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
                 Smem4<T>::store(tile_k + r * D + c0, wk);
                 Smem4<T>::store(tile_v + r * D + c0, wv);
                 if (ck) {
-                    const long long tt = tc0 + r;
+                    const long long tt = (long long)p.t0 + tc0 + r;
                     long long row0, row1;
                     cache_rows_of(tt, Dh, Wh, S, p.grid, row0, row1);
                     const long long e0 = row0 >= 0 ? crow(row0) : -1;
@@ -581,7 +581,7 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
                 asm volatile(
                     "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"(
                         reinterpret_cast<uint64_t>(&p.tmap[3 + i])),
-                    "r"(0), "r"(h), "r"(tc0), "r"(b), "r"(smem_u32(sbuf + i * kTile))
+                    "r"(0), "r"(h), "r"(p.t0 + tc0), "r"(b), "r"(smem_u32(sbuf + i * kTile))
                     : "memory");
             asm volatile("cp.async.bulk.commit_group;" ::: "memory");
             // the stores must have read shared memory before the CTA exits

@@ -148,6 +148,7 @@ __global__ void __launch_bounds__(kThreads) topk_decode_kernel(const TopkParams 
         const size_t e = bh * D + tid;
         float a[2] = {0.f, 0.f}, oma[2] = {1.f, 1.f};   // keys, values
         if (p.recur[h]) {
+#pragma unroll
             for (int i = 0; i < 2; ++i) {
                 // separate gates: the value gate is the second [B,H,d] tensor
                 const size_t ge = (p.sep && i == 1) ? (size_t)p.B * p.H * D + e : e;

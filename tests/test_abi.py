@@ -157,6 +157,18 @@ def test_paged_cache_descriptor_checks(lib):
                                      None) == rat.RAT_ERR_INVALID
 
 
+
+def test_chunked_prefill_arguments(lib):
+    # t_cap must hold the history; a chunk after the first needs the caller's kt/vt
+    assert lib.rat_workspace_size(cfg(t0=100, t_cap=150).ref(), rat.RAT_OP_SCAN, 0) == 0     # T = 100
+    assert lib.rat_workspace_size(cfg(t0=100, t_cap=200).ref(), rat.RAT_OP_SCAN, 0) > 0
+    assert lib.rat_workspace_size(cfg(t0=-1).ref(), rat.RAT_OP_SCAN, 0) == 0
+    c = cfg(t0=100)
+    P = 16
+    rc = lib.rat_mix_prefill(c.ref(), P, P, P, P, None, None, P, None, None, None, None, None, 256, 1 << 40, None)
+    assert rc == rat.RAT_ERR_INVALID
+
+
 def call_scan(lib, c, **ptrs):
     P = dict(k=16, v=16, g=16, init_k=None, init_v=None, kt=16, vt=16, fk=None, fv=None, ck=None, cv=None, cap=0,
              ws=256, wsb=1 << 40)

@@ -22,10 +22,11 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def make_cfg(B, T, H, d, dtype, dil, win, recur=None, scale=0.0, grid=False, dedupe=False, sep=False):
+def make_cfg(B, T, H, d, dtype, dil, win, recur=None, scale=0.0, grid=False, dedupe=False, sep=False, t0=0,
+             t_cap=0):
     flags = (rat.RAT_FLAG_GRID_DILATION if grid else 0) | (rat.RAT_FLAG_DEDUPE if dedupe else 0)
     flags |= rat.RAT_FLAG_SEPARATE_GATES if sep else 0
-    return rat.Config(B, T, H, d, dtype, dil, win, recur, scale, flags)
+    return rat.Config(B, T, H, d, dtype, dil, win, recur, scale, flags, t0, t_cap)
 
 
 def inputs(B, T, H, d, dtype, mu=2.0, seed=0, device="cpu"):
@@ -818,6 +819,71 @@ def test_paged_decode_invalid_page_is_reported():
     assert torch.count_nonzero(o[1]) == 0
     assert torch.count_nonzero(o[0]) > 0 and torch.count_nonzero(o[2]) > 0
     table.copy_(ok)
+
+
+# ------------------------------------------------------------- chunked prefill
+
+
+@pytest.mark.parametrize("grid", [False, True])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("chunks", [[1024, 512, 448], [1000, 600, 384]])
+def test_chunked_prefill_equals_one_shot(grid, dtype, chunks):
+    # the chunks carry the recurrent state and share one kt/vt history buffer
+    # (t_cap rows per batch entry); the second chunk list starts chunks at
+    # 1000 and 1600, which D = 64 does not divide (those heads run on CUDA cores)
+    B, H, d = 2, 3, 128
+    dil, win, recur = [1, 8, 64], [0, 32, 300], [0, 1, 1]
+    Ttot = sum(chunks)
+    cap = Ttot + 8
+    q, k, v, g = inputs(B, Ttot, H, d, dtype, seed=81)
+    kt = torch.zeros(B, cap, H, d, dtype=dtype, device=DEV)
+    vt = torch.zeros_like(kt)
+    sk = sv = None
+    R = rat.rat_cache_rows(make_cfg(B, 1, H, d, dtype, dil, win, recur, grid=grid), cap)
+    ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
+    cv = torch.zeros_like(ck)
+    outs, lses = [], []
+    t0 = 0
+    for Tc in chunks:
+        cfg = make_cfg(B, Tc, H, d, dtype, dil, win, recur, grid=grid, t0=t0, t_cap=cap)
+        sl = np.s_[:, t0:t0 + Tc]
+        o = torch.empty(B, Tc, H, d, dtype=dtype, device=DEV)
+        lse = torch.empty(B, H, Tc, device=DEV)
+        fk, fv = torch.empty(B, H, d, device=DEV), torch.empty(B, H, d, device=DEV)
+        ws = rat.workspace(cfg, rat.RAT_OP_MIX_CALLER_KV)
+        rat.rat_mix_prefill(cfg, q[sl].contiguous(), k[sl].contiguous(), v[sl].contiguous(), g[sl].contiguous(),
+                            sk, sv, o, lse, kt, vt, fk, fv, ws)
+        # the decode cache of the same chunk (its rows go to positions t0 + t)
+        wss = rat.workspace(cfg, rat.RAT_OP_SCAN)
+        rat.rat_scan_prefill(cfg, k[sl].contiguous(), v[sl].contiguous(), g[sl].contiguous(), sk, sv, None, None,
+                             None, None, ck, cv, cap, wss)
+        rat.rat_check_status(ws)
+        rat.rat_check_status(wss)
+        outs.append(o)
+        lses.append(lse)
+        sk, sv = fk, fv
+        t0 += Tc
+    rk, rfk = oracle.scan(f64(k), f64(g), None, recur)
+    rv, rfv = oracle.scan(f64(v), f64(g), None, recur)
+    ro, rl = oracle.attention(f64(q), rk, rv, dil, win, grid=grid)
+    ft = torch.float32 if dtype == torch.float32 else dtype
+    assert_close(torch.cat(outs, 1), ro, dtype, "o")
+    assert_close(torch.cat(lses, 2), rl, ft, "lse")
+    assert_close(kt[:, :Ttot], rk, dtype, "kt history")
+    assert_close(sk, rfk, ft, "final_k")
+    # every position's cache row (the layout of include/rat.h) holds the
+    # oracle's augmented key and value, written chunk by chunk
+    ckh, cvh = f64(ck), f64(cv)
+    for h, (D, W) in enumerate(zip(dil, win)):
+        S = -(-cap // D)
+        for j in range(Ttot):
+            if grid:
+                rows = ([j // D] if j % D == D - 1 else []) + ([S + j % W] if D > 1 and W > 0 and j >= Ttot - W else [])
+            else:
+                rows = [(j % D) * S + j // D]
+            for r in rows:
+                np.testing.assert_allclose(ckh[:, h, r], rk[:, j, h], rtol=2e-2, atol=2e-2)
+                np.testing.assert_allclose(cvh[:, h, r], rv[:, j, h], rtol=2e-2, atol=2e-2)
 
 
 def test_decode_bad_position_is_reported():
