@@ -249,11 +249,11 @@ def attn_pairs(T, D, W):
     return pairs
 
 
-def variant_pairs(T, D, W, grid=False, dedupe=False):
-    """Unmasked (query, key) pairs of one head under the fixed-grid reading
-    (keys j <= t with j mod D == D-1, plus t once) and/or dedupe (the window
-    part skips the dilated set's keys), in closed form per row."""
-    t = np.arange(T, dtype=np.int64)
+def variant_pairs(T, D, W, grid=False, dedupe=False, t_from=0):
+    """Unmasked (query, key) pairs of one head's rows t_from .. T-1 under the
+    fixed-grid reading (keys j <= t with j mod D == D-1, plus t once) and/or
+    dedupe (the window part skips the dilated set's keys), in closed form per row."""
+    t = np.arange(t_from, T, dtype=np.int64)
     lo = np.maximum(0, t - W + 1)
     if grid:
         on = (t % D) == D - 1
@@ -491,12 +491,16 @@ def bench_decode(rat, w, ctx, steps, warmup, world, rank, dev, fill_chunk=8, fla
     return dict(ms=ms, bytes=byts, launches=launches, ctx=ctx)
 
 
-def bench_attn_variant(rat, w, flags, steps, warmup, world, rank, dev):
+def bench_attn_variant(rat, w, flags, steps, warmup, world, rank, dev, t0=0):
     """The attention step alone (rat_dilated_attn_prefill) on the prefill
-    workload under RAT_FLAG_* `flags`; returns ms per launch."""
+    workload under RAT_FLAG_* `flags`; with t0 > 0, only the queries of
+    positions t0 .. T-1 (the last chunk of a chunked prefill) over the whole
+    history.  Returns ms per launch."""
     dtype = w.torch_dtype
     q, k, v, _ = wl.prefill_inputs(w.B, w.T, w.H, w.d, w.gate_mean, dtype, device=dev, seed=11 + rank)
-    cfg = rat.Config(w.B, w.T, w.H, w.d, dtype, w.dil, w.win, w.recur, flags=flags)
+    if t0 > 0:
+        q = q[:, t0:].contiguous()
+    cfg = rat.Config(w.B, w.T - t0, w.H, w.d, dtype, w.dil, w.win, w.recur, flags=flags, t0=t0)
     o = torch.empty_like(q)
     ws = rat.workspace(cfg, rat.RAT_OP_ATTN, device=dev)
     stream = torch.cuda.current_stream()
@@ -706,6 +710,7 @@ def main():
                                            page_rows=256)
         att_var = {name: bench_attn_variant(rat, w, f, 3, args.warmup, world, rank, dev)
                    for name, f in (("grid", rat.RAT_FLAG_GRID_DILATION), ("dedupe", rat.RAT_FLAG_DEDUPE))}
+        att_var["chunked"] = bench_attn_variant(rat, w, 0, 3, args.warmup, world, rank, dev, t0=w.T * 3 // 4)
         nxt["topk_decode"] = bench_topk(rat, wd.decode_batch, wd.H, wd.d, 16384, 64, 16, rat.RAT_TOPK_QUEST,
                                         args.decode_steps, args.warmup, world, rank, dev)
 
@@ -766,13 +771,15 @@ def main():
     if nxt:
         line["attention_variants"] = {}
         for name, r in att_var.items():
+            t_from = w.T * 3 // 4 if name == "chunked" else 0
             fl = sum(w.B * 4.0 * w.d * variant_pairs(w.T, w.dil[h], w.win[h], grid=name == "grid",
-                                                     dedupe=name == "dedupe") for h in range(w.H))
+                                                     dedupe=name == "dedupe", t_from=t_from) for h in range(w.H))
             tf = fl / (r["ms"] * 1e-3) / 1e12
             line["attention_variants"][name] = {
                 "what": {"grid": "fixed-grid dilation (j mod D == D-1, plus t)",
-                         "dedupe": "window part without the dilated set's keys"}[name],
-                "ms_per_launch": r["ms"], "value": w.B * w.T * world / (r["ms"] * 1e-3), "unit": "tok/s",
+                         "dedupe": "window part without the dilated set's keys",
+                         "chunked": "last quarter of the prefill as a chunk (t0 = 3T/4) over the whole history"}[name],
+                "ms_per_launch": r["ms"], "value": w.B * (w.T - t_from) * world / (r["ms"] * 1e-3), "unit": "tok/s",
                 "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                              "frac": tf / peaks["bf16_tflops"], "traffic": None},
                 "gpu_launches": r["launches"]}

@@ -89,5 +89,9 @@ def test_variant_pairs_count_the_reading_key_sets(grid, dedupe, T, D, W):
         win = {j for j in range(t + 1) if W > 0 and j >= t - W + 1}
         n += len(dil) + len(win - dil if dedupe else win)
     assert bench.variant_pairs(T, D, W, grid=grid, dedupe=dedupe) == n
+    # a chunk's rows alone: the whole minus the rows before it
+    t_from = T // 3
+    n_before = bench.variant_pairs(t_from, D, W, grid=grid, dedupe=dedupe) if t_from else 0.0
+    assert bench.variant_pairs(T, D, W, grid=grid, dedupe=dedupe, t_from=t_from) == n - n_before
     if not grid and not dedupe:
         assert bench.attn_pairs(T, D, W) == n
