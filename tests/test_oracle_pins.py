@@ -240,6 +240,20 @@ def test_merge_is_one_softmax_over_both_sets(T, D, W):
         assert abs(lse[0, 0, t] - torch.logsumexp(z, 0).item()) < 1e-12
 
 
+def test_huge_scores_select_the_best_key():
+    # scale -> infinity: each row's softmax collapses onto its largest-score key
+    # (no overflow: the max is taken out before exponentiating)
+    B, T, H, d = 1, 40, 1, 8
+    q, k, v = rand_qkv(B, T, H, d)
+    o, lse = oracle.attention(q, k, v, [3], [5], scale=1e6)
+    for t in range(T):
+        keys = sorted({j for j in range(t + 1) if (t - j) % 3 == 0} | set(range(max(0, t - 4), t + 1)))
+        z = k[0, keys, 0] @ q[0, t, 0]
+        best = keys[int(np.argmax(z))]
+        np.testing.assert_allclose(o[0, t, 0], v[0, best, 0], rtol=0, atol=1e-9)
+        assert np.isfinite(lse[0, 0, t])
+
+
 def test_first_row_and_convex_hull():
     B, T, H, d = 2, 30, 2, 6
     q, k, v = rand_qkv(B, T, H, d)
