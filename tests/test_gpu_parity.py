@@ -886,6 +886,26 @@ def test_chunked_prefill_equals_one_shot(grid, dtype, chunks):
                 np.testing.assert_allclose(cvh[:, h, r], rv[:, j, h], rtol=2e-2, atol=2e-2)
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_attention_with_large_scores(dtype):
+    # q scaled by 8: scores of tens in the log2 domain, so the running max
+    # grows by more than the lazy-rescale threshold between tiles and P must
+    # stay bounded; the outputs still match the oracle
+    B, T, H, d = 1, 4096, 2, 128
+    q, kt, vt, _ = inputs(B, T, H, d, dtype, seed=91)
+    q = (q.float() * 8).to(dtype)
+    dil, win = [16, 1], [256, 0]
+    cfg = make_cfg(B, T, H, d, dtype, dil, win)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, T, device=DEV)
+    ws = rat.workspace(cfg, rat.RAT_OP_ATTN)
+    rat.rat_dilated_attn_prefill(cfg, q, kt, vt, o, lse, ws)
+    rat.rat_check_status(ws)
+    ro, rl = oracle.attention(f64(q), f64(kt), f64(vt), dil, win)
+    assert_close(o, ro, dtype, "o")
+    assert_close(lse, rl, dtype if dtype == torch.bfloat16 else torch.float32, "lse")
+
+
 def test_decode_bad_position_is_reported():
     B, H, d = 2, 2, 64
     cfg = make_cfg(B, 1, H, d, torch.bfloat16, [2, 2], [0, 0])
