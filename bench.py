@@ -249,6 +249,27 @@ def attn_pairs(T, D, W):
     return pairs
 
 
+def variant_pairs(T, D, W, grid=False, dedupe=False, t_from=0):
+    """Unmasked (query, key) pairs of one head's rows t_from .. T-1 under the
+    fixed-grid reading (keys j <= t with j mod D == D-1, plus t once) and/or
+    dedupe (the window part skips the dilated set's keys), in closed form per row."""
+    t = np.arange(t_from, T, dtype=np.int64)
+    lo = np.maximum(0, t - W + 1)
+    if grid:
+        on = (t % D) == D - 1
+        n_dil = (t + 1) // D + np.where(on, 0, 1)
+    else:
+        n_dil = t // D + 1
+    n_win = np.minimum(W, t + 1) if W > 0 else np.zeros_like(t)
+    if dedupe and W > 0:
+        if grid:    # grid positions in [lo, t], plus t itself when it is off the grid
+            shared = (t + 1) // D - lo // D + np.where(on, 0, 1)
+        else:       # t, t-D, ... down to lo
+            shared = (t - lo) // D + 1
+        n_win = n_win - shared
+    return float(np.sum(n_dil + n_win))
+
+
 def prefill_work(w):
     """(attention FLOPs, scan bytes) of one prefill step: 4*d FLOPs per pair;
     10 bytes per (token, channel) of a recurrent head (k, v, g read; kt, vt written)."""
@@ -393,19 +414,21 @@ def bench_prefill(rat, w, steps, warmup, world, rank, dev, e2e_steps):
 # ---------------------------------------------------------------- decode
 
 
-def bench_decode(rat, w, ctx, steps, warmup, world, rank, dev, fill_chunk=8):
+def bench_decode(rat, w, ctx, steps, warmup, world, rank, dev, fill_chunk=8, flags=0, page_rows=0):
     """Fill the cache of `ctx` tokens with batch-chunked rat_scan_prefill, then
-    time `steps` decode steps (positions ctx+warmup .. )."""
+    time `steps` decode steps (positions ctx+warmup .. ).  flags: RAT_FLAG_*;
+    page_rows > 0: the decode reads a paged copy of the cache (pages in
+    reverse order, so no two consecutive pages of a sequence are adjacent)."""
     dtype = w.torch_dtype
     B = w.decode_batch
     cap = ctx + warmup + steps
-    cfg = rat.Config(B, ctx, w.H, w.d, dtype, w.dil, w.win, w.recur)
+    cfg = rat.Config(B, ctx, w.H, w.d, dtype, w.dil, w.win, w.recur, flags=flags)
     R = rat.rat_cache_rows(cfg, cap)
     ck = torch.empty(B, w.H, R, w.d, dtype=dtype, device=dev)
     cv = torch.empty_like(ck)
     sk = torch.empty(B, w.H, w.d, dtype=torch.float32, device=dev)
     sv = torch.empty_like(sk)
-    ccfg = rat.Config(fill_chunk, ctx, w.H, w.d, dtype, w.dil, w.win, w.recur)
+    ccfg = rat.Config(fill_chunk, ctx, w.H, w.d, dtype, w.dil, w.win, w.recur, flags=flags)
     wsc = rat.workspace(ccfg, rat.RAT_OP_SCAN, device=dev)
     per_b = w.H * R * w.d
     for b0 in range(0, B, fill_chunk):
@@ -417,6 +440,21 @@ def bench_decode(rat, w, ctx, steps, warmup, world, rank, dev, fill_chunk=8):
         del k, v, g
     rat.rat_check_status(wsc)
     del wsc
+    cache = None
+    if page_rows > 0:
+        # the same logical rows moved into shuffled pages
+        pps = -(-R // page_rows)
+        table = torch.arange(B * pps - 1, -1, -1, dtype=torch.int32, device=dev).view(B, pps)
+        pool_k = torch.zeros(B * pps, w.H, page_rows, w.d, dtype=dtype, device=dev)
+        pool_v = torch.zeros_like(pool_k)
+        r = torch.arange(R, device=dev)
+        for b in range(B):
+            pg = table[b, r // page_rows].long()
+            pool_k[pg, :, r % page_rows] = ck[b].transpose(0, 1)
+            pool_v[pg, :, r % page_rows] = cv[b].transpose(0, 1)
+        del ck, cv
+        ck = cv = None
+        cache = rat.paged_cache(cfg, pool_k, pool_v, table, cap)
     n = warmup + steps
     toks = [wl.token_inputs(B, w.H, w.d, w.gate_mean, dtype, device=dev, seed=5000 + i) for i in range(n)]
     poss = [torch.full((B,), ctx + i, dtype=torch.int32, device=dev) for i in range(n)]
@@ -426,7 +464,10 @@ def bench_decode(rat, w, ctx, steps, warmup, world, rank, dev, fill_chunk=8):
 
     def step(i):
         tq, tk, tv, tg = toks[i]
-        rat.rat_decode_step(cfg, tq, tk, tv, tg, sk, sv, ck, cv, cap, poss[i], o, None, ws=wsd, stream=stream)
+        if cache is not None:
+            rat.rat_decode_step_paged(cfg, tq, tk, tv, tg, sk, sv, cache, cap, poss[i], o, None, ws=wsd, stream=stream)
+        else:
+            rat.rat_decode_step(cfg, tq, tk, tv, tg, sk, sv, ck, cv, cap, poss[i], o, None, ws=wsd, stream=stream)
 
     for i in range(warmup):
         step(i)
@@ -445,7 +486,111 @@ def bench_decode(rat, w, ctx, steps, warmup, world, rank, dev, fill_chunk=8):
     ms = max_over_ranks(a.elapsed_time(b), world, dev) / steps
     t_mid = ctx + warmup + steps // 2
     byts = decode_bytes(B, w.H, w.d, t_mid, w.dil, w.win)
-    del ck, cv, toks
+    del ck, cv, toks, cache
+    torch.cuda.empty_cache()
+    return dict(ms=ms, bytes=byts, launches=launches, ctx=ctx)
+
+
+def bench_attn_variant(rat, w, flags, steps, warmup, world, rank, dev, t0=0):
+    """The attention step alone (rat_dilated_attn_prefill) on the prefill
+    workload under RAT_FLAG_* `flags`; with t0 > 0, only the queries of
+    positions t0 .. T-1 (the last chunk of a chunked prefill) over the whole
+    history.  Returns ms per launch."""
+    dtype = w.torch_dtype
+    q, k, v, _ = wl.prefill_inputs(w.B, w.T, w.H, w.d, w.gate_mean, dtype, device=dev, seed=11 + rank)
+    if t0 > 0:
+        q = q[:, t0:].contiguous()
+    cfg = rat.Config(w.B, w.T - t0, w.H, w.d, dtype, w.dil, w.win, w.recur, flags=flags, t0=t0)
+    o = torch.empty_like(q)
+    ws = rat.workspace(cfg, rat.RAT_OP_ATTN, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        rat.rat_dilated_attn_prefill(cfg, q, k, v, o, None, ws, stream=stream)
+    rat.rat_check_status(ws)
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = rat.rat_launch_count()
+    a.record(stream)
+    for _ in range(steps):
+        rat.rat_dilated_attn_prefill(cfg, q, k, v, o, None, ws, stream=stream)
+    b.record(stream)
+    torch.cuda.synchronize()
+    launches = rat.rat_launch_count() - n0
+    rat.rat_check_status(ws)
+    ms = max_over_ranks(a.elapsed_time(b), world, dev) / steps
+    del q, k, v, o, ws
+    torch.cuda.empty_cache()
+    return dict(ms=ms, launches=launches)
+
+
+def topk_decode_bytes(B, H, d, t, block, K, elt=2):
+    """Algorithmic HBM bytes of one top-k decode step at position t: the fp32
+    statistics of the candidate blocks, the old rows (before t) of the first,
+    local and selected blocks (K~ and V~), the token's q,k,v,g, o, the state,
+    and the new row plus its block's statistics (the new row itself is
+    attended from registers, as in decode_bytes)."""
+    c = t // block
+    ncand = max(0, c - 1)
+    rows = t if c == 0 else block + min(K, ncand) * block + (t - c * block)
+    stats = ncand * 2 * d * 4
+    return B * H * (stats + rows * 2 * d * elt + d * (5 * elt + 16 + 2 * elt) + 2 * 2 * d * 4)
+
+
+def bench_topk(rat, B, H, d, ctx, block, K, mode, steps, warmup, world, rank, dev, fill_chunk=8, gate_mean=2.0):
+    """Top-k block decode over a dense cache of `ctx` tokens: batch-chunked
+    prefill into the cache, block statistics, then `steps` timed steps."""
+    dtype = torch.bfloat16
+    cap = ctx + warmup + steps
+    dil, win = [1] * H, [0] * H
+    cfg = rat.Config(B, ctx, H, d, dtype, dil, win)
+    R = rat.rat_cache_rows(cfg, cap)
+    ck = torch.empty(B, H, R, d, dtype=dtype, device=dev)
+    cv = torch.empty_like(ck)
+    sk = torch.empty(B, H, d, device=dev)
+    sv = torch.empty_like(sk)
+    ccfg = rat.Config(fill_chunk, ctx, H, d, dtype, dil, win)
+    wsc = rat.workspace(ccfg, rat.RAT_OP_SCAN, device=dev)
+    per_b = H * R * d
+    for b0 in range(0, B, fill_chunk):
+        k, v, g = wl.prefill_inputs(fill_chunk, ctx, H, d, gate_mean, dtype, device=dev, seed=3000 + rank * 997 + b0)[1:]
+        rat.rat_scan_prefill(ccfg, k, v, g, None, None, None, None, sk[b0:b0 + fill_chunk], sv[b0:b0 + fill_chunk],
+                             ck.view(-1)[b0 * per_b:(b0 + fill_chunk) * per_b],
+                             cv.view(-1)[b0 * per_b:(b0 + fill_chunk) * per_b], cap, ws=wsc)
+        del k, v, g
+    rat.rat_check_status(wsc)
+    del wsc
+    stats = torch.empty(rat.topk_stats_shape(cfg, block, cap), device=dev)
+    rat.rat_topk_build_stats(cfg, block, mode, ck, cap, stats)
+    n = warmup + steps
+    toks = [wl.token_inputs(B, H, d, gate_mean, dtype, device=dev, seed=7000 + i) for i in range(n)]
+    poss = [torch.full((B,), ctx + i, dtype=torch.int32, device=dev) for i in range(n)]
+    o = torch.empty(B, H, d, dtype=dtype, device=dev)
+    wsd = rat.workspace(cfg, rat.RAT_OP_TOPK_DECODE, cap, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        tq, tk, tv, tg = toks[i]
+        rat.rat_topk_decode_step(cfg, block, K, mode, tq, tk, tv, tg, sk, sv, ck, cv, cap, stats, poss[i], o, None,
+                                 None, ws=wsd, stream=stream)
+
+    for i in range(warmup):
+        step(i)
+    rat.rat_check_status(wsd)
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = rat.rat_launch_count()
+    a.record(stream)
+    for i in range(warmup, n):
+        step(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    launches = rat.rat_launch_count() - n0
+    rat.rat_check_status(wsd)
+    ms = max_over_ranks(a.elapsed_time(b), world, dev) / steps
+    byts = topk_decode_bytes(B, H, d, ctx + warmup + steps // 2, block, K)
+    del ck, cv, stats, toks
     torch.cuda.empty_cache()
     return dict(ms=ms, bytes=byts, launches=launches, ctx=ctx)
 
@@ -524,6 +669,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=2048, help="oracle rows timed for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=512, help="oracle rows per reference-arm step")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the decode variants (fixed grid, paged cache, top-k blocks)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -553,6 +700,19 @@ def main():
     dec = []
     for ctx in [int(c) for c in args.decode_ctx.split(",") if c]:
         dec.append(bench_decode(rat, wl.DECODE_D16, ctx, args.decode_steps, args.warmup, world, rank, dev))
+
+    nxt = {}
+    if not args.no_next_rows:
+        wd = wl.DECODE_D16
+        nxt["grid_decode"] = bench_decode(rat, wd, 4096, args.decode_steps, args.warmup, world, rank, dev,
+                                          flags=rat.RAT_FLAG_GRID_DILATION)
+        nxt["paged_decode"] = bench_decode(rat, wd, 4096, args.decode_steps, args.warmup, world, rank, dev,
+                                           page_rows=256)
+        att_var = {name: bench_attn_variant(rat, w, f, 3, args.warmup, world, rank, dev)
+                   for name, f in (("grid", rat.RAT_FLAG_GRID_DILATION), ("dedupe", rat.RAT_FLAG_DEDUPE))}
+        att_var["chunked"] = bench_attn_variant(rat, w, 0, 3, args.warmup, world, rank, dev, t0=w.T * 3 // 4)
+        nxt["topk_decode"] = bench_topk(rat, wd.decode_batch, wd.H, wd.d, 16384, 64, 16, rat.RAT_TOPK_QUEST,
+                                        args.decode_steps, args.warmup, world, rank, dev)
 
     if rank != 0:
         return
@@ -608,6 +768,32 @@ def main():
                                      "traffic": profile_traffic("decode_batch256", "decode_ctx%d" % r["ctx"])},
                         "gpu_launches": r["launches"]} for r in dec],
         }
+    if nxt:
+        line["attention_variants"] = {}
+        for name, r in att_var.items():
+            t_from = w.T * 3 // 4 if name == "chunked" else 0
+            fl = sum(w.B * 4.0 * w.d * variant_pairs(w.T, w.dil[h], w.win[h], grid=name == "grid",
+                                                     dedupe=name == "dedupe", t_from=t_from) for h in range(w.H))
+            tf = fl / (r["ms"] * 1e-3) / 1e12
+            line["attention_variants"][name] = {
+                "what": {"grid": "fixed-grid dilation (j mod D == D-1, plus t)",
+                         "dedupe": "window part without the dilated set's keys",
+                         "chunked": "last quarter of the prefill as a chunk (t0 = 3T/4) over the whole history"}[name],
+                "ms_per_launch": r["ms"], "value": w.B * (w.T - t_from) * world / (r["ms"] * 1e-3), "unit": "tok/s",
+                "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": tf / peaks["bf16_tflops"], "traffic": None},
+                "gpu_launches": r["launches"]}
+        wd = wl.DECODE_D16
+        desc = {"grid_decode": "fixed-grid dilation, grid cache + window ring, ctx 4096",
+                "paged_decode": "residue cache in 256-row pages (shuffled), ctx 4096",
+                "topk_decode": "top-k blocks (Quest, block 64, K 16) over a dense cache, ctx 16384"}
+        line["decode_variants"] = {
+            name: {"what": desc[name], "value": wd.decode_batch * world / (r["ms"] * 1e-3), "unit": "tok/s",
+                   "ms_per_step": r["ms"],
+                   "roofline": {"bound": "hbm", "achieved": r["bytes"] / (r["ms"] * 1e-3) / 1e9,
+                                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                "frac": r["bytes"] / (r["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"], "traffic": None},
+                   "gpu_launches": r["launches"]} for name, r in nxt.items()}
     if not args.no_cpu and world == 1:
         v, secs = oracle_sample(w, args.cpu_rows)
         line["cpu_baseline"] = {"value": v, "unit": "tok/s", "cores": host_cores(), "kind": "oracle",

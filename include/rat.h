@@ -20,13 +20,18 @@
  * Definitions used by every entry point (the pages give the method at the
  * level of captions; these are the plain readings of them):
  *   recurrence   s_t = a_t * s_{t-1} + (1 - a_t) * x_t per channel, for x = k
- *                and x = v, with a_t = sigmoid(g_t) from one gate tensor g;
+ *                and x = v, with a_t = sigmoid(g_t) from one gate tensor g
+ *                (one per tensor with RAT_FLAG_SEPARATE_GATES);
  *                s_{-1} = init (zero when not given).  A head with recur = 0
  *                has a = 0: its augmented keys/values are the raw ones.
- *   dilation     query t attends to { j <= t : (t - j) mod D == 0 }.
+ *   dilation     query t attends to { j <= t : (t - j) mod D == 0 }.  With
+ *                RAT_FLAG_GRID_DILATION it attends instead to the fixed grid
+ *                { j <= t : j mod D == D - 1 } plus itself (j = t, once): the
+ *                chunk-end keys of the RAT page's Approach (chunk size D),
+ *                which a decode can keep in a cache D times smaller.
  *   window       W > 0 adds a second softmax over { max(0, t-W+1) <= j <= t }.
  *   merge        the two softmaxes are merged by log-sum-exp (a key in both
- *                sets counts in both).
+ *                sets counts in both; with RAT_FLAG_DEDUPE, once).
  *   scale        scores are scale * <q_t, k~_j>, scale = 1/sqrt(d) by default.
  *
  * Conventions shared by all calls
@@ -90,7 +95,8 @@ typedef enum {
     RAT_OP_ATTN = 1,          /* rat_dilated_attn_prefill */
     RAT_OP_MIX = 2,           /* rat_mix_prefill with kt = vt = NULL (K~/V~ kept in ws) */
     RAT_OP_MIX_CALLER_KV = 3, /* rat_mix_prefill with caller-provided kt and vt */
-    RAT_OP_DECODE = 4         /* rat_decode_step */
+    RAT_OP_DECODE = 4,        /* rat_decode_step */
+    RAT_OP_TOPK_DECODE = 5    /* rat_topk_decode_step */
 } rat_op;
 
 /*
@@ -99,7 +105,17 @@ typedef enum {
  * window) and recurrence flag recur[h] (0 = no recurrence; NULL = all heads
  * recurrent) -- the hybrid head compositions of the RAT+ Abstract.
  * Limits of this library version: d in {64, 128}; 1 <= H <= 256; B, T >= 0;
- * B*T*H*d < 2^40 elements.  An empty batch or sequence (B*T == 0) launches
+ * B*T*H*d < 2^40 elements.
+ *
+ * Chunked prefill (t0 > 0): a call covers positions t0 .. t0+T-1 of its
+ * sequences.  Token inputs (q, k, v, g) and outputs (o, lse) hold those T
+ * positions; the augmented keys/values kt, vt are history buffers
+ * [B, t_cap, H, d] (t_cap = 0 means t0 + T) whose rows 0 .. t0+T-1 hold
+ * positions 0 .. t0+T-1, so one buffer serves every chunk: the scan writes rows t0 ..
+ * t0+T-1 (init_k/init_v carry the state after position t0-1) and the
+ * attention reads all rows, so the chunks of a prefill give the one-shot
+ * result.  Decode-cache rows go to positions t0 + t.  rat_mix_prefill then
+ * needs caller kt/vt.  Decode steps ignore t0.  An empty batch or sequence (B*T == 0) launches
  * no kernel; a prefill then only copies init (or zero) to final.
  */
 typedef struct {
@@ -109,7 +125,21 @@ typedef struct {
     const int32_t *win;      /* host [H] */
     const uint8_t *recur;    /* host [H] or NULL */
     float scale;             /* <= 0 selects 1/sqrt(d) */
+    uint32_t flags;          /* RAT_FLAG_* bits, 0 = the defaults above */
+    int t0;                  /* position of this call's first token (chunked prefill), 0 = a whole prefill */
+    int t_cap;               /* rows per batch entry of the kt/vt history, >= t0 + T; 0 = t0 + T */
 } rat_cfg;
+
+/* Fixed-grid reading of dilation (see "dilation" above) for every head of the
+ * call, and the matching decode-cache layout (see rat_cache_rows). */
+#define RAT_FLAG_GRID_DILATION 1u
+/* A key in both the dilated set and the window counts once: the window part
+ * skips the keys the dilated set holds (with D = 1 the window adds nothing). */
+#define RAT_FLAG_DEDUPE 2u
+/* Separate gates for keys and values: the gate tensor g holds two tensors of
+ * the usual shape, g[0] for the key recurrence and g[1] for the value
+ * recurrence ([2, B, T, H, d] in a prefill, [2, B, H, d] in a decode step). */
+#define RAT_FLAG_SEPARATE_GATES 4u
 
 /* Bytes of workspace `op` needs for `cfg` (cache_cap: decode capacity, else
  * ignored).  Returns 0 when cfg is invalid. */
@@ -125,6 +155,11 @@ RAT_API rat_status rat_workspace_init(void *ws, size_t ws_bytes, rat_stream_t st
  *     (j mod D_h) * ceil(cap / D_h) + floor(j / D_h)
  * i.e. residue-major: the rows a decode query at position t reads for its
  * dilated part (all j == t mod D_h, j <= t) form one contiguous slab.
+ * With RAT_FLAG_GRID_DILATION a head keeps only its grid: position j with
+ * j mod D_h == D_h - 1 at row floor(j / D_h), rows [0, ceil(cap / D_h)).  A
+ * head with D_h > 1 and a window W_h > 0 also keeps a ring of its last W_h
+ * positions after the grid: position j at row ceil(cap / D_h) + (j mod W_h).
+ * R is the largest head's row count in either layout.
  * Returns 0 when cfg or cap is invalid.
  */
 RAT_API int64_t rat_cache_rows(const rat_cfg *cfg, int cap);
@@ -138,7 +173,9 @@ RAT_API int64_t rat_cache_rows(const rat_cfg *cfg, int cap);
  *                        is given (recur = 0 heads receive a copy of k / v)
  *   final_k, final_v out [B,H,d] fp32 s_{T-1}, or NULL
  *   cache_k, cache_v out decode cache tensors (layout above) for positions
- *                        0..T-1, or NULL; requires T <= cache_cap
+ *                        0..T-1 (under the fixed grid: the grid rows, and
+ *                        the ring rows of positions T-W_h .. T-1), or NULL;
+ *                        requires T <= cache_cap
  * At least one of (kt, vt) or (cache_k, cache_v) must be given, as pairs.
  */
 RAT_API rat_status rat_scan_prefill(const rat_cfg *cfg, const void *k, const void *v, const void *g,
@@ -178,12 +215,15 @@ RAT_API rat_status rat_mix_prefill(const rat_cfg *cfg, const void *q, const void
  *   1. s <- a*s + (1-a)*x for x = k and v (a = sigmoid(g), a = 0 if recur = 0),
  *      updating state_k / state_v in place (fp32 [B,H,d]);
  *   2. the new augmented key/value (rounded to cfg->dtype) is stored at t's
- *      cache row;
+ *      cache row (under the fixed grid: at its grid row when t is on the
+ *      grid, and at its ring row when the head keeps a ring);
  *   3. o[b,h] = merged attention of q over the cache rows j <= t of the
  *      dilated set (and window) of t.
  *   q, k, v, g   in  [B,H,d]
  *   cache_k/v    in/out [B,H,R,d], R = rat_cache_rows(cfg, cache_cap); rows of
  *                positions < pos[b] must hold earlier augmented keys/values
+ *                (under the fixed grid: the grid rows below t and the ring
+ *                rows of t-W_h+1 .. t-1)
  *   pos          in  DEVICE int32 [B], 0 <= pos[b] < cache_cap (a position out
  *                of range makes the kernel skip that entry and record
  *                RAT_ERR_INVALID for rat_check_status)
@@ -197,6 +237,38 @@ RAT_API rat_status rat_decode_step(const rat_cfg *cfg, const void *q, const void
                            const void *g, float *state_k, float *state_v, void *cache_k,
                            void *cache_v, int cache_cap, const int32_t *pos, void *o, float *lse,
                            void *ws, size_t ws_bytes, rat_stream_t stream);
+
+/*
+ * Paged decode cache, for serving engines that hand out KV memory in pages.
+ * The logical rows of a (b, h) block -- the layout of rat_cache_rows, in
+ * either dilation reading -- live in pages of page_rows rows: logical row r of
+ * batch entry b, head h is row (r mod page_rows) of page
+ * page_table[b * pages_per_seq + r / page_rows] of the pools, which are
+ * [num_pages, H, page_rows, d] in cfg->dtype.  pages_per_seq * page_rows must
+ * cover rat_cache_rows(cfg, cache_cap).  Only the pages of the rows a call
+ * touches need valid entries; a touched entry outside [0, num_pages) is never
+ * dereferenced: the prefill leaves that row unwritten and the decode step
+ * skips each (b, h) whose step touches it (o = 0, state unchanged), and either
+ * records RAT_ERR_INVALID for rat_check_status.  The caller owns pools and
+ * table (device memory).
+ */
+typedef struct {
+    void *pool_k, *pool_v;        /* [num_pages, H, page_rows, d] */
+    const int32_t *page_table;    /* device int32 [B, pages_per_seq] */
+    int page_rows, pages_per_seq, num_pages;
+} rat_paged_cache;
+
+/* rat_scan_prefill writing a paged cache (cache_cap as there). */
+RAT_API rat_status rat_scan_prefill_paged(const rat_cfg *cfg, const void *k, const void *v, const void *g,
+                                          const float *init_k, const float *init_v, void *kt, void *vt,
+                                          float *final_k, float *final_v, const rat_paged_cache *cache,
+                                          int cache_cap, void *ws, size_t ws_bytes, rat_stream_t stream);
+
+/* rat_decode_step over a paged cache; the ring's copies split at page ends. */
+RAT_API rat_status rat_decode_step_paged(const rat_cfg *cfg, const void *q, const void *k, const void *v,
+                                         const void *g, float *state_k, float *state_v,
+                                         const rat_paged_cache *cache, int cache_cap, const int32_t *pos,
+                                         void *o, float *lse, void *ws, size_t ws_bytes, rat_stream_t stream);
 
 /*
  * rat_decode_step without a workspace, for callers that cannot allocate
@@ -226,6 +298,54 @@ RAT_API rat_status rat_decode_step_noalloc(const rat_cfg *cfg, const void *q, co
                                            const void *g, float *state_k, float *state_v, void *cache_k,
                                            void *cache_v, int cache_cap, const int32_t *pos, void *o,
                                            float *lse, rat_stream_t stream);
+
+/*
+ * Top-k block attention for decoding over the augmented keys/values (RAT+
+ * Figure 3 and Tables 17-18; Exponentially Decaying Memory, section 2.2,
+ * sparse inference settings).  Keys are grouped in blocks of `block`
+ * consecutive positions.  The query at t (block c = t / block) attends, in one
+ * softmax, to the rows j <= t of block 0, of block c, and of the `topk` best
+ * of blocks 1 .. c-1 (all of them when there are fewer), ranked by
+ *   RAT_TOPK_QUEST  sum_ch max(q_ch * kmin_ch, q_ch * kmax_ch) over the block's
+ *                   per-channel key range (an upper bound of q.k in the block)
+ *   RAT_TOPK_MOBA   q . mean of the block's keys
+ * with equal scores going to the lower block.  The cache is the dense layout:
+ * every head must have dil = 1 and win = 0 (the sparse selection replaces
+ * dilation and window), so position j of a head is row j.
+ *
+ * Block statistics: `stats` is caller memory of rat_topk_stats_size() bytes,
+ * fp32 [B, H, ceil(cache_cap / block), 2, d]: per block the channel minima and
+ * maxima (Quest), or the channel sums and zeros (MoBA), of the cached keys.
+ * Limits: 1 <= block; 0 <= topk <= 64; ceil(cache_cap / block) <= 16384.
+ */
+typedef enum { RAT_TOPK_QUEST = 0, RAT_TOPK_MOBA = 1 } rat_topk_mode;
+
+/* Bytes of the block-statistics buffer (0 when an argument is invalid). */
+RAT_API size_t rat_topk_stats_size(const rat_cfg *cfg, int block, int cache_cap);
+
+/*
+ * Statistics of the blocks of positions 0 .. cfg->T - 1 (the tokens a prefill
+ * wrote into cache_k with rat_scan_prefill), in `mode`; a last partial block
+ * covers the positions it has.  Blocks at or past cfg->T are left as they are.
+ */
+RAT_API rat_status rat_topk_build_stats(const rat_cfg *cfg, int block, int mode, const void *cache_k,
+                                        int cache_cap, float *stats, rat_stream_t stream);
+
+/*
+ * One decode step with top-k block attention.  As rat_decode_step (the state
+ * update, the append of the new row at row t = pos[b], ragged positions, the
+ * error behaviour), plus: the new key is folded into its block's statistics,
+ * which must hold blocks 0 .. c of the positions before t; `sel` (nullable,
+ * device int32 [B, H, topk]) receives the selected blocks in selection order,
+ * -1 where fewer were available.  ws: rat_workspace_size(cfg,
+ * RAT_OP_TOPK_DECODE, cache_cap) bytes.  One kernel per step, no other CUDA
+ * call after the first on a device (graph-capturable).
+ */
+RAT_API rat_status rat_topk_decode_step(const rat_cfg *cfg, int block, int topk, int mode, const void *q,
+                                        const void *k, const void *v, const void *g, float *state_k,
+                                        float *state_v, void *cache_k, void *cache_v, int cache_cap,
+                                        float *stats, const int32_t *pos, void *o, float *lse, int32_t *sel,
+                                        void *ws, size_t ws_bytes, rat_stream_t stream);
 
 /*
  * Synchronises `stream`, returns the first device-side error recorded in `ws`

@@ -20,12 +20,17 @@ LIB_PATH = os.path.join(HERE, "librat.so")
 
 RAT_OK, RAT_ERR_INVALID, RAT_ERR_UNSUPPORTED, RAT_ERR_CUDA, RAT_ERR_TIMEOUT, RAT_ERR_WORKSPACE = range(6)
 RAT_F32, RAT_BF16 = 0, 1
-RAT_OP_SCAN, RAT_OP_ATTN, RAT_OP_MIX, RAT_OP_MIX_CALLER_KV, RAT_OP_DECODE = range(5)
+RAT_OP_SCAN, RAT_OP_ATTN, RAT_OP_MIX, RAT_OP_MIX_CALLER_KV, RAT_OP_DECODE, RAT_OP_TOPK_DECODE = range(6)
+RAT_TOPK_QUEST, RAT_TOPK_MOBA = 0, 1
+RAT_FLAG_GRID_DILATION = 1
+RAT_FLAG_DEDUPE = 2
+RAT_FLAG_SEPARATE_GATES = 4
 
 EXPORTS = ["rat_workspace_size", "rat_workspace_init", "rat_cache_rows", "rat_scan_prefill",
            "rat_dilated_attn_prefill", "rat_mix_prefill", "rat_decode_step", "rat_check_status",
            "rat_status_string", "rat_last_error", "rat_version", "rat_launch_count", "rat_debug_set_scan_stall",
-           "rat_decode_step_noalloc"]
+           "rat_decode_step_noalloc", "rat_topk_stats_size", "rat_topk_build_stats", "rat_topk_decode_step",
+           "rat_scan_prefill_paged", "rat_decode_step_paged"]
 
 
 class RatError(RuntimeError):
@@ -42,7 +47,12 @@ class rat_cfg(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("dil", ctypes.POINTER(ctypes.c_int32)),
                 ("win", ctypes.POINTER(ctypes.c_int32)), ("recur", ctypes.POINTER(ctypes.c_uint8)),
-                ("scale", ctypes.c_float)]
+                ("scale", ctypes.c_float), ("flags", ctypes.c_uint32), ("t0", ctypes.c_int), ("t_cap", ctypes.c_int)]
+
+
+class rat_paged_cache(ctypes.Structure):
+    _fields_ = [("pool_k", ctypes.c_void_p), ("pool_v", ctypes.c_void_p), ("page_table", ctypes.c_void_p),
+                ("page_rows", ctypes.c_int), ("pages_per_seq", ctypes.c_int), ("num_pages", ctypes.c_int)]
 
 
 _lib = None
@@ -68,6 +78,13 @@ def load_library(path=LIB_PATH):
     lib.rat_mix_prefill.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P]
     lib.rat_decode_step.argtypes = [cfgp, P, P, P, P, P, P, P, P, I, P, P, P, P, S, P]
     lib.rat_decode_step_noalloc.argtypes = [cfgp, P, P, P, P, P, P, P, P, I, P, P, P, P]
+    lib.rat_topk_stats_size.argtypes = [cfgp, I, I]
+    lib.rat_topk_stats_size.restype = S
+    lib.rat_topk_build_stats.argtypes = [cfgp, I, I, P, I, P, P]
+    lib.rat_topk_decode_step.argtypes = [cfgp, I, I, I, P, P, P, P, P, P, P, P, I, P, P, P, P, P, P, S, P]
+    pcp = ctypes.POINTER(rat_paged_cache)
+    lib.rat_scan_prefill_paged.argtypes = [cfgp, P, P, P, P, P, P, P, P, P, pcp, I, P, S, P]
+    lib.rat_decode_step_paged.argtypes = [cfgp, P, P, P, P, P, P, pcp, I, P, P, P, P, S, P]
     lib.rat_check_status.argtypes = [P, P]
     lib.rat_status_string.argtypes = [I]
     lib.rat_status_string.restype = ctypes.c_char_p
@@ -77,7 +94,9 @@ def load_library(path=LIB_PATH):
     lib.rat_launch_count.restype = ctypes.c_longlong
     lib.rat_debug_set_scan_stall.argtypes = [P, S, ctypes.c_int64, ctypes.c_int64, P]
     for name in ("rat_workspace_init", "rat_scan_prefill", "rat_dilated_attn_prefill", "rat_mix_prefill",
-                 "rat_decode_step", "rat_check_status", "rat_debug_set_scan_stall", "rat_decode_step_noalloc"):
+                 "rat_decode_step", "rat_check_status", "rat_debug_set_scan_stall", "rat_decode_step_noalloc",
+                 "rat_topk_build_stats", "rat_topk_decode_step", "rat_scan_prefill_paged",
+                 "rat_decode_step_paged"):
         getattr(lib, name).restype = I
     _lib = lib
     return lib
@@ -86,7 +105,7 @@ def load_library(path=LIB_PATH):
 class Config:
     """Owns a rat_cfg and the host arrays it points to."""
 
-    def __init__(self, B, T, H, d, dtype, dil, win, recur=None, scale=0.0):
+    def __init__(self, B, T, H, d, dtype, dil, win, recur=None, scale=0.0, flags=0, t0=0, t_cap=0):
         self.dil = np.ascontiguousarray(dil, dtype=np.int32)
         self.win = np.ascontiguousarray(win, dtype=np.int32)
         self.recur = None if recur is None else np.ascontiguousarray(recur, dtype=np.uint8)
@@ -97,7 +116,7 @@ class Config:
                          self.dil.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
                          self.win.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
                          None if self.recur is None else self.recur.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)),
-                         float(scale))
+                         float(scale), int(flags), int(t0), int(t_cap))
 
     @property
     def torch_dtype(self):
@@ -105,12 +124,23 @@ class Config:
 
     def replace(self, **kw):
         args = dict(B=self.c.B, T=self.c.T, H=self.c.H, d=self.c.d, dtype=self.c.dtype, dil=self.dil,
-                    win=self.win, recur=self.recur, scale=self.c.scale)
+                    win=self.win, recur=self.recur, scale=self.c.scale, flags=self.c.flags, t0=self.c.t0,
+                    t_cap=self.c.t_cap)
         args.update(kw)
         return Config(**args)
 
     def ref(self):
         return ctypes.byref(self.c)
+
+    @property
+    def history_shape(self):
+        """Shape of kt / vt: [B, t_cap or t0 + T, H, d] (the history in a chunked prefill)."""
+        return (self.c.B, self.c.t_cap or self.c.t0 + self.c.T, self.c.H, self.c.d)
+
+    def gate_shape(self, tok):
+        """Shape of the gate tensor for token tensors of shape `tok` (a second,
+        leading axis of 2 with separate key and value gates)."""
+        return ((2,) + tuple(tok)) if self.c.flags & RAT_FLAG_SEPARATE_GATES else tuple(tok)
 
 
 def _ptr(t, name, dtype=None, shape=None, optional=False):
@@ -184,9 +214,9 @@ def rat_scan_prefill(cfg, k, v, g, init_k=None, init_v=None, kt=None, vt=None, f
     tok = (c.B, c.T, c.H, c.d)
     st = (c.B, c.H, c.d)
     dt = cfg.torch_dtype
-    args = [_ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, tok),
+    args = [_ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
             _ptr(init_k, "init_k", torch.float32, st, True), _ptr(init_v, "init_v", torch.float32, st, True),
-            _ptr(kt, "kt", dt, tok, True), _ptr(vt, "vt", dt, tok, True),
+            _ptr(kt, "kt", dt, cfg.history_shape, True), _ptr(vt, "vt", dt, cfg.history_shape, True),
             _ptr(final_k, "final_k", torch.float32, st, True), _ptr(final_v, "final_v", torch.float32, st, True),
             _ptr(cache_k, "cache_k", dt, None, True), _ptr(cache_v, "cache_v", dt, None, True), int(cache_cap),
             _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream)]
@@ -197,7 +227,8 @@ def rat_dilated_attn_prefill(cfg, q, kt, vt, o, lse=None, ws=None, stream=None):
     c = cfg.c
     tok = (c.B, c.T, c.H, c.d)
     dt = cfg.torch_dtype
-    args = [_ptr(q, "q", dt, tok), _ptr(kt, "kt", dt, tok), _ptr(vt, "vt", dt, tok), _ptr(o, "o", dt, tok),
+    args = [_ptr(q, "q", dt, tok), _ptr(kt, "kt", dt, cfg.history_shape), _ptr(vt, "vt", dt, cfg.history_shape),
+            _ptr(o, "o", dt, tok),
             _ptr(lse, "lse", torch.float32, (c.B, c.H, c.T), True), _ptr(ws, "ws", torch.uint8), ws.numel(),
             _stream(stream)]
     _check(load_library().rat_dilated_attn_prefill(cfg.ref(), *args), "rat_dilated_attn_prefill")
@@ -209,10 +240,10 @@ def rat_mix_prefill(cfg, q, k, v, g, init_k=None, init_v=None, o=None, lse=None,
     tok = (c.B, c.T, c.H, c.d)
     st = (c.B, c.H, c.d)
     dt = cfg.torch_dtype
-    args = [_ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, tok),
+    args = [_ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
             _ptr(init_k, "init_k", torch.float32, st, True), _ptr(init_v, "init_v", torch.float32, st, True),
             _ptr(o, "o", dt, tok), _ptr(lse, "lse", torch.float32, (c.B, c.H, c.T), True),
-            _ptr(kt, "kt", dt, tok, True), _ptr(vt, "vt", dt, tok, True),
+            _ptr(kt, "kt", dt, cfg.history_shape, True), _ptr(vt, "vt", dt, cfg.history_shape, True),
             _ptr(final_k, "final_k", torch.float32, st, True), _ptr(final_v, "final_v", torch.float32, st, True),
             _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream)]
     _check(load_library().rat_mix_prefill(cfg.ref(), *args), "rat_mix_prefill")
@@ -225,7 +256,7 @@ def rat_decode_step(cfg, q, k, v, g, state_k, state_v, cache_k, cache_v, cache_c
     dt = cfg.torch_dtype
     R = rat_cache_rows(cfg, cache_cap)
     cshape = (c.B, c.H, R, c.d)
-    args = [_ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, tok),
+    args = [_ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
             _ptr(state_k, "state_k", torch.float32, tok), _ptr(state_v, "state_v", torch.float32, tok),
             _ptr(cache_k, "cache_k", dt, cshape), _ptr(cache_v, "cache_v", dt, cshape), int(cache_cap),
             _ptr(pos, "pos", torch.int32, (c.B,)), _ptr(o, "o", dt, tok),
@@ -244,12 +275,97 @@ def rat_decode_step_noalloc(cfg, q, k, v, g, state_k, state_v, cache_k, cache_v,
     dt = cfg.torch_dtype
     R = rat_cache_rows(cfg, cache_cap)
     cshape = (c.B, c.H, R, c.d)
-    args = [_ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, tok),
+    args = [_ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
             _ptr(state_k, "state_k", torch.float32, tok), _ptr(state_v, "state_v", torch.float32, tok),
             _ptr(cache_k, "cache_k", dt, cshape), _ptr(cache_v, "cache_v", dt, cshape), int(cache_cap),
             _ptr(pos, "pos", torch.int32, (c.B,)), _ptr(o, "o", dt, tok),
             _ptr(lse, "lse", torch.float32, (c.B, c.H), True), _stream(stream)]
     _check(load_library().rat_decode_step_noalloc(cfg.ref(), *args), "rat_decode_step_noalloc")
+
+
+def rat_topk_stats_size(cfg, block, cache_cap):
+    n = load_library().rat_topk_stats_size(cfg.ref(), int(block), int(cache_cap))
+    if n == 0:
+        raise RatError(RAT_ERR_INVALID, "rat_topk_stats_size: " + load_library().rat_last_error().decode())
+    return n
+
+
+def topk_stats_shape(cfg, block, cache_cap):
+    """Shape of the fp32 block-statistics tensor: [B, H, ceil(cap / block), 2, d]."""
+    c = cfg.c
+    return (c.B, c.H, -(-int(cache_cap) // int(block)), 2, c.d)
+
+
+def rat_topk_build_stats(cfg, block, mode, cache_k, cache_cap, stats, stream=None):
+    c = cfg.c
+    R = rat_cache_rows(cfg, cache_cap)
+    args = [int(block), int(mode), _ptr(cache_k, "cache_k", cfg.torch_dtype, (c.B, c.H, R, c.d)), int(cache_cap),
+            _ptr(stats, "stats", torch.float32, topk_stats_shape(cfg, block, cache_cap)), _stream(stream)]
+    _check(load_library().rat_topk_build_stats(cfg.ref(), *args), "rat_topk_build_stats")
+
+
+def rat_topk_decode_step(cfg, block, topk, mode, q, k, v, g, state_k, state_v, cache_k, cache_v, cache_cap, stats,
+                         pos, o, lse=None, sel=None, ws=None, stream=None):
+    c = cfg.c
+    tok = (c.B, c.H, c.d)
+    dt = cfg.torch_dtype
+    R = rat_cache_rows(cfg, cache_cap)
+    cshape = (c.B, c.H, R, c.d)
+    args = [int(block), int(topk), int(mode),
+            _ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
+            _ptr(state_k, "state_k", torch.float32, tok), _ptr(state_v, "state_v", torch.float32, tok),
+            _ptr(cache_k, "cache_k", dt, cshape), _ptr(cache_v, "cache_v", dt, cshape), int(cache_cap),
+            _ptr(stats, "stats", torch.float32, topk_stats_shape(cfg, block, cache_cap)),
+            _ptr(pos, "pos", torch.int32, (c.B,)), _ptr(o, "o", dt, tok),
+            _ptr(lse, "lse", torch.float32, (c.B, c.H), True),
+            _ptr(sel, "sel", torch.int32, (c.B, c.H, int(topk)), True),
+            _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream)]
+    _check(load_library().rat_topk_decode_step(cfg.ref(), *args), "rat_topk_decode_step")
+
+
+def paged_cache(cfg, pool_k, pool_v, page_table, cache_cap):
+    """A rat_paged_cache over torch tensors: pools [num_pages, H, page_rows, d]
+    in the cfg's dtype and a device int32 table [B, pages_per_seq]."""
+    c = cfg.c
+    if pool_k.dim() != 4 or pool_k.shape[1] != c.H or pool_k.shape[3] != c.d:
+        raise ValueError("pool_k must be [num_pages, H, page_rows, d]")
+    n, _, P, _ = pool_k.shape
+    _ptr(pool_k, "pool_k", cfg.torch_dtype)
+    _ptr(pool_v, "pool_v", cfg.torch_dtype, tuple(pool_k.shape))
+    _ptr(page_table, "page_table", torch.int32)
+    if page_table.dim() != 2 or page_table.shape[0] != c.B:
+        raise ValueError("page_table must be [B, pages_per_seq]")
+    return rat_paged_cache(pool_k.data_ptr(), pool_v.data_ptr(), page_table.data_ptr(), int(P),
+                           int(page_table.shape[1]), int(n))
+
+
+def rat_scan_prefill_paged(cfg, k, v, g, init_k=None, init_v=None, kt=None, vt=None, final_k=None, final_v=None,
+                           cache=None, cache_cap=0, ws=None, stream=None):
+    """rat_scan_prefill into a paged cache (a rat_paged_cache from paged_cache())."""
+    c = cfg.c
+    tok = (c.B, c.T, c.H, c.d)
+    st = (c.B, c.H, c.d)
+    dt = cfg.torch_dtype
+    args = [_ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
+            _ptr(init_k, "init_k", torch.float32, st, True), _ptr(init_v, "init_v", torch.float32, st, True),
+            _ptr(kt, "kt", dt, cfg.history_shape, True), _ptr(vt, "vt", dt, cfg.history_shape, True),
+            _ptr(final_k, "final_k", torch.float32, st, True), _ptr(final_v, "final_v", torch.float32, st, True),
+            ctypes.byref(cache), int(cache_cap), _ptr(ws, "ws", torch.uint8), ws.numel(), _stream(stream)]
+    _check(load_library().rat_scan_prefill_paged(cfg.ref(), *args), "rat_scan_prefill_paged")
+
+
+def rat_decode_step_paged(cfg, q, k, v, g, state_k, state_v, cache, cache_cap, pos, o, lse=None, ws=None,
+                          stream=None):
+    """rat_decode_step over a paged cache (a rat_paged_cache from paged_cache())."""
+    c = cfg.c
+    tok = (c.B, c.H, c.d)
+    dt = cfg.torch_dtype
+    args = [_ptr(q, "q", dt, tok), _ptr(k, "k", dt, tok), _ptr(v, "v", dt, tok), _ptr(g, "g", dt, cfg.gate_shape(tok)),
+            _ptr(state_k, "state_k", torch.float32, tok), _ptr(state_v, "state_v", torch.float32, tok),
+            ctypes.byref(cache), int(cache_cap), _ptr(pos, "pos", torch.int32, (c.B,)), _ptr(o, "o", dt, tok),
+            _ptr(lse, "lse", torch.float32, (c.B, c.H), True), _ptr(ws, "ws", torch.uint8), ws.numel(),
+            _stream(stream)]
+    _check(load_library().rat_decode_step_paged(cfg.ref(), *args), "rat_decode_step_paged")
 
 
 def rat_check_status(ws, stream=None):
@@ -266,8 +382,11 @@ def rat_debug_set_scan_stall(ws, ticket, spin_limit_ns=0, stream=None):
 
 
 def mix_prefill(cfg, q, k, v, g, init_k=None, init_v=None, want_kv=False, want_lse=True, ws=None, stream=None):
-    """Allocate outputs with torch and run rat_mix_prefill.  Returns a dict."""
+    """Allocate outputs with torch and run rat_mix_prefill.  Returns a dict.
+    (A chunked prefill, t0 > 0, calls rat_mix_prefill with its kt/vt history.)"""
     c = cfg.c
+    if c.t0 > 0:
+        raise ValueError("mix_prefill allocates its own kt/vt: with t0 > 0 call rat_mix_prefill with the history")
     dev = q.device
     o = torch.empty_like(q)
     lse = torch.empty((c.B, c.H, c.T), dtype=torch.float32, device=dev) if want_lse else None

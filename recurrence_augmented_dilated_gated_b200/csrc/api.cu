@@ -73,18 +73,39 @@ rat_status check_cfg(const rat_cfg *c, bool need_T = true) {
     const double elems = (double)c->B * (need_T ? (double)c->T : 1.0) * c->H * c->d;
     if (elems >= 1099511627776.0) return fail(RAT_ERR_INVALID, "B*T*H*d too large");
     if (!(c->scale == c->scale)) return fail(RAT_ERR_INVALID, "scale is NaN");
+    if (c->t0 < 0 || (long long)c->t0 + c->T > 0x7fffffffLL) return fail(RAT_ERR_INVALID, "t0 %d out of range", c->t0);
+    if (c->t_cap != 0 && (long long)c->t_cap < (long long)c->t0 + c->T)
+        return fail(RAT_ERR_INVALID, "t_cap %d < t0 + T", c->t_cap);
+    if (need_T && (double)c->B * ((double)c->t0 + c->T + c->t_cap) * c->H * c->d >= 1099511627776.0)
+        return fail(RAT_ERR_INVALID, "B*(t0+T)*H*d too large");
+    if (c->flags & ~(RAT_FLAG_GRID_DILATION | RAT_FLAG_DEDUPE | RAT_FLAG_SEPARATE_GATES))
+        return fail(RAT_ERR_INVALID, "unknown flags 0x%x", c->flags);
     return RAT_OK;
 }
 
 bool head_recur(const rat_cfg *c, int h) { return c->recur == nullptr || c->recur[h] != 0; }
 
+bool grid_mode(const rat_cfg *c) { return (c->flags & RAT_FLAG_GRID_DILATION) != 0; }
+
+// rows per batch entry of the kt/vt history (t0 + T unless the caller's buffer is longer)
+int hist_rows(const rat_cfg *c) { return c->t_cap ? c->t_cap : c->t0 + c->T; }
+
+bool dedupe_mode(const rat_cfg *c) { return (c->flags & RAT_FLAG_DEDUPE) != 0; }
+
+// The window a head's attention runs: with dedupe a D = 1 head's window keys
+// all lie in its dilated set, so it has no window part.
+int attn_window(const rat_cfg *c, int h) { return dedupe_mode(c) && c->dil[h] == 1 ? 0 : c->win[h]; }
+
 float scale_of(const rat_cfg *c) { return c->scale > 0.f ? c->scale : 1.0f / sqrtf((float)c->d); }
 
+// Rows of one (b, h) block of the decode cache: residue-major, all positions;
+// or, under the fixed grid, the grid rows plus the window ring (D > 1, W > 0).
 int64_t cache_rows(const rat_cfg *c, int cap) {
     int64_t R = 0;
     for (int h = 0; h < c->H; ++h) {
-        const int64_t D = c->dil[h];
-        R = std::max<int64_t>(R, D * ((cap + D - 1) / D));
+        const int64_t D = c->dil[h], S = (cap + D - 1) / D;
+        const int64_t rows = grid_mode(c) ? S + (D > 1 ? (int64_t)c->win[h] : 0) : D * S;
+        R = std::max<int64_t>(R, rows);
     }
     return R;
 }
@@ -168,12 +189,39 @@ rat_status empty_prefill_state(const rat_cfg *c, const float *ik, const float *i
     return RAT_OK;
 }
 
+bool separate_gates(const rat_cfg *c) { return (c->flags & RAT_FLAG_SEPARATE_GATES) != 0; }
+
+// One scan launch: tensor maps of its operands, zeroed ticket and chunk flags.
+rat_status scan_pass(const rat_cfg *c, const Layout &L, ScanParams &p, char *ws, cudaStream_t s) {
+    // the one-tensor form reads slot 1 of neither list: repeat slot 0 there
+    const void *srcs[5] = {p.x[0], p.x[1] ? p.x[1] : p.x[0], p.g, p.out[0], p.out[1] ? p.out[1] : p.out[0]};
+    p.use_tma_out = p.out[0] != nullptr ? 1 : 0;
+    // inputs hold the call's T positions; kt / vt are the [B, t0+T, H, d] history
+    for (int i = 0; i < (p.use_tma_out ? 5 : 3); ++i)
+        if (!encode_map_tokens(&p.tmap[i], srcs[i], c->dtype, c->B, i < 3 ? c->T : c->t0 + c->T,
+                               i < 3 ? c->T : hist_rows(c), c->H, c->d, p.chunk_len))
+            return fail(RAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (scan operand %d)", i);
+    // zero the ticket and the chunk flags (one contiguous range)
+    cudaError_t e = cudaMemsetAsync(ws + L.ticket, 0, L.agg - L.ticket, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(scan flags)");
+    e = launch_scan(p, c->dtype, s);
+    if (e != cudaSuccess) return cuda_fail(e, "scan launch");
+    return RAT_OK;
+}
+
 // Scan of the selected heads into kt/vt and/or the cache.
 rat_status run_scan(const rat_cfg *c, const Layout &L, const void *k, const void *v, const void *g,
                     const float *ik, const float *iv, void *kt, void *vt, float *fk, float *fv,
-                    void *ck, void *cv, int cap, char *ws, bool only_recurrent, cudaStream_t s) {
+                    void *ck, void *cv, int cap, char *ws, bool only_recurrent, cudaStream_t s,
+                    const rat_paged_cache *pc = nullptr) {
     ScanParams p;
     memset(&p, 0, sizeof(p));
+    if (pc) {
+        p.page_table = pc->page_table;
+        p.page_rows = pc->page_rows;
+        p.pps = pc->pages_per_seq;
+        p.num_pages = pc->num_pages;
+    }
     p.x[0] = k; p.x[1] = v; p.g = g;
     p.init[0] = ik; p.init[1] = iv;
     p.out[0] = kt; p.out[1] = vt;
@@ -181,12 +229,15 @@ rat_status run_scan(const rat_cfg *c, const Layout &L, const void *k, const void
     p.cache[0] = ck; p.cache[1] = cv;
     p.cap = cap;
     p.cache_R = ck ? cache_rows(c, cap) : 0;
+    p.grid = grid_mode(c) ? 1 : 0;
     p.B = c->B; p.T = c->T; p.H = c->H; p.d = c->d;
+    p.t0 = c->t0;
     int n = 0, n_plain = 0;
     unsigned char plain[kMaxHeads];
     for (int h = 0; h < c->H; ++h) {
         p.head_recur[h] = head_recur(c, h) ? 1 : 0;
         p.head_dil[h] = c->dil[h];
+        p.head_win[h] = c->win[h];
         if (!only_recurrent || p.head_recur[h]) p.head_list[n++] = (unsigned char)h;
         else plain[n_plain++] = (unsigned char)h;
     }
@@ -203,49 +254,63 @@ rat_status run_scan(const rat_cfg *c, const Layout &L, const void *k, const void
     p.nslices = c->B * n;
     p.nchunks = L.nchunks;
     p.chunk_len = scan_chunk_len(c->d);
-    const void *srcs[5] = {k, v, g, kt, vt};
-    p.use_tma_out = kt != nullptr ? 1 : 0;
-    for (int i = 0; i < (p.use_tma_out ? 5 : 3); ++i)
-        if (!encode_map_tokens(&p.tmap[i], srcs[i], c->dtype, c->B, c->T, c->H, c->d, p.chunk_len))
-            return fail(RAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (scan operand %d)", i);
     p.ticket = reinterpret_cast<unsigned *>(ws + L.ticket);
     p.flags = reinterpret_cast<int *>(ws + L.flags);
     p.agg = reinterpret_cast<float *>(ws + L.agg);
     p.incl = reinterpret_cast<float *>(ws + L.incl);
     p.hdr = reinterpret_cast<WsHeader *>(ws);
-    // zero the ticket and the chunk flags (one contiguous range)
-    cudaError_t e = cudaMemsetAsync(ws + L.ticket, 0, L.agg - L.ticket, s);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(scan flags)");
-    e = launch_scan(p, c->dtype, s);
-    if (e != cudaSuccess) return cuda_fail(e, "scan launch");
-    return RAT_OK;
+    if (!separate_gates(c)) return scan_pass(c, L, p, ws, s);
+    // separate gates: the keys with g[0], then the values with g[1], each in
+    // the one-tensor form of the scan (ordered on the stream, one workspace)
+    ScanParams pk = p, pv = p;
+    pk.one = pv.one = 1;
+    pk.x[1] = nullptr; pk.init[1] = nullptr; pk.out[1] = nullptr; pk.fin[1] = nullptr; pk.cache[1] = nullptr;
+    pv.x[0] = v; pv.init[0] = iv; pv.out[0] = vt; pv.fin[0] = fv; pv.cache[0] = cv;
+    pv.x[1] = nullptr; pv.init[1] = nullptr; pv.out[1] = nullptr; pv.fin[1] = nullptr; pv.cache[1] = nullptr;
+    pv.g = static_cast<const char *>(g) + (size_t)c->B * c->T * c->H * c->d * elt_size(c->dtype);
+    rat_status st = scan_pass(c, L, pk, ws, s);
+    if (st != RAT_OK) return st;
+    return scan_pass(c, L, pv, ws, s);
 }
+
+// Kind of a head's dilated part on the tensor cores: the residue subsequences,
+// or (fixed grid, D > 1) every position against the grid subsequence.
+bool grid_head(const rat_cfg *c, int h) { return grid_mode(c) && c->dil[h] > 1; }
 
 // A head runs on the tensor-core kernel when its operands are bf16 and its
 // dilation divides T (the strided TMA view needs whole subsequences);
 // otherwise the fp32 CUDA-core kernel computes it.
-bool tc_head(const rat_cfg *c, int h) { return c->dtype == RAT_BF16 && c->T % c->dil[h] == 0; }
+// (A chunked prefill also needs t0 % D == 0: its residues line up with the
+// history's.)
+bool tc_head(const rat_cfg *c, int h) {
+    return c->dtype == RAT_BF16 && c->T % c->dil[h] == 0 && c->t0 % c->dil[h] == 0;
+}
 
-// One tensor-core launch over `heads` (dilated part, or window part when
-// window_mode), grouped into classes of equal (dilation, K/V source).
-rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, bool window_mode, const void *q,
+// One tensor-core launch over `heads` (kind kTcDilated, kTcWindow or kTcGrid),
+// grouped into classes of equal (dilation, K/V source).
+rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, int kind, const void *q,
                           const void *kt, const void *vt, const void *kraw, const void *vraw,
                           const bool *raw_head, void *o, float *lse, float *lse_dil, char *ws, unsigned *tickets,
                           int *n_launch, cudaStream_t s) {
-    struct Key { int D; int raw; };
+    struct Key { int D; int raw; int xd; };
     int done = 0;
     bool taken[kMaxHeads] = {false};
     while (done < nheads) {
         TcParams P;
         memset(&P, 0, sizeof(P));
         P.B = c->B; P.T = c->T; P.H = c->H;
-        P.window_mode = window_mode ? 1 : 0;
+        P.kind = kind;
+        P.q = q;
+        P.t0 = c->t0;
+        P.Tk = c->t0 + c->T;
+        P.Th = hist_rows(c);
         P.scale_log2 = scale_of(c) * 1.4426950408889634f;
         P.o = o; P.lse_user = lse; P.lse_dil = lse_dil;
         P.hdr = reinterpret_cast<WsHeader *>(ws);
         if (*n_launch >= kAttnTickets) return fail(RAT_ERR_UNSUPPORTED, "more than %d attention launches", kAttnTickets);
         P.ticket = tickets + (*n_launch)++;
-        for (int h = 0; h < c->H; ++h) P.win[h] = c->win[h];
+        P.grid = grid_mode(c) ? 1 : 0;
+        for (int h = 0; h < c->H; ++h) P.win[h] = attn_window(c, h);
         // collect up to kTcMaxClasses classes
         Key keys[kTcMaxClasses];
         int ncls = 0, nh = 0;
@@ -254,10 +319,12 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, bool w
         for (int i = 0; i < nheads; ++i) {
             const int h = heads[i];
             if (taken[i]) continue;
-            const Key k{window_mode ? 1 : c->dil[h], raw_head[h] ? 1 : 0};
+            const bool win_kind = kind == kTcWindow || kind == kTcWindowDedupe;
+            // the dedupe window launch also tells the heads' dilations apart
+            const Key k{win_kind ? 1 : c->dil[h], raw_head[h] ? 1 : 0, kind == kTcWindowDedupe ? c->dil[h] : 1};
             int ci = -1;
             for (int j = 0; j < ncls; ++j)
-                if (keys[j].D == k.D && keys[j].raw == k.raw) ci = j;
+                if (keys[j].D == k.D && keys[j].raw == k.raw && keys[j].xd == k.xd) ci = j;
             if (ci < 0) {
                 if (ncls == kTcMaxClasses) continue;  // next launch
                 ci = ncls++;
@@ -277,18 +344,26 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, bool w
             const int ci = order[oi];
             TcClass &C = P.cls[oi];
             C.D = keys[ci].D;
-            C.n = c->T / C.D;
+            // query rows per group: a residue subsequence, or every position
+            C.n = kind == kTcDilated ? c->T / C.D : c->T;
+            C.nres = kind == kTcDilated ? C.D : 1;
+            C.kres = kind == kTcGrid ? C.D - 1 : 0;   // the grid is residue D-1
+            C.xd = keys[ci].xd;
             C.mtiles = (C.n + 255) / 256;   // 256-row units per (b, h, residue) group
             C.nheads = cls_n[ci];
             C.head0 = nh;
             for (int j = 0; j < cls_n[ci]; ++j) P.heads[nh++] = (unsigned char)cls_heads[ci][j];
             P.prefix[oi] = pref;
-            pref += (long long)c->B * C.nheads * C.D * C.mtiles;
+            pref += (long long)c->B * C.nheads * C.nres * C.mtiles;
             const void *kb = keys[ci].raw ? kraw : kt;
             const void *vb = keys[ci].raw ? vraw : vt;
-            if (!encode_map_5d(&P.tq[oi], q, c->B, c->T, c->H, c->d, C.D, kTcRowsQ) ||
-                !encode_map_5d(&P.tk[oi], kb, c->B, c->T, c->H, c->d, C.D, kTcRowsKV) ||
-                !encode_map_5d(&P.tv[oi], vb, c->B, c->T, c->H, c->d, C.D, kTcRowsKV))
+            P.kself[oi] = kb;
+            P.vself[oi] = vb;
+            // raw k / v (heads without recurrence, mix prefill) hold the call's rows only
+            const int kv_rows = keys[ci].raw ? c->T : P.Th;
+            if (!encode_map_5d(&P.tq[oi], q, c->B, c->T, c->T, c->H, c->d, kind == kTcGrid ? 1 : C.D, kTcRowsQ) ||
+                !encode_map_5d(&P.tk[oi], kb, c->B, P.Tk, kv_rows, c->H, c->d, C.D, kTcRowsKV) ||
+                !encode_map_5d(&P.tv[oi], vb, c->B, P.Tk, kv_rows, c->H, c->d, C.D, kTcRowsKV))
                 return fail(RAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (dilation %d)", C.D);
         }
         P.prefix[ncls] = pref;
@@ -303,30 +378,37 @@ rat_status run_attn(const rat_cfg *c, const Layout &L, const void *q, const void
                     const void *kraw, const void *vraw, bool raw_for_plain_heads, void *o, float *lse,
                     char *ws, cudaStream_t s) {
     bool raw_head[kMaxHeads];
-    int tc_all[kMaxHeads], tc_win[kMaxHeads];
-    int n_tc = 0, n_win = 0, n_simt = 0;
+    int tc_all[kMaxHeads], tc_grid[kMaxHeads], tc_win[kMaxHeads];
+    int n_tc = 0, n_grid = 0, n_win = 0, n_simt = 0;
     for (int h = 0; h < c->H; ++h) {
         raw_head[h] = raw_for_plain_heads && !head_recur(c, h);
         if (tc_head(c, h)) {
-            tc_all[n_tc++] = h;
-            if (c->win[h] > 0) tc_win[n_win++] = h;
+            if (grid_head(c, h)) tc_grid[n_grid++] = h;
+            else tc_all[n_tc++] = h;
+            if (attn_window(c, h) > 0) tc_win[n_win++] = h;
         } else {
             ++n_simt;
         }
     }
     float *lse_dil = reinterpret_cast<float *>(ws + L.lse_dil);
-    if (n_tc > 0) {
+    if (n_tc + n_grid > 0) {
         unsigned *tickets = reinterpret_cast<unsigned *>(ws + L.att_ticket);
         int n_launch = 0;
         cudaError_t e = cudaMemsetAsync(tickets, 0, kAttnTickets * sizeof(unsigned), s);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(attention tickets)");
         // The sort in launch_tc_part orders classes by dilation; with T fixed,
         // a smaller dilation means longer subsequences, i.e. more query tiles.
-        rat_status st = launch_tc_part(c, tc_all, n_tc, false, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws,
-                                       tickets, &n_launch, s);
+        rat_status st = RAT_OK;
+        if (n_tc > 0)
+            st = launch_tc_part(c, tc_all, n_tc, kTcDilated, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws,
+                                tickets, &n_launch, s);
+        if (st != RAT_OK) return st;
+        if (n_grid > 0)
+            st = launch_tc_part(c, tc_grid, n_grid, kTcGrid, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws,
+                                tickets, &n_launch, s);
         if (st != RAT_OK) return st;
         if (n_win > 0) {
-            st = launch_tc_part(c, tc_win, n_win, true, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws,
+            st = launch_tc_part(c, tc_win, n_win, dedupe_mode(c) ? kTcWindowDedupe : kTcWindow, q, kt, vt, kraw, vraw, raw_head, o, lse, lse_dil, ws,
                                 tickets, &n_launch, s);
             if (st != RAT_OK) return st;
         }
@@ -337,10 +419,14 @@ rat_status run_attn(const rat_cfg *c, const Layout &L, const void *q, const void
         p.q = q; p.kt = kt; p.vt = vt; p.kraw = kraw; p.vraw = vraw;
         p.o = o; p.lse = lse;
         p.B = c->B; p.T = c->T; p.H = c->H; p.d = c->d;
+        p.t0 = c->t0;
+        p.Th = hist_rows(c);
         p.scale_log2 = scale_of(c) * 1.4426950408889634f;
+        p.grid = grid_mode(c) ? 1 : 0;
+        p.dedupe = dedupe_mode(c) ? 1 : 0;
         for (int h = 0; h < c->H; ++h) {
             p.dil[h] = c->dil[h];
-            p.win[h] = c->win[h];
+            p.win[h] = attn_window(c, h);
             p.use_raw[h] = raw_head[h] ? 1 : 0;
             p.skip[h] = tc_head(c, h) ? 1 : 0;
         }
@@ -351,11 +437,97 @@ rat_status run_attn(const rat_cfg *c, const Layout &L, const void *q, const void
     return RAT_OK;
 }
 
+// A paged cache descriptor: pools and table given, pages cover the logical rows.
+rat_status check_paged(const rat_cfg *c, const rat_paged_cache *pc, int cap) {
+    if (!pc) return fail(RAT_ERR_INVALID, "paged cache descriptor is NULL");
+    CHECK_PTR(pc->pool_k, "pool_k"); CHECK_PTR(pc->pool_v, "pool_v"); CHECK_PTR(pc->page_table, "page_table");
+    if (pc->page_rows < 1 || pc->num_pages < 1 || pc->pages_per_seq < 1)
+        return fail(RAT_ERR_INVALID, "page_rows %d, num_pages %d, pages_per_seq %d must be >= 1", pc->page_rows,
+                    pc->num_pages, pc->pages_per_seq);
+    if (cap < 1) return fail(RAT_ERR_INVALID, "cache_cap %d < 1", cap);
+    const long long R = cache_rows(c, cap);
+    if ((long long)pc->pages_per_seq * pc->page_rows < R)
+        return fail(RAT_ERR_INVALID, "pages_per_seq x page_rows < %lld cache rows", R);
+    return RAT_OK;
+}
+
+// rat_decode_step with a dense cache (pc = NULL) or a paged one.
+rat_status decode_step(const rat_cfg *cfg, const void *q, const void *k, const void *v, const void *g,
+                       float *state_k, float *state_v, void *cache_k, void *cache_v, const rat_paged_cache *pc,
+                       int cache_cap, const int32_t *pos, void *o, float *lse, void *ws, size_t ws_bytes,
+                       rat_stream_t stream) {
+    rat_status st = check_cfg(cfg, false);
+    if (st != RAT_OK) return st;
+    if (cfg->B == 0) return RAT_OK;
+    CHECK_PTR(q, "q"); CHECK_PTR(k, "k"); CHECK_PTR(v, "v"); CHECK_PTR(g, "g");
+    CHECK_PTR(state_k, "state_k"); CHECK_PTR(state_v, "state_v");
+    CHECK_PTR(cache_k, "cache_k"); CHECK_PTR(cache_v, "cache_v");
+    CHECK_PTR(pos, "pos"); CHECK_PTR(o, "o"); CHECK_OPT(lse, "lse");
+    if (cache_cap < 1) return fail(RAT_ERR_INVALID, "cache_cap %d < 1", cache_cap);
+    Layout L;
+    st = check_ws(cfg, RAT_OP_DECODE, cache_cap, ws, ws_bytes, &L);
+    if (st != RAT_OK) return st;
+    DecodeParams p;
+    memset(&p, 0, sizeof(p));
+    decode_plan(cfg, cache_cap, &p);
+    p.q = q; p.k = k; p.v = v; p.g = g;
+    p.state[0] = state_k; p.state[1] = state_v;
+    p.cache[0] = cache_k; p.cache[1] = cache_v;
+    if (pc) {
+        p.page_table = pc->page_table;
+        p.page_rows = pc->page_rows;
+        p.pps = pc->pages_per_seq;
+        p.num_pages = pc->num_pages;
+    }
+    p.pos = pos; p.o = o; p.lse = lse;
+    char *w = static_cast<char *>(ws);
+    p.part = reinterpret_cast<float *>(w + L.part);
+    const size_t part_bytes = align256((size_t)cfg->B * p.items_per_b * (cfg->d + 2) * sizeof(float));
+    p.counter = reinterpret_cast<int *>(w + L.part + part_bytes);
+    p.cap = cache_cap; p.B = cfg->B; p.H = cfg->H; p.d = cfg->d;
+    p.scale_log2 = scale_of(cfg) * 1.4426950408889634f;
+    p.hdr = reinterpret_cast<WsHeader *>(ws);
+    // per-(b,h) completion counters start from zero on every call
+    cudaError_t ez = cudaMemsetAsync(p.counter, 0, (size_t)cfg->B * cfg->H * sizeof(int), (cudaStream_t)stream);
+    if (ez != cudaSuccess) return cuda_fail(ez, "cudaMemsetAsync(decode counters)");
+    cudaError_t e = launch_decode(p, cfg->dtype, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    return RAT_OK;
+}
+
+// rat_scan_prefill with a dense cache (pc = NULL) or a paged one.
+rat_status scan_prefill(const rat_cfg *cfg, const void *k, const void *v, const void *g, const float *init_k,
+                        const float *init_v, void *kt, void *vt, float *final_k, float *final_v, void *cache_k,
+                        void *cache_v, const rat_paged_cache *pc, int cache_cap, void *ws, size_t ws_bytes,
+                        rat_stream_t stream) {
+    rat_status st = check_cfg(cfg);
+    if (st != RAT_OK) return st;
+    CHECK_OPT(init_k, "init_k"); CHECK_OPT(init_v, "init_v");
+    CHECK_OPT(final_k, "final_k"); CHECK_OPT(final_v, "final_v");
+    if (empty(cfg)) return empty_prefill_state(cfg, init_k, init_v, final_k, final_v, (cudaStream_t)stream);
+    CHECK_PTR(k, "k"); CHECK_PTR(v, "v"); CHECK_PTR(g, "g");
+    CHECK_OPT(init_k, "init_k"); CHECK_OPT(init_v, "init_v");
+    CHECK_OPT(kt, "kt"); CHECK_OPT(vt, "vt");
+    CHECK_OPT(final_k, "final_k"); CHECK_OPT(final_v, "final_v");
+    CHECK_OPT(cache_k, "cache_k"); CHECK_OPT(cache_v, "cache_v");
+    if ((kt == nullptr) != (vt == nullptr)) return fail(RAT_ERR_INVALID, "kt and vt must be given together");
+    if ((cache_k == nullptr) != (cache_v == nullptr))
+        return fail(RAT_ERR_INVALID, "cache_k and cache_v must be given together");
+    if (!kt && !cache_k) return fail(RAT_ERR_INVALID, "no output: give kt/vt and/or cache_k/cache_v");
+    if (cache_k && cache_cap < (long long)cfg->t0 + cfg->T)
+        return fail(RAT_ERR_INVALID, "cache_cap %d < t0 + T = %lld", cache_cap, (long long)cfg->t0 + cfg->T);
+    Layout L;
+    st = check_ws(cfg, RAT_OP_SCAN, 0, ws, ws_bytes, &L);
+    if (st != RAT_OK) return st;
+    return run_scan(cfg, L, k, v, g, init_k, init_v, kt, vt, final_k, final_v, cache_k, cache_v,
+                    cache_cap, static_cast<char *>(ws), false, (cudaStream_t)stream, pc);
+}
+
 }  // namespace
 
 extern "C" {
 
-int rat_version(void) { return 100; }
+int rat_version(void) { return 101; }
 
 long long rat_launch_count(void) { return rat::g_launches.load(std::memory_order_relaxed); }
 
@@ -374,9 +546,11 @@ const char *rat_status_string(rat_status s) {
 }
 
 size_t rat_workspace_size(const rat_cfg *cfg, int op, int cache_cap) {
-    if (op < RAT_OP_SCAN || op > RAT_OP_DECODE) return 0;
-    if (check_cfg(cfg, op != RAT_OP_DECODE) != RAT_OK) return 0;
-    if (op == RAT_OP_DECODE && cache_cap < 1) return 0;
+    if (op < RAT_OP_SCAN || op > RAT_OP_TOPK_DECODE) return 0;
+    const bool dec = op == RAT_OP_DECODE || op == RAT_OP_TOPK_DECODE;
+    if (check_cfg(cfg, !dec) != RAT_OK) return 0;
+    if (dec && cache_cap < 1) return 0;
+    if (op == RAT_OP_TOPK_DECODE) return sizeof(WsHeader);   // the status word only
     return layout(cfg, op, cache_cap).total;
 }
 
@@ -396,26 +570,20 @@ rat_status rat_scan_prefill(const rat_cfg *cfg, const void *k, const void *v, co
                             const float *init_k, const float *init_v, void *kt, void *vt,
                             float *final_k, float *final_v, void *cache_k, void *cache_v,
                             int cache_cap, void *ws, size_t ws_bytes, rat_stream_t stream) {
+    return scan_prefill(cfg, k, v, g, init_k, init_v, kt, vt, final_k, final_v, cache_k, cache_v, nullptr,
+                        cache_cap, ws, ws_bytes, stream);
+}
+
+rat_status rat_scan_prefill_paged(const rat_cfg *cfg, const void *k, const void *v, const void *g,
+                                  const float *init_k, const float *init_v, void *kt, void *vt, float *final_k,
+                                  float *final_v, const rat_paged_cache *cache, int cache_cap, void *ws,
+                                  size_t ws_bytes, rat_stream_t stream) {
     rat_status st = check_cfg(cfg);
     if (st != RAT_OK) return st;
-    CHECK_OPT(init_k, "init_k"); CHECK_OPT(init_v, "init_v");
-    CHECK_OPT(final_k, "final_k"); CHECK_OPT(final_v, "final_v");
-    if (empty(cfg)) return empty_prefill_state(cfg, init_k, init_v, final_k, final_v, (cudaStream_t)stream);
-    CHECK_PTR(k, "k"); CHECK_PTR(v, "v"); CHECK_PTR(g, "g");
-    CHECK_OPT(init_k, "init_k"); CHECK_OPT(init_v, "init_v");
-    CHECK_OPT(kt, "kt"); CHECK_OPT(vt, "vt");
-    CHECK_OPT(final_k, "final_k"); CHECK_OPT(final_v, "final_v");
-    CHECK_OPT(cache_k, "cache_k"); CHECK_OPT(cache_v, "cache_v");
-    if ((kt == nullptr) != (vt == nullptr)) return fail(RAT_ERR_INVALID, "kt and vt must be given together");
-    if ((cache_k == nullptr) != (cache_v == nullptr))
-        return fail(RAT_ERR_INVALID, "cache_k and cache_v must be given together");
-    if (!kt && !cache_k) return fail(RAT_ERR_INVALID, "no output: give kt/vt and/or cache_k/cache_v");
-    if (cache_k && cache_cap < cfg->T) return fail(RAT_ERR_INVALID, "cache_cap %d < T %d", cache_cap, cfg->T);
-    Layout L;
-    st = check_ws(cfg, RAT_OP_SCAN, 0, ws, ws_bytes, &L);
+    st = check_paged(cfg, cache, cache_cap);
     if (st != RAT_OK) return st;
-    return run_scan(cfg, L, k, v, g, init_k, init_v, kt, vt, final_k, final_v, cache_k, cache_v,
-                    cache_cap, static_cast<char *>(ws), false, (cudaStream_t)stream);
+    return scan_prefill(cfg, k, v, g, init_k, init_v, kt, vt, final_k, final_v, cache->pool_k, cache->pool_v,
+                        cache, cache_cap, ws, ws_bytes, stream);
 }
 
 rat_status rat_dilated_attn_prefill(const rat_cfg *cfg, const void *q, const void *kt, const void *vt,
@@ -447,6 +615,10 @@ rat_status rat_mix_prefill(const rat_cfg *cfg, const void *q, const void *k, con
     CHECK_OPT(final_k, "final_k"); CHECK_OPT(final_v, "final_v");
     if ((kt == nullptr) != (vt == nullptr)) return fail(RAT_ERR_INVALID, "kt and vt must be given together");
     const bool caller_kv = kt != nullptr;
+    if (cfg->t0 > 0 && !caller_kv)
+        return fail(RAT_ERR_INVALID, "a chunked prefill (t0 > 0) needs the caller's kt/vt history");
+    if (!caller_kv && cfg->t_cap != 0 && cfg->t_cap != cfg->T)
+        return fail(RAT_ERR_INVALID, "t_cap describes the caller's kt/vt; the workspace keeps T rows");
     Layout L;
     st = check_ws(cfg, caller_kv ? RAT_OP_MIX_CALLER_KV : RAT_OP_MIX, 0, ws, ws_bytes, &L);
     if (st != RAT_OK) return st;
@@ -468,36 +640,99 @@ rat_status rat_decode_step(const rat_cfg *cfg, const void *q, const void *k, con
                            const void *g, float *state_k, float *state_v, void *cache_k,
                            void *cache_v, int cache_cap, const int32_t *pos, void *o, float *lse,
                            void *ws, size_t ws_bytes, rat_stream_t stream) {
+    return decode_step(cfg, q, k, v, g, state_k, state_v, cache_k, cache_v, nullptr, cache_cap, pos, o, lse, ws,
+                       ws_bytes, stream);
+}
+
+rat_status rat_decode_step_paged(const rat_cfg *cfg, const void *q, const void *k, const void *v, const void *g,
+                                 float *state_k, float *state_v, const rat_paged_cache *cache, int cache_cap,
+                                 const int32_t *pos, void *o, float *lse, void *ws, size_t ws_bytes,
+                                 rat_stream_t stream) {
     rat_status st = check_cfg(cfg, false);
+    if (st != RAT_OK) return st;
+    st = check_paged(cfg, cache, cache_cap);
+    if (st != RAT_OK) return st;
+    return decode_step(cfg, q, k, v, g, state_k, state_v, cache->pool_k, cache->pool_v, cache, cache_cap, pos, o,
+                       lse, ws, ws_bytes, stream);
+}
+
+// ---------------------------------------------------------- top-k block decode
+
+namespace {
+
+rat_status check_topk(const rat_cfg *c, int block, int topk, int mode, int cap) {
+    rat_status st = check_cfg(c, false);
+    if (st != RAT_OK) return st;
+    if (block < 1) return fail(RAT_ERR_INVALID, "block %d < 1", block);
+    if (topk < 0 || topk > kTopkMaxK) return fail(RAT_ERR_INVALID, "topk %d outside [0, %d]", topk, kTopkMaxK);
+    if (mode != RAT_TOPK_QUEST && mode != RAT_TOPK_MOBA) return fail(RAT_ERR_INVALID, "top-k mode %d", mode);
+    if (cap < 1) return fail(RAT_ERR_INVALID, "cache_cap %d < 1", cap);
+    if ((cap + (long long)block - 1) / block > kTopkMaxBlocks)
+        return fail(RAT_ERR_UNSUPPORTED, "ceil(cache_cap / block) exceeds %d blocks", kTopkMaxBlocks);
+    for (int h = 0; h < c->H; ++h)
+        if (c->dil[h] != 1 || c->win[h] != 0)
+            return fail(RAT_ERR_INVALID, "top-k decoding needs dil = 1 and win = 0 (head %d)", h);
+    return RAT_OK;
+}
+
+TopkParams topk_params(const rat_cfg *c, int block, int topk, int mode, int cap, float *stats) {
+    TopkParams p;
+    memset(&p, 0, sizeof(p));
+    p.cache_R = cache_rows(c, cap);
+    p.cap = cap; p.B = c->B; p.H = c->H; p.d = c->d;
+    p.bs = block; p.K = topk; p.mode = mode;
+    p.sep = separate_gates(c) ? 1 : 0;
+    p.nblk = (int)((cap + (long long)block - 1) / block);
+    p.stats = stats;
+    p.scale_log2 = scale_of(c) * 1.4426950408889634f;
+    for (int h = 0; h < c->H; ++h) p.recur[h] = head_recur(c, h) ? 1 : 0;
+    return p;
+}
+
+}  // namespace
+
+size_t rat_topk_stats_size(const rat_cfg *cfg, int block, int cache_cap) {
+    if (check_topk(cfg, block, 0, RAT_TOPK_QUEST, cache_cap) != RAT_OK) return 0;
+    const size_t nblk = (size_t)((cache_cap + (long long)block - 1) / block);
+    return (size_t)cfg->B * cfg->H * nblk * 2 * cfg->d * sizeof(float);
+}
+
+rat_status rat_topk_build_stats(const rat_cfg *cfg, int block, int mode, const void *cache_k, int cache_cap,
+                                float *stats, rat_stream_t stream) {
+    rat_status st = check_topk(cfg, block, 0, mode, cache_cap);
+    if (st != RAT_OK) return st;
+    if (cfg->T < 0 || cfg->T > cache_cap) return fail(RAT_ERR_INVALID, "T %d outside [0, cache_cap]", cfg->T);
+    if ((size_t)cfg->B * cfg->T == 0) return RAT_OK;
+    CHECK_PTR(cache_k, "cache_k"); CHECK_PTR(stats, "stats");
+    TopkParams p = topk_params(cfg, block, 0, mode, cache_cap, stats);
+    p.cache[0] = const_cast<void *>(cache_k);
+    cudaError_t e = launch_topk_stats(p, cfg->T, cfg->dtype, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "top-k statistics launch");
+    return RAT_OK;
+}
+
+rat_status rat_topk_decode_step(const rat_cfg *cfg, int block, int topk, int mode, const void *q, const void *k,
+                                const void *v, const void *g, float *state_k, float *state_v, void *cache_k,
+                                void *cache_v, int cache_cap, float *stats, const int32_t *pos, void *o,
+                                float *lse, int32_t *sel, void *ws, size_t ws_bytes, rat_stream_t stream) {
+    rat_status st = check_topk(cfg, block, topk, mode, cache_cap);
     if (st != RAT_OK) return st;
     if (cfg->B == 0) return RAT_OK;
     CHECK_PTR(q, "q"); CHECK_PTR(k, "k"); CHECK_PTR(v, "v"); CHECK_PTR(g, "g");
     CHECK_PTR(state_k, "state_k"); CHECK_PTR(state_v, "state_v");
-    CHECK_PTR(cache_k, "cache_k"); CHECK_PTR(cache_v, "cache_v");
-    CHECK_PTR(pos, "pos"); CHECK_PTR(o, "o"); CHECK_OPT(lse, "lse");
-    if (cache_cap < 1) return fail(RAT_ERR_INVALID, "cache_cap %d < 1", cache_cap);
+    CHECK_PTR(cache_k, "cache_k"); CHECK_PTR(cache_v, "cache_v"); CHECK_PTR(stats, "stats");
+    CHECK_PTR(pos, "pos"); CHECK_PTR(o, "o"); CHECK_OPT(lse, "lse"); CHECK_OPT(sel, "sel");
     Layout L;
-    st = check_ws(cfg, RAT_OP_DECODE, cache_cap, ws, ws_bytes, &L);
+    st = check_ws(cfg, RAT_OP_TOPK_DECODE, cache_cap, ws, ws_bytes, &L);
     if (st != RAT_OK) return st;
-    DecodeParams p;
-    memset(&p, 0, sizeof(p));
-    decode_plan(cfg, cache_cap, &p);
+    TopkParams p = topk_params(cfg, block, topk, mode, cache_cap, stats);
     p.q = q; p.k = k; p.v = v; p.g = g;
     p.state[0] = state_k; p.state[1] = state_v;
     p.cache[0] = cache_k; p.cache[1] = cache_v;
-    p.pos = pos; p.o = o; p.lse = lse;
-    char *w = static_cast<char *>(ws);
-    p.part = reinterpret_cast<float *>(w + L.part);
-    const size_t part_bytes = align256((size_t)cfg->B * p.items_per_b * (cfg->d + 2) * sizeof(float));
-    p.counter = reinterpret_cast<int *>(w + L.part + part_bytes);
-    p.cap = cache_cap; p.B = cfg->B; p.H = cfg->H; p.d = cfg->d;
-    p.scale_log2 = scale_of(cfg) * 1.4426950408889634f;
+    p.pos = pos; p.o = o; p.lse = lse; p.sel = sel;
     p.hdr = reinterpret_cast<WsHeader *>(ws);
-    // per-(b,h) completion counters start from zero on every call
-    cudaError_t ez = cudaMemsetAsync(p.counter, 0, (size_t)cfg->B * cfg->H * sizeof(int), (cudaStream_t)stream);
-    if (ez != cudaSuccess) return cuda_fail(ez, "cudaMemsetAsync(decode counters)");
-    cudaError_t e = launch_decode(p, cfg->dtype, (cudaStream_t)stream);
-    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    cudaError_t e = launch_topk_decode(p, cfg->dtype, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "top-k decode launch");
     return RAT_OK;
 }
 

@@ -28,6 +28,15 @@
 // and lse; heads with one write o (bf16) and lse into scratch.  Launch 2
 // (window part): 256 consecutive positions against the key tiles covering
 // [t0-W+1, t0+255]; the epilogue merges with launch 1's (o, lse) by LSE.
+// Under the fixed-grid reading of dilation (query t attends to the keys
+// j <= t with j mod D == D-1, plus its own key) the dilated launch is replaced
+// by a grid launch: units are 256 consecutive positions against the key tiles
+// of the residue-(D-1) subsequence up to the last row's grid key, masked per
+// row; the epilogue adds the row's own key (when it is off the grid) by LSE,
+// scoring it from q and K~ in global memory.
+// With dedupe the window launch also masks, in every tile, the keys of the
+// row's dilated set (a periodic bit pattern per 32-column chunk), so a key in
+// both sets counts once.
 //
 // Every mbarrier wait is bounded (globaltimer); on expiry the CTA records
 // RAT_ERR_TIMEOUT, raises a shared abort flag, waits (bounded) for its own
@@ -194,8 +203,8 @@ __device__ __forceinline__ Unit decode_unit(const TcParams &p, long long u) {
     Unit out;
     out.cls = c;
     out.m = C.mtiles - 1 - (int)(rem % C.mtiles);
-    out.r = (int)(g % C.D);
-    g /= C.D;
+    out.r = (int)(g % C.nres);
+    g /= C.nres;
     out.h = p.heads[C.head0 + (int)(g % C.nheads)];
     out.b = (int)(g / C.nheads);
     return out;
@@ -209,18 +218,37 @@ struct Plan {
     bool valid[kSub];
 };
 
-__device__ __forceinline__ Plan make_plan(const TcParams &p, const Unit &u, int n) {
+// Where a unit's query rows sit in the key rows: a chunked prefill's queries
+// start at position t0, i.e. subsequence row t0 / D of the dilated part (t0 is
+// a multiple of D there) and position t0 of the window and grid parts.
+template <int kKind>
+__device__ __forceinline__ int query_offset(const TcParams &p, const TcClass &C) {
+    return kKind == kTcDilated ? p.t0 / C.D : p.t0;
+}
+
+template <int kKind>
+__device__ __forceinline__ Plan make_plan(const TcParams &p, const Unit &u) {
     Plan pl;
+    const TcClass &C = p.cls[u.cls];
+    const int n = C.n;
     const int q0 = 2 * BM * u.m;
     const int W = p.win[u.h];
+    const int qo = query_offset<kKind>(p, C);
     for (int i = 0; i < kSub; ++i) {
         const int qmin = q0 + BM * i;
         pl.valid[i] = qmin < n;
-        pl.hi[i] = qmin / BN;
-        if (!p.window_mode) {
+        const int qlast = qo + min(qmin + BM - 1, n - 1);   // the sub-tile's last row, in key units
+        if (kKind == kTcGrid) {
+            // grid keys g <= (t+1)/D - 1 for the sub-tile's last row t; a tile
+            // whose rows have no grid key yet keeps tile 0, fully masked
+            pl.hi[i] = max(0, ((qlast + 1) / C.D - 1) / BN);
+        } else {
+            pl.hi[i] = qlast / BN;
+        }
+        if (kKind != kTcWindow && kKind != kTcWindowDedupe) {
             pl.lo[i] = 0;
         } else {
-            const int first = qmin - W + 1;  // earliest key of the sub-tile's first row
+            const int first = qo + qmin - W + 1;  // earliest key of the sub-tile's first row
             pl.lo[i] = first > 0 ? first / BN : 0;
         }
     }
@@ -328,6 +356,87 @@ __device__ __forceinline__ float row_exp_s(uint32_t t_s, int lo, int lim, float 
     return ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
 }
 
+// Keys the dilated set already holds, for the window part with dedupe: in a
+// tile, key k is excluded when k == e0 (mod xd).  base has a bit at every
+// multiple of xd below 32 (one bit when xd > 32); e is the offset of the first
+// excluded key of the current 32-column chunk, d32 = 32 mod xd steps it on.
+struct Excl {
+    uint32_t base;
+    int d32, xd;
+};
+
+__device__ __forceinline__ Excl make_excl(int xd) {
+    Excl x;
+    x.xd = xd;
+    x.d32 = 32 % xd;
+    x.base = 0u;
+    for (int k = 0; k < 32; k += xd) x.base |= 1u << k;
+    return x;
+}
+
+__device__ __forceinline__ uint32_t excl_word(const Excl &x, int e) { return e < 32 ? x.base << e : 0u; }
+
+__device__ __forceinline__ int excl_next(const Excl &x, int e) {
+    e -= x.d32;
+    return e < 0 ? e + x.xd : e;
+}
+
+// row_max_s / row_exp_s with the masked test and the exclusion pattern
+// starting at offset e0 of the tile.
+__device__ __forceinline__ float row_max_x(uint32_t t_s, int lo, int lim, const Excl &x, int e0) {
+    float mx4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) mx4[k] = -INFINITY;
+    int e = e0;
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+        uint32_t sr[32];
+        tmem_ld32(t_s + 32 * q, sr);
+        const uint32_t xw = excl_word(x, e);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            float a = __uint_as_float(sr[2 * k]), b = __uint_as_float(sr[2 * k + 1]);
+            a = key_ok<2>(32 * q + 2 * k, lo, lim) && !((xw >> (2 * k)) & 1u) ? a : -INFINITY;
+            b = key_ok<2>(32 * q + 2 * k + 1, lo, lim) && !((xw >> (2 * k + 1)) & 1u) ? b : -INFINITY;
+            mx4[k & 3] = max3(mx4[k & 3], a, b);
+        }
+        e = excl_next(x, e);
+    }
+    return max3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+}
+
+__device__ __forceinline__ float row_exp_x(uint32_t t_s, int lo, int lim, const Excl &x, int e0, float c,
+                                           float m) {
+    uint64_t rs2[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) rs2[k] = f2_pack(0.f, 0.f);
+    const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m, -m);
+    int e = e0;
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+        uint32_t sr[32];
+        tmem_ld32(t_s + 32 * q, sr);
+        const uint32_t xw = excl_word(x, e);
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            float t0, t1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])), c2, nm2), t0, t1);
+            float e0_ = ex2(t0), e1_ = ex2(t1);
+            e0_ = key_ok<2>(32 * q + 2 * k, lo, lim) && !((xw >> (2 * k)) & 1u) ? e0_ : 0.f;
+            e1_ = key_ok<2>(32 * q + 2 * k + 1, lo, lim) && !((xw >> (2 * k + 1)) & 1u) ? e1_ : 0.f;
+            rs2[k & 3] = f2_add(rs2[k & 3], f2_pack(e0_, e1_));
+            pk[k] = pack_bf16(e0_, e1_);
+        }
+        tmem_st16(t_s + 16 * q, pk);
+        e = excl_next(x, e);
+    }
+    float r[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) f2_unpack(rs2[k], r[2 * k], r[2 * k + 1]);
+    return ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
+}
+
 template <int HD>
 struct Smem {
     static constexpr int kTile = BM * HD * 2;   // one 128-row tile of Q, K or V (bytes)
@@ -348,9 +457,12 @@ struct Smem {
 // for that warpgroup's next P, which it writes only after its epilogue has
 // read O_i (ordered by the tcgen05 fences around bar_pfull).  Unit tickets
 // reach the other roles through a 2-slot ring in shared memory.
-template <int HD, bool kWin>
+template <int HD, int kKind>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
     using L = Smem<HD>;
+    constexpr bool kWin = kKind == kTcWindow || kKind == kTcWindowDedupe;
+    constexpr bool kGrid = kKind == kTcGrid;
+    constexpr bool kDedupe = kKind == kTcWindowDedupe;
     constexpr int NCB = HD / 64;  // 64-column (128-byte) blocks of a head row
     extern __shared__ uint8_t dsmem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) & ~uintptr_t(1023));
@@ -411,11 +523,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 mbar_arrive(&bar_ufull[slot]);
                 if (un >= p.total_units) break;
                 const Unit u = decode_unit(p, un);
-                const Plan pl = make_plan(p, u, p.cls[u.cls].n);
+                const Plan pl = make_plan<kKind>(p, u);
                 const int ntiles = pl.jhi - pl.jlo + 1;
                 const CUtensorMap *mq = &p.tq[u.cls];
                 const CUtensorMap *mk = &p.tk[u.cls];
                 const CUtensorMap *mv = &p.tv[u.cls];
+                const int rk = u.r + p.cls[u.cls].kres;   // K/V residue coordinate
                 // Q of the previous unit has been read by its last QK
                 if (it >= 1 && !(ok = mbar_wait(&bar_qempty, (uint32_t)(it - 1) & 1u, &s_abort))) break;
                 const int nq = pl.valid[1] ? 2 : 1;
@@ -433,13 +546,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     mbar_expect_tx(&bar_kfull[st], L::kTile);
                     for (int cb = 0; cb < NCB; ++cb)
                         tma_load_5d(sbase + L::kK + st * L::kTile + cb * BN * 128, mk, &bar_kfull[st], cb * 64,
-                                    u.h, u.r, krow, u.b);
+                                    u.h, rk, krow, u.b);
                     ++nk;
                     if (nv >= 2 && !(ok = mbar_wait(&bar_vempty[st], ph ^ 1u, &s_abort))) break;
                     mbar_expect_tx(&bar_vfull[st], L::kTile);
                     for (int cb = 0; cb < NCB; ++cb)
                         tma_load_5d(sbase + L::kV + st * L::kTile + cb * BN * 128, mv, &bar_vfull[st], cb * 64,
-                                    u.h, u.r, krow, u.b);
+                                    u.h, rk, krow, u.b);
                     ++nv;
                 }
             }
@@ -498,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 mbar_arrive(&bar_uempty[slot]);
                 if (un >= p.total_units) break;
                 const Unit u = decode_unit(p, un);
-                const Plan pl = make_plan(p, u, p.cls[u.cls].n);
+                const Plan pl = make_plan<kKind>(p, u);
                 const int ntiles = pl.jhi - pl.jlo + 1;
                 ok = mbar_wait(&bar_q, (uint32_t)it & 1u, &s_abort);
                 if (ok) ok = mbar_wait(&bar_kfull[kv & 1], (uint32_t)(kv >> 1) & 1u, &s_abort);
@@ -577,12 +690,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (un >= p.total_units) break;
             const Unit u = decode_unit(p, un);
             const TcClass &C = p.cls[u.cls];
-            const Plan pl = make_plan(p, u, C.n);
+            const Plan pl = make_plan<kKind>(p, u);
             const int qmin = 2 * BM * u.m + BM * sub;                 // first row of the sub-tile
             const int qi = qmin + row;                                // subsequence row / position
             const int W = p.win[u.h];
+            const int qo = query_offset<kKind>(p, C);
             const int lo_s = sub ? pl.lo[1] : pl.lo[0];
             const int nt = (sub ? pl.valid[1] : pl.valid[0]) ? (sub ? pl.hi[1] : pl.hi[0]) - lo_s + 1 : 0;
+            Excl xcl;
+            if constexpr (kDedupe) xcl = make_excl(C.xd);
             float m_run = -INFINITY, l_run = 0.f;
             for (int c = 0; c < nt; ++c) {
                 const int j = lo_s + c;
@@ -590,16 +706,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 if (!ok) break;
                 ++n_s;
                 tc_fence_after();
-                // mask: causal on subsequence rows (dilated part); keys in (qi - W, qi] (window part)
+                // mask: causal on subsequence rows (dilated part); keys in (qi - W, qi] (window
+                // part); grid keys g <= (qi+1)/D - 1 (grid part)
                 const int ks = BN * j;
-                const bool full = !kWin ? (ks + BN - 1 <= qmin)
-                                                 : (ks + BN - 1 <= qmin && ks > qmin + BM - 1 - W);
-                // row limits in keys from the tile's first column
-                const int lim = qi - ks;            // key k valid iff k <= lim (both parts)
+                const int qa = qo + qi, qamin = qo + qmin;   // the row and the sub-tile's first, in key units
+                const bool full = kGrid ? (ks + BN - 1 <= (qamin + 1) / C.D - 1)
+                                  : !kWin ? (ks + BN - 1 <= qamin)
+                                          : (ks + BN - 1 <= qamin && ks > qamin + BM - 1 - W);
+                // row limits in keys from the tile's first column: key k valid iff k <= lim
+                const int lim = kGrid ? (qa + 1) / C.D - 1 - ks : qa - ks;
                 // window part: and k > lo (no lower limit in the dilated part)
-                const int lo = kWin ? qi - W - ks : INT_MIN / 2;
+                const int lo = kWin ? qa - W - ks : INT_MIN / 2;
                 const int mode = full ? 0 : 2;
-                const float mraw = mode == 0 ? row_max_s<0>(t_s, lo, lim) : row_max_s<2>(t_s, lo, lim);
+                // dedupe: the dilated set's keys in this tile are k == e0 (mod xd):
+                // k == lim for the residue reading (the row's own key among them);
+                // the grid positions ks + k == xd - 1 (mod xd) for the fixed grid,
+                // whose own key leaves through the limit instead
+                int e0 = 0, limx = lim;
+                if constexpr (kDedupe) {
+                    const int r0 = p.grid ? (C.xd - 1 - ks) % C.xd : lim % C.xd;
+                    e0 = r0 < 0 ? r0 + C.xd : r0;
+                    if (p.grid) limx = lim - 1;
+                }
+                float mraw;
+                if constexpr (kDedupe) mraw = row_max_x(t_s, lo, limx, xcl, e0);
+                else mraw = mode == 0 ? row_max_s<0>(t_s, lo, lim) : row_max_s<2>(t_s, lo, lim);
                 const float mx = mraw * p.scale_log2;   // scale > 0 commutes with max
                 // running max with lazy rescale: keep the stale max unless the new
                 // one exceeds it by more than 8 (P stays <= 2^8)
@@ -626,8 +757,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                         }
                     }
                 }
-                const float rs = mode == 0 ? row_exp_s<0>(t_s, lo, lim, p.scale_log2, m_use)
-                                           : row_exp_s<2>(t_s, lo, lim, p.scale_log2, m_use);
+                float rs;
+                if constexpr (kDedupe) rs = row_exp_x(t_s, lo, limx, xcl, e0, p.scale_log2, m_use);
+                else rs = mode == 0 ? row_exp_s<0>(t_s, lo, lim, p.scale_log2, m_use)
+                                    : row_exp_s<2>(t_s, lo, lim, p.scale_log2, m_use);
                 l_run = l_run * alpha + rs;
                 m_run = m_new;
                 tc_fence_before();
@@ -637,20 +770,51 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (!ok) break;
             if (nt > 0) {
                 const bool valid_row = qi < C.n;
-                const long long t = kWin ? (long long)qi : (long long)u.r + (long long)C.D * qi;
+                const long long t = kKind != kTcDilated ? (long long)qi : (long long)u.r + (long long)C.D * qi;
                 const size_t orow = (((size_t)u.b * p.T + (size_t)t) * p.H + u.h) * HD;
                 const size_t lrow = ((size_t)u.b * p.H + u.h) * p.T + (size_t)t;
                 __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.o);
-                constexpr bool merge = kWin;
-                // The window launch merges with the dilated part's row (o, lse),
-                // written by the previous launch: fetch it while the last PV runs.
+                constexpr bool merge = kWin || kGrid;
+                // The row's other part, merged by LSE: for the window launch the
+                // dilated part's row (o, lse) written by the previous launch; for
+                // the grid launch the row's own key (V~_t, score s q_t.K~_t) when
+                // t is off the grid.  Fetched while the last PV runs.
+                const bool mrow = merge && valid_row && (!kGrid || (p.t0 + t) % C.D != C.D - 1);
                 uint4 prev[HD / 8];
                 float ld2 = 0.f;
-                if (merge && valid_row) {
-                    const uint4 *src = reinterpret_cast<const uint4 *>(o + orow);
+                if (mrow) {
+                    if constexpr (kGrid) {
+                        const uint4 *qs = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.q) + orow);
+                        // the row's own key and value: row t0 + t of the [B, t0+T, H, d] history
+                        const size_t hrow = (((size_t)u.b * p.Th + (size_t)(p.t0 + t)) * p.H + u.h) * HD;
+                        const uint4 *ks4 =
+                            reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.kself[u.cls]) + hrow);
+                        const uint4 *vs4 =
+                            reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.vself[u.cls]) + hrow);
+                        float z = 0.f;
 #pragma unroll
-                    for (int q = 0; q < HD / 8; ++q) prev[q] = src[q];
-                    ld2 = p.lse_dil[lrow] * 1.4426950408889634f;
+                        for (int q = 0; q < HD / 8; ++q) {
+                            const uint4 a = qs[q], k4 = ks4[q];
+                            const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, kw[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&aw[i]));
+                                const float2 fk = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kw[i]));
+                                z = fmaf(fa.x, fk.x, z);
+                                z = fmaf(fa.y, fk.y, z);
+                            }
+                            prev[q] = vs4[q];
+                        }
+                        ld2 = z * p.scale_log2;
+                    } else {
+                        const uint4 *src = reinterpret_cast<const uint4 *>(o + orow);
+#pragma unroll
+                        for (int q = 0; q < HD / 8; ++q) prev[q] = src[q];
+                        ld2 = p.lse_dil[lrow] * 1.4426950408889634f;
+                    }
+                } else if constexpr (merge) {
+#pragma unroll
+                    for (int q = 0; q < HD / 8; ++q) prev[q] = make_uint4(0u, 0u, 0u, 0u);
                 }
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar_pvdone[sub], (uint32_t)n_pv & 1u, &s_abort));
                 if (!ok) break;
@@ -659,9 +823,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 // ---- epilogue: o = O / l, lse = ln(2) * (m + log2 l)
                 const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
                 float lse2 = l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY;  // log2 domain
+                // weights of this launch's part (w_self) and of the other part (w_dil)
                 float w_self = 1.f, w_dil = 0.f;
-                if (merge && valid_row) {
-                    // merge with the dilated part: weights e^(lse_i - max) / sum
+                if (mrow) {
+                    // merge with the other part: weights e^(lse_i - max) / sum
                     const float mm = fmaxf(ld2, lse2);
                     const float e1 = ex2(ld2 - mm), e2 = ex2(lse2 - mm);
                     w_dil = e1 / (e1 + e2);
@@ -745,7 +910,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 }
                 if (valid_row) {
                     const float lse = lse2 * 0.69314718055994531f;
-                    if (!merge && p.win[u.h] > 0) p.lse_dil[lrow] = lse;  // the window launch merges later
+                    if (!kWin && p.win[u.h] > 0) p.lse_dil[lrow] = lse;  // the window launch merges later
                     else if (p.lse_user) p.lse_user[lrow] = lse;
                 }
             }
@@ -789,12 +954,12 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int H, int d, int D, int box_rows) {
+bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int Ts, int H, int d, int D, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn || D < 1 || T % D != 0) return false;
     const cuuint64_t e = 2;  // bf16
     const cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)D, (cuuint64_t)(T / D), (cuuint64_t)B};
-    const cuuint64_t strides[4] = {e * d, e * d * H, e * d * H * D, e * d * H * T};
+    const cuuint64_t strides[4] = {e * d, e * d * H, e * d * H * D, e * d * H * Ts};
     const cuuint32_t box[5] = {64, 1, 1, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
@@ -804,12 +969,13 @@ bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int H, int 
 
 // One CTA per SM: each CTA allocates all 512 TMEM columns, so the d = 64
 // variant also asks for more than half of the shared memory.
-bool encode_map_tokens(CUtensorMap *map, const void *base, int dtype, int B, int T, int H, int d, int box_rows) {
+bool encode_map_tokens(CUtensorMap *map, const void *base, int dtype, int B, int T, int Ts, int H, int d,
+                       int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t e = dtype == RAT_BF16 ? 2 : 4;
     const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {e * d, e * d * H, e * d * H * T};
+    const cuuint64_t strides[3] = {e * d, e * d * H, e * d * H * Ts};
     const cuuint32_t box[4] = {(cuuint32_t)d, 1, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(map, dtype == RAT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
@@ -823,13 +989,23 @@ size_t attn_tc_smem_bytes(int hd) {
     return need > 120 * 1024 ? need : 120 * 1024;
 }
 
-template <int HD, bool kWin>
+template <int HD, int kKind>
 cudaError_t launch_inst(const TcParams &p, unsigned grid, size_t smem, cudaStream_t s) {
     static std::atomic<unsigned long long> smem_set{0};
-    cudaError_t e = ensure_smem_limit(attn_tc_kernel<HD, kWin>, smem, smem_set);
+    cudaError_t e = ensure_smem_limit(attn_tc_kernel<HD, kKind>, smem, smem_set);
     if (e != cudaSuccess) return e;
-    attn_tc_kernel<HD, kWin><<<grid, kThreads, smem, s>>>(p);
+    attn_tc_kernel<HD, kKind><<<grid, kThreads, smem, s>>>(p);
     return cudaSuccess;
+}
+
+template <int HD>
+cudaError_t launch_kind(const TcParams &p, unsigned grid, size_t smem, cudaStream_t s) {
+    switch (p.kind) {
+    case kTcWindow: return launch_inst<HD, kTcWindow>(p, grid, smem, s);
+    case kTcGrid: return launch_inst<HD, kTcGrid>(p, grid, smem, s);
+    case kTcWindowDedupe: return launch_inst<HD, kTcWindowDedupe>(p, grid, smem, s);
+    default: return launch_inst<HD, kTcDilated>(p, grid, smem, s);
+    }
 }
 
 cudaError_t launch_attn_tc(const TcParams &p, int hd, cudaStream_t s) {
@@ -841,10 +1017,9 @@ cudaError_t launch_attn_tc(const TcParams &p, int hd, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM (the shared memory and TMEM of one CTA fill an SM)
     const unsigned grid = (unsigned)std::min<long long>(p.total_units, (long long)nsm);
-    // the dilated and window launches are separate instantiations, so each
-    // carries only its own epilogue and masks (instruction-cache footprint)
-    if (hd == 128) e = p.window_mode ? launch_inst<128, true>(p, grid, smem, s) : launch_inst<128, false>(p, grid, smem, s);
-    else e = p.window_mode ? launch_inst<64, true>(p, grid, smem, s) : launch_inst<64, false>(p, grid, smem, s);
+    // each launch kind is its own instantiation, carrying only its own
+    // epilogue and masks (instruction-cache footprint)
+    e = hd == 128 ? launch_kind<128>(p, grid, smem, s) : launch_kind<64>(p, grid, smem, s);
     if (e != cudaSuccess) return e;
     count_launches(1);
     return cudaGetLastError();

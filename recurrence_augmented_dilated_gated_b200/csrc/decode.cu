@@ -7,6 +7,13 @@
 //   s <- a*s + (1-a)*x (x = k, v; a = sigmoid(g), a = 0 without recurrence),
 //   the new augmented row is stored at cache row (t mod D)*S + t/D,
 //   o = softmax over the multiset  { j <= t, j == t mod D }  (+)  { t-W+1..t }.
+// Under the fixed-grid reading the dilated set is { j < t, j mod D == D-1 }
+// plus t, the slab is the grid (rows 0 .. t/D - 1, the same count), the new
+// row is stored at its grid row only when t is on the grid, and the window
+// rows come from a ring of the last W positions (D > 1).  A paged cache
+// (kPaged) keeps the same logical rows in pages named by a page table; the
+// ring's bulk copies split where a run of rows crosses a page.  With dedupe the
+// window part skips the keys of the dilated set, the new row among them.
 // Softmaxes over disjoint pieces of a key multiset combine exactly by
 // log-sum-exp, so the step is split into independent work items:
 //   * item i of (b, h) streams its run of old rows of the residue slab
@@ -131,13 +138,15 @@ struct Acc8 {
     float m, l, o[8];
 };
 
-// Adds the first n <= NB keys (scores s[], values v[][]) in one rescale;
-// fully unrolled and predicated so the arrays stay in registers.
+// Adds the first n <= NB keys (scores s[], values v[][]) in one rescale,
+// leaving out key u when bit u of `skip` is set; fully unrolled and predicated
+// so the arrays stay in registers.
 template <int NB>
-__device__ __forceinline__ void acc_add_batch(Acc8 &a, const float *s, const float (*v)[8], int n) {
+__device__ __forceinline__ void acc_add_batch(Acc8 &a, const float *s, const float (*v)[8], int n,
+                                              unsigned skip = 0u) {
     float mb = -INFINITY;
 #pragma unroll
-    for (int u = 0; u < NB; ++u) mb = u < n ? fmaxf(mb, s[u]) : mb;
+    for (int u = 0; u < NB; ++u) mb = (u < n && !((skip >> u) & 1u)) ? fmaxf(mb, s[u]) : mb;
     const float mn = fmaxf(a.m, mb);
     const float corr = a.m == -INFINITY ? 0.f : exp2f(a.m - mn);
     a.l *= corr;
@@ -145,7 +154,7 @@ __device__ __forceinline__ void acc_add_batch(Acc8 &a, const float *s, const flo
     for (int i = 0; i < 8; ++i) a.o[i] *= corr;
 #pragma unroll
     for (int u = 0; u < NB; ++u) {
-        const float pj = u < n ? exp2f(s[u] - mn) : 0.f;
+        const float pj = (u < n && !((skip >> u) & 1u)) ? exp2f(s[u] - mn) : 0.f;
         a.l += pj;
 #pragma unroll
         for (int i = 0; i < 8; ++i) a.o[i] += pj * v[u][i];
@@ -153,7 +162,7 @@ __device__ __forceinline__ void acc_add_batch(Acc8 &a, const float *s, const flo
     a.m = mn;
 }
 
-template <typename T, int D>
+template <typename T, int D, bool kPaged>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) {
     constexpr int LPR = D / 8;                 // lanes per cache row (8 channels each)
     constexpr int NG = kCompute / LPR;         // row groups
@@ -182,13 +191,38 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     const int Dh = p.dil[h], W = p.win[h];
     const long long S = p.slab[h];
     const int r = valid_pos ? t % Dh : 0;
-    const int n_old = valid_pos ? t / Dh : 0;    // old rows of the residue slab
+    const int n_old = valid_pos ? t / Dh : 0;    // old rows of the residue slab (or grid)
+    const size_t slab0 = p.grid ? 0 : (size_t)r * S;   // first cache row of the slab
     const int i0 = li * p.rows_per_item[h];      // this item's run of old rows: [i0, i1)
     const int i1 = min(i0 + p.rows_per_item[h], n_old);
     const int nrows = max(0, i1 - i0);
     const int nst = (nrows + RS - 1) / RS;       // ring stages this item streams
-    const T *ck = static_cast<const T *>(p.cache[0]) + bh * (size_t)p.cache_R * D;
-    const T *cv = static_cast<const T *>(p.cache[1]) + bh * (size_t)p.cache_R * D;
+    const T *ck = static_cast<const T *>(p.cache[0]);   // cache bases: rows at row_off(row)
+    const T *cv = static_cast<const T *>(p.cache[1]);
+    // element offset of logical cache row `row` of (b, h); -1 for a page the
+    // table does not name validly
+    auto row_off = [&](long long row) -> long long {
+        if (kPaged) return cache_offset(p.page_table, p.pps, p.page_rows, p.num_pages, p.cache_R, p.H, D, b, h, row);
+        return ((long long)bh * p.cache_R + row) * D;
+    };
+    // a paged cache: every page the step of (b, h) touches must be valid, else
+    // the pair is skipped (o = 0) and reported like an invalid position.  Every
+    // item checks the pages of the whole step, so all items of (b, h) agree.
+    int bad = 0;
+    if (kPaged && valid_pos) {
+        if (n_old > 0)
+            for (long long pg = (long long)slab0 / p.page_rows + tid;
+                 pg <= (long long)(slab0 + n_old - 1) / p.page_rows; pg += kThreads)
+                bad |= row_off(pg * p.page_rows) < 0;
+        long long ra, rb;
+        cache_rows_of(t, Dh, W, S, p.grid, ra, rb);
+        if (tid == 0) bad |= (ra >= 0 && row_off(ra) < 0) || (rb >= 0 && row_off(rb) < 0);
+        if (W > 0)
+            for (int jj = max(0, t - W + 1) + tid; jj < t; jj += kThreads) {
+                cache_rows_of(jj, Dh, W, S, p.grid, ra, rb);
+                bad |= row_off(rb >= 0 ? rb : ra) < 0;
+            }
+    }
 
     if (tid == 0) {
         s_abort = 0;
@@ -200,7 +234,9 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         if (!valid_pos) report_error(p.hdr, RAT_ERR_INVALID, b);
     }
-    __syncthreads();
+    bad = __syncthreads_or(bad);
+    const bool valid = valid_pos && !bad;
+    if (tid == 0 && valid_pos && bad) report_error(p.hdr, RAT_ERR_INVALID, b);
 
     Acc8 acc;
     acc.m = -INFINITY;
@@ -212,9 +248,9 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     if (warp == kCompute / 32) {
         // ------------------------------------------------ producer: stream the
         // item's contiguous run of K~ and V~ rows through the ring
-        if ((tid & 31) == 0 && valid_pos) {
-            const char *kb = reinterpret_cast<const char *>(ck + ((size_t)r * S + i0) * D);
-            const char *vb = reinterpret_cast<const char *>(cv + ((size_t)r * S + i0) * D);
+        if ((tid & 31) == 0 && valid) {
+            const char *kb = reinterpret_cast<const char *>(ck + (kPaged ? 0 : row_off(slab0 + i0)));
+            const char *vb = reinterpret_cast<const char *>(cv + (kPaged ? 0 : row_off(slab0 + i0)));
             int sidx = 0;
             bool ok = true;
             for (; sidx < nst; ++sidx) {
@@ -232,14 +268,34 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                 const size_t off = (size_t)sidx * RS * kRowBytes;
                 asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full), "r"(2 * bytes)
                              : "memory");
-                asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                                 dk),
-                             "l"(kb + off), "r"(bytes), "r"(full)
-                             : "memory");
-                asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                                 dv),
-                             "l"(vb + off), "r"(bytes), "r"(full)
-                             : "memory");
+                if (!kPaged) {
+                    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                                     dk),
+                                 "l"(kb + off), "r"(bytes), "r"(full)
+                                 : "memory");
+                    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                                     dv),
+                                 "l"(vb + off), "r"(bytes), "r"(full)
+                                 : "memory");
+                } else {
+                    // one copy per page the stage's rows touch (all validated above)
+                    const long long ra = (long long)(slab0 + i0) + (long long)sidx * RS;
+                    for (int done = 0; done < nr;) {
+                        const long long row = ra + done;
+                        const int n = (int)min((long long)(nr - done), (long long)p.page_rows - row % p.page_rows);
+                        const long long ofs = row_off(row);
+                        const uint32_t nb = (uint32_t)n * kRowBytes, so = (uint32_t)done * kRowBytes;
+                        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                                         dk + so),
+                                     "l"(ck + ofs), "r"(nb), "r"(full)
+                                     : "memory");
+                        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                                         dv + so),
+                                     "l"(cv + ofs), "r"(nb), "r"(full)
+                                     : "memory");
+                        done += n;
+                    }
+                }
             }
             if (!ok) {
                 s_abort = 1;
@@ -249,7 +305,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                     mbar_wait(smem_u32(&s_full[q % kStages]), (uint32_t)(q / kStages) & 1u, &never);
             }
         }
-    } else if (valid_pos) {
+    } else if (valid) {
         // ------------------------------------------------ scoring warps
         const unsigned gmask = group_mask<LPR>();
         float q[8];
@@ -261,12 +317,16 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         // loaded now and used after the old rows, so their latency overlaps
         // the stream (channel tid; kCompute >= D)
         static_assert(kCompute >= D, "one channel per scoring thread");
-        float in_k = 0.f, in_v = 0.f, in_g = 0.f, st_k = 0.f, st_v = 0.f;
+        float in_k = 0.f, in_v = 0.f, in_g = 0.f, in_gv = 0.f, st_k = 0.f, st_v = 0.f;
         const size_t e_new = bh * D + tid;
         if (last && tid < D) {
             in_k = (float)static_cast<const T *>(p.k)[e_new];
             in_v = (float)static_cast<const T *>(p.v)[e_new];
-            if (p.recur[h]) in_g = (float)static_cast<const T *>(p.g)[e_new];
+            if (p.recur[h]) {
+                in_g = (float)static_cast<const T *>(p.g)[e_new];
+                // separate gates: the value gate is the second [B,H,d] tensor
+                in_gv = p.sep ? (float)static_cast<const T *>(p.g)[(size_t)p.B * p.H * D + e_new] : in_g;
+            }
             st_k = p.state[0][e_new];
             st_v = p.state[1][e_new];
         }
@@ -313,20 +373,37 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         if (last) {
             // step update and append of the new row (no item reads it this step)
             if (tid < D) {
-                float a = 0.f, oma = 1.f;
+                float a = 0.f, oma = 1.f, av = 0.f, omav = 1.f;
                 if (p.recur[h]) {
                     const float gl_ = fminf(fmaxf(in_g, -80.f), 80.f);
                     const float ex = expf(-gl_);
                     a = 1.f / (1.f + ex);
                     oma = ex * a;
+                    av = a;
+                    omav = oma;
+                    if (p.sep) {
+                        const float gv_ = fminf(fmaxf(in_gv, -80.f), 80.f);
+                        const float exv = expf(-gv_);
+                        av = 1.f / (1.f + exv);
+                        omav = exv * av;
+                    }
                 }
                 const float sk = a * st_k + oma * in_k;
-                const float sv = a * st_v + oma * in_v;
+                const float sv = av * st_v + omav * in_v;
                 p.state[0][e_new] = sk;
                 p.state[1][e_new] = sv;
-                const size_t row = (size_t)r * S + n_old;
-                static_cast<T *>(p.cache[0])[bh * (size_t)p.cache_R * D + row * D + tid] = to_t<T>(sk);
-                static_cast<T *>(p.cache[1])[bh * (size_t)p.cache_R * D + row * D + tid] = to_t<T>(sv);
+                long long row0, row1;
+                cache_rows_of(t, Dh, W, S, p.grid, row0, row1);
+                T *dk = static_cast<T *>(p.cache[0]) + tid;
+                T *dv = static_cast<T *>(p.cache[1]) + tid;
+                if (row0 >= 0) {
+                    dk[row_off(row0)] = to_t<T>(sk);
+                    dv[row_off(row0)] = to_t<T>(sv);
+                }
+                if (row1 >= 0) {  // the ring slot of t - W, which no window needs any more
+                    dk[row_off(row1)] = to_t<T>(sk);
+                    dv[row_off(row1)] = to_t<T>(sv);
+                }
                 s_new[0][tid] = round_to<T>(sk);
                 s_new[1][tid] = round_to<T>(sv);
             }
@@ -337,13 +414,17 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                 for (int j = j0 + grp * kBatch; j < t; j += NG * kBatch) {
                     float kf[kBatch][8], vf[kBatch][8], sc[kBatch];
                     const int n = min(kBatch, t - j);
+                    unsigned skip = 0u;
 #pragma unroll
                     for (int u = 0; u < kBatch; ++u) {
                         if (u < n) {
                             const int jj = j + u;
-                            const size_t row = (size_t)(jj % Dh) * S + (size_t)(jj / Dh);
-                            IO8<T>::load(ck + row * D + c0, kf[u]);
-                            IO8<T>::load(cv + row * D + c0, vf[u]);
+                            if (p.dedupe && (p.grid ? jj % Dh == Dh - 1 : (t - jj) % Dh == 0)) skip |= 1u << u;
+                            long long row0, row1;
+                            cache_rows_of(jj, Dh, W, S, p.grid, row0, row1);
+                            const long long ofs = row_off(row1 >= 0 ? row1 : row0);
+                            IO8<T>::load(ck + ofs + c0, kf[u]);
+                            IO8<T>::load(cv + ofs + c0, vf[u]);
                         } else {
 #pragma unroll
                             for (int c = 0; c < 8; ++c) kf[u][c] = vf[u][c] = 0.f;
@@ -356,10 +437,11 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                         for (int c = 0; c < 8; ++c) s2 += q[c] * kf[u][c];
                         sc[u] = group_sum<LPR>(s2, gmask);
                     }
-                    acc_add_batch<kBatch>(acc, sc, vf, n);
+                    acc_add_batch<kBatch>(acc, sc, vf, n, skip);
                 }
             }
             // the new row: once in the dilated set, once more in the window
+            // (not with dedupe)
             if (grp == 0) {
                 float kv[2][8], sc[2];
 #pragma unroll
@@ -373,7 +455,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                 s2 = group_sum<LPR>(s2, gmask);
                 sc[0] = s2;
                 sc[1] = s2;
-                acc_add_batch<2>(acc, sc, kv, W > 0 ? 2 : 1);
+                acc_add_batch<2>(acc, sc, kv, W > 0 && !p.dedupe ? 2 : 1);
             }
         }
     }
@@ -452,15 +534,20 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     if (tid == 0) p.counter[bh] = 0;  // ready for the next step
 }
 
-template <typename T, int D>
-cudaError_t launch_typed(const DecodeParams &p, unsigned grid, cudaStream_t s) {
+template <typename T, int D, bool kPaged>
+cudaError_t launch_form(const DecodeParams &p, unsigned grid, cudaStream_t s) {
     constexpr int RS = (kCompute / (D / 8)) * kBatch;
     const size_t smem = (size_t)kStages * 2 * RS * D * sizeof(T);
     static std::atomic<unsigned long long> smem_set{0};
-    cudaError_t e = ensure_smem_limit(decode_kernel<T, D>, smem, smem_set);
+    cudaError_t e = ensure_smem_limit(decode_kernel<T, D, kPaged>, smem, smem_set);
     if (e != cudaSuccess) return e;
-    decode_kernel<T, D><<<grid, kThreads, smem, s>>>(p);
+    decode_kernel<T, D, kPaged><<<grid, kThreads, smem, s>>>(p);
     return cudaSuccess;
+}
+
+template <typename T, int D>
+cudaError_t launch_typed(const DecodeParams &p, unsigned grid, cudaStream_t s) {
+    return p.page_table ? launch_form<T, D, true>(p, grid, s) : launch_form<T, D, false>(p, grid, s);
 }
 
 }  // namespace
@@ -486,15 +573,21 @@ size_t decode_plan(const rat_cfg *c, int cap, DecodeParams *p) {
         const int ns = (slab + target - 1) / target;
         const int n = ns > 0 ? ns : 1;
         p->dil[h] = D;
-        p->win[h] = c->win[h];
+        // with dedupe a D = 1 head's window keys are all in its dilated set
+        p->win[h] = (c->flags & RAT_FLAG_DEDUPE) && D == 1 ? 0 : c->win[h];
         p->slab[h] = slab;
         p->nsplit[h] = n;
         p->rows_per_item[h] = (slab + n - 1) / n;   // balanced runs
         p->item0[h] = items;
         p->recur[h] = (c->recur == nullptr || c->recur[h] != 0) ? 1 : 0;
         items += n;
-        R = R > (long long)D * slab ? R : (long long)D * slab;
+        const bool grid = (c->flags & RAT_FLAG_GRID_DILATION) != 0;
+        const long long rows = grid ? (long long)slab + (D > 1 ? c->win[h] : 0) : (long long)D * slab;
+        R = R > rows ? R : rows;
     }
+    p->grid = (c->flags & RAT_FLAG_GRID_DILATION) ? 1 : 0;
+    p->dedupe = (c->flags & RAT_FLAG_DEDUPE) ? 1 : 0;
+    p->sep = (c->flags & RAT_FLAG_SEPARATE_GATES) ? 1 : 0;
     p->item0[c->H] = items;
     p->items_per_b = items;
     p->cache_R = R;

@@ -92,6 +92,33 @@ __device__ __forceinline__ float f4get(const float4 &v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
+// Decode-cache rows of position j for a head with dilation D, window W and
+// S = ceil(cap / D) (layout in include/rat.h).  Residue-major: one row.  Fixed
+// grid: the grid row when j is on the grid (j mod D == D - 1), and the window
+// ring row when the head keeps a ring (D > 1, W > 0); -1 where there is none.
+__host__ __device__ __forceinline__ void cache_rows_of(long long j, int D, int W, long long S, int grid,
+                                                       long long &grid_row, long long &ring_row) {
+    if (!grid) {
+        grid_row = (j % D) * S + j / D;
+        ring_row = -1;
+        return;
+    }
+    grid_row = (j % D == D - 1) ? j / D : -1;
+    ring_row = (D > 1 && W > 0) ? S + j % W : -1;
+}
+
+// Element offset of (logical row `row`, channel 0) of (b, h) in a cache: the
+// dense [B,H,R,d] block, or the page the table names ([num_pages,H,P,d]); -1
+// when the table names no valid page.
+__host__ __device__ __forceinline__ long long cache_offset(const int *table, int pps, int page_rows, int num_pages,
+                                                           long long cache_R, int H, int d, int b, int h,
+                                                           long long row) {
+    if (!table) return (((long long)b * H + h) * cache_R + row) * d;
+    const int pg = table[(long long)b * pps + row / page_rows];
+    if (pg < 0 || pg >= num_pages) return -1;
+    return (((long long)pg * H + h) * page_rows + row % page_rows) * d;
+}
+
 // --------------------------------------------------------------- scan (K1)
 struct ScanParams {
     // 4-D TMA maps (d, H, T, B) of k, v, g (loads) and kt, vt (stores), box
@@ -106,6 +133,11 @@ struct ScanParams {
     void *cache[2];         // decode cache [B,H,R,d] or null
     long long cache_R;      // rows per (b,h) cache block
     int cap;
+    int grid;               // cache layout of the fixed-grid reading (grid rows + window ring)
+    int one;                // one-tensor form: x[0], g -> out[0] (separate gates, run per tensor)
+    int t0;                 // position of the call's first token: out rows and cache positions are t0 + t
+    const int *page_table;  // paged cache (null: dense), as DecodeParams
+    int page_rows, pps, num_pages;
     int B, T, H, d;
     int nslices;            // B * nheads
     int nchunks;            // chunks along T per slice
@@ -114,6 +146,7 @@ struct ScanParams {
     unsigned char head_list[kMaxHeads];
     unsigned char head_recur[kMaxHeads];
     int head_dil[kMaxHeads];
+    int head_win[kMaxHeads];
     unsigned int *ticket;   // dynamic chunk ticket counter (zeroed per launch)
     int *flags;             // [nslices * nchunks] 0 none, 1 aggregate, 2 inclusive
     float *agg;             // [nslices * nchunks][3][d]  (A, b_k, b_v)
@@ -130,6 +163,10 @@ struct AttnParams {
     float *lse;             // [B,H,T] or null
     int B, T, H, d;
     float scale_log2;       // scale * log2(e)
+    int t0;                 // chunked prefill: rows are positions t0 + t; kt/vt hold t0 + T rows
+    int Th;                 // rows per batch entry of kt/vt
+    int grid;               // fixed-grid reading of dilation
+    int dedupe;             // the window part skips the dilated set's keys
     int dil[kMaxHeads];
     int win[kMaxHeads];
     unsigned char use_raw[kMaxHeads];
@@ -150,6 +187,13 @@ struct DecodeParams {
     long long cache_R;
     int cap, B, H, d;
     int items_per_b;             // sum over heads of nsplit
+    int grid;                    // fixed-grid reading and its cache layout
+    int dedupe;                  // the window part skips the dilated set's keys
+    int sep;                     // separate key and value gates: g is [2,B,H,d]
+    // paged cache (null table: one dense [B,H,R,d] block): logical row r of
+    // (b, h) at page table[b * pps + r / page_rows], [num_pages, H, page_rows, d]
+    const int *page_table;
+    int page_rows, pps, num_pages;
     float scale_log2;
     int dil[kMaxHeads];
     int win[kMaxHeads];
@@ -157,6 +201,28 @@ struct DecodeParams {
     int nsplit[kMaxHeads];       // work items of head h (the last also does the step update)
     int rows_per_item[kMaxHeads];// slab rows per work item
     int item0[kMaxHeads + 1];    // first item of head h within a batch entry
+    unsigned char recur[kMaxHeads];
+    WsHeader *hdr;
+};
+
+// -------------------------------------------------- top-k block decode (K6)
+constexpr int kTopkMaxK = 64;          // selected blocks per query, at most
+constexpr int kTopkMaxBlocks = 16384;  // blocks of one (b, h) cache, at most (scores in shared memory)
+
+struct TopkParams {
+    const void *q, *k, *v, *g;   // [B,H,d]
+    float *state[2];             // [B,H,d] fp32, in place
+    void *cache[2];              // [B,H,R,d], dense layout: position j at row j
+    float *stats;                // [B,H,nblk,2,d] fp32 block statistics
+    const int *pos;              // device [B]
+    void *o;                     // [B,H,d]
+    float *lse;                  // [B,H] or null
+    int *sel;                    // [B,H,K] selected blocks or null
+    long long cache_R;
+    int cap, B, H, d;
+    int bs, K, mode, nblk;       // block size, blocks to select, RAT_TOPK_*, ceil(cap / bs)
+    int sep;                     // separate key and value gates: g is [2,B,H,d]
+    float scale_log2;
     unsigned char recur[kMaxHeads];
     WsHeader *hdr;
 };
@@ -176,11 +242,16 @@ rat_status set_last_error(rat_status s, const char *msg);
 cudaError_t launch_scan(const ScanParams &p, int dtype, cudaStream_t s);
 // tokens per scan chunk for head dimension d
 int scan_chunk_tokens(int d);
-// 4-D TMA map (d, H, T, B) of a [B,T,H,d] tensor, box (d, 1, box_rows, 1), no swizzle
-bool encode_map_tokens(CUtensorMap *map, const void *base, int dtype, int B, int T, int H, int d, int box_rows);
+// 4-D TMA map (d, H, T, B) of the first T rows of a [B,Ts,H,d] tensor (Ts rows
+// per batch entry), box (d, 1, box_rows, 1), no swizzle
+bool encode_map_tokens(CUtensorMap *map, const void *base, int dtype, int B, int T, int Ts, int H, int d,
+                       int box_rows);
 // final state of the heads in p.head_list, which have no recurrence
 cudaError_t launch_final_of_plain_heads(const ScanParams &p, int dtype, cudaStream_t s);
 cudaError_t launch_attn_simt(const AttnParams &p, int dtype, cudaStream_t s);
 cudaError_t launch_decode(const DecodeParams &p, int dtype, cudaStream_t s);
+// block statistics of positions [0, n_tok) of the cache
+cudaError_t launch_topk_stats(const TopkParams &p, int n_tok, int dtype, cudaStream_t s);
+cudaError_t launch_topk_decode(const TopkParams &p, int dtype, cudaStream_t s);
 
 }  // namespace rat

@@ -25,6 +25,9 @@
 //     overwriting k and v in shared memory with K~ and V~, which two TMA
 //     stores write back (and decode-cache rows are written directly).
 // HBM traffic is the algorithmic 3 reads + 2 writes per (token, channel).
+// With separate gates for keys and values the scan runs twice in its
+// one-tensor form (kOne: x and g in, x~ out), once per tensor: 2 reads and 1
+// write each, again the algorithmic traffic.
 // Every wait is bounded by the workspace's spin limit; on expiry the CTA
 // records RAT_ERR_TIMEOUT, continues from a zero state and still publishes, so
 // no successor waits forever.
@@ -130,7 +133,7 @@ template <> struct Smem4<float> {
     static __device__ __forceinline__ void store(float *p, float4 v) { IO4<float>::store(p, v); }
 };
 
-template <typename T, int D>
+template <typename T, int D, bool kOne>
 __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ ScanParams p) {
     constexpr int LPR = D / 4;             // threads per token row (4 channels each)
     constexpr int G = kThreads / LPR;      // thread groups (sub-chunks) per CTA
@@ -171,9 +174,10 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
     if (tid == 0) {
         const uint32_t bar = smem_u32(&s_bar);
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
-                     "r"((rec ? 3u : 2u) * kTile)
+                     "r"((rec ? 3u : 2u) * kTile - (kOne ? kTile : 0u))
                      : "memory");
         for (int i = 0; i < (rec ? 3 : 2); ++i)
+            if (!kOne || i != 1)   // the one-tensor form has no second tensor
             asm volatile(
                 "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
                 " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(sbuf + i * kTile)),
@@ -212,7 +216,7 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
         for (int r = r0; r < r0 + kSub; ++r) {
             if (r < r1) {
                 const uint2 kw = *reinterpret_cast<const uint2 *>(tile_k + r * D + c0);
-                const uint2 vw = *reinterpret_cast<const uint2 *>(tile_v + r * D + c0);
+                const uint2 vw = kOne ? make_uint2(0u, 0u) : *reinterpret_cast<const uint2 *>(tile_v + r * D + c0);
                 const uint2 gw = *reinterpret_cast<const uint2 *>(tile_g + r * D + c0);
                 const uint32_t kq[2] = {kw.x, kw.y}, vq[2] = {vw.x, vw.y}, gq[2] = {gw.x, gw.y};
                 uint32_t oh[2];
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
         for (int r = r0; r < r0 + kSub; ++r) {
             if (r < r1) {
                 const float4 kk = Smem4<T>::load(tile_k + r * D + c0);
-                const float4 vv = Smem4<T>::load(tile_v + r * D + c0);
+                const float4 vv = kOne ? make_float4(0.f, 0.f, 0.f, 0.f) : Smem4<T>::load(tile_v + r * D + c0);
                 const float4 gg = rec ? Smem4<T>::load(tile_g + r * D + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
                 float om[4];
 #pragma unroll
@@ -464,9 +468,18 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
     }
     T *ck = static_cast<T *>(p.cache[0]);
     T *cv = static_cast<T *>(p.cache[1]);
-    const int Dh = p.head_dil[h];
+    const int Dh = p.head_dil[h], Wh = p.head_win[h];
     const long long S = ((long long)p.cap + Dh - 1) / Dh;
-    const size_t cbase = ((size_t)b * p.H + h) * (size_t)p.cache_R * D + c0;
+    // the window ring keeps the prefill's last W positions (one writer per row)
+    const long long ring_from = (long long)p.t0 + p.T - Wh;
+    // element offset of (cache row `row`, channel c0) of this head: the dense
+    // block or a page of a paged cache; a page the table does not name validly
+    // is reported and the row left unwritten
+    auto crow = [&](long long row) -> long long {
+        const long long o = cache_offset(p.page_table, p.pps, p.page_rows, p.num_pages, p.cache_R, p.H, D, b, h, row);
+        if (o < 0) report_error(p.hdr, RAT_ERR_INVALID, (int)ticket);
+        return o < 0 ? -1 : o + c0;
+    };
     if (loaded && !kAccurate && rec) {
         // bf16: a = 1 - (1 - a) from the fp16 cache, channel pairs in f32x2
         uint64_t sk2[2] = {f2(sk[0], sk[1]), f2(sk[2], sk[3])}, sv2[2] = {f2(sv[0], sv[1]), f2(sv[2], sv[3])};
@@ -474,7 +487,7 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
         for (int r = r0; r < r0 + kSub; ++r) {
             if (r < r1) {
                 const uint2 kw = *reinterpret_cast<const uint2 *>(tile_k + r * D + c0);
-                const uint2 vw = *reinterpret_cast<const uint2 *>(tile_v + r * D + c0);
+                const uint2 vw = kOne ? make_uint2(0u, 0u) : *reinterpret_cast<const uint2 *>(tile_v + r * D + c0);
                 const uint2 ow = *reinterpret_cast<const uint2 *>(tile_g + r * D + c0);
                 const uint32_t kq[2] = {kw.x, kw.y}, vq[2] = {vw.x, vw.y}, oq[2] = {ow.x, ow.y};
                 uint32_t wk[2], wv[2];
@@ -491,11 +504,19 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
                 *reinterpret_cast<uint2 *>(tile_k + r * D + c0) = make_uint2(wk[0], wk[1]);
                 *reinterpret_cast<uint2 *>(tile_v + r * D + c0) = make_uint2(wv[0], wv[1]);
                 if (ck) {
-                    const long long tt = tc0 + r;
-                    const long long row = (tt % Dh) * S + tt / Dh;
-                    const size_t e = cbase + (size_t)row * D;
-                    *reinterpret_cast<uint2 *>(ck + e) = make_uint2(wk[0], wk[1]);
-                    *reinterpret_cast<uint2 *>(cv + e) = make_uint2(wv[0], wv[1]);
+                    const long long tt = (long long)p.t0 + tc0 + r;
+                    long long row0, row1;
+                    cache_rows_of(tt, Dh, Wh, S, p.grid, row0, row1);
+                    const long long e0 = row0 >= 0 ? crow(row0) : -1;
+                    if (e0 >= 0) {
+                        *reinterpret_cast<uint2 *>(ck + e0) = make_uint2(wk[0], wk[1]);
+                        if (!kOne) *reinterpret_cast<uint2 *>(cv + e0) = make_uint2(wv[0], wv[1]);
+                    }
+                    const long long e1 = (row1 >= 0 && tt >= ring_from) ? crow(row1) : -1;
+                    if (e1 >= 0) {
+                        *reinterpret_cast<uint2 *>(ck + e1) = make_uint2(wk[0], wk[1]);
+                        if (!kOne) *reinterpret_cast<uint2 *>(cv + e1) = make_uint2(wv[0], wv[1]);
+                    }
                 }
             }
         }
@@ -534,11 +555,19 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
                 Smem4<T>::store(tile_k + r * D + c0, wk);
                 Smem4<T>::store(tile_v + r * D + c0, wv);
                 if (ck) {
-                    const long long tt = tc0 + r;
-                    const long long row = (tt % Dh) * S + tt / Dh;
-                    const size_t e = cbase + (size_t)row * D;
-                    IO4<T>::store(ck + e, wk);
-                    IO4<T>::store(cv + e, wv);
+                    const long long tt = (long long)p.t0 + tc0 + r;
+                    long long row0, row1;
+                    cache_rows_of(tt, Dh, Wh, S, p.grid, row0, row1);
+                    const long long e0 = row0 >= 0 ? crow(row0) : -1;
+                    if (e0 >= 0) {
+                        IO4<T>::store(ck + e0, wk);
+                        if (!kOne) IO4<T>::store(cv + e0, wv);
+                    }
+                    const long long e1 = (row1 >= 0 && tt >= ring_from) ? crow(row1) : -1;
+                    if (e1 >= 0) {
+                        IO4<T>::store(ck + e1, wk);
+                        if (!kOne) IO4<T>::store(cv + e1, wv);
+                    }
                 }
             }
         }
@@ -548,11 +577,11 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncthreads();
         if (tid == 0) {
-            for (int i = 0; i < 2; ++i)
+            for (int i = 0; i < (kOne ? 1 : 2); ++i)
                 asm volatile(
                     "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"(
                         reinterpret_cast<uint64_t>(&p.tmap[3 + i])),
-                    "r"(0), "r"(h), "r"(tc0), "r"(b), "r"(smem_u32(sbuf + i * kTile))
+                    "r"(0), "r"(h), "r"(p.t0 + tc0), "r"(b), "r"(smem_u32(sbuf + i * kTile))
                     : "memory");
             asm volatile("cp.async.bulk.commit_group;" ::: "memory");
             // the stores must have read shared memory before the CTA exits
@@ -582,14 +611,19 @@ size_t scan_smem() {
     return 3 * (size_t)C * D * sizeof(T);   // k, v, g of one chunk
 }
 
-template <typename T, int D>
-cudaError_t launch_one(const ScanParams &p, unsigned tickets, cudaStream_t s) {
+template <typename T, int D, bool kOne>
+cudaError_t launch_form(const ScanParams &p, unsigned tickets, cudaStream_t s) {
     const size_t smem = scan_smem<T, D>();
     static std::atomic<unsigned long long> smem_set{0};
-    cudaError_t e = ensure_smem_limit(scan_kernel<T, D>, smem, smem_set);
+    cudaError_t e = ensure_smem_limit(scan_kernel<T, D, kOne>, smem, smem_set);
     if (e != cudaSuccess) return e;
-    scan_kernel<T, D><<<tickets, kThreads, smem, s>>>(p);
+    scan_kernel<T, D, kOne><<<tickets, kThreads, smem, s>>>(p);
     return cudaSuccess;
+}
+
+template <typename T, int D>
+cudaError_t launch_one(const ScanParams &p, unsigned tickets, cudaStream_t s) {
+    return p.one ? launch_form<T, D, true>(p, tickets, s) : launch_form<T, D, false>(p, tickets, s);
 }
 
 }  // namespace

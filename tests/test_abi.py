@@ -36,7 +36,7 @@ def test_header_declares_the_binding_exports():
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert lib.rat_version() == 100
+    assert lib.rat_version() == 101
 
 
 def test_status_strings(lib):
@@ -96,6 +96,77 @@ def test_cache_rows_layout(lib):
         expect = max(D * -(-cap // D) for D in (1, 16, 64))
         assert lib.rat_cache_rows(c.ref(), cap) == expect
     assert lib.rat_cache_rows(c.ref(), 0) == 0
+
+
+
+def test_cache_rows_layout_fixed_grid(lib):
+    # fixed grid: ceil(cap / D) grid rows, plus a ring of W rows when D > 1 and W > 0
+    c = cfg(H=4, dil=[1, 16, 64, 8], win=[32, 0, 256, 0], flags=rat.RAT_FLAG_GRID_DILATION)
+    for cap in (1, 63, 64, 65, 4096, 33792):
+        expect = max(-(-cap // D) + (W if D > 1 else 0) for D, W in ((1, 32), (16, 0), (64, 256), (8, 0)))
+        assert lib.rat_cache_rows(c.ref(), cap) == expect
+    # the decode plan strides the cache by the same row count (workspace stays defined)
+    assert lib.rat_workspace_size(c.ref(), rat.RAT_OP_DECODE, 4096) > 0
+
+
+def test_unknown_flags_are_rejected(lib):
+    assert lib.rat_workspace_size(cfg(flags=8).ref(), rat.RAT_OP_MIX, 0) == 0
+    for f in (rat.RAT_FLAG_GRID_DILATION, rat.RAT_FLAG_DEDUPE, rat.RAT_FLAG_SEPARATE_GATES,
+              rat.RAT_FLAG_GRID_DILATION | rat.RAT_FLAG_DEDUPE | rat.RAT_FLAG_SEPARATE_GATES):
+        assert lib.rat_workspace_size(cfg(flags=f).ref(), rat.RAT_OP_MIX, 0) > 0
+
+
+
+def test_topk_sizes_and_argument_checks(lib):
+    c = cfg(B=2, H=2, dil=[1, 1], win=[0, 0])
+    # statistics: [B, H, ceil(cap / block), 2, d] fp32
+    assert lib.rat_topk_stats_size(c.ref(), 64, 4000) == 2 * 2 * 63 * 2 * 128 * 4
+    assert lib.rat_topk_stats_size(cfg().ref(), 64, 4096) == 0          # dilated heads: not the dense layout
+    assert lib.rat_topk_stats_size(cfg(dil=[1, 1]).ref(), 64, 4096) == 0  # a window
+    assert lib.rat_topk_stats_size(c.ref(), 0, 4096) == 0
+    assert lib.rat_topk_stats_size(c.ref(), 1, 16385) == 0               # more blocks than the kernel holds
+    assert lib.rat_workspace_size(c.ref(), rat.RAT_OP_TOPK_DECODE, 4096) == 256
+    P = 16
+    for block, topk, mode in ((64, 65, 0), (64, -1, 0), (64, 4, 2), (0, 4, 0)):
+        rc = lib.rat_topk_decode_step(c.ref(), block, topk, mode, P, P, P, P, P, P, P, P, 4096, P, P, P, None,
+                                      None, 256, 256, None)
+        assert rc == rat.RAT_ERR_INVALID, (block, topk, mode)
+    rc = lib.rat_topk_build_stats(c.replace(T=5000).ref(), 64, 0, P, 4096, P, None)
+    assert rc == rat.RAT_ERR_INVALID     # more tokens than the cache holds
+
+
+
+def test_paged_cache_descriptor_checks(lib):
+    # host-side checks of the page descriptor, before any launch
+    c = cfg(B=2, H=2, dil=[1, 4], win=[0, 8])
+    cap = 1000
+    R = lib.rat_cache_rows(c.ref(), cap)
+    P = 16
+
+    def step(desc):
+        return lib.rat_decode_step_paged(c.ref(), P, P, P, P, P, P, ctypes.byref(desc), cap, P, P, None, 256, 1 << 30,
+                                         None)
+
+    good = dict(pool_k=16, pool_v=32, page_table=48, page_rows=64, pages_per_seq=-(-R // 64), num_pages=64)
+    for bad in (dict(page_rows=0), dict(num_pages=0), dict(pages_per_seq=-(-R // 64) - 1), dict(pool_k=None),
+                dict(page_table=8)):
+        d = dict(good)
+        d.update(bad)
+        assert step(rat.rat_paged_cache(**d)) == rat.RAT_ERR_INVALID, bad
+    assert lib.rat_decode_step_paged(c.ref(), P, P, P, P, P, P, None, cap, P, P, None, 256, 1 << 30,
+                                     None) == rat.RAT_ERR_INVALID
+
+
+
+def test_chunked_prefill_arguments(lib):
+    # t_cap must hold the history; a chunk after the first needs the caller's kt/vt
+    assert lib.rat_workspace_size(cfg(t0=100, t_cap=150).ref(), rat.RAT_OP_SCAN, 0) == 0     # T = 100
+    assert lib.rat_workspace_size(cfg(t0=100, t_cap=200).ref(), rat.RAT_OP_SCAN, 0) > 0
+    assert lib.rat_workspace_size(cfg(t0=-1).ref(), rat.RAT_OP_SCAN, 0) == 0
+    c = cfg(t0=100)
+    P = 16
+    rc = lib.rat_mix_prefill(c.ref(), P, P, P, P, None, None, P, None, None, None, None, None, 256, 1 << 40, None)
+    assert rc == rat.RAT_ERR_INVALID
 
 
 def call_scan(lib, c, **ptrs):

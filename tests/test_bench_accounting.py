@@ -65,3 +65,33 @@ def test_profile_traffic_needs_the_captured_source(tmp_path, monkeypatch):
     assert bench.profile_traffic("missing") is None
     src.write_text("kernel source, changed\n")
     assert bench.profile_traffic("k_case", "x") is None       # the counters belong to older code
+
+
+@pytest.mark.parametrize("t,block,K", [(0, 4, 2), (3, 4, 2), (4, 4, 2), (9, 4, 2), (40, 4, 2), (40, 4, 64),
+                                       (16450, 64, 16)])
+def test_topk_decode_bytes_read_the_kept_rows_and_the_candidates(t, block, K):
+    B, H, d, elt = 2, 3, 128, 2
+    c = t // block
+    cand = list(range(1, c))
+    kept = {0, c} | set(cand[:K])          # which K does not matter for the byte count
+    rows = sum(1 for j in range(t) if j // block in kept)      # old rows; the new one is in registers
+    per = len(cand) * 2 * d * 4 + rows * 2 * d * elt + d * (5 * elt + 16 + 2 * elt) + 2 * 2 * d * 4
+    assert bench.topk_decode_bytes(B, H, d, t, block, K, elt) == B * H * per
+
+
+@pytest.mark.parametrize("grid", [False, True])
+@pytest.mark.parametrize("dedupe", [False, True])
+@pytest.mark.parametrize("T,D,W", [(1, 1, 0), (37, 4, 5), (50, 7, 100), (64, 1, 8), (100, 9, 1), (90, 30, 61)])
+def test_variant_pairs_count_the_reading_key_sets(grid, dedupe, T, D, W):
+    n = 0
+    for t in range(T):
+        dil = {j for j in range(t + 1) if ((j % D == D - 1 or j == t) if grid else (t - j) % D == 0)}
+        win = {j for j in range(t + 1) if W > 0 and j >= t - W + 1}
+        n += len(dil) + len(win - dil if dedupe else win)
+    assert bench.variant_pairs(T, D, W, grid=grid, dedupe=dedupe) == n
+    # a chunk's rows alone: the whole minus the rows before it
+    t_from = T // 3
+    n_before = bench.variant_pairs(t_from, D, W, grid=grid, dedupe=dedupe) if t_from else 0.0
+    assert bench.variant_pairs(T, D, W, grid=grid, dedupe=dedupe, t_from=t_from) == n - n_before
+    if not grid and not dedupe:
+        assert bench.attn_pairs(T, D, W) == n

@@ -22,8 +22,11 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def make_cfg(B, T, H, d, dtype, dil, win, recur=None, scale=0.0):
-    return rat.Config(B, T, H, d, dtype, dil, win, recur, scale)
+def make_cfg(B, T, H, d, dtype, dil, win, recur=None, scale=0.0, grid=False, dedupe=False, sep=False, t0=0,
+             t_cap=0):
+    flags = (rat.RAT_FLAG_GRID_DILATION if grid else 0) | (rat.RAT_FLAG_DEDUPE if dedupe else 0)
+    flags |= rat.RAT_FLAG_SEPARATE_GATES if sep else 0
+    return rat.Config(B, T, H, d, dtype, dil, win, recur, scale, flags, t0, t_cap)
 
 
 def inputs(B, T, H, d, dtype, mu=2.0, seed=0, device="cpu"):
@@ -277,21 +280,26 @@ def test_decode_cache_layout_from_scan():
 
 
 def run_decode_case(B, T, steps, H, d, dtype, dil, win, recur, mu, seed, cap=None, check_b=None, check_h=None,
-                    gen_device="cpu"):
+                    gen_device="cpu", grid=False, dedupe=False, sep=False):
     """Prefill T tokens into the cache with rat_scan_prefill, then decode `steps`
     tokens with rat_decode_step; compare every step with the oracle's rows
-    (on the batch entries check_b and heads check_h; all by default)."""
+    (on the batch entries check_b and heads check_h; all by default).  grid:
+    the fixed-grid reading of dilation and its cache layout; dedupe: a key in
+    both parts counts once; sep: separate key and value gates."""
     Tt = T + steps
     cap = cap or Tt
     q, k, v, g = inputs(B, Tt, H, d, dtype, mu=mu, seed=seed, device=gen_device)
-    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur)
+    gv = inputs(B, Tt, H, d, dtype, mu=mu, seed=seed + 1000, device=gen_device)[3] if sep else g
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur, grid=grid, dedupe=dedupe, sep=sep)
+    # the gate argument: [2, B, T, H, d] with separate gates
+    gate = (lambda sl: torch.stack([g[sl], gv[sl]]).contiguous()) if sep else (lambda sl: g[sl].contiguous())
     R = rat.rat_cache_rows(cfg, cap)
     ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
     cv = torch.zeros_like(ck)
     sk = torch.empty(B, H, d, device=DEV)
     sv = torch.empty_like(sk)
     ws = rat.workspace(cfg, rat.RAT_OP_SCAN)
-    rat.rat_scan_prefill(cfg, k[:, :T].contiguous(), v[:, :T].contiguous(), g[:, :T].contiguous(), None, None,
+    rat.rat_scan_prefill(cfg, k[:, :T].contiguous(), v[:, :T].contiguous(), gate(np.s_[:, :T]), None, None,
                          None, None, sk, sv, ck, cv, cap, ws)
     rat.rat_check_status(ws)
     del ws
@@ -303,7 +311,7 @@ def run_decode_case(B, T, steps, H, d, dtype, dil, win, recur, mu, seed, cap=Non
         o = torch.empty(B, H, d, dtype=dtype, device=DEV)
         lse = torch.empty(B, H, device=DEV)
         rat.rat_decode_step(cfg, q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(),
-                            g[:, t].contiguous(), sk, sv, ck, cv, cap, pos, o, lse, wsd)
+                            gate(np.s_[:, t]), sk, sv, ck, cv, cap, pos, o, lse, wsd)
         outs.append((o, lse))
     rat.rat_check_status(wsd)
     bsel = list(range(B)) if check_b is None else check_b
@@ -311,9 +319,9 @@ def run_decode_case(B, T, steps, H, d, dtype, dil, win, recur, mu, seed, cap=Non
     sl = lambda x: f64(x[bsel][:, :, hsel])
     dsel, wsel, rsel = [dil[h] for h in hsel], [win[h] for h in hsel], [recur[h] for h in hsel]
     kt, fk = oracle.scan(sl(k), sl(g), None, rsel)
-    vt, fv = oracle.scan(sl(v), sl(g), None, rsel)
+    vt, fv = oracle.scan(sl(v), sl(gv), None, rsel)
     rows = np.array([(b, i, t) for b in range(len(bsel)) for i in range(len(hsel)) for t in range(T, Tt)])
-    ro, rl = oracle.attn_rows(sl(q), kt, vt, dsel, wsel, rows, parts=3)
+    ro, rl = oracle.attn_rows(sl(q), kt, vt, dsel, wsel, rows, parts=3, grid=grid, dedupe=dedupe)
     ro = ro.reshape(len(bsel), len(hsel), steps, d)
     rl = rl.reshape(len(bsel), len(hsel), steps)
     ft = torch.float32 if dtype == torch.float32 else dtype
@@ -440,6 +448,462 @@ def test_decode_step_replays_from_a_cuda_graph():
     assert_close(sk, fk, dtype, "state_k after the replays")
     assert_close(sv, fv, dtype, "state_v after the replays")
     del graph
+
+
+# ------------------------------------------------- fixed-grid reading of dilation
+# Query t attends to { j <= t : j mod D == D-1 } plus itself, and the decode
+# cache keeps only the grid rows plus a ring of the last W positions.
+
+GRID_CASES = [
+    # (B, T, dil per head, win per head)
+    (2, 2048, [4, 64], [0, 100]),        # tensor-core grid launch, one head windowed
+    (1, 12800, [64, 128], [1, 3000]),    # 200 and 100 grid rows: full and partial key tiles
+    (2, 1024, [256, 1], [0, 64]),        # D = 256: the first query tiles have no grid key yet
+    (2, 1000, [8, 3], [127, 0]),         # 3 does not divide T: that head runs on CUDA cores
+]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("case", range(len(GRID_CASES)))
+def test_grid_attention_every_element(dtype, d, case):
+    B, T, dil, win = GRID_CASES[case]
+    H = len(dil)
+    q, kt, vt, _ = inputs(B, T, H, d, dtype, seed=700 + case)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, grid=True)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, T, device=DEV)
+    ws = rat.workspace(cfg, rat.RAT_OP_ATTN)
+    rat.rat_dilated_attn_prefill(cfg, q, kt, vt, o, lse, ws)
+    rat.rat_check_status(ws)
+    ro, rl = oracle.attention(f64(q), f64(kt), f64(vt), dil, win, grid=True)
+    assert_close(o, ro, dtype, "o")
+    assert_close(lse, rl, dtype if dtype == torch.bfloat16 else torch.float32, "lse")
+    err = np.linalg.norm(f64(o) - ro, axis=-1) / np.maximum(np.linalg.norm(ro, axis=-1), 1e-30)
+    assert float(err.max()) < 5e-2, "worst row rel err %.3g" % float(err.max())
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_grid_mix_hybrid_heads_every_element(dtype):
+    # a dense head without recurrence next to dilated recurrent heads
+    B, T, d = 2, 1536, 128
+    dil, win, recur = [1, 16, 64], [0, 0, 256], [0, 1, 1]
+    H = len(dil)
+    q, k, v, g = inputs(B, T, H, d, dtype, seed=77)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur, grid=True)
+    out = rat.mix_prefill(cfg, q, k, v, g)
+    rat.rat_check_status(out["ws"])
+    rk, _ = oracle.scan(f64(k), f64(g), None, recur)
+    rv, _ = oracle.scan(f64(v), f64(g), None, recur)
+    ro, rl = oracle.attention(f64(q), rk, rv, dil, win, grid=True)
+    assert_close(out["o"], ro, dtype, "o")
+    assert_close(out["lse"], rl, dtype if dtype == torch.bfloat16 else torch.float32, "lse")
+
+
+def test_grid_decode_cache_layout_from_scan():
+    # grid row of j (j mod D == D-1): j // D; ring row (D > 1, W > 0) of the
+    # prefill's last W positions: ceil(cap / D) + j mod W
+    B, T, H, d = 2, 300, 4, 64
+    dtype = torch.bfloat16
+    dil, win = [1, 4, 7, 16], [5, 0, 40, 512]
+    cap = 333
+    q, k, v, g = inputs(B, T, H, d, dtype, seed=19)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, grid=True)
+    R = rat.rat_cache_rows(cfg, cap)
+    ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
+    cv = torch.zeros_like(ck)
+    kt, vt = torch.empty_like(k), torch.empty_like(v)
+    ws = rat.workspace(cfg, rat.RAT_OP_SCAN)
+    rat.rat_scan_prefill(cfg, k, v, g, None, None, kt, vt, None, None, ck, cv, cap, ws)
+    rat.rat_check_status(ws)
+    for h, (D, W) in enumerate(zip(dil, win)):
+        S = -(-cap // D)
+        j = torch.arange(D - 1, T, D, device=DEV)
+        assert torch.equal(ck[:, h, j // D], kt[:, j, h])
+        assert torch.equal(cv[:, h, j // D], vt[:, j, h])
+        if D > 1 and W > 0:
+            j = torch.arange(max(0, T - W), T, device=DEV)
+            assert torch.equal(ck[:, h, S + j % W], kt[:, j, h])
+            assert torch.equal(cv[:, h, S + j % W], vt[:, j, h])
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+def test_grid_decode_steps_every_element(dtype, d):
+    # positions 1500..1504 put t on the grid of D = 4, 16 and 3 once each
+    run_decode_case(B=3, T=1500, steps=5, H=4, d=d, dtype=dtype, dil=[1, 4, 16, 3], win=[0, 0, 64, 1500],
+                    recur=[0, 1, 1, 1], mu=2.0, seed=21, grid=True)
+
+
+def test_grid_decode_from_empty_history():
+    # the ring fills while the first positions are decoded (cap 8 < W for one head)
+    run_decode_case(B=2, T=1, steps=6, H=3, d=128, dtype=torch.bfloat16, dil=[2, 1, 3], win=[3, 0, 10],
+                    recur=[1, 0, 1], mu=2.0, seed=5, cap=8, grid=True)
+
+
+def test_grid_decode_long_slab_spans_several_splits():
+    run_decode_case(B=1, T=5000, steps=2, H=2, d=128, dtype=torch.bfloat16, dil=[2, 1], win=[9, 7],
+                    recur=[1, 1], mu=2.0, seed=6, grid=True)
+
+
+# ------------------------------------------------- dedupe: a shared key counts once
+
+DEDUPE_CASES = [
+    # (B, T, dil per head, win per head): windows wider and narrower than D
+    (2, 2048, [4, 64], [100, 512]),
+    (1, 1056, [1, 33], [64, 1000]),       # D = 1: no window part; D = 33 > 32 (one key per chunk)
+    (2, 768, [2, 3], [1, 300]),           # W = 1 leaves the window part empty (residue reading)
+    (2, 1000, [8, 7], [127, 50]),         # 7 does not divide T: CUDA cores
+]
+
+
+@pytest.mark.parametrize("grid", [False, True])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("case", range(len(DEDUPE_CASES)))
+def test_dedupe_attention_every_element(grid, dtype, case):
+    B, T, dil, win = DEDUPE_CASES[case]
+    H, d = len(dil), 128
+    q, kt, vt, _ = inputs(B, T, H, d, dtype, seed=900 + case)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, grid=grid, dedupe=True)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, T, device=DEV)
+    ws = rat.workspace(cfg, rat.RAT_OP_ATTN)
+    rat.rat_dilated_attn_prefill(cfg, q, kt, vt, o, lse, ws)
+    rat.rat_check_status(ws)
+    ro, rl = oracle.attention(f64(q), f64(kt), f64(vt), dil, win, grid=grid, dedupe=True)
+    assert_close(o, ro, dtype, "o")
+    assert_close(lse, rl, dtype if dtype == torch.bfloat16 else torch.float32, "lse")
+    err = np.linalg.norm(f64(o) - ro, axis=-1) / np.maximum(np.linalg.norm(ro, axis=-1), 1e-30)
+    assert float(err.max()) < 5e-2, "worst row rel err %.3g" % float(err.max())
+
+
+@pytest.mark.parametrize("grid", [False, True])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_dedupe_decode_steps_every_element(grid, dtype):
+    run_decode_case(B=3, T=1500, steps=5, H=4, d=128, dtype=dtype, dil=[1, 4, 16, 3], win=[8, 9, 64, 1500],
+                    recur=[0, 1, 1, 1], mu=2.0, seed=23, grid=grid, dedupe=True)
+
+
+# ------------------------------------------- top-k block attention for decoding
+
+
+def run_topk_case(B, T, steps, H, d, dtype, block, topk, mode, recur, seed, cap=None, margin=0.02):
+    """Prefill T tokens into a dense cache, build the block statistics, decode
+    `steps` tokens with rat_topk_decode_step; compare with the oracle's top-k
+    rows.  The block choice is an integer decision: the oracle takes it on its
+    K~ rounded to the cache's precision, as the kernel does, and rows whose
+    K-th and (K+1)-th block scores lie within `margin` (rounding could swap
+    them) are only checked for a valid selection."""
+    Tt = T + steps
+    cap = cap or Tt
+    q, k, v, g = inputs(B, Tt, H, d, dtype, mu=2.0, seed=seed)
+    cfg = make_cfg(B, T, H, d, dtype, [1] * H, [0] * H, recur)
+    R = rat.rat_cache_rows(cfg, cap)
+    ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
+    cv = torch.zeros_like(ck)
+    sk = torch.empty(B, H, d, device=DEV)
+    sv = torch.empty_like(sk)
+    ws = rat.workspace(cfg, rat.RAT_OP_SCAN)
+    rat.rat_scan_prefill(cfg, k[:, :T].contiguous(), v[:, :T].contiguous(), g[:, :T].contiguous(), None, None,
+                         None, None, sk, sv, ck, cv, cap, ws)
+    rat.rat_check_status(ws)
+    stats = torch.full(rat.topk_stats_shape(cfg, block, cap), float("nan"), device=DEV)
+    rat.rat_topk_build_stats(cfg, block, mode, ck, cap, stats)
+    wsd = rat.workspace(cfg, rat.RAT_OP_TOPK_DECODE, cap)
+    outs = []
+    for s in range(steps):
+        t = T + s
+        pos = torch.full((B,), t, dtype=torch.int32, device=DEV)
+        o = torch.empty(B, H, d, dtype=dtype, device=DEV)
+        lse = torch.empty(B, H, device=DEV)
+        sel = torch.empty(B, H, topk, dtype=torch.int32, device=DEV)
+        rat.rat_topk_decode_step(cfg, block, topk, mode, q[:, t].contiguous(), k[:, t].contiguous(),
+                                 v[:, t].contiguous(), g[:, t].contiguous(), sk, sv, ck, cv, cap, stats, pos, o,
+                                 lse, sel, wsd)
+        outs.append((o, lse, sel))
+    rat.rat_check_status(wsd)
+    kt, fk = oracle.scan(f64(k), f64(g), None, recur)
+    vt, fv = oracle.scan(f64(v), f64(g), None, recur)
+    ft = torch.float32 if dtype == torch.float32 else dtype
+    assert_close(ck[:, :, :Tt].transpose(1, 2), kt, dtype, "cache_k")
+    assert_close(cv[:, :, :Tt].transpose(1, 2), vt, dtype, "cache_v")
+    assert_close(sk, fk, ft, "state_k")
+    # the cache's precision for the oracle's keys and values
+    kq = torch.from_numpy(kt).to(dtype).double().numpy()
+    vq = torch.from_numpy(vt).to(dtype).double().numpy()
+    name = {rat.RAT_TOPK_QUEST: "quest", rat.RAT_TOPK_MOBA: "moba"}[mode]
+    rows = np.array([(b, h, t) for b in range(B) for h in range(H) for t in range(T, Tt)])
+    ro, rl = oracle.attn_rows_topk(f64(q), kq, vq, block, topk, name, rows)
+    rsel, gap = oracle.topk_select(f64(q), kq, block, topk, name, rows)
+    got_o = np.stack([f64(o) for o, _, _ in outs], axis=2).reshape(-1, d)      # (b, h, step) order
+    got_l = np.stack([f64(l) for _, l, _ in outs], axis=2).reshape(-1)
+    got_s = np.stack([x[2].cpu().numpy() for x in outs], axis=2).reshape(-1, topk)
+    clear = gap > margin
+    assert clear.mean() >= 0.6, "too many near-ties: %d of %d rows" % (int((~clear).sum()), len(clear))
+    for i in np.nonzero(clear)[0]:
+        assert sorted(got_s[i]) == sorted(rsel[i]), (rows[i], got_s[i], rsel[i])
+    assert_close(got_o[clear], ro[clear], dtype, "top-k o")
+    assert_close(got_l[clear], rl[clear], ft, "top-k lse")
+    for i in np.nonzero(~clear)[0]:   # a near-tie: any valid selection of distinct candidates
+        c = rows[i][2] // block
+        picked = [x for x in got_s[i] if x >= 0]
+        assert len(set(picked)) == len(picked) == min(topk, max(0, c - 1))
+        assert all(1 <= x < c for x in picked)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+def test_topk_decode_steps(mode, dtype, d):
+    # positions 1021 .. 1025 cross into a new 64-row block at 1024
+    run_topk_case(B=2, T=1021, steps=5, H=3, d=d, dtype=dtype, block=64, topk=4, mode=mode, recur=[0, 1, 1],
+                  seed=31 + mode)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_topk_decode_from_empty_history(mode):
+    # blocks of 4 from t = 1: no candidates, then fewer than K, then more
+    run_topk_case(B=2, T=1, steps=30, H=2, d=128, dtype=torch.bfloat16, block=4, topk=3, mode=mode,
+                  recur=[1, 0], seed=41, cap=40)
+
+
+def test_topk_decode_keeps_every_block_when_k_is_large():
+    # K >= number of candidates: the step is dense causal attention
+    run_topk_case(B=1, T=500, steps=3, H=2, d=128, dtype=torch.bfloat16, block=32, topk=64, mode=0,
+                  recur=[1, 1], seed=43)
+
+
+# ------------------------------------------------- separate key and value gates
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("T", [77, 5003])
+def test_separate_gates_scan_every_element(dtype, d, T):
+    B, H = 2, 3
+    q, k, v, g = inputs(B, T, H, d, dtype, seed=T + 1)
+    gv = inputs(B, T, H, d, dtype, mu=0.5, seed=T + 2)[3]
+    init_k = wl.random_state(B, H, d, seed=3).to(DEV)
+    init_v = wl.random_state(B, H, d, seed=4).to(DEV)
+    recur = [1, 0, 1]
+    cap = T + 5
+    cfg = make_cfg(B, T, H, d, dtype, [1, 4, 7], [0, 0, 9], recur, sep=True)
+    kt, vt = torch.empty_like(k), torch.empty_like(v)
+    fk = torch.empty(B, H, d, device=DEV)
+    fv = torch.empty_like(fk)
+    R = rat.rat_cache_rows(cfg, cap)
+    ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
+    cv = torch.zeros_like(ck)
+    ws = rat.workspace(cfg, rat.RAT_OP_SCAN)
+    rat.rat_scan_prefill(cfg, k, v, torch.stack([g, gv]).contiguous(), init_k, init_v, kt, vt, fk, fv, ck, cv,
+                         cap, ws)
+    rat.rat_check_status(ws)
+    rk, rfk = oracle.scan(f64(k), f64(g), f64(init_k), recur)
+    rv, rfv = oracle.scan(f64(v), f64(gv), f64(init_v), recur)
+    ft = torch.float32 if dtype == torch.float32 else dtype
+    assert_close(kt, rk, dtype, "kt")
+    assert_close(vt, rv, dtype, "vt")
+    assert_close(fk, rfk, ft, "final_k")
+    assert_close(fv, rfv, ft, "final_v")
+    for h, D in enumerate([1, 4, 7]):   # both caches written, each from its own pass
+        S = -(-cap // D)
+        j = torch.arange(T, device=DEV)
+        rows = (j % D) * S + j // D
+        assert torch.equal(ck[:, h, rows], kt[:, :, h]) and torch.equal(cv[:, h, rows], vt[:, :, h])
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_separate_gates_mix_every_element(dtype):
+    B, T, H, d = 2, 2048, 3, 128
+    dil, win, recur = [1, 16, 64], [0, 0, 256], [0, 1, 1]
+    q, k, v, g = inputs(B, T, H, d, dtype, seed=51)
+    gv = inputs(B, T, H, d, dtype, mu=-1.0, seed=52)[3]
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur, sep=True)
+    out = rat.mix_prefill(cfg, q, k, v, torch.stack([g, gv]).contiguous())
+    rat.rat_check_status(out["ws"])
+    rk, rfk = oracle.scan(f64(k), f64(g), None, recur)
+    rv, rfv = oracle.scan(f64(v), f64(gv), None, recur)
+    ro, rl = oracle.attention(f64(q), rk, rv, dil, win)
+    ft = torch.float32 if dtype == torch.float32 else dtype
+    assert_close(out["o"], ro, dtype, "o")
+    assert_close(out["lse"], rl, ft, "lse")
+    assert_close(out["final_k"], rfk, ft, "final_k")
+    assert_close(out["final_v"], rfv, ft, "final_v")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_separate_gates_decode_steps(dtype):
+    run_decode_case(B=3, T=1500, steps=4, H=4, d=128, dtype=dtype, dil=[1, 4, 16, 3], win=[0, 0, 64, 1500],
+                    recur=[0, 1, 1, 1], mu=2.0, seed=25, sep=True)
+
+
+# ---------------------------------------------------------- paged decode cache
+
+
+def _paged_setup(grid):
+    B, T, steps, H, d = 3, 700, 4, 3, 128
+    dil, win, recur = [1, 4, 7], [0, 16, 100], [0, 1, 1]
+    cap = T + steps
+    dtype = torch.bfloat16
+    q, k, v, g = inputs(B, T + steps, H, d, dtype, seed=61)
+    cfg = make_cfg(B, T, H, d, dtype, dil, win, recur, grid=grid)
+    R = rat.rat_cache_rows(cfg, cap)
+    P = 48                      # not a multiple of a ring stage (64 rows): stages straddle pages
+    pps = -(-R // P)
+    num_pages = B * pps + 5
+    perm = torch.randperm(num_pages, generator=torch.Generator().manual_seed(7))[:B * pps]
+    table = perm.view(B, pps).to(torch.int32).to(DEV)
+    return B, T, steps, H, d, cap, dtype, q, k, v, g, cfg, R, P, num_pages, table
+
+
+@pytest.mark.parametrize("grid", [False, True])
+def test_paged_decode_equals_dense(grid):
+    # the same logical rows in shuffled pages: every output bit-identical
+    B, T, steps, H, d, cap, dtype, q, k, v, g, cfg, R, P, num_pages, table = _paged_setup(grid)
+    ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
+    cv = torch.zeros_like(ck)
+    pool_k = torch.zeros(num_pages, H, P, d, dtype=dtype, device=DEV)
+    pool_v = torch.zeros_like(pool_k)
+    cache = rat.paged_cache(cfg, pool_k, pool_v, table, cap)
+    states = [torch.empty(B, H, d, device=DEV) for _ in range(4)]
+    ws = rat.workspace(cfg, rat.RAT_OP_SCAN)
+    pre = (k[:, :T].contiguous(), v[:, :T].contiguous(), g[:, :T].contiguous())
+    rat.rat_scan_prefill(cfg, *pre, None, None, None, None, states[0], states[1], ck, cv, cap, ws)
+    rat.rat_scan_prefill_paged(cfg, *pre, None, None, None, None, states[2], states[3], cache=cache, cache_cap=cap,
+                               ws=ws)
+    rat.rat_check_status(ws)
+    wsd = rat.workspace(cfg, rat.RAT_OP_DECODE, cap)
+    for s in range(steps):
+        t = T + s
+        pos = torch.full((B,), t, dtype=torch.int32, device=DEV)
+        tok = (q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(), g[:, t].contiguous())
+        o1, o2 = torch.empty(B, H, d, dtype=dtype, device=DEV), torch.empty(B, H, d, dtype=dtype, device=DEV)
+        l1, l2 = torch.empty(B, H, device=DEV), torch.empty(B, H, device=DEV)
+        rat.rat_decode_step(cfg, *tok, states[0], states[1], ck, cv, cap, pos, o1, l1, wsd)
+        rat.rat_decode_step_paged(cfg, *tok, states[2], states[3], cache, cap, pos, o2, l2, wsd)
+        rat.rat_check_status(wsd)
+        assert torch.equal(o1, o2) and torch.equal(l1, l2), "step %d" % s
+    assert torch.equal(states[0], states[2]) and torch.equal(states[1], states[3])
+    # every logical row sits in the page the table names
+    r = torch.arange(R, device=DEV)
+    for b in range(B):
+        pg = table[b, r // P].long()
+        for h in range(H):
+            assert torch.equal(pool_k[pg, h, r % P], ck[b, h]) and torch.equal(pool_v[pg, h, r % P], cv[b, h])
+
+
+def test_paged_decode_invalid_page_is_reported():
+    # a table entry of -1 on a page the step reads: every head of entry 1 reads
+    # logical rows from 0 at t = 700 (residue 0 of D = 1, 4, 7), so all are
+    # skipped (o = 0) and RAT_ERR_INVALID recorded; the other entries are not
+    B, T, steps, H, d, cap, dtype, q, k, v, g, cfg, R, P, num_pages, table = _paged_setup(False)
+    pool_k = torch.zeros(num_pages, H, P, d, dtype=dtype, device=DEV)
+    pool_v = torch.zeros_like(pool_k)
+    cache = rat.paged_cache(cfg, pool_k, pool_v, table, cap)
+    sk, sv = torch.empty(B, H, d, device=DEV), torch.empty(B, H, d, device=DEV)
+    ws = rat.workspace(cfg, rat.RAT_OP_SCAN)
+    rat.rat_scan_prefill_paged(cfg, k[:, :T].contiguous(), v[:, :T].contiguous(), g[:, :T].contiguous(), None,
+                               None, None, None, sk, sv, cache=cache, cache_cap=cap, ws=ws)
+    rat.rat_check_status(ws)
+    ok = table.clone()
+    table[1, 0] = -1            # head 0 of entry 1 (D = 1) reads logical rows from 0
+    t = T
+    pos = torch.full((B,), t, dtype=torch.int32, device=DEV)
+    o = torch.empty(B, H, d, dtype=dtype, device=DEV)
+    wsd = rat.workspace(cfg, rat.RAT_OP_DECODE, cap)
+    rat.rat_decode_step_paged(cfg, q[:, t].contiguous(), k[:, t].contiguous(), v[:, t].contiguous(),
+                              g[:, t].contiguous(), sk, sv, cache, cap, pos, o, None, wsd)
+    with pytest.raises(rat.RatError) as err:
+        rat.rat_check_status(wsd)
+    assert err.value.status == rat.RAT_ERR_INVALID
+    assert torch.count_nonzero(o[1]) == 0
+    assert torch.count_nonzero(o[0]) > 0 and torch.count_nonzero(o[2]) > 0
+    table.copy_(ok)
+
+
+# ------------------------------------------------------------- chunked prefill
+
+
+@pytest.mark.parametrize("grid", [False, True])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("chunks", [[1024, 512, 448], [1000, 600, 384]])
+def test_chunked_prefill_equals_one_shot(grid, dtype, chunks):
+    # the chunks carry the recurrent state and share one kt/vt history buffer
+    # (t_cap rows per batch entry); the second chunk list starts chunks at
+    # 1000 and 1600, which D = 64 does not divide (those heads run on CUDA cores)
+    B, H, d = 2, 3, 128
+    dil, win, recur = [1, 8, 64], [0, 32, 300], [0, 1, 1]
+    Ttot = sum(chunks)
+    cap = Ttot + 8
+    q, k, v, g = inputs(B, Ttot, H, d, dtype, seed=81)
+    kt = torch.zeros(B, cap, H, d, dtype=dtype, device=DEV)
+    vt = torch.zeros_like(kt)
+    sk = sv = None
+    R = rat.rat_cache_rows(make_cfg(B, 1, H, d, dtype, dil, win, recur, grid=grid), cap)
+    ck = torch.zeros(B, H, R, d, dtype=dtype, device=DEV)
+    cv = torch.zeros_like(ck)
+    outs, lses = [], []
+    t0 = 0
+    for Tc in chunks:
+        cfg = make_cfg(B, Tc, H, d, dtype, dil, win, recur, grid=grid, t0=t0, t_cap=cap)
+        sl = np.s_[:, t0:t0 + Tc]
+        o = torch.empty(B, Tc, H, d, dtype=dtype, device=DEV)
+        lse = torch.empty(B, H, Tc, device=DEV)
+        fk, fv = torch.empty(B, H, d, device=DEV), torch.empty(B, H, d, device=DEV)
+        ws = rat.workspace(cfg, rat.RAT_OP_MIX_CALLER_KV)
+        rat.rat_mix_prefill(cfg, q[sl].contiguous(), k[sl].contiguous(), v[sl].contiguous(), g[sl].contiguous(),
+                            sk, sv, o, lse, kt, vt, fk, fv, ws)
+        # the decode cache of the same chunk (its rows go to positions t0 + t)
+        wss = rat.workspace(cfg, rat.RAT_OP_SCAN)
+        rat.rat_scan_prefill(cfg, k[sl].contiguous(), v[sl].contiguous(), g[sl].contiguous(), sk, sv, None, None,
+                             None, None, ck, cv, cap, wss)
+        rat.rat_check_status(ws)
+        rat.rat_check_status(wss)
+        outs.append(o)
+        lses.append(lse)
+        sk, sv = fk, fv
+        t0 += Tc
+    rk, rfk = oracle.scan(f64(k), f64(g), None, recur)
+    rv, rfv = oracle.scan(f64(v), f64(g), None, recur)
+    ro, rl = oracle.attention(f64(q), rk, rv, dil, win, grid=grid)
+    ft = torch.float32 if dtype == torch.float32 else dtype
+    assert_close(torch.cat(outs, 1), ro, dtype, "o")
+    assert_close(torch.cat(lses, 2), rl, ft, "lse")
+    assert_close(kt[:, :Ttot], rk, dtype, "kt history")
+    assert_close(sk, rfk, ft, "final_k")
+    # every position's cache row (the layout of include/rat.h) holds the
+    # oracle's augmented key and value, written chunk by chunk
+    ckh, cvh = f64(ck), f64(cv)
+    for h, (D, W) in enumerate(zip(dil, win)):
+        S = -(-cap // D)
+        for j in range(Ttot):
+            if grid:
+                rows = ([j // D] if j % D == D - 1 else []) + ([S + j % W] if D > 1 and W > 0 and j >= Ttot - W else [])
+            else:
+                rows = [(j % D) * S + j // D]
+            for r in rows:
+                np.testing.assert_allclose(ckh[:, h, r], rk[:, j, h], rtol=2e-2, atol=2e-2)
+                np.testing.assert_allclose(cvh[:, h, r], rv[:, j, h], rtol=2e-2, atol=2e-2)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_attention_with_large_scores(dtype):
+    # q scaled by 8: scores of tens in the log2 domain, so the running max
+    # grows by more than the lazy-rescale threshold between tiles and P must
+    # stay bounded; the outputs still match the oracle
+    B, T, H, d = 1, 4096, 2, 128
+    q, kt, vt, _ = inputs(B, T, H, d, dtype, seed=91)
+    q = (q.float() * 8).to(dtype)
+    dil, win = [16, 1], [256, 0]
+    cfg = make_cfg(B, T, H, d, dtype, dil, win)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, T, device=DEV)
+    ws = rat.workspace(cfg, rat.RAT_OP_ATTN)
+    rat.rat_dilated_attn_prefill(cfg, q, kt, vt, o, lse, ws)
+    rat.rat_check_status(ws)
+    ro, rl = oracle.attention(f64(q), f64(kt), f64(vt), dil, win)
+    assert_close(o, ro, dtype, "o")
+    assert_close(lse, rl, dtype if dtype == torch.bfloat16 else torch.float32, "lse")
 
 
 def test_decode_bad_position_is_reported():
