@@ -40,6 +40,7 @@ import workloads as wl  # noqa: E402
 
 METRIC = "temporal-mix prefill tok/s @262K & decode tok/s; % of HBM/tensor roofline"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_HBM_GBS = 8000.0   # the ~8 TB/s nominal HBM3e figure, reported beside the measured copy peak
 
 
 # ----------------------------------------------------------------- plumbing
@@ -296,7 +297,15 @@ def decode_bytes(B, H, d, t, dil, win, elt=2):
 # --------------------------------------------------------------- prefill
 
 
-def bench_prefill(rat, w, steps, warmup, world, rank, dev, e2e_steps):
+def bench_prefill(rat, w, steps, warmup, world, rank, dev, e2e_steps, mix=False):
+    """Time `steps` prefill steps of workload w.  By default a step is
+    rat_scan_prefill then rat_dilated_attn_prefill (= rat_mix_prefill with
+    caller K~/V~), with events around each stage.  mix=True times
+    rat_mix_prefill itself with K~/V~ kept in its workspace, as a user calls
+    it (heads without recurrence then attend to k/v without a copy), and the
+    attention stage alone in a second timed loop."""
+    if mix:
+        return bench_prefill_mix(rat, w, steps, warmup, world, rank, dev)
     dtype = w.torch_dtype
     q, k, v, g = wl.prefill_inputs(w.B, w.T, w.H, w.d, w.gate_mean, dtype, device=dev, seed=rank)
     cfg = rat.Config(w.B, w.T, w.H, w.d, dtype, w.dil, w.win, w.recur)
@@ -409,6 +418,67 @@ def bench_prefill(rat, w, steps, warmup, world, rank, dev, e2e_steps):
     del q, k, v, g, o, lse, ws
     torch.cuda.empty_cache()
     return res
+
+
+def bench_prefill_mix(rat, w, steps, warmup, world, rank, dev):
+    dtype = w.torch_dtype
+    q, k, v, g = wl.prefill_inputs(w.B, w.T, w.H, w.d, w.gate_mean, dtype, device=dev, seed=rank)
+    cfg = rat.Config(w.B, w.T, w.H, w.d, dtype, w.dil, w.win, w.recur)
+    o = torch.empty_like(q)
+    lse = torch.empty(w.B, w.H, w.T, dtype=torch.float32, device=dev)
+    fk = torch.empty(w.B, w.H, w.d, dtype=torch.float32, device=dev)
+    fv = torch.empty_like(fk)
+    ws = rat.workspace(cfg, rat.RAT_OP_MIX, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, n):
+        barrier(world)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n0 = rat.rat_launch_count()
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(a.elapsed_time(b), world, dev), rat.rat_launch_count() - n0
+
+    mix = lambda: rat.rat_mix_prefill(cfg, q, k, v, g, None, None, o, lse, None, None, fk, fv, ws=ws,
+                                      stream=stream)
+    clk = ClockSampler(torch.cuda.current_device()).start()
+    for _ in range(warmup):
+        mix()
+    rat.rat_check_status(ws)
+    t_host0 = time.time()
+    total_ms, launches = timed(mix, steps)
+    t_host1 = time.time()
+    clk.stop()
+    rat.rat_check_status(ws)
+    del ws
+    torch.cuda.empty_cache()
+    # the scan stage alone (rat_scan_prefill into caller K~/V~, which also
+    # copies the k/v of heads without recurrence), then the attention stage
+    # alone over those augmented keys/values
+    kt, vt = torch.empty_like(k), torch.empty_like(v)
+    wss = rat.workspace(cfg, rat.RAT_OP_SCAN, device=dev)
+    scan = lambda: rat.rat_scan_prefill(cfg, k, v, g, None, None, kt, vt, fk, fv, ws=wss, stream=stream)
+    for _ in range(warmup):
+        scan()
+    scan_total, _ = timed(scan, steps)
+    rat.rat_check_status(wss)
+    del wss, k, v, g
+    wsa = rat.workspace(cfg, rat.RAT_OP_ATTN, device=dev)
+    attn = lambda: rat.rat_dilated_attn_prefill(cfg, q, kt, vt, o, lse, ws=wsa, stream=stream)
+    for _ in range(warmup):
+        attn()
+    attn_total, _ = timed(attn, steps)
+    rat.rat_check_status(wsa)
+    del q, kt, vt, o, lse, wsa
+    torch.cuda.empty_cache()
+    plain = sum(1 for h in range(w.H) if not w.recur[h])
+    return dict(total_ms=total_ms, attn_ms=attn_total / steps, scan_ms=scan_total / steps,
+                scan_copy_bytes=float(w.B * w.T * plain * w.d * 4 * (2 if w.dtype == "bf16" else 4)),
+                launches=launches, clocks=clk.summary(t_host0, t_host1))
 
 
 # ---------------------------------------------------------------- decode
@@ -599,26 +669,58 @@ def bench_topk(rat, B, H, d, ctx, block, K, mode, steps, warmup, world, rank, de
 
 
 def oracle_sample(w, n_rows, seed=0, rows_offset=0.5):
-    """Time the CPU oracle on head 0 of the workload: the full-length scan of k
-    and v, then `n_rows` query rows spread evenly over T.  Returns the
-    extrapolated whole-operator throughput (tokens/s over all heads)."""
+    """Time the CPU oracle on one head of each head class of the workload (a
+    class = heads with the same dilation, window and recurrence flag): the
+    full-length scan of k and v, then `n_rows` query rows spread evenly over T.
+    Returns the extrapolated whole-operator throughput (tokens/s over all
+    heads and batch entries) and the seconds the sample took."""
     import oracle
 
-    q, k, v, g = wl.prefill_inputs(w.B, w.T, 1, w.d, w.gate_mean, w.torch_dtype, device="cpu", seed=seed)
+    classes = {}
+    for h in range(w.H):
+        classes.setdefault((w.dil[h], w.win[h], w.recur[h]), []).append(h)
+    q, k, v, g = wl.prefill_inputs(1, w.T, 1, w.d, w.gate_mean, w.torch_dtype, device="cpu", seed=seed)
     f = lambda x: x.float().numpy().astype(np.float64)
     q, k, v, g = f(q), f(k), f(v), f(g)
-    t0 = time.perf_counter()
-    kt, _ = oracle.scan(k, g, None, [w.recur[0]])
-    vt, _ = oracle.scan(v, g, None, [w.recur[0]])
-    t_scan = time.perf_counter() - t0
     ts = ((np.arange(n_rows) + rows_offset) * w.T / n_rows).astype(np.int64)
     rows = np.stack([np.zeros_like(ts), np.zeros_like(ts), ts], axis=1)
-    t0 = time.perf_counter()
-    oracle.attn_rows(q, kt, vt, [w.dil[0]], [w.win[0]], rows, parts=3)
-    t_rows = time.perf_counter() - t0
-    per_head = t_scan + t_rows * (w.T / n_rows)
-    tok_s = w.B * w.T / (per_head * w.H)
-    return tok_s, t_scan + t_rows
+    per_seq, spent = 0.0, 0.0
+    for (D, W, rec), heads in classes.items():
+        t0 = time.perf_counter()
+        kt, _ = oracle.scan(k, g, None, [rec])
+        vt, _ = oracle.scan(v, g, None, [rec])
+        t_scan = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        oracle.attn_rows(q, kt, vt, [D], [W], rows, parts=3)
+        t_rows = time.perf_counter() - t0
+        per_seq += len(heads) * (t_scan + t_rows * (w.T / n_rows))
+        spent += t_scan + t_rows
+    tok_s = w.T / per_seq
+    return tok_s, spent
+
+
+def oracle_decode_sample(w, ctx, seed=0):
+    """Time one oracle decode step of one batch entry (all heads) at position
+    ctx over a random history; a step of the whole batch costs B times that.
+    Returns (tokens/s, seconds spent)."""
+    import oracle
+
+    H, d = w.H, w.d
+    rng = np.random.default_rng(seed)
+    # the oracle's work does not depend on the values: a constant history
+    hist_k = np.full((1, ctx + 1, H, d), 0.25)
+    hist_v = np.full((1, ctx + 1, H, d), 0.5)
+    sk, sv = rng.standard_normal((1, H, d)), rng.standard_normal((1, H, d))
+    q, k, v = (rng.standard_normal((1, H, d)) for _ in range(3))
+    g = rng.standard_normal((1, H, d)) + w.gate_mean
+    n, t0 = 0, time.perf_counter()
+    while True:   # repeat the step (same position) for at least 0.2 s
+        oracle.decode_step(q, k, v, g, sk, sv, hist_k, hist_v, [ctx], w.dil, w.win, w.recur)
+        n += 1
+        sec = time.perf_counter() - t0
+        if sec >= 0.2:
+            break
+    return n / sec, sec
 
 
 def host_cores():
@@ -657,6 +759,55 @@ def run_reference(args, world, rank):
 # ------------------------------------------------------------------ main
 
 
+def hbm_roofline(byts, ms, peaks, traffic=None):
+    gbs = byts / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": gbs / peaks["hbm_gbs"], "frac_of_nominal_8tbs": gbs / NOMINAL_HBM_GBS, "traffic": traffic,
+            "peak_source": peaks["_source"] + " copy"}
+
+
+def tensor_roofline(flops, ms, peaks, traffic=None, kernel=None):
+    tf = flops / (ms * 1e-3) / 1e12
+    r = {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+         "frac": tf / peaks["bf16_tflops"], "traffic": traffic, "peak_source": peaks["_source"] + " bf16 dense burst"}
+    if kernel:
+        r = dict(kernel=kernel, **r)
+    return r
+
+
+def prefill_entry(w, r, steps, world, peaks, cpu=None):
+    """One prefill workload's line: whole-step tok/s, the attention stage
+    against the bf16 tensor peak and the scan stage against HBM."""
+    flops, scan_bytes = prefill_work(w)
+    scan_bytes += r.get("scan_copy_bytes", 0.0)
+    step_ms = r["total_ms"] / steps
+    e = {"workload": w.name, "value": w.B * w.T * world / (step_ms * 1e-3), "unit": "tok/s",
+         "ms_per_step": step_ms, "kernels_ms": {"scan": r["scan_ms"], "attention": r["attn_ms"]},
+         "roofline": tensor_roofline(flops, r["attn_ms"], peaks, kernel="attention"),
+         "scan_roofline": hbm_roofline(scan_bytes, r["scan_ms"], peaks) if r["scan_ms"] > 0 else None,
+         "gpu_launches": r["launches"], "clocks": r["clocks"]}
+    if "scan_copy_bytes" in r:
+        e["step"] = ("rat_mix_prefill (K~/V~ in its workspace, heads without recurrence read k/v directly); "
+                     "the scan (into caller K~/V~, copying those heads' k/v: 4 B per token-channel each way) "
+                     "and the attention timed alone")
+    if cpu:
+        e["cpu_baseline"] = cpu
+    return e
+
+
+def decode_entry(w, r, steps, world, peaks, traffic=None, cpu=None):
+    e = {"ctx": r["ctx"], "value": w.decode_batch * world / (r["ms"] * 1e-3), "unit": "tok/s",
+         "ms_per_step": r["ms"], "steps": steps, "roofline": hbm_roofline(r["bytes"], r["ms"], peaks, traffic),
+         "gpu_launches": r["launches"]}
+    if cpu:
+        e["cpu_baseline"] = cpu
+    return e
+
+
+def cpu_entry(v, secs, what):
+    return {"value": v, "unit": "tok/s", "cores": host_cores(), "kind": "oracle", "sample": "%s (%.1f s)" % (what, secs)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -664,11 +815,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-ctx", type=str, default="4096,16384,32768")
-    ap.add_argument("--decode-steps", type=int, default=64)
+    ap.add_argument("--decode-steps", type=int, default=0,
+                    help="decode steps per context (0: the workload's own horizon, 1024 and 256)")
     ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--cpu-rows", type=int, default=2048, help="oracle rows timed for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=512, help="oracle rows per reference-arm step")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads (16K prefill, hybrid prefill and decode)")
     ap.add_argument("--no-next-rows", action="store_true",
                     help="skip the decode variants (fixed grid, paged cache, top-k blocks)")
     args = ap.parse_args()
@@ -689,6 +843,7 @@ def main():
     init_dist(world, "nccl")
     rat.load_library()
     peaks = load_peaks()
+    cpu_ok = not args.no_cpu and world == 1
 
     w = wl.PREFILL_262K
     pre = bench_prefill(rat, w, args.steps, args.warmup, world, rank, dev, args.e2e_steps)
@@ -697,22 +852,32 @@ def main():
     step_ms = pre["total_ms"] / args.steps
     value = tokens / (step_ms * 1e-3)
 
+    wd = wl.DECODE_D16
+    dsteps = args.decode_steps or wd.decode_steps
     dec = []
     for ctx in [int(c) for c in args.decode_ctx.split(",") if c]:
-        dec.append(bench_decode(rat, wl.DECODE_D16, ctx, args.decode_steps, args.warmup, world, rank, dev))
+        dec.append(bench_decode(rat, wd, ctx, dsteps, args.warmup, world, rank, dev))
+
+    cfgs = {}
+    if not args.no_configs:
+        w2, w5 = wl.PREFILL_16K, wl.HYBRID
+        cfgs["prefill_16k"] = (w2, bench_prefill(rat, w2, args.steps, args.warmup, world, rank, dev, 0))
+        cfgs["prefill_hybrid"] = (w5, bench_prefill(rat, w5, args.steps, args.warmup, world, rank, dev, 0, mix=True))
+        h_steps = args.decode_steps or w5.decode_steps
+        cfgs["decode_hybrid"] = (w5, bench_decode(rat, w5, w5.decode_ctx[0], h_steps, args.warmup, world, rank, dev,
+                                                  fill_chunk=4), h_steps)
 
     nxt = {}
     if not args.no_next_rows:
-        wd = wl.DECODE_D16
-        nxt["grid_decode"] = bench_decode(rat, wd, 4096, args.decode_steps, args.warmup, world, rank, dev,
+        vsteps = min(dsteps, 64)
+        nxt["grid_decode"] = bench_decode(rat, wd, 4096, vsteps, args.warmup, world, rank, dev,
                                           flags=rat.RAT_FLAG_GRID_DILATION)
-        nxt["paged_decode"] = bench_decode(rat, wd, 4096, args.decode_steps, args.warmup, world, rank, dev,
-                                           page_rows=256)
+        nxt["paged_decode"] = bench_decode(rat, wd, 4096, vsteps, args.warmup, world, rank, dev, page_rows=256)
         att_var = {name: bench_attn_variant(rat, w, f, 3, args.warmup, world, rank, dev)
                    for name, f in (("grid", rat.RAT_FLAG_GRID_DILATION), ("dedupe", rat.RAT_FLAG_DEDUPE))}
         att_var["chunked"] = bench_attn_variant(rat, w, 0, 3, args.warmup, world, rank, dev, t0=w.T * 3 // 4)
         nxt["topk_decode"] = bench_topk(rat, wd.decode_batch, wd.H, wd.d, 16384, 64, 16, rat.RAT_TOPK_QUEST,
-                                        args.decode_steps, args.warmup, world, rank, dev)
+                                        vsteps, args.warmup, world, rank, dev)
 
     if rank != 0:
         return
@@ -741,10 +906,8 @@ def main():
                      "traffic": profile_traffic("attn_prefill262k"),
                      "algorithmic": "%.4g FLOP per launch (4*d per unmasked pair)" % flops,
                      "peak_source": peaks["_source"] + " bf16 dense burst"},
-        "scan_roofline": {"bound": "hbm", "achieved": scan_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                          "frac": scan_gbs / peaks["hbm_gbs"], "traffic": profile_traffic("scan_prefill262k"),
-                          "algorithmic": "%.4g bytes per launch (10 B per token-channel)" % scan_bytes,
-                          "peak_source": peaks["_source"] + " copy"},
+        "scan_roofline": dict(hbm_roofline(scan_bytes, pre["scan_ms"], peaks, profile_traffic("scan_prefill262k")),
+                              algorithmic="%.4g bytes per launch (10 B per token-channel)" % scan_bytes),
         "kernels_ms": {"scan": pre["scan_ms"], "attention": pre["attn_ms"]},
         "gpu_launches": pre["launches"],
         "clocks": pre["clocks"],
@@ -756,45 +919,58 @@ def main():
                        "pipelined": "copy-in of step i+1 and copy-out of step i-1 overlap step i (three streams, "
                                     "double-buffered device tensors); timed from the first copy-in to the last copy-out"}
     if dec:
-        wd = wl.DECODE_D16
         line["decode"] = {
             "metric": "decode tok/s (batch %d, H%d d%d D%d)" % (wd.decode_batch, wd.H, wd.d, wd.dil[0]),
-            "unit": "tok/s",
-            "steps": args.decode_steps,
-            "by_ctx": [{"ctx": r["ctx"], "value": wd.decode_batch * world / (r["ms"] * 1e-3), "ms_per_step": r["ms"],
-                        "roofline": {"bound": "hbm", "achieved": r["bytes"] / (r["ms"] * 1e-3) / 1e9,
-                                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                     "frac": r["bytes"] / (r["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                                     "traffic": profile_traffic("decode_batch256", "decode_ctx%d" % r["ctx"])},
-                        "gpu_launches": r["launches"]} for r in dec],
+            "workload": wd.name, "unit": "tok/s", "steps": dsteps,
+            "by_ctx": [decode_entry(wd, r, dsteps, world, peaks,
+                                    traffic=profile_traffic("decode_batch256", "decode_ctx%d" % r["ctx"]),
+                                    cpu=cpu_entry(*oracle_decode_sample(wd, r["ctx"]),
+                                                  "one batch entry's step (all heads) at position %d, repeated; "
+                                                  "times the batch" % r["ctx"]) if cpu_ok else None)
+                       for r in dec],
         }
+    if cfgs:
+        line["configs"] = {}
+        for name, item in cfgs.items():
+            wc, r = item[0], item[1]
+            if name.startswith("prefill"):
+                cpu = None
+                if cpu_ok:
+                    n_rows = 256
+                    v, secs = oracle_sample(wc, n_rows)
+                    cpu = cpu_entry(v, secs, "one head per head class: full scan + %d query rows spread over T; "
+                                             "extrapolated to all heads" % n_rows)
+                line["configs"][name] = prefill_entry(wc, r, args.steps, world, peaks, cpu)
+            else:
+                cpu = None
+                if cpu_ok:
+                    v, secs = oracle_decode_sample(wc, r["ctx"])
+                    cpu = cpu_entry(v, secs, "one batch entry's step (all heads) at position %d, repeated; "
+                                             "times the batch" % r["ctx"])
+                e = decode_entry(wc, r, item[2], world, peaks, cpu=cpu)
+                e["workload"] = wc.name + " decode batch %d" % wc.decode_batch
+                line["configs"][name] = e
     if nxt:
         line["attention_variants"] = {}
         for name, r in att_var.items():
             t_from = w.T * 3 // 4 if name == "chunked" else 0
             fl = sum(w.B * 4.0 * w.d * variant_pairs(w.T, w.dil[h], w.win[h], grid=name == "grid",
                                                      dedupe=name == "dedupe", t_from=t_from) for h in range(w.H))
-            tf = fl / (r["ms"] * 1e-3) / 1e12
             line["attention_variants"][name] = {
                 "what": {"grid": "fixed-grid dilation (j mod D == D-1, plus t)",
                          "dedupe": "window part without the dilated set's keys",
                          "chunked": "last quarter of the prefill as a chunk (t0 = 3T/4) over the whole history"}[name],
                 "ms_per_launch": r["ms"], "value": w.B * (w.T - t_from) * world / (r["ms"] * 1e-3), "unit": "tok/s",
-                "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                             "frac": tf / peaks["bf16_tflops"], "traffic": None},
+                "roofline": tensor_roofline(fl, r["ms"], peaks),
                 "gpu_launches": r["launches"]}
-        wd = wl.DECODE_D16
         desc = {"grid_decode": "fixed-grid dilation, grid cache + window ring, ctx 4096",
                 "paged_decode": "residue cache in 256-row pages (shuffled), ctx 4096",
                 "topk_decode": "top-k blocks (Quest, block 64, K 16) over a dense cache, ctx 16384"}
         line["decode_variants"] = {
             name: {"what": desc[name], "value": wd.decode_batch * world / (r["ms"] * 1e-3), "unit": "tok/s",
-                   "ms_per_step": r["ms"],
-                   "roofline": {"bound": "hbm", "achieved": r["bytes"] / (r["ms"] * 1e-3) / 1e9,
-                                "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                "frac": r["bytes"] / (r["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"], "traffic": None},
+                   "ms_per_step": r["ms"], "roofline": hbm_roofline(r["bytes"], r["ms"], peaks),
                    "gpu_launches": r["launches"]} for name, r in nxt.items()}
-    if not args.no_cpu and world == 1:
+    if cpu_ok:
         v, secs = oracle_sample(w, args.cpu_rows)
         line["cpu_baseline"] = {"value": v, "unit": "tok/s", "cores": host_cores(), "kind": "oracle",
                                 "sample": "head 0 of %d: full scan over T=%d + %d query rows spread over T "

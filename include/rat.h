@@ -284,8 +284,13 @@ RAT_API rat_status rat_decode_step_paged(const rat_cfg *cfg, const void *q, cons
  *     (down to 256) while B * items < 592; a larger step returns
  *     RAT_ERR_UNSUPPORTED with the sizes in rat_last_error().
  *   - The first call on a device (with that device current) looks up the
- *     array's device address (cudaGetSymbolAddress) and caches it; make that
- *     first call before any stream capture.
+ *     array's device address (cudaGetSymbolAddress) and caches it with the
+ *     device's current context; make that first call before any stream
+ *     capture.  If that context is later destroyed (cudaDeviceReset), the next
+ *     call sees a new context and looks the address up again, so it too
+ *     should come before any capture.
+ *   - Arguments are checked by the same code as rat_decode_step, so a bad
+ *     call returns the same status and rat_last_error() text.
  *   - All calls share the one array and it keeps the last call's contents;
  *     each call clears the part that must start at zero (its completion
  *     counters) itself.  Calls whose kernels overlap on a GPU race on it:

@@ -456,14 +456,9 @@ rat_status decode_step(const rat_cfg *cfg, const void *q, const void *k, const v
                        float *state_k, float *state_v, void *cache_k, void *cache_v, const rat_paged_cache *pc,
                        int cache_cap, const int32_t *pos, void *o, float *lse, void *ws, size_t ws_bytes,
                        rat_stream_t stream) {
-    rat_status st = check_cfg(cfg, false);
+    rat_status st = check_decode_args(cfg, q, k, v, g, state_k, state_v, cache_k, cache_v, cache_cap, pos, o, lse);
     if (st != RAT_OK) return st;
     if (cfg->B == 0) return RAT_OK;
-    CHECK_PTR(q, "q"); CHECK_PTR(k, "k"); CHECK_PTR(v, "v"); CHECK_PTR(g, "g");
-    CHECK_PTR(state_k, "state_k"); CHECK_PTR(state_v, "state_v");
-    CHECK_PTR(cache_k, "cache_k"); CHECK_PTR(cache_v, "cache_v");
-    CHECK_PTR(pos, "pos"); CHECK_PTR(o, "o"); CHECK_OPT(lse, "lse");
-    if (cache_cap < 1) return fail(RAT_ERR_INVALID, "cache_cap %d < 1", cache_cap);
     Layout L;
     st = check_ws(cfg, RAT_OP_DECODE, cache_cap, ws, ws_bytes, &L);
     if (st != RAT_OK) return st;
@@ -524,6 +519,23 @@ rat_status scan_prefill(const rat_cfg *cfg, const void *k, const void *v, const 
 }
 
 }  // namespace
+
+// The argument rules of a decode step, shared by every decode entry point
+// (with and without a workspace) so that they accept and refuse alike.
+rat_status rat::check_decode_args(const rat_cfg *cfg, const void *q, const void *k, const void *v, const void *g,
+                                  const float *state_k, const float *state_v, const void *cache_k,
+                                  const void *cache_v, int cache_cap, const int32_t *pos, const void *o,
+                                  const float *lse) {
+    rat_status st = check_cfg(cfg, false);
+    if (st != RAT_OK) return st;
+    if (cfg->B == 0) return RAT_OK;
+    CHECK_PTR(q, "q"); CHECK_PTR(k, "k"); CHECK_PTR(v, "v"); CHECK_PTR(g, "g");
+    CHECK_PTR(state_k, "state_k"); CHECK_PTR(state_v, "state_v");
+    CHECK_PTR(cache_k, "cache_k"); CHECK_PTR(cache_v, "cache_v");
+    CHECK_PTR(pos, "pos"); CHECK_PTR(o, "o"); CHECK_OPT(lse, "lse");
+    if (cache_cap < 1) return fail(RAT_ERR_INVALID, "cache_cap %d < 1", cache_cap);
+    return RAT_OK;
+}
 
 extern "C" {
 

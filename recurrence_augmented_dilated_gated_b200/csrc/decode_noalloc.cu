@@ -11,9 +11,11 @@
 // GPU loading this library holds until the process exits.
 //
 // Host code must not hand the array's name to a kernel: on the host it names a
-// stand-in, not device memory.  The device address is fetched once per device
-// with cudaGetSymbolAddress, on the first call made while that device is
-// current, and cached.
+// stand-in, not device memory.  The device address is fetched with
+// cudaGetSymbolAddress on the first call made while a device is current, and
+// cached together with that device's current context: a call that finds a
+// different context there (the old one was destroyed, e.g. by
+// cudaDeviceReset, and the module loaded again) fetches the address anew.
 #include <math.h>
 #include <stdio.h>
 #include <string.h>
@@ -32,28 +34,56 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
 std::mutex g_setup_mutex;
-void *g_scratch_addr[kMaxDevices];  // device address of g_decode_scratch, per device
+void *g_scratch_addr[kMaxDevices];   // device address of g_decode_scratch, per device
+CUcontext g_scratch_ctx[kMaxDevices];  // the context that address belongs to
 
-// Device address of the scratch on the current device (set up on first use).
+// The driver's cuCtxGetCurrent, looked up once through the runtime.
+using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+CtxGetCurrentFn ctx_get_current() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+    });
+    return fn;
+}
+
+// Device address of the scratch on the current device: looked up on the first
+// call in each context of the device, then reused.
 rat_status scratch_on_current_device(void **out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return set_last_error(RAT_ERR_CUDA, "rat_decode_step_noalloc: cudaGetDevice failed");
     if (dev < 0 || dev >= kMaxDevices)
         return set_last_error(RAT_ERR_UNSUPPORTED, "rat_decode_step_noalloc: device ordinal above 63");
+    CtxGetCurrentFn get_ctx = ctx_get_current();
+    if (!get_ctx) return set_last_error(RAT_ERR_CUDA, "rat_decode_step_noalloc: cuCtxGetCurrent unavailable");
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_decode_scratch);
-        if (e != cudaSuccess || !p)
-            return set_last_error(RAT_ERR_CUDA, "rat_decode_step_noalloc: cudaGetSymbolAddress of the scratch failed");
-        g_scratch_addr[dev] = p;
+    CUcontext ctx = nullptr;
+    if (g_scratch_addr[dev]) {
+        // a context is current once the device has been used; compare it
+        if (get_ctx(&ctx) != CUDA_SUCCESS)
+            return set_last_error(RAT_ERR_CUDA, "rat_decode_step_noalloc: cuCtxGetCurrent failed");
+        if (ctx == g_scratch_ctx[dev]) {
+            *out = g_scratch_addr[dev];
+            return RAT_OK;
+        }
     }
-    *out = g_scratch_addr[dev];
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);  // also makes the device's primary context current
+    if (e != cudaSuccess || !p)
+        return set_last_error(RAT_ERR_CUDA, "rat_decode_step_noalloc: cudaGetSymbolAddress of the scratch failed");
+    if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx)
+        return set_last_error(RAT_ERR_CUDA, "rat_decode_step_noalloc: cuCtxGetCurrent failed");
+    g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
+    *out = p;
     return RAT_OK;
 }
-
-bool a16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 }  // namespace
 
@@ -61,24 +91,9 @@ extern "C" rat_status rat_decode_step_noalloc(const rat_cfg *cfg, const void *q,
                                               const void *g, float *state_k, float *state_v, void *cache_k,
                                               void *cache_v, int cache_cap, const int32_t *pos, void *o,
                                               float *lse, rat_stream_t stream) {
-    // the same argument rules as rat_decode_step
-    const char *bad = nullptr;
-    if (!cfg) bad = "cfg is NULL";
-    else if (cfg->B < 0 || cfg->H < 1 || cfg->H > kMaxHeads || (cfg->d != 64 && cfg->d != 128))
-        bad = "need B >= 0, 1 <= H <= 256, d in {64, 128}";
-    else if (cfg->dtype != RAT_F32 && cfg->dtype != RAT_BF16) bad = "invalid dtype";
-    else if (!cfg->dil || !cfg->win) bad = "cfg->dil / cfg->win is NULL";
-    else if (!(cfg->scale == cfg->scale)) bad = "scale is NaN";
-    else if (cache_cap < 1) bad = "cache_cap < 1";
-    if (!bad && cfg->B > 0) {
-        for (int h = 0; h < cfg->H && !bad; ++h)
-            if (cfg->dil[h] < 1 || cfg->win[h] < 0) bad = "dil[h] must be >= 1 and win[h] >= 0";
-        const void *req[] = {q, k, v, g, state_k, state_v, cache_k, cache_v, pos, o};
-        for (const void *ptr : req)
-            if (!bad && (!ptr || !a16(ptr))) bad = "a required pointer is NULL or not 16-byte aligned";
-        if (!bad && lse && !a16(lse)) bad = "lse is not 16-byte aligned";
-    }
-    if (bad) return set_last_error(RAT_ERR_INVALID, bad);
+    // the argument rules of rat_decode_step, from the same checker
+    rat_status st = check_decode_args(cfg, q, k, v, g, state_k, state_v, cache_k, cache_v, cache_cap, pos, o, lse);
+    if (st != RAT_OK) return st;
     if (cfg->B == 0) return RAT_OK;
 
     DecodeParams p;
@@ -92,7 +107,7 @@ extern "C" rat_status rat_decode_step_noalloc(const rat_cfg *cfg, const void *q,
         return set_last_error(RAT_ERR_UNSUPPORTED, msg);
     }
     void *scratch = nullptr;
-    rat_status st = scratch_on_current_device(&scratch);
+    st = scratch_on_current_device(&scratch);
     if (st != RAT_OK) return st;
 
     p.q = q; p.k = k; p.v = v; p.g = g;

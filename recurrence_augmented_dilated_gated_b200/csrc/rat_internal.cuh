@@ -237,6 +237,11 @@ void count_launches(int n);
 
 // Record the calling thread's rat_last_error() message; returns s.
 rat_status set_last_error(rat_status s, const char *msg);
+// Argument checks of a decode step (cfg, pointers, cache_cap), the same for
+// every decode entry point; sets the last-error string on failure.
+rat_status check_decode_args(const rat_cfg *cfg, const void *q, const void *k, const void *v, const void *g,
+                             const float *state_k, const float *state_v, const void *cache_k, const void *cache_v,
+                             int cache_cap, const int32_t *pos, const void *o, const float *lse);
 
 // launchers (defined in the kernel files); return cudaGetLastError()
 cudaError_t launch_scan(const ScanParams &p, int dtype, cudaStream_t s);

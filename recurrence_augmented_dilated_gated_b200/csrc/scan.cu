@@ -184,24 +184,28 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
                 "l"(reinterpret_cast<uint64_t>(&p.tmap[i])), "r"(0), "r"(h), "r"(tc0), "r"(b), "r"(bar)
                 : "memory");
         // bounded wait for the bytes to land
-        const unsigned long long t0 = global_ns();
-        int ok = 1;
-        for (uint32_t w = 0;; ++w) {
-            uint32_t done;
-            asm volatile(
-                "{\n\t.reg .pred q;\n\tmbarrier.try_wait.parity.shared::cta.b64 q, [%1], 0;\n\t"
-                "selp.u32 %0, 1, 0, q;\n\t}\n"
-                : "=r"(done)
-                : "r"(bar)
-                : "memory");
-            if (done) break;
-            if ((w & 63u) == 63u && (long long)(global_ns() - t0) > limit) {
-                ok = 0;
-                break;
+        auto landed = [&]() -> int {
+            const unsigned long long t0 = global_ns();
+            for (uint32_t w = 0;; ++w) {
+                uint32_t done;
+                asm volatile(
+                    "{\n\t.reg .pred q;\n\tmbarrier.try_wait.parity.shared::cta.b64 q, [%1], 0;\n\t"
+                    "selp.u32 %0, 1, 0, q;\n\t}\n"
+                    : "=r"(done)
+                    : "r"(bar)
+                    : "memory");
+                if (done) return 1;
+                if ((w & 63u) == 63u && (long long)(global_ns() - t0) > limit) return 0;
             }
-        }
+        };
+        const int ok = landed();
         s_load_ok = ok;
-        if (!ok) report_error(p.hdr, RAT_ERR_TIMEOUT, (int)ticket);
+        if (!ok) {
+            report_error(p.hdr, RAT_ERR_TIMEOUT, (int)ticket);
+            // the chunk is skipped, but the CTA must not exit while its copies
+            // may still write its shared memory: one more bounded wait for them
+            (void)landed();
+        }
     }
     __syncthreads();
     const bool loaded = s_load_ok != 0;

@@ -949,13 +949,23 @@ def test_scan_lookback_timeout_is_reported_and_recovers():
 # ------------------------------------------------------ full-size workloads
 
 
+def worst_row_error(got, ref):
+    """Largest relative L2 error of one row (last axis) of got against ref."""
+    got, ref = f64(got) if isinstance(got, torch.Tensor) else got, ref
+    e = np.linalg.norm(got - ref, axis=-1) / np.maximum(np.linalg.norm(ref, axis=-1), 1e-30)
+    return float(e.max())
+
+
 def large_prefill_check(w, heads, n_random=24, seed=0):
     """Run the whole operator at the workload's full size on the GPU; compare
-    sampled heads and rows with the oracle (which runs on those heads only)."""
+    sampled heads and rows with the oracle (which runs on those heads only).
+    Besides the pooled bar, every sampled output row and EVERY row of the
+    augmented keys/values of the sampled heads (all scan chunks, with their
+    boundaries and carries) must be within 5e-2 on its own."""
     dtype = w.torch_dtype
     q, k, v, g = wl.prefill_inputs(w.B, w.T, w.H, w.d, w.gate_mean, dtype, device=DEV, seed=seed)
     cfg = make_cfg(w.B, w.T, w.H, w.d, dtype, w.dil, w.win, w.recur)
-    out = rat.mix_prefill(cfg, q, k, v, g)
+    out = rat.mix_prefill(cfg, q, k, v, g, want_kv=True)
     rat.rat_check_status(out["ws"])
     sl = lambda x: x[:, :, heads]
     dil = [w.dil[h] for h in heads]
@@ -976,7 +986,16 @@ def large_prefill_check(w, heads, n_random=24, seed=0):
     got_l = out["lse"][rows[:, 0], hsel, rows[:, 2]]
     assert_close(got_o, ro, dtype, "o rows")
     assert_close(got_l, rl, dtype, "lse rows")
+    e = worst_row_error(got_o, ro)
+    assert e < 5e-2, "worst sampled output row: rel err %.3g" % e
     assert_close(out["final_k"][:, heads], fk, dtype, "final_k")
+    assert_close(out["final_v"][:, heads], fv, dtype, "final_v")
+    for name, ref in (("kt", kt), ("vt", vt)):
+        got = f64(sl(out[name]))
+        assert_close(got, ref, dtype, name + " (all rows of the sampled heads)")
+        e = worst_row_error(got, ref)
+        assert e < 5e-2, "worst %s row: rel err %.3g" % (name, e)
+        del got
     del out, q, k, v, g
     torch.cuda.empty_cache()
 
