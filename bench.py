@@ -40,6 +40,7 @@ import workloads as wl  # noqa: E402
 
 METRIC = "temporal-mix prefill tok/s @262K & decode tok/s; % of HBM/tensor roofline"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+RAGGED_T = 262144 - 23   # a long prefill whose length the dilation does not divide
 NOMINAL_HBM_GBS = 8000.0   # the ~8 TB/s nominal HBM3e figure, reported beside the measured copy peak
 
 
@@ -561,16 +562,17 @@ def bench_decode(rat, w, ctx, steps, warmup, world, rank, dev, fill_chunk=8, fla
     return dict(ms=ms, bytes=byts, launches=launches, ctx=ctx)
 
 
-def bench_attn_variant(rat, w, flags, steps, warmup, world, rank, dev, t0=0):
+def bench_attn_variant(rat, w, flags, steps, warmup, world, rank, dev, t0=0, T=None):
     """The attention step alone (rat_dilated_attn_prefill) on the prefill
     workload under RAT_FLAG_* `flags`; with t0 > 0, only the queries of
     positions t0 .. T-1 (the last chunk of a chunked prefill) over the whole
-    history.  Returns ms per launch."""
+    history; T overrides the workload's length.  Returns ms per launch."""
     dtype = w.torch_dtype
-    q, k, v, _ = wl.prefill_inputs(w.B, w.T, w.H, w.d, w.gate_mean, dtype, device=dev, seed=11 + rank)
+    T = T or w.T
+    q, k, v, _ = wl.prefill_inputs(w.B, T, w.H, w.d, w.gate_mean, dtype, device=dev, seed=11 + rank)
     if t0 > 0:
         q = q[:, t0:].contiguous()
-    cfg = rat.Config(w.B, w.T - t0, w.H, w.d, dtype, w.dil, w.win, w.recur, flags=flags, t0=t0)
+    cfg = rat.Config(w.B, T - t0, w.H, w.d, dtype, w.dil, w.win, w.recur, flags=flags, t0=t0)
     o = torch.empty_like(q)
     ws = rat.workspace(cfg, rat.RAT_OP_ATTN, device=dev)
     stream = torch.cuda.current_stream()
@@ -876,6 +878,7 @@ def main():
         att_var = {name: bench_attn_variant(rat, w, f, 3, args.warmup, world, rank, dev)
                    for name, f in (("grid", rat.RAT_FLAG_GRID_DILATION), ("dedupe", rat.RAT_FLAG_DEDUPE))}
         att_var["chunked"] = bench_attn_variant(rat, w, 0, 3, args.warmup, world, rank, dev, t0=w.T * 3 // 4)
+        att_var["ragged"] = bench_attn_variant(rat, w, 0, 3, args.warmup, world, rank, dev, T=RAGGED_T)
         nxt["topk_decode"] = bench_topk(rat, wd.decode_batch, wd.H, wd.d, 16384, 64, 16, rat.RAT_TOPK_QUEST,
                                         vsteps, args.warmup, world, rank, dev)
 
@@ -954,13 +957,16 @@ def main():
         line["attention_variants"] = {}
         for name, r in att_var.items():
             t_from = w.T * 3 // 4 if name == "chunked" else 0
-            fl = sum(w.B * 4.0 * w.d * variant_pairs(w.T, w.dil[h], w.win[h], grid=name == "grid",
+            Tv = RAGGED_T if name == "ragged" else w.T
+            fl = sum(w.B * 4.0 * w.d * variant_pairs(Tv, w.dil[h], w.win[h], grid=name == "grid",
                                                      dedupe=name == "dedupe", t_from=t_from) for h in range(w.H))
             line["attention_variants"][name] = {
                 "what": {"grid": "fixed-grid dilation (j mod D == D-1, plus t)",
                          "dedupe": "window part without the dilated set's keys",
-                         "chunked": "last quarter of the prefill as a chunk (t0 = 3T/4) over the whole history"}[name],
-                "ms_per_launch": r["ms"], "value": w.B * (w.T - t_from) * world / (r["ms"] * 1e-3), "unit": "tok/s",
+                         "chunked": "last quarter of the prefill as a chunk (t0 = 3T/4) over the whole history",
+                         "ragged": "T = %d, which D = 64 does not divide (two residue groups of %d and %d rows)"
+                                   % (RAGGED_T, -(-RAGGED_T // 64), RAGGED_T // 64)}[name],
+                "ms_per_launch": r["ms"], "value": w.B * (Tv - t_from) * world / (r["ms"] * 1e-3), "unit": "tok/s",
                 "roofline": tensor_roofline(fl, r["ms"], peaks),
                 "gpu_launches": r["launches"]}
         desc = {"grid_decode": "fixed-grid dilation, grid cache + window ring, ctx 4096",

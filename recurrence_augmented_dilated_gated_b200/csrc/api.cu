@@ -277,14 +277,13 @@ rat_status run_scan(const rat_cfg *c, const Layout &L, const void *k, const void
 // or (fixed grid, D > 1) every position against the grid subsequence.
 bool grid_head(const rat_cfg *c, int h) { return grid_mode(c) && c->dil[h] > 1; }
 
-// A head runs on the tensor-core kernel when its operands are bf16 and its
-// dilation divides T (the strided TMA view needs whole subsequences);
-// otherwise the fp32 CUDA-core kernel computes it.
-// (A chunked prefill also needs t0 % D == 0: its residues line up with the
-// history's.)
-bool tc_head(const rat_cfg *c, int h) {
-    return c->dtype == RAT_BF16 && c->T % c->dil[h] == 0 && c->t0 % c->dil[h] == 0;
-}
+// A head runs on the tensor-core kernel when its operands are bf16; otherwise
+// the fp32 CUDA-core kernel computes it.  Any T works: the residues of a
+// dilation D that does not divide T fall into two classes of equal length
+// (ceil(T/D) and floor(T/D) rows), each read through its own strided view.
+// A chunked prefill also needs t0 % D == 0, so that the chunk's residues line
+// up with the history's.
+bool tc_head(const rat_cfg *c, int h) { return c->dtype == RAT_BF16 && c->t0 % c->dil[h] == 0; }
 
 // One tensor-core launch over `heads` (kind kTcDilated, kTcWindow or kTcGrid),
 // grouped into classes of equal (dilation, K/V source).
@@ -292,7 +291,9 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, int ki
                           const void *kt, const void *vt, const void *kraw, const void *vraw,
                           const bool *raw_head, void *o, float *lse, float *lse_dil, char *ws, unsigned *tickets,
                           int *n_launch, cudaStream_t s) {
-    struct Key { int D; int raw; int xd; };
+    // part: 0 every residue of the dilation (or natural order); with D not
+    // dividing T, 1 the residues r < T mod D (ceil(T/D) rows) and 2 the rest
+    struct Key { int D; int raw; int xd; int part; };
     int done = 0;
     bool taken[kMaxHeads] = {false};
     while (done < nheads) {
@@ -321,33 +322,56 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, int ki
             if (taken[i]) continue;
             const bool win_kind = kind == kTcWindow || kind == kTcWindowDedupe;
             // the dedupe window launch also tells the heads' dilations apart
-            const Key k{win_kind ? 1 : c->dil[h], raw_head[h] ? 1 : 0, kind == kTcWindowDedupe ? c->dil[h] : 1};
-            int ci = -1;
-            for (int j = 0; j < ncls; ++j)
-                if (keys[j].D == k.D && keys[j].raw == k.raw && keys[j].xd == k.xd) ci = j;
-            if (ci < 0) {
-                if (ncls == kTcMaxClasses) continue;  // next launch
-                ci = ncls++;
-                keys[ci] = k;
+            const int D = win_kind ? 1 : c->dil[h];
+            const int xd = kind == kTcWindowDedupe ? c->dil[h] : 1;
+            const int rem = c->T % D, qd = c->T / D;
+            Key want[2];
+            int nk = 0;
+            if (kind != kTcDilated || rem == 0) {
+                want[nk++] = Key{D, raw_head[h] ? 1 : 0, xd, 0};
+            } else {
+                want[nk++] = Key{D, raw_head[h] ? 1 : 0, xd, 1};
+                if (qd > 0) want[nk++] = Key{D, raw_head[h] ? 1 : 0, xd, 2};
             }
-            cls_heads[ci][cls_n[ci]++] = h;
+            // the head joins a launch only with all of its classes
+            int ci[2] = {-1, -1}, fresh = 0;
+            for (int w = 0; w < nk; ++w)
+                for (int j = 0; j < ncls; ++j)
+                    if (keys[j].D == want[w].D && keys[j].raw == want[w].raw && keys[j].xd == want[w].xd &&
+                        keys[j].part == want[w].part)
+                        ci[w] = j;
+            for (int w = 0; w < nk; ++w) fresh += ci[w] < 0;
+            if (ncls + fresh > kTcMaxClasses) continue;  // next launch
+            for (int w = 0; w < nk; ++w) {
+                if (ci[w] < 0) {
+                    ci[w] = ncls++;
+                    keys[ci[w]] = want[w];
+                }
+                cls_heads[ci[w]][cls_n[ci[w]]++] = h;
+            }
             taken[i] = true;
             ++done;
         }
         // order classes by query tiles per subsequence, descending (heaviest first)
         int order[kTcMaxClasses];
         for (int i = 0; i < ncls; ++i) order[i] = i;
-        std::sort(order, order + ncls, [&](int a, int b) { return keys[a].D < keys[b].D; });
+        std::sort(order, order + ncls, [&](int a, int b) {
+            return keys[a].D != keys[b].D ? keys[a].D < keys[b].D : keys[a].part < keys[b].part;
+        });
         P.ncls = ncls;
         long long pref = 0;
         for (int oi = 0; oi < ncls; ++oi) {
             const int ci = order[oi];
             TcClass &C = P.cls[oi];
             C.D = keys[ci].D;
-            // query rows per group: a residue subsequence, or every position
-            C.n = kind == kTcDilated ? c->T / C.D : c->T;
-            C.nres = kind == kTcDilated ? C.D : 1;
-            C.kres = kind == kTcGrid ? C.D - 1 : 0;   // the grid is residue D-1
+            const int part = keys[ci].part, rem = c->T % C.D, qd = c->T / C.D;
+            // query rows per group: a residue subsequence, or every position;
+            // residues r0 .. r0+nres-1 (with D not dividing T: those before
+            // T mod D have one row more than the rest)
+            C.r0 = part == 2 ? rem : 0;
+            C.nres = kind != kTcDilated ? 1 : part == 0 ? C.D : part == 1 ? rem : C.D - rem;
+            C.n = kind != kTcDilated ? c->T : part == 1 ? qd + 1 : qd;
+            C.kres = 0;   // every K/V map starts at its class's first residue
             C.xd = keys[ci].xd;
             C.mtiles = (C.n + 255) / 256;   // 256-row units per (b, h, residue) group
             C.nheads = cls_n[ci];
@@ -361,9 +385,33 @@ rat_status launch_tc_part(const rat_cfg *c, const int *heads, int nheads, int ki
             P.vself[oi] = vb;
             // raw k / v (heads without recurrence, mix prefill) hold the call's rows only
             const int kv_rows = keys[ci].raw ? c->T : P.Th;
-            if (!encode_map_5d(&P.tq[oi], q, c->B, c->T, c->T, c->H, c->d, kind == kTcGrid ? 1 : C.D, kTcRowsQ) ||
-                !encode_map_5d(&P.tk[oi], kb, c->B, P.Tk, kv_rows, c->H, c->d, C.D, kTcRowsKV) ||
-                !encode_map_5d(&P.tv[oi], vb, c->B, P.Tk, kv_rows, c->H, c->d, C.D, kTcRowsKV))
+            // K/V views over the history's Tk = t0 + T positions: the class's
+            // residues (dilated part; t0 is a multiple of D, so they are the
+            // queries' residues), the grid (residue D - 1), or natural order
+            const int krem = P.Tk % C.D, kq = P.Tk / C.D;
+            int kr0 = 0, knres = 1, kn = P.Tk;
+            if (kind == kTcDilated) {
+                kr0 = C.r0;
+                knres = C.nres;
+                kn = part == 0 ? kq : part == 1 ? kq + 1 : kq;
+            } else if (kind == kTcGrid) {
+                kr0 = C.D - 1;
+                kn = kq;
+            }
+            (void)krem;
+            // Q: the class's residues of the call's T rows, or natural order
+            const bool ok_q = kind == kTcDilated
+                                  ? encode_map_res(&P.tq[oi], q, c->B, c->T, c->H, c->d, C.D, C.r0, C.nres, C.n, kTcRowsQ)
+                                  : encode_map_res(&P.tq[oi], q, c->B, c->T, c->H, c->d, 1, 0, 1, c->T, kTcRowsQ);
+            if (kn < 1) {
+                // a grid with no key yet (Tk < D): every row attends to itself
+                // only; point the maps at the first row (never read: the plan
+                // of every row masks its one tile completely)
+                kr0 = 0;
+                kn = 1;
+            }
+            if (!ok_q || !encode_map_res(&P.tk[oi], kb, c->B, kv_rows, c->H, c->d, C.D, kr0, knres, kn, kTcRowsKV) ||
+                !encode_map_res(&P.tv[oi], vb, c->B, kv_rows, c->H, c->d, C.D, kr0, knres, kn, kTcRowsKV))
                 return fail(RAT_ERR_CUDA, "cuTensorMapEncodeTiled failed (dilation %d)", C.D);
         }
         P.prefix[ncls] = pref;

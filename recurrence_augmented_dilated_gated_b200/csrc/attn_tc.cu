@@ -356,6 +356,97 @@ __device__ __forceinline__ float row_exp_s(uint32_t t_s, int lo, int lim, float 
     return ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
 }
 
+// A masked tile, 32 columns at a time.  The 32 rows of a warp are
+// consecutive, so a causal or window boundary crosses at most one or two
+// 32-column chunks of the warp's rows: every other chunk is either valid for
+// all 32 rows (the unmasked body) or masked for all of them (skipped: no TMEM
+// load, no exponentials, P = 0).  Only the chunks the boundary crosses run the
+// masked body.  The decision is warp-uniform (votes), as the TMEM loads need.
+// 0: every key masked for every row of the warp; 1: every key valid; 2: mixed.
+__device__ __forceinline__ int chunk_kind(int q, int lo, int lim) {
+    const int k0 = 32 * q, k1 = 32 * q + 31;
+    if (__all_sync(0xffffffffu, k1 <= lo || k0 > lim)) return 0;
+    if (__all_sync(0xffffffffu, k0 > lo && k1 <= lim)) return 1;
+    return 2;
+}
+
+// row_max_s over a masked tile, chunk by chunk (same result, bit for bit).
+__device__ __forceinline__ float row_max_m(uint32_t t_s, int lo, int lim) {
+    float mx4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) mx4[k] = -INFINITY;
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+        const int kind = chunk_kind(q, lo, lim);
+        if (kind == 0) continue;
+        uint32_t sr[32];
+        tmem_ld32(t_s + 32 * q, sr);
+        if (kind == 1) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                mx4[k & 3] = max3(mx4[k & 3], __uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1]));
+        } else {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                float a = __uint_as_float(sr[2 * k]), b = __uint_as_float(sr[2 * k + 1]);
+                a = key_ok<2>(32 * q + 2 * k, lo, lim) ? a : -INFINITY;
+                b = key_ok<2>(32 * q + 2 * k + 1, lo, lim) ? b : -INFINITY;
+                mx4[k & 3] = max3(mx4[k & 3], a, b);
+            }
+        }
+    }
+    return max3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+}
+
+// row_exp_s over a masked tile, chunk by chunk (same P and row sum, bit for
+// bit: a skipped chunk's zeros add nothing to the sum).
+__device__ __forceinline__ float row_exp_m(uint32_t t_s, int lo, int lim, float c, float m) {
+    uint64_t rs2[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) rs2[k] = f2_pack(0.f, 0.f);
+    const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m, -m);
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+        const int kind = chunk_kind(q, lo, lim);
+        uint32_t pk[16];
+        if (kind == 0) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) pk[k] = 0u;
+        } else {
+            uint32_t sr[32];
+            tmem_ld32(t_s + 32 * q, sr);
+            if (kind == 1) {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    float t0, t1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])), c2, nm2),
+                              t0, t1);
+                    const float e0 = ex2(t0), e1 = ex2(t1);
+                    rs2[k & 3] = f2_add(rs2[k & 3], f2_pack(e0, e1));
+                    pk[k] = pack_bf16(e0, e1);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    float t0, t1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])), c2, nm2),
+                              t0, t1);
+                    float e0 = ex2(t0), e1 = ex2(t1);
+                    e0 = key_ok<2>(32 * q + 2 * k, lo, lim) ? e0 : 0.f;
+                    e1 = key_ok<2>(32 * q + 2 * k + 1, lo, lim) ? e1 : 0.f;
+                    rs2[k & 3] = f2_add(rs2[k & 3], f2_pack(e0, e1));
+                    pk[k] = pack_bf16(e0, e1);
+                }
+            }
+        }
+        tmem_st16(t_s + 16 * q, pk);
+    }
+    float r[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) f2_unpack(rs2[k], r[2 * k], r[2 * k + 1]);
+    return ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
+}
+
 // Keys the dilated set already holds, for the window part with dedupe: in a
 // tile, key k is excluded when k == e0 (mod xd).  base has a bit at every
 // multiple of xd below 32 (one bit when xd > 32); e is the offset of the first
@@ -730,7 +821,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 }
                 float mraw;
                 if constexpr (kDedupe) mraw = row_max_x(t_s, lo, limx, xcl, e0);
-                else mraw = mode == 0 ? row_max_s<0>(t_s, lo, lim) : row_max_s<2>(t_s, lo, lim);
+                else mraw = mode == 0 ? row_max_s<0>(t_s, lo, lim) : row_max_m(t_s, lo, lim);
                 const float mx = mraw * p.scale_log2;   // scale > 0 commutes with max
                 // running max with lazy rescale: keep the stale max unless the new
                 // one exceeds it by more than 8 (P stays <= 2^8)
@@ -760,7 +851,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 float rs;
                 if constexpr (kDedupe) rs = row_exp_x(t_s, lo, limx, xcl, e0, p.scale_log2, m_use);
                 else rs = mode == 0 ? row_exp_s<0>(t_s, lo, lim, p.scale_log2, m_use)
-                                    : row_exp_s<2>(t_s, lo, lim, p.scale_log2, m_use);
+                                    : row_exp_m(t_s, lo, lim, p.scale_log2, m_use);
                 l_run = l_run * alpha + rs;
                 m_run = m_new;
                 tc_fence_before();
@@ -770,7 +861,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (!ok) break;
             if (nt > 0) {
                 const bool valid_row = qi < C.n;
-                const long long t = kKind != kTcDilated ? (long long)qi : (long long)u.r + (long long)C.D * qi;
+                const long long t = kKind != kTcDilated ? (long long)qi : (long long)(u.r + C.r0) + (long long)C.D * qi;
                 const size_t orow = (((size_t)u.b * p.T + (size_t)t) * p.H + u.h) * HD;
                 const size_t lrow = ((size_t)u.b * p.H + u.h) * p.T + (size_t)t;
                 __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.o);
@@ -954,17 +1045,25 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int Ts, int H, int d, int D, int box_rows) {
+bool encode_map_res(CUtensorMap *map, const void *base, int B, int Ts, int H, int d, int D, int r0, int nres, int n,
+                    int box_rows) {
     EncodeTiledFn fn = encode_fn();
-    if (!fn || D < 1 || T % D != 0) return false;
+    if (!fn || D < 1 || r0 < 0 || nres < 1 || n < 1 || (long long)r0 + nres - 1 + (long long)(n - 1) * D >= Ts)
+        return false;
     const cuuint64_t e = 2;  // bf16
-    const cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)D, (cuuint64_t)(T / D), (cuuint64_t)B};
+    const cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)nres, (cuuint64_t)n, (cuuint64_t)B};
     const cuuint64_t strides[4] = {e * d, e * d * H, e * d * H * D, e * d * H * Ts};
     const cuuint32_t box[5] = {64, 1, 1, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
+    const char *origin = static_cast<const char *>(base) + (size_t)r0 * H * d * e;
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<char *>(origin), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int Ts, int H, int d, int D, int box_rows) {
+    if (D < 1 || T % D != 0 || T < D) return false;
+    return encode_map_res(map, base, B, Ts, H, d, D, 0, D, T / D, box_rows);
 }
 
 // One CTA per SM: each CTA allocates all 512 TMEM columns, so the d = 64

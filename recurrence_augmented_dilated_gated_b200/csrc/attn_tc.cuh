@@ -24,9 +24,10 @@ struct TcClass {
     int mtiles;  // 256-row work units per group, ceil(n / 256)
     int nheads;  // heads in the class
     int head0;   // first entry of the class in TcParams::heads
-    int nres;    // groups per (b, h): D residues (dilated part), else 1
-    int kres;    // residue coordinate of K/V relative to Q's (D - 1 for the grid)
+    int nres;    // groups per (b, h): residues r0 .. r0+nres-1 (dilated part), else 1
+    int kres;    // residue coordinate of K/V relative to Q's in their maps
     int xd;      // dilation of the heads (the dedupe window launch), else 1
+    int r0;      // residue of the class's first group (its maps start there)
 };
 
 struct TcParams {
@@ -51,7 +52,7 @@ struct TcParams {
     WsHeader *hdr;
     unsigned int *ticket;           // work-unit counter of this launch (zero at launch)
     long long total_units;
-    unsigned char heads[kMaxHeads];
+    unsigned char heads[2 * kMaxHeads];  // class lists (a head with D not dividing T is in two)
     int win[kMaxHeads];
 };
 
@@ -61,5 +62,12 @@ cudaError_t launch_attn_tc(const TcParams &p, int hd, cudaStream_t s);
 // batch entry) viewed as (d, H, D, T/D, B), box (64, 1, 1, box_rows, 1);
 // requires T % D == 0.
 bool encode_map_5d(CUtensorMap *map, const void *base, int B, int T, int Ts, int H, int d, int D, int box_rows);
+// 5-D TMA map of residues r0 .. r0+nres-1 of a [B,Ts,H,d] bf16 tensor under
+// dilation D, n rows each: element (c, h, r, j, b) is channel c of head h at
+// position r0 + r + j*D of batch entry b; box (64, 1, 1, box_rows, 1).  Every
+// element of the view must lie inside the tensor (r0 + nres - 1 + (n-1)*D < Ts);
+// box rows past n read as zero.
+bool encode_map_res(CUtensorMap *map, const void *base, int B, int Ts, int H, int d, int D, int r0, int nres, int n,
+                    int box_rows);
 
 }  // namespace rat

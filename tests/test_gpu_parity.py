@@ -110,13 +110,19 @@ def test_attention_every_element(dtype, d, case):
 
 
 TC_CASES = [
-    # (B, T, dil per head, win per head): every dilation divides T, so every head
-    # runs on the tensor-core kernel; n = T/D spans full and partial 128-row tiles
+    # (B, T, dil per head, win per head): bf16 operands, so every head runs on
+    # the tensor-core kernel; n = T/D spans full and partial 128-row tiles
     (2, 2048, [1, 4], [0, 0]),
     (2, 2048, [64, 1], [512, 100]),
     (1, 12800, [64, 64], [1, 3000]),       # n = 200: one full and one partial tile
     (2, 1000, [8, 1], [127, 128]),         # n = 125 < 128; window edges at tile size
     (1, 4096, [16, 2], [256, 4096]),
+    # D not dividing T: the residues before T mod D have one row more; each of
+    # the two groups runs through its own strided view, still on the tensor cores
+    (2, 2000, [64, 3], [512, 0]),          # T mod D = 16 and 2
+    (1, 12801, [64, 7], [1, 3000]),        # 201 / 200 and 1829 / 1828 rows per residue
+    (2, 130, [400, 129], [0, 5]),          # D > T (130 one-row residues) and D = T - 1
+    (1, 4097, [16, 1], [256, 0]),          # one residue of 257 rows, fifteen of 256
 ]
 
 
@@ -459,7 +465,9 @@ GRID_CASES = [
     (2, 2048, [4, 64], [0, 100]),        # tensor-core grid launch, one head windowed
     (1, 12800, [64, 128], [1, 3000]),    # 200 and 100 grid rows: full and partial key tiles
     (2, 1024, [256, 1], [0, 64]),        # D = 256: the first query tiles have no grid key yet
-    (2, 1000, [8, 3], [127, 0]),         # 3 does not divide T: that head runs on CUDA cores
+    (2, 1000, [8, 3], [127, 0]),         # 3 does not divide T: the grid is 333 rows of residue 2
+    (1, 5003, [64, 7], [512, 0]),        # T mod D = 11 and 5: ragged grids on the tensor cores
+    (2, 100, [128, 101], [0, 7]),        # D > T: no grid key anywhere, every row attends to itself
 ]
 
 
