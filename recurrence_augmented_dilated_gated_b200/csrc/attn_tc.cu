@@ -447,6 +447,92 @@ __device__ __forceinline__ float row_exp_m(uint32_t t_s, int lo, int lim, float 
     return ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
 }
 
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// P of this row's first `nq` chunks of a tile (bf16 pairs in TMEM columns
+// [0, 16 nq)) times f (1 leaves a row's P unchanged, bit for bit).  Rare path
+// of the one-pass softmax, kept out of line; called by all lanes of a warp.
+__device__ __noinline__ void rescale_p(uint32_t t_s, int nq, float f) {
+    for (int q = 0; q < nq; ++q) {
+        uint32_t pk[16];
+        tmem_ld16(t_s + 16 * q, pk);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(&pk[k]);
+            const float2 x = __bfloat1622float2(v);
+            pk[k] = pack_bf16(x.x * f, x.y * f);
+        }
+        tmem_st16(t_s + 16 * q, pk);
+    }
+}
+
+// One-pass softmax of a full tile against the row's running reference m (log2
+// domain, finite): P = 2^(s c - m), with no separate pass for the tile's max.
+// The reference need not be the maximum (softmax does not depend on it) as
+// long as P stays bounded: a chunk whose sum of P exceeds 2^32 (some score far
+// above m) first raises m for its rows to an upper bound of their maximum so
+// far (the earlier chunks' scores lie below m + 32), rescales the P already
+// written and the partial sum, and is computed again.  Returns the row sum of
+// P against the final m, which the caller compares with the m it passed in.
+__device__ __forceinline__ float row_exp_1p(uint32_t t_s, float c, float &m) {
+    uint64_t rs2[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) rs2[k] = f2_pack(0.f, 0.f);
+    const uint64_t c2 = f2_pack(c, c);
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+        uint32_t sr[32];
+        tmem_ld32(t_s + 32 * q, sr);
+        uint32_t pk[16];
+        uint64_t cs2[4];
+#pragma unroll 1
+        for (int pass = 0;; ++pass) {
+            const uint64_t nm2 = f2_pack(-m, -m);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) cs2[k] = f2_pack(0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                float t0, t1;
+                f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])), c2, nm2), t0,
+                          t1);
+                const float e0 = ex2(t0), e1 = ex2(t1);
+                cs2[k & 3] = f2_add(cs2[k & 3], f2_pack(e0, e1));
+                pk[k] = pack_bf16(e0, e1);
+            }
+            float a[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) f2_unpack(cs2[k], a[2 * k], a[2 * k + 1]);
+            const float csum = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+            const bool hit = csum > 4294967296.f;   // 2^32 (an infinite sum too)
+            if (pass > 0 || !__any_sync(0xffffffffu, hit)) break;
+            float mn = m;
+            if (hit) {
+                float mx = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) mx = max3(mx, __uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1]));
+                mn = fmaxf(m + 32.f, mx * c);
+            }
+            const float f = hit ? ex2(m - mn) : 1.f;
+            if (q > 0) rescale_p(t_s, q, f);
+            const uint64_t f2v = f2_pack(f, f);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) rs2[k] = f2_mul(rs2[k], f2v);
+            m = mn;
+        }
+        tmem_st16(t_s + 16 * q, pk);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) rs2[k] = f2_add(rs2[k], cs2[k]);
+    }
+    float r[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) f2_unpack(rs2[k], r[2 * k], r[2 * k + 1]);
+    return ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
+}
+
 // Keys the dilated set already holds, for the window part with dedupe: in a
 // tile, key k is excluded when k == e0 (mod xd).  base has a bit at every
 // multiple of xd below 32 (one bit when xd > 32); e is the offset of the first
@@ -818,6 +904,35 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     const int r0 = p.grid ? (C.xd - 1 - ks) % C.xd : lim % C.xd;
                     e0 = r0 < 0 ? r0 + C.xd : r0;
                     if (p.grid) limx = lim - 1;
+                }
+                if constexpr (!kDedupe) {
+                    // a full tile after the row's first: one pass against the
+                    // running reference (warp-uniform choice: TMEM accesses are
+                    // warp-collective)
+                    if (mode == 0 && __all_sync(0xffffffffu, m_run != -INFINITY)) {
+                        float m = m_run;
+                        const float rs = row_exp_1p(t_s, p.scale_log2, m);
+                        const bool raised = m != m_run;
+                        const float alpha = raised ? ex2(m_run - m) : 1.f;
+                        // O holds tiles 0..c-1 (S(c) completes after every earlier
+                        // MMA): bring it to the raised reference before PV(c)
+                        if (__any_sync(0xffffffffu, raised)) {
+#pragma unroll 1
+                            for (int cc = 0; cc < HD / 32; ++cc) {
+                                uint32_t o[32];
+                                tmem_ld32(t_o + cc * 32, o);
+#pragma unroll
+                                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                                tmem_st32(t_o + cc * 32, o);
+                            }
+                        }
+                        l_run = l_run * alpha + rs;
+                        m_run = m;
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&bar_pfull[sub]);
+                        continue;
+                    }
                 }
                 float mraw;
                 if constexpr (kDedupe) mraw = row_max_x(t_s, lo, limx, xcl, e0);

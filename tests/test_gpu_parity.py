@@ -894,14 +894,18 @@ def test_chunked_prefill_equals_one_shot(grid, dtype, chunks):
                 np.testing.assert_allclose(cvh[:, h, r], rv[:, j, h], rtol=2e-2, atol=2e-2)
 
 
+@pytest.mark.parametrize("qscale", [8, 32])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_attention_with_large_scores(dtype):
+def test_attention_with_large_scores(dtype, qscale):
     # q scaled by 8: scores of tens in the log2 domain, so the running max
     # grows by more than the lazy-rescale threshold between tiles and P must
-    # stay bounded; the outputs still match the oracle
+    # stay bounded; by 32: later tiles hold scores more than 32 above the
+    # running reference, so the one-pass softmax of full tiles must raise it
+    # mid-tile and rescale the P it has written; the outputs still match the
+    # oracle
     B, T, H, d = 1, 4096, 2, 128
     q, kt, vt, _ = inputs(B, T, H, d, dtype, seed=91)
-    q = (q.float() * 8).to(dtype)
+    q = (q.float() * qscale).to(dtype)
     dil, win = [16, 1], [256, 0]
     cfg = make_cfg(B, T, H, d, dtype, dil, win)
     o = torch.empty_like(q)
