@@ -13,7 +13,8 @@
 // One CTA computes one work unit: 256 query rows as two 128-row sub-tiles that
 // share every K/V tile load (ping-pong, as in FlashAttention-4):
 //   warp 0      TMA producer: Q0/Q1 once, then K and V tiles (2-stage rings)
-//   warp 1      TMEM owner and MMA issuer (one elected thread), in the order
+//   warp 1      TMEM owner and MMA issuer (the warp runs converged; one
+//               elected lane issues every MMA and commit), in the order
 //               PV0(j) QK0(j+1) PV1(j) QK1(j+1), so the tensor core works on
 //               one sub-tile while the softmax of the other runs
 //   warps 2..9  two softmax warpgroups, one per sub-tile; thread i of a group
@@ -129,6 +130,38 @@ __device__ __forceinline__ void tc_fence_before() {
 }
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// The MMA issuer's warp runs converged; one elected lane issues each MMA and
+// commit (always the same lane, so its commits track its own MMAs), while the
+// descriptors and TMEM addresses are warp-uniform values.
+__device__ __forceinline__ void umma_ss_e(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_ts_e(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit_e(uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(
+            smem_u32(bar))
+        : "memory");
 }
 
 // D(tmem) (+)= A(smem) * B(smem)
@@ -747,35 +780,41 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        {
             const uint32_t id_qk = idesc_bf16(BM, BN, 0);
             const uint32_t id_pv = idesc_bf16(BM, HD, 1);
             int n_pv[kSub] = {0, 0};   // PV MMAs issued per sub-tile (pfull phases)
+            // Descriptors of the tiles at their first K step; later steps add
+            // their byte offset / 16 to the start-address field (shared memory
+            // lies below 256 KB, so the field never carries into the next).
+            const uint64_t dq0 = sdesc(sbase + L::kQ, 16, 1024);
+            const uint64_t dk0 = sdesc(sbase + L::kK, 16, 1024);
+            const uint64_t dv0 = sdesc(sbase + L::kV, BN * 128, 1024);
+            constexpr uint64_t kTileD = L::kTile >> 4;   // one tile, in 16-byte units
             auto qk = [&](int i, int n) {  // S_i = Q_i K(ring tile n)
-                const uint32_t tq = sbase + L::kQ + i * L::kTile;
-                const uint32_t tk = sbase + L::kK + (n & 1) * L::kTile;
+                const uint64_t aq = dq0 + i * kTileD, bk = dk0 + (n & 1) * kTileD;
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint64_t a = sdesc(tq + (kk >> 2) * (BM * 128) + (kk & 3) * 32, 16, 1024);
-                    const uint64_t b = sdesc(tk + (kk >> 2) * (BN * 128) + (kk & 3) * 32, 16, 1024);
-                    umma_ss(tmem + BM * i, a, b, id_qk, kk > 0 ? 1u : 0u);
+                    const uint64_t a = aq + (uint64_t)(((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4);
+                    const uint64_t b = bk + (uint64_t)(((kk >> 2) * (BN * 128) + (kk & 3) * 32) >> 4);
+                    umma_ss_e(tmem + BM * i, a, b, id_qk, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&bar_sfull[i]);
+                umma_commit_e(&bar_sfull[i]);
             };
             // O_i (+)= P_i V(ring tile n), P_i read from TMEM over S_i.  Only the
             // unit's last PV of a sub-tile signals bar_pvdone (for the epilogue):
             // the commit after QK_i(j+1), issued after PV_i(j), already tells the
             // softmax that O_i holds tile j when S_i(j+1) is ready.
             auto pv = [&](int i, int n, bool acc, bool last) -> bool {
-                if (!mbar_wait(&bar_pfull[i], (uint32_t)n_pv[i] & 1u, &s_abort)) return false;
+                if (!__all_sync(0xffffffffu, mbar_wait(&bar_pfull[i], (uint32_t)n_pv[i] & 1u, &s_abort))) return false;
                 tc_fence_after();
-                const uint32_t tv = sbase + L::kV + (n & 1) * L::kTile;
+                const uint64_t bv = dv0 + (n & 1) * kTileD;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t b = sdesc(tv + kk * 16 * 128, BN * 128, 1024);
-                    umma_ts(tmem + 256 + HD * i, tmem + BM * i + 8 * kk, b, id_pv, (acc || kk > 0) ? 1u : 0u);
+                    const uint64_t b = bv + (uint64_t)((kk * 16 * 128) >> 4);
+                    umma_ts_e(tmem + 256 + HD * i, tmem + BM * i + 8 * kk, b, id_pv, (acc || kk > 0) ? 1u : 0u);
                 }
-                if (last) umma_commit(&bar_pvdone[i]);
+                if (last) umma_commit_e(&bar_pvdone[i]);
                 ++n_pv[i];
                 return true;
             };
@@ -783,22 +822,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             bool ok = true;
             for (int it = 0; ok; ++it) {
                 const int slot = it & 1;
-                if (!(ok = mbar_wait(&bar_ufull[slot], (uint32_t)(it >> 1) & 1u, &s_abort))) break;
+                if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bar_ufull[slot], (uint32_t)(it >> 1) & 1u, &s_abort)))) break;
                 const long long un = s_unit[slot];
-                mbar_arrive(&bar_uempty[slot]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_uempty[slot]);
                 if (un >= p.total_units) break;
                 const Unit u = decode_unit(p, un);
                 const Plan pl = make_plan<kKind>(p, u);
                 const int ntiles = pl.jhi - pl.jlo + 1;
-                ok = mbar_wait(&bar_q, (uint32_t)it & 1u, &s_abort);
-                if (ok) ok = mbar_wait(&bar_kfull[kv & 1], (uint32_t)(kv >> 1) & 1u, &s_abort);
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar_q, (uint32_t)it & 1u, &s_abort));
+                if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar_kfull[kv & 1], (uint32_t)(kv >> 1) & 1u, &s_abort));
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll
                 for (int i = 0; i < kSub; ++i)
                     if (takes(pl, i, pl.jlo)) qk(i, kv);
-                umma_commit(&bar_kempty[kv & 1]);
-                if (ntiles == 1) umma_commit(&bar_qempty);
+                umma_commit_e(&bar_kempty[kv & 1]);
+                if (ntiles == 1) umma_commit_e(&bar_qempty);
                 bool started[kSub] = {false, false};  // a PV of this unit has written O_i (accumulate)
                 for (int t = 0; t < ntiles && ok; ++t) {
                     const int j = pl.jlo + t;
@@ -809,7 +849,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                         if (!ok) break;
                         if (takes(pl, i, j)) {
                             if (!v_ready) {
-                                ok = mbar_wait(&bar_vfull[cur & 1], (uint32_t)(cur >> 1) & 1u, &s_abort);
+                                ok = __all_sync(0xffffffffu, mbar_wait(&bar_vfull[cur & 1], (uint32_t)(cur >> 1) & 1u, &s_abort));
                                 if (!ok) break;
                                 v_ready = true;
                             }
@@ -819,7 +859,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                         }
                         if (t + 1 < ntiles && takes(pl, i, j + 1)) {
                             if (!k_ready) {
-                                ok = mbar_wait(&bar_kfull[nxt & 1], (uint32_t)(nxt >> 1) & 1u, &s_abort);
+                                ok = __all_sync(0xffffffffu, mbar_wait(&bar_kfull[nxt & 1], (uint32_t)(nxt >> 1) & 1u, &s_abort));
                                 if (!ok) break;
                                 tc_fence_after();
                                 k_ready = true;
@@ -828,24 +868,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                         }
                     }
                     if (!ok) break;
-                    umma_commit(&bar_vempty[cur & 1]);
+                    umma_commit_e(&bar_vempty[cur & 1]);
                     if (t + 1 < ntiles) {
-                        if (!k_ready) ok = mbar_wait(&bar_kfull[nxt & 1], (uint32_t)(nxt >> 1) & 1u, &s_abort);
-                        umma_commit(&bar_kempty[nxt & 1]);
-                        if (t + 2 == ntiles) umma_commit(&bar_qempty);  // the unit's last QK is issued
+                        if (!k_ready) ok = __all_sync(0xffffffffu, mbar_wait(&bar_kfull[nxt & 1], (uint32_t)(nxt >> 1) & 1u, &s_abort));
+                        umma_commit_e(&bar_kempty[nxt & 1]);
+                        if (t + 2 == ntiles) umma_commit_e(&bar_qempty);  // the unit's last QK is issued
                     }
                 }
                 kv += ntiles;
             }
-            if (!ok) {
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok && lane == 0) {
                 s_abort = 1;
                 report_error(p.hdr, RAT_ERR_TIMEOUT, (int)blockIdx.x);
             }
             // every MMA already issued must finish before TMEM is released
             // (a commit arrives once all prior tcgen05 operations are done)
-            umma_commit(&bar_drain);
+            umma_commit_e(&bar_drain);
             volatile int never = 0;
-            mbar_wait(&bar_drain, 0, &never);
+            __all_sync(0xffffffffu, mbar_wait(&bar_drain, 0, &never));
         }
     } else {
         // ------------------------------------------------ softmax warpgroups
