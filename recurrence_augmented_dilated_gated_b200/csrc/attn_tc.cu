@@ -135,26 +135,6 @@ __device__ __forceinline__ void tc_fence_after() {
 // The MMA issuer's warp runs converged; one elected lane issues each MMA and
 // commit (always the same lane, so its commits track its own MMAs), while the
 // descriptors and TMEM addresses are warp-uniform values.
-__device__ __forceinline__ void umma_ss_e(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-__device__ __forceinline__ void umma_ts_e(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p, e;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
 __device__ __forceinline__ void umma_commit_e(uint64_t *bar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t"
@@ -164,32 +144,68 @@ __device__ __forceinline__ void umma_commit_e(uint64_t *bar) {
         : "memory");
 }
 
-// D(tmem) (+)= A(smem) * B(smem)
-__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate) {
+// One K/V tile's worth of MMAs of one sub-tile in one statement: a single
+// lane election and predicate set-up for the group instead of one per MMA.
+// QK: S (+)= Q K^T over NK K steps of 16 (both operands in shared memory);
+// descriptors a[i] / b[i] address step i.  The first step overwrites S.
+template <int NK>
+__device__ __forceinline__ void umma_ss_group(uint32_t d_tmem, const uint64_t *a, const uint64_t *b, uint32_t idesc);
+template <>
+__device__ __forceinline__ void umma_ss_group<8>(uint32_t d_tmem, const uint64_t *a, const uint64_t *b, uint32_t idesc) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "{\n\t.reg .pred e, z, t;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 z, %1, %1;\n\t"
+        "setp.eq.b32 t, %1, %1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %3, %1, z;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %5, %1, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %6, %7, %1, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %8, %9, %1, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %10, %11, %1, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %12, %13, %1, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %14, %15, %1, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %16, %17, %1, t;\n\t}\n" ::"r"(d_tmem),
+        "r"(idesc), "l"(a[0]), "l"(b[0]), "l"(a[1]), "l"(b[1]), "l"(a[2]), "l"(b[2]), "l"(a[3]), "l"(b[3]),
+        "l"(a[4]), "l"(b[4]), "l"(a[5]), "l"(b[5]), "l"(a[6]), "l"(b[6]), "l"(a[7]), "l"(b[7])
         : "memory");
 }
-
-// D(tmem) (+)= A(tmem) * B(smem)
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate) {
+template <>
+__device__ __forceinline__ void umma_ss_group<4>(uint32_t d_tmem, const uint64_t *a, const uint64_t *b, uint32_t idesc) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "{\n\t.reg .pred e, z, t;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 z, %1, %1;\n\t"
+        "setp.eq.b32 t, %1, %1;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %3, %1, z;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %5, %1, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %6, %7, %1, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %8, %9, %1, t;\n\t}\n" ::"r"(d_tmem),
+        "r"(idesc), "l"(a[0]), "l"(b[0]), "l"(a[1]), "l"(b[1]), "l"(a[2]), "l"(b[2]), "l"(a[3]), "l"(b[3])
         : "memory");
 }
-
-__device__ __forceinline__ void umma_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     smem_u32(bar))
-                 : "memory");
+// PV: O (+)= P V over the tile's 128 keys in 8 K steps of 16, P from TMEM
+// columns a_tmem + 8 i (bf16 pairs), V descriptors b[i]; the first step
+// accumulates only when acc != 0.
+__device__ __forceinline__ void umma_ts_group8(uint32_t d_tmem, uint32_t a_tmem, const uint64_t *b, uint32_t idesc,
+                                               uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred e, f, t;\n\t.reg .b32 a1, a2, a3, a4, a5, a6, a7;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 f, %3, 0;\n\t"
+        "setp.eq.b32 t, %2, %2;\n\t"
+        "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\tadd.u32 a4, %1, 32;\n\t"
+        "add.u32 a5, %1, 40;\n\tadd.u32 a6, %1, 48;\n\tadd.u32 a7, %1, 56;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %4, %2, f;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], %5, %2, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], %6, %2, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], %7, %2, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a4], %8, %2, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a5], %9, %2, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a6], %10, %2, t;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a7], %11, %2, t;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(idesc), "r"(acc), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]), "l"(b[4]), "l"(b[5]),
+        "l"(b[6]), "l"(b[7])
+        : "memory");
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -793,12 +809,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             constexpr uint64_t kTileD = L::kTile >> 4;   // one tile, in 16-byte units
             auto qk = [&](int i, int n) {  // S_i = Q_i K(ring tile n)
                 const uint64_t aq = dq0 + i * kTileD, bk = dk0 + (n & 1) * kTileD;
+                uint64_t a[HD / 16], b[HD / 16];
 #pragma unroll
                 for (int kk = 0; kk < HD / 16; ++kk) {
-                    const uint64_t a = aq + (uint64_t)(((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4);
-                    const uint64_t b = bk + (uint64_t)(((kk >> 2) * (BN * 128) + (kk & 3) * 32) >> 4);
-                    umma_ss_e(tmem + BM * i, a, b, id_qk, kk > 0 ? 1u : 0u);
+                    a[kk] = aq + (uint64_t)(((kk >> 2) * (BM * 128) + (kk & 3) * 32) >> 4);
+                    b[kk] = bk + (uint64_t)(((kk >> 2) * (BN * 128) + (kk & 3) * 32) >> 4);
                 }
+                umma_ss_group<HD / 16>(tmem + BM * i, a, b, id_qk);
                 umma_commit_e(&bar_sfull[i]);
             };
             // O_i (+)= P_i V(ring tile n), P_i read from TMEM over S_i.  Only the
@@ -809,11 +826,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 if (!__all_sync(0xffffffffu, mbar_wait(&bar_pfull[i], (uint32_t)n_pv[i] & 1u, &s_abort))) return false;
                 tc_fence_after();
                 const uint64_t bv = dv0 + (n & 1) * kTileD;
+                uint64_t b[BN / 16];
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t b = bv + (uint64_t)((kk * 16 * 128) >> 4);
-                    umma_ts_e(tmem + 256 + HD * i, tmem + BM * i + 8 * kk, b, id_pv, (acc || kk > 0) ? 1u : 0u);
-                }
+                for (int kk = 0; kk < BN / 16; ++kk) b[kk] = bv + (uint64_t)((kk * 16 * 128) >> 4);
+                static_assert(BN / 16 == 8, "eight K steps of P V per tile");
+                umma_ts_group8(tmem + 256 + HD * i, tmem + BM * i, b, id_pv, acc ? 1u : 0u);
                 if (last) umma_commit_e(&bar_pvdone[i]);
                 ++n_pv[i];
                 return true;
