@@ -397,7 +397,7 @@ __device__ __forceinline__ float row_exp_s(uint32_t t_s, int lo, int lim, float 
             rs2[k & 3] = f2_add(rs2[k & 3], f2_pack(e0, e1));
             pk[k] = pack_bf16(e0, e1);
         }
-        tmem_st16(t_s + 16 * q, pk);
+        tmem_st16_async(t_s + 16 * q, pk);
     }
     float r[8];
 #pragma unroll
@@ -488,7 +488,7 @@ __device__ __forceinline__ float row_exp_m(uint32_t t_s, int lo, int lim, float 
                 }
             }
         }
-        tmem_st16(t_s + 16 * q, pk);
+        tmem_st16_async(t_s + 16 * q, pk);
     }
     float r[8];
 #pragma unroll
@@ -506,6 +506,7 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
 // [0, 16 nq)) times f (1 leaves a row's P unchanged, bit for bit).  Rare path
 // of the one-pass softmax, kept out of line; called by all lanes of a warp.
 __device__ __noinline__ void rescale_p(uint32_t t_s, int nq, float f) {
+    tmem_wait_st();   // the chunks' P stores have landed
     for (int q = 0; q < nq; ++q) {
         uint32_t pk[16];
         tmem_ld16(t_s + 16 * q, pk);
@@ -572,7 +573,7 @@ __device__ __forceinline__ float row_exp_1p(uint32_t t_s, float c, float &m) {
             for (int k = 0; k < 4; ++k) rs2[k] = f2_mul(rs2[k], f2v);
             m = mn;
         }
-        tmem_st16(t_s + 16 * q, pk);
+        tmem_st16_async(t_s + 16 * q, pk);
 #pragma unroll
         for (int k = 0; k < 4; ++k) rs2[k] = f2_add(rs2[k], cs2[k]);
     }
@@ -654,7 +655,7 @@ __device__ __forceinline__ float row_exp_x(uint32_t t_s, int lo, int lim, const 
             rs2[k & 3] = f2_add(rs2[k & 3], f2_pack(e0_, e1_));
             pk[k] = pack_bf16(e0_, e1_);
         }
-        tmem_st16(t_s + 16 * q, pk);
+        tmem_st16_async(t_s + 16 * q, pk);
         e = excl_next(x, e);
     }
     float r[8];
@@ -986,6 +987,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                         }
                         l_run = l_run * alpha + rs;
                         m_run = m;
+                        tmem_wait_st();   // P is in TMEM before the MMA warp reads it
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&bar_pfull[sub]);
@@ -1027,6 +1029,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                                     : row_exp_m(t_s, lo, lim, p.scale_log2, m_use);
                 l_run = l_run * alpha + rs;
                 m_run = m_new;
+                tmem_wait_st();   // P is in TMEM before the MMA warp reads it
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar_pfull[sub]);

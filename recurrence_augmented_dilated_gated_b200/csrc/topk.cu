@@ -229,6 +229,9 @@ __global__ void __launch_bounds__(kThreads) topk_decode_kernel(const TopkParams 
                     v = s_rv[w];
                     i = s_ri[w];
                 }
+            // every remaining score NaN (NaN inputs): take a block in range
+            // rather than index past the score array
+            if (i < 1 || i >= c) i = 1 + k;
             s_pick[k] = i;
             s_score[i] = __int_as_float(0x7fffffff);   // NaN: out of the later rounds
         }
