@@ -14,8 +14,11 @@
 //   * a CTA takes a dynamic ticket -> (slice = one (b,h) head, chunk of time);
 //     tickets are handed out in launch order, so every predecessor chunk of a
 //     running CTA has already started (forward progress);
-//   * three TMA loads stage the chunk's k, v, g rows (d channels of one head)
-//     in shared memory; nothing else reads HBM;
+//   * TMA loads stage the chunk's k and v rows (d channels of one head) in
+//     shared memory; the gate logits g either go the same way or, for bf16
+//     with d = 128, straight from global memory into the registers of the
+//     thread that uses them (coalesced across the warp), which leaves room
+//     for three CTAs per SM instead of two;
 //   * pass 1: each group of d/4 threads (4 channels per thread) folds its
 //     sub-chunk of rows into (A, b_k, b_v);
 //   * the CTA folds its groups, publishes its aggregate, looks back over
@@ -23,7 +26,10 @@
 //     entering the chunk, and publishes its inclusive state;
 //   * pass 2: each group replays its sub-chunk from its carried-in state,
 //     overwriting k and v in shared memory with K~ and V~, which two TMA
-//     stores write back (and decode-cache rows are written directly).
+//     stores write back (and decode-cache rows are written directly).  The
+//     gate comes from an fp16 copy of 1 - a that pass 1 left over g in shared
+//     memory, or, when g was not staged, from the logits read again (an L2
+//     hit) and the same fp32 arithmetic as pass 1.
 // HBM traffic is the algorithmic 3 reads + 2 writes per (token, channel).
 // With separate gates for keys and values the scan runs twice in its
 // one-tensor form (kOne: x and g in, x~ out), once per tensor: 2 reads and 1
@@ -133,23 +139,35 @@ template <> struct Smem4<float> {
     static __device__ __forceinline__ void store(float *p, float4 v) { IO4<float>::store(p, v); }
 };
 
+// bf16 with d = 128: the gate logits bypass shared memory (each thread reads
+// its own, coalesced across the warp, in both passes; the second read hits
+// L2), so a chunk stages only k and v and three CTAs fit on an SM; group 0
+// (warp 0, which runs the look-back) keeps its aggregate in registers, which
+// keeps the static shared memory small enough for the third CTA.
+template <typename T, int D>
+constexpr bool gate_in_regs() { return sizeof(T) == 2 && D == 128; }
+
 template <typename T, int D, bool kOne>
-__global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ ScanParams p) {
+__global__ void __launch_bounds__(kThreads, gate_in_regs<T, D>() ? 3 : 1)
+    scan_kernel(const __grid_constant__ ScanParams p) {
     constexpr int LPR = D / 4;             // threads per token row (4 channels each)
     constexpr int G = kThreads / LPR;      // thread groups (sub-chunks) per CTA
     constexpr int C = G * kSub;            // tokens per chunk
     constexpr uint32_t kTile = C * D * sizeof(T);
     constexpr bool kAccurate = sizeof(T) == 4;
+    constexpr bool kRegG = gate_in_regs<T, D>();
+    static_assert(!kRegG || LPR == 32, "group 0 is warp 0");
+    constexpr int G0 = kRegG ? 1 : 0;      // groups whose aggregate stays in registers
     extern __shared__ __align__(128) uint8_t sbuf[];
     T *tile_k = reinterpret_cast<T *>(sbuf);
     T *tile_v = reinterpret_cast<T *>(sbuf + kTile);
-    T *tile_g = reinterpret_cast<T *>(sbuf + 2 * kTile);
+    T *tile_g = reinterpret_cast<T *>(sbuf + 2 * kTile);   // staged only when !kRegG
     __shared__ unsigned s_ticket;
     __shared__ __align__(8) uint64_t s_bar;
     __shared__ int s_load_ok;
-    // per group (A, b_k, b_v); after the look-back, slots 1 and 2 hold the
-    // state entering the group's sub-chunk (k and v)
-    __shared__ float s_agg[G][3][D];
+    // per group g >= G0, at index g - G0: (A, b_k, b_v); after the look-back,
+    // slots 1 and 2 hold the state entering the group's sub-chunk (k and v)
+    __shared__ float s_agg[G - G0][3][D];
 
     const int tid = threadIdx.x;
     if (tid == 0) {
@@ -170,13 +188,28 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
     const int r1 = min(r0 + kSub, p.T - tc0);                    // rows of this group (may be <= r0)
     const long long limit = p.hdr->spin_limit_ns > 0 ? p.hdr->spin_limit_ns : kDefaultSpinNs;
 
+    // gate logits of this thread's rows and channels (kRegG), read while the
+    // chunk's k and v are being staged
+    const __nv_bfloat16 *grow = nullptr;   // row r0 of this thread's channels
+    const size_t gstride = (size_t)p.H * D;
+    uint2 gr[kSub];
+    if constexpr (kRegG) {
+        if (rec) {
+            grow = static_cast<const __nv_bfloat16 *>(p.g) + (((size_t)b * p.T + tc0 + r0) * p.H + h) * D + c0;
+#pragma unroll
+            for (int i = 0; i < kSub; ++i)
+                gr[i] = r0 + i < r1 ? __ldg(reinterpret_cast<const uint2 *>(grow + i * gstride)) : make_uint2(0u, 0u);
+        }
+    }
+
     // ---- stage the chunk: TMA loads of k, v (and g) rows of this head
     if (tid == 0) {
         const uint32_t bar = smem_u32(&s_bar);
+        const int ntile = rec && !kRegG ? 3 : 2;
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
-                     "r"((rec ? 3u : 2u) * kTile - (kOne ? kTile : 0u))
+                     "r"((uint32_t)ntile * kTile - (kOne ? kTile : 0u))
                      : "memory");
-        for (int i = 0; i < (rec ? 3 : 2); ++i)
+        for (int i = 0; i < ntile; ++i)
             if (!kOne || i != 1)   // the one-tensor form has no second tensor
             asm volatile(
                 "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
@@ -221,7 +254,7 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
             if (r < r1) {
                 const uint2 kw = *reinterpret_cast<const uint2 *>(tile_k + r * D + c0);
                 const uint2 vw = kOne ? make_uint2(0u, 0u) : *reinterpret_cast<const uint2 *>(tile_v + r * D + c0);
-                const uint2 gw = *reinterpret_cast<const uint2 *>(tile_g + r * D + c0);
+                const uint2 gw = kRegG ? gr[r - r0] : *reinterpret_cast<const uint2 *>(tile_g + r * D + c0);
                 const uint32_t kq[2] = {kw.x, kw.y}, vq[2] = {vw.x, vw.y}, gq[2] = {gw.x, gw.y};
                 uint32_t oh[2];
 #pragma unroll
@@ -237,7 +270,7 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
                 }
                 // keep 1 - a for pass 2 (fp16: relative precision 2^-11)
                 // over the gate logits this thread has just consumed
-                *reinterpret_cast<uint2 *>(tile_g + r * D + c0) = make_uint2(oh[0], oh[1]);
+                if constexpr (!kRegG) *reinterpret_cast<uint2 *>(tile_g + r * D + c0) = make_uint2(oh[0], oh[1]);
             }
         }
 #pragma unroll
@@ -274,28 +307,40 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
             }
         }
     }
+    if (grp >= G0) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        s_agg[grp][0][c0 + c] = A[c];
-        s_agg[grp][1][c0 + c] = bk[c];
-        s_agg[grp][2][c0 + c] = bv[c];
+        for (int c = 0; c < 4; ++c) {
+            s_agg[grp - G0][0][c0 + c] = A[c];
+            s_agg[grp - G0][1][c0 + c] = bk[c];
+            s_agg[grp - G0][2][c0 + c] = bv[c];
+        }
     }
     __syncthreads();
 
     // ---- chunk aggregate, look-back, inclusive publish (warp 0)
+    float sk0[4], sv0[4];   // kRegG: the state entering group 0's sub-chunk (warp 0)
     if (tid < 32) {
         const int lane = tid;
         const bool owns = lane < LPR;          // lanes holding 4 channels each
         const int cc = lane * 4;
         float TA[4] = {1.f, 1.f, 1.f, 1.f}, Tk[4] = {0.f, 0.f, 0.f, 0.f}, Tv[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (kRegG) {
+            // group 0 is this warp: its aggregate is in registers
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                TA[c] = A[c];
+                Tk[c] = bk[c];
+                Tv[c] = bv[c];
+            }
+        }
         if (owns) {
-            for (int gi = 0; gi < G; ++gi) {
+            for (int gi = G0; gi < G; ++gi) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    float a = s_agg[gi][0][cc + c];
+                    float a = s_agg[gi - G0][0][cc + c];
                     TA[c] *= a;
-                    Tk[c] = a * Tk[c] + s_agg[gi][1][cc + c];
-                    Tv[c] = a * Tv[c] + s_agg[gi][2][cc + c];
+                    Tk[c] = a * Tk[c] + s_agg[gi - G0][1][cc + c];
+                    Tv[c] = a * Tv[c] + s_agg[gi - G0][2][cc + c];
                 }
             }
         }
@@ -446,14 +491,23 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
             }
         }
         // state entering each group's sub-chunk (over the consumed b_k, b_v slots)
+        if constexpr (kRegG) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                sk0[c] = sk[c];
+                sv0[c] = sv[c];
+                sk[c] = A[c] * sk[c] + bk[c];
+                sv[c] = A[c] * sv[c] + bv[c];
+            }
+        }
         if (owns) {
-            for (int gi = 0; gi < G; ++gi) {
+            for (int gi = G0; gi < G; ++gi) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const float a = s_agg[gi][0][cc + c];
-                    const float ak = s_agg[gi][1][cc + c], av = s_agg[gi][2][cc + c];
-                    s_agg[gi][1][cc + c] = sk[c];
-                    s_agg[gi][2][cc + c] = sv[c];
+                    const float a = s_agg[gi - G0][0][cc + c];
+                    const float ak = s_agg[gi - G0][1][cc + c], av = s_agg[gi - G0][2][cc + c];
+                    s_agg[gi - G0][1][cc + c] = sk[c];
+                    s_agg[gi - G0][2][cc + c] = sv[c];
                     sk[c] = a * sk[c] + ak;
                     sv[c] = a * sv[c] + av;
                 }
@@ -465,10 +519,18 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
     // ---- pass 2: replay the sub-chunk from its carried-in state; K~ and V~
     // overwrite k and v in shared memory (same thread, same slot)
     float sk[4], sv[4];
+    if (kRegG && grp == 0) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        sk[c] = s_agg[grp][1][c0 + c];
-        sv[c] = s_agg[grp][2][c0 + c];
+        for (int c = 0; c < 4; ++c) {
+            sk[c] = sk0[c];
+            sv[c] = sv0[c];
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            sk[c] = s_agg[grp - G0][1][c0 + c];
+            sv[c] = s_agg[grp - G0][2][c0 + c];
+        }
     }
     T *ck = static_cast<T *>(p.cache[0]);
     T *cv = static_cast<T *>(p.cache[1]);
@@ -485,21 +547,32 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ 
         return o < 0 ? -1 : o + c0;
     };
     if (loaded && !kAccurate && rec) {
-        // bf16: a = 1 - (1 - a) from the fp16 cache, channel pairs in f32x2
+        // bf16: a = 1 - (1 - a) from the fp16 cache, channel pairs in f32x2;
+        // kRegG: the gate recomputed from the logits, read again (from L2)
         uint64_t sk2[2] = {f2(sk[0], sk[1]), f2(sk[2], sk[3])}, sv2[2] = {f2(sv[0], sv[1]), f2(sv[2], sv[3])};
+        if constexpr (kRegG) {
+#pragma unroll
+            for (int i = 0; i < kSub; ++i)
+                gr[i] = r0 + i < r1 ? __ldg(reinterpret_cast<const uint2 *>(grow + i * gstride)) : make_uint2(0u, 0u);
+        }
 #pragma unroll
         for (int r = r0; r < r0 + kSub; ++r) {
             if (r < r1) {
                 const uint2 kw = *reinterpret_cast<const uint2 *>(tile_k + r * D + c0);
                 const uint2 vw = kOne ? make_uint2(0u, 0u) : *reinterpret_cast<const uint2 *>(tile_v + r * D + c0);
-                const uint2 ow = *reinterpret_cast<const uint2 *>(tile_g + r * D + c0);
+                const uint2 ow = kRegG ? gr[r - r0] : *reinterpret_cast<const uint2 *>(tile_g + r * D + c0);
                 const uint32_t kq[2] = {kw.x, kw.y}, vq[2] = {vw.x, vw.y}, oq[2] = {ow.x, ow.y};
                 uint32_t wk[2], wv[2];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const float2 of = __half22float2(*reinterpret_cast<const __half2 *>(&oq[h]));
-                    const uint64_t oma = f2(of.x, of.y);
-                    const uint64_t a = f2_fma(oma, f2(-1.f, -1.f), f2(1.f, 1.f));
+                    uint64_t a, oma;
+                    if constexpr (kRegG) {
+                        gate2(oq[h], a, oma);   // the same arithmetic as pass 1
+                    } else {
+                        const float2 of = __half22float2(*reinterpret_cast<const __half2 *>(&oq[h]));
+                        oma = f2(of.x, of.y);
+                        a = f2_fma(oma, f2(-1.f, -1.f), f2(1.f, 1.f));
+                    }
                     sk2[h] = f2_fma(a, sk2[h], f2_mul(oma, bf2_f2(kq[h])));
                     sv2[h] = f2_fma(a, sv2[h], f2_mul(oma, bf2_f2(vq[h])));
                     wk[h] = f2_bf2(sk2[h]);
@@ -612,7 +685,8 @@ __global__ void final_of_plain_heads_kernel(const __grid_constant__ ScanParams p
 template <typename T, int D>
 size_t scan_smem() {
     constexpr int C = (kThreads / (D / 4)) * kSub;
-    return 3 * (size_t)C * D * sizeof(T);   // k, v, g of one chunk
+    // k, v (and g unless each thread reads its own gate logits) of one chunk
+    return (gate_in_regs<T, D>() ? 2 : 3) * (size_t)C * D * sizeof(T);
 }
 
 template <typename T, int D, bool kOne>
@@ -621,6 +695,20 @@ cudaError_t launch_form(const ScanParams &p, unsigned tickets, cudaStream_t s) {
     static std::atomic<unsigned long long> smem_set{0};
     cudaError_t e = ensure_smem_limit(scan_kernel<T, D, kOne>, smem, smem_set);
     if (e != cudaSuccess) return e;
+    if (gate_in_regs<T, D>()) {
+        // three CTAs per SM need the largest shared-memory carve-out
+        static std::atomic<unsigned long long> carve_set{0};
+        int dev = 0;
+        e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+        if (!bit || !(carve_set.load(std::memory_order_acquire) & bit)) {
+            e = cudaFuncSetAttribute(scan_kernel<T, D, kOne>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared);
+            if (e != cudaSuccess) return e;
+            if (bit) carve_set.fetch_or(bit, std::memory_order_acq_rel);
+        }
+    }
     scan_kernel<T, D, kOne><<<tickets, kThreads, smem, s>>>(p);
     return cudaSuccess;
 }
