@@ -520,7 +520,7 @@ __device__ __noinline__ void rescale_p(uint32_t t_s, int nq, float f) {
     }
 }
 
-// One-pass softmax of a full tile against the row's running reference m (log2
+// One-pass softmax of a tile against the row's running reference m (log2
 // domain, finite): P = 2^(s c - m), with no separate pass for the tile's max.
 // The reference need not be the maximum (softmax does not depend on it) as
 // long as P stays bounded: a chunk whose sum of P exceeds 2^32 (some score far
@@ -528,17 +528,34 @@ __device__ __noinline__ void rescale_p(uint32_t t_s, int nq, float f) {
 // far (the earlier chunks' scores lie below m + 32), rescales the P already
 // written and the partial sum, and is computed again.  Returns the row sum of
 // P against the final m, which the caller compares with the m it passed in.
-__device__ __forceinline__ float row_exp_1p(uint32_t t_s, float c, float &m) {
+// kMasked: a masked tile (key k valid iff lo < k <= lim), its 32-column chunks
+// classified as in row_exp_m: chunks masked for every row of the warp are
+// skipped (P = 0), chunks valid for all of them take the unmasked body.
+template <bool kMasked>
+__device__ __forceinline__ float row_exp_1p(uint32_t t_s, float c, float &m, int lo, int lim) {
     uint64_t rs2[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) rs2[k] = f2_pack(0.f, 0.f);
     const uint64_t c2 = f2_pack(c, c);
 #pragma unroll 1
     for (int q = 0; q < 4; ++q) {
-        uint32_t sr[32];
-        tmem_ld32(t_s + 32 * q, sr);
+        const int kind = kMasked ? chunk_kind(q, lo, lim) : 1;
         uint32_t pk[16];
         uint64_t cs2[4];
+        if (kMasked && kind == 0) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) pk[k] = 0u;
+            tmem_st16_async(t_s + 16 * q, pk);
+            continue;
+        }
+        uint32_t sr[32];
+        tmem_ld32(t_s + 32 * q, sr);
+        if (kMasked && kind == 2) {
+            // masked scores out of the way once: -inf gives P = 0 and no max
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+                if (!key_ok<2>(32 * q + k, lo, lim)) sr[k] = __float_as_uint(-INFINITY);
+        }
 #pragma unroll 1
         for (int pass = 0;; ++pass) {
             const uint64_t nm2 = f2_pack(-m, -m);
@@ -965,12 +982,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     if (p.grid) limx = lim - 1;
                 }
                 if constexpr (!kDedupe) {
-                    // a full tile after the row's first: one pass against the
+                    // a tile after the row's first: one pass against the
                     // running reference (warp-uniform choice: TMEM accesses are
                     // warp-collective)
-                    if (mode == 0 && __all_sync(0xffffffffu, m_run != -INFINITY)) {
+                    if (__all_sync(0xffffffffu, m_run != -INFINITY)) {
                         float m = m_run;
-                        const float rs = row_exp_1p(t_s, p.scale_log2, m);
+                        const float rs = mode == 0 ? row_exp_1p<false>(t_s, p.scale_log2, m, lo, lim)
+                                                   : row_exp_1p<true>(t_s, p.scale_log2, m, lo, lim);
                         const bool raised = m != m_run;
                         const float alpha = raised ? ex2(m_run - m) : 1.f;
                         // O holds tiles 0..c-1 (S(c) completes after every earlier
