@@ -210,10 +210,15 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
     // item checks the pages of the whole step, so all items of (b, h) agree.
     int bad = 0;
     if (kPaged && valid_pos) {
-        if (n_old > 0)
-            for (long long pg = (long long)slab0 / p.page_rows + tid;
-                 pg <= (long long)(slab0 + n_old - 1) / p.page_rows; pg += kThreads)
-                bad |= row_off(pg * p.page_rows) < 0;
+        if (n_old > 0) {
+            // first and last page of the step's slab (32-bit divisions when the
+            // rows fit, as they do for any cache a sequence can hold)
+            const long long r_lo = (long long)slab0, r_hi = (long long)slab0 + n_old - 1;
+            const bool fits = r_hi <= 0x7fffffffLL;
+            const long long pg_lo = fits ? (long long)((unsigned)r_lo / (unsigned)p.page_rows) : r_lo / p.page_rows;
+            const long long pg_hi = fits ? (long long)((unsigned)r_hi / (unsigned)p.page_rows) : r_hi / p.page_rows;
+            for (long long pg = pg_lo + tid; pg <= pg_hi; pg += kThreads) bad |= row_off(pg * p.page_rows) < 0;
+        }
         long long ra, rb;
         cache_rows_of(t, Dh, W, S, p.grid, ra, rb);
         if (tid == 0) bad |= (ra >= 0 && row_off(ra) < 0) || (rb >= 0 && row_off(rb) < 0);
@@ -282,7 +287,10 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
                     const long long ra = (long long)(slab0 + i0) + (long long)sidx * RS;
                     for (int done = 0; done < nr;) {
                         const long long row = ra + done;
-                        const int n = (int)min((long long)(nr - done), (long long)p.page_rows - row % p.page_rows);
+                        const long long in_page = row <= 0x7fffffffLL
+                                                      ? (long long)((unsigned)row % (unsigned)p.page_rows)
+                                                      : row % p.page_rows;
+                        const int n = (int)min((long long)(nr - done), (long long)p.page_rows - in_page);
                         const long long ofs = row_off(row);
                         const uint32_t nb = (uint32_t)n * kRowBytes, so = (uint32_t)done * kRowBytes;
                         asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(

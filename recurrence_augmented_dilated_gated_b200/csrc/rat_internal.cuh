@@ -114,9 +114,20 @@ __host__ __device__ __forceinline__ long long cache_offset(const int *table, int
                                                            long long cache_R, int H, int d, int b, int h,
                                                            long long row) {
     if (!table) return (((long long)b * H + h) * cache_R + row) * d;
-    const int pg = table[(long long)b * pps + row / page_rows];
+    // one 32-bit division (a row of one sequence's cache fits in 32 bits; a
+    // 64-bit division and remainder cost several times as many instructions)
+    long long pi, pr;
+    if (row >= 0 && row <= 0x7fffffffLL) {
+        const unsigned r32 = (unsigned)row, q = r32 / (unsigned)page_rows;
+        pi = q;
+        pr = r32 - q * (unsigned)page_rows;
+    } else {
+        pi = row / page_rows;
+        pr = row % page_rows;
+    }
+    const int pg = table[(long long)b * pps + pi];
     if (pg < 0 || pg >= num_pages) return -1;
-    return (((long long)pg * H + h) * page_rows + row % page_rows) * d;
+    return (((long long)pg * H + h) * page_rows + pr) * d;
 }
 
 // --------------------------------------------------------------- scan (K1)
