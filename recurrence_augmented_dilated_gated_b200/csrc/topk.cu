@@ -27,6 +27,21 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+// The candidates' statistics and the kept blocks' K~/V~ rows are contiguous
+// runs in global memory: they stream through a double buffer in shared memory
+// (cp.async, 16 bytes per thread and copy), the next chunk in flight while the
+// CTA works on the current one.
+constexpr int kStageBytes = 16384;
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// this thread's copies of all but the most recent `n` groups have landed
+template <int n>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(n) : "memory"); }
 
 template <typename T> struct Row8;
 template <> struct Row8<__nv_bfloat16> {
@@ -115,7 +130,9 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kThreads) topk_decode_kernel(const TopkParams p) {
     constexpr int LPR = D / 8;             // lanes per row (8 channels each)
     constexpr int NG = kThreads / LPR;     // row groups
-    extern __shared__ float s_score[];     // [nblk] candidate scores
+    extern __shared__ __align__(16) unsigned char s_dyn[];   // double buffer, then the candidate scores
+    unsigned char *ring = s_dyn;                            // 2 x kStageBytes
+    float *s_score = reinterpret_cast<float *>(s_dyn + 2 * kStageBytes);   // [nblk]
     __shared__ float s_q[D];
     __shared__ float s_rv[kWarps];
     __shared__ int s_ri[kWarps];
@@ -179,19 +196,46 @@ __global__ void __launch_bounds__(kThreads) topk_decode_kernel(const TopkParams 
     }
     __syncthreads();
 
-    // (B) scores of the candidate blocks 1 .. c-1, one warp per block
+    // (B) scores of the candidate blocks 1 .. c-1, block g by warp (g - 1) mod
+    // kWarps; their statistics stream through the double buffer, CB blocks
+    // per chunk
     const int ncand = c > 1 ? c - 1 : 0;
-    for (int g = 1 + warp; g < c; g += kWarps) {
-        const float *sg = st + (size_t)g * 2 * D;
-        float s = 0.f;
-        for (int ch = lane; ch < D; ch += 32) {
-            const float qc = s_q[ch];
-            if (p.mode == RAT_TOPK_QUEST) s += fmaxf(qc * sg[ch], qc * sg[D + ch]);
-            else s += qc * sg[ch];
-        }
+    {
+        constexpr int CB = kStageBytes / (2 * D * (int)sizeof(float));
+        const int nch = (ncand + CB - 1) / CB;
+        auto load = [&](int sidx, int buf) {
+            const int g0 = 1 + sidx * CB, n = min(CB, c - g0);
+            const unsigned char *src = reinterpret_cast<const unsigned char *>(st + (size_t)g0 * 2 * D);
+            unsigned char *dst = ring + buf * kStageBytes;
+            const int pieces = n * 2 * D * (int)sizeof(float) / 16;
+            for (int i = tid; i < pieces; i += kThreads) cp_async16(dst + 16 * i, src + 16 * i);
+            cp_async_commit();
+        };
+        if (nch > 0) load(0, 0);
+        for (int sidx = 0; sidx < nch; ++sidx) {
+            if (sidx + 1 < nch) {
+                load(sidx + 1, (sidx + 1) & 1);
+                cp_async_wait<1>();
+            } else {
+                cp_async_wait<0>();
+            }
+            __syncthreads();   // every thread's copies of this chunk have landed
+            const float *base = reinterpret_cast<const float *>(ring + (sidx & 1) * kStageBytes);
+            const int g0 = 1 + sidx * CB, g1 = min(c, g0 + CB);
+            for (int g = g0 + (((1 + warp - g0) % kWarps) + kWarps) % kWarps; g < g1; g += kWarps) {
+                const float *sg = base + (size_t)(g - g0) * 2 * D;
+                float s = 0.f;
+                for (int ch = lane; ch < D; ch += 32) {
+                    const float qc = s_q[ch];
+                    if (p.mode == RAT_TOPK_QUEST) s += fmaxf(qc * sg[ch], qc * sg[D + ch]);
+                    else s += qc * sg[ch];
+                }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        if (lane == 0) s_score[g] = p.mode == RAT_TOPK_QUEST ? s : s / (float)bs;
+                for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+                if (lane == 0) s_score[g] = p.mode == RAT_TOPK_QUEST ? s : s / (float)bs;
+            }
+            __syncthreads();   // the buffer is free for the chunk after next
+        }
     }
     __syncthreads();
 
@@ -266,19 +310,66 @@ __global__ void __launch_bounds__(kThreads) topk_decode_kernel(const TopkParams 
     acc.l = 0.f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc.o[i] = 0.f;
-    int blk = 0;
-    for (int r = grp; r < nrows; r += NG) {
-        while (r >= s_off[blk + 1]) ++blk;
-        const int j = s_blk[blk] * bs + (r - s_off[blk]);
-        float kf[8], vf[8];
-        Row8<T>::load(ck + (size_t)j * D + c0, kf);
-        Row8<T>::load(cv + (size_t)j * D + c0, vf);
-        float s = 0.f;
+    // The kept rows in order (block by block), cut into chunks of at most SR
+    // rows that stream through the double buffer (K~ rows, then V~ rows).  Row
+    // r of the concatenation still goes to group r mod NG, in order.
+    {
+        constexpr int SR = kStageBytes / (2 * D * (int)sizeof(T));
+        (void)nrows;
+        auto rows_of = [&](int bi, int ro) { return min(SR, (s_off[bi + 1] - s_off[bi]) - ro); };
+        auto advance = [&](int &bi, int &ro) {
+            ro += SR;
+            if (ro >= s_off[bi + 1] - s_off[bi]) {
+                ++bi;
+                ro = 0;
+            }
+        };
+        auto load = [&](int bi, int ro, int buf) {
+            const int n = rows_of(bi, ro);
+            const size_t j0 = (size_t)s_blk[bi] * bs + ro;   // first cache row
+            const unsigned char *sk = reinterpret_cast<const unsigned char *>(ck + j0 * D);
+            const unsigned char *sv = reinterpret_cast<const unsigned char *>(cv + j0 * D);
+            unsigned char *dk = ring + buf * kStageBytes, *dv = dk + SR * D * sizeof(T);
+            const int pieces = n * D * (int)sizeof(T) / 16;
+            for (int i = tid; i < pieces; i += kThreads) {
+                cp_async16(dk + 16 * i, sk + 16 * i);
+                cp_async16(dv + 16 * i, sv + 16 * i);
+            }
+            cp_async_commit();
+        };
+        int lb = 0, lr = 0;   // next chunk to load
+        int cb = 0, cr = 0;   // chunk to score
+        if (nb > 0) {
+            load(0, 0, 0);
+            advance(lb, lr);
+        }
+        for (int k = 0; cb < nb; ++k) {
+            const bool more = lb < nb;
+            if (more) {
+                load(lb, lr, (k + 1) & 1);
+                cp_async_wait<1>();
+            } else {
+                cp_async_wait<0>();
+            }
+            __syncthreads();   // every thread's copies of this chunk have landed
+            const T *bkr = reinterpret_cast<const T *>(ring + (k & 1) * kStageBytes);
+            const T *bvr = bkr + SR * D;
+            const int n = rows_of(cb, cr), rg0 = s_off[cb] + cr;   // the chunk's first row in the concatenation
+            for (int rr = ((grp - rg0) % NG + NG) % NG; rr < n; rr += NG) {
+                float kf[8], vf[8];
+                Row8<T>::load(bkr + (size_t)rr * D + c0, kf);
+                Row8<T>::load(bvr + (size_t)rr * D + c0, vf);
+                float s = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) s += q8[i] * kf[i];
+                for (int i = 0; i < 8; ++i) s += q8[i] * kf[i];
 #pragma unroll
-        for (int off = LPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(gmask, s, off);
-        acc_add(acc, s, vf);
+                for (int off = LPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(gmask, s, off);
+                acc_add(acc, s, vf);
+            }
+            __syncthreads();   // the buffer is free for the chunk after next
+            if (more) advance(lb, lr);
+            advance(cb, cr);
+        }
     }
     if (tid % LPR == 0) {
         s_m[grp] = acc.m;
@@ -304,10 +395,11 @@ __global__ void __launch_bounds__(kThreads) topk_decode_kernel(const TopkParams 
 
 template <typename T, int D>
 cudaError_t launch_decode_typed(const TopkParams &p, cudaStream_t s) {
-    const size_t smem = (size_t)p.nblk * sizeof(float);
+    const size_t smem = 2 * (size_t)kStageBytes + (size_t)p.nblk * sizeof(float);
     // the limit is raised once per device, so to the largest score array any call can need
     static std::atomic<unsigned long long> smem_set{0};
-    cudaError_t e = ensure_smem_limit(topk_decode_kernel<T, D>, (size_t)kTopkMaxBlocks * sizeof(float), smem_set);
+    cudaError_t e = ensure_smem_limit(topk_decode_kernel<T, D>,
+                                      2 * (size_t)kStageBytes + (size_t)kTopkMaxBlocks * sizeof(float), smem_set);
     if (e != cudaSuccess) return e;
     topk_decode_kernel<T, D><<<(unsigned)(p.B * p.H), kThreads, smem, s>>>(p);
     return cudaSuccess;
