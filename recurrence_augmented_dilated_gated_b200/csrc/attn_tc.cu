@@ -681,6 +681,70 @@ __device__ __forceinline__ float row_exp_x(uint32_t t_s, int lo, int lim, const 
     return ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
 }
 
+// row_exp_1p for the dedupe window: keys outside (lo, lim] and the dilated
+// set's keys (the exclusion pattern from offset e0) get score -inf, then one
+// pass against the running reference m, as in row_exp_1p.
+__device__ __forceinline__ float row_exp_1px(uint32_t t_s, float c, float &m, int lo, int lim, const Excl &x, int e0) {
+    uint64_t rs2[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) rs2[k] = f2_pack(0.f, 0.f);
+    const uint64_t c2 = f2_pack(c, c);
+    int e = e0;
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+        uint32_t sr[32];
+        tmem_ld32(t_s + 32 * q, sr);
+        const uint32_t xw = excl_word(x, e);
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+            if (!(key_ok<2>(32 * q + k, lo, lim) && !((xw >> k) & 1u))) sr[k] = __float_as_uint(-INFINITY);
+        uint32_t pk[16];
+        uint64_t cs2[4];
+#pragma unroll 1
+        for (int pass = 0;; ++pass) {
+            const uint64_t nm2 = f2_pack(-m, -m);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) cs2[k] = f2_pack(0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                float t0, t1;
+                f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1])), c2, nm2), t0,
+                          t1);
+                const float e0_ = ex2(t0), e1_ = ex2(t1);
+                cs2[k & 3] = f2_add(cs2[k & 3], f2_pack(e0_, e1_));
+                pk[k] = pack_bf16(e0_, e1_);
+            }
+            float a[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) f2_unpack(cs2[k], a[2 * k], a[2 * k + 1]);
+            const float csum = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+            const bool hit = csum > 4294967296.f;   // 2^32 (an infinite sum too)
+            if (pass > 0 || !__any_sync(0xffffffffu, hit)) break;
+            float mn = m;
+            if (hit) {
+                float mx = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < 16; ++k) mx = max3(mx, __uint_as_float(sr[2 * k]), __uint_as_float(sr[2 * k + 1]));
+                mn = fmaxf(m + 32.f, mx * c);
+            }
+            const float f = hit ? ex2(m - mn) : 1.f;
+            if (q > 0) rescale_p(t_s, q, f);
+            const uint64_t f2v = f2_pack(f, f);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) rs2[k] = f2_mul(rs2[k], f2v);
+            m = mn;
+        }
+        tmem_st16_async(t_s + 16 * q, pk);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) rs2[k] = f2_add(rs2[k], cs2[k]);
+        e = excl_next(x, e);
+    }
+    float r[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) f2_unpack(rs2[k], r[2 * k], r[2 * k + 1]);
+    return ((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7]));
+}
+
 template <int HD>
 struct Smem {
     static constexpr int kTile = BM * HD * 2;   // one 128-row tile of Q, K or V (bytes)
@@ -981,14 +1045,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                     e0 = r0 < 0 ? r0 + C.xd : r0;
                     if (p.grid) limx = lim - 1;
                 }
-                if constexpr (!kDedupe) {
+                {
                     // a tile after the row's first: one pass against the
                     // running reference (warp-uniform choice: TMEM accesses are
                     // warp-collective)
                     if (__all_sync(0xffffffffu, m_run != -INFINITY)) {
                         float m = m_run;
-                        const float rs = mode == 0 ? row_exp_1p<false>(t_s, p.scale_log2, m, lo, lim)
-                                                   : row_exp_1p<true>(t_s, p.scale_log2, m, lo, lim);
+                        float rs;
+                        if constexpr (kDedupe) rs = row_exp_1px(t_s, p.scale_log2, m, lo, limx, xcl, e0);
+                        else rs = mode == 0 ? row_exp_1p<false>(t_s, p.scale_log2, m, lo, lim)
+                                            : row_exp_1p<true>(t_s, p.scale_log2, m, lo, lim);
                         const bool raised = m != m_run;
                         const float alpha = raised ? ex2(m_run - m) : 1.f;
                         // O holds tiles 0..c-1 (S(c) completes after every earlier
