@@ -18,7 +18,9 @@
 // One CTA per (b, h) runs the step: (A) recurrence update, cache append and
 // statistics update of block c; (B) candidate scores into shared memory, one
 // warp per block; (C) K rounds of a block-wide argmax; (D) an online softmax
-// over the kept blocks' rows, row groups of d/8 lanes, folded by LSE.
+// over the kept blocks' rows, row groups of d/8 lanes, folded by LSE.  (B)
+// and (D) read contiguous runs (the candidates' statistics; each kept block's
+// rows), which stream through a shared-memory double buffer by cp.async.
 #include "rat_internal.cuh"
 
 namespace rat {
@@ -299,7 +301,7 @@ __global__ void __launch_bounds__(kThreads) topk_decode_kernel(const TopkParams 
         s_nb = nb;
     }
     __syncthreads();
-    const int nb = s_nb, nrows = s_off[nb];
+    const int nb = s_nb;
     const int grp = tid / LPR, c0 = (tid % LPR) * 8;
     float q8[8];
 #pragma unroll
@@ -315,7 +317,6 @@ __global__ void __launch_bounds__(kThreads) topk_decode_kernel(const TopkParams 
     // r of the concatenation still goes to group r mod NG, in order.
     {
         constexpr int SR = kStageBytes / (2 * D * (int)sizeof(T));
-        (void)nrows;
         auto rows_of = [&](int bi, int ro) { return min(SR, (s_off[bi + 1] - s_off[bi]) - ro); };
         auto advance = [&](int &bi, int &ro) {
             ro += SR;
