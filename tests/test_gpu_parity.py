@@ -675,6 +675,19 @@ def test_topk_decode_from_empty_history(mode):
                   recur=[1, 0], seed=41, cap=40)
 
 
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("d,block,dtype", [(128, 37, torch.bfloat16), (128, 100, torch.bfloat16),
+                                           (64, 37, torch.bfloat16), (128, 37, torch.float32)])
+def test_topk_decode_many_candidates_odd_blocks(mode, d, block, dtype):
+    # more candidates than one shared-memory chunk of statistics holds (16 per
+    # chunk at d = 128, 32 at d = 64: 19 to 53 here), and blocks whose rows are
+    # not a multiple of the row chunk (32 bf16 rows at d = 128, 16 fp32 rows,
+    # 64 bf16 rows at d = 64), so both streams wrap their double buffer and
+    # row groups realign at every block
+    run_topk_case(B=2, T=2000, steps=3, H=2, d=d, dtype=dtype, block=block, topk=8, mode=mode, recur=[1, 1],
+                  seed=47 + mode)
+
+
 def test_topk_decode_keeps_every_block_when_k_is_large():
     # K >= number of candidates: the step is dense causal attention
     run_topk_case(B=1, T=500, steps=3, H=2, d=128, dtype=torch.bfloat16, block=32, topk=64, mode=0,
