@@ -20,8 +20,11 @@
 //   warps 2..9  two softmax warpgroups, one per sub-tile; thread i of a group
 //               owns query row i (TMEM lane i).  Online softmax in the log2
 //               domain; P (bf16) is written back into TMEM over its own S and
-//               read from there by the PV MMA; O is rescaled in TMEM only when
-//               the running max grows by more than 8 (P stays <= 2^8).
+//               read from there by the PV MMA.  A row's first tile takes two
+//               passes (its max, then P), and O is rescaled in TMEM only when
+//               the running max grows by more than 8; every later tile, masked
+//               or not, takes one pass against the running reference, raised
+//               only where a 32-key chunk's sum of P would pass 2^32.
 // TMEM: S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [256+d,256+2d).
 // Launch 1 (dilated part): units are (b, h, residue, 256-row block), grouped
 // by (b, h, residue) with the heaviest block first, so the blocks that share a
