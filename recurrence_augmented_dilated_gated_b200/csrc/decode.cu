@@ -221,12 +221,19 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
         }
         long long ra, rb;
         cache_rows_of(t, Dh, W, S, p.grid, ra, rb);
-        if (tid == 0) bad |= (ra >= 0 && row_off(ra) < 0) || (rb >= 0 && row_off(rb) < 0);
-        if (W > 0)
-            for (int jj = max(0, t - W + 1) + tid; jj < t; jj += kThreads) {
+        // the new row's two slots, each by a thread of another warp than the
+        // slab's first pages, so that every page-table load is in flight at once
+        if (tid == 32 && ra >= 0) bad |= row_off(ra) < 0;
+        if (tid == 64 && rb >= 0) bad |= row_off(rb) < 0;
+        if (W > 0) {
+            // the window's old rows, four independent lookups per thread at a time
+            const int jlo = max(0, t - W + 1);
+#pragma unroll 4
+            for (int jj = jlo + tid; jj < t; jj += kThreads) {
                 cache_rows_of(jj, Dh, W, S, p.grid, ra, rb);
                 bad |= row_off(rb >= 0 ? rb : ra) < 0;
             }
+        }
     }
 
     if (tid == 0) {
