@@ -168,6 +168,10 @@ __global__ void __launch_bounds__(kThreads, gate_in_regs<T, D>() ? 3 : 1)
     // per group g >= G0, at index g - G0: (A, b_k, b_v); after the look-back,
     // slots 1 and 2 hold the state entering the group's sub-chunk (k and v)
     __shared__ float s_agg[G - G0][3][D];
+    // three CTAs per SM: staged k and v, this table and the small words above,
+    // plus the 1 KB the hardware reserves per CTA, within the SM's 228 KB
+    static_assert(!kRegG || 3 * (2 * (size_t)kTile + sizeof(s_agg) + 64 + 1024) <= 228 * 1024,
+                  "three CTAs must fit in an SM's shared memory");
 
     const int tid = threadIdx.x;
     if (tid == 0) {
