@@ -7,6 +7,8 @@ converted to fp64 on the host).  Bar: max-abs 1e-4 (fp32), relative L2 1e-2
 sampled heads and rows that always include t=0, t<D, residue and window
 boundaries and the last rows.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -1033,6 +1035,14 @@ def test_full_prefill_16k():
 @pytest.mark.slow
 def test_full_prefill_262k_window():
     large_prefill_check(wl.PREFILL_262K, heads=[0, 9], n_random=16)
+
+
+@pytest.mark.slow
+def test_full_prefill_262k_ragged():
+    # T = 262121: D = 64 does not divide it (residues 0..40 have one row more),
+    # so the dilated part runs as two classes of strided views at full size
+    w = dataclasses.replace(wl.PREFILL_262K, T=wl.PREFILL_262K.T - 23)
+    large_prefill_check(w, heads=[0, 9], n_random=16, seed=5)
 
 
 @pytest.mark.slow
