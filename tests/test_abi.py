@@ -133,6 +133,17 @@ def test_topk_sizes_and_argument_checks(lib):
         assert rc == rat.RAT_ERR_INVALID, (block, topk, mode)
     rc = lib.rat_topk_build_stats(c.replace(T=5000).ref(), 64, 0, P, 4096, P, None)
     assert rc == rat.RAT_ERR_INVALID     # more tokens than the cache holds
+    # the step streams cache rows and block statistics through shared memory in
+    # 16-byte copies: a cache or statistics pointer off that alignment is
+    # refused before anything is launched (the other arguments are valid)
+    good = dict(q=P, k=P, v=P, g=P, sk=P, sv=P, ck=P, cv=P, stats=P, pos=P, o=P)
+    for name in ("ck", "cv", "stats"):
+        a = dict(good)
+        a[name] = P + 4
+        rc = lib.rat_topk_decode_step(c.ref(), 64, 4, 0, a["q"], a["k"], a["v"], a["g"], a["sk"], a["sv"], a["ck"],
+                                      a["cv"], 4096, a["stats"], a["pos"], a["o"], None, None, 256, 256, None)
+        assert rc == rat.RAT_ERR_INVALID, name
+        assert b"16-byte aligned" in lib.rat_last_error(), name
 
 
 
